@@ -1,0 +1,503 @@
+"""Benchmark of the MLA decode hot path on B200 (one JSON line on rank 0).
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference] [--workload I]
+
+A step is one pass of the whole path over one batch: the split-KV plan
+(mla_get_metadata), the split-KV decode kernel and the log-sum-exp combine
+(mla_decode), on inputs already resident in HBM.  The workload defaults to
+batch 16, s_q 1, h_q 128, lengths uniform in [1024, 4096] (64-token pages,
+1.25x shuffled pool, bf16 N(0, 1)).  Calls rotate over several independent
+pools whose total size is at least 3x the L2 cache, so each step reads its
+cache from HBM.  The timed region replays CUDA graphs of those steps (exactly
+K steps), bracketed by a barrier and a device synchronisation, timed with CUDA
+events on the launching stream; the split-KV kernel is also timed on its own
+through events recorded around it inside the graphs.
+
+With --gpus N > 1 (launched by torchrun, one process per GPU, NCCL), every
+rank runs its own batch (batch rows are independent: weak scaling, no
+collective on the data path); the reported time is the maximum over ranks.
+
+--impl reference times the fp64 CPU oracle on this host's cores instead (rank
+0 only), one batch row per step, scaled to a full call.
+"""
+
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import math
+import os
+import re
+import sys
+import threading
+import time
+
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from mla_decode_attention_13_b200 import binding, inputs  # noqa: E402
+
+METRIC = "MLA decode µs/call, achieved HBM GB/s and TFLOPS vs B200 roofline (1 GPU)"
+FALLBACK_HBM_GBS = 6650.0
+FALLBACK_BF16_TFLOPS = 1590.0
+KERNEL_SOURCES = ("mla_decode.cu", "sm100_ptx.cuh", "mla_internal.h")
+
+
+# ----------------------------------------------------------------------------
+# work accounting
+# ----------------------------------------------------------------------------
+
+def visible_pairs(lens, h_q, s_q, causal):
+    n = 0
+    for L in lens:
+        for t in range(s_q):
+            vis = min(max((L - s_q + t + 1) if causal else L, 0), L)
+            n += h_q * vis
+    return n
+
+
+def algorithmic_work(lens, h_q, s_q, causal):
+    """Bytes the decode kernel must move and FLOPs it must do.
+
+    Bytes: every cached row once (576 bf16), Q (576 bf16 per query row), the
+    bf16 output (512 per row), fp32 lse, one block-table entry per page and one
+    length per row.  FLOPs: 2 * (576 + 512) per visible (query row, token).
+    """
+    rows = s_q * h_q
+    tokens = sum(lens)
+    pages = sum((L + 63) // 64 for L in lens)
+    nbytes = tokens * 576 * 2 + len(lens) * rows * (576 * 2 + 512 * 2 + 4) + pages * 4 + len(lens) * 4
+    flops = 2 * (576 + 512) * visible_pairs(lens, h_q, s_q, causal)
+    return nbytes, flops
+
+
+def measured_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            d = json.load(f)
+        return float(d["hbm_gbs"]), float(d["bf16_tflops"]), float(d.get("bf16_tflops_sustained", d["bf16_tflops"])), "measured"
+    except Exception:
+        return FALLBACK_HBM_GBS, FALLBACK_BF16_TFLOPS, 1400.0, "fallback"
+
+
+def kernel_source_sha():
+    h = hashlib.sha256()
+    for name in KERNEL_SOURCES:
+        with open(os.path.join(ROOT, "mla_decode_attention_13_b200", "csrc", name), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()[:16]
+
+
+def committed_traffic(workload_name):
+    """DRAM bytes per decode-kernel launch from the committed ncu summary, if
+    it was taken on the current kernel source (else None)."""
+    path = os.path.join(ROOT, "profiles", "mla_decode_kernel_traffic.md")
+    if not os.path.exists(path):
+        return None
+    sha = kernel_source_sha()
+    pat = re.compile(r"traffic_bytes_per_launch:\s*(\d+)\s+workload:\s*(\S+)\s+source_sha:\s*([0-9a-f]+)")
+    for line in open(path):
+        m = pat.search(line)
+        if m and m.group(2) == workload_name and m.group(3) == sha:
+            return int(m.group(1))
+    return None
+
+
+# ----------------------------------------------------------------------------
+# clocks during the timed region
+# ----------------------------------------------------------------------------
+
+class ClockSampler:
+    """Polls SM clock and clock-event reasons through NVML (read-only)."""
+
+    REASONS = {
+        0x1: "gpu_idle", 0x2: "applications_clocks_setting", 0x4: "sw_power_cap", 0x8: "hw_slowdown",
+        0x10: "sync_boost", 0x20: "sw_thermal_slowdown", 0x40: "hw_thermal_slowdown", 0x80: "hw_power_brake_slowdown",
+        0x100: "display_clock_setting",
+    }
+
+    def __init__(self, index):
+        self.samples, self.reasons, self.max_mhz = [], 0, None
+        self._stop = threading.Event()
+        self._thread = None
+        try:
+            import pynvml
+
+            pynvml.nvmlInit()
+            self._nv = pynvml
+            try:
+                nvml_index = torch.cuda._get_nvml_device_index(index)
+            except Exception:
+                nvml_index = index
+            self._h = pynvml.nvmlDeviceGetHandleByIndex(nvml_index)
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self._h, pynvml.NVML_CLOCK_SM)
+            self._reasons = getattr(pynvml, "nvmlDeviceGetCurrentClocksEventReasons", None) or \
+                pynvml.nvmlDeviceGetCurrentClocksThrottleReasons
+        except Exception:
+            self._nv = None
+
+    def _run(self):
+        nv = self._nv
+        while not self._stop.is_set():
+            try:
+                self.samples.append(nv.nvmlDeviceGetClockInfo(self._h, nv.NVML_CLOCK_SM))
+                self.reasons |= self._reasons(self._h)
+            except Exception:
+                pass
+            time.sleep(0.001)
+
+    def __enter__(self):
+        if self._nv is not None:
+            self._thread = threading.Thread(target=self._run, daemon=True)
+            self._thread.start()
+        return self
+
+    def __exit__(self, *exc):
+        self._stop.set()
+        if self._thread:
+            self._thread.join()
+
+    def summary(self):
+        if not self.samples:
+            return {"sm_mhz": None, "sm_max_mhz": self.max_mhz, "reasons": ["unavailable"]}
+        s = sorted(self.samples)
+        names = [n for bit, n in self.REASONS.items() if self.reasons & bit and n != "gpu_idle"]
+        return {"sm_mhz": s[len(s) // 2], "sm_max_mhz": self.max_mhz, "reasons": names, "samples": len(s)}
+
+
+# ----------------------------------------------------------------------------
+# distributed plumbing (one process per GPU)
+# ----------------------------------------------------------------------------
+
+def dist_setup(backend="nccl"):
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import datetime
+
+        import torch.distributed as dist
+
+        os.environ.setdefault("MASTER_ADDR", "127.0.0.1")
+        if backend == "nccl":
+            torch.cuda.set_device(local)
+        dist.init_process_group(backend, timeout=datetime.timedelta(seconds=120))
+    return world, rank, local
+
+
+def max_over_ranks(value: float, world: int, device) -> float:
+    if world == 1:
+        return value
+    import torch.distributed as dist
+
+    t = torch.tensor([value], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def barrier(world: int):
+    if world > 1:
+        import torch.distributed as dist
+
+        dist.barrier()
+
+
+def dist_teardown(world: int):
+    if world > 1:
+        import torch.distributed as dist
+
+        dist.destroy_process_group()
+
+
+# ----------------------------------------------------------------------------
+# the reference arm: the fp64 CPU oracle
+# ----------------------------------------------------------------------------
+
+def cpu_threads():
+    try:
+        from threadpoolctl import threadpool_info
+
+        n = [i.get("num_threads", 1) for i in threadpool_info() if i.get("user_api") == "blas"]
+        return max(n) if n else 1
+    except Exception:
+        return 1
+
+
+def time_oracle_rows(x, rows_per_step, steps, warmup):
+    from oracle import mla_oracle
+
+    times = []
+    b = x.batch
+    for k in range(warmup + steps):
+        rows = [(k * rows_per_step + j) % b for j in range(rows_per_step)]
+        t0 = time.perf_counter()
+        mla_oracle.decode(x.q, x.kv_cache, x.block_table, x.seqlens, x.softmax_scale, x.causal, rows=rows)
+        dt = time.perf_counter() - t0
+        if k >= warmup:
+            times.append(dt)
+    return times
+
+
+def cpu_baseline(idx, budget_s):
+    """The oracle, as it stands, on whole calls of the workload for about budget_s."""
+    from oracle import mla_oracle
+
+    x = inputs.workload_inputs(idx)
+    times = []
+    t_start = time.perf_counter()
+    while not times or (time.perf_counter() - t_start < budget_s and len(times) < 50):
+        t0 = time.perf_counter()
+        mla_oracle.decode(x.q, x.kv_cache, x.block_table, x.seqlens, x.softmax_scale, x.causal)
+        times.append(time.perf_counter() - t0)
+    per_call = sum(times) / len(times)
+    return {"value": round(per_call * 1e6, 1), "unit": "us/call", "cores": cpu_threads(), "kind": "oracle",
+            "sample": f"{len(times)} whole oracle calls (fp64 NumPy, all {x.batch} rows) of the same workload"}
+
+
+def reference_arm(args, world, rank):
+    if rank != 0:
+        return
+    idx = args.workload
+    wl = inputs.WORKLOADS[idx]
+    x = inputs.workload_inputs(idx)
+    lens = x.seqlens.tolist()
+    # calibrate one row, then keep the whole run within a few minutes
+    t_row = min(time_oracle_rows(x, 1, 2, 0))
+    steps, warmup = args.steps, args.warmup
+    t0 = time.perf_counter()
+    times = time_oracle_rows(x, 1, steps, warmup)
+    elapsed = time.perf_counter() - t0
+    per_row = sum(times) / len(times)
+    us_per_call = per_row * x.batch * 1e6
+    nbytes, flops = algorithmic_work(lens, wl.h_q, wl.s_q, wl.causal)
+    line = {
+        "impl": "reference", "metric": METRIC, "value": round(us_per_call, 3), "unit": "us/call", "n_gpus": world,
+        "steps": steps, "warmup": warmup, "ms_per_step": round(per_row * 1e3, 4), "higher_is_better": False,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": workload_config(wl, idx, lens, None),
+        "achieved_gbs": round(nbytes / (us_per_call * 1e-6) / 1e9, 3),
+        "achieved_tflops": round(flops / (us_per_call * 1e-6) / 1e12, 6),
+        "cpu_baseline": {"value": round(us_per_call, 3), "unit": "us/call", "cores": cpu_threads(), "kind": "oracle",
+                         "sample": f"one batch row per step (of {x.batch}), {steps} timed steps, scaled x{x.batch}; "
+                                   f"calibration {t_row * 1e3:.1f} ms/row, run {elapsed:.1f} s"},
+        "e2e": {"value": round(us_per_call, 3), "unit": "us/call", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+def workload_config(wl, idx, lens, l2_note):
+    rec = wl.lengths
+    c = {"workload": wl.name, "batch": wl.batch, "s_q": wl.s_q, "h_q": wl.h_q, "h_kv": 1, "d_qk": 576, "d_v": 512,
+         "page": 64, "causal": wl.causal, "lengths": str(rec[0]) + str(list(rec[1:]))[:60],
+         "tokens": int(sum(lens)), "seed": 1000 + idx}
+    if l2_note:
+        c["l2"] = l2_note
+    return c
+
+
+# ----------------------------------------------------------------------------
+# our arm
+# ----------------------------------------------------------------------------
+
+def ours(args, world, rank, local):
+    dev = torch.device("cuda", local)
+    torch.cuda.set_device(dev)
+    idx = args.workload
+    wl = inputs.WORKLOADS[idx]
+    gen = torch.Generator()
+    gen.manual_seed(1000 + idx)
+    lens = inputs.draw_lengths(wl.lengths, wl.batch, gen)
+    l2 = torch.cuda.get_device_properties(dev).L2_cache_size
+    one = None
+    pools = []
+    total = 0
+    while len(pools) < 2 or total < 3 * l2:
+        seed = 1000 + idx + 7919 * (len(pools) + 1) + 104729 * rank
+        one = inputs.make_inputs(lens, wl.h_q, wl.s_q, seed=seed, causal=wl.causal, softmax_scale=wl.softmax_scale,
+                                 pool_factor=wl.pool_factor, device=str(dev), name=wl.name)
+        pools.append(one)
+        total += one.kv_cache.numel() * 2 + one.q.numel() * 2
+        if len(pools) >= 64:
+            break
+    npool = len(pools)
+    stream = torch.cuda.Stream(dev)
+    ws_bytes = max(binding.mla_workspace_bytes(wl.batch, wl.h_q, wl.s_q), 16)
+    with torch.cuda.stream(stream):
+        metas = [torch.empty(binding.mla_metadata_bytes(wl.batch, wl.h_q, wl.s_q) // 4, dtype=torch.int32, device=dev)
+                 for _ in range(npool)]
+        ws = torch.empty(ws_bytes, dtype=torch.uint8, device=dev)
+        out = torch.empty(wl.batch, wl.s_q, wl.h_q, 512, dtype=torch.bfloat16, device=dev)
+        lse = torch.empty(wl.batch, wl.h_q, wl.s_q, dtype=torch.float32, device=dev)
+    torch.cuda.synchronize(dev)
+
+    def step(r, events=None):
+        x = pools[r]
+        binding.mla_get_metadata(x.seqlens, x.h_q, x.s_q, metadata=metas[r], stream=stream)
+        binding.mla_decode(x.q, x.kv_cache, x.block_table, x.seqlens, x.softmax_scale, x.causal, metas[r],
+                           workspace=ws, out=out, lse=lse, stream=stream, events=events)
+
+    # warm-up (eager), and a check that no device error was raised
+    for k in range(max(args.warmup, 1)):
+        step(k % npool)
+    stream.synchronize()
+    for m in metas:
+        err = binding.mla_check_device_error(m, stream=stream)
+        if err:
+            raise RuntimeError(f"device error word {err:#x} during warm-up")
+
+    # CUDA graphs: one cycle over all pools (with events around each split-KV
+    # kernel) and one single-step graph per pool, so that exactly K steps run.
+    ev_pairs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(npool)]
+    for a, b in ev_pairs:
+        a.record(stream)
+        b.record(stream)
+    stream.synchronize()
+    cycle = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(cycle, stream=stream):
+        for r in range(npool):
+            step(r, events=ev_pairs[r])
+    singles = []
+    for r in range(npool):
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g, stream=stream):
+            step(r)
+        singles.append(g)
+    with torch.cuda.stream(stream):
+        for _ in range(2):
+            cycle.replay()
+    stream.synchronize()
+
+    K = args.steps
+    reps, rem = divmod(K, npool)
+    start = torch.cuda.Event(enable_timing=True)
+    end = torch.cuda.Event(enable_timing=True)
+    barrier(world)
+    torch.cuda.synchronize(dev)
+    with ClockSampler(local) as clocks:
+        with torch.cuda.stream(stream):
+            start.record(stream)
+            for _ in range(reps):
+                cycle.replay()
+            for r in range(rem):
+                singles[r].replay()
+            end.record(stream)
+        stream.synchronize()
+    torch.cuda.synchronize(dev)
+    barrier(world)
+    ms_total = start.elapsed_time(end)
+    ms_total = max_over_ranks(ms_total, world, dev)
+    ms_step = ms_total / K
+    k2_ms = [a.elapsed_time(b) for a, b in ev_pairs] if reps > 0 else []
+    k2_avg_ms = sum(k2_ms) / len(k2_ms) if k2_ms else float("nan")
+    for m in metas:
+        err = binding.mla_check_device_error(m, stream=stream)
+        if err:
+            raise RuntimeError(f"device error word {err:#x} in the timed region")
+
+    # end to end through the API: pinned host inputs in, result out, every step
+    e2e_steps = min(K, 500)
+    x0 = pools[0]
+    h_q_host = x0.q.cpu().pin_memory()
+    h_table = x0.block_table.cpu().pin_memory()
+    h_lens = x0.seqlens.cpu().pin_memory()
+    h_out = torch.empty(out.shape, dtype=out.dtype).pin_memory()
+    h_lse = torch.empty(lse.shape, dtype=lse.dtype).pin_memory()
+    d_q = torch.empty_like(x0.q)
+    d_table = torch.empty_like(x0.block_table)
+    d_lens = torch.empty_like(x0.seqlens)
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    barrier(world)
+    torch.cuda.synchronize(dev)
+    with torch.cuda.stream(stream):
+        e0.record(stream)
+        for _ in range(e2e_steps):
+            d_q.copy_(h_q_host, non_blocking=True)
+            d_table.copy_(h_table, non_blocking=True)
+            d_lens.copy_(h_lens, non_blocking=True)
+            binding.mla_get_metadata(d_lens, x0.h_q, x0.s_q, metadata=metas[0], stream=stream)
+            binding.mla_decode(d_q, x0.kv_cache, d_table, d_lens, x0.softmax_scale, x0.causal, metas[0],
+                               workspace=ws, out=out, lse=lse, stream=stream)
+            h_out.copy_(out, non_blocking=True)
+            h_lse.copy_(lse, non_blocking=True)
+        e1.record(stream)
+    stream.synchronize()
+    e2e_ms = max_over_ranks(e0.elapsed_time(e1) / e2e_steps, world, dev)
+    h2d = h_q_host.numel() * 2 + h_table.numel() * 4 + h_lens.numel() * 4
+    d2h = h_out.numel() * 2 + h_lse.numel() * 4
+
+    nbytes, flops = algorithmic_work(lens, wl.h_q, wl.s_q, wl.causal)
+    hbm_peak, tf_peak, tf_sustained, peak_kind = measured_peaks()
+    k2_s = k2_avg_ms * 1e-3
+    achieved_k2 = nbytes / k2_s / 1e9 if k2_s > 0 else None
+    line = {
+        "metric": METRIC,
+        "value": round(ms_step * 1e3, 3),
+        "unit": "us/call",
+        "n_gpus": world,
+        "steps": K,
+        "warmup": args.warmup,
+        "ms_per_step": round(ms_step, 6),
+        "higher_is_better": False,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": "bf16",
+        "data": "synthetic",
+        "config": workload_config(wl, idx, lens, f"{npool} rotating pools, {total / 2**20:.0f} MiB > 3x "
+                                                 f"{l2 / 2**20:.0f} MiB L2; timed via CUDA graph replay"),
+        "achieved_gbs": round(nbytes / (ms_step * 1e-3) / 1e9, 1),
+        "achieved_tflops": round(flops / (ms_step * 1e-3) / 1e12, 2),
+        "calls_per_s_all_ranks": round(world / (ms_step * 1e-3), 1),
+        "decode_kernel_us": round(k2_avg_ms * 1e3, 3),
+        "roofline": {
+            "bound": "hbm",
+            "achieved": round(achieved_k2, 1) if achieved_k2 else None,
+            "peak": hbm_peak,
+            "unit": "GB/s",
+            "frac": round(achieved_k2 / hbm_peak, 4) if achieved_k2 else None,
+            "traffic": committed_traffic(wl.name),
+            "kernel": "mla_decode_kernel",
+            "algorithmic_bytes_per_launch": nbytes,
+            "peak_source": f"{peak_kind} hbm_gbs",
+            "tensor_frac_of_measured_bf16": round(flops / k2_s / 1e12 / tf_peak, 4) if k2_s > 0 else None,
+        },
+        "e2e": {"value": round(e2e_ms * 1e3, 3), "unit": "us/call", "h2d_bytes_per_step": h2d,
+                "d2h_bytes_per_step": d2h, "steps": e2e_steps,
+                "note": "pinned q/block_table/seqlens in, out/lse back, every step; cache resident in HBM"},
+        "gpu_launches": 3 * K,
+        "clocks": clocks.summary(),
+    }
+    if world == 1 and rank == 0 and not args.no_cpu_baseline:
+        line["cpu_baseline"] = cpu_baseline(idx, budget_s=10.0)
+    del cycle, singles
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+
+
+def main():
+    ap = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawDescriptionHelpFormatter)
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=3000)
+    ap.add_argument("--warmup", type=int, default=10)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--workload", type=int, default=1, help="index into inputs.WORKLOADS (1 = headline)")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        args.warmup = 3
+    world, rank, local = dist_setup("nccl" if args.impl == "ours" else "gloo")
+    try:
+        if args.impl == "reference":
+            reference_arm(args, world, rank)
+        else:
+            ours(args, world, rank, local)
+    finally:
+        dist_teardown(world)
+
+
+if __name__ == "__main__":
+    main()

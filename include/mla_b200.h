@@ -1,0 +1,168 @@
+/*
+ * mla_b200.h — C ABI of libmla_b200.so: Multi-head Latent Attention (MLA)
+ * decode over a paged, compressed latent KV cache, on one NVIDIA B200
+ * (sm_100a).
+ *
+ * The operation.  "MLA 和 MHA 的 Kernel 区别" (sealessland.top), sections
+ * "内存布局和 KV Cache 大小 / MLA" and "Decode 阶段的 HBM 访问模式 / MLA Decode":
+ * the cache holds one compressed latent vector per token; a decode step scores
+ * the new query against every cached token, applies a softmax and sums the
+ * values.  In absorbed form each cached token is one 576-element bf16 row
+ * (512 latent dims, then 64 rope dims); each query head is a 576-element row;
+ * the score is softmax_scale * <q, k_j> over all 576 dims and the value is the
+ * first 512 dims of the same row.  For batch row i, query token t, head h:
+ *
+ *     z_j  = softmax_scale * <q[i][t][h][:], kv_row(i, j)>,   j visible
+ *     lse  = ln sum_j exp(z_j)
+ *     out  = sum_j exp(z_j - lse) * kv_row(i, j)[0:512]
+ *
+ * "FlashMLA overview" (nullthought.net FlashMLA walkthrough): bf16 cache,
+ * paged in blocks of 64 tokens, variable-length rows.  Token j of row i lives
+ * in page block_table[i][j / 64], slot j % 64.  Visible tokens are j < L_i;
+ * with causal = 1 query token t sees j <= L_i - s_q + t (the s_q new tokens
+ * are the last s_q cache positions).  A query with no visible token returns
+ * out = 0 and lse = -inf.
+ *
+ * The two calls follow the same page's account of the FlashMLA API
+ * ("flash_api.cpp"): a metadata call prepares the tile-scheduler plan once per
+ * decode step and is reused for every layer; then the attention call runs once
+ * per layer.  Splitting long rows across processors and merging the pieces by
+ * log-sum-exp is the flash-decoding scheme of "Unlocking GPU Potential: The
+ * Impact of FlashAttention and KV Cache Optimization in Long-Text Inference"
+ * (decode has query length 1, so a small batch leaves most SMs idle).
+ *
+ * Conventions for every function below.
+ *   - Pointers marked [device] are CUDA device pointers owned by the caller;
+ *     the library never allocates, frees or keeps them.  Tensors are dense
+ *     and row-major in the stated shape.
+ *   - `stream` is a cudaStream_t passed as void* (NULL = legacy default
+ *     stream).  Calls enqueue work asynchronously and never synchronise the
+ *     host, except mla_check_device_error.
+ *   - Argument errors are found on the host, before anything is enqueued, and
+ *     returned as a negative status.  Errors only the GPU can see (a length
+ *     past the block table, a page id outside the pool, a plan that does not
+ *     match the call, a wait that ran past its time limit) set bits in an error
+ *     word inside `metadata`; the kernels skip the offending work instead of
+ *     faulting, and mla_check_device_error reports the word.
+ *   - No exception or C++ type crosses the ABI.  The functions are
+ *     thread-compatible: concurrent calls must use distinct metadata and
+ *     workspace buffers.
+ */
+#ifndef MLA_B200_H
+#define MLA_B200_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* Status codes returned by every int-valued function. */
+#define MLA_OK 0
+#define MLA_ERR_ARG (-1)         /* NULL pointer, bad size, bad alignment  */
+#define MLA_ERR_UNSUPPORTED (-2) /* shape outside what the kernels handle  */
+#define MLA_ERR_CUDA (-3)        /* a CUDA runtime or driver call failed   */
+#define MLA_ERR_WORKSPACE (-4)   /* workspace smaller than required        */
+#define MLA_ERR_DEVICE (-5)      /* the device error word is non-zero      */
+
+/* Bits of the device error word (see mla_check_device_error). */
+#define MLA_DEVERR_SEQLEN 0x1u   /* L_i < 0 or L_i > 64 * max_pages_per_seq */
+#define MLA_DEVERR_PAGE 0x2u     /* block-table entry outside [0, num_pages) */
+#define MLA_DEVERR_TIMEOUT 0x4u  /* a bounded wait inside a kernel gave up   */
+#define MLA_DEVERR_PLAN 0x8u     /* metadata does not match this call        */
+
+/* Fixed dimensions of the absorbed cache row and of a page. */
+#define MLA_D_QK 576
+#define MLA_D_V 512
+#define MLA_PAGE 64
+
+/*
+ * Bytes of the metadata buffer mla_get_metadata fills for this shape.
+ * batch >= 1, 1 <= h_q <= 128, 1 <= s_q <= 16; returns 0 otherwise.
+ */
+size_t mla_metadata_bytes(int batch, int h_q, int s_q);
+
+/*
+ * Bytes of scratch ("workspace") mla_decode needs for this shape on the
+ * current CUDA device: the fp32 partial outputs and log-sum-exps of rows that
+ * the plan splits across SM pairs.  Returns 0 for an unsupported shape.  When
+ * no CUDA device can be queried the bound for the largest supported GPU is
+ * returned, which is never too small.
+ */
+size_t mla_workspace_bytes(int batch, int h_q, int s_q);
+
+/*
+ * Number of 2-CTA clusters (SM pairs) the decode kernel runs on the current
+ * device; the plan is cut into this many pieces.  Negative status on error.
+ */
+int mla_num_sm_pairs(void);
+
+/*
+ * Build the split-KV tile-scheduler plan for one decode step ("FlashMLA
+ * overview", flash_api.cpp: get_mla_metadata).
+ *
+ *   seqlens   [device] int32 [batch]: cached tokens L_i of each row.
+ *   batch, h_q, s_q: as for mla_decode.
+ *   metadata  [device] mla_metadata_bytes(batch, h_q, s_q) bytes, 16-byte
+ *             aligned; overwritten by the plan, and its error word cleared.
+ *
+ * One kernel on `stream`; no host synchronisation.  The same metadata serves
+ * any number of mla_decode calls (one per layer) with the same seqlens.
+ */
+int mla_get_metadata(const int32_t* seqlens, int batch, int h_q, int s_q, void* metadata, void* stream);
+
+/*
+ * MLA decode ("FlashMLA overview", flash_api.cpp: flash_mla_with_kvcache).
+ *
+ *   q            [device] bf16 [batch][s_q][h_q][576], 16-byte aligned.
+ *   kv_cache     [device] bf16 [num_pages][64][1][576], 16-byte aligned;
+ *                one latent-plus-rope row per cached token, h_kv = 1.
+ *   num_pages    pages in the pool, 1 <= num_pages <= 2^25.
+ *   block_table  [device] int32 [batch][max_pages_per_seq]; entries past a
+ *                row's ceil(L_i / 64) pages are never read.
+ *   seqlens      [device] int32 [batch], 0 <= L_i <= 64 * max_pages_per_seq;
+ *                must hold the values the metadata was built from.
+ *   softmax_scale  multiplies <q, k>; finite.
+ *   causal       0 or 1 (see the header comment).
+ *   out          [device] bf16 [batch][s_q][h_q][512], 16-byte aligned.
+ *   lse          [device] fp32 [batch][h_q][s_q]: natural log of
+ *                sum_j exp(softmax_scale * <q, k_j>).
+ *   metadata     [device] from mla_get_metadata for (seqlens, batch, h_q, s_q);
+ *                its error word may be set by this call.
+ *   workspace    [device] at least mla_workspace_bytes(batch, h_q, s_q)
+ *                bytes, 16-byte aligned; workspace_bytes says how many.
+ *
+ * Enqueues the split-KV decode kernel and the log-sum-exp combine kernel on
+ * `stream`.  Supported: 1 <= h_q <= 128, 1 <= s_q <= 16, batch >= 1.
+ */
+int mla_decode(const void* q, const void* kv_cache, int64_t num_pages, const int32_t* block_table,
+               int max_pages_per_seq, const int32_t* seqlens, int batch, int s_q, int h_q, float softmax_scale,
+               int causal, void* out, float* lse, void* metadata, void* workspace, size_t workspace_bytes,
+               void* stream);
+
+/*
+ * mla_decode, plus CUDA events recorded on `stream` immediately before and
+ * after the split-KV decode kernel (either may be NULL), so that a caller can
+ * time that kernel alone.  The events are cudaEvent_t passed as void*.
+ */
+int mla_decode_timed(const void* q, const void* kv_cache, int64_t num_pages, const int32_t* block_table,
+                     int max_pages_per_seq, const int32_t* seqlens, int batch, int s_q, int h_q,
+                     float softmax_scale, int causal, void* out, float* lse, void* metadata, void* workspace,
+                     size_t workspace_bytes, void* stream, void* event_before_decode, void* event_after_decode);
+
+/*
+ * Synchronise `stream` and read the device error word from `metadata`.
+ * Writes the word to *error_word (if not NULL).  Returns MLA_OK when it is
+ * zero, MLA_ERR_DEVICE when not, MLA_ERR_CUDA if the copy or sync failed.
+ */
+int mla_check_device_error(const void* metadata, void* stream, uint32_t* error_word);
+
+/* Static text for a status code. */
+const char* mla_error_string(int status);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* MLA_B200_H */

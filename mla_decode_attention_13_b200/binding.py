@@ -1,0 +1,173 @@
+"""ctypes binding of libmla_b200.so (the C ABI in include/mla_b200.h).
+
+Argument marshalling only: tensors are passed as raw device pointers with the
+current CUDA stream; every step of the decode runs in the library's kernels.
+The functions keep the C names.  There is no CPU fallback: if the library is
+missing, or a call returns a non-zero status, a RuntimeError is raised.
+"""
+
+from __future__ import annotations
+
+import ctypes
+import os
+from typing import Optional, Tuple
+
+import torch
+
+LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libmla_b200.so")
+
+MLA_OK = 0
+MLA_ERR_ARG = -1
+MLA_ERR_UNSUPPORTED = -2
+MLA_ERR_CUDA = -3
+MLA_ERR_WORKSPACE = -4
+MLA_ERR_DEVICE = -5
+
+MLA_DEVERR_SEQLEN = 0x1
+MLA_DEVERR_PAGE = 0x2
+MLA_DEVERR_TIMEOUT = 0x4
+MLA_DEVERR_PLAN = 0x8
+
+EXPORTED = (
+    "mla_metadata_bytes",
+    "mla_workspace_bytes",
+    "mla_num_sm_pairs",
+    "mla_get_metadata",
+    "mla_decode",
+    "mla_decode_timed",
+    "mla_check_device_error",
+    "mla_error_string",
+)
+
+_lib = None
+_vp = ctypes.c_void_p
+_i32p = ctypes.POINTER(ctypes.c_int32)
+
+
+class MLAError(RuntimeError):
+    def __init__(self, func: str, status: int):
+        self.status = status
+        super().__init__(f"{func} failed: {status} ({mla_error_string(status)})")
+
+
+def lib() -> ctypes.CDLL:
+    """Open the library once (RuntimeError if it was not built)."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIB_PATH):
+            raise RuntimeError(f"{LIB_PATH} is missing: build it with `python -m mla_decode_attention_13_b200.build`")
+        L = ctypes.CDLL(LIB_PATH)
+        L.mla_metadata_bytes.restype = ctypes.c_size_t
+        L.mla_metadata_bytes.argtypes = [ctypes.c_int] * 3
+        L.mla_workspace_bytes.restype = ctypes.c_size_t
+        L.mla_workspace_bytes.argtypes = [ctypes.c_int] * 3
+        L.mla_num_sm_pairs.restype = ctypes.c_int
+        L.mla_num_sm_pairs.argtypes = []
+        L.mla_get_metadata.restype = ctypes.c_int
+        L.mla_get_metadata.argtypes = [_vp, ctypes.c_int, ctypes.c_int, ctypes.c_int, _vp, _vp]
+        dec = [_vp, _vp, ctypes.c_int64, _vp, ctypes.c_int, _vp, ctypes.c_int, ctypes.c_int, ctypes.c_int,
+               ctypes.c_float, ctypes.c_int, _vp, _vp, _vp, _vp, ctypes.c_size_t, _vp]
+        L.mla_decode.restype = ctypes.c_int
+        L.mla_decode.argtypes = dec
+        L.mla_decode_timed.restype = ctypes.c_int
+        L.mla_decode_timed.argtypes = dec + [_vp, _vp]
+        L.mla_check_device_error.restype = ctypes.c_int
+        L.mla_check_device_error.argtypes = [_vp, _vp, ctypes.POINTER(ctypes.c_uint32)]
+        L.mla_error_string.restype = ctypes.c_char_p
+        L.mla_error_string.argtypes = [ctypes.c_int]
+        _lib = L
+    return _lib
+
+
+def mla_error_string(status: int) -> str:
+    return lib().mla_error_string(int(status)).decode()
+
+
+def mla_metadata_bytes(batch: int, h_q: int, s_q: int) -> int:
+    return int(lib().mla_metadata_bytes(batch, h_q, s_q))
+
+
+def mla_workspace_bytes(batch: int, h_q: int, s_q: int) -> int:
+    return int(lib().mla_workspace_bytes(batch, h_q, s_q))
+
+
+def mla_num_sm_pairs() -> int:
+    n = int(lib().mla_num_sm_pairs())
+    if n < 0:
+        raise MLAError("mla_num_sm_pairs", n)
+    return n
+
+
+def _stream_ptr(stream) -> Optional[int]:
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return int(stream.cuda_stream) if hasattr(stream, "cuda_stream") else int(stream)
+
+
+def _ptr(t: Optional[torch.Tensor]) -> Optional[int]:
+    return None if t is None else int(t.data_ptr())
+
+
+def _check(func: str, status: int) -> None:
+    if status != MLA_OK:
+        raise MLAError(func, status)
+
+
+def mla_get_metadata(seqlens: torch.Tensor, h_q: int, s_q: int, metadata: Optional[torch.Tensor] = None,
+                     stream=None) -> torch.Tensor:
+    """Split-KV plan for one decode step; returns the (device) metadata buffer."""
+    batch = int(seqlens.shape[0])
+    nbytes = mla_metadata_bytes(batch, h_q, s_q)
+    if nbytes == 0:
+        raise MLAError("mla_metadata_bytes", MLA_ERR_UNSUPPORTED)
+    if metadata is None:
+        metadata = torch.empty(nbytes // 4, dtype=torch.int32, device=seqlens.device)
+    _check("mla_get_metadata",
+           lib().mla_get_metadata(_ptr(seqlens), batch, h_q, s_q, _ptr(metadata), _stream_ptr(stream)))
+    return metadata
+
+
+def mla_decode(q: torch.Tensor, kv_cache: torch.Tensor, block_table: torch.Tensor, seqlens: torch.Tensor,
+               softmax_scale: float, causal: bool, metadata: torch.Tensor, workspace: Optional[torch.Tensor] = None,
+               out: Optional[torch.Tensor] = None, lse: Optional[torch.Tensor] = None, stream=None,
+               events: Optional[Tuple] = None) -> Tuple[torch.Tensor, torch.Tensor]:
+    """MLA decode; returns (out [b, s_q, h_q, 512] bf16, lse [b, h_q, s_q] fp32).
+
+    ``events`` = (before, after) torch.cuda.Event recorded around the split-KV
+    kernel (timing only).
+    """
+    batch, s_q, h_q, d = q.shape
+    if d != 576 or kv_cache.shape[-1] != 576 or q.dtype != torch.bfloat16 or kv_cache.dtype != torch.bfloat16:
+        raise MLAError("mla_decode", MLA_ERR_ARG)
+    for t in (q, kv_cache, block_table, seqlens):
+        if not t.is_contiguous():
+            raise MLAError("mla_decode", MLA_ERR_ARG)
+    if out is None:
+        out = torch.empty(batch, s_q, h_q, 512, dtype=torch.bfloat16, device=q.device)
+    if lse is None:
+        lse = torch.empty(batch, h_q, s_q, dtype=torch.float32, device=q.device)
+    if workspace is None:
+        workspace = torch.empty(max(mla_workspace_bytes(batch, h_q, s_q), 16), dtype=torch.uint8, device=q.device)
+    args = [_ptr(q), _ptr(kv_cache), int(kv_cache.shape[0]), _ptr(block_table), int(block_table.shape[1]),
+            _ptr(seqlens), batch, s_q, h_q, float(softmax_scale), int(bool(causal)), _ptr(out), _ptr(lse),
+            _ptr(metadata), _ptr(workspace), int(workspace.numel() * workspace.element_size()), _stream_ptr(stream)]
+    if events is None:
+        status = lib().mla_decode(*args)
+    else:
+        ev = []
+        for e in events:
+            if e is not None and int(e.cuda_event) == 0:
+                e.record()  # torch creates the CUDA event lazily, on first record
+            ev.append(None if e is None else int(e.cuda_event))
+        status = lib().mla_decode_timed(*args, *ev)
+    _check("mla_decode", status)
+    return out, lse
+
+
+def mla_check_device_error(metadata: torch.Tensor, stream=None) -> int:
+    """Synchronise and return the device error word (0 = no error)."""
+    word = ctypes.c_uint32(0)
+    status = lib().mla_check_device_error(_ptr(metadata), _stream_ptr(stream), ctypes.byref(word))
+    if status not in (MLA_OK, MLA_ERR_DEVICE):
+        raise MLAError("mla_check_device_error", status)
+    return int(word.value)

@@ -1,0 +1,250 @@
+// Host side of the C ABI declared in include/mla_b200.h: argument checks,
+// TMA tensor-map encoding, per-device launch geometry, and the launches.
+#include <cudaTypedefs.h>
+
+#include <cmath>
+#include <mutex>
+
+#include "mla_internal.h"
+
+#define MLA_API extern "C" __attribute__((visibility("default")))
+
+namespace mla {
+namespace {
+
+constexpr int kMaxDevices = 64;
+
+struct DeviceInfo {
+  int pairs = 0;  // co-resident 2-CTA clusters of the decode kernel
+  int sms = 0;
+  bool ready = false;
+};
+
+std::mutex g_mu;
+DeviceInfo g_dev[kMaxDevices];
+PFN_cuTensorMapEncodeTiled_v12000 g_encode = nullptr;
+
+int current_device_info(DeviceInfo* out) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) {
+    cudaGetLastError();
+    return MLA_ERR_CUDA;
+  }
+  if (dev < 0 || dev >= kMaxDevices) return MLA_ERR_UNSUPPORTED;
+  std::lock_guard<std::mutex> lock(g_mu);
+  DeviceInfo& d = g_dev[dev];
+  if (!d.ready) {
+    int major = 0;
+    if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess) return MLA_ERR_CUDA;
+    if (major != 10) return MLA_ERR_UNSUPPORTED;  // built for sm_100a only
+    if (cudaDeviceGetAttribute(&d.sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return MLA_ERR_CUDA;
+    if (decode_kernel_pairs(&d.pairs) != cudaSuccess) {
+      cudaGetLastError();
+      return MLA_ERR_CUDA;
+    }
+    if (d.pairs < 1) return MLA_ERR_UNSUPPORTED;
+    d.ready = true;
+  }
+  *out = d;
+  return MLA_OK;
+}
+
+int tensor_map_encoder(PFN_cuTensorMapEncodeTiled_v12000* fn) {
+  std::lock_guard<std::mutex> lock(g_mu);
+  if (!g_encode) {
+    void* ptr = nullptr;
+    cudaDriverEntryPointQueryResult q = cudaDriverEntryPointSymbolNotFound;
+    const cudaError_t e = cudaGetDriverEntryPointByVersion("cuTensorMapEncodeTiled", &ptr, 12000, cudaEnableDefault, &q);
+    if (e != cudaSuccess || q != cudaDriverEntryPointSuccess || ptr == nullptr) {
+      cudaGetLastError();
+      return MLA_ERR_CUDA;
+    }
+    g_encode = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(ptr);
+  }
+  *fn = g_encode;
+  return MLA_OK;
+}
+
+// A [rows][576] bf16 row-major tensor, tiled in boxes of box_cols x box_rows.
+int encode_rows576(PFN_cuTensorMapEncodeTiled_v12000 enc, CUtensorMap* map, const void* base, uint64_t rows,
+                   uint32_t box_cols, uint32_t box_rows, CUtensorMapSwizzle swizzle) {
+  const cuuint64_t dims[2] = {static_cast<cuuint64_t>(kDqk), static_cast<cuuint64_t>(rows)};
+  const cuuint64_t strides[1] = {static_cast<cuuint64_t>(kDqk) * 2};
+  const cuuint32_t box[2] = {box_cols, box_rows};
+  const cuuint32_t elem[2] = {1, 1};
+  const CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box, elem,
+                         CU_TENSOR_MAP_INTERLEAVE_NONE, swizzle, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                         CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS ? MLA_OK : MLA_ERR_CUDA;
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+bool shape_ok(int batch, int h_q, int s_q) {
+  return batch >= 1 && h_q >= 1 && h_q <= kMaxHq && s_q >= 1 && s_q <= kMaxSq &&
+         static_cast<long long>(batch) * s_q * h_q <= (1LL << 30);
+}
+
+int decode_impl(const void* q, const void* kv_cache, int64_t num_pages, const int32_t* block_table,
+                int max_pages_per_seq, const int32_t* seqlens, int batch, int s_q, int h_q, float softmax_scale,
+                int causal, void* out, float* lse, void* metadata, void* workspace, size_t workspace_bytes,
+                void* stream, void* ev_before, void* ev_after) {
+  if (!q || !kv_cache || !block_table || !seqlens || !out || !lse || !metadata) return MLA_ERR_ARG;
+  if (batch < 1 || h_q < 1 || s_q < 1 || max_pages_per_seq < 1 || num_pages < 1) return MLA_ERR_ARG;
+  if (causal != 0 && causal != 1) return MLA_ERR_ARG;
+  if (!std::isfinite(softmax_scale)) return MLA_ERR_ARG;
+  if (!aligned16(q) || !aligned16(kv_cache) || !aligned16(out) || !aligned16(metadata)) return MLA_ERR_ARG;
+  if (workspace && !aligned16(workspace)) return MLA_ERR_ARG;
+  if (!shape_ok(batch, h_q, s_q)) return MLA_ERR_UNSUPPORTED;
+  if (num_pages > (1LL << 25)) return MLA_ERR_UNSUPPORTED;  // row coordinates stay below 2^31
+
+  DeviceInfo dev;
+  int st = current_device_info(&dev);
+  if (st != MLA_OK) return st;
+  const size_t need = workspace_bytes_for(dev.pairs, h_q, s_q);
+  if (workspace_bytes < need || (need > 0 && workspace == nullptr)) return MLA_ERR_WORKSPACE;
+  PFN_cuTensorMapEncodeTiled_v12000 enc = nullptr;
+  if ((st = tensor_map_encoder(&enc)) != MLA_OK) return st;
+
+  const int R = s_q * h_q;
+  const int tr = tile_rows(h_q, s_q);
+  const int slots = max_slots(dev.pairs);
+  DecodeParams p;
+  const uint64_t kv_rows = static_cast<uint64_t>(num_pages) * kPage;
+  const uint64_t q_rows = static_cast<uint64_t>(batch) * R;
+  if ((st = encode_rows576(enc, &p.tm_kv_lat, kv_cache, kv_rows, 64, kPage, CU_TENSOR_MAP_SWIZZLE_128B)) != MLA_OK ||
+      (st = encode_rows576(enc, &p.tm_kv_rope, kv_cache, kv_rows, 32, kPage, CU_TENSOR_MAP_SWIZZLE_64B)) != MLA_OK ||
+      (st = encode_rows576(enc, &p.tm_q_lat, q, q_rows, 64, static_cast<uint32_t>(tr), CU_TENSOR_MAP_SWIZZLE_128B)) !=
+          MLA_OK ||
+      (st = encode_rows576(enc, &p.tm_q_rope, q, q_rows, 32, static_cast<uint32_t>(tr), CU_TENSOR_MAP_SWIZZLE_64B)) !=
+          MLA_OK)
+    return st;
+  p.block_table = block_table;
+  p.seqlens = seqlens;
+  p.out = out;
+  p.lse = lse;
+  p.o_part = static_cast<float*>(workspace);
+  p.lse_part = workspace ? static_cast<float*>(workspace) + static_cast<size_t>(slots) * tr * kDv : nullptr;
+  p.meta = static_cast<int32_t*>(metadata);
+  p.num_pages = num_pages;
+  p.max_pages = max_pages_per_seq;
+  p.batch = batch;
+  p.s_q = s_q;
+  p.h_q = h_q;
+  p.R = R;
+  p.n_mt = ceil_div(R, kMTile);
+  p.causal = causal;
+  p.q_box_rows = tr;
+  p.tile_rows = tr;
+  p.max_slots = slots;
+  p.scale_log2 = softmax_scale * 1.4426950408889634f;
+
+  CombineParams cp;
+  cp.meta = static_cast<const int32_t*>(metadata);
+  cp.o_part = p.o_part;
+  cp.lse_part = p.lse_part;
+  cp.out = out;
+  cp.lse = lse;
+  cp.batch = batch;
+  cp.s_q = s_q;
+  cp.h_q = h_q;
+  cp.R = R;
+  cp.tile_rows = tr;
+  cp.pairs = dev.pairs;
+  cp.max_slots = slots;
+
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  if (ev_before && cudaEventRecord(static_cast<cudaEvent_t>(ev_before), s) != cudaSuccess) return MLA_ERR_CUDA;
+  if (launch_decode(p, dev.pairs, s) != cudaSuccess) return MLA_ERR_CUDA;
+  if (ev_after && cudaEventRecord(static_cast<cudaEvent_t>(ev_after), s) != cudaSuccess) return MLA_ERR_CUDA;
+  if (launch_combine(cp, 2 * dev.sms, s) != cudaSuccess) return MLA_ERR_CUDA;
+  return MLA_OK;
+}
+
+}  // namespace
+}  // namespace mla
+
+using namespace mla;
+
+MLA_API size_t mla_metadata_bytes(int batch, int h_q, int s_q) {
+  if (!shape_ok(batch, h_q, s_q)) return 0;
+  return meta_layout(batch, h_q, s_q).words * sizeof(int32_t);
+}
+
+MLA_API size_t mla_workspace_bytes(int batch, int h_q, int s_q) {
+  if (!shape_ok(batch, h_q, s_q)) return 0;
+  DeviceInfo dev;
+  if (current_device_info(&dev) != MLA_OK) return workspace_bytes_for(kMaxPairs, h_q, s_q);
+  return workspace_bytes_for(dev.pairs, h_q, s_q);
+}
+
+MLA_API int mla_num_sm_pairs(void) {
+  DeviceInfo dev;
+  const int st = current_device_info(&dev);
+  return st == MLA_OK ? dev.pairs : st;
+}
+
+MLA_API int mla_get_metadata(const int32_t* seqlens, int batch, int h_q, int s_q, void* metadata, void* stream) {
+  if (!seqlens || !metadata) return MLA_ERR_ARG;
+  if (batch < 1 || h_q < 1 || s_q < 1) return MLA_ERR_ARG;
+  if (!aligned16(metadata)) return MLA_ERR_ARG;
+  if (!shape_ok(batch, h_q, s_q)) return MLA_ERR_UNSUPPORTED;
+  DeviceInfo dev;
+  const int st = current_device_info(&dev);
+  if (st != MLA_OK) return st;
+  if (launch_sched(seqlens, batch, h_q, s_q, dev.pairs, static_cast<int32_t*>(metadata),
+                   static_cast<cudaStream_t>(stream)) != cudaSuccess)
+    return MLA_ERR_CUDA;
+  return MLA_OK;
+}
+
+MLA_API int mla_decode(const void* q, const void* kv_cache, int64_t num_pages, const int32_t* block_table,
+                       int max_pages_per_seq, const int32_t* seqlens, int batch, int s_q, int h_q, float softmax_scale,
+                       int causal, void* out, float* lse, void* metadata, void* workspace, size_t workspace_bytes,
+                       void* stream) {
+  return decode_impl(q, kv_cache, num_pages, block_table, max_pages_per_seq, seqlens, batch, s_q, h_q, softmax_scale,
+                     causal, out, lse, metadata, workspace, workspace_bytes, stream, nullptr, nullptr);
+}
+
+MLA_API int mla_decode_timed(const void* q, const void* kv_cache, int64_t num_pages, const int32_t* block_table,
+                             int max_pages_per_seq, const int32_t* seqlens, int batch, int s_q, int h_q,
+                             float softmax_scale, int causal, void* out, float* lse, void* metadata, void* workspace,
+                             size_t workspace_bytes, void* stream, void* event_before_decode,
+                             void* event_after_decode) {
+  return decode_impl(q, kv_cache, num_pages, block_table, max_pages_per_seq, seqlens, batch, s_q, h_q, softmax_scale,
+                     causal, out, lse, metadata, workspace, workspace_bytes, stream, event_before_decode,
+                     event_after_decode);
+}
+
+MLA_API int mla_check_device_error(const void* metadata, void* stream, uint32_t* error_word) {
+  if (!metadata) return MLA_ERR_ARG;
+  uint32_t word = 0;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  if (cudaMemcpyAsync(&word, static_cast<const int32_t*>(metadata) + kHError, sizeof(word), cudaMemcpyDeviceToHost,
+                      s) != cudaSuccess ||
+      cudaStreamSynchronize(s) != cudaSuccess) {
+    cudaGetLastError();
+    return MLA_ERR_CUDA;
+  }
+  if (error_word) *error_word = word;
+  return word == 0 ? MLA_OK : MLA_ERR_DEVICE;
+}
+
+MLA_API const char* mla_error_string(int status) {
+  switch (status) {
+    case MLA_OK:
+      return "ok";
+    case MLA_ERR_ARG:
+      return "invalid argument (null pointer, bad size or misaligned pointer)";
+    case MLA_ERR_UNSUPPORTED:
+      return "unsupported shape or device";
+    case MLA_ERR_CUDA:
+      return "CUDA runtime or driver call failed";
+    case MLA_ERR_WORKSPACE:
+      return "workspace smaller than mla_workspace_bytes()";
+    case MLA_ERR_DEVICE:
+      return "device error word set (see MLA_DEVERR_* bits)";
+    default:
+      return "unknown status";
+  }
+}

@@ -1,0 +1,128 @@
+// Internal layout shared by the host code and the three kernels of the
+// decode path: the metadata (tile-scheduler plan) word layout, the workspace
+// layout, and the kernels' launch entry points.
+#pragma once
+
+#include <cstddef>
+#include <cstdint>
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include "mla_b200.h"
+
+namespace mla {
+
+constexpr int kDqk = 576;
+constexpr int kDv = 512;
+constexpr int kPage = 64;
+constexpr int kMTile = 128;       // query rows per work row (UMMA M)
+constexpr int kMaxPairs = 160;    // upper bound on SM pairs of any sm_100 part
+constexpr int kMaxHq = 128;
+constexpr int kMaxSq = 16;
+constexpr int kKappa = 2;         // fixed per-piece cost of the plan, in pages
+constexpr uint32_t kMagic = 0x314C4D42u;  // "BML1"
+
+// ---------------------------------------------------------------------------
+// Metadata: int32 words.
+//   header [kHdrWords]
+//   pair_off  [kMaxPairs + 1]           segment range of each pair
+//   segs      [W + kMaxPairs][4]        (work row, first page, end page, slot)
+//   row_info  [W][2]                    (first slot or -1, pieces)
+//   split_rows [W]                      work rows cut into >1 pieces
+//   empty_rows [W]                      work rows with no pages
+// A work row is (batch row i, m-tile mt) with index w = mt * batch + i.
+// ---------------------------------------------------------------------------
+enum HeaderWord : int {
+  kHMagic = 0,
+  kHError = 1,
+  kHPairs = 2,
+  kHWorkRows = 3,
+  kHSegments = 4,
+  kHSlots = 5,
+  kHRows = 6,      // R = s_q * h_q
+  kHMTiles = 7,
+  kHBatch = 8,
+  kHKappa = 9,
+  kHSplitRows = 10,
+  kHEmptyRows = 11,
+  kHHq = 12,
+  kHSq = 13,
+  kHCap = 14,
+  kHdrWords = 32,
+};
+
+struct MetaLayout {
+  int W;
+  size_t pair_off, segs, row_info, split_rows, empty_rows, words;
+};
+
+__host__ __device__ inline int ceil_div(int a, int b) { return (a + b - 1) / b; }
+
+__host__ __device__ inline MetaLayout meta_layout(int batch, int h_q, int s_q) {
+  MetaLayout L;
+  L.W = batch * ceil_div(s_q * h_q, kMTile);
+  L.pair_off = kHdrWords;
+  L.segs = (L.pair_off + kMaxPairs + 1 + 3) & ~size_t(3);
+  L.row_info = L.segs + size_t(4) * (L.W + kMaxPairs);
+  L.split_rows = L.row_info + size_t(2) * L.W;
+  L.empty_rows = L.split_rows + L.W;
+  L.words = L.empty_rows + L.W;
+  return L;
+}
+
+// Rows of a work row that hold real query rows: min(R, 128).
+__host__ __device__ inline int tile_rows(int h_q, int s_q) {
+  int R = s_q * h_q;
+  return R < kMTile ? R : kMTile;
+}
+
+// Workspace: o_part [slots][tile_rows][512] fp32, then lse_part [slots][tile_rows].
+// A plan over P pairs cuts rows at most P - 1 times, and every cut row has one
+// more piece than cuts, so at most 2 (P - 1) slots are used.
+__host__ __device__ inline int max_slots(int pairs) { return pairs > 1 ? 2 * (pairs - 1) : 0; }
+
+__host__ __device__ inline size_t workspace_bytes_for(int pairs, int h_q, int s_q) {
+  size_t rows = size_t(max_slots(pairs)) * tile_rows(h_q, s_q);
+  return rows * (kDv + 1) * sizeof(float);
+}
+
+// ---------------------------------------------------------------------------
+// Split-KV decode kernel parameters.
+// ---------------------------------------------------------------------------
+struct DecodeParams {
+  CUtensorMap tm_kv_lat;   // cache as [num_pages*64][576]: box 64 cols x 64 rows, 128B swizzle
+  CUtensorMap tm_kv_rope;  // same tensor: box 32 cols x 64 rows, 64B swizzle
+  CUtensorMap tm_q_lat;    // q as [batch*R][576]: box 64 cols x min(R,128) rows, 128B swizzle
+  CUtensorMap tm_q_rope;   // same tensor: box 32 cols x min(R,128) rows, 64B swizzle
+  const int32_t* block_table;
+  const int32_t* seqlens;
+  void* out;               // bf16
+  float* lse;
+  float* o_part;
+  float* lse_part;
+  int32_t* meta;
+  long long num_pages;
+  int max_pages;
+  int batch, s_q, h_q, R, n_mt, causal, q_box_rows, tile_rows, max_slots;
+  float scale_log2;        // softmax_scale * log2(e)
+};
+
+struct CombineParams {
+  const int32_t* meta;
+  const float* o_part;
+  const float* lse_part;
+  void* out;
+  float* lse;
+  int batch, s_q, h_q, R, tile_rows, pairs, max_slots;
+};
+
+// Launch wrappers (each returns a cudaError_t).
+cudaError_t launch_sched(const int32_t* seqlens, int batch, int h_q, int s_q, int pairs, int32_t* meta,
+                         cudaStream_t stream);
+cudaError_t decode_kernel_prepare();
+cudaError_t decode_kernel_pairs(int* pairs);
+size_t decode_kernel_smem_bytes();
+cudaError_t launch_decode(const DecodeParams& p, int pairs, cudaStream_t stream);
+cudaError_t launch_combine(const CombineParams& p, int grid, cudaStream_t stream);
+
+}  // namespace mla

@@ -86,12 +86,20 @@ def token_location(j: np.ndarray) -> Tuple[np.ndarray, np.ndarray]:
     return j // PAGE, j % PAGE
 
 
-def depage(kv_pool: np.ndarray, table_row: np.ndarray, length: int) -> np.ndarray:
-    """Gather the first ``length`` cache rows of one sequence: [length, 576]."""
+def depage(kv_pool, table_row: np.ndarray, length: int) -> np.ndarray:
+    """Gather the first ``length`` cache rows of one sequence: [length, 576] float64.
+
+    ``kv_pool`` may be a float array or a (bf16) torch tensor; only the rows
+    gathered are converted.
+    """
     j = np.arange(length, dtype=np.int64)
     page, slot = token_location(j)
     phys = table_row[page]
-    return kv_pool[phys, slot, 0, :]
+    if hasattr(kv_pool, "detach"):
+        import torch  # local: the oracle itself does not need torch
+
+        return as_f64(kv_pool[torch.from_numpy(phys), torch.from_numpy(slot), 0, :])
+    return np.asarray(kv_pool[phys, slot, 0, :], dtype=np.float64)
 
 
 def key_of(rows: np.ndarray) -> np.ndarray:
@@ -169,7 +177,7 @@ def decode(q, kv_cache, block_table, seqlens, softmax_scale: float, causal: bool
     the work to those batch rows (the others stay zero / -inf).
     """
     q = as_f64(q)
-    pool = as_f64(kv_cache)
+    pool = kv_cache if hasattr(kv_cache, "detach") else as_f64(kv_cache)
     table = as_int(block_table)
     lens = as_int(seqlens)
     batch, s_q, h_q, _ = q.shape
