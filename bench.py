@@ -391,8 +391,19 @@ def ours(args, world, rank, local):
     ms_total = start.elapsed_time(end)
     ms_total = max_over_ranks(ms_total, world, dev)
     ms_step = ms_total / K
-    k2_ms = [a.elapsed_time(b) for a, b in ev_pairs] if reps > 0 else []
-    k2_avg_ms = sum(k2_ms) / len(k2_ms) if k2_ms else float("nan")
+    k2_source = "events around the split-KV kernel inside the timed graphs (last cycle)"
+    try:
+        k2_ms = [a.elapsed_time(b) for a, b in ev_pairs] if reps > 0 else []
+    except Exception:
+        k2_ms = []
+    if not k2_ms:
+        # Eager launches with the same events, right after the timed region.
+        k2_source = "events around the split-KV kernel, eager launches after the timed region"
+        for r in range(npool):
+            step(r, events=ev_pairs[r])
+        stream.synchronize()
+        k2_ms = [a.elapsed_time(b) for a, b in ev_pairs]
+    k2_avg_ms = sum(k2_ms) / len(k2_ms)
     for m in metas:
         err = binding.mla_check_device_error(m, stream=stream)
         if err:
@@ -464,6 +475,7 @@ def ours(args, world, rank, local):
             "algorithmic_bytes_per_launch": nbytes,
             "peak_source": f"{peak_kind} hbm_gbs",
             "tensor_frac_of_measured_bf16": round(flops / k2_s / 1e12 / tf_peak, 4) if k2_s > 0 else None,
+            "timing": k2_source,
         },
         "e2e": {"value": round(e2e_ms * 1e3, 3), "unit": "us/call", "h2d_bytes_per_step": h2d,
                 "d2h_bytes_per_step": d2h, "steps": e2e_steps,

@@ -123,7 +123,7 @@ int mla_get_metadata(const int32_t* seqlens, int batch, int h_q, int s_q, void* 
  *                row's ceil(L_i / 64) pages are never read.
  *   seqlens      [device] int32 [batch], 0 <= L_i <= 64 * max_pages_per_seq;
  *                must hold the values the metadata was built from.
- *   softmax_scale  multiplies <q, k>; finite.
+ *   softmax_scale  multiplies <q, k>; finite and >= 0.
  *   causal       0 or 1 (see the header comment).
  *   out          [device] bf16 [batch][s_q][h_q][512], 16-byte aligned.
  *   lse          [device] fp32 [batch][h_q][s_q]: natural log of

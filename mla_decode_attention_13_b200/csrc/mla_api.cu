@@ -92,7 +92,7 @@ int decode_impl(const void* q, const void* kv_cache, int64_t num_pages, const in
   if (!q || !kv_cache || !block_table || !seqlens || !out || !lse || !metadata) return MLA_ERR_ARG;
   if (batch < 1 || h_q < 1 || s_q < 1 || max_pages_per_seq < 1 || num_pages < 1) return MLA_ERR_ARG;
   if (causal != 0 && causal != 1) return MLA_ERR_ARG;
-  if (!std::isfinite(softmax_scale)) return MLA_ERR_ARG;
+  if (!std::isfinite(softmax_scale) || softmax_scale < 0.0f) return MLA_ERR_ARG;
   if (!aligned16(q) || !aligned16(kv_cache) || !aligned16(out) || !aligned16(metadata)) return MLA_ERR_ARG;
   if (workspace && !aligned16(workspace)) return MLA_ERR_ARG;
   if (!shape_ok(batch, h_q, s_q)) return MLA_ERR_UNSUPPORTED;
@@ -112,12 +112,9 @@ int decode_impl(const void* q, const void* kv_cache, int64_t num_pages, const in
   DecodeParams p;
   const uint64_t kv_rows = static_cast<uint64_t>(num_pages) * kPage;
   const uint64_t q_rows = static_cast<uint64_t>(batch) * R;
-  if ((st = encode_rows576(enc, &p.tm_kv_lat, kv_cache, kv_rows, 64, kPage, CU_TENSOR_MAP_SWIZZLE_128B)) != MLA_OK ||
-      (st = encode_rows576(enc, &p.tm_kv_rope, kv_cache, kv_rows, 32, kPage, CU_TENSOR_MAP_SWIZZLE_64B)) != MLA_OK ||
-      (st = encode_rows576(enc, &p.tm_q_lat, q, q_rows, 64, static_cast<uint32_t>(tr), CU_TENSOR_MAP_SWIZZLE_128B)) !=
-          MLA_OK ||
-      (st = encode_rows576(enc, &p.tm_q_rope, q, q_rows, 32, static_cast<uint32_t>(tr), CU_TENSOR_MAP_SWIZZLE_64B)) !=
-          MLA_OK)
+  if ((st = encode_rows576(enc, &p.tm_k, kv_cache, kv_rows, 64, kPage / 2, CU_TENSOR_MAP_SWIZZLE_128B)) != MLA_OK ||
+      (st = encode_rows576(enc, &p.tm_v, kv_cache, kv_rows, 64, kPage, CU_TENSOR_MAP_SWIZZLE_128B)) != MLA_OK ||
+      (st = encode_rows576(enc, &p.tm_q, q, q_rows, 64, kMTile / 2, CU_TENSOR_MAP_SWIZZLE_128B)) != MLA_OK)
     return st;
   p.block_table = block_table;
   p.seqlens = seqlens;
@@ -134,7 +131,6 @@ int decode_impl(const void* q, const void* kv_cache, int64_t num_pages, const in
   p.R = R;
   p.n_mt = ceil_div(R, kMTile);
   p.causal = causal;
-  p.q_box_rows = tr;
   p.tile_rows = tr;
   p.max_slots = slots;
   p.scale_log2 = softmax_scale * 1.4426950408889634f;
@@ -154,9 +150,19 @@ int decode_impl(const void* q, const void* kv_cache, int64_t num_pages, const in
   cp.max_slots = slots;
 
   cudaStream_t s = static_cast<cudaStream_t>(stream);
-  if (ev_before && cudaEventRecord(static_cast<cudaEvent_t>(ev_before), s) != cudaSuccess) return MLA_ERR_CUDA;
+  // Inside a stream capture the events must become event-record nodes of the
+  // graph (external events), or they would never be recorded at replay.
+  unsigned int ev_flags = cudaEventRecordDefault;
+  if (ev_before || ev_after) {
+    cudaStreamCaptureStatus cs = cudaStreamCaptureStatusNone;
+    if (cudaStreamIsCapturing(s, &cs) != cudaSuccess) return MLA_ERR_CUDA;
+    if (cs == cudaStreamCaptureStatusActive) ev_flags = cudaEventRecordExternal;
+  }
+  if (ev_before && cudaEventRecordWithFlags(static_cast<cudaEvent_t>(ev_before), s, ev_flags) != cudaSuccess)
+    return MLA_ERR_CUDA;
   if (launch_decode(p, dev.pairs, s) != cudaSuccess) return MLA_ERR_CUDA;
-  if (ev_after && cudaEventRecord(static_cast<cudaEvent_t>(ev_after), s) != cudaSuccess) return MLA_ERR_CUDA;
+  if (ev_after && cudaEventRecordWithFlags(static_cast<cudaEvent_t>(ev_after), s, ev_flags) != cudaSuccess)
+    return MLA_ERR_CUDA;
   if (launch_combine(cp, 2 * dev.sms, s) != cudaSuccess) return MLA_ERR_CUDA;
   return MLA_OK;
 }

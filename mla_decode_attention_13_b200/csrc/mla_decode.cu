@@ -3,38 +3,43 @@
 // What it computes: for every query row (batch row i, query token t, head h)
 // the absorbed-form attention over that row's cached latent tokens ("MLA 和
 // MHA 的 Kernel 区别", sections "MLA Decode" and "MLA 的 FlashAttention": load
-// each latent tile from HBM once, decompress/score it on chip, reuse it for
-// every head).  Scores use all 576 dims of a cached row (512 latent + 64
-// rope); values are the first 512 dims of the same row, so every cached tile
-// is read once and serves as both K and V.
+// each latent tile from HBM once, score it on chip, reuse it for every head).
+// Scores use all 576 dims of a cached row (512 latent + 64 rope); values are
+// the first 512 dims of the same row.
 //
-// How, per SM pair (one 2-CTA cluster, persistent over the plan's segments):
-//   * The 576 columns are split between the two CTAs: CTA c owns latent
-//     columns [256c, 256c + 256) and rope columns [512 + 32c, 512 + 32c + 32).
-//     Each CTA TMA-loads only its 288 columns of every 64-token page, so each
-//     cache byte leaves HBM once.  Pages are gathered through the block table
-//     ("FlashMLA overview": paged kvcache, block size 64).
-//   * QK^T: each CTA computes a partial S = Q[:, own cols] K[:, own cols]^T on
-//     tcgen05 (M = 128 query rows, N = 64 tokens, 18 K-steps of 16) into TMEM.
-//     The two partials are exchanged through distributed shared memory
-//     (st.async with mbarrier byte counts) and added; both CTAs then hold the
-//     same S and run the same online softmax (one thread per query row).
-//   * PV: P (bf16, 128 x 64, written to shared memory in the 128-byte swizzled
-//     K-major layout) times V (the CTA's 256 latent columns of the same tile,
-//     read MN-major) accumulates into O (128 x 256 fp32) in TMEM.  Per SM the
-//     TMEM holds O (256 columns) and two S buffers (2 x 64 columns).
-//   * Online softmax with a lazy rescale: the running max only moves when a
-//     block's max exceeds it by more than kTau (log2 units); O and the running
-//     sum are rescaled together, so the result is exact.
-//   * A row that the plan splits writes fp32 (O / l, lse) partials to the
-//     workspace for the combine kernel; an unsplit row writes bf16 out and lse.
+// How: one persistent 2-CTA cluster per SM pair walks the plan's segments.
+// The pair works on a tile of 128 query rows (a work row); CTA c owns query
+// rows [64c, 64c + 64).  Both products run as pair MMAs (tcgen05.mma
+// cta_group::2, M = 128), issued by the leader CTA: each CTA supplies its 64
+// rows of the A operand and half of the B operand's columns from its own
+// shared memory at the same offsets; the tensor cores share the B halves, and
+// each CTA's 64 rows of the result land in its own TMEM spread over all 128
+// lanes (lanes 0-63 hold the first N/2 columns, lanes 64-127 the rest).
+//   * QK^T: A = Q (64 rows x 576, shared memory, loaded once per segment),
+//     B = the page's cache rows: CTA c TMA-loads tokens [32c, 32c + 32) of each
+//     64-token page, all 576 columns, so the page's keys are read once for
+//     the pair.  S (64 rows x 64 tokens per CTA) lands in 32 TMEM columns:
+//     lane r < 64 holds tokens 0-31 of row r, lane r + 64 tokens 32-63.
+//   * Softmax: thread r (= TMEM lane r) handles row r mod 64, 32 tokens; the
+//     two threads of a row trade their block maxima through shared memory.
+//     Online softmax in the log2 domain with a lazy rescale (the running max
+//     only moves when a block's max exceeds it by more than kTau; O and the
+//     running sums are rescaled together, so the result is exact).  The
+//     bf16-rounded weights P go to shared memory (A operand of PV); the
+//     normaliser and lse use their unrounded fp32 sum.
+//   * PV: O (64 rows x 512 per CTA, 256 TMEM columns) += P V in two MMAs of
+//     N = 256; for each, CTA c supplies latent columns [128c, 128c + 128) of
+//     that half for all 64 tokens (its own TMA load of the page's V columns).
+//   Pages are gathered through the block table ("FlashMLA overview": paged
+//   kvcache, block size 64); the producer warp reads page ids 32 at a time.
+// A row the plan splits writes fp32 (O / l, lse) partials to the workspace
+// for the combine kernel; an unsplit row writes bf16 out and lse.
 // Warp roles per CTA (256 threads): warp 0 = TMA producer, warp 1 = TMEM
-// owner and UMMA issuer, warps 4-7 = softmax + epilogue (one thread per query
-// row / TMEM lane), warps 2-3 idle.
+// owner and (leader only) MMA issuer, warps 4-7 = softmax and epilogue.
 //
 // Every mbarrier wait is bounded by %globaltimer; on expiry the kernel sets
 // MLA_DEVERR_TIMEOUT in the metadata error word, tells the peer CTA to stop,
-// drains its own copies and MMAs, frees TMEM and returns.
+// drains its own MMAs, frees TMEM and returns.
 #include <cuda_bf16.h>
 
 #include "mla_internal.h"
@@ -49,59 +54,64 @@ constexpr int kThreads = 256;
 constexpr int kStages = 2;
 constexpr float kTau = 8.0f;  // lazy-rescale threshold, log2 units
 constexpr uint64_t kTimeoutNs = 500ull * 1000ull * 1000ull;
+constexpr int kRowsCta = kMTile / 2;  // 64 query rows per CTA
 
-// Shared-memory layout (offsets from a 1024-byte aligned base).
-constexpr uint32_t kQPanel = kMTile * 128;                // 128 rows x 64 bf16 (128B swizzle)
-constexpr uint32_t kQRope = kMTile * 64;                  // 128 rows x 32 bf16 (64B swizzle)
-constexpr uint32_t kQBytes = 4 * kQPanel + kQRope;        // 73728
-constexpr uint32_t kKvPanel = kPage * 128;                // 64 tokens x 64 bf16
-constexpr uint32_t kKvRope = kPage * 64;                  // 64 tokens x 32 bf16
-constexpr uint32_t kStageBytes = 4 * kKvPanel + kKvRope;  // 36864
-constexpr uint32_t kPBytes = kMTile * 128;                // 128 rows x 64 bf16
-constexpr uint32_t kXBytes = kMTile * 64 * 4;             // 128 rows x 64 fp32
+// Shared-memory layout (offsets from a 1024-byte aligned base).  All operand
+// tiles are 128-byte swizzled panels of 64 bf16 columns.
+constexpr uint32_t kQPanel = kRowsCta * 128;               // 64 rows x 64 cols
+constexpr uint32_t kQBytes = 9 * kQPanel;                  // 576 cols
+constexpr uint32_t kKPanel = (kPage / 2) * 128;            // 32 tokens x 64 cols
+constexpr uint32_t kKBytes = 9 * kKPanel;                  // this CTA's 32 tokens, 576 cols
+constexpr uint32_t kVPanel = kPage * 128;                  // 64 tokens x 64 cols
+constexpr uint32_t kVBytes = 4 * kVPanel;                  // 64 tokens x this CTA's 256 V cols
+constexpr uint32_t kStageBytes = kKBytes + kVBytes;        // 69632
+constexpr uint32_t kPBytes = kRowsCta * 128;               // 64 rows x 64 tokens bf16
 constexpr uint32_t kOffQ = 0;
-constexpr uint32_t kOffKv = kOffQ + kQBytes;
-constexpr uint32_t kOffP = kOffKv + kStages * kStageBytes;
-constexpr uint32_t kOffX = kOffP + kPBytes;
-constexpr uint32_t kOffBar = kOffX + kXBytes;
+constexpr uint32_t kOffStage = kOffQ + kQBytes;
+constexpr uint32_t kOffP = kOffStage + kStages * kStageBytes;
+constexpr uint32_t kOffMax = kOffP + kPBytes;               // float [2][128]
+constexpr uint32_t kOffBar = kOffMax + 2 * 128 * 4;
 constexpr uint32_t kSmemUsed = kOffBar + 256;
 constexpr uint32_t kSmemBytes = kSmemUsed + 1024;  // slack for aligning the base
 
 enum Bar : uint32_t {
-  kBarKvFull = 0,   // [2] TMA -> MMA (tx bytes)
-  kBarKvEmpty = 2,  // [2] MMA commit -> TMA
-  kBarQFull = 4,
-  kBarQEmpty = 5,
-  kBarSFull = 6,    // [2] MMA commit -> softmax
-  kBarSEmpty = 8,   // [2] softmax (4 warps) -> MMA
-  kBarPFull = 10,   // softmax (4 warps) -> MMA
-  kBarPvDone = 11,  // MMA commit -> softmax
-  kBarXFull = 12,   // peer st.async bytes + own expect_tx
-  kBarXEmpty = 13,  // peer's 4 softmax warps -> me
-  kBarOEmpty = 14,  // softmax (4 warps) -> MMA
-  kBarFinal = 15,   // MMA drain at teardown
-  kNumBars = 16,
+  kBarKFull = 0,                  // [kStages] (leader) both CTAs' key halves landed
+  kBarVFull = kStages,            // [kStages] (leader) both CTAs' V columns landed
+  kBarStageEmpty = 2 * kStages,   // [kStages] (both) pair MMAs done with the stage
+  kBarQFull = 3 * kStages,        // (leader) both CTAs' Q rows landed
+  kBarQEmpty = 3 * kStages + 1,   // (both) last QK of the segment done
+  kBarSFull = 3 * kStages + 2,    // [2] (both) S buffer written
+  kBarSEmpty = 3 * kStages + 4,   // [2] (leader) 8 softmax warps read it
+  kBarPFull = 3 * kStages + 6,    // (leader) 8 warps wrote P and rescaled O
+  kBarPvDone = 3 * kStages + 7,   // (both) PV done
+  kBarOEmpty = 3 * kStages + 8,   // (leader) 8 warps read O out
+  kBarFinal = 3 * kStages + 9,    // (leader) MMA drain at teardown
+  kBarXMax = 3 * kStages + 10,    // (both) 4 softmax warps published their row maxima / sums
+  kNumBars = 3 * kStages + 11,
 };
 constexpr uint32_t kOffTmemSlot = kOffBar + 8 * kNumBars;  // u32
 constexpr uint32_t kOffAbort = kOffTmemSlot + 4;           // u32
+static_assert(kOffAbort + 4 <= kSmemUsed, "barrier area");
+static_assert(kSmemBytes <= 232448, "shared memory budget");
 
+// Tensor-memory columns (per CTA; the pair allocation mirrors them).
 constexpr uint32_t kTmemCols = 512;
-constexpr uint32_t kColO = 0;
-constexpr uint32_t kColS = 256;
+constexpr uint32_t kColO = 0;    // 256: lanes 0-63 / 64-127 hold the two column halves of each N=256 product
+constexpr uint32_t kColS = 256;  // 2 x 32
 
 constexpr uint32_t kIdescQK = idesc_bf16_f32(kMTile, kPage, false);
 constexpr uint32_t kIdescPV = idesc_bf16_f32(kMTile, 256, true);
 
-static_assert(kSmemBytes <= 232448, "shared memory budget");
-
 struct Ctx {
-  uint32_t base;          // shared::cta address of the aligned base
-  uint8_t* gbase;         // generic pointer to the same place
-  uint32_t cta, peer;
-  uint32_t peer_x, peer_xfull, peer_xempty, peer_abort;
+  uint32_t base;     // shared::cta address of the aligned base
+  uint8_t* gbase;    // generic pointer to the same place
+  uint32_t cta;      // rank in the pair; 0 is the leader
+  uint32_t peer_abort;
+  uint32_t lead_bars;  // shared::cluster address of the leader's barrier block
   volatile uint32_t* abort_flag;
   int32_t* meta;
   __device__ uint32_t bar(uint32_t k) const { return base + kOffBar + 8 * k; }
+  __device__ uint32_t lead_bar(uint32_t k) const { return lead_bars + 8 * k; }
 };
 
 __device__ void raise_abort(const Ctx& c, uint32_t err_bits) {
@@ -129,6 +139,13 @@ __device__ bool wait_bar(const Ctx& c, uint32_t bar, uint32_t parity, bool clust
       }
     }
   }
+}
+
+// Arrive on one of the leader's barriers (locally in the leader, remotely from
+// the other CTA).
+__device__ __forceinline__ void arrive_leader(const Ctx& c, uint32_t k) {
+  if (c.cta == 0) mbar_arrive(c.bar(k));
+  else mbar_arrive_remote(c.lead_bar(k));
 }
 
 struct Segment {
@@ -159,118 +176,137 @@ __device__ __forceinline__ Segment load_segment(const DecodeParams& p, int s) {
 }
 
 // ------------------------------------------------------------- producer --
+// Whole warp 0 of each CTA: lanes read 32 page ids at a time (one chunk
+// ahead); lane 0 waits for a free stage and loads this CTA's key half (32
+// tokens, 576 columns) and V columns (64 tokens, 256 columns) of each page,
+// completing bytes on the leader's barriers.
+__device__ __forceinline__ int load_page(const DecodeParams& p, const Ctx& c, const int32_t* table, int blk,
+                                         int end) {
+  if (blk >= end) return 0;
+  int page = table[blk];
+  if (page < 0 || page >= p.num_pages) {
+    atomicOr(reinterpret_cast<unsigned int*>(c.meta + kHError), MLA_DEVERR_PAGE);
+    page = 0;  // keep the copy inside the pool; the result is flagged
+  }
+  return page;
+}
+
 __device__ void producer(const DecodeParams& p, const Ctx& c, int s_begin, int s_end) {
-  const uint32_t q_bytes = static_cast<uint32_t>(p.q_box_rows) * (4 * 128 + 64);  // rows x 288 bf16
+  const int lane = threadIdx.x & 31;
   uint32_t kv_cnt = 0, seg_it = 0;
   bool ok = true;
   for (int s = s_begin; s < s_end && ok; ++s) {
     const Segment g = load_segment(p, s);
     if (g.bad) continue;
-    if (seg_it > 0 && !(ok = wait_bar(c, c.bar(kBarQEmpty), (seg_it - 1) & 1))) break;
-    mbar_arrive_expect_tx(c.bar(kBarQFull), q_bytes);
-    const int y = g.i * p.R + g.mt * kMTile;
-    for (int k = 0; k < 4; ++k)
-      tma_load_2d(c.base + kOffQ + k * kQPanel, &p.tm_q_lat, c.bar(kBarQFull), c.cta * 256 + k * 64, y);
-    tma_load_2d(c.base + kOffQ + 4 * kQPanel, &p.tm_q_rope, c.bar(kBarQFull), 512 + c.cta * 32, y);
-    const int32_t* table = p.block_table + static_cast<long long>(g.i) * p.max_pages;
-    for (int blk = g.b0; blk < g.b1; ++blk) {
-      const uint32_t stage = kv_cnt & 1;
-      if (!(ok = wait_bar(c, c.bar(kBarKvEmpty + stage), ((kv_cnt >> 1) & 1) ^ 1))) break;
-      int page = table[blk];
-      if (page < 0 || page >= p.num_pages) {
-        atomicOr(reinterpret_cast<unsigned int*>(c.meta + kHError), MLA_DEVERR_PAGE);
-        page = 0;  // keep the copy inside the pool; the result is flagged
+    // Q rows of this CTA (once per segment, after the previous segment's QKs).
+    if (lane == 0) {
+      ok = seg_it == 0 || wait_bar(c, c.bar(kBarQEmpty), (seg_it - 1) & 1, true);
+      if (ok) {
+        if (c.cta == 0) mbar_arrive_expect_tx(c.bar(kBarQFull), 2 * kQBytes);
+        const int y = g.i * p.R + g.mt * kMTile + c.cta * kRowsCta;
+#pragma unroll
+        for (int q = 0; q < 9; ++q)
+          tma_load_2d_pair(c.base + kOffQ + q * kQPanel, &p.tm_q, c.lead_bar(kBarQFull), q * 64, y);
       }
-      const uint32_t dst = c.base + kOffKv + stage * kStageBytes;
-      mbar_arrive_expect_tx(c.bar(kBarKvFull + stage), kStageBytes);
-      for (int k = 0; k < 4; ++k)
-        tma_load_2d(dst + k * kKvPanel, &p.tm_kv_lat, c.bar(kBarKvFull + stage), c.cta * 256 + k * 64, page * kPage);
-      tma_load_2d(dst + 4 * kKvPanel, &p.tm_kv_rope, c.bar(kBarKvFull + stage), 512 + c.cta * 32, page * kPage);
-      ++kv_cnt;
     }
+    ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
+    if (!ok) break;
     ++seg_it;
-  }
-  if (!ok) {
-    // Aborting: let the copies already issued land before the CTA can exit.
-    for (uint32_t k = 0; k < 2 && k < kv_cnt; ++k) {
-      const uint32_t last = kv_cnt - 1 - k;
-      const uint64_t t0 = globaltimer();
-      while (!mbar_try_wait(c.bar(kBarKvFull + (last & 1)), (last >> 1) & 1) && globaltimer() - t0 < kTimeoutNs) {
+    const int32_t* table = p.block_table + static_cast<long long>(g.i) * p.max_pages;
+    int cur = load_page(p, c, table, g.b0 + lane, g.b1);
+    for (int c0 = g.b0; c0 < g.b1 && ok; c0 += 32) {
+      const int nxt = load_page(p, c, table, c0 + 32 + lane, g.b1);
+      const int n = min(32, g.b1 - c0);
+      for (int k = 0; k < n; ++k) {
+        const int page = __shfl_sync(0xffffffffu, cur, k);
+        const uint32_t stage = kv_cnt % kStages;
+        int good = 1;
+        if (lane == 0) {
+          good = wait_bar(c, c.bar(kBarStageEmpty + stage), ((kv_cnt / kStages) & 1) ^ 1, true) ? 1 : 0;
+          if (good) {
+            const uint32_t dst = c.base + kOffStage + stage * kStageBytes;
+            const uint32_t kfull = c.lead_bar(kBarKFull + stage);
+            const uint32_t vfull = c.lead_bar(kBarVFull + stage);
+            if (c.cta == 0) {
+              mbar_arrive_expect_tx(c.bar(kBarKFull + stage), 2 * kKBytes);
+              mbar_arrive_expect_tx(c.bar(kBarVFull + stage), 2 * kVBytes);
+            }
+            const int ky = page * kPage + c.cta * (kPage / 2);
+#pragma unroll
+            for (int q = 0; q < 9; ++q) tma_load_2d_pair(dst + q * kKPanel, &p.tm_k, kfull, q * 64, ky);
+#pragma unroll
+            for (int q = 0; q < 4; ++q)
+              tma_load_2d_pair(dst + kKBytes + q * kVPanel, &p.tm_v, vfull,
+                               (q >> 1) * 256 + c.cta * 128 + (q & 1) * 64, page * kPage);
+          }
+        }
+        good = __shfl_sync(0xffffffffu, good, 0);
+        if (!good) {
+          ok = false;
+          break;
+        }
+        ++kv_cnt;
       }
-    }
-    const uint64_t t0 = globaltimer();
-    while (seg_it > 0 && !mbar_try_wait(c.bar(kBarQFull), (seg_it - 1) & 1) && globaltimer() - t0 < kTimeoutNs) {
+      cur = nxt;
     }
   }
 }
 
-// ------------------------------------------------------------------ MMA --
+// ------------------------------------------------------ MMA (leader only) --
 __device__ __forceinline__ void issue_qk(const Ctx& c, uint32_t tmem, uint32_t stage, uint32_t sb) {
   const uint32_t q = c.base + kOffQ;
-  const uint32_t kv = c.base + kOffKv + stage * kStageBytes;
-  const uint32_t d = tmem + kColS + sb * kPage;
+  const uint32_t k = c.base + kOffStage + stage * kStageBytes;
 #pragma unroll
-  for (int k = 0; k < 16; ++k) {
-    const uint32_t off = (k & 3) * 32;
-    const uint64_t a = smem_desc(q + (k >> 2) * kQPanel + off, 16, 1024, kSwizzle128B);
-    const uint64_t b = smem_desc(kv + (k >> 2) * kKvPanel + off, 16, 1024, kSwizzle128B);
-    umma_ss(d, a, b, kIdescQK, k > 0 ? 1u : 0u);
-  }
-#pragma unroll
-  for (int k = 0; k < 2; ++k) {
-    const uint64_t a = smem_desc(q + 4 * kQPanel + k * 32, 16, 512, kSwizzle64B);
-    const uint64_t b = smem_desc(kv + 4 * kKvPanel + k * 32, 16, 512, kSwizzle64B);
-    umma_ss(d, a, b, kIdescQK, 1u);
+  for (int s = 0; s < 36; ++s) {
+    const uint32_t off = (s & 3) * 32;
+    const uint64_t a = smem_desc(q + (s >> 2) * kQPanel + off, 16, 1024, kSwizzle128B);
+    const uint64_t b = smem_desc(k + (s >> 2) * kKPanel + off, 16, 1024, kSwizzle128B);
+    umma_ss_pair(tmem + kColS + 32 * sb, a, b, kIdescQK, s > 0 ? 1u : 0u);
   }
 }
 
 __device__ void mma_issuer(const DecodeParams& p, const Ctx& c, uint32_t tmem, int s_begin, int s_end) {
   uint32_t kv_cnt = 0, q_cnt = 0, pv_cnt = 0, seg_it = 0;
+  const uint16_t both = 0x3;
   for (int s = s_begin; s < s_end; ++s) {
     const Segment g = load_segment(p, s);
     if (g.bad) continue;
     const int n = g.b1 - g.b0;
-    if (!wait_bar(c, c.bar(kBarQFull), seg_it & 1)) return;
-    tc_fence_after();
-    // QK(0)
-    {
-      const uint32_t stage = kv_cnt & 1, sb = q_cnt & 1;
-      if (!wait_bar(c, c.bar(kBarKvFull + stage), (kv_cnt >> 1) & 1)) return;
-      if (!wait_bar(c, c.bar(kBarSEmpty + sb), ((q_cnt >> 1) & 1) ^ 1)) return;
-      tc_fence_after();
-      issue_qk(c, tmem, stage, sb);
-      umma_commit(c.bar(kBarSFull + sb));
-      ++q_cnt;
-    }
-    for (int j = 0; j < n; ++j) {
+    if (!wait_bar(c, c.bar(kBarQFull), seg_it & 1, true)) return;
+    for (int j = -1; j < n; ++j) {
+      // QK(j + 1) first, so that it runs while the softmax works on block j.
       if (j + 1 < n) {
-        const uint32_t kvi = kv_cnt + j + 1;
-        const uint32_t stage = kvi & 1, sb = q_cnt & 1;
-        if (!wait_bar(c, c.bar(kBarKvFull + stage), (kvi >> 1) & 1)) return;
-        if (!wait_bar(c, c.bar(kBarSEmpty + sb), ((q_cnt >> 1) & 1) ^ 1)) return;
+        const uint32_t kvi = kv_cnt + j + 1, sb = q_cnt & 1;
+        if (!wait_bar(c, c.bar(kBarKFull + kvi % kStages), (kvi / kStages) & 1, true)) return;
+        if (!wait_bar(c, c.bar(kBarSEmpty + sb), ((q_cnt >> 1) & 1) ^ 1, true)) return;
         tc_fence_after();
-        issue_qk(c, tmem, stage, sb);
-        umma_commit(c.bar(kBarSFull + sb));
+        issue_qk(c, tmem, kvi % kStages, sb);
+        umma_commit_pair(c.bar(kBarSFull + sb), both);
         ++q_cnt;
-      } else {
-        umma_commit(c.bar(kBarQEmpty));  // Q no longer read once the last QK is done
+        if (j + 1 == n - 1) umma_commit_pair(c.bar(kBarQEmpty), both);  // Q free once the last QK is done
       }
-      if (!wait_bar(c, c.bar(kBarPFull), pv_cnt & 1)) return;
-      if (j == 0 && seg_it > 0 && !wait_bar(c, c.bar(kBarOEmpty), (seg_it - 1) & 1)) return;
+      if (j < 0) continue;
+      // PV(j)
+      const uint32_t kvj = kv_cnt + j, stage = kvj % kStages;
+      if (!wait_bar(c, c.bar(kBarVFull + stage), (kvj / kStages) & 1, true)) return;
+      if (!wait_bar(c, c.bar(kBarPFull), pv_cnt & 1, true)) return;
+      if (j == 0 && seg_it > 0 && !wait_bar(c, c.bar(kBarOEmpty), (seg_it - 1) & 1, true)) return;
       tc_fence_after();
-      const uint32_t stage = (kv_cnt + j) & 1;
       const uint32_t pbuf = c.base + kOffP;
-      const uint32_t vbuf = c.base + kOffKv + stage * kStageBytes;
+      const uint32_t vbuf = c.base + kOffStage + stage * kStageBytes + kKBytes;
 #pragma unroll
-      for (int k = 0; k < 4; ++k) {
-        const uint64_t a = smem_desc(pbuf + k * 32, 16, 1024, kSwizzle128B);
-        // V: K = 16 tokens starting at token 16k, N = 256 latent columns
-        // spread over 4 panels (leading byte offset = panel stride).
-        const uint64_t b = smem_desc(vbuf + k * 16 * 128, kKvPanel, 1024, kSwizzle128B);
-        umma_ss(tmem + kColO, a, b, kIdescPV, (j > 0 || k > 0) ? 1u : 0u);
+      for (int h = 0; h < 2; ++h) {
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+          const uint64_t a = smem_desc(pbuf + k * 32, 16, 1024, kSwizzle128B);
+          // V: K = 16 tokens from token 16k; this CTA's N/2 = 128 columns of
+          // the half are two panels (leading byte offset = panel stride).
+          const uint64_t b = smem_desc(vbuf + h * 2 * kVPanel + k * 16 * 128, kVPanel, 1024, kSwizzle128B);
+          umma_ss_pair(tmem + kColO + 128 * h, a, b, kIdescPV, (j > 0 || k > 0) ? 1u : 0u);
+        }
       }
-      umma_commit(c.bar(kBarKvEmpty + stage));
-      umma_commit(c.bar(kBarPvDone));
+      umma_commit_pair(c.bar(kBarStageEmpty + stage), both);
+      umma_commit_pair(c.bar(kBarPvDone), both);
       ++pv_cnt;
     }
     kv_cnt += n;
@@ -278,17 +314,32 @@ __device__ void mma_issuer(const DecodeParams& p, const Ctx& c, uint32_t tmem, i
   }
 }
 
-// -------------------------------------------------------------- softmax --
+// ---------------------------------------------------- softmax, epilogue --
 __device__ void softmax_epilogue(const DecodeParams& p, const Ctx& c, uint32_t tmem, int s_begin, int s_end) {
-  const int r = threadIdx.x - 128;       // query row within the tile = TMEM lane
+  const int r = threadIdx.x - 128;  // TMEM lane
   const int lane = threadIdx.x & 31;
+  const int hr = r & (kRowsCta - 1);  // query row within this CTA
+  const int half = r >> 6;            // 0: tokens 0-31 / first column half; 1: the rest
   const uint32_t lane_off = static_cast<uint32_t>(r & ~31) << 16;
   const uint32_t t_s = tmem + lane_off + kColS;
   const uint32_t t_o = tmem + lane_off + kColO;
-  float* xbuf = reinterpret_cast<float*>(c.gbase + kOffX);
-  const uint32_t my_xfull = c.bar(kBarXFull);
-  const uint32_t peer_row = c.peer_x + r * 256;
-  uint32_t s_cnt = 0, pv_cnt = 0, x_cnt = 0, blk_cnt = 0;
+  float* smax = reinterpret_cast<float*>(c.gbase + kOffMax);
+  const float sl2 = p.scale_log2;
+  // blk_cnt: pages consumed (selects the V stage); x_cnt: row exchanges with
+  // the partner thread (selects the exchange slot and the barrier phase).
+  uint32_t s_cnt = 0, pv_cnt = 0, blk_cnt = 0, x_cnt = 0;
+  // Publish v for the partner thread (same row, other half) and return its
+  // value; the 4 warps meet on an mbarrier (bounded wait).
+  auto trade = [&](float v, float* out) -> bool {
+    float* buf = smax + (x_cnt & 1) * 128;
+    buf[r] = v;
+    __syncwarp();
+    if (lane == 0) mbar_arrive(c.bar(kBarXMax));
+    const bool ok = wait_bar(c, c.bar(kBarXMax), x_cnt & 1);
+    ++x_cnt;
+    *out = buf[r ^ 64];
+    return ok;
+  };
 
   for (int s = s_begin; s < s_end; ++s) {
     const Segment g = load_segment(p, s);
@@ -297,8 +348,9 @@ __device__ void softmax_epilogue(const DecodeParams& p, const Ctx& c, uint32_t t
       continue;
     }
     const int n = g.b1 - g.b0;
-    const int row_g = g.mt * kMTile + r;
-    const bool row_valid = r < p.tile_rows && row_g < p.R;
+    const int q_row = c.cta * kRowsCta + hr;  // row within the 128-row tile
+    const int row_g = g.mt * kMTile + q_row;
+    const bool row_valid = q_row < p.tile_rows && row_g < p.R;
     const int t = row_g / p.h_q;
     const int hh = row_g - t * p.h_q;
     int limit = 0;
@@ -307,81 +359,71 @@ __device__ void softmax_epilogue(const DecodeParams& p, const Ctx& c, uint32_t t
       limit = limit < 0 ? 0 : (limit > g.L ? g.L : limit);
     }
     const int last_page = ceil_div(g.L, kPage) - 1;
-    // l: sum of the bf16-rounded weights actually fed to PV (normalises O, so
-    // the output is an exact convex combination of those weights); le: the
-    // same sum before rounding (gives lse without the bf16 rounding bias).
-    float m = -INFINITY, l = 0.0f, le = 0.0f;
 
+    float m = -INFINITY, l = 0.0f;  // l: this thread's half of the row sum
     for (int j = 0; j < n; ++j) {
       const int blk = g.b0 + j;
       const uint32_t sb = s_cnt & 1;
-      if (!wait_bar(c, c.bar(kBarSFull + sb), (s_cnt >> 1) & 1)) return;
+      if (!wait_bar(c, c.bar(kBarSFull + sb), (s_cnt >> 1) & 1, true)) return;
       tc_fence_after();
-      float sv[64];
-      tmem_ld32(t_s + sb * kPage, *reinterpret_cast<float(*)[32]>(&sv[0]));
-      tmem_ld32(t_s + sb * kPage + 32, *reinterpret_cast<float(*)[32]>(&sv[32]));
+      float sv[32];
+      tmem_ld32(t_s + 32 * sb, sv);
       tmem_wait_ld();
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive(c.bar(kBarSEmpty + sb));
+      if (lane == 0) arrive_leader(c, kBarSEmpty + sb);
       ++s_cnt;
 
-      // ---- exchange the partial S with the peer CTA and add ----
-      if (x_cnt > 0 && !wait_bar(c, c.bar(kBarXEmpty), (x_cnt - 1) & 1, true)) return;
-      if (r == 0) mbar_arrive_expect_tx(my_xfull, kXBytes);
+      // ---- mask; block max over both halves of the row ----
+      int nvalid = limit - blk * kPage - 32 * half;
+      nvalid = nvalid < 0 ? 0 : (nvalid > 32 ? 32 : nvalid);
+      if (nvalid < 32) {
 #pragma unroll
-      for (int q4 = 0; q4 < 16; ++q4) {
-        const uint32_t dst = peer_row + ((q4 ^ (r & 15)) << 4);
-        st_async_v4(dst, c.peer_xfull, sv[4 * q4 + 0], sv[4 * q4 + 1], sv[4 * q4 + 2], sv[4 * q4 + 3]);
+        for (int k = 0; k < 32; ++k) sv[k] = (k < nvalid) ? sv[k] : -INFINITY;
       }
-      if (!wait_bar(c, my_xfull, x_cnt & 1, true)) return;
+      float mx;
       {
-        const float4* row = reinterpret_cast<const float4*>(xbuf + r * 64);
+        float a[16];
 #pragma unroll
-        for (int q4 = 0; q4 < 16; ++q4) {
-          const float4 u = row[q4 ^ (r & 15)];
-          sv[4 * q4 + 0] += u.x;
-          sv[4 * q4 + 1] += u.y;
-          sv[4 * q4 + 2] += u.z;
-          sv[4 * q4 + 3] += u.w;
-        }
-      }
-      __syncwarp();
-      if (lane == 0) mbar_arrive_remote(c.peer_xempty);
-      ++x_cnt;
-
-      // ---- mask, online softmax (log2 domain) ----
-      int nvalid = limit - blk * kPage;
-      nvalid = nvalid < 0 ? 0 : (nvalid > kPage ? kPage : nvalid);
-      float mx = -INFINITY;
+        for (int k = 0; k < 16; ++k) a[k] = fmaxf(sv[k], sv[k + 16]);
 #pragma unroll
-      for (int k = 0; k < 64; ++k) {
-        const float x = (k < nvalid) ? sv[k] * p.scale_log2 : -INFINITY;
-        sv[k] = x;
-        mx = fmaxf(mx, x);
+        for (int k = 0; k < 8; ++k) a[k] = fmaxf(a[k], a[k + 8]);
+#pragma unroll
+        for (int k = 0; k < 4; ++k) a[k] = fmaxf(a[k], a[k + 4]);
+        mx = fmaxf(fmaxf(a[0], a[2]), fmaxf(a[1], a[3]));
       }
+      mx = (nvalid > 0) ? mx * sl2 : -INFINITY;  // softmax_scale >= 0
+      float mx_peer;
+      if (!trade(mx, &mx_peer)) return;
+      mx = fmaxf(mx, mx_peer);
       float m_new = m;
       if (mx > m + kTau) m_new = mx;  // also true for the first finite block
       const float alpha = (m_new == m) ? 1.0f : ex2(m - m_new);  // 0 when m was -inf
-      const float m_use = (m_new == -INFINITY) ? 0.0f : m_new;
-      uint32_t packed[32];
-      float psum = 0.0f, esum = 0.0f;
+      const float neg_m = (m_new == -INFINITY) ? 0.0f : -m_new;
+      uint32_t packed[16];
+      float e[16];
 #pragma unroll
-      for (int k = 0; k < 32; ++k) {
-        const float a = ex2(sv[2 * k] - m_use), b = ex2(sv[2 * k + 1] - m_use);
-        esum += a + b;
+      for (int k = 0; k < 16; ++k) {
+        float a = ex2(fmaf(sv[2 * k], sl2, neg_m));
+        float b = ex2(fmaf(sv[2 * k + 1], sl2, neg_m));
+        if (nvalid < 32) {
+          a = (2 * k < nvalid) ? a : 0.0f;
+          b = (2 * k + 1 < nvalid) ? b : 0.0f;
+        }
+        e[k] = a + b;
         const __nv_bfloat162 pr = __floats2bfloat162_rn(a, b);
-        const float2 back = __bfloat1622float2(pr);
-        psum += back.x + back.y;
         packed[k] = *reinterpret_cast<const uint32_t*>(&pr);
       }
-      l = l * alpha + psum;
-      le = le * alpha + esum;
+#pragma unroll
+      for (int k = 0; k < 8; ++k) e[k] += e[k + 8];
+#pragma unroll
+      for (int k = 0; k < 4; ++k) e[k] += e[k + 4];
+      l = l * alpha + ((e[0] + e[2]) + (e[1] + e[3]));
       m = m_new;
 
-      // ---- wait for the previous PV: P buffer free, O up to date ----
+      // ---- previous PV done: P buffer free, O up to date ----
       if (j > 0) {
-        if (!wait_bar(c, c.bar(kBarPvDone), pv_cnt & 1)) return;
+        if (!wait_bar(c, c.bar(kBarPvDone), pv_cnt & 1, true)) return;
         ++pv_cnt;
         tc_fence_after();
         const bool need = alpha < 1.0f;
@@ -398,49 +440,55 @@ __device__ void softmax_epilogue(const DecodeParams& p, const Ctx& c, uint32_t t
           tmem_wait_st();
         }
       }
-
-      // ---- P to shared memory (128B-swizzled K-major rows) ----
+      // ---- P row hr, this thread's 32 tokens = 4 swizzled 16-byte chunks ----
       {
-        uint8_t* prow = c.gbase + kOffP + (r >> 3) * 1024 + (r & 7) * 128;
+        uint8_t* prow = c.gbase + kOffP + (hr >> 3) * 1024 + (hr & 7) * 128;
 #pragma unroll
-        for (int ch = 0; ch < 8; ++ch) {
-          uint4 v = make_uint4(packed[4 * ch + 0], packed[4 * ch + 1], packed[4 * ch + 2], packed[4 * ch + 3]);
-          *reinterpret_cast<uint4*>(prow + ((ch ^ (r & 7)) << 4)) = v;
+        for (int q = 0; q < 4; ++q) {
+          const int ch = 4 * half + q;
+          *reinterpret_cast<uint4*>(prow + ((ch ^ (hr & 7)) << 4)) =
+              make_uint4(packed[4 * q], packed[4 * q + 1], packed[4 * q + 2], packed[4 * q + 3]);
         }
       }
       // ---- the last page of a row may hold garbage (even NaN) past L: zero
-      //      those V rows so that 0 * garbage cannot reach O ----
+      //      this CTA's V rows there so that 0 * garbage cannot reach O ----
       if (blk == last_page && (g.L & (kPage - 1))) {
         const int first_bad = g.L - blk * kPage;
         const int chunks = (kPage - first_bad) * 4 * 8;  // rows x panels x 16-byte chunks
-        uint8_t* stage = c.gbase + kOffKv + (blk_cnt & 1) * kStageBytes;
-        for (int e = r; e < chunks; e += 128) {
-          const int row = first_bad + (e >> 5);
-          const int panel = (e >> 3) & 3;
-          const int ch = e & 7;
-          *reinterpret_cast<uint4*>(stage + panel * kKvPanel + row * 128 + ch * 16) = make_uint4(0, 0, 0, 0);
+        uint8_t* vst = c.gbase + kOffStage + (blk_cnt % kStages) * kStageBytes + kKBytes;
+        for (int e2 = r; e2 < chunks; e2 += 128) {
+          const int row = first_bad + (e2 >> 5);
+          const int panel = (e2 >> 3) & 3;
+          const int ch = e2 & 7;
+          *reinterpret_cast<uint4*>(vst + panel * kVPanel + row * 128 + ch * 16) = make_uint4(0, 0, 0, 0);
         }
       }
       fence_proxy_async_smem();
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive(c.bar(kBarPFull));
+      if (lane == 0) arrive_leader(c, kBarPFull);
       ++blk_cnt;
     }
 
     // ---- epilogue ----
-    if (!wait_bar(c, c.bar(kBarPvDone), pv_cnt & 1)) return;
+    if (!wait_bar(c, c.bar(kBarPvDone), pv_cnt & 1, true)) return;
     ++pv_cnt;
     tc_fence_after();
-    const float inv_l = l > 0.0f ? 1.0f / l : 0.0f;
+    float l_peer;
+    if (!trade(l, &l_peer)) return;
+    const float lt = l + l_peer;
+    const float inv_l = lt > 0.0f ? 1.0f / lt : 0.0f;
+    const float lse_v = lt > 0.0f ? (m + __log2f(lt)) * 0.69314718055994530942f : -INFINITY;
+    // This thread's O columns: for each half h of the 512, columns
+    // [256h + 128*half, 256h + 128*half + 128).
     if (g.slot < 0) {
-      __nv_bfloat16* orow = reinterpret_cast<__nv_bfloat16*>(p.out) +
-                            (static_cast<long long>(g.i) * p.R + row_g) * kDv + c.cta * 256;
+      __nv_bfloat16* orow = reinterpret_cast<__nv_bfloat16*>(p.out) + (static_cast<long long>(g.i) * p.R + row_g) * kDv;
 #pragma unroll 1
       for (int cc = 0; cc < 256; cc += 32) {
         float o[32];
         tmem_ld32(t_o + cc, o);
         tmem_wait_ld();
+        const int col = (cc >> 7) * 256 + 128 * half + (cc & 127);
         if (row_valid) {
 #pragma unroll
           for (int k = 0; k < 32; k += 8) {
@@ -453,36 +501,31 @@ __device__ void softmax_epilogue(const DecodeParams& p, const Ctx& c, uint32_t t
             v.y = *reinterpret_cast<uint32_t*>(&h1);
             v.z = *reinterpret_cast<uint32_t*>(&h2);
             v.w = *reinterpret_cast<uint32_t*>(&h3);
-            *reinterpret_cast<uint4*>(orow + cc + k) = v;
+            *reinterpret_cast<uint4*>(orow + col + k) = v;
           }
         }
       }
-      if (row_valid && c.cta == 0) {
-        const float lse = le > 0.0f ? (m + __log2f(le)) * 0.69314718055994530942f : -INFINITY;
-        p.lse[(static_cast<long long>(g.i) * p.h_q + hh) * p.s_q + t] = lse;
-      }
+      if (row_valid && half == 0) p.lse[(static_cast<long long>(g.i) * p.h_q + hh) * p.s_q + t] = lse_v;
     } else {
-      float* orow = p.o_part + (static_cast<long long>(g.slot) * p.tile_rows + r) * kDv + c.cta * 256;
+      float* orow = p.o_part + (static_cast<long long>(g.slot) * p.tile_rows + q_row) * kDv;
 #pragma unroll 1
       for (int cc = 0; cc < 256; cc += 32) {
         float o[32];
         tmem_ld32(t_o + cc, o);
         tmem_wait_ld();
+        const int col = (cc >> 7) * 256 + 128 * half + (cc & 127);
         if (row_valid) {
 #pragma unroll
           for (int k = 0; k < 32; k += 4)
-            *reinterpret_cast<float4*>(orow + cc + k) =
+            *reinterpret_cast<float4*>(orow + col + k) =
                 make_float4(o[k] * inv_l, o[k + 1] * inv_l, o[k + 2] * inv_l, o[k + 3] * inv_l);
         }
       }
-      if (row_valid && c.cta == 0) {
-        const float lse = le > 0.0f ? (m + __log2f(le)) * 0.69314718055994530942f : -INFINITY;
-        p.lse_part[static_cast<long long>(g.slot) * p.tile_rows + r] = lse;
-      }
+      if (row_valid && half == 0) p.lse_part[static_cast<long long>(g.slot) * p.tile_rows + q_row] = lse_v;
     }
     tc_fence_before();
     __syncwarp();
-    if (lane == 0) mbar_arrive(c.bar(kBarOEmpty));
+    if (lane == 0) arrive_leader(c, kBarOEmpty);
   }
 }
 
@@ -495,68 +538,49 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
   c.base = base;
   c.gbase = smem_raw + (base - raw);
   c.cta = cluster_ctarank();
-  c.peer = c.cta ^ 1u;
   c.meta = p.meta;
   c.abort_flag = reinterpret_cast<volatile uint32_t*>(c.gbase + kOffAbort);
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
 
   if (threadIdx.x == 0) {
-    mbar_init(c.bar(kBarKvFull + 0), 1);
-    mbar_init(c.bar(kBarKvFull + 1), 1);
-    mbar_init(c.bar(kBarKvEmpty + 0), 1);
-    mbar_init(c.bar(kBarKvEmpty + 1), 1);
+    // Barriers of the leader's pipeline are only used in the leader, the
+    // rest in both CTAs; initialise all of them everywhere.
+    for (int k = 0; k < kStages; ++k) {
+      mbar_init(c.bar(kBarKFull + k), 1);
+      mbar_init(c.bar(kBarVFull + k), 1);
+      mbar_init(c.bar(kBarStageEmpty + k), 1);
+    }
     mbar_init(c.bar(kBarQFull), 1);
     mbar_init(c.bar(kBarQEmpty), 1);
     mbar_init(c.bar(kBarSFull + 0), 1);
     mbar_init(c.bar(kBarSFull + 1), 1);
-    mbar_init(c.bar(kBarSEmpty + 0), 4);
-    mbar_init(c.bar(kBarSEmpty + 1), 4);
-    mbar_init(c.bar(kBarPFull), 4);
+    mbar_init(c.bar(kBarSEmpty + 0), 8);
+    mbar_init(c.bar(kBarSEmpty + 1), 8);
+    mbar_init(c.bar(kBarPFull), 8);
     mbar_init(c.bar(kBarPvDone), 1);
-    mbar_init(c.bar(kBarXFull), 1);
-    mbar_init(c.bar(kBarXEmpty), 4);
-    mbar_init(c.bar(kBarOEmpty), 4);
+    mbar_init(c.bar(kBarOEmpty), 8);
     mbar_init(c.bar(kBarFinal), 1);
+    mbar_init(c.bar(kBarXMax), 4);
     *c.abort_flag = 0u;
     fence_mbar_init_cluster();
   }
-  // Query rows past the tile's real rows are never written by TMA: zero them
-  // once so that the padded MMA rows stay finite.
-  if (p.q_box_rows < kMTile) {
-    const int rows = kMTile - p.q_box_rows;
-    const int per_panel128 = rows * 8;  // 16-byte chunks
-    for (int e = threadIdx.x; e < per_panel128 * 4; e += kThreads) {
-      const int panel = e / per_panel128;
-      const int rem = e - panel * per_panel128;
-      *reinterpret_cast<uint4*>(c.gbase + kOffQ + panel * kQPanel + (p.q_box_rows + rem / 8) * 128 + (rem & 7) * 16) =
-          make_uint4(0, 0, 0, 0);
-    }
-    for (int e = threadIdx.x; e < rows * 4; e += kThreads) {
-      *reinterpret_cast<uint4*>(c.gbase + kOffQ + 4 * kQPanel + (p.q_box_rows + e / 4) * 64 + (e & 3) * 16) =
-          make_uint4(0, 0, 0, 0);
-    }
-    fence_proxy_async_smem();
-  }
   if (warp == 1) {
-    tmem_alloc(base + kOffTmemSlot, kTmemCols);
-    tmem_relinquish();
+    tmem_alloc_pair(base + kOffTmemSlot, kTmemCols);
+    tmem_relinquish_pair();
   }
   if (warp == 0 && lane == 0) {
-    tma_prefetch_desc(&p.tm_kv_lat);
-    tma_prefetch_desc(&p.tm_kv_rope);
-    tma_prefetch_desc(&p.tm_q_lat);
-    tma_prefetch_desc(&p.tm_q_rope);
+    tma_prefetch_desc(&p.tm_k);
+    tma_prefetch_desc(&p.tm_v);
+    tma_prefetch_desc(&p.tm_q);
   }
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
-  cluster_sync();  // the peer's barriers exist before any remote arrival
+  cluster_sync();  // both CTAs' barriers exist before any remote arrival
   const uint32_t tmem = *reinterpret_cast<volatile uint32_t*>(c.gbase + kOffTmemSlot);
-  c.peer_x = map_to_rank(base + kOffX, c.peer);
-  c.peer_xfull = map_to_rank(c.bar(kBarXFull), c.peer);
-  c.peer_xempty = map_to_rank(c.bar(kBarXEmpty), c.peer);
-  c.peer_abort = map_to_rank(base + kOffAbort, c.peer);
+  c.peer_abort = map_to_rank(base + kOffAbort, c.cta ^ 1u);
+  c.lead_bars = map_to_rank(base + kOffBar, 0);
 
   // The plan must be the one built for this call's shape on this many pairs.
   const int pair = static_cast<int>(blockIdx.x >> 1);
@@ -573,33 +597,32 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
   }
 
   if (warp == 0) {
-    if (lane == 0) producer(p, c, s_begin, s_end);
-    __syncwarp();
+    producer(p, c, s_begin, s_end);
   } else if (warp == 1) {
-    if (lane == 0) mma_issuer(p, c, tmem, s_begin, s_end);
+    if (lane == 0 && c.cta == 0) mma_issuer(p, c, tmem, s_begin, s_end);
     __syncwarp();
   } else if (warp >= 4) {
     softmax_epilogue(p, c, tmem, s_begin, s_end);
   }
 
-  // ---- teardown: drain MMAs, wait for the peer, free TMEM ----
+  // ---- teardown: drain the pair MMAs, wait for the peer, free TMEM ----
   __syncthreads();
-  if (warp == 1) {
+  if (warp == 1 && c.cta == 0) {
     if (lane == 0) {
-      umma_commit(c.bar(kBarFinal));
+      umma_commit_pair(c.bar(kBarFinal), 0x1);
       const uint64_t t0 = globaltimer();
       while (!mbar_try_wait(c.bar(kBarFinal), 0) && globaltimer() - t0 < kTimeoutNs) {
       }
     }
     __syncwarp();
   }
-  if (*c.abort_flag) __nanosleep(20000);  // let a peer's in-flight DSMEM stores land
+  if (*c.abort_flag) __nanosleep(20000);  // let in-flight copies and arrivals land
   tc_fence_before();
   __syncthreads();
   cluster_sync();
   if (warp == 1) {
     tc_fence_after();
-    tmem_dealloc(tmem, kTmemCols);
+    tmem_dealloc_pair(tmem, kTmemCols);
   }
 }
 

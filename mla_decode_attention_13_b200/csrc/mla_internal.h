@@ -30,6 +30,8 @@ constexpr uint32_t kMagic = 0x314C4D42u;  // "BML1"
 //   row_info  [W][2]                    (first slot or -1, pieces)
 //   split_rows [W]                      work rows cut into >1 pieces
 //   empty_rows [W]                      work rows with no pages
+//   scratch   [W][4]                    plan construction: end cost (int64),
+//                                       first segment, first pair
 // A work row is (batch row i, m-tile mt) with index w = mt * batch + i.
 // ---------------------------------------------------------------------------
 enum HeaderWord : int {
@@ -53,7 +55,7 @@ enum HeaderWord : int {
 
 struct MetaLayout {
   int W;
-  size_t pair_off, segs, row_info, split_rows, empty_rows, words;
+  size_t pair_off, segs, row_info, split_rows, empty_rows, scratch, words;
 };
 
 __host__ __device__ inline int ceil_div(int a, int b) { return (a + b - 1) / b; }
@@ -66,7 +68,8 @@ __host__ __device__ inline MetaLayout meta_layout(int batch, int h_q, int s_q) {
   L.row_info = L.segs + size_t(4) * (L.W + kMaxPairs);
   L.split_rows = L.row_info + size_t(2) * L.W;
   L.empty_rows = L.split_rows + L.W;
-  L.words = L.empty_rows + L.W;
+  L.scratch = (L.empty_rows + L.W + 1) & ~size_t(1);  // 8-byte aligned
+  L.words = L.scratch + size_t(4) * L.W;
   return L;
 }
 
@@ -90,10 +93,9 @@ __host__ __device__ inline size_t workspace_bytes_for(int pairs, int h_q, int s_
 // Split-KV decode kernel parameters.
 // ---------------------------------------------------------------------------
 struct DecodeParams {
-  CUtensorMap tm_kv_lat;   // cache as [num_pages*64][576]: box 64 cols x 64 rows, 128B swizzle
-  CUtensorMap tm_kv_rope;  // same tensor: box 32 cols x 64 rows, 64B swizzle
-  CUtensorMap tm_q_lat;    // q as [batch*R][576]: box 64 cols x min(R,128) rows, 128B swizzle
-  CUtensorMap tm_q_rope;   // same tensor: box 32 cols x min(R,128) rows, 64B swizzle
+  CUtensorMap tm_k;  // cache as [num_pages*64][576]: box 64 cols x 32 rows, 128B swizzle (key halves)
+  CUtensorMap tm_v;  // same tensor: box 64 cols x 64 rows, 128B swizzle (V columns)
+  CUtensorMap tm_q;  // q as [batch*R][576]: box 64 cols x 64 rows, 128B swizzle
   const int32_t* block_table;
   const int32_t* seqlens;
   void* out;               // bf16
@@ -103,7 +105,7 @@ struct DecodeParams {
   int32_t* meta;
   long long num_pages;
   int max_pages;
-  int batch, s_q, h_q, R, n_mt, causal, q_box_rows, tile_rows, max_slots;
+  int batch, s_q, h_q, R, n_mt, causal, tile_rows, max_slots;
   float scale_log2;        // softmax_scale * log2(e)
 };
 

@@ -7,28 +7,66 @@
 // pieces merged.  "FlashMLA overview" (flash_api.cpp): the plan is computed
 // once per decode step (get_mla_metadata) and reused by every layer.
 //
-// The plan cuts the concatenation of all work rows' 64-token pages into one
-// contiguous range per SM pair (2-CTA cluster):
-//   * a work row is one batch row's tile of up to 128 query rows; work rows
-//     are ordered m-tile major, w = mt * batch + i, so the m-tiles of one batch
-//     row (which read the same pages) land on pairs far apart in the order and
-//     run at about the same time;
-//   * a row with n pages costs n + kappa (kappa: fixed per-piece cost: Q load,
-//     pipeline fill, epilogue), T is the total, and each pair may hold
-//     cap = ceil(T / P) + 2 kappa;
-//   * walking rows in order, the current pair takes as many pages of the row as
-//     fit in cap - used - kappa (at least one); when nothing fits, the next pair
-//     starts; the last pair takes whatever is left;
-//   * a row cut into k > 1 pieces gets k consecutive partial slots (row order).
-// One CTA: all threads compute the page counts and their total, then thread 0
-// walks the rows (O(W + P) steps).
+// The plan is a cost-interval partition of all work rows' 64-token pages over
+// the P SM pairs (2-CTA clusters):
+//   * a work row is one batch row's tile of up to 128 query rows, ordered
+//     m-tile major (w = mt * batch + i), so the m-tiles of one batch row, which
+//     read the same pages, land on pairs far apart and run at the same time;
+//   * a row with n > 0 pages costs n + kappa (kappa: fixed cost of starting a
+//     row: Q load, pipeline fill, epilogue); C_w is the cost of the rows before
+//     w and T the total; cap = max(1, ceil(T / P));
+//   * page b of row w sits at cost position C_w + kappa + b and belongs to pair
+//     floor(position / cap), so every pair takes one contiguous page range;
+//   * a row whose pages land on k > 1 pairs is cut into k pieces with k
+//     consecutive partial slots (row order); its output comes from the combine.
+// Everything follows from prefix sums, so one CTA computes it with block-wide
+// scans over chunks of 1024 rows and one binary search per pair.
 #include "mla_internal.h"
 
 namespace mla {
 namespace {
 
-constexpr int kSchedThreads = 256;
-constexpr int kSmemRows = 8192;
+constexpr int kSchedThreads = 1024;
+constexpr int kWarps = kSchedThreads / 32;
+
+// Block-wide exclusive scan of one value per thread; returns the exclusive
+// prefix and writes the block total to *total.  All threads must call it.
+template <typename T>
+__device__ T block_exclusive_scan(T v, T* warp_tot, T* total) {
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  T incl = v;
+#pragma unroll
+  for (int off = 1; off < 32; off <<= 1) {
+    const T o = __shfl_up_sync(0xffffffffu, incl, off);
+    if (lane >= off) incl += o;
+  }
+  if (lane == 31) warp_tot[warp] = incl;
+  __syncthreads();
+  if (warp == 0) {
+    T t = lane < kWarps ? warp_tot[lane] : T(0);
+    T ti = t;
+#pragma unroll
+    for (int off = 1; off < 32; off <<= 1) {
+      const T o = __shfl_up_sync(0xffffffffu, ti, off);
+      if (lane >= off) ti += o;
+    }
+    if (lane < kWarps) warp_tot[lane] = ti - t;  // exclusive warp offsets
+    if (lane == kWarps - 1) *total = ti;
+  }
+  __syncthreads();
+  const T res = warp_tot[warp] + incl - v;
+  __syncthreads();
+  return res;
+}
+
+__device__ __forceinline__ int row_pages(const int32_t* seqlens, int batch, int w, int* err) {
+  int L = seqlens[w % batch];
+  if (L < 0) {
+    *err = 1;
+    L = 0;
+  }
+  return ceil_div(L, kPage);
+}
 
 __global__ void __launch_bounds__(kSchedThreads) mla_sched_kernel(const int32_t* __restrict__ seqlens, int batch,
                                                                   int h_q, int s_q, int pairs, int32_t* meta) {
@@ -41,104 +79,121 @@ __global__ void __launch_bounds__(kSchedThreads) mla_sched_kernel(const int32_t*
   int32_t* row_info = meta + lo.row_info;
   int32_t* split_rows = meta + lo.split_rows;
   int32_t* empty_rows = meta + lo.empty_rows;
+  long long* end_cost = reinterpret_cast<long long*>(meta + lo.scratch);  // [W]
+  int32_t* first_seg = meta + lo.scratch + 2 * W;                         // [W]
+  int32_t* first_pair = meta + lo.scratch + 3 * W;                        // [W]
 
-  __shared__ int32_t s_pages[kSmemRows];
-  __shared__ long long s_red[kSchedThreads / 32];
+  __shared__ long long s_wl[kWarps];
+  __shared__ int s_wi[kWarps];
+  __shared__ long long s_tot_l;
+  __shared__ int s_tot_i;
   __shared__ int s_err;
-  // Pages per work row live in shared memory when they fit, else in the
-  // empty_rows area (rewritten after the walk).
-  int32_t* pages = (W <= kSmemRows) ? s_pages : empty_rows;
-
   if (threadIdx.x == 0) s_err = 0;
   __syncthreads();
+  int err = 0;
+
+  // Pass 1: total cost T.
   long long local = 0;
-  for (int w = threadIdx.x; w < W; w += blockDim.x) {
-    const int i = w % batch;
-    int L = seqlens[i];
-    if (L < 0) {
-      s_err = 1;
-      L = 0;
-    }
-    const int n = ceil_div(L, kPage);
-    pages[w] = n;
+  for (int w = threadIdx.x; w < W; w += kSchedThreads) {
+    const int n = row_pages(seqlens, batch, w, &err);
     if (n > 0) local += n + kKappa;
   }
-  for (int off = 16; off > 0; off >>= 1) local += __shfl_xor_sync(0xffffffffu, local, off);
-  if ((threadIdx.x & 31) == 0) s_red[threadIdx.x >> 5] = local;
-  __syncthreads();
-  if (threadIdx.x != 0) return;
+  block_exclusive_scan<long long>(local, s_wl, &s_tot_l);
+  const long long T = s_tot_l;
+  const long long cap = T > 0 ? (T + pairs - 1) / pairs : 1;
 
-  long long T = 0;
-  for (int k = 0; k < kSchedThreads / 32; ++k) T += s_red[k];
-  const long long cap = (T + pairs - 1) / pairs + 2 * kKappa;
-
-  int p = 0, nseg = 0, nslots = 0;
-  long long used = 0;
-  for (int k = 0; k <= pairs; ++k) pair_off[k] = 0;
-  for (int w = 0; w < W; ++w) {
-    const int n = pages[w];
-    const int first = nseg;
-    int b0 = 0;
-    while (b0 < n) {
-      const long long room = cap - used - kKappa;
-      if (room < 1 && p < pairs - 1) {
-        ++p;
-        pair_off[p] = nseg;
-        used = 0;
-        continue;
-      }
-      long long take = n - b0;
-      if (p != pairs - 1) {
-        const long long fit = room > 1 ? room : 1;
-        if (fit < take) take = fit;
-      }
-      int32_t* s = segs + 4 * nseg;
-      s[0] = w;
-      s[1] = b0;
-      s[2] = b0 + static_cast<int>(take);
-      s[3] = -1;
-      ++nseg;
-      used += take + kKappa;
-      b0 += static_cast<int>(take);
+  // Pass 2: per-row prefix sums (cost, segments, slots, split and empty
+  // lists), chunk by chunk with carries.
+  long long carry_cost = 0;
+  int carry_seg = 0, carry_slot = 0, carry_split = 0, carry_empty = 0;
+  for (int base = 0; base < W; base += kSchedThreads) {
+    const int w = base + threadIdx.x;
+    const bool in = w < W;
+    const int n = in ? row_pages(seqlens, batch, w, &err) : 0;
+    const long long c = n > 0 ? n + kKappa : 0;
+    const long long C = carry_cost + block_exclusive_scan<long long>(c, s_wl, &s_tot_l);
+    const long long chunk_cost = s_tot_l;
+    int f = 0, pieces = 0;
+    if (n > 0) {
+      f = static_cast<int>((C + kKappa) / cap);
+      const int l = static_cast<int>((C + kKappa + n - 1) / cap);
+      pieces = l - f + 1;
     }
-    const int pieces = nseg - first;
-    row_info[2 * w + 0] = -1;
-    row_info[2 * w + 1] = pieces;
-    if (pieces > 1) {
-      row_info[2 * w + 0] = nslots;
-      for (int k = 0; k < pieces; ++k) segs[4 * (first + k) + 3] = nslots + k;
-      nslots += pieces;
+    const int seg0 = carry_seg + block_exclusive_scan<int>(pieces, s_wi, &s_tot_i);
+    const int chunk_seg = s_tot_i;
+    const int slot0 = carry_slot + block_exclusive_scan<int>(pieces > 1 ? pieces : 0, s_wi, &s_tot_i);
+    const int chunk_slot = s_tot_i;
+    const int split_i = carry_split + block_exclusive_scan<int>(pieces > 1 ? 1 : 0, s_wi, &s_tot_i);
+    const int chunk_split = s_tot_i;
+    const int empty_i = carry_empty + block_exclusive_scan<int>(in && n == 0 ? 1 : 0, s_wi, &s_tot_i);
+    const int chunk_empty = s_tot_i;
+    if (in) {
+      row_info[2 * w + 0] = pieces > 1 ? slot0 : -1;
+      row_info[2 * w + 1] = pieces;
+      for (int k = 0; k < pieces; ++k) {
+        const long long p = f + k;
+        const long long b0 = p * cap - C - kKappa;
+        const long long b1 = (p + 1) * cap - C - kKappa;
+        int4 sg;
+        sg.x = w;
+        sg.y = b0 > 0 ? static_cast<int>(b0) : 0;
+        sg.z = b1 < n ? static_cast<int>(b1) : n;
+        sg.w = pieces > 1 ? slot0 + k : -1;
+        *reinterpret_cast<int4*>(segs + 4 * (seg0 + k)) = sg;
+      }
+      if (pieces > 1) split_rows[split_i] = w;
+      if (n == 0) empty_rows[empty_i] = w;
+      end_cost[w] = C + c;
+      first_seg[w] = seg0;
+      first_pair[w] = f;
     }
+    carry_cost += chunk_cost;
+    carry_seg += chunk_seg;
+    carry_slot += chunk_slot;
+    carry_split += chunk_split;
+    carry_empty += chunk_empty;
   }
-  // Pairs after the last one that received work own empty ranges.
-  for (int k = p + 1; k <= pairs; ++k) pair_off[k] = nseg;
+  if (err) s_err = 1;
+  __syncthreads();  // scratch written and visible to the whole CTA
 
-  int n_split = 0, n_empty = 0;
-  for (int w = 0; w < W; ++w) {
-    const int pieces = row_info[2 * w + 1];
-    if (pieces > 1) split_rows[n_split++] = w;
-  }
-  for (int w = 0; w < W; ++w) {
-    if (row_info[2 * w + 1] == 0) empty_rows[n_empty++] = w;
+  // Pass 3: pair p starts at the first row whose pages reach cost position
+  // p * cap (end cost > p * cap); its first segment there is p - first pair.
+  for (int p = threadIdx.x; p <= pairs; p += kSchedThreads) {
+    int off = carry_seg;
+    if (p < pairs) {
+      const long long x = static_cast<long long>(p) * cap;
+      int lo_w = 0, hi_w = W;  // first w with end_cost[w] > x
+      while (lo_w < hi_w) {
+        const int mid = (lo_w + hi_w) >> 1;
+        if (end_cost[mid] > x) hi_w = mid; else lo_w = mid + 1;
+      }
+      if (lo_w < W) {
+        const int d = p - first_pair[lo_w];
+        off = first_seg[lo_w] + (d > 0 ? d : 0);
+      }
+    }
+    pair_off[p] = off;
   }
 
-  uint32_t err = s_err ? MLA_DEVERR_SEQLEN : 0u;
-  if (nslots > max_slots(pairs)) err |= MLA_DEVERR_PLAN;
-  meta[kHMagic] = static_cast<int32_t>(kMagic);
-  meta[kHError] = static_cast<int32_t>(err);
-  meta[kHPairs] = pairs;
-  meta[kHWorkRows] = W;
-  meta[kHSegments] = nseg;
-  meta[kHSlots] = nslots;
-  meta[kHRows] = R;
-  meta[kHMTiles] = n_mt;
-  meta[kHBatch] = batch;
-  meta[kHKappa] = kKappa;
-  meta[kHSplitRows] = n_split;
-  meta[kHEmptyRows] = n_empty;
-  meta[kHHq] = h_q;
-  meta[kHSq] = s_q;
-  meta[kHCap] = static_cast<int32_t>(cap);
+  if (threadIdx.x == 0) {
+    uint32_t e = s_err ? MLA_DEVERR_SEQLEN : 0u;
+    if (carry_slot > max_slots(pairs)) e |= MLA_DEVERR_PLAN;
+    meta[kHMagic] = static_cast<int32_t>(kMagic);
+    meta[kHError] = static_cast<int32_t>(e);
+    meta[kHPairs] = pairs;
+    meta[kHWorkRows] = W;
+    meta[kHSegments] = carry_seg;
+    meta[kHSlots] = carry_slot;
+    meta[kHRows] = R;
+    meta[kHMTiles] = n_mt;
+    meta[kHBatch] = batch;
+    meta[kHKappa] = kKappa;
+    meta[kHSplitRows] = carry_split;
+    meta[kHEmptyRows] = carry_empty;
+    meta[kHHq] = h_q;
+    meta[kHSq] = s_q;
+    meta[kHCap] = static_cast<int32_t>(cap < 0x7fffffffLL ? cap : 0x7fffffffLL);
+  }
 }
 
 }  // namespace

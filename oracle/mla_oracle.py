@@ -274,17 +274,17 @@ def combine_partials(parts: List[Tuple[np.ndarray, np.ndarray]]) -> Tuple[np.nda
 # The split-KV plan (integer; compared bit for bit with the metadata kernel)
 # --------------------------------------------------------------------------
 
-def split_plan(seqlens, h_q: int, s_q: int, num_pairs: int, kappa: int) -> dict:
-    """Greedy contiguous partition of all (work row, page) units over ``num_pairs``.
+def split_plan(seqlens, h_q, s_q, num_pairs: int, kappa: int) -> dict:
+    """Cost-interval partition of all (work row, page) units over ``num_pairs``.
 
     A work row is one batch row's block of up to 128 query rows; work rows are
-    ordered m-tile major (w = mt * batch + i).  Each work row with n > 0 pages
-    costs n + kappa (kappa: the fixed per-piece cost in page units).  With
-    T = total cost, each pair may hold cap = ceil(T / P) + 2 * kappa.  Walking
-    the rows in order, the current pair takes as many pages of the current row
-    as fit in cap - used - kappa (at least one); when nothing fits it closes and
-    the next pair starts.  The last pair takes whatever is left.  A work row cut
-    into k > 1 pieces gets k consecutive partial slots, numbered in row order.
+    ordered m-tile major (w = mt * batch + i).  A work row with n > 0 pages
+    costs c = n + kappa (kappa: the fixed cost of starting a row, in page
+    units), else 0.  With C_w the cost of the rows before w and T the total,
+    page b of row w sits at cost position C_w + kappa + b and belongs to pair
+    floor(position / cap), cap = max(1, ceil(T / P)).  Each pair thus takes one
+    contiguous range of pages; a row whose pages land on k > 1 pairs is cut
+    into k pieces and gets k consecutive partial slots, numbered in row order.
     """
     lens = [int(x) for x in as_int(seqlens)]
     batch = len(lens)
@@ -294,26 +294,25 @@ def split_plan(seqlens, h_q: int, s_q: int, num_pairs: int, kappa: int) -> dict:
     n_blk = [0] * W
     for mt in range(n_mt):
         for i in range(batch):
-            n_blk[mt * batch + i] = (lens[i] + PAGE - 1) // PAGE
-    T = sum(n + kappa for n in n_blk if n > 0)
-    cap = (T + num_pairs - 1) // num_pairs + 2 * kappa
+            n_blk[mt * batch + i] = (max(lens[i], 0) + PAGE - 1) // PAGE
+    cost = [(n + kappa) if n > 0 else 0 for n in n_blk]
+    T = sum(cost)
+    cap = max(1, (T + num_pairs - 1) // num_pairs)
     segs = []  # (pair, w, b0, b1)
-    p, used = 0, 0
+    C = 0
     for w in range(W):
         n = n_blk[w]
-        b0 = 0
-        while b0 < n:
-            room = cap - used - kappa
-            if room < 1 and p < num_pairs - 1:
-                p, used = p + 1, 0
-                continue
-            take = (n - b0) if p == num_pairs - 1 else min(n - b0, max(room, 1))
-            segs.append([p, w, b0, b0 + take])
-            used += take + kappa
-            b0 += take
+        if n > 0:
+            first = (C + kappa) // cap
+            last = (C + kappa + n - 1) // cap
+            for p in range(first, last + 1):
+                b0 = max(0, p * cap - C - kappa)
+                b1 = min(n, (p + 1) * cap - C - kappa)
+                segs.append([p, w, b0, b1])
+        C += cost[w]
     pieces = [0] * W
-    for s in segs:
-        pieces[s[1]] += 1
+    for sg in segs:
+        pieces[sg[1]] += 1
     slot_base = [-1] * W
     nslots = 0
     for w in range(W):
@@ -322,22 +321,22 @@ def split_plan(seqlens, h_q: int, s_q: int, num_pairs: int, kappa: int) -> dict:
             nslots += pieces[w]
     seen = [0] * W
     seg_slots = []
-    for s in segs:
-        w = s[1]
+    for sg in segs:
+        w = sg[1]
         if pieces[w] > 1:
             seg_slots.append(slot_base[w] + seen[w])
             seen[w] += 1
         else:
             seg_slots.append(-1)
     pair_off = [0] * (num_pairs + 1)
-    for s in segs:
-        pair_off[s[0] + 1] += 1
+    for sg in segs:
+        pair_off[sg[0] + 1] += 1
     for k in range(num_pairs):
         pair_off[k + 1] += pair_off[k]
     return {
         "num_pairs": num_pairs, "work_rows": W, "n_mt": n_mt, "cap": cap,
-        "segments": [(s[1], s[2], s[3], sl) for s, sl in zip(segs, seg_slots)],
-        "segment_pair": [s[0] for s in segs],
+        "segments": [(sg[1], sg[2], sg[3], sl) for sg, sl in zip(segs, seg_slots)],
+        "segment_pair": [sg[0] for sg in segs],
         "pair_offsets": pair_off,
         "pieces": pieces, "slot_base": slot_base, "num_slots": nslots,
         "split_rows": [w for w in range(W) if pieces[w] > 1],

@@ -98,6 +98,7 @@ def _decode_args(**over):
     (dict(causal=2), binding.MLA_ERR_ARG),
     (dict(scale=float("nan")), binding.MLA_ERR_ARG),
     (dict(scale=float("inf")), binding.MLA_ERR_ARG),
+    (dict(scale=-0.1), binding.MLA_ERR_ARG),
     (dict(h_q=129), binding.MLA_ERR_UNSUPPORTED),
     (dict(s_q=17), binding.MLA_ERR_UNSUPPORTED),
     (dict(num_pages=(1 << 25) + 1), binding.MLA_ERR_UNSUPPORTED),

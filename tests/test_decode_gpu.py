@@ -5,14 +5,14 @@ mean-abs <= 1e-3 on the bf16 output and |lse difference| <= 1e-3, with -inf
 exactly where the oracle has no visible token.  The edge cases keep the
 mean-abs and lse bars; their per-element max-abs bar is the larger of 8e-3 and
 the bound the arithmetic allows when a few tokens carry most of the weight:
-the kernel feeds bf16 weights p~ = p (1 + e), |e| <= 2^-8, to the PV product
-and rounds the output to bf16, so
-    |out_gpu - out| <= 2^-8 (|out| + 2 sum_j w_j |v_j - out|) + 1e-4
-(the factor 2 covers rows split across SM pairs, whose pieces are each
-normalised by their own rounded weights; 1e-4 covers fp32 accumulation and the
-ex2 approximation).  For rows of one to a few tokens with N(0, 1) values this
-bound reaches 1-2e-2, above 8e-3; over the workloads' hundreds to thousands of
-tokens it stays below 8e-3.
+the kernel feeds bf16 weights p~ = p (1 + e), |e| <= 2^-8, to the PV product,
+normalises by the unrounded fp32 sum of the weights (per piece, for rows split
+across SM pairs, whose pieces are then merged with exact weights) and rounds
+the output to bf16, so
+    |out_gpu - out| <= 1.01 * 2^-8 (|out| + sum_j w_j |v_j|) + 1e-4
+(1e-4 covers fp32 accumulation and the ex2 approximation).  For rows of one to
+a few tokens with N(0, 1) values this bound reaches 1-2e-2, above 8e-3; over
+the workloads' hundreds to thousands of tokens it stays below 8e-3.
 
 The plan (metadata) is integer work and must match the oracle's plan bit for
 bit.
@@ -43,7 +43,7 @@ def run(x, check_error=True):
 
 
 def bf16_weight_bound(x, want_o, rows):
-    """Per-element bound 2^-8 (|out| + 2 sum_j w_j |v_j - out|) + 1e-4 (module docstring)."""
+    """Per-element bound 1.01 * 2^-8 (|out| + sum_j w_j |v_j|) + 1e-4 (module docstring)."""
     B = np.zeros_like(want_o)
     for n, i in enumerate(rows):
         L = int(x.seqlens[i])
@@ -59,8 +59,8 @@ def bf16_weight_bound(x, want_o, rows):
                 z = x.softmax_scale * (kv[:lim] @ q[h])
                 w = np.exp(z - z.max())
                 w /= w.sum()
-                spread = w @ np.abs(kv[:lim, :512] - o)
-                B[n, t, h] = 2.0 ** -8 * (np.abs(o) + 2.0 * spread) + 1e-4
+                mag = w @ np.abs(kv[:lim, :512])
+                B[n, t, h] = 1.01 * 2.0 ** -8 * (np.abs(o) + mag) + 1e-4
     return B
 
 

@@ -342,7 +342,7 @@ def test_plan_covers_every_page_once_and_balances(case, kappa):
     load = [0] * P
     for (w, b0, b1, _), p in zip(plan["segments"], plan["segment_pair"]):
         load[p] += b1 - b0 + kappa
-    assert max(load, default=0) <= plan["cap"] + (0 if kappa else 1)
+    assert max(load, default=0) <= plan["cap"] + 2 * kappa
     # pair offsets index the segment list
     offs = plan["pair_offsets"]
     assert offs[0] == 0 and offs[-1] == len(plan["segments"])
