@@ -64,31 +64,33 @@ constexpr uint32_t kKPanel = (kPage / 2) * 128;            // 32 tokens x 64 col
 constexpr uint32_t kKBytes = 9 * kKPanel;                  // this CTA's 32 tokens, 576 cols
 constexpr uint32_t kVPanel = kPage * 128;                  // 64 tokens x 64 cols
 constexpr uint32_t kVBytes = 4 * kVPanel;                  // 64 tokens x this CTA's 256 V cols
-constexpr uint32_t kStageBytes = kKBytes + kVBytes;        // 69632
 constexpr uint32_t kPBytes = kRowsCta * 128;               // 64 rows x 64 tokens bf16
 constexpr uint32_t kOffQ = 0;
-constexpr uint32_t kOffStage = kOffQ + kQBytes;
-constexpr uint32_t kOffP = kOffStage + kStages * kStageBytes;
-constexpr uint32_t kOffMax = kOffP + kPBytes;               // float [2][128]
+constexpr uint32_t kOffK = kOffQ + kQBytes;                 // key-half ring
+constexpr uint32_t kOffV = kOffK + kStages * kKBytes;       // V ring
+constexpr uint32_t kOffP = kOffV + kStages * kVBytes;       // 2 P buffers
+constexpr uint32_t kOffMax = kOffP + 2 * kPBytes;           // float [2][128]
 constexpr uint32_t kOffBar = kOffMax + 2 * 128 * 4;
 constexpr uint32_t kSmemUsed = kOffBar + 256;
 constexpr uint32_t kSmemBytes = kSmemUsed + 1024;  // slack for aligning the base
 
 enum Bar : uint32_t {
   kBarKFull = 0,                  // [kStages] (leader) both CTAs' key halves landed
-  kBarVFull = kStages,            // [kStages] (leader) both CTAs' V columns landed
-  kBarStageEmpty = 2 * kStages,   // [kStages] (both) pair MMAs done with the stage
-  kBarQFull = 3 * kStages,        // (leader) both CTAs' Q rows landed
-  kBarQEmpty = 3 * kStages + 1,   // (both) last QK of the segment done
-  kBarSFull = 3 * kStages + 2,    // [2] (both) S buffer written
-  kBarSEmpty = 3 * kStages + 4,   // [2] (leader) 8 softmax warps read it
-  kBarPFull = 3 * kStages + 6,    // (leader) 8 warps wrote P and rescaled O
-  kBarPvDone = 3 * kStages + 7,   // (both) PV done
-  kBarOEmpty = 3 * kStages + 8,   // (leader) 8 warps read O out
-  kBarFinal = 3 * kStages + 9,    // (leader) MMA drain at teardown
-  kBarXMax = 3 * kStages + 10,    // (both) 4 softmax warps published their row maxima / sums
-  kNumBars = 3 * kStages + 11,
+  kBarKEmpty = 2,                 // [kStages] (both) QK done with the key stage
+  kBarVFull = 4,                  // [kStages] (leader) both CTAs' V columns landed
+  kBarVEmpty = 6,                 // [kStages] (both) PV done with the V stage
+  kBarQFull = 8,                  // (leader) both CTAs' Q rows landed
+  kBarQEmpty = 9,                 // (both) last QK of the segment done
+  kBarSFull = 10,                 // [2] (both) S buffer written
+  kBarPFull = 12,                 // [2] (leader) P buffer written and O rescaled: 4 local warps + relay
+  kBarPLocal = 14,                // [2] (non-leader) its 4 softmax warps, forwarded by the relay
+  kBarPvDone = 16,                // [2] (both) PV of that P buffer done
+  kBarOEmpty = 18,                // (leader) 8 softmax warps read O out
+  kBarFinal = 19,                 // (leader) MMA drain at teardown
+  kBarXMax = 20,                  // (both) 4 softmax warps published their row maxima / sums
+  kNumBars = 21,
 };
+static_assert(kStages == 2, "barrier layout assumes two stages per ring");
 constexpr uint32_t kOffTmemSlot = kOffBar + 8 * kNumBars;  // u32
 constexpr uint32_t kOffAbort = kOffTmemSlot + 4;           // u32
 static_assert(kOffAbort + 4 <= kSmemUsed, "barrier area");
@@ -193,8 +195,33 @@ __device__ __forceinline__ int load_page(const DecodeParams& p, const Ctx& c, co
 
 __device__ void producer(const DecodeParams& p, const Ctx& c, int s_begin, int s_end) {
   const int lane = threadIdx.x & 31;
-  uint32_t kv_cnt = 0, seg_it = 0;
+  uint32_t k_cnt = 0, v_cnt = 0, seg_it = 0;
   bool ok = true;
+  // Key halves run one page ahead of the V columns: the key stage frees after
+  // QK, the V stage only after PV.
+  auto load_k = [&](int page) -> bool {
+    const uint32_t st = k_cnt % kStages;
+    if (!wait_bar(c, c.bar(kBarKEmpty + st), ((k_cnt / kStages) & 1) ^ 1, true)) return false;
+    if (c.cta == 0) mbar_arrive_expect_tx(c.bar(kBarKFull + st), 2 * kKBytes);
+    const uint32_t dst = c.base + kOffK + st * kKBytes;
+    const int ky = page * kPage + c.cta * (kPage / 2);
+#pragma unroll
+    for (int q = 0; q < 9; ++q) tma_load_2d_pair(dst + q * kKPanel, &p.tm_k, c.lead_bar(kBarKFull + st), q * 64, ky);
+    ++k_cnt;
+    return true;
+  };
+  auto load_v = [&](int page) -> bool {
+    const uint32_t st = v_cnt % kStages;
+    if (!wait_bar(c, c.bar(kBarVEmpty + st), ((v_cnt / kStages) & 1) ^ 1, true)) return false;
+    if (c.cta == 0) mbar_arrive_expect_tx(c.bar(kBarVFull + st), 2 * kVBytes);
+    const uint32_t dst = c.base + kOffV + st * kVBytes;
+#pragma unroll
+    for (int q = 0; q < 4; ++q)
+      tma_load_2d_pair(dst + q * kVPanel, &p.tm_v, c.lead_bar(kBarVFull + st),
+                       (q >> 1) * 256 + c.cta * 128 + (q & 1) * 64, page * kPage);
+    ++v_cnt;
+    return true;
+  };
   for (int s = s_begin; s < s_end && ok; ++s) {
     const Segment g = load_segment(p, s);
     if (g.bad) continue;
@@ -214,48 +241,35 @@ __device__ void producer(const DecodeParams& p, const Ctx& c, int s_begin, int s
     ++seg_it;
     const int32_t* table = p.block_table + static_cast<long long>(g.i) * p.max_pages;
     int cur = load_page(p, c, table, g.b0 + lane, g.b1);
+    int prev_page = 0;
     for (int c0 = g.b0; c0 < g.b1 && ok; c0 += 32) {
       const int nxt = load_page(p, c, table, c0 + 32 + lane, g.b1);
       const int n = min(32, g.b1 - c0);
       for (int k = 0; k < n; ++k) {
         const int page = __shfl_sync(0xffffffffu, cur, k);
-        const uint32_t stage = kv_cnt % kStages;
         int good = 1;
         if (lane == 0) {
-          good = wait_bar(c, c.bar(kBarStageEmpty + stage), ((kv_cnt / kStages) & 1) ^ 1, true) ? 1 : 0;
-          if (good) {
-            const uint32_t dst = c.base + kOffStage + stage * kStageBytes;
-            const uint32_t kfull = c.lead_bar(kBarKFull + stage);
-            const uint32_t vfull = c.lead_bar(kBarVFull + stage);
-            if (c.cta == 0) {
-              mbar_arrive_expect_tx(c.bar(kBarKFull + stage), 2 * kKBytes);
-              mbar_arrive_expect_tx(c.bar(kBarVFull + stage), 2 * kVBytes);
-            }
-            const int ky = page * kPage + c.cta * (kPage / 2);
-#pragma unroll
-            for (int q = 0; q < 9; ++q) tma_load_2d_pair(dst + q * kKPanel, &p.tm_k, kfull, q * 64, ky);
-#pragma unroll
-            for (int q = 0; q < 4; ++q)
-              tma_load_2d_pair(dst + kKBytes + q * kVPanel, &p.tm_v, vfull,
-                               (q >> 1) * 256 + c.cta * 128 + (q & 1) * 64, page * kPage);
-          }
+          good = load_k(page) ? 1 : 0;
+          if (good && c0 + k > g.b0) good = load_v(prev_page) ? 1 : 0;  // V of the previous page
         }
         good = __shfl_sync(0xffffffffu, good, 0);
         if (!good) {
           ok = false;
           break;
         }
-        ++kv_cnt;
+        prev_page = page;
       }
       cur = nxt;
     }
+    if (ok && lane == 0) ok = load_v(prev_page);  // V of the segment's last page
+    ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
   }
 }
 
 // ------------------------------------------------------ MMA (leader only) --
 __device__ __forceinline__ void issue_qk(const Ctx& c, uint32_t tmem, uint32_t stage, uint32_t sb) {
   const uint32_t q = c.base + kOffQ;
-  const uint32_t k = c.base + kOffStage + stage * kStageBytes;
+  const uint32_t k = c.base + kOffK + stage * kKBytes;
 #pragma unroll
   for (int s = 0; s < 36; ++s) {
     const uint32_t off = (s & 3) * 32;
@@ -265,8 +279,11 @@ __device__ __forceinline__ void issue_qk(const Ctx& c, uint32_t tmem, uint32_t s
   }
 }
 
+// Issue order per segment: QK(0), then for each page j: QK(j+1), PV(j).
+// The S buffer QK(j+1) writes held S(j-1), which both CTAs had read before
+// signalling P(j-1) ready, and PV(j-1) was issued after that signal.
 __device__ void mma_issuer(const DecodeParams& p, const Ctx& c, uint32_t tmem, int s_begin, int s_end) {
-  uint32_t kv_cnt = 0, q_cnt = 0, pv_cnt = 0, seg_it = 0;
+  uint32_t kv_cnt = 0, q_cnt = 0, seg_it = 0;
   const uint16_t both = 0x3;
   for (int s = s_begin; s < s_end; ++s) {
     const Segment g = load_segment(p, s);
@@ -274,26 +291,24 @@ __device__ void mma_issuer(const DecodeParams& p, const Ctx& c, uint32_t tmem, i
     const int n = g.b1 - g.b0;
     if (!wait_bar(c, c.bar(kBarQFull), seg_it & 1, true)) return;
     for (int j = -1; j < n; ++j) {
-      // QK(j + 1) first, so that it runs while the softmax works on block j.
       if (j + 1 < n) {
-        const uint32_t kvi = kv_cnt + j + 1, sb = q_cnt & 1;
-        if (!wait_bar(c, c.bar(kBarKFull + kvi % kStages), (kvi / kStages) & 1, true)) return;
-        if (!wait_bar(c, c.bar(kBarSEmpty + sb), ((q_cnt >> 1) & 1) ^ 1, true)) return;
+        const uint32_t kvi = kv_cnt + j + 1, st = kvi % kStages, sb = q_cnt & 1;
+        if (!wait_bar(c, c.bar(kBarKFull + st), (kvi / kStages) & 1, true)) return;
         tc_fence_after();
-        issue_qk(c, tmem, kvi % kStages, sb);
+        issue_qk(c, tmem, st, sb);
         umma_commit_pair(c.bar(kBarSFull + sb), both);
+        umma_commit_pair(c.bar(kBarKEmpty + st), both);
         ++q_cnt;
         if (j + 1 == n - 1) umma_commit_pair(c.bar(kBarQEmpty), both);  // Q free once the last QK is done
       }
       if (j < 0) continue;
-      // PV(j)
-      const uint32_t kvj = kv_cnt + j, stage = kvj % kStages;
-      if (!wait_bar(c, c.bar(kBarVFull + stage), (kvj / kStages) & 1, true)) return;
-      if (!wait_bar(c, c.bar(kBarPFull), pv_cnt & 1, true)) return;
+      const uint32_t kvj = kv_cnt + j, st = kvj % kStages, pb = kvj & 1;
+      if (!wait_bar(c, c.bar(kBarVFull + st), (kvj / kStages) & 1, true)) return;
+      if (!wait_bar(c, c.bar(kBarPFull + pb), (kvj >> 1) & 1, true)) return;
       if (j == 0 && seg_it > 0 && !wait_bar(c, c.bar(kBarOEmpty), (seg_it - 1) & 1, true)) return;
       tc_fence_after();
-      const uint32_t pbuf = c.base + kOffP;
-      const uint32_t vbuf = c.base + kOffStage + stage * kStageBytes + kKBytes;
+      const uint32_t pbuf = c.base + kOffP + pb * kPBytes;
+      const uint32_t vbuf = c.base + kOffV + st * kVBytes;
 #pragma unroll
       for (int h = 0; h < 2; ++h) {
 #pragma unroll
@@ -305,12 +320,25 @@ __device__ void mma_issuer(const DecodeParams& p, const Ctx& c, uint32_t tmem, i
           umma_ss_pair(tmem + kColO + 128 * h, a, b, kIdescPV, (j > 0 || k > 0) ? 1u : 0u);
         }
       }
-      umma_commit_pair(c.bar(kBarStageEmpty + stage), both);
-      umma_commit_pair(c.bar(kBarPvDone), both);
-      ++pv_cnt;
+      umma_commit_pair(c.bar(kBarVEmpty + st), both);
+      umma_commit_pair(c.bar(kBarPvDone + pb), both);
     }
     kv_cnt += n;
     ++seg_it;
+  }
+}
+
+// Non-leader only: forwards "P buffer ready" from its 4 softmax warps to the
+// leader, so that the release at cluster scope does not stall the softmax.
+__device__ void relay(const DecodeParams& p, const Ctx& c, int s_begin, int s_end) {
+  uint32_t k = 0;
+  for (int s = s_begin; s < s_end; ++s) {
+    const Segment g = load_segment(p, s);
+    if (g.bad) continue;
+    for (int j = g.b0; j < g.b1; ++j, ++k) {
+      if (!wait_bar(c, c.bar(kBarPLocal + (k & 1)), (k >> 1) & 1)) return;
+      mbar_arrive_remote(c.lead_bar(kBarPFull + (k & 1)));
+    }
   }
 }
 
@@ -327,7 +355,9 @@ __device__ void softmax_epilogue(const DecodeParams& p, const Ctx& c, uint32_t t
   const float sl2 = p.scale_log2;
   // blk_cnt: pages consumed (selects the V stage); x_cnt: row exchanges with
   // the partner thread (selects the exchange slot and the barrier phase).
-  uint32_t s_cnt = 0, pv_cnt = 0, blk_cnt = 0, x_cnt = 0;
+  uint32_t s_cnt = 0, blk_cnt = 0, x_cnt = 0;
+  // Wait until the PV of global page k (P buffer k & 1) has completed.
+  auto pv_done = [&](uint32_t k) -> bool { return wait_bar(c, c.bar(kBarPvDone + (k & 1)), (k >> 1) & 1, true); };
   // Publish v for the partner thread (same row, other half) and return its
   // value; the 4 warps meet on an mbarrier (bounded wait).
   auto trade = [&](float v, float* out) -> bool {
@@ -369,9 +399,6 @@ __device__ void softmax_epilogue(const DecodeParams& p, const Ctx& c, uint32_t t
       float sv[32];
       tmem_ld32(t_s + 32 * sb, sv);
       tmem_wait_ld();
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) arrive_leader(c, kBarSEmpty + sb);
       ++s_cnt;
 
       // ---- mask; block max over both halves of the row ----
@@ -421,13 +448,13 @@ __device__ void softmax_epilogue(const DecodeParams& p, const Ctx& c, uint32_t t
       l = l * alpha + ((e[0] + e[2]) + (e[1] + e[3]));
       m = m_new;
 
-      // ---- previous PV done: P buffer free, O up to date ----
+      // ---- P buffer free (PV two pages back); O up to date for a rescale ----
+      if (blk_cnt >= 2 && !pv_done(blk_cnt - 2)) return;
       if (j > 0) {
-        if (!wait_bar(c, c.bar(kBarPvDone), pv_cnt & 1, true)) return;
-        ++pv_cnt;
-        tc_fence_after();
         const bool need = alpha < 1.0f;
         if (__any_sync(0xffffffffu, need)) {
+          if (!pv_done(blk_cnt - 1)) return;
+          tc_fence_after();
 #pragma unroll 1
           for (int cc = 0; cc < 256; cc += 32) {
             float o[32];
@@ -442,7 +469,7 @@ __device__ void softmax_epilogue(const DecodeParams& p, const Ctx& c, uint32_t t
       }
       // ---- P row hr, this thread's 32 tokens = 4 swizzled 16-byte chunks ----
       {
-        uint8_t* prow = c.gbase + kOffP + (hr >> 3) * 1024 + (hr & 7) * 128;
+        uint8_t* prow = c.gbase + kOffP + (blk_cnt & 1) * kPBytes + (hr >> 3) * 1024 + (hr & 7) * 128;
 #pragma unroll
         for (int q = 0; q < 4; ++q) {
           const int ch = 4 * half + q;
@@ -455,7 +482,7 @@ __device__ void softmax_epilogue(const DecodeParams& p, const Ctx& c, uint32_t t
       if (blk == last_page && (g.L & (kPage - 1))) {
         const int first_bad = g.L - blk * kPage;
         const int chunks = (kPage - first_bad) * 4 * 8;  // rows x panels x 16-byte chunks
-        uint8_t* vst = c.gbase + kOffStage + (blk_cnt % kStages) * kStageBytes + kKBytes;
+        uint8_t* vst = c.gbase + kOffV + (blk_cnt % kStages) * kVBytes;
         for (int e2 = r; e2 < chunks; e2 += 128) {
           const int row = first_bad + (e2 >> 5);
           const int panel = (e2 >> 3) & 3;
@@ -466,13 +493,12 @@ __device__ void softmax_epilogue(const DecodeParams& p, const Ctx& c, uint32_t t
       fence_proxy_async_smem();
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) arrive_leader(c, kBarPFull);
+      if (lane == 0) mbar_arrive(c.bar((c.cta == 0 ? kBarPFull : kBarPLocal) + (blk_cnt & 1)));
       ++blk_cnt;
     }
 
     // ---- epilogue ----
-    if (!wait_bar(c, c.bar(kBarPvDone), pv_cnt & 1, true)) return;
-    ++pv_cnt;
+    if (!pv_done(blk_cnt - 1)) return;
     tc_fence_after();
     float l_peer;
     if (!trade(l, &l_peer)) return;
@@ -546,19 +572,18 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
   if (threadIdx.x == 0) {
     // Barriers of the leader's pipeline are only used in the leader, the
     // rest in both CTAs; initialise all of them everywhere.
-    for (int k = 0; k < kStages; ++k) {
+    for (int k = 0; k < 2; ++k) {
       mbar_init(c.bar(kBarKFull + k), 1);
+      mbar_init(c.bar(kBarKEmpty + k), 1);
       mbar_init(c.bar(kBarVFull + k), 1);
-      mbar_init(c.bar(kBarStageEmpty + k), 1);
+      mbar_init(c.bar(kBarVEmpty + k), 1);
+      mbar_init(c.bar(kBarSFull + k), 1);
+      mbar_init(c.bar(kBarPFull + k), 5);
+      mbar_init(c.bar(kBarPLocal + k), 4);
+      mbar_init(c.bar(kBarPvDone + k), 1);
     }
     mbar_init(c.bar(kBarQFull), 1);
     mbar_init(c.bar(kBarQEmpty), 1);
-    mbar_init(c.bar(kBarSFull + 0), 1);
-    mbar_init(c.bar(kBarSFull + 1), 1);
-    mbar_init(c.bar(kBarSEmpty + 0), 8);
-    mbar_init(c.bar(kBarSEmpty + 1), 8);
-    mbar_init(c.bar(kBarPFull), 8);
-    mbar_init(c.bar(kBarPvDone), 1);
     mbar_init(c.bar(kBarOEmpty), 8);
     mbar_init(c.bar(kBarFinal), 1);
     mbar_init(c.bar(kBarXMax), 4);
@@ -600,6 +625,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     producer(p, c, s_begin, s_end);
   } else if (warp == 1) {
     if (lane == 0 && c.cta == 0) mma_issuer(p, c, tmem, s_begin, s_end);
+    __syncwarp();
+  } else if (warp == 2) {
+    if (lane == 0 && c.cta == 1) relay(p, c, s_begin, s_end);
     __syncwarp();
   } else if (warp >= 4) {
     softmax_epilogue(p, c, tmem, s_begin, s_end);
