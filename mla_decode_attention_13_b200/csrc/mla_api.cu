@@ -65,15 +65,17 @@ int tensor_map_encoder(PFN_cuTensorMapEncodeTiled_v12000* fn) {
   return MLA_OK;
 }
 
-// A [rows][576] bf16 row-major tensor, tiled in boxes of box_cols x box_rows.
-int encode_rows576(PFN_cuTensorMapEncodeTiled_v12000 enc, CUtensorMap* map, const void* base, uint64_t rows,
-                   uint32_t box_cols, uint32_t box_rows, CUtensorMapSwizzle swizzle) {
-  const cuuint64_t dims[2] = {static_cast<cuuint64_t>(kDqk), static_cast<cuuint64_t>(rows)};
-  const cuuint64_t strides[1] = {static_cast<cuuint64_t>(kDqk) * 2};
-  const cuuint32_t box[2] = {box_cols, box_rows};
-  const cuuint32_t elem[2] = {1, 1};
-  const CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box, elem,
-                         CU_TENSOR_MAP_INTERLEAVE_NONE, swizzle, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+// A [rows][576] bf16 row-major tensor viewed as (64 cols, rows, 9 panels)
+// with strides (1152 B, 128 B): a box (64, box_rows, box_panels) lands in
+// shared memory as box_panels panels of box_rows x 128 bytes, 128B-swizzled.
+int encode_panels576(PFN_cuTensorMapEncodeTiled_v12000 enc, CUtensorMap* map, const void* base, uint64_t rows,
+                     uint32_t box_rows, uint32_t box_panels) {
+  const cuuint64_t dims[3] = {64, static_cast<cuuint64_t>(rows), static_cast<cuuint64_t>(kDqk / 64)};
+  const cuuint64_t strides[2] = {static_cast<cuuint64_t>(kDqk) * 2, 128};
+  const cuuint32_t box[3] = {64, box_rows, box_panels};
+  const cuuint32_t elem[3] = {1, 1, 1};
+  const CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box, elem,
+                         CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                          CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   return r == CUDA_SUCCESS ? MLA_OK : MLA_ERR_CUDA;
 }
@@ -112,10 +114,10 @@ int decode_impl(const void* q, const void* kv_cache, int64_t num_pages, const in
   DecodeParams p;
   const uint64_t kv_rows = static_cast<uint64_t>(num_pages) * kPage;
   const uint64_t q_rows = static_cast<uint64_t>(batch) * R;
-  if ((st = encode_rows576(enc, &p.tm_k, kv_cache, kv_rows, 64, kPage / 2, CU_TENSOR_MAP_SWIZZLE_128B)) != MLA_OK ||
-      (st = encode_rows576(enc, &p.tm_v, kv_cache, kv_rows, 64, kPage, CU_TENSOR_MAP_SWIZZLE_128B)) != MLA_OK ||
-      (st = encode_rows576(enc, &p.tm_q, q, q_rows, 64, kMTile / 2, CU_TENSOR_MAP_SWIZZLE_128B)) != MLA_OK)
+  if ((st = encode_panels576(enc, &p.tm_k, kv_cache, kv_rows, kPage / 2, 1)) != MLA_OK ||
+      (st = encode_panels576(enc, &p.tm_q, q, q_rows, kMTile / 2, kDqk / 64)) != MLA_OK)
     return st;
+  p.kv = kv_cache;
   p.block_table = block_table;
   p.seqlens = seqlens;
   p.out = out;

@@ -15,93 +15,131 @@
 // shared memory at the same offsets; the tensor cores share the B halves, and
 // each CTA's 64 rows of the result land in its own TMEM spread over all 128
 // lanes (lanes 0-63 hold the first N/2 columns, lanes 64-127 the rest).
+// Pages go through the pipeline two at a time (a group): a tcgen05.mma costs
+// at least ~64 cycles whatever its size, and QK over one 64-token page (N =
+// 64) would waste three quarters of every instruction.
+//   * Group stage: for each of the group's pages, CTA c TMA-loads its key
+//     half, tokens [32c, 32c + 32) with all 576 columns, so a page leaves HBM
+//     once for the pair.  The stage is nine panels of 64 columns x 64 rows
+//     (rows 0-31: first page, 32-63: second page), 128B-swizzled.
 //   * QK^T: A = Q (64 rows x 576, shared memory, loaded once per segment),
-//     B = the page's cache rows: CTA c TMA-loads tokens [32c, 32c + 32) of each
-//     64-token page, all 576 columns, so the page's keys are read once for
-//     the pair.  S (64 rows x 64 tokens per CTA) lands in 32 TMEM columns:
-//     lane r < 64 holds tokens 0-31 of row r, lane r + 64 tokens 32-63.
-//   * Softmax: thread r (= TMEM lane r) handles row r mod 64, 32 tokens; the
-//     two threads of a row trade their block maxima through shared memory.
-//     Online softmax in the log2 domain with a lazy rescale (the running max
-//     only moves when a block's max exceeds it by more than kTau; O and the
-//     running sums are rescaled together, so the result is exact).  The
-//     bf16-rounded weights P go to shared memory (A operand of PV); the
-//     normaliser and lse use their unrounded fp32 sum.
+//     B = the stage's nine panels, N = 128.  S (64 rows x 128 tokens per CTA)
+//     lands in 64 TMEM columns: lane r < 64 holds tokens 0-31 of both pages
+//     for row r, lane r + 64 tokens 32-63.
+//   * V in place: for PV, CTA c needs all 64 tokens of both pages in its own
+//     value columns [256h + 128c, 256h + 128c + 128) (h = 0, 1), at the same
+//     offsets as its partner.  Its own tokens of those columns are already in
+//     the stage; the four panels that hold the partner's value columns are
+//     dead once QK is done, so CTA c overwrites them with the partner's tokens
+//     of its own value columns (an L2 hit: the partner has just read them).
+//     Panel positions 4h, 4h+1 then hold tokens 0-31 and 4h+2, 4h+3 tokens
+//     32-63 (of both pages) of each CTA's value columns.
+//   * Softmax: thread r (= TMEM lane r) handles row r mod 64, 64 scores (32
+//     tokens of each page); the two threads of a row trade their maxima
+//     through shared memory.  Online softmax in the log2 domain with a lazy
+//     rescale (the running max only moves when a block's max exceeds it by
+//     more than kTau; O and the running sums are rescaled together, so the
+//     result is exact).  The bf16-rounded weights P go to shared memory as
+//     the A operand of PV, tokens 0-31 of both pages (from threads r < 64) in
+//     a buffer of their own, tokens 32-63 (threads r >= 64) in the stage's
+//     rope panel, dead after QK; the normaliser and lse use the unrounded
+//     fp32 sum.
 //   * PV: O (64 rows x 512 per CTA, 256 TMEM columns) += P V in two MMAs of
-//     N = 256; for each, CTA c supplies latent columns [128c, 128c + 128) of
-//     that half for all 64 tokens (its own TMA load of the page's V columns).
+//     N = 256, four K = 16 steps per page.
 //   Pages are gathered through the block table ("FlashMLA overview": paged
-//   kvcache, block size 64); the producer warp reads page ids 32 at a time.
+//   kvcache, block size 64); the producer warps read page ids 32 at a time.
 // A row the plan splits writes fp32 (O / l, lse) partials to the workspace
 // for the combine kernel; an unsplit row writes bf16 out and lse.
-// Warp roles per CTA (256 threads): warp 0 = TMA producer, warp 1 = TMEM
-// owner and (leader only) MMA issuer, warps 4-7 = softmax and epilogue.
+// Warp roles per CTA (256 threads): warp 0 = key/Q producer, warp 1 = TMEM
+// owner and (leader only) MMA issuer, warp 2 = value producer, warp 3 = L2
+// prefetcher (keeps this CTA's key halves of the pages kPrefetchGroups groups
+// ahead of the key loads in L2, so that a stage waits for an L2 hit rather
+// than for DRAM), warps 4-7 = softmax and epilogue.
 //
-// Every mbarrier wait is bounded by %globaltimer; on expiry the kernel sets
-// MLA_DEVERR_TIMEOUT in the metadata error word, tells the peer CTA to stop,
-// drains its own MMAs, frees TMEM and returns.
+// Cross-CTA signals are relaxed arrivals after a CTA-scope fence (see
+// mbar_arrive_remote) and every wait is at CTA scope.  Every mbarrier wait is
+// bounded by %globaltimer; on expiry the kernel sets MLA_DEVERR_TIMEOUT in the
+// metadata error word, tells the peer CTA to stop, drains its own MMAs, frees
+// TMEM and returns.
 #include <cuda_bf16.h>
 
 #include "mla_internal.h"
 #include "sm100_ptx.cuh"
 
 namespace mla {
+
+// Optional clock64 timeline of the pipeline roles, for profiling builds only
+// (compile with -DMLA_DECODE_TRACE; the default build records nothing).
+#ifdef MLA_DECODE_TRACE
+__device__ unsigned long long g_mla_trace[4][16][512];  // [traced CTA][event][page]
+#define MLA_TRACE(ev, k)                                                                     \
+  do {                                                                                       \
+    const int tr_pair_ = static_cast<int>(blockIdx.x >> 1);                                  \
+    const int tr_slot_ = tr_pair_ == 0 ? 0 : (tr_pair_ == 37 ? 2 : -1);                      \
+    if (tr_slot_ >= 0 && (k) < 512) g_mla_trace[tr_slot_ + (blockIdx.x & 1)][ev][k] = clock64(); \
+  } while (0)
+#else
+#define MLA_TRACE(ev, k) \
+  do {                   \
+  } while (0)
+#endif
 namespace {
 
 using namespace ptx;
 
 constexpr int kThreads = 256;
-constexpr int kStages = 2;
-constexpr float kTau = 8.0f;  // lazy-rescale threshold, log2 units
+constexpr int kStages = 2;            // group stages
+constexpr int kGroup = 2;             // pages per group
+constexpr float kTau = 8.0f;          // lazy-rescale threshold, log2 units
 constexpr uint64_t kTimeoutNs = 500ull * 1000ull * 1000ull;
 constexpr int kRowsCta = kMTile / 2;  // 64 query rows per CTA
+constexpr int kHalfPage = kPage / 2;  // 32 tokens of a page per CTA
+constexpr uint32_t kPrefetchGroups = 2;  // L2 prefetch distance ahead of the key loads, in groups
 
 // Shared-memory layout (offsets from a 1024-byte aligned base).  All operand
-// tiles are 128-byte swizzled panels of 64 bf16 columns.
-constexpr uint32_t kQPanel = kRowsCta * 128;               // 64 rows x 64 cols
-constexpr uint32_t kQBytes = 9 * kQPanel;                  // 576 cols
-constexpr uint32_t kKPanel = (kPage / 2) * 128;            // 32 tokens x 64 cols
-constexpr uint32_t kKBytes = 9 * kKPanel;                  // this CTA's 32 tokens, 576 cols
-constexpr uint32_t kVPanel = kPage * 128;                  // 64 tokens x 64 cols
-constexpr uint32_t kVBytes = 4 * kVPanel;                  // 64 tokens x this CTA's 256 V cols
-constexpr uint32_t kPBytes = kRowsCta * 128;               // 64 rows x 64 tokens bf16
+// tiles are 128-byte swizzled panels of 64 bf16 columns x 64 rows.
+constexpr uint32_t kPanel = 64 * 128;            // 8 KB
+constexpr uint32_t kQBytes = 9 * kPanel;         // 64 query rows x 576 cols
+constexpr uint32_t kStageBytes = 9 * kPanel;     // a group: 2 pages x 32 tokens x 576 cols
+constexpr uint32_t kHalfPageBytes = kHalfPage * 128;  // 32 token rows of one panel
+constexpr uint32_t kKBytesPage = 9 * kHalfPageBytes;  // one page's key half (36 KB)
+constexpr uint32_t kVxBytesPage = 4 * kHalfPageBytes; // the partner's tokens of this CTA's value panels (16 KB)
+constexpr uint32_t kRopePos = 8;                 // stage panel that holds P tokens 32-63 after QK
 constexpr uint32_t kOffQ = 0;
-constexpr uint32_t kOffK = kOffQ + kQBytes;                 // key-half ring
-constexpr uint32_t kOffV = kOffK + kStages * kKBytes;       // V ring
-constexpr uint32_t kOffP = kOffV + kStages * kVBytes;       // 2 P buffers
-constexpr uint32_t kOffMax = kOffP + 2 * kPBytes;           // float [2][128]
-constexpr uint32_t kOffBar = kOffMax + 2 * 128 * 4;
-constexpr uint32_t kSmemUsed = kOffBar + 256;
-constexpr uint32_t kSmemBytes = kSmemUsed + 1024;  // slack for aligning the base
+constexpr uint32_t kOffStage = kOffQ + kQBytes;
+constexpr uint32_t kOffP0 = kOffStage + kStages * kStageBytes;  // P tokens 0-31 of both pages
+constexpr uint32_t kOffX = kOffP0 + kPanel;                      // float [2][128] row exchange
+constexpr uint32_t kOffBar = kOffX + 2 * 128 * 4;
 
 enum Bar : uint32_t {
-  kBarKFull = 0,                  // [kStages] (leader) both CTAs' key halves landed
-  kBarKEmpty = 2,                 // [kStages] (both) QK done with the key stage
-  kBarVFull = 4,                  // [kStages] (leader) both CTAs' V columns landed
-  kBarVEmpty = 6,                 // [kStages] (both) PV done with the V stage
-  kBarQFull = 8,                  // (leader) both CTAs' Q rows landed
-  kBarQEmpty = 9,                 // (both) last QK of the segment done
-  kBarSFull = 10,                 // [2] (both) S buffer written
-  kBarPFull = 12,                 // [2] (leader) P buffer written and O rescaled: 4 local warps + relay
-  kBarPLocal = 14,                // [2] (non-leader) its 4 softmax warps, forwarded by the relay
-  kBarPvDone = 16,                // [2] (both) PV of that P buffer done
-  kBarOEmpty = 18,                // (leader) 8 softmax warps read O out
-  kBarFinal = 19,                 // (leader) MMA drain at teardown
-  kBarXMax = 20,                  // (both) 4 softmax warps published their row maxima / sums
-  kNumBars = 21,
+  kBarKFull = 0,                          // [kStages] (leader) both CTAs' key halves landed
+  kBarKEmpty = kBarKFull + kStages,       // [kStages] (both) PV done: stage free
+  kBarQkDone = kBarKEmpty + kStages,      // [kStages] (both) QK done: dead panels may be overwritten
+  kBarVxFull = kBarQkDone + kStages,      // [kStages] (both, local) partner tokens' value panels landed
+  kBarQFull = kBarVxFull + kStages,       // (leader) both CTAs' Q rows landed
+  kBarQEmpty = kBarQFull + 1,             // (both) last QK of the segment done
+  kBarSFull = kBarQEmpty + 1,             // [2] (both) S buffer written
+  kBarPFull = kBarSFull + 2,              // [2] (leader) P written by both CTAs' 4 softmax warps
+  kBarPvDone = kBarPFull + 2,             // [2] (both) PV of that group done
+  kBarOEmpty = kBarPvDone + 2,            // (leader) both CTAs' softmax warps read O out
+  kBarFinal = kBarOEmpty + 1,             // (leader) MMA drain at teardown
+  kBarXch = kBarFinal + 1,                // [2] (both) warps 4+6 / 5+7 published row values
+  kNumBars = kBarXch + 2,
 };
-static_assert(kStages == 2, "barrier layout assumes two stages per ring");
 constexpr uint32_t kOffTmemSlot = kOffBar + 8 * kNumBars;  // u32
 constexpr uint32_t kOffAbort = kOffTmemSlot + 4;           // u32
-static_assert(kOffAbort + 4 <= kSmemUsed, "barrier area");
+constexpr uint32_t kOffKProg = kOffAbort + 4;              // u32: groups whose key loads are issued
+constexpr uint32_t kSmemUsed = kOffKProg + 4;
+constexpr uint32_t kSmemBytes = kSmemUsed + 1024;  // slack for aligning the base
 static_assert(kSmemBytes <= 232448, "shared memory budget");
+static_assert(kOffStage % 1024 == 0 && kStageBytes % 1024 == 0 && kOffP0 % 1024 == 0, "1024-byte aligned tiles");
 
 // Tensor-memory columns (per CTA; the pair allocation mirrors them).
 constexpr uint32_t kTmemCols = 512;
 constexpr uint32_t kColO = 0;    // 256: lanes 0-63 / 64-127 hold the two column halves of each N=256 product
-constexpr uint32_t kColS = 256;  // 2 x 32
+constexpr uint32_t kColS = 256;  // 2 x 64
 
-constexpr uint32_t kIdescQK = idesc_bf16_f32(kMTile, kPage, false);
+constexpr uint32_t kIdescQK = idesc_bf16_f32(kMTile, kGroup * kPage, false);
 constexpr uint32_t kIdescPV = idesc_bf16_f32(kMTile, 256, true);
 
 struct Ctx {
@@ -111,9 +149,11 @@ struct Ctx {
   uint32_t peer_abort;
   uint32_t lead_bars;  // shared::cluster address of the leader's barrier block
   volatile uint32_t* abort_flag;
+  volatile uint32_t* k_prog;
   int32_t* meta;
   __device__ uint32_t bar(uint32_t k) const { return base + kOffBar + 8 * k; }
   __device__ uint32_t lead_bar(uint32_t k) const { return lead_bars + 8 * k; }
+  __device__ uint32_t stage(uint32_t st) const { return base + kOffStage + st * kStageBytes; }
 };
 
 __device__ void raise_abort(const Ctx& c, uint32_t err_bits) {
@@ -124,13 +164,12 @@ __device__ void raise_abort(const Ctx& c, uint32_t err_bits) {
 
 // Bounded wait on an mbarrier phase.  Returns false when the kernel is
 // aborting (this wait timed out, or another role or the peer CTA gave up).
-__device__ bool wait_bar(const Ctx& c, uint32_t bar, uint32_t parity, bool cluster_scope = false) {
+__device__ bool wait_bar(const Ctx& c, uint32_t bar, uint32_t parity) {
   uint32_t spins = 0;
   uint64_t t0 = 0;
   while (true) {
-    const bool ok = cluster_scope ? mbar_try_wait_cluster(bar, parity) : mbar_try_wait(bar, parity);
-    if (ok) return true;
-    if ((++spins & 127u) == 0) {
+    if (mbar_try_wait(bar, parity)) return true;
+    if ((++spins & 63u) == 0) {
       if (*c.abort_flag) return false;
       const uint64_t now = globaltimer();
       if (t0 == 0) {
@@ -144,10 +183,15 @@ __device__ bool wait_bar(const Ctx& c, uint32_t bar, uint32_t parity, bool clust
 }
 
 // Arrive on one of the leader's barriers (locally in the leader, remotely from
-// the other CTA).
+// the other CTA).  The caller's warp has written what the arrival publishes
+// (shared memory of its own CTA, or TMEM reads that completed) and synced.
 __device__ __forceinline__ void arrive_leader(const Ctx& c, uint32_t k) {
-  if (c.cta == 0) mbar_arrive(c.bar(k));
-  else mbar_arrive_remote(c.lead_bar(k));
+  if (c.cta == 0) {
+    mbar_arrive(c.bar(k));
+  } else {
+    fence_cta();
+    mbar_arrive_remote(c.lead_bar(k));
+  }
 }
 
 struct Segment {
@@ -177,11 +221,6 @@ __device__ __forceinline__ Segment load_segment(const DecodeParams& p, int s) {
   return g;
 }
 
-// ------------------------------------------------------------- producer --
-// Whole warp 0 of each CTA: lanes read 32 page ids at a time (one chunk
-// ahead); lane 0 waits for a free stage and loads this CTA's key half (32
-// tokens, 576 columns) and V columns (64 tokens, 256 columns) of each page,
-// completing bytes on the leader's barriers.
 __device__ __forceinline__ int load_page(const DecodeParams& p, const Ctx& c, const int32_t* table, int blk,
                                          int end) {
   if (blk >= end) return 0;
@@ -193,312 +232,429 @@ __device__ __forceinline__ int load_page(const DecodeParams& p, const Ctx& c, co
   return page;
 }
 
-__device__ void producer(const DecodeParams& p, const Ctx& c, int s_begin, int s_end) {
+// A group: up to kGroup consecutive pages of one segment.
+struct Group {
+  int blk;        // first page (logical block index within the row)
+  int np;         // pages in the group, 1 or 2
+  int page[kGroup];
+  bool first;     // first group of its segment
+  bool last;      // last group of its segment
+};
+
+// Walks this pair's segments in plan order and calls fn(segment, group) for
+// every group, with the page ids read 32 at a time by the whole warp (one
+// chunk ahead).  fn runs on every lane and returns false to stop the walk.
+template <typename Fn>
+__device__ __forceinline__ void walk_groups(const DecodeParams& p, const Ctx& c, int s_begin, int s_end, Fn&& fn) {
   const int lane = threadIdx.x & 31;
-  uint32_t k_cnt = 0, v_cnt = 0, seg_it = 0;
-  bool ok = true;
-  // Key halves run one page ahead of the V columns: the key stage frees after
-  // QK, the V stage only after PV.
-  auto load_k = [&](int page) -> bool {
-    const uint32_t st = k_cnt % kStages;
-    if (!wait_bar(c, c.bar(kBarKEmpty + st), ((k_cnt / kStages) & 1) ^ 1, true)) return false;
-    if (c.cta == 0) mbar_arrive_expect_tx(c.bar(kBarKFull + st), 2 * kKBytes);
-    const uint32_t dst = c.base + kOffK + st * kKBytes;
-    const int ky = page * kPage + c.cta * (kPage / 2);
-#pragma unroll
-    for (int q = 0; q < 9; ++q) tma_load_2d_pair(dst + q * kKPanel, &p.tm_k, c.lead_bar(kBarKFull + st), q * 64, ky);
-    ++k_cnt;
-    return true;
-  };
-  auto load_v = [&](int page) -> bool {
-    const uint32_t st = v_cnt % kStages;
-    if (!wait_bar(c, c.bar(kBarVEmpty + st), ((v_cnt / kStages) & 1) ^ 1, true)) return false;
-    if (c.cta == 0) mbar_arrive_expect_tx(c.bar(kBarVFull + st), 2 * kVBytes);
-    const uint32_t dst = c.base + kOffV + st * kVBytes;
-#pragma unroll
-    for (int q = 0; q < 4; ++q)
-      tma_load_2d_pair(dst + q * kVPanel, &p.tm_v, c.lead_bar(kBarVFull + st),
-                       (q >> 1) * 256 + c.cta * 128 + (q & 1) * 64, page * kPage);
-    ++v_cnt;
-    return true;
-  };
-  for (int s = s_begin; s < s_end && ok; ++s) {
-    const Segment g = load_segment(p, s);
-    if (g.bad) continue;
-    // Q rows of this CTA (once per segment, after the previous segment's QKs).
-    if (lane == 0) {
-      ok = seg_it == 0 || wait_bar(c, c.bar(kBarQEmpty), (seg_it - 1) & 1, true);
-      if (ok) {
-        if (c.cta == 0) mbar_arrive_expect_tx(c.bar(kBarQFull), 2 * kQBytes);
-        const int y = g.i * p.R + g.mt * kMTile + c.cta * kRowsCta;
-#pragma unroll
-        for (int q = 0; q < 9; ++q)
-          tma_load_2d_pair(c.base + kOffQ + q * kQPanel, &p.tm_q, c.lead_bar(kBarQFull), q * 64, y);
-      }
-    }
-    ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
-    if (!ok) break;
-    ++seg_it;
-    const int32_t* table = p.block_table + static_cast<long long>(g.i) * p.max_pages;
-    int cur = load_page(p, c, table, g.b0 + lane, g.b1);
-    int prev_page = 0;
-    for (int c0 = g.b0; c0 < g.b1 && ok; c0 += 32) {
-      const int nxt = load_page(p, c, table, c0 + 32 + lane, g.b1);
-      const int n = min(32, g.b1 - c0);
-      for (int k = 0; k < n; ++k) {
-        const int page = __shfl_sync(0xffffffffu, cur, k);
-        int good = 1;
-        if (lane == 0) {
-          good = load_k(page) ? 1 : 0;
-          if (good && c0 + k > g.b0) good = load_v(prev_page) ? 1 : 0;  // V of the previous page
-        }
-        good = __shfl_sync(0xffffffffu, good, 0);
-        if (!good) {
-          ok = false;
-          break;
-        }
-        prev_page = page;
+  for (int s = s_begin; s < s_end; ++s) {
+    const Segment sg = load_segment(p, s);
+    if (sg.bad) continue;
+    const int32_t* table = p.block_table + static_cast<long long>(sg.i) * p.max_pages;
+    int cur = load_page(p, c, table, sg.b0 + lane, sg.b1);
+    for (int c0 = sg.b0; c0 < sg.b1; c0 += 32) {  // 32 is a multiple of kGroup
+      const int nxt = load_page(p, c, table, c0 + 32 + lane, sg.b1);
+      const int n = min(32, sg.b1 - c0);
+      for (int k = 0; k < n; k += kGroup) {
+        Group gr;
+        gr.blk = c0 + k;
+        gr.np = min(kGroup, n - k);
+        gr.page[0] = __shfl_sync(0xffffffffu, cur, k);
+        gr.page[1] = __shfl_sync(0xffffffffu, cur, (k + 1) & 31);
+        gr.first = gr.blk == sg.b0;
+        gr.last = gr.blk + gr.np == sg.b1;
+        if (!fn(sg, gr)) return;
       }
       cur = nxt;
     }
-    if (ok && lane == 0) ok = load_v(prev_page);  // V of the segment's last page
-    ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
   }
+}
+
+// ------------------------------------------------------------- producers --
+// Warp 0: each segment's Q rows of this CTA, then this CTA's key half of
+// every page into the group stages (bytes complete on the leader's barriers).
+__device__ void producer_k(const DecodeParams& p, const Ctx& c, int s_begin, int s_end) {
+  const int lane = threadIdx.x & 31;
+  uint32_t gi = 0, seg_it = 0;  // groups loaded, segments started
+  walk_groups(p, c, s_begin, s_end, [&](const Segment& sg, const Group& gr) -> bool {
+    int good = 1;
+    if (lane == 0) {
+      if (gr.first) {  // the segment's Q rows first
+        good = seg_it == 0 || wait_bar(c, c.bar(kBarQEmpty), (seg_it - 1) & 1);
+        if (good) {
+          if (c.cta == 0) mbar_arrive_expect_tx(c.bar(kBarQFull), 2 * kQBytes);
+          const int y = sg.i * p.R + sg.mt * kMTile + c.cta * kRowsCta;
+          tma_load_3d_pair(c.base + kOffQ, &p.tm_q, c.lead_bar(kBarQFull), 0, y, 0);
+        }
+      }
+      const uint32_t st = gi % kStages;
+      if (good && gi >= kStages) good = wait_bar(c, c.bar(kBarKEmpty + st), ((gi / kStages) - 1) & 1);
+      if (good) {
+        MLA_TRACE(0, gi);
+        const uint32_t bar = c.lead_bar(kBarKFull + st);
+        if (c.cta == 0) mbar_arrive_expect_tx(c.bar(kBarKFull + st), 2 * gr.np * kKBytesPage);
+        for (int q = 0; q < gr.np; ++q) {
+          const int y = gr.page[q] * kPage + static_cast<int>(c.cta) * kHalfPage;
+#pragma unroll
+          for (int pn = 0; pn < 9; ++pn)
+            tma_load_3d_pair(c.stage(st) + pn * kPanel + q * kHalfPageBytes, &p.tm_k, bar, 0, y, pn);
+        }
+      }
+    }
+    if (gr.first) ++seg_it;
+    ++gi;
+    if (lane == 0) *c.k_prog = gi;
+    return __shfl_sync(0xffffffffu, good, 0) != 0;
+  });
+}
+
+// Warp 3: L2 prefetch of this CTA's key half of each page (contiguous: 32
+// token rows of 1152 bytes), at most kPrefetchGroups groups ahead of the key
+// loads.
+__device__ void prefetcher(const DecodeParams& p, const Ctx& c, int s_begin, int s_end) {
+  const int lane = threadIdx.x & 31;
+  uint32_t gi = 0;
+  const uint8_t* kv = static_cast<const uint8_t*>(p.kv);
+  walk_groups(p, c, s_begin, s_end, [&](const Segment&, const Group& gr) -> bool {
+    int good = 1;
+    if (lane == 0) {
+      uint64_t t0 = 0;
+      while (gi >= *c.k_prog + kPrefetchGroups) {
+        if (*c.abort_flag) {
+          good = 0;
+          break;
+        }
+        const uint64_t now = globaltimer();
+        if (t0 == 0) {
+          t0 = now;
+        } else if (now - t0 > kTimeoutNs) {
+          raise_abort(c, MLA_DEVERR_TIMEOUT);
+          good = 0;
+          break;
+        }
+        __nanosleep(256);
+      }
+      if (good) {
+        for (int q = 0; q < gr.np; ++q)
+          prefetch_l2_bulk(kv + (static_cast<long long>(gr.page[q]) * kPage + c.cta * kHalfPage) * (kDqk * 2),
+                           kKBytesPage);
+      }
+    }
+    ++gi;
+    return __shfl_sync(0xffffffffu, good, 0) != 0;
+  });
+}
+
+// Warp 2: once QK of a group is done, overwrite the stage's four panels that
+// held the partner's value columns with the partner's tokens of this CTA's
+// value columns (bytes complete on this CTA's own barrier; the softmax warps
+// wait for it before releasing P, so PV never runs ahead of it).
+__device__ void producer_v(const DecodeParams& p, const Ctx& c, int s_begin, int s_end) {
+  const int lane = threadIdx.x & 31;
+  uint32_t gi = 0;
+  const uint32_t other = c.cta ^ 1u;
+  walk_groups(p, c, s_begin, s_end, [&](const Segment&, const Group& gr) -> bool {
+    int good = 1;
+    if (lane == 0) {
+      const uint32_t st = gi % kStages;
+      good = wait_bar(c, c.bar(kBarQkDone + st), (gi / kStages) & 1);
+      if (good) {
+        MLA_TRACE(3, gi);
+        const uint32_t bar = c.bar(kBarVxFull + st);
+        mbar_arrive_expect_tx(bar, gr.np * kVxBytesPage);
+        for (int q = 0; q < gr.np; ++q) {
+          const int y = gr.page[q] * kPage + static_cast<int>(other) * kHalfPage;
+#pragma unroll
+          for (int v = 0; v < 4; ++v) {
+            const int h = v >> 1, e = v & 1;
+            tma_load_3d(c.stage(st) + (4 * h + 2 * other + e) * kPanel + q * kHalfPageBytes, &p.tm_k, bar, 0, y,
+                        4 * h + 2 * c.cta + e);
+          }
+        }
+      }
+    }
+    ++gi;
+    return __shfl_sync(0xffffffffu, good, 0) != 0;
+  });
 }
 
 // ------------------------------------------------------ MMA (leader only) --
-__device__ __forceinline__ void issue_qk(const Ctx& c, uint32_t tmem, uint32_t stage, uint32_t sb) {
+__device__ __forceinline__ void issue_qk(const Ctx& c, uint32_t tmem, uint32_t st, uint32_t sb) {
   const uint32_t q = c.base + kOffQ;
-  const uint32_t k = c.base + kOffK + stage * kKBytes;
+  const uint32_t k = c.stage(st);
 #pragma unroll
   for (int s = 0; s < 36; ++s) {
     const uint32_t off = (s & 3) * 32;
-    const uint64_t a = smem_desc(q + (s >> 2) * kQPanel + off, 16, 1024, kSwizzle128B);
-    const uint64_t b = smem_desc(k + (s >> 2) * kKPanel + off, 16, 1024, kSwizzle128B);
-    umma_ss_pair(tmem + kColS + 32 * sb, a, b, kIdescQK, s > 0 ? 1u : 0u);
+    const uint64_t a = smem_desc(q + (s >> 2) * kPanel + off, 16, 1024, kSwizzle128B);
+    const uint64_t b = smem_desc(k + (s >> 2) * kPanel + off, 16, 1024, kSwizzle128B);
+    umma_ss_pair(tmem + kColS + 64 * sb, a, b, kIdescQK, s > 0 ? 1u : 0u);
   }
 }
 
-// Issue order per segment: QK(0), then for each page j: QK(j+1), PV(j).
-// The S buffer QK(j+1) writes held S(j-1), which both CTAs had read before
-// signalling P(j-1) ready, and PV(j-1) was issued after that signal.
+// O (+)= P V over the group's np pages.  K step k (16 tokens) of the N = 256
+// half h: P chunk k >> 2 (tokens 0-31 or 32-63 of both pages), its 32-byte
+// column block k & 3; V at panel position 4h (+2 for chunk 1), rows 16 (k & 3)
+// (page k >> 1 & 1), this CTA's 128 value columns being two adjacent panels
+// (leading byte offset = one panel).
+__device__ __forceinline__ void issue_pv(const Ctx& c, uint32_t tmem, uint32_t st, int np, bool first) {
+  const uint32_t v = c.stage(st);
+  const uint32_t chunk[2] = {c.base + kOffP0, v + kRopePos * kPanel};
+#pragma unroll
+  for (int h = 0; h < 2; ++h) {
+    bool acc = !first;
+#pragma unroll
+    for (int k = 0; k < 8; ++k) {
+      if (((k >> 1) & 1) >= np) continue;  // the second page is absent
+      const uint64_t a = smem_desc(chunk[k >> 2] + (k & 3) * 32, 16, 1024, kSwizzle128B);
+      const uint32_t pos = 4 * h + ((k >> 2) << 1);
+      const uint64_t b = smem_desc(v + pos * kPanel + (k & 3) * 2048, kPanel, 1024, kSwizzle128B);
+      umma_ss_pair(tmem + kColO + 128 * h, a, b, kIdescPV, acc ? 1u : 0u);
+      acc = true;
+    }
+  }
+}
+
+// Per segment the MMAs go out as QK(0), then QK(j+1) and PV(j) for each group
+// j, whichever becomes ready first: QK(j+1) when its keys have landed (and
+// PV(j-1) is out: QK(j+1) overwrites the S buffer of group j-1, which both
+// CTAs had read before signalling P(j-1) ready), PV(j) when both CTAs' P(j)
+// is written.  Letting PV(j) overtake a QK whose keys are late frees stage j
+// for the next loads sooner.
 __device__ void mma_issuer(const DecodeParams& p, const Ctx& c, uint32_t tmem, int s_begin, int s_end) {
-  uint32_t kv_cnt = 0, q_cnt = 0, seg_it = 0;
+  uint32_t g0 = 0, seg_it = 0;
   const uint16_t both = 0x3;
   for (int s = s_begin; s < s_end; ++s) {
-    const Segment g = load_segment(p, s);
-    if (g.bad) continue;
-    const int n = g.b1 - g.b0;
-    if (!wait_bar(c, c.bar(kBarQFull), seg_it & 1, true)) return;
-    for (int j = -1; j < n; ++j) {
-      if (j + 1 < n) {
-        const uint32_t kvi = kv_cnt + j + 1, st = kvi % kStages, sb = q_cnt & 1;
-        if (!wait_bar(c, c.bar(kBarKFull + st), (kvi / kStages) & 1, true)) return;
-        tc_fence_after();
-        issue_qk(c, tmem, st, sb);
-        umma_commit_pair(c.bar(kBarSFull + sb), both);
-        umma_commit_pair(c.bar(kBarKEmpty + st), both);
-        ++q_cnt;
-        if (j + 1 == n - 1) umma_commit_pair(c.bar(kBarQEmpty), both);  // Q free once the last QK is done
-      }
-      if (j < 0) continue;
-      const uint32_t kvj = kv_cnt + j, st = kvj % kStages, pb = kvj & 1;
-      if (!wait_bar(c, c.bar(kBarVFull + st), (kvj / kStages) & 1, true)) return;
-      if (!wait_bar(c, c.bar(kBarPFull + pb), (kvj >> 1) & 1, true)) return;
-      if (j == 0 && seg_it > 0 && !wait_bar(c, c.bar(kBarOEmpty), (seg_it - 1) & 1, true)) return;
-      tc_fence_after();
-      const uint32_t pbuf = c.base + kOffP + pb * kPBytes;
-      const uint32_t vbuf = c.base + kOffV + st * kVBytes;
-#pragma unroll
-      for (int h = 0; h < 2; ++h) {
-#pragma unroll
-        for (int k = 0; k < 4; ++k) {
-          const uint64_t a = smem_desc(pbuf + k * 32, 16, 1024, kSwizzle128B);
-          // V: K = 16 tokens from token 16k; this CTA's N/2 = 128 columns of
-          // the half are two panels (leading byte offset = panel stride).
-          const uint64_t b = smem_desc(vbuf + h * 2 * kVPanel + k * 16 * 128, kVPanel, 1024, kSwizzle128B);
-          umma_ss_pair(tmem + kColO + 128 * h, a, b, kIdescPV, (j > 0 || k > 0) ? 1u : 0u);
+    const Segment sg = load_segment(p, s);
+    if (sg.bad) continue;
+    const int n = sg.b1 - sg.b0;
+    const int ng = ceil_div(n, kGroup);
+    if (!wait_bar(c, c.bar(kBarQFull), seg_it & 1)) return;
+    int jq = 0, jp = 0;  // next QK, next PV (groups of this segment)
+    uint64_t t0 = 0;
+    while (jp < ng) {
+      bool did = false;
+      if (jq < ng && jq <= jp + 1) {
+        const uint32_t g = g0 + jq, st = g % kStages, sb = g & 1;
+        if (mbar_test_wait(c.bar(kBarKFull + st), (g / kStages) & 1)) {
+          MLA_TRACE(1, g);
+          tc_fence_after();
+          issue_qk(c, tmem, st, sb);
+          umma_commit_pair(c.bar(kBarSFull + sb), both);
+          umma_commit_pair(c.bar(kBarQkDone + st), both);
+          if (jq == ng - 1) umma_commit_pair(c.bar(kBarQEmpty), both);  // Q free once the last QK is done
+          ++jq;
+          did = true;
         }
       }
-      umma_commit_pair(c.bar(kBarVEmpty + st), both);
-      umma_commit_pair(c.bar(kBarPvDone + pb), both);
+      if (!did && jp < jq) {
+        const uint32_t g = g0 + jp, st = g % kStages, pb = g & 1;
+        if (mbar_test_wait(c.bar(kBarPFull + pb), (g >> 1) & 1) &&
+            (jp > 0 || seg_it == 0 || mbar_test_wait(c.bar(kBarOEmpty), (seg_it - 1) & 1))) {
+          MLA_TRACE(2, g);
+          tc_fence_after();
+          issue_pv(c, tmem, st, min(kGroup, n - kGroup * jp), jp == 0);
+          umma_commit_pair(c.bar(kBarKEmpty + st), both);
+          umma_commit_pair(c.bar(kBarPvDone + pb), both);
+          ++jp;
+          did = true;
+        }
+      }
+      if (did) {
+        t0 = 0;
+        continue;
+      }
+      if (*c.abort_flag) return;
+      const uint64_t now = globaltimer();
+      if (t0 == 0) {
+        t0 = now;
+      } else if (now - t0 > kTimeoutNs) {
+        raise_abort(c, MLA_DEVERR_TIMEOUT);
+        return;
+      }
+      __nanosleep(32);
     }
-    kv_cnt += n;
+    g0 += ng;
     ++seg_it;
-  }
-}
-
-// Non-leader only: forwards "P buffer ready" from its 4 softmax warps to the
-// leader, so that the release at cluster scope does not stall the softmax.
-__device__ void relay(const DecodeParams& p, const Ctx& c, int s_begin, int s_end) {
-  uint32_t k = 0;
-  for (int s = s_begin; s < s_end; ++s) {
-    const Segment g = load_segment(p, s);
-    if (g.bad) continue;
-    for (int j = g.b0; j < g.b1; ++j, ++k) {
-      if (!wait_bar(c, c.bar(kBarPLocal + (k & 1)), (k >> 1) & 1)) return;
-      mbar_arrive_remote(c.lead_bar(kBarPFull + (k & 1)));
-    }
   }
 }
 
 // ---------------------------------------------------- softmax, epilogue --
+// Masks the scores past `nvalid` and returns their maximum (-inf if none).
+__device__ __forceinline__ float masked_max(float (&sv)[32], int nvalid) {
+  if (nvalid < 32) {
+#pragma unroll
+    for (int k = 0; k < 32; ++k) sv[k] = (k < nvalid) ? sv[k] : -INFINITY;
+  }
+  float a[16];
+#pragma unroll
+  for (int k = 0; k < 16; ++k) a[k] = fmaxf(sv[k], sv[k + 16]);
+#pragma unroll
+  for (int k = 0; k < 8; ++k) a[k] = fmaxf(a[k], a[k + 8]);
+#pragma unroll
+  for (int k = 0; k < 4; ++k) a[k] = fmaxf(a[k], a[k + 4]);
+  return fmaxf(fmaxf(a[0], a[2]), fmaxf(a[1], a[3]));
+}
+
+// p = 2^(s * sl2 - m) for the first nvalid scores, 0 past them; packs the
+// bf16-rounded weights in pairs and returns their unrounded fp32 sum.
+__device__ __forceinline__ float exp_pack(const float (&sv)[32], int nvalid, float sl2, float neg_m,
+                                          uint32_t* packed) {
+  float e[16];
+#pragma unroll
+  for (int k = 0; k < 16; ++k) {
+    float a = ex2(fmaf(sv[2 * k], sl2, neg_m));
+    float b = ex2(fmaf(sv[2 * k + 1], sl2, neg_m));
+    if (nvalid < 32) {
+      a = (2 * k < nvalid) ? a : 0.0f;
+      b = (2 * k + 1 < nvalid) ? b : 0.0f;
+    }
+    e[k] = a + b;
+    const __nv_bfloat162 pr = __floats2bfloat162_rn(a, b);
+    packed[k] = *reinterpret_cast<const uint32_t*>(&pr);
+  }
+#pragma unroll
+  for (int k = 0; k < 8; ++k) e[k] += e[k + 8];
+#pragma unroll
+  for (int k = 0; k < 4; ++k) e[k] += e[k + 4];
+  return (e[0] + e[2]) + (e[1] + e[3]);
+}
+
 __device__ void softmax_epilogue(const DecodeParams& p, const Ctx& c, uint32_t tmem, int s_begin, int s_end) {
   const int r = threadIdx.x - 128;  // TMEM lane
   const int lane = threadIdx.x & 31;
   const int hr = r & (kRowsCta - 1);  // query row within this CTA
-  const int half = r >> 6;            // 0: tokens 0-31 / first column half; 1: the rest
+  const int half = r >> 6;            // 0: tokens 0-31 of each page / first column half; 1: the rest
   const uint32_t lane_off = static_cast<uint32_t>(r & ~31) << 16;
   const uint32_t t_s = tmem + lane_off + kColS;
   const uint32_t t_o = tmem + lane_off + kColO;
-  float* smax = reinterpret_cast<float*>(c.gbase + kOffMax);
+  const uint32_t xbar = c.bar(kBarXch + ((r >> 5) & 1));  // warps 4+6 and 5+7 hold the two halves of rows
+  float* xbuf = reinterpret_cast<float*>(c.gbase + kOffX);
+  // This thread's row of P: 128 bytes, 16-byte chunks swizzled by the row.
+  const uint32_t prow_off = (hr >> 3) * 1024 + (hr & 7) * 128;
   const float sl2 = p.scale_log2;
-  // blk_cnt: pages consumed (selects the V stage); x_cnt: row exchanges with
-  // the partner thread (selects the exchange slot and the barrier phase).
-  uint32_t s_cnt = 0, blk_cnt = 0, x_cnt = 0;
-  // Wait until the PV of global page k (P buffer k & 1) has completed.
-  auto pv_done = [&](uint32_t k) -> bool { return wait_bar(c, c.bar(kBarPvDone + (k & 1)), (k >> 1) & 1, true); };
+  // gi: groups consumed so far (selects S and stage buffers and phases);
+  // x_cnt: row exchanges with the partner thread.
+  uint32_t gi = 0, x_cnt = 0;
+  auto pv_done = [&](uint32_t k) -> bool { return wait_bar(c, c.bar(kBarPvDone + (k & 1)), (k >> 1) & 1); };
   // Publish v for the partner thread (same row, other half) and return its
-  // value; the 4 warps meet on an mbarrier (bounded wait).
+  // value; the two warps meet on an mbarrier (bounded wait).
   auto trade = [&](float v, float* out) -> bool {
-    float* buf = smax + (x_cnt & 1) * 128;
+    float* buf = xbuf + (x_cnt & 1) * 128;
     buf[r] = v;
     __syncwarp();
-    if (lane == 0) mbar_arrive(c.bar(kBarXMax));
-    const bool ok = wait_bar(c, c.bar(kBarXMax), x_cnt & 1);
+    if (lane == 0) mbar_arrive(xbar);
+    const bool ok = wait_bar(c, xbar, x_cnt & 1);
     ++x_cnt;
     *out = buf[r ^ 64];
     return ok;
   };
 
   for (int s = s_begin; s < s_end; ++s) {
-    const Segment g = load_segment(p, s);
-    if (g.bad) {
+    const Segment sg = load_segment(p, s);
+    if (sg.bad) {
       if (r == 0 && c.cta == 0) atomicOr(reinterpret_cast<unsigned int*>(c.meta + kHError), MLA_DEVERR_SEQLEN);
       continue;
     }
-    const int n = g.b1 - g.b0;
+    const int n = sg.b1 - sg.b0;
     const int q_row = c.cta * kRowsCta + hr;  // row within the 128-row tile
-    const int row_g = g.mt * kMTile + q_row;
+    const int row_g = sg.mt * kMTile + q_row;
     const bool row_valid = q_row < p.tile_rows && row_g < p.R;
     const int t = row_g / p.h_q;
     const int hh = row_g - t * p.h_q;
     int limit = 0;
     if (row_valid) {
-      limit = p.causal ? g.L - p.s_q + t + 1 : g.L;
-      limit = limit < 0 ? 0 : (limit > g.L ? g.L : limit);
+      limit = p.causal ? sg.L - p.s_q + t + 1 : sg.L;
+      limit = limit < 0 ? 0 : (limit > sg.L ? sg.L : limit);
     }
-    const int last_page = ceil_div(g.L, kPage) - 1;
+    const int last_page = ceil_div(sg.L, kPage) - 1;
 
     float m = -INFINITY, l = 0.0f;  // l: this thread's half of the row sum
-    for (int j = 0; j < n; ++j) {
-      const int blk = g.b0 + j;
-      const uint32_t sb = s_cnt & 1;
-      if (!wait_bar(c, c.bar(kBarSFull + sb), (s_cnt >> 1) & 1, true)) return;
+    for (int j = 0; j < n; j += kGroup, ++gi) {
+      const int blk = sg.b0 + j;
+      const int np = min(kGroup, n - j);
+      const uint32_t sb = gi & 1, st = gi % kStages;
+      if (!wait_bar(c, c.bar(kBarSFull + sb), (gi >> 1) & 1)) return;
+      if (r == 0) MLA_TRACE(4, gi);
       tc_fence_after();
-      float sv[32];
-      tmem_ld32(t_s + 32 * sb, sv);
+      float sv0[32], sv1[32];
+      tmem_ld32(t_s + 64 * sb, sv0);
+      tmem_ld32(t_s + 64 * sb + 32, sv1);
       tmem_wait_ld();
-      ++s_cnt;
 
-      // ---- mask; block max over both halves of the row ----
-      int nvalid = limit - blk * kPage - 32 * half;
-      nvalid = nvalid < 0 ? 0 : (nvalid > 32 ? 32 : nvalid);
-      if (nvalid < 32) {
-#pragma unroll
-        for (int k = 0; k < 32; ++k) sv[k] = (k < nvalid) ? sv[k] : -INFINITY;
-      }
-      float mx;
-      {
-        float a[16];
-#pragma unroll
-        for (int k = 0; k < 16; ++k) a[k] = fmaxf(sv[k], sv[k + 16]);
-#pragma unroll
-        for (int k = 0; k < 8; ++k) a[k] = fmaxf(a[k], a[k + 8]);
-#pragma unroll
-        for (int k = 0; k < 4; ++k) a[k] = fmaxf(a[k], a[k + 4]);
-        mx = fmaxf(fmaxf(a[0], a[2]), fmaxf(a[1], a[3]));
-      }
-      mx = (nvalid > 0) ? mx * sl2 : -INFINITY;  // softmax_scale >= 0
+      // ---- mask; max over both pages and both halves of the row ----
+      int nv0 = limit - blk * kPage - kHalfPage * half;
+      nv0 = nv0 < 0 ? 0 : (nv0 > 32 ? 32 : nv0);
+      int nv1 = limit - (blk + 1) * kPage - kHalfPage * half;
+      nv1 = (np < 2 || nv1 < 0) ? 0 : (nv1 > 32 ? 32 : nv1);
+      float mx = fmaxf(masked_max(sv0, nv0), masked_max(sv1, nv1));
+      mx = (nv0 + nv1 > 0) ? mx * sl2 : -INFINITY;  // softmax_scale >= 0
       float mx_peer;
       if (!trade(mx, &mx_peer)) return;
+      if (r == 0) MLA_TRACE(5, gi);
       mx = fmaxf(mx, mx_peer);
       float m_new = m;
       if (mx > m + kTau) m_new = mx;  // also true for the first finite block
       const float alpha = (m_new == m) ? 1.0f : ex2(m - m_new);  // 0 when m was -inf
       const float neg_m = (m_new == -INFINITY) ? 0.0f : -m_new;
-      uint32_t packed[16];
-      float e[16];
-#pragma unroll
-      for (int k = 0; k < 16; ++k) {
-        float a = ex2(fmaf(sv[2 * k], sl2, neg_m));
-        float b = ex2(fmaf(sv[2 * k + 1], sl2, neg_m));
-        if (nvalid < 32) {
-          a = (2 * k < nvalid) ? a : 0.0f;
-          b = (2 * k + 1 < nvalid) ? b : 0.0f;
-        }
-        e[k] = a + b;
-        const __nv_bfloat162 pr = __floats2bfloat162_rn(a, b);
-        packed[k] = *reinterpret_cast<const uint32_t*>(&pr);
-      }
-#pragma unroll
-      for (int k = 0; k < 8; ++k) e[k] += e[k + 8];
-#pragma unroll
-      for (int k = 0; k < 4; ++k) e[k] += e[k + 4];
-      l = l * alpha + ((e[0] + e[2]) + (e[1] + e[3]));
+      uint32_t packed[32];
+      const float e = exp_pack(sv0, nv0, sl2, neg_m, packed) + exp_pack(sv1, nv1, sl2, neg_m, packed + 16);
+      l = l * alpha + e;
       m = m_new;
 
-      // ---- P buffer free (PV two pages back); O up to date for a rescale ----
-      if (blk_cnt >= 2 && !pv_done(blk_cnt - 2)) return;
-      if (j > 0) {
-        const bool need = alpha < 1.0f;
-        if (__any_sync(0xffffffffu, need)) {
-          if (!pv_done(blk_cnt - 1)) return;
-          tc_fence_after();
+      // ---- the previous group's PV is done: the P buffer of tokens 0-31 is
+      //      free and O is up to date for a rescale ----
+      if (r == 0) MLA_TRACE(6, gi);
+      const bool rescale = j > 0 && __any_sync(0xffffffffu, alpha < 1.0f);
+      if (gi >= 1 && (half == 0 || rescale) && !pv_done(gi - 1)) return;
+      if (rescale) {
+        tc_fence_after();
 #pragma unroll 1
-          for (int cc = 0; cc < 256; cc += 32) {
-            float o[32];
-            tmem_ld32(t_o + cc, o);
-            tmem_wait_ld();
+        for (int cc = 0; cc < 256; cc += 32) {
+          float o[32];
+          tmem_ld32(t_o + cc, o);
+          tmem_wait_ld();
 #pragma unroll
-            for (int k = 0; k < 32; ++k) o[k] *= alpha;
-            tmem_st32(t_o + cc, o);
-          }
-          tmem_wait_st();
+          for (int k = 0; k < 32; ++k) o[k] *= alpha;
+          tmem_st32(t_o + cc, o);
         }
+        tmem_wait_st();
       }
-      // ---- P row hr, this thread's 32 tokens = 4 swizzled 16-byte chunks ----
+      // ---- P row hr: tokens [32 half, 32 half + 32) of both pages ----
+      if (r == 0) MLA_TRACE(7, gi);
       {
-        uint8_t* prow = c.gbase + kOffP + (blk_cnt & 1) * kPBytes + (hr >> 3) * 1024 + (hr & 7) * 128;
+        uint8_t* prow = (half == 0 ? c.gbase + kOffP0 : c.gbase + kOffStage + st * kStageBytes + kRopePos * kPanel) +
+                        prow_off;
 #pragma unroll
-        for (int q = 0; q < 4; ++q) {
-          const int ch = 4 * half + q;
-          *reinterpret_cast<uint4*>(prow + ((ch ^ (hr & 7)) << 4)) =
-              make_uint4(packed[4 * q], packed[4 * q + 1], packed[4 * q + 2], packed[4 * q + 3]);
-        }
+        for (int ci = 0; ci < 8; ++ci)
+          *reinterpret_cast<uint4*>(prow + ((ci ^ (hr & 7)) << 4)) =
+              make_uint4(packed[4 * ci], packed[4 * ci + 1], packed[4 * ci + 2], packed[4 * ci + 3]);
       }
-      // ---- the last page of a row may hold garbage (even NaN) past L: zero
-      //      this CTA's V rows there so that 0 * garbage cannot reach O ----
-      if (blk == last_page && (g.L & (kPage - 1))) {
-        const int first_bad = g.L - blk * kPage;
-        const int chunks = (kPage - first_bad) * 4 * 8;  // rows x panels x 16-byte chunks
-        uint8_t* vst = c.gbase + kOffV + (blk_cnt % kStages) * kVBytes;
+      // ---- the partner's value panels have landed; the last page of a row
+      //      may hold garbage (even NaN) past L: zero the value rows there
+      //      that PV reads, so that 0 * garbage cannot reach O ----
+      if (!wait_bar(c, c.bar(kBarVxFull + st), (gi / kStages) & 1)) return;
+      if (r == 0) MLA_TRACE(8, gi);
+      if ((sg.L & (kPage - 1)) && last_page >= blk && last_page < blk + np) {
+        const int q = last_page - blk;
+        const int first_bad = sg.L - last_page * kPage;
+        const int chunks = (kPage - first_bad) * 4 * 8;  // tokens x panels x 16-byte chunks
+        uint8_t* stg = c.gbase + kOffStage + st * kStageBytes + q * kHalfPageBytes;
         for (int e2 = r; e2 < chunks; e2 += 128) {
-          const int row = first_bad + (e2 >> 5);
-          const int panel = (e2 >> 3) & 3;
-          const int ch = e2 & 7;
-          *reinterpret_cast<uint4*>(vst + panel * kVPanel + row * 128 + ch * 16) = make_uint4(0, 0, 0, 0);
+          const int tok = first_bad + (e2 >> 5);
+          const int v = (e2 >> 3) & 3;
+          const int pos = (v & 1) + 4 * (v >> 1) + (tok >= kHalfPage ? 2 : 0);
+          *reinterpret_cast<uint4*>(stg + pos * kPanel + (tok & 31) * 128 + (e2 & 7) * 16) = make_uint4(0, 0, 0, 0);
         }
       }
       fence_proxy_async_smem();
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive(c.bar((c.cta == 0 ? kBarPFull : kBarPLocal) + (blk_cnt & 1)));
-      ++blk_cnt;
+      if (lane == 0) arrive_leader(c, kBarPFull + sb);
+      if (r == 0) MLA_TRACE(9, gi);
     }
 
     // ---- epilogue ----
-    if (!pv_done(blk_cnt - 1)) return;
+    if (!pv_done(gi - 1)) return;
     tc_fence_after();
     float l_peer;
     if (!trade(l, &l_peer)) return;
@@ -507,8 +663,8 @@ __device__ void softmax_epilogue(const DecodeParams& p, const Ctx& c, uint32_t t
     const float lse_v = lt > 0.0f ? (m + __log2f(lt)) * 0.69314718055994530942f : -INFINITY;
     // This thread's O columns: for each half h of the 512, columns
     // [256h + 128*half, 256h + 128*half + 128).
-    if (g.slot < 0) {
-      __nv_bfloat16* orow = reinterpret_cast<__nv_bfloat16*>(p.out) + (static_cast<long long>(g.i) * p.R + row_g) * kDv;
+    if (sg.slot < 0) {
+      __nv_bfloat16* orow = reinterpret_cast<__nv_bfloat16*>(p.out) + (static_cast<long long>(sg.i) * p.R + row_g) * kDv;
 #pragma unroll 1
       for (int cc = 0; cc < 256; cc += 32) {
         float o[32];
@@ -531,9 +687,9 @@ __device__ void softmax_epilogue(const DecodeParams& p, const Ctx& c, uint32_t t
           }
         }
       }
-      if (row_valid && half == 0) p.lse[(static_cast<long long>(g.i) * p.h_q + hh) * p.s_q + t] = lse_v;
+      if (row_valid && half == 0) p.lse[(static_cast<long long>(sg.i) * p.h_q + hh) * p.s_q + t] = lse_v;
     } else {
-      float* orow = p.o_part + (static_cast<long long>(g.slot) * p.tile_rows + q_row) * kDv;
+      float* orow = p.o_part + (static_cast<long long>(sg.slot) * p.tile_rows + q_row) * kDv;
 #pragma unroll 1
       for (int cc = 0; cc < 256; cc += 32) {
         float o[32];
@@ -547,7 +703,7 @@ __device__ void softmax_epilogue(const DecodeParams& p, const Ctx& c, uint32_t t
                 make_float4(o[k] * inv_l, o[k + 1] * inv_l, o[k + 2] * inv_l, o[k + 3] * inv_l);
         }
       }
-      if (row_valid && half == 0) p.lse_part[static_cast<long long>(g.slot) * p.tile_rows + q_row] = lse_v;
+      if (row_valid && half == 0) p.lse_part[static_cast<long long>(sg.slot) * p.tile_rows + q_row] = lse_v;
     }
     tc_fence_before();
     __syncwarp();
@@ -566,28 +722,31 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
   c.cta = cluster_ctarank();
   c.meta = p.meta;
   c.abort_flag = reinterpret_cast<volatile uint32_t*>(c.gbase + kOffAbort);
+  c.k_prog = reinterpret_cast<volatile uint32_t*>(c.gbase + kOffKProg);
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
 
   if (threadIdx.x == 0) {
     // Barriers of the leader's pipeline are only used in the leader, the
     // rest in both CTAs; initialise all of them everywhere.
-    for (int k = 0; k < 2; ++k) {
+    for (int k = 0; k < kStages; ++k) {
       mbar_init(c.bar(kBarKFull + k), 1);
       mbar_init(c.bar(kBarKEmpty + k), 1);
-      mbar_init(c.bar(kBarVFull + k), 1);
-      mbar_init(c.bar(kBarVEmpty + k), 1);
+      mbar_init(c.bar(kBarQkDone + k), 1);
+      mbar_init(c.bar(kBarVxFull + k), 1);
+    }
+    for (int k = 0; k < 2; ++k) {
       mbar_init(c.bar(kBarSFull + k), 1);
-      mbar_init(c.bar(kBarPFull + k), 5);
-      mbar_init(c.bar(kBarPLocal + k), 4);
+      mbar_init(c.bar(kBarPFull + k), 8);
       mbar_init(c.bar(kBarPvDone + k), 1);
+      mbar_init(c.bar(kBarXch + k), 2);
     }
     mbar_init(c.bar(kBarQFull), 1);
     mbar_init(c.bar(kBarQEmpty), 1);
     mbar_init(c.bar(kBarOEmpty), 8);
     mbar_init(c.bar(kBarFinal), 1);
-    mbar_init(c.bar(kBarXMax), 4);
     *c.abort_flag = 0u;
+    *c.k_prog = 0u;
     fence_mbar_init_cluster();
   }
   if (warp == 1) {
@@ -596,7 +755,6 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
   }
   if (warp == 0 && lane == 0) {
     tma_prefetch_desc(&p.tm_k);
-    tma_prefetch_desc(&p.tm_v);
     tma_prefetch_desc(&p.tm_q);
   }
   tc_fence_before();
@@ -622,14 +780,15 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
   }
 
   if (warp == 0) {
-    producer(p, c, s_begin, s_end);
+    producer_k(p, c, s_begin, s_end);
   } else if (warp == 1) {
     if (lane == 0 && c.cta == 0) mma_issuer(p, c, tmem, s_begin, s_end);
     __syncwarp();
   } else if (warp == 2) {
-    if (lane == 0 && c.cta == 1) relay(p, c, s_begin, s_end);
-    __syncwarp();
-  } else if (warp >= 4) {
+    producer_v(p, c, s_begin, s_end);
+  } else if (warp == 3) {
+    prefetcher(p, c, s_begin, s_end);
+  } else {
     softmax_epilogue(p, c, tmem, s_begin, s_end);
   }
 
@@ -655,6 +814,16 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
 }
 
 }  // namespace
+
+#ifdef MLA_DECODE_TRACE
+extern "C" __attribute__((visibility("default"))) int mla_trace_read(void* host) {
+  return static_cast<int>(cudaMemcpyFromSymbol(host, g_mla_trace, sizeof(g_mla_trace)));
+}
+extern "C" __attribute__((visibility("default"))) int mla_trace_clear() {
+  static unsigned long long zero[4][16][512];
+  return static_cast<int>(cudaMemcpyToSymbol(g_mla_trace, zero, sizeof(zero)));
+}
+#endif
 
 size_t decode_kernel_smem_bytes() { return kSmemBytes; }
 
