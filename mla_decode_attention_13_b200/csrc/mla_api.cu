@@ -115,6 +115,7 @@ int decode_impl(const void* q, const void* kv_cache, int64_t num_pages, const in
   const uint64_t kv_rows = static_cast<uint64_t>(num_pages) * kPage;
   const uint64_t q_rows = static_cast<uint64_t>(batch) * R;
   if ((st = encode_panels576(enc, &p.tm_k, kv_cache, kv_rows, kPage / 2, 1)) != MLA_OK ||
+      (st = encode_panels576(enc, &p.tm_v, kv_cache, kv_rows, kPage, 2)) != MLA_OK ||
       (st = encode_panels576(enc, &p.tm_q, q, q_rows, kMTile / 2, kDqk / 64)) != MLA_OK)
     return st;
   p.kv = kv_cache;

@@ -15,46 +15,42 @@
 // shared memory at the same offsets; the tensor cores share the B halves, and
 // each CTA's 64 rows of the result land in its own TMEM spread over all 128
 // lanes (lanes 0-63 hold the first N/2 columns, lanes 64-127 the rest).
-// Pages go through the pipeline two at a time (a group): a tcgen05.mma costs
-// at least ~64 cycles whatever its size, and QK over one 64-token page (N =
-// 64) would waste three quarters of every instruction.
-//   * Group stage: for each of the group's pages, CTA c TMA-loads its key
-//     half, tokens [32c, 32c + 32) with all 576 columns, so a page leaves HBM
-//     once for the pair.  The stage is nine panels of 64 columns x 64 rows
-//     (rows 0-31: first page, 32-63: second page), 128B-swizzled.
+//
+// A tcgen05.mma costs at least ~64 cycles whatever its size, and a pair MMA
+// only reaches the tensor peak at N = 256, so QK^T runs over four pages at a
+// time (a group, 256 tokens); PV runs page by page at N = 256.
+//   * Keys: CTA c supplies tokens [32c, 32c + 32) of each page of the group,
+//     all 576 columns, so a page leaves HBM once for the pair.  They stream
+//     through a ring of panels (64 columns x 128 token rows, 16 KB); a panel
+//     is free again as soon as its four K = 16 MMAs are done.
 //   * QK^T: A = Q (64 rows x 576, shared memory, loaded once per segment),
-//     B = the stage's nine panels, N = 128.  S (64 rows x 128 tokens per CTA)
-//     lands in 64 TMEM columns: lane r < 64 holds tokens 0-31 of both pages
-//     for row r, lane r + 64 tokens 32-63.
-//   * V in place: for PV, CTA c needs all 64 tokens of both pages in its own
-//     value columns [256h + 128c, 256h + 128c + 128) (h = 0, 1), at the same
-//     offsets as its partner.  Its own tokens of those columns are already in
-//     the stage; the four panels that hold the partner's value columns are
-//     dead once QK is done, so CTA c overwrites them with the partner's tokens
-//     of its own value columns (an L2 hit: the partner has just read them).
-//     Panel positions 4h, 4h+1 then hold tokens 0-31 and 4h+2, 4h+3 tokens
-//     32-63 (of both pages) of each CTA's value columns.
-//   * Softmax: thread r (= TMEM lane r) handles row r mod 64, 64 scores (32
+//     B = the group's panels, N = 256.  S (64 rows x 256 tokens per CTA)
+//     lands in 128 TMEM columns: lane r < 64 holds tokens 0-31 of the four
+//     pages for row r, lane r + 64 tokens 32-63.
+//   * Values: for PV, CTA c needs all 64 tokens of a page in its value
+//     columns [256h + 128c, 256h + 128c + 128) (h = 0, 1): a 32 KB tile per
+//     page, read from L2 (the pair has just brought the page in), in a ring
+//     of two.
+//   * Softmax: thread r (= TMEM lane r) handles row r mod 64, 128 scores (32
 //     tokens of each page); the two threads of a row trade their maxima
 //     through shared memory.  Online softmax in the log2 domain with a lazy
 //     rescale (the running max only moves when a block's max exceeds it by
 //     more than kTau; O and the running sums are rescaled together, so the
-//     result is exact).  The bf16-rounded weights P go to shared memory as
-//     the A operand of PV, tokens 0-31 of both pages (from threads r < 64) in
-//     a buffer of their own, tokens 32-63 (threads r >= 64) in the stage's
-//     rope panel, dead after QK; the normaliser and lse use the unrounded
-//     fp32 sum.
-//   * PV: O (64 rows x 512 per CTA, 256 TMEM columns) += P V in two MMAs of
-//     N = 256, four K = 16 steps per page.
-//   Pages are gathered through the block table ("FlashMLA overview": paged
-//   kvcache, block size 64); the producer warps read page ids 32 at a time.
+//     result is exact).  The bf16-rounded weights P of each page go to a ring
+//     of two shared-memory tiles (A operand of PV); the normaliser and lse use
+//     the unrounded fp32 sum.
+//   * PV: O (64 rows x 512 per CTA, 256 TMEM columns) += P V per page, in two
+//     MMAs of N = 256 (four K = 16 steps each).
+//   Two threads issue the MMAs, one the QK panels and one the PV pages, so
+//   that the next group's QK overlaps this group's PV.  Pages are gathered through the
+//   block table ("FlashMLA overview": paged kvcache, block size 64); the
+//   producer warps read page ids 32 at a time.
 // A row the plan splits writes fp32 (O / l, lse) partials to the workspace
 // for the combine kernel; an unsplit row writes bf16 out and lse.
 // Warp roles per CTA (256 threads): warp 0 = key/Q producer, warp 1 = TMEM
-// owner and (leader only) MMA issuer, warp 2 = value producer, warp 3 = L2
-// prefetcher (keeps this CTA's key halves of the pages kPrefetchGroups groups
-// ahead of the key loads in L2, so that a stage waits for an L2 hit rather
-// than for DRAM), warps 4-7 = softmax and epilogue.
+// owner and (leader only) QK issuer, warp 2 = value producer, warp 3 =
+// (leader only) PV issuer, warps 4-7 = softmax and epilogue.  (A bulk L2 prefetch of the pages ahead of the key
+// loads was measured on B200 and made the kernel slower; there is none.)
 //
 // Cross-CTA signals are relaxed arrivals after a CTA-scope fence (see
 // mbar_arrive_remote) and every wait is at CTA scope.  Every mbarrier wait is
@@ -71,11 +67,11 @@ namespace mla {
 // Optional clock64 timeline of the pipeline roles, for profiling builds only
 // (compile with -DMLA_DECODE_TRACE; the default build records nothing).
 #ifdef MLA_DECODE_TRACE
-__device__ unsigned long long g_mla_trace[4][16][512];  // [traced CTA][event][page]
-#define MLA_TRACE(ev, k)                                                                     \
-  do {                                                                                       \
-    const int tr_pair_ = static_cast<int>(blockIdx.x >> 1);                                  \
-    const int tr_slot_ = tr_pair_ == 0 ? 0 : (tr_pair_ == 37 ? 2 : -1);                      \
+__device__ unsigned long long g_mla_trace[4][16][512];  // [traced CTA][event][index]
+#define MLA_TRACE(ev, k)                                                                         \
+  do {                                                                                           \
+    const int tr_pair_ = static_cast<int>(blockIdx.x >> 1);                                      \
+    const int tr_slot_ = tr_pair_ == 0 ? 0 : (tr_pair_ == 37 ? 2 : -1);                          \
     if (tr_slot_ >= 0 && (k) < 512) g_mla_trace[tr_slot_ + (blockIdx.x & 1)][ev][k] = clock64(); \
   } while (0)
 #else
@@ -83,61 +79,62 @@ __device__ unsigned long long g_mla_trace[4][16][512];  // [traced CTA][event][p
   do {                   \
   } while (0)
 #endif
+
 namespace {
 
 using namespace ptx;
 
 constexpr int kThreads = 256;
-constexpr int kStages = 2;            // group stages
-constexpr int kGroup = 2;             // pages per group
+constexpr int kGroup = 4;             // pages per QK group
+constexpr int kKRing = 4;             // key panel slots
+constexpr int kVRing = 2;             // value tiles (and P tiles)
 constexpr float kTau = 8.0f;          // lazy-rescale threshold, log2 units
 constexpr uint64_t kTimeoutNs = 500ull * 1000ull * 1000ull;
 constexpr int kRowsCta = kMTile / 2;  // 64 query rows per CTA
 constexpr int kHalfPage = kPage / 2;  // 32 tokens of a page per CTA
-constexpr uint32_t kPrefetchGroups = 2;  // L2 prefetch distance ahead of the key loads, in groups
 
 // Shared-memory layout (offsets from a 1024-byte aligned base).  All operand
-// tiles are 128-byte swizzled panels of 64 bf16 columns x 64 rows.
-constexpr uint32_t kPanel = 64 * 128;            // 8 KB
-constexpr uint32_t kQBytes = 9 * kPanel;         // 64 query rows x 576 cols
-constexpr uint32_t kStageBytes = 9 * kPanel;     // a group: 2 pages x 32 tokens x 576 cols
-constexpr uint32_t kHalfPageBytes = kHalfPage * 128;  // 32 token rows of one panel
-constexpr uint32_t kKBytesPage = 9 * kHalfPageBytes;  // one page's key half (36 KB)
-constexpr uint32_t kVxBytesPage = 4 * kHalfPageBytes; // the partner's tokens of this CTA's value panels (16 KB)
-constexpr uint32_t kRopePos = 8;                 // stage panel that holds P tokens 32-63 after QK
+// tiles are 128-byte swizzled panels of 64 bf16 columns.
+constexpr uint32_t kQPanel = kRowsCta * 128;            // 64 rows x 64 cols
+constexpr uint32_t kQBytes = 9 * kQPanel;               // 64 query rows x 576 cols
+constexpr uint32_t kHalfPageBytes = kHalfPage * 128;    // 32 token rows x 64 cols
+constexpr uint32_t kKSlot = kGroup * kHalfPageBytes;    // one panel of a group: 128 token rows
+constexpr uint32_t kVPanel = kPage * 128;               // 64 tokens x 64 cols
+constexpr uint32_t kVTile = 4 * kVPanel;                // 64 tokens x this CTA's 256 value cols
+constexpr uint32_t kPTile = kRowsCta * 128;             // 64 rows x 64 tokens bf16
 constexpr uint32_t kOffQ = 0;
-constexpr uint32_t kOffStage = kOffQ + kQBytes;
-constexpr uint32_t kOffP0 = kOffStage + kStages * kStageBytes;  // P tokens 0-31 of both pages
-constexpr uint32_t kOffX = kOffP0 + kPanel;                      // float [2][128] row exchange
+constexpr uint32_t kOffK = kOffQ + kQBytes;
+constexpr uint32_t kOffV = kOffK + kKRing * kKSlot;
+constexpr uint32_t kOffP = kOffV + kVRing * kVTile;
+constexpr uint32_t kOffX = kOffP + kVRing * kPTile;     // float [2][128] row exchange
 constexpr uint32_t kOffBar = kOffX + 2 * 128 * 4;
 
 enum Bar : uint32_t {
-  kBarKFull = 0,                          // [kStages] (leader) both CTAs' key halves landed
-  kBarKEmpty = kBarKFull + kStages,       // [kStages] (both) PV done: stage free
-  kBarQkDone = kBarKEmpty + kStages,      // [kStages] (both) QK done: dead panels may be overwritten
-  kBarVxFull = kBarQkDone + kStages,      // [kStages] (both, local) partner tokens' value panels landed
-  kBarQFull = kBarVxFull + kStages,       // (leader) both CTAs' Q rows landed
-  kBarQEmpty = kBarQFull + 1,             // (both) last QK of the segment done
-  kBarSFull = kBarQEmpty + 1,             // [2] (both) S buffer written
-  kBarPFull = kBarSFull + 2,              // [2] (leader) P written by both CTAs' 4 softmax warps
-  kBarPvDone = kBarPFull + 2,             // [2] (both) PV of that group done
-  kBarOEmpty = kBarPvDone + 2,            // (leader) both CTAs' softmax warps read O out
-  kBarFinal = kBarOEmpty + 1,             // (leader) MMA drain at teardown
-  kBarXch = kBarFinal + 1,                // [2] (both) warps 4+6 / 5+7 published row values
+  kBarKFull = 0,                       // [kKRing] (leader) both CTAs' key panel landed
+  kBarKEmpty = kBarKFull + kKRing,     // [kKRing] (both) the panel's QK MMAs are done
+  kBarVFull = kBarKEmpty + kKRing,     // [kVRing] (both, local) this CTA's value tile landed
+  kBarPFull = kBarVFull + kVRing,      // [kVRing] (leader) P written by both CTAs' 4 softmax warps
+  kBarPvDone = kBarPFull + kVRing,     // [kVRing] (both) PV of that page done: P and value tiles free
+  kBarSFull = kBarPvDone + kVRing,     // [2] (both) S buffer written
+  kBarSEmpty = kBarSFull + 2,          // [2] (leader) both CTAs' softmax warps read the S buffer
+  kBarQFull = kBarSEmpty + 2,          // (leader) both CTAs' Q rows landed
+  kBarQEmpty = kBarQFull + 1,          // (both) last QK of the segment done
+  kBarOEmpty = kBarQEmpty + 1,         // (leader) both CTAs' softmax warps read O out
+  kBarFinal = kBarOEmpty + 1,          // (leader) MMA drain at teardown: both issuer threads
+  kBarXch = kBarFinal + 1,             // [2] (both) warps 4+6 / 5+7 published row values
   kNumBars = kBarXch + 2,
 };
 constexpr uint32_t kOffTmemSlot = kOffBar + 8 * kNumBars;  // u32
 constexpr uint32_t kOffAbort = kOffTmemSlot + 4;           // u32
-constexpr uint32_t kOffKProg = kOffAbort + 4;              // u32: groups whose key loads are issued
-constexpr uint32_t kSmemUsed = kOffKProg + 4;
+constexpr uint32_t kSmemUsed = kOffAbort + 4;
 constexpr uint32_t kSmemBytes = kSmemUsed + 1024;  // slack for aligning the base
 static_assert(kSmemBytes <= 232448, "shared memory budget");
-static_assert(kOffStage % 1024 == 0 && kStageBytes % 1024 == 0 && kOffP0 % 1024 == 0, "1024-byte aligned tiles");
+static_assert(kOffK % 1024 == 0 && kOffV % 1024 == 0 && kOffP % 1024 == 0, "1024-byte aligned tiles");
 
 // Tensor-memory columns (per CTA; the pair allocation mirrors them).
 constexpr uint32_t kTmemCols = 512;
 constexpr uint32_t kColO = 0;    // 256: lanes 0-63 / 64-127 hold the two column halves of each N=256 product
-constexpr uint32_t kColS = 256;  // 2 x 64
+constexpr uint32_t kColS = 256;  // 2 x 128
 
 constexpr uint32_t kIdescQK = idesc_bf16_f32(kMTile, kGroup * kPage, false);
 constexpr uint32_t kIdescPV = idesc_bf16_f32(kMTile, 256, true);
@@ -149,11 +146,12 @@ struct Ctx {
   uint32_t peer_abort;
   uint32_t lead_bars;  // shared::cluster address of the leader's barrier block
   volatile uint32_t* abort_flag;
-  volatile uint32_t* k_prog;
   int32_t* meta;
   __device__ uint32_t bar(uint32_t k) const { return base + kOffBar + 8 * k; }
   __device__ uint32_t lead_bar(uint32_t k) const { return lead_bars + 8 * k; }
-  __device__ uint32_t stage(uint32_t st) const { return base + kOffStage + st * kStageBytes; }
+  __device__ uint32_t kslot(uint32_t k) const { return base + kOffK + k * kKSlot; }
+  __device__ uint32_t vtile(uint32_t k) const { return base + kOffV + k * kVTile; }
+  __device__ uint32_t ptile(uint32_t k) const { return base + kOffP + k * kPTile; }
 };
 
 __device__ void raise_abort(const Ctx& c, uint32_t err_bits) {
@@ -235,10 +233,9 @@ __device__ __forceinline__ int load_page(const DecodeParams& p, const Ctx& c, co
 // A group: up to kGroup consecutive pages of one segment.
 struct Group {
   int blk;        // first page (logical block index within the row)
-  int np;         // pages in the group, 1 or 2
+  int np;         // pages in the group, 1 to kGroup
   int page[kGroup];
   bool first;     // first group of its segment
-  bool last;      // last group of its segment
 };
 
 // Walks this pair's segments in plan order and calls fn(segment, group) for
@@ -246,23 +243,23 @@ struct Group {
 // chunk ahead).  fn runs on every lane and returns false to stop the walk.
 template <typename Fn>
 __device__ __forceinline__ void walk_groups(const DecodeParams& p, const Ctx& c, int s_begin, int s_end, Fn&& fn) {
+  static_assert(32 % kGroup == 0, "groups never straddle a chunk of page ids");
   const int lane = threadIdx.x & 31;
   for (int s = s_begin; s < s_end; ++s) {
     const Segment sg = load_segment(p, s);
     if (sg.bad) continue;
     const int32_t* table = p.block_table + static_cast<long long>(sg.i) * p.max_pages;
     int cur = load_page(p, c, table, sg.b0 + lane, sg.b1);
-    for (int c0 = sg.b0; c0 < sg.b1; c0 += 32) {  // 32 is a multiple of kGroup
+    for (int c0 = sg.b0; c0 < sg.b1; c0 += 32) {
       const int nxt = load_page(p, c, table, c0 + 32 + lane, sg.b1);
       const int n = min(32, sg.b1 - c0);
       for (int k = 0; k < n; k += kGroup) {
         Group gr;
         gr.blk = c0 + k;
         gr.np = min(kGroup, n - k);
-        gr.page[0] = __shfl_sync(0xffffffffu, cur, k);
-        gr.page[1] = __shfl_sync(0xffffffffu, cur, (k + 1) & 31);
+#pragma unroll
+        for (int q = 0; q < kGroup; ++q) gr.page[q] = __shfl_sync(0xffffffffu, cur, k + q);
         gr.first = gr.blk == sg.b0;
-        gr.last = gr.blk + gr.np == sg.b1;
         if (!fn(sg, gr)) return;
       }
       cur = nxt;
@@ -271,11 +268,12 @@ __device__ __forceinline__ void walk_groups(const DecodeParams& p, const Ctx& c,
 }
 
 // ------------------------------------------------------------- producers --
-// Warp 0: each segment's Q rows of this CTA, then this CTA's key half of
-// every page into the group stages (bytes complete on the leader's barriers).
+// Warp 0: each segment's Q rows of this CTA, then this CTA's key half of the
+// group's pages, panel by panel, into the key ring (bytes complete on the
+// leader's barriers).
 __device__ void producer_k(const DecodeParams& p, const Ctx& c, int s_begin, int s_end) {
   const int lane = threadIdx.x & 31;
-  uint32_t gi = 0, seg_it = 0;  // groups loaded, segments started
+  uint32_t gi = 0, seg_it = 0, ks = 0;  // groups, segments started, key panels loaded
   walk_groups(p, c, s_begin, s_end, [&](const Segment& sg, const Group& gr) -> bool {
     int good = 1;
     if (lane == 0) {
@@ -287,193 +285,135 @@ __device__ void producer_k(const DecodeParams& p, const Ctx& c, int s_begin, int
           tma_load_3d_pair(c.base + kOffQ, &p.tm_q, c.lead_bar(kBarQFull), 0, y, 0);
         }
       }
-      const uint32_t st = gi % kStages;
-      if (good && gi >= kStages) good = wait_bar(c, c.bar(kBarKEmpty + st), ((gi / kStages) - 1) & 1);
-      if (good) {
-        MLA_TRACE(0, gi);
-        const uint32_t bar = c.lead_bar(kBarKFull + st);
-        if (c.cta == 0) mbar_arrive_expect_tx(c.bar(kBarKFull + st), 2 * gr.np * kKBytesPage);
-        for (int q = 0; q < gr.np; ++q) {
-          const int y = gr.page[q] * kPage + static_cast<int>(c.cta) * kHalfPage;
-#pragma unroll
-          for (int pn = 0; pn < 9; ++pn)
-            tma_load_3d_pair(c.stage(st) + pn * kPanel + q * kHalfPageBytes, &p.tm_k, bar, 0, y, pn);
+      if (good) MLA_TRACE(0, gi);
+      for (int pn = 0; pn < 9 && good; ++pn, ++ks) {
+        const uint32_t slot = ks % kKRing;
+        if (ks >= kKRing) good = wait_bar(c, c.bar(kBarKEmpty + slot), ((ks / kKRing) - 1) & 1);
+        if (good) {
+          MLA_TRACE(10, ks);
+          if (c.cta == 0) mbar_arrive_expect_tx(c.bar(kBarKFull + slot), 2 * gr.np * kHalfPageBytes);
+          for (int q = 0; q < gr.np; ++q)
+            tma_load_3d_pair(c.kslot(slot) + q * kHalfPageBytes, &p.tm_k, c.lead_bar(kBarKFull + slot), 0,
+                             gr.page[q] * kPage + static_cast<int>(c.cta) * kHalfPage, pn);
         }
       }
     }
     if (gr.first) ++seg_it;
     ++gi;
-    if (lane == 0) *c.k_prog = gi;
     return __shfl_sync(0xffffffffu, good, 0) != 0;
   });
 }
 
-// Warp 3: L2 prefetch of this CTA's key half of each page (contiguous: 32
-// token rows of 1152 bytes), at most kPrefetchGroups groups ahead of the key
-// loads.
-__device__ void prefetcher(const DecodeParams& p, const Ctx& c, int s_begin, int s_end) {
-  const int lane = threadIdx.x & 31;
-  uint32_t gi = 0;
-  const uint8_t* kv = static_cast<const uint8_t*>(p.kv);
-  walk_groups(p, c, s_begin, s_end, [&](const Segment&, const Group& gr) -> bool {
-    int good = 1;
-    if (lane == 0) {
-      uint64_t t0 = 0;
-      while (gi >= *c.k_prog + kPrefetchGroups) {
-        if (*c.abort_flag) {
-          good = 0;
-          break;
-        }
-        const uint64_t now = globaltimer();
-        if (t0 == 0) {
-          t0 = now;
-        } else if (now - t0 > kTimeoutNs) {
-          raise_abort(c, MLA_DEVERR_TIMEOUT);
-          good = 0;
-          break;
-        }
-        __nanosleep(256);
-      }
-      if (good) {
-        for (int q = 0; q < gr.np; ++q)
-          prefetch_l2_bulk(kv + (static_cast<long long>(gr.page[q]) * kPage + c.cta * kHalfPage) * (kDqk * 2),
-                           kKBytesPage);
-      }
-    }
-    ++gi;
-    return __shfl_sync(0xffffffffu, good, 0) != 0;
-  });
-}
-
-// Warp 2: once QK of a group is done, overwrite the stage's four panels that
-// held the partner's value columns with the partner's tokens of this CTA's
-// value columns (bytes complete on this CTA's own barrier; the softmax warps
-// wait for it before releasing P, so PV never runs ahead of it).
+// Warp 2: this CTA's value tile of every page (all 64 tokens, its 256 value
+// columns) into the value ring once PV two pages back has released the slot;
+// bytes complete on this CTA's own barrier (the softmax warps wait for it
+// before releasing P, so PV never runs ahead of it).
 __device__ void producer_v(const DecodeParams& p, const Ctx& c, int s_begin, int s_end) {
   const int lane = threadIdx.x & 31;
-  uint32_t gi = 0;
-  const uint32_t other = c.cta ^ 1u;
+  uint32_t ps = 0;  // pages
   walk_groups(p, c, s_begin, s_end, [&](const Segment&, const Group& gr) -> bool {
     int good = 1;
     if (lane == 0) {
-      const uint32_t st = gi % kStages;
-      good = wait_bar(c, c.bar(kBarQkDone + st), (gi / kStages) & 1);
-      if (good) {
-        MLA_TRACE(3, gi);
-        const uint32_t bar = c.bar(kBarVxFull + st);
-        mbar_arrive_expect_tx(bar, gr.np * kVxBytesPage);
-        for (int q = 0; q < gr.np; ++q) {
-          const int y = gr.page[q] * kPage + static_cast<int>(other) * kHalfPage;
+      for (int q = 0; q < gr.np && good; ++q, ++ps) {
+        const uint32_t slot = ps % kVRing;
+        if (ps >= kVRing) good = wait_bar(c, c.bar(kBarPvDone + slot), ((ps - kVRing) / kVRing) & 1);
+        if (good) {
+          MLA_TRACE(3, ps);
+          const uint32_t bar = c.bar(kBarVFull + slot);
+          mbar_arrive_expect_tx(bar, kVTile);
 #pragma unroll
-          for (int v = 0; v < 4; ++v) {
-            const int h = v >> 1, e = v & 1;
-            tma_load_3d(c.stage(st) + (4 * h + 2 * other + e) * kPanel + q * kHalfPageBytes, &p.tm_k, bar, 0, y,
-                        4 * h + 2 * c.cta + e);
-          }
+          for (int h = 0; h < 2; ++h)
+            tma_load_3d(c.vtile(slot) + h * 2 * kVPanel, &p.tm_v, bar, 0, gr.page[q] * kPage,
+                        4 * h + 2 * static_cast<int>(c.cta));
         }
       }
     }
-    ++gi;
     return __shfl_sync(0xffffffffu, good, 0) != 0;
   });
 }
 
 // ------------------------------------------------------ MMA (leader only) --
-__device__ __forceinline__ void issue_qk(const Ctx& c, uint32_t tmem, uint32_t st, uint32_t sb) {
-  const uint32_t q = c.base + kOffQ;
-  const uint32_t k = c.stage(st);
+// One key panel of QK^T: four K = 16 steps over its 64 columns.
+__device__ __forceinline__ void issue_qk_panel(const Ctx& c, uint32_t tmem, uint32_t slot, int pn, uint32_t sb) {
+  const uint32_t q = c.base + kOffQ + pn * kQPanel;
+  const uint32_t k = c.kslot(slot);
 #pragma unroll
-  for (int s = 0; s < 36; ++s) {
-    const uint32_t off = (s & 3) * 32;
-    const uint64_t a = smem_desc(q + (s >> 2) * kPanel + off, 16, 1024, kSwizzle128B);
-    const uint64_t b = smem_desc(k + (s >> 2) * kPanel + off, 16, 1024, kSwizzle128B);
-    umma_ss_pair(tmem + kColS + 64 * sb, a, b, kIdescQK, s > 0 ? 1u : 0u);
+  for (int s = 0; s < 4; ++s) {
+    const uint64_t a = smem_desc(q + s * 32, 16, 1024, kSwizzle128B);
+    const uint64_t b = smem_desc(k + s * 32, 16, 1024, kSwizzle128B);
+    umma_ss_pair(tmem + kColS + 128 * sb, a, b, kIdescQK, (pn > 0 || s > 0) ? 1u : 0u);
   }
 }
 
-// O (+)= P V over the group's np pages.  K step k (16 tokens) of the N = 256
-// half h: P chunk k >> 2 (tokens 0-31 or 32-63 of both pages), its 32-byte
-// column block k & 3; V at panel position 4h (+2 for chunk 1), rows 16 (k & 3)
-// (page k >> 1 & 1), this CTA's 128 value columns being two adjacent panels
-// (leading byte offset = one panel).
-__device__ __forceinline__ void issue_pv(const Ctx& c, uint32_t tmem, uint32_t st, int np, bool first) {
-  const uint32_t v = c.stage(st);
-  const uint32_t chunk[2] = {c.base + kOffP0, v + kRopePos * kPanel};
+// O (+)= P V for one page.  For the N = 256 half h, each CTA's 128 value
+// columns are two adjacent panels (leading byte offset = one panel); K step k
+// takes tokens [16k, 16k + 16).
+__device__ __forceinline__ void issue_pv_page(const Ctx& c, uint32_t tmem, uint32_t slot, bool first) {
+  const uint32_t pt = c.ptile(slot);
+  const uint32_t vt = c.vtile(slot);
 #pragma unroll
   for (int h = 0; h < 2; ++h) {
-    bool acc = !first;
 #pragma unroll
-    for (int k = 0; k < 8; ++k) {
-      if (((k >> 1) & 1) >= np) continue;  // the second page is absent
-      const uint64_t a = smem_desc(chunk[k >> 2] + (k & 3) * 32, 16, 1024, kSwizzle128B);
-      const uint32_t pos = 4 * h + ((k >> 2) << 1);
-      const uint64_t b = smem_desc(v + pos * kPanel + (k & 3) * 2048, kPanel, 1024, kSwizzle128B);
-      umma_ss_pair(tmem + kColO + 128 * h, a, b, kIdescPV, acc ? 1u : 0u);
-      acc = true;
+    for (int k = 0; k < 4; ++k) {
+      const uint64_t a = smem_desc(pt + k * 32, 16, 1024, kSwizzle128B);
+      const uint64_t b = smem_desc(vt + h * 2 * kVPanel + k * 16 * 128, kVPanel, 1024, kSwizzle128B);
+      umma_ss_pair(tmem + kColO + 128 * h, a, b, kIdescPV, (!first || k > 0) ? 1u : 0u);
     }
   }
 }
 
-// Per segment the MMAs go out as QK(0), then QK(j+1) and PV(j) for each group
-// j, whichever becomes ready first: QK(j+1) when its keys have landed (and
-// PV(j-1) is out: QK(j+1) overwrites the S buffer of group j-1, which both
-// CTAs had read before signalling P(j-1) ready), PV(j) when both CTAs' P(j)
-// is written.  Letting PV(j) overtake a QK whose keys are late frees stage j
-// for the next loads sooner.
-__device__ void mma_issuer(const DecodeParams& p, const Ctx& c, uint32_t tmem, int s_begin, int s_end) {
-  uint32_t g0 = 0, seg_it = 0;
+// The MMAs go out as two independent streams, each from its own thread of the
+// leader CTA, so that one waiting (or blocked on a full tensor-core queue)
+// never holds the other back.  The two share no TMEM: QK writes the S
+// buffers, PV accumulates O.
+//   * QK (warp 1): per group, one panel at a time as the key panels land; a
+//     group may start once both CTAs have read the S buffer it overwrites.
+//   * PV (warp 3): per page, in order, once both CTAs have written its P
+//     (which they do after reading S, so QK of its group is complete); the
+//     first page of a segment also waits until O has been read out.
+__device__ void qk_issuer(const DecodeParams& p, const Ctx& c, uint32_t tmem, int s_begin, int s_end) {
+  uint32_t gi = 0, ks = 0, seg_it = 0;  // groups, key panels consumed, segments
+  const uint16_t both = 0x3;
+  for (int s = s_begin; s < s_end; ++s) {
+    const Segment sg = load_segment(p, s);
+    if (sg.bad) continue;
+    const int ng = ceil_div(sg.b1 - sg.b0, kGroup);
+    if (!wait_bar(c, c.bar(kBarQFull), seg_it & 1)) return;
+    for (int gq = 0; gq < ng; ++gq, ++gi) {
+      const uint32_t sb = gi & 1;
+      if (gi >= 2 && !wait_bar(c, c.bar(kBarSEmpty + sb), ((gi - 2) >> 1) & 1)) return;
+      MLA_TRACE(1, gi);
+      for (int pn = 0; pn < 9; ++pn, ++ks) {
+        const uint32_t slot = ks % kKRing;
+        if (!wait_bar(c, c.bar(kBarKFull + slot), (ks / kKRing) & 1)) return;
+        MLA_TRACE(9, ks);
+        tc_fence_after();
+        issue_qk_panel(c, tmem, slot, pn, sb);
+        umma_commit_pair(c.bar(kBarKEmpty + slot), both);
+      }
+      umma_commit_pair(c.bar(kBarSFull + sb), both);
+    }
+    umma_commit_pair(c.bar(kBarQEmpty), both);  // Q free once the segment's last QK is done
+    ++seg_it;
+  }
+}
+
+__device__ void pv_issuer(const DecodeParams& p, const Ctx& c, uint32_t tmem, int s_begin, int s_end) {
+  uint32_t pg = 0, seg_it = 0;  // pages, segments
   const uint16_t both = 0x3;
   for (int s = s_begin; s < s_end; ++s) {
     const Segment sg = load_segment(p, s);
     if (sg.bad) continue;
     const int n = sg.b1 - sg.b0;
-    const int ng = ceil_div(n, kGroup);
-    if (!wait_bar(c, c.bar(kBarQFull), seg_it & 1)) return;
-    int jq = 0, jp = 0;  // next QK, next PV (groups of this segment)
-    uint64_t t0 = 0;
-    while (jp < ng) {
-      bool did = false;
-      if (jq < ng && jq <= jp + 1) {
-        const uint32_t g = g0 + jq, st = g % kStages, sb = g & 1;
-        if (mbar_test_wait(c.bar(kBarKFull + st), (g / kStages) & 1)) {
-          MLA_TRACE(1, g);
-          tc_fence_after();
-          issue_qk(c, tmem, st, sb);
-          umma_commit_pair(c.bar(kBarSFull + sb), both);
-          umma_commit_pair(c.bar(kBarQkDone + st), both);
-          if (jq == ng - 1) umma_commit_pair(c.bar(kBarQEmpty), both);  // Q free once the last QK is done
-          ++jq;
-          did = true;
-        }
-      }
-      if (!did && jp < jq) {
-        const uint32_t g = g0 + jp, st = g % kStages, pb = g & 1;
-        if (mbar_test_wait(c.bar(kBarPFull + pb), (g >> 1) & 1) &&
-            (jp > 0 || seg_it == 0 || mbar_test_wait(c.bar(kBarOEmpty), (seg_it - 1) & 1))) {
-          MLA_TRACE(2, g);
-          tc_fence_after();
-          issue_pv(c, tmem, st, min(kGroup, n - kGroup * jp), jp == 0);
-          umma_commit_pair(c.bar(kBarKEmpty + st), both);
-          umma_commit_pair(c.bar(kBarPvDone + pb), both);
-          ++jp;
-          did = true;
-        }
-      }
-      if (did) {
-        t0 = 0;
-        continue;
-      }
-      if (*c.abort_flag) return;
-      const uint64_t now = globaltimer();
-      if (t0 == 0) {
-        t0 = now;
-      } else if (now - t0 > kTimeoutNs) {
-        raise_abort(c, MLA_DEVERR_TIMEOUT);
-        return;
-      }
-      __nanosleep(32);
+    for (int jp = 0; jp < n; ++jp, ++pg) {
+      const uint32_t slot = pg % kVRing;
+      if (!wait_bar(c, c.bar(kBarPFull + slot), (pg / kVRing) & 1)) return;
+      if (jp == 0 && seg_it > 0 && !wait_bar(c, c.bar(kBarOEmpty), (seg_it - 1) & 1)) return;
+      MLA_TRACE(2, pg);
+      tc_fence_after();
+      issue_pv_page(c, tmem, slot, jp == 0);
+      umma_commit_pair(c.bar(kBarPvDone + slot), both);
     }
-    g0 += ng;
     ++seg_it;
   }
 }
@@ -498,7 +438,7 @@ __device__ __forceinline__ float masked_max(float (&sv)[32], int nvalid) {
 // p = 2^(s * sl2 - m) for the first nvalid scores, 0 past them; packs the
 // bf16-rounded weights in pairs and returns their unrounded fp32 sum.
 __device__ __forceinline__ float exp_pack(const float (&sv)[32], int nvalid, float sl2, float neg_m,
-                                          uint32_t* packed) {
+                                          uint32_t (&packed)[16]) {
   float e[16];
 #pragma unroll
   for (int k = 0; k < 16; ++k) {
@@ -529,13 +469,14 @@ __device__ void softmax_epilogue(const DecodeParams& p, const Ctx& c, uint32_t t
   const uint32_t t_o = tmem + lane_off + kColO;
   const uint32_t xbar = c.bar(kBarXch + ((r >> 5) & 1));  // warps 4+6 and 5+7 hold the two halves of rows
   float* xbuf = reinterpret_cast<float*>(c.gbase + kOffX);
-  // This thread's row of P: 128 bytes, 16-byte chunks swizzled by the row.
+  // This thread's 32 weights of a page: 64 bytes of P row hr, 16-byte chunks
+  // 4 half .. 4 half + 3, swizzled by the row.
   const uint32_t prow_off = (hr >> 3) * 1024 + (hr & 7) * 128;
   const float sl2 = p.scale_log2;
-  // gi: groups consumed so far (selects S and stage buffers and phases);
+  // gi: groups, ps: pages consumed so far (select buffers and phases);
   // x_cnt: row exchanges with the partner thread.
-  uint32_t gi = 0, x_cnt = 0;
-  auto pv_done = [&](uint32_t k) -> bool { return wait_bar(c, c.bar(kBarPvDone + (k & 1)), (k >> 1) & 1); };
+  uint32_t gi = 0, ps = 0, x_cnt = 0;
+  auto pv_done = [&](uint32_t k) -> bool { return wait_bar(c, c.bar(kBarPvDone + k % kVRing), (k / kVRing) & 1); };
   // Publish v for the partner thread (same row, other half) and return its
   // value; the two warps meet on an mbarrier (bounded wait).
   auto trade = [&](float v, float* out) -> bool {
@@ -572,22 +513,28 @@ __device__ void softmax_epilogue(const DecodeParams& p, const Ctx& c, uint32_t t
     for (int j = 0; j < n; j += kGroup, ++gi) {
       const int blk = sg.b0 + j;
       const int np = min(kGroup, n - j);
-      const uint32_t sb = gi & 1, st = gi % kStages;
+      const uint32_t sb = gi & 1;
       if (!wait_bar(c, c.bar(kBarSFull + sb), (gi >> 1) & 1)) return;
       if (r == 0) MLA_TRACE(4, gi);
       tc_fence_after();
-      float sv0[32], sv1[32];
-      tmem_ld32(t_s + 64 * sb, sv0);
-      tmem_ld32(t_s + 64 * sb + 32, sv1);
+      float sv[kGroup][32];
+#pragma unroll
+      for (int q = 0; q < kGroup; ++q) tmem_ld32(t_s + 128 * sb + 32 * q, sv[q]);
       tmem_wait_ld();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) arrive_leader(c, kBarSEmpty + sb);  // S buffer read
 
-      // ---- mask; max over both pages and both halves of the row ----
-      int nv0 = limit - blk * kPage - kHalfPage * half;
-      nv0 = nv0 < 0 ? 0 : (nv0 > 32 ? 32 : nv0);
-      int nv1 = limit - (blk + 1) * kPage - kHalfPage * half;
-      nv1 = (np < 2 || nv1 < 0) ? 0 : (nv1 > 32 ? 32 : nv1);
-      float mx = fmaxf(masked_max(sv0, nv0), masked_max(sv1, nv1));
-      mx = (nv0 + nv1 > 0) ? mx * sl2 : -INFINITY;  // softmax_scale >= 0
+      // ---- mask; max over the group's pages and both halves of the row ----
+      int nv[kGroup];
+      float mx = -INFINITY;
+#pragma unroll
+      for (int q = 0; q < kGroup; ++q) {
+        int v = limit - (blk + q) * kPage - kHalfPage * half;
+        nv[q] = (q >= np || v < 0) ? 0 : (v > 32 ? 32 : v);
+        mx = fmaxf(mx, masked_max(sv[q], nv[q]));
+      }
+      mx = (nv[0] > 0) ? mx * sl2 : -INFINITY;  // tokens are valid from the left; softmax_scale >= 0
       float mx_peer;
       if (!trade(mx, &mx_peer)) return;
       if (r == 0) MLA_TRACE(5, gi);
@@ -596,17 +543,10 @@ __device__ void softmax_epilogue(const DecodeParams& p, const Ctx& c, uint32_t t
       if (mx > m + kTau) m_new = mx;  // also true for the first finite block
       const float alpha = (m_new == m) ? 1.0f : ex2(m - m_new);  // 0 when m was -inf
       const float neg_m = (m_new == -INFINITY) ? 0.0f : -m_new;
-      uint32_t packed[32];
-      const float e = exp_pack(sv0, nv0, sl2, neg_m, packed) + exp_pack(sv1, nv1, sl2, neg_m, packed + 16);
-      l = l * alpha + e;
-      m = m_new;
 
-      // ---- the previous group's PV is done: the P buffer of tokens 0-31 is
-      //      free and O is up to date for a rescale ----
-      if (r == 0) MLA_TRACE(6, gi);
-      const bool rescale = j > 0 && __any_sync(0xffffffffu, alpha < 1.0f);
-      if (gi >= 1 && (half == 0 || rescale) && !pv_done(gi - 1)) return;
-      if (rescale) {
+      // ---- rescale O (rare): after PV of every earlier page of the segment ----
+      if (j > 0 && __any_sync(0xffffffffu, alpha < 1.0f)) {
+        if (!pv_done(ps - 1)) return;
         tc_fence_after();
 #pragma unroll 1
         for (int cc = 0; cc < 256; cc += 32) {
@@ -619,42 +559,52 @@ __device__ void softmax_epilogue(const DecodeParams& p, const Ctx& c, uint32_t t
         }
         tmem_wait_st();
       }
-      // ---- P row hr: tokens [32 half, 32 half + 32) of both pages ----
-      if (r == 0) MLA_TRACE(7, gi);
-      {
-        uint8_t* prow = (half == 0 ? c.gbase + kOffP0 : c.gbase + kOffStage + st * kStageBytes + kRopePos * kPanel) +
-                        prow_off;
+
+      float lsum = 0.0f;
 #pragma unroll
-        for (int ci = 0; ci < 8; ++ci)
-          *reinterpret_cast<uint4*>(prow + ((ci ^ (hr & 7)) << 4)) =
-              make_uint4(packed[4 * ci], packed[4 * ci + 1], packed[4 * ci + 2], packed[4 * ci + 3]);
-      }
-      // ---- the partner's value panels have landed; the last page of a row
-      //      may hold garbage (even NaN) past L: zero the value rows there
-      //      that PV reads, so that 0 * garbage cannot reach O ----
-      if (!wait_bar(c, c.bar(kBarVxFull + st), (gi / kStages) & 1)) return;
-      if (r == 0) MLA_TRACE(8, gi);
-      if ((sg.L & (kPage - 1)) && last_page >= blk && last_page < blk + np) {
-        const int q = last_page - blk;
-        const int first_bad = sg.L - last_page * kPage;
-        const int chunks = (kPage - first_bad) * 4 * 8;  // tokens x panels x 16-byte chunks
-        uint8_t* stg = c.gbase + kOffStage + st * kStageBytes + q * kHalfPageBytes;
-        for (int e2 = r; e2 < chunks; e2 += 128) {
-          const int tok = first_bad + (e2 >> 5);
-          const int v = (e2 >> 3) & 3;
-          const int pos = (v & 1) + 4 * (v >> 1) + (tok >= kHalfPage ? 2 : 0);
-          *reinterpret_cast<uint4*>(stg + pos * kPanel + (tok & 31) * 128 + (e2 & 7) * 16) = make_uint4(0, 0, 0, 0);
+      for (int q = 0; q < kGroup; ++q) {
+        if (q >= np) break;
+        uint32_t packed[16];
+        lsum += exp_pack(sv[q], nv[q], sl2, neg_m, packed);
+        const uint32_t slot = ps % kVRing;
+        // ---- P tile free (PV two pages back) ----
+        if (ps >= kVRing && !pv_done(ps - kVRing)) return;
+        if (r == 0) MLA_TRACE(6, ps);
+        {
+          uint8_t* prow = c.gbase + kOffP + slot * kPTile + prow_off;
+#pragma unroll
+          for (int ci = 0; ci < 4; ++ci)
+            *reinterpret_cast<uint4*>(prow + (((4 * half + ci) ^ (hr & 7)) << 4)) =
+                make_uint4(packed[4 * ci], packed[4 * ci + 1], packed[4 * ci + 2], packed[4 * ci + 3]);
         }
+        // ---- this CTA's value tile has landed; the last page of a row may
+        //      hold garbage (even NaN) past L: zero the value rows there, so
+        //      that 0 * garbage cannot reach O ----
+        if (!wait_bar(c, c.bar(kBarVFull + slot), (ps / kVRing) & 1)) return;
+        if (r == 0) MLA_TRACE(7, ps);
+        if (blk + q == last_page && (sg.L & (kPage - 1))) {
+          const int first_bad = sg.L - last_page * kPage;
+          const int chunks = (kPage - first_bad) * 4 * 8;  // tokens x panels x 16-byte chunks
+          uint8_t* vt = c.gbase + kOffV + slot * kVTile;
+          for (int e2 = r; e2 < chunks; e2 += 128) {
+            const int tok = first_bad + (e2 >> 5);
+            *reinterpret_cast<uint4*>(vt + ((e2 >> 3) & 3) * kVPanel + tok * 128 + (e2 & 7) * 16) =
+                make_uint4(0, 0, 0, 0);
+          }
+        }
+        fence_proxy_async_smem();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) arrive_leader(c, kBarPFull + slot);
+        if (r == 0) MLA_TRACE(8, ps);
+        ++ps;
       }
-      fence_proxy_async_smem();
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) arrive_leader(c, kBarPFull + sb);
-      if (r == 0) MLA_TRACE(9, gi);
+      l = l * alpha + lsum;
+      m = m_new;
     }
 
     // ---- epilogue ----
-    if (!pv_done(gi - 1)) return;
+    if (!pv_done(ps - 1)) return;
     tc_fence_after();
     float l_peer;
     if (!trade(l, &l_peer)) return;
@@ -722,31 +672,31 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
   c.cta = cluster_ctarank();
   c.meta = p.meta;
   c.abort_flag = reinterpret_cast<volatile uint32_t*>(c.gbase + kOffAbort);
-  c.k_prog = reinterpret_cast<volatile uint32_t*>(c.gbase + kOffKProg);
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
 
   if (threadIdx.x == 0) {
     // Barriers of the leader's pipeline are only used in the leader, the
     // rest in both CTAs; initialise all of them everywhere.
-    for (int k = 0; k < kStages; ++k) {
+    for (int k = 0; k < kKRing; ++k) {
       mbar_init(c.bar(kBarKFull + k), 1);
       mbar_init(c.bar(kBarKEmpty + k), 1);
-      mbar_init(c.bar(kBarQkDone + k), 1);
-      mbar_init(c.bar(kBarVxFull + k), 1);
+    }
+    for (int k = 0; k < kVRing; ++k) {
+      mbar_init(c.bar(kBarVFull + k), 1);
+      mbar_init(c.bar(kBarPFull + k), 8);
+      mbar_init(c.bar(kBarPvDone + k), 1);
     }
     for (int k = 0; k < 2; ++k) {
       mbar_init(c.bar(kBarSFull + k), 1);
-      mbar_init(c.bar(kBarPFull + k), 8);
-      mbar_init(c.bar(kBarPvDone + k), 1);
+      mbar_init(c.bar(kBarSEmpty + k), 8);
       mbar_init(c.bar(kBarXch + k), 2);
     }
     mbar_init(c.bar(kBarQFull), 1);
     mbar_init(c.bar(kBarQEmpty), 1);
     mbar_init(c.bar(kBarOEmpty), 8);
-    mbar_init(c.bar(kBarFinal), 1);
+    mbar_init(c.bar(kBarFinal), 2);
     *c.abort_flag = 0u;
-    *c.k_prog = 0u;
     fence_mbar_init_cluster();
   }
   if (warp == 1) {
@@ -755,6 +705,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
   }
   if (warp == 0 && lane == 0) {
     tma_prefetch_desc(&p.tm_k);
+    tma_prefetch_desc(&p.tm_v);
     tma_prefetch_desc(&p.tm_q);
   }
   tc_fence_before();
@@ -782,21 +733,23 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
   if (warp == 0) {
     producer_k(p, c, s_begin, s_end);
   } else if (warp == 1) {
-    if (lane == 0 && c.cta == 0) mma_issuer(p, c, tmem, s_begin, s_end);
+    if (lane == 0 && c.cta == 0) qk_issuer(p, c, tmem, s_begin, s_end);
     __syncwarp();
   } else if (warp == 2) {
     producer_v(p, c, s_begin, s_end);
   } else if (warp == 3) {
-    prefetcher(p, c, s_begin, s_end);
+    if (lane == 0 && c.cta == 0) pv_issuer(p, c, tmem, s_begin, s_end);
+    __syncwarp();
   } else {
     softmax_epilogue(p, c, tmem, s_begin, s_end);
   }
 
   // ---- teardown: drain the pair MMAs, wait for the peer, free TMEM ----
   __syncthreads();
+  if (warp == 3 && c.cta == 0 && lane == 0) umma_commit_pair(c.bar(kBarFinal), 0x1);  // PV issuer's MMAs
   if (warp == 1 && c.cta == 0) {
     if (lane == 0) {
-      umma_commit_pair(c.bar(kBarFinal), 0x1);
+      umma_commit_pair(c.bar(kBarFinal), 0x1);  // QK issuer's MMAs
       const uint64_t t0 = globaltimer();
       while (!mbar_try_wait(c.bar(kBarFinal), 0) && globaltimer() - t0 < kTimeoutNs) {
       }

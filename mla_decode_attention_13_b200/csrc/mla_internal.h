@@ -93,10 +93,11 @@ __host__ __device__ inline size_t workspace_bytes_for(int pairs, int h_q, int s_
 // Split-KV decode kernel parameters.
 // ---------------------------------------------------------------------------
 struct DecodeParams {
-  // Both view a [rows][576] bf16 tensor as (64 cols, rows, 9 panels),
+  // All three view a [rows][576] bf16 tensor as (64 cols, rows, 9 panels),
   // strides (1152 B, 128 B), so that a 3-D box lands as panels of 64
   // columns x box rows, 128B-swizzled.
-  CUtensorMap tm_k;  // cache: box (64, 32, 1), one panel of 32 tokens
+  CUtensorMap tm_k;  // cache: box (64, 32, 1), one panel of a page's 32 key tokens
+  CUtensorMap tm_v;  // cache: box (64, 64, 2), two value panels of a page's 64 tokens
   CUtensorMap tm_q;  // q: box (64, 64, 9), 64 query rows
   const void* kv;          // cache base (bf16 [num_pages*64][576]), for L2 prefetch
   const int32_t* block_table;
