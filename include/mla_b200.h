@@ -65,6 +65,7 @@ extern "C" {
 #define MLA_ERR_CUDA (-3)        /* a CUDA runtime or driver call failed   */
 #define MLA_ERR_WORKSPACE (-4)   /* workspace smaller than required        */
 #define MLA_ERR_DEVICE (-5)      /* the device error word is non-zero      */
+#define MLA_ERR_SCRATCH (-6)     /* needs more than the fixed scratch holds */
 
 /* Bits of the device error word (see mla_check_device_error). */
 #define MLA_DEVERR_SEQLEN 0x1u   /* L_i < 0 or L_i > 64 * max_pages_per_seq */
@@ -150,6 +151,48 @@ int mla_decode_timed(const void* q, const void* kv_cache, int64_t num_pages, con
                      int max_pages_per_seq, const int32_t* seqlens, int batch, int s_q, int h_q,
                      float softmax_scale, int causal, void* out, float* lse, void* metadata, void* workspace,
                      size_t workspace_bytes, void* stream, void* event_before_decode, void* event_after_decode);
+
+/*
+ * Size in bytes of the library's fixed, statically allocated scratch buffer
+ * used by mla_decode_noalloc: 40 MiB.
+ */
+#define MLA_NOALLOC_SCRATCH_BYTES (40u * 1024u * 1024u)
+
+/*
+ * mla_decode without a caller-supplied workspace, for callers that cannot
+ * allocate device memory at the point of the call: code running inside a
+ * framework that owns the device allocator, a fixed-footprint inference
+ * engine that sizes all its memory before it starts serving, or a capture or
+ * replay of a graph whose memory plan is frozen.  None of these can call
+ * cudaMalloc (nor ask torch for a tensor) in the decode loop, but all of them
+ * can pass the inputs, outputs and metadata they already own.  (The pages
+ * this library follows have no counterpart to this call; it only changes
+ * where the scratch lives.)
+ *
+ * Arguments and results are those of mla_decode, without workspace and
+ * workspace_bytes.  The scratch that mla_decode takes from the caller (the
+ * fp32 partial outputs of rows the plan splits) lives instead in one
+ * statically allocated device array of MLA_NOALLOC_SCRATCH_BYTES, which every
+ * GPU that loads the library holds until the process exits.
+ *
+ *   - Returns MLA_ERR_SCRATCH, before enqueueing anything, when this shape
+ *     could need more scratch than that (mla_workspace_bytes(batch, h_q, s_q)
+ *     > MLA_NOALLOC_SCRATCH_BYTES); then use mla_decode with a workspace.
+ *     On B200 every supported shape fits.
+ *   - The first call on each device looks up the array's device address (no
+ *     allocation); make that first call before any stream capture.
+ *   - Nothing in the array needs to start at zero: the decode kernel writes
+ *     every partial it assigns before the combine kernel reads it, so the
+ *     contents left by an earlier call are never used.
+ *   - All calls on a device share the one array: calls whose kernels overlap
+ *     on the GPU (different streams, or different host threads, without an
+ *     ordering between them) race on it and give wrong results.  Order them
+ *     on one stream, or use mla_decode with separate workspaces.
+ *   - Calls no cudaMalloc, cudaFree or other allocating routine.
+ */
+int mla_decode_noalloc(const void* q, const void* kv_cache, int64_t num_pages, const int32_t* block_table,
+                       int max_pages_per_seq, const int32_t* seqlens, int batch, int s_q, int h_q,
+                       float softmax_scale, int causal, void* out, float* lse, void* metadata, void* stream);
 
 /*
  * Synchronise `stream` and read the device error word from `metadata`.

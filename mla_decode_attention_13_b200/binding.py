@@ -22,6 +22,7 @@ MLA_ERR_UNSUPPORTED = -2
 MLA_ERR_CUDA = -3
 MLA_ERR_WORKSPACE = -4
 MLA_ERR_DEVICE = -5
+MLA_ERR_SCRATCH = -6
 
 MLA_DEVERR_SEQLEN = 0x1
 MLA_DEVERR_PAGE = 0x2
@@ -35,6 +36,7 @@ EXPORTED = (
     "mla_get_metadata",
     "mla_decode",
     "mla_decode_timed",
+    "mla_decode_noalloc",
     "mla_check_device_error",
     "mla_error_string",
 )
@@ -71,6 +73,8 @@ def lib() -> ctypes.CDLL:
         L.mla_decode.argtypes = dec
         L.mla_decode_timed.restype = ctypes.c_int
         L.mla_decode_timed.argtypes = dec + [_vp, _vp]
+        L.mla_decode_noalloc.restype = ctypes.c_int
+        L.mla_decode_noalloc.argtypes = dec[:14] + [_vp]
         L.mla_check_device_error.restype = ctypes.c_int
         L.mla_check_device_error.argtypes = [_vp, _vp, ctypes.POINTER(ctypes.c_uint32)]
         L.mla_error_string.restype = ctypes.c_char_p
@@ -161,6 +165,33 @@ def mla_decode(q: torch.Tensor, kv_cache: torch.Tensor, block_table: torch.Tenso
             ev.append(None if e is None else int(e.cuda_event))
         status = lib().mla_decode_timed(*args, *ev)
     _check("mla_decode", status)
+    return out, lse
+
+
+def mla_decode_noalloc(q: torch.Tensor, kv_cache: torch.Tensor, block_table: torch.Tensor, seqlens: torch.Tensor,
+                       softmax_scale: float, causal: bool, metadata: torch.Tensor, out: torch.Tensor,
+                       lse: torch.Tensor, stream=None) -> Tuple[torch.Tensor, torch.Tensor]:
+    """MLA decode with the library's fixed scratch instead of a workspace.
+
+    For callers that cannot allocate device memory in the decode loop: every
+    buffer (q, cache, table, lengths, metadata, out, lse) is passed in, and
+    nothing is allocated here or in the library.  Calls that overlap on the GPU
+    share the one scratch array and race.
+    """
+    batch, s_q, h_q, d = q.shape
+    if d != 576 or kv_cache.shape[-1] != 576 or q.dtype != torch.bfloat16 or kv_cache.dtype != torch.bfloat16:
+        raise MLAError("mla_decode_noalloc", MLA_ERR_ARG)
+    for t in (q, kv_cache, block_table, seqlens, out, lse):
+        if not t.is_contiguous():
+            raise MLAError("mla_decode_noalloc", MLA_ERR_ARG)
+    if tuple(out.shape) != (batch, s_q, h_q, 512) or out.dtype != torch.bfloat16:
+        raise MLAError("mla_decode_noalloc", MLA_ERR_ARG)
+    if tuple(lse.shape) != (batch, h_q, s_q) or lse.dtype != torch.float32:
+        raise MLAError("mla_decode_noalloc", MLA_ERR_ARG)
+    _check("mla_decode_noalloc",
+           lib().mla_decode_noalloc(_ptr(q), _ptr(kv_cache), int(kv_cache.shape[0]), _ptr(block_table),
+                                    int(block_table.shape[1]), _ptr(seqlens), batch, s_q, h_q, float(softmax_scale),
+                                    int(bool(causal)), _ptr(out), _ptr(lse), _ptr(metadata), _stream_ptr(stream)))
     return out, lse
 
 

@@ -80,6 +80,36 @@ int encode_panels576(PFN_cuTensorMapEncodeTiled_v12000 enc, CUtensorMap* map, co
   return r == CUDA_SUCCESS ? MLA_OK : MLA_ERR_CUDA;
 }
 
+// Scratch of mla_decode_noalloc: one fixed device array per GPU that loads
+// the library (held until the process exits), shared by every call on that
+// device.  In host code the name stands for a host-side shadow, not a device
+// address, so the address is looked up per device with cudaGetSymbolAddress.
+static_assert(MLA_NOALLOC_SCRATCH_BYTES % 16 == 0, "scratch size");
+static __device__ __align__(256) unsigned char g_noalloc_scratch[MLA_NOALLOC_SCRATCH_BYTES];
+void* g_noalloc_ptr[kMaxDevices] = {};
+
+// Device address of g_noalloc_scratch on the current device (looked up on the
+// first call there; no allocation).
+int noalloc_scratch(void** out) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) {
+    cudaGetLastError();
+    return MLA_ERR_CUDA;
+  }
+  if (dev < 0 || dev >= kMaxDevices) return MLA_ERR_UNSUPPORTED;
+  std::lock_guard<std::mutex> lock(g_mu);
+  if (!g_noalloc_ptr[dev]) {
+    void* ptr = nullptr;
+    if (cudaGetSymbolAddress(&ptr, g_noalloc_scratch) != cudaSuccess || ptr == nullptr) {
+      cudaGetLastError();
+      return MLA_ERR_CUDA;
+    }
+    g_noalloc_ptr[dev] = ptr;
+  }
+  *out = g_noalloc_ptr[dev];
+  return MLA_OK;
+}
+
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
 bool shape_ok(int batch, int h_q, int s_q) {
@@ -225,6 +255,20 @@ MLA_API int mla_decode_timed(const void* q, const void* kv_cache, int64_t num_pa
                      event_after_decode);
 }
 
+MLA_API int mla_decode_noalloc(const void* q, const void* kv_cache, int64_t num_pages, const int32_t* block_table,
+                               int max_pages_per_seq, const int32_t* seqlens, int batch, int s_q, int h_q,
+                               float softmax_scale, int causal, void* out, float* lse, void* metadata, void* stream) {
+  if (!shape_ok(batch, h_q, s_q)) return batch < 1 || h_q < 1 || s_q < 1 ? MLA_ERR_ARG : MLA_ERR_UNSUPPORTED;
+  DeviceInfo dev;
+  int st = current_device_info(&dev);
+  if (st != MLA_OK) return st;
+  if (workspace_bytes_for(dev.pairs, h_q, s_q) > MLA_NOALLOC_SCRATCH_BYTES) return MLA_ERR_SCRATCH;
+  void* scratch = nullptr;
+  if ((st = noalloc_scratch(&scratch)) != MLA_OK) return st;
+  return decode_impl(q, kv_cache, num_pages, block_table, max_pages_per_seq, seqlens, batch, s_q, h_q, softmax_scale,
+                     causal, out, lse, metadata, scratch, MLA_NOALLOC_SCRATCH_BYTES, stream, nullptr, nullptr);
+}
+
 MLA_API int mla_check_device_error(const void* metadata, void* stream, uint32_t* error_word) {
   if (!metadata) return MLA_ERR_ARG;
   uint32_t word = 0;
@@ -253,6 +297,8 @@ MLA_API const char* mla_error_string(int status) {
       return "workspace smaller than mla_workspace_bytes()";
     case MLA_ERR_DEVICE:
       return "device error word set (see MLA_DEVERR_* bits)";
+    case MLA_ERR_SCRATCH:
+      return "shape needs more scratch than the fixed no-allocation buffer holds (use mla_decode with a workspace)";
     default:
       return "unknown status";
   }

@@ -47,7 +47,7 @@ def test_library_has_no_driver_link_dependency(lib):
 
 
 def test_error_strings(lib):
-    for code in (0, -1, -2, -3, -4, -5, 7):
+    for code in (0, -1, -2, -3, -4, -5, -6, 7):
         assert isinstance(binding.mla_error_string(code), str) and binding.mla_error_string(code)
 
 
