@@ -10,18 +10,26 @@
 //
 // Grid-stride over items (work row, group of 8 query rows); one warp per query
 // row, each lane owning 16 of the 512 output columns as 4 float4 strips, so a
-// warp reads and writes whole contiguous rows.  Memory-light, CUDA cores.
+// warp reads and writes whole contiguous rows.  Lane q reads piece q's lse
+// once; the pieces' rows are then fetched kBatch at a time with all their
+// loads in flight together, because the kernel is bound by memory latency,
+// not bandwidth.  Launched as the decode kernel's programmatic dependent: it
+// waits for the decode kernel's completion before reading the partials.
 #include <cuda_bf16.h>
 
 #include "mla_internal.h"
+#include "sm100_ptx.cuh"
 
 namespace mla {
 namespace {
 
 constexpr int kCombineThreads = 256;
 constexpr int kRowsPerItem = kCombineThreads / 32;
+constexpr int kBatch = 4;  // pieces whose rows are in flight at once
 
 __global__ void __launch_bounds__(kCombineThreads) mla_combine_kernel(const CombineParams p) {
+  ptx::griddep_launch_dependents();
+  ptx::griddep_wait();  // the decode kernel's partials and the plan are complete
   const int32_t* meta = p.meta;
   const MetaLayout lo = meta_layout(p.batch, p.h_q, p.s_q);
   // Only a plan built for this call's shape on this many pairs is used.
@@ -60,30 +68,53 @@ __global__ void __launch_bounds__(kCombineThreads) mla_combine_kernel(const Comb
     if (!empty) {
       const int base = meta[lo.row_info + 2 * w + 0];
       const int pieces = meta[lo.row_info + 2 * w + 1];
-      if (base < 0 || pieces < 2 || base + pieces > p.max_slots) continue;
+      if (base < 0 || pieces < 2 || pieces > 32 * 8 || base + pieces > p.max_slots) continue;
+      // lse of piece lane + 32 k, held by that lane.
+      float lv[8];
       float mx = -INFINITY;
-      for (int q = lane; q < pieces; q += 32) {
-        mx = fmaxf(mx, p.lse_part[static_cast<long long>(base + q) * p.tile_rows + r]);
+#pragma unroll
+      for (int k = 0; k < 8; ++k) {
+        const int q = lane + 32 * k;
+        lv[k] = q < pieces ? p.lse_part[static_cast<long long>(base + q) * p.tile_rows + r] : -INFINITY;
+        mx = fmaxf(mx, lv[k]);
       }
       for (int off = 16; off > 0; off >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, off));
       if (mx != -INFINITY) {
         float sum = 0.0f;
-        for (int q = lane; q < pieces; q += 32) {
-          sum += __expf(p.lse_part[static_cast<long long>(base + q) * p.tile_rows + r] - mx);
-        }
+#pragma unroll
+        for (int k = 0; k < 8; ++k) sum += __expf(lv[k] - mx);  // exp(-inf) = 0 for absent pieces
         for (int off = 16; off > 0; off >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, off);
         lse = mx + __logf(sum);
-        for (int q = 0; q < pieces; ++q) {
-          const long long slot_row = static_cast<long long>(base + q) * p.tile_rows + r;
-          const float wgt = __expf(p.lse_part[slot_row] - lse);
-          const float4* src = reinterpret_cast<const float4*>(p.o_part + slot_row * kDv);
+        float wl[8];  // weight of piece lane + 32 k
 #pragma unroll
-          for (int c = 0; c < 4; ++c) {
-            const float4 v = src[c * 32 + lane];
-            acc[4 * c + 0] += wgt * v.x;
-            acc[4 * c + 1] += wgt * v.y;
-            acc[4 * c + 2] += wgt * v.z;
-            acc[4 * c + 3] += wgt * v.w;
+        for (int k = 0; k < 8; ++k) wl[k] = __expf(lv[k] - lse);
+        for (int q0 = 0; q0 < pieces; q0 += kBatch) {
+          float4 v[kBatch][4];
+#pragma unroll
+          for (int b = 0; b < kBatch; ++b) {
+            const int q = q0 + b < pieces ? q0 + b : pieces - 1;  // clamp; weight 0 below
+            const float4* src =
+                reinterpret_cast<const float4*>(p.o_part + (static_cast<long long>(base + q) * p.tile_rows + r) * kDv);
+#pragma unroll
+            for (int c = 0; c < 4; ++c) v[b][c] = src[c * 32 + lane];
+          }
+#pragma unroll
+          for (int b = 0; b < kBatch; ++b) {
+            const int q = q0 + b;
+            float wgt = 0.0f;
+#pragma unroll
+            for (int k = 0; k < 8; ++k) {
+              const float wk = __shfl_sync(0xffffffffu, wl[k], q & 31);
+              if ((q >> 5) == k) wgt = wk;
+            }
+            if (q >= pieces) wgt = 0.0f;
+#pragma unroll
+            for (int c = 0; c < 4; ++c) {
+              acc[4 * c + 0] += wgt * v[b][c].x;
+              acc[4 * c + 1] += wgt * v[b][c].y;
+              acc[4 * c + 2] += wgt * v[b][c].z;
+              acc[4 * c + 3] += wgt * v[b][c].w;
+            }
           }
         }
       }
@@ -104,8 +135,16 @@ __global__ void __launch_bounds__(kCombineThreads) mla_combine_kernel(const Comb
 }  // namespace
 
 cudaError_t launch_combine(const CombineParams& p, int grid, cudaStream_t stream) {
-  mla_combine_kernel<<<grid, kCombineThreads, 0, stream>>>(p);
-  return cudaGetLastError();
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(static_cast<unsigned>(grid), 1, 1);
+  cfg.blockDim = dim3(kCombineThreads, 1, 1);
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, mla_combine_kernel, p);
 }
 
 }  // namespace mla

@@ -68,6 +68,7 @@ namespace mla {
 // (compile with -DMLA_DECODE_TRACE; the default build records nothing).
 #ifdef MLA_DECODE_TRACE
 __device__ unsigned long long g_mla_trace[4][16][512];  // [traced CTA][event][index]
+__device__ unsigned long long g_mla_span[160][4];  // [pair][start, end, segments, pages] (globaltimer)
 #define MLA_TRACE(ev, k)                                                                         \
   do {                                                                                           \
     const int tr_pair_ = static_cast<int>(blockIdx.x >> 1);                                      \
@@ -280,6 +281,7 @@ __device__ void producer_k(const DecodeParams& p, const Ctx& c, int s_begin, int
       if (gr.first) {  // the segment's Q rows first
         good = seg_it == 0 || wait_bar(c, c.bar(kBarQEmpty), (seg_it - 1) & 1);
         if (good) {
+          MLA_TRACE(14, seg_it);
           if (c.cta == 0) mbar_arrive_expect_tx(c.bar(kBarQFull), 2 * kQBytes);
           const int y = sg.i * p.R + sg.mt * kMTile + c.cta * kRowsCta;
           tma_load_3d_pair(c.base + kOffQ, &p.tm_q, c.lead_bar(kBarQFull), 0, y, 0);
@@ -605,6 +607,7 @@ __device__ void softmax_epilogue(const DecodeParams& p, const Ctx& c, uint32_t t
 
     // ---- epilogue ----
     if (!pv_done(ps - 1)) return;
+    if (r == 0) MLA_TRACE(12, s - s_begin);
     tc_fence_after();
     float l_peer;
     if (!trade(l, &l_peer)) return;
@@ -658,6 +661,7 @@ __device__ void softmax_epilogue(const DecodeParams& p, const Ctx& c, uint32_t t
     tc_fence_before();
     __syncwarp();
     if (lane == 0) arrive_leader(c, kBarOEmpty);
+    if (r == 0) MLA_TRACE(13, s - s_begin);
   }
 }
 
@@ -715,6 +719,12 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
   const uint32_t tmem = *reinterpret_cast<volatile uint32_t*>(c.gbase + kOffTmemSlot);
   c.peer_abort = map_to_rank(base + kOffAbort, c.cta ^ 1u);
   c.lead_bars = map_to_rank(base + kOffBar, 0);
+  // Programmatic dependent launch: the set-up above overlapped the previous
+  // kernel (the plan, or the previous call's combine); wait for its
+  // completion before reading the plan or writing any output.  The combine
+  // may start launching now (it waits for this kernel in turn).
+  griddep_launch_dependents();
+  griddep_wait();
 
   // The plan must be the one built for this call's shape on this many pairs.
   const int pair = static_cast<int>(blockIdx.x >> 1);
@@ -730,6 +740,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     atomicOr(reinterpret_cast<unsigned int*>(c.meta + kHError), MLA_DEVERR_PLAN);
   }
 
+  if (threadIdx.x == 128) MLA_TRACE(11, 0);
+#ifdef MLA_DECODE_TRACE
+  if (threadIdx.x == 0 && c.cta == 0) g_mla_span[blockIdx.x >> 1][0] = globaltimer();
+#endif
   if (warp == 0) {
     producer_k(p, c, s_begin, s_end);
   } else if (warp == 1) {
@@ -756,6 +770,12 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     }
     __syncwarp();
   }
+#ifdef MLA_DECODE_TRACE
+  if (threadIdx.x == 0 && c.cta == 0) {
+    g_mla_span[blockIdx.x >> 1][1] = globaltimer();
+    g_mla_span[blockIdx.x >> 1][2] = s_end - s_begin;
+  }
+#endif
   if (*c.abort_flag) __nanosleep(20000);  // let in-flight copies and arrivals land
   tc_fence_before();
   __syncthreads();
@@ -771,6 +791,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
 #ifdef MLA_DECODE_TRACE
 extern "C" __attribute__((visibility("default"))) int mla_trace_read(void* host) {
   return static_cast<int>(cudaMemcpyFromSymbol(host, g_mla_trace, sizeof(g_mla_trace)));
+}
+extern "C" __attribute__((visibility("default"))) int mla_trace_span(void* host) {
+  return static_cast<int>(cudaMemcpyFromSymbol(host, g_mla_span, sizeof(g_mla_span)));
 }
 extern "C" __attribute__((visibility("default"))) int mla_trace_clear() {
   static unsigned long long zero[4][16][512];
@@ -810,8 +833,17 @@ cudaError_t decode_kernel_pairs(int* pairs) {
 }
 
 cudaError_t launch_decode(const DecodeParams& p, int pairs, cudaStream_t stream) {
-  mla_decode_kernel<<<dim3(2 * pairs), dim3(kThreads), kSmemBytes, stream>>>(p);
-  return cudaGetLastError();
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(static_cast<unsigned>(2 * pairs), 1, 1);
+  cfg.blockDim = dim3(kThreads, 1, 1);
+  cfg.dynamicSmemBytes = kSmemBytes;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, mla_decode_kernel, p);
 }
 
 }  // namespace mla

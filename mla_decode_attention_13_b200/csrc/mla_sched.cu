@@ -22,6 +22,7 @@
 // Everything follows from prefix sums, so one CTA computes it with block-wide
 // scans over chunks of 1024 rows and one binary search per pair.
 #include "mla_internal.h"
+#include "sm100_ptx.cuh"
 
 namespace mla {
 namespace {
@@ -70,6 +71,11 @@ __device__ __forceinline__ int row_pages(const int32_t* seqlens, int batch, int 
 
 __global__ void __launch_bounds__(kSchedThreads) mla_sched_kernel(const int32_t* __restrict__ seqlens, int batch,
                                                                   int h_q, int s_q, int pairs, int32_t* meta) {
+  // Programmatic dependent launch: the decode kernel may start its set-up now;
+  // this kernel itself waits until the previous kernel in the stream (which
+  // may still read the metadata, or have written the lengths) has completed.
+  ptx::griddep_launch_dependents();
+  ptx::griddep_wait();
   const MetaLayout lo = meta_layout(batch, h_q, s_q);
   const int W = lo.W;
   const int R = s_q * h_q;
@@ -200,8 +206,16 @@ __global__ void __launch_bounds__(kSchedThreads) mla_sched_kernel(const int32_t*
 
 cudaError_t launch_sched(const int32_t* seqlens, int batch, int h_q, int s_q, int pairs, int32_t* meta,
                          cudaStream_t stream) {
-  mla_sched_kernel<<<1, kSchedThreads, 0, stream>>>(seqlens, batch, h_q, s_q, pairs, meta);
-  return cudaGetLastError();
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(1, 1, 1);
+  cfg.blockDim = dim3(kSchedThreads, 1, 1);
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, mla_sched_kernel, seqlens, batch, h_q, s_q, pairs, meta);
 }
 
 }  // namespace mla
