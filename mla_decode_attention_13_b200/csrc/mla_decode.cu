@@ -123,7 +123,8 @@ enum Bar : uint32_t {
   kBarOEmpty = kBarQEmpty + 1,         // (leader) both CTAs' softmax warps read O out
   kBarFinal = kBarOEmpty + 1,          // (leader) MMA drain at teardown: both issuer threads
   kBarXch = kBarFinal + 1,             // [2] (both) warps 4+6 / 5+7 published row values
-  kNumBars = kBarXch + 2,
+  kBarStageFree = kBarXch + 2,         // (both, local) the epilogue's stores have read their staging
+  kNumBars = kBarStageFree + 1,
 };
 constexpr uint32_t kOffTmemSlot = kOffBar + 8 * kNumBars;  // u32
 constexpr uint32_t kOffAbort = kOffTmemSlot + 4;           // u32
@@ -312,10 +313,13 @@ __device__ void producer_k(const DecodeParams& p, const Ctx& c, int s_begin, int
 // before releasing P, so PV never runs ahead of it).
 __device__ void producer_v(const DecodeParams& p, const Ctx& c, int s_begin, int s_end) {
   const int lane = threadIdx.x & 31;
-  uint32_t ps = 0;  // pages
+  uint32_t ps = 0, seg_it = 0;  // pages, segments
   walk_groups(p, c, s_begin, s_end, [&](const Segment&, const Group& gr) -> bool {
     int good = 1;
     if (lane == 0) {
+      // The epilogue of the previous segment stages its output in the value
+      // ring: a new segment's first tile waits until those stores have read it.
+      if (gr.first && seg_it > 0) good = wait_bar(c, c.bar(kBarStageFree), (seg_it - 1) & 1);
       for (int q = 0; q < gr.np && good; ++q, ++ps) {
         const uint32_t slot = ps % kVRing;
         if (ps >= kVRing) good = wait_bar(c, c.bar(kBarPvDone + slot), ((ps - kVRing) / kVRing) & 1);
@@ -330,6 +334,7 @@ __device__ void producer_v(const DecodeParams& p, const Ctx& c, int s_begin, int
         }
       }
     }
+    if (gr.first) ++seg_it;
     return __shfl_sync(0xffffffffu, good, 0) != 0;
   });
 }
@@ -614,55 +619,93 @@ __device__ void softmax_epilogue(const DecodeParams& p, const Ctx& c, uint32_t t
     const float lt = l + l_peer;
     const float inv_l = lt > 0.0f ? 1.0f / lt : 0.0f;
     const float lse_v = lt > 0.0f ? (m + __log2f(lt)) * 0.69314718055994530942f : -INFINITY;
-    // This thread's O columns: for each half h of the 512, columns
+    // Output through TMA stores: each warp stages its 32 rows x 128 bytes of
+    // columns in shared memory (128B-swizzled, two buffers per warp in the
+    // value ring, idle now) and stores the box; rows past R (or tile_rows)
+    // lie outside the store tensor and are dropped by the copy engine.  This
+    // thread's O columns: for each half h of the 512, columns
     // [256h + 128*half, 256h + 128*half + 128).
+    const int wq = r >> 5;  // softmax warp 0-3: rows 32 (wq & 1) .., column half wq >> 1
+    const uint32_t stage0 = c.base + kOffV + wq * 8192;
+    uint8_t* stage0_g = c.gbase + kOffV + wq * 8192;
+    const int row0 = c.cta * kRowsCta + 32 * (wq & 1);  // first row of this warp's box in the tile
+    const uint32_t swz = lane & 7;
     if (sg.slot < 0) {
-      __nv_bfloat16* orow = reinterpret_cast<__nv_bfloat16*>(p.out) + (static_cast<long long>(sg.i) * p.R + row_g) * kDv;
+      const int y = sg.mt * kMTile + row0;
+      const bool any = y < p.R;
 #pragma unroll 1
-      for (int cc = 0; cc < 256; cc += 32) {
-        float o[32];
-        tmem_ld32(t_o + cc, o);
+      for (int k = 0; k < 4; ++k) {  // 64 columns (128 bytes of bf16) per box
+        float o[64];
+        tmem_ld32(t_o + 64 * k, *reinterpret_cast<float(*)[32]>(o));
+        tmem_ld32(t_o + 64 * k + 32, *reinterpret_cast<float(*)[32]>(o + 32));
         tmem_wait_ld();
-        const int col = (cc >> 7) * 256 + 128 * half + (cc & 127);
-        if (row_valid) {
-#pragma unroll
-          for (int k = 0; k < 32; k += 8) {
-            uint4 v;
-            __nv_bfloat162 h0 = __floats2bfloat162_rn(o[k + 0] * inv_l, o[k + 1] * inv_l);
-            __nv_bfloat162 h1 = __floats2bfloat162_rn(o[k + 2] * inv_l, o[k + 3] * inv_l);
-            __nv_bfloat162 h2 = __floats2bfloat162_rn(o[k + 4] * inv_l, o[k + 5] * inv_l);
-            __nv_bfloat162 h3 = __floats2bfloat162_rn(o[k + 6] * inv_l, o[k + 7] * inv_l);
-            v.x = *reinterpret_cast<uint32_t*>(&h0);
-            v.y = *reinterpret_cast<uint32_t*>(&h1);
-            v.z = *reinterpret_cast<uint32_t*>(&h2);
-            v.w = *reinterpret_cast<uint32_t*>(&h3);
-            *reinterpret_cast<uint4*>(orow + col + k) = v;
-          }
+        const uint32_t buf = k & 1;
+        if (k >= 2) {
+          if (lane == 0) bulk_wait_group_read<1>();
+          __syncwarp();
         }
+        uint8_t* srow = stage0_g + buf * 4096 + lane * 128;
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {
+          __nv_bfloat162 h0 = __floats2bfloat162_rn(o[8 * j + 0] * inv_l, o[8 * j + 1] * inv_l);
+          __nv_bfloat162 h1 = __floats2bfloat162_rn(o[8 * j + 2] * inv_l, o[8 * j + 3] * inv_l);
+          __nv_bfloat162 h2 = __floats2bfloat162_rn(o[8 * j + 4] * inv_l, o[8 * j + 5] * inv_l);
+          __nv_bfloat162 h3 = __floats2bfloat162_rn(o[8 * j + 6] * inv_l, o[8 * j + 7] * inv_l);
+          uint4 v;
+          v.x = *reinterpret_cast<uint32_t*>(&h0);
+          v.y = *reinterpret_cast<uint32_t*>(&h1);
+          v.z = *reinterpret_cast<uint32_t*>(&h2);
+          v.w = *reinterpret_cast<uint32_t*>(&h3);
+          *reinterpret_cast<uint4*>(srow + ((j ^ swz) << 4)) = v;
+        }
+        fence_proxy_async_smem();
+        __syncwarp();
+        if (lane == 0 && any) {
+          const int col = (k >> 1) * 256 + 128 * half + (k & 1) * 64;
+          tma_store_3d(&p.tm_out, stage0 + buf * 4096, col, y, sg.i);
+        }
+        if (lane == 0) bulk_commit_group();
       }
       if (row_valid && half == 0) p.lse[(static_cast<long long>(sg.i) * p.h_q + hh) * p.s_q + t] = lse_v;
     } else {
-      float* orow = p.o_part + (static_cast<long long>(sg.slot) * p.tile_rows + q_row) * kDv;
+      const bool any = row0 < p.tile_rows;
 #pragma unroll 1
-      for (int cc = 0; cc < 256; cc += 32) {
+      for (int k = 0; k < 8; ++k) {  // 32 columns (128 bytes of fp32) per box
         float o[32];
-        tmem_ld32(t_o + cc, o);
+        tmem_ld32(t_o + 32 * k, o);
         tmem_wait_ld();
-        const int col = (cc >> 7) * 256 + 128 * half + (cc & 127);
-        if (row_valid) {
-#pragma unroll
-          for (int k = 0; k < 32; k += 4)
-            *reinterpret_cast<float4*>(orow + col + k) =
-                make_float4(o[k] * inv_l, o[k + 1] * inv_l, o[k + 2] * inv_l, o[k + 3] * inv_l);
+        const uint32_t buf = k & 1;
+        if (k >= 2) {
+          if (lane == 0) bulk_wait_group_read<1>();
+          __syncwarp();
         }
+        uint8_t* srow = stage0_g + buf * 4096 + lane * 128;
+#pragma unroll
+        for (int j = 0; j < 8; ++j)
+          *reinterpret_cast<float4*>(srow + ((j ^ swz) << 4)) =
+              make_float4(o[4 * j] * inv_l, o[4 * j + 1] * inv_l, o[4 * j + 2] * inv_l, o[4 * j + 3] * inv_l);
+        fence_proxy_async_smem();
+        __syncwarp();
+        if (lane == 0 && any) {
+          const int col = (k >> 2) * 256 + 128 * half + (k & 3) * 32;
+          tma_store_3d(&p.tm_opart, stage0 + buf * 4096, col, row0, sg.slot);
+        }
+        if (lane == 0) bulk_commit_group();
       }
       if (row_valid && half == 0) p.lse_part[static_cast<long long>(sg.slot) * p.tile_rows + q_row] = lse_v;
     }
     tc_fence_before();
     __syncwarp();
-    if (lane == 0) arrive_leader(c, kBarOEmpty);
+    if (lane == 0) arrive_leader(c, kBarOEmpty);  // O is read out: the next segment's PV may overwrite it
+    if (lane == 0) {
+      bulk_wait_group_read<0>();
+      mbar_arrive(c.bar(kBarStageFree));  // staging read: the value ring may be refilled
+    }
+    __syncwarp();
     if (r == 0) MLA_TRACE(13, s - s_begin);
   }
+  if (lane == 0) bulk_wait_group_all();  // this warp's output stores have landed
+  __syncwarp();
 }
 
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
@@ -700,6 +743,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     mbar_init(c.bar(kBarQEmpty), 1);
     mbar_init(c.bar(kBarOEmpty), 8);
     mbar_init(c.bar(kBarFinal), 2);
+    mbar_init(c.bar(kBarStageFree), 4);
     *c.abort_flag = 0u;
     fence_mbar_init_cluster();
   }
