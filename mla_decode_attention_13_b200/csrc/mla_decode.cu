@@ -243,13 +243,21 @@ struct Group {
 // Walks this pair's segments in plan order and calls fn(segment, group) for
 // every group, with the page ids read 32 at a time by the whole warp (one
 // chunk ahead).  fn runs on every lane and returns false to stop the walk.
-template <typename Fn>
-__device__ __forceinline__ void walk_groups(const DecodeParams& p, const Ctx& c, int s_begin, int s_end, Fn&& fn) {
+// on_segment(segment) runs on every lane before the segment's page ids are
+// read, and returns false to stop the walk.
+struct NoSegmentHook {
+  __device__ bool operator()(const Segment&) const { return true; }
+};
+
+template <typename Fn, typename SegFn = NoSegmentHook>
+__device__ __forceinline__ void walk_groups(const DecodeParams& p, const Ctx& c, int s_begin, int s_end, Fn&& fn,
+                                            SegFn&& on_segment = SegFn()) {
   static_assert(32 % kGroup == 0, "groups never straddle a chunk of page ids");
   const int lane = threadIdx.x & 31;
   for (int s = s_begin; s < s_end; ++s) {
     const Segment sg = load_segment(p, s);
     if (sg.bad) continue;
+    if (!on_segment(sg)) return;
     const int32_t* table = p.block_table + static_cast<long long>(sg.i) * p.max_pages;
     int cur = load_page(p, c, table, sg.b0 + lane, sg.b1);
     for (int c0 = sg.b0; c0 < sg.b1; c0 += 32) {
@@ -276,19 +284,25 @@ __device__ __forceinline__ void walk_groups(const DecodeParams& p, const Ctx& c,
 __device__ void producer_k(const DecodeParams& p, const Ctx& c, int s_begin, int s_end) {
   const int lane = threadIdx.x & 31;
   uint32_t gi = 0, seg_it = 0, ks = 0;  // groups, segments started, key panels loaded
+  // The segment's Q rows first, before its page ids are even read.
+  auto load_q = [&](const Segment& sg) -> bool {
+    int good = 1;
+    if (lane == 0) {
+      good = seg_it == 0 || wait_bar(c, c.bar(kBarQEmpty), (seg_it - 1) & 1);
+      if (good) {
+        MLA_TRACE(14, seg_it);
+        if (c.cta == 0) mbar_arrive_expect_tx(c.bar(kBarQFull), 2 * kQBytes);
+        const int y = sg.i * p.R + sg.mt * kMTile + c.cta * kRowsCta;
+        tma_load_3d_pair(c.base + kOffQ, &p.tm_q, c.lead_bar(kBarQFull), 0, y, 0);
+      }
+    }
+    ++seg_it;
+    return __shfl_sync(0xffffffffu, good, 0) != 0;
+  };
   walk_groups(p, c, s_begin, s_end, [&](const Segment& sg, const Group& gr) -> bool {
     int good = 1;
     if (lane == 0) {
-      if (gr.first) {  // the segment's Q rows first
-        good = seg_it == 0 || wait_bar(c, c.bar(kBarQEmpty), (seg_it - 1) & 1);
-        if (good) {
-          MLA_TRACE(14, seg_it);
-          if (c.cta == 0) mbar_arrive_expect_tx(c.bar(kBarQFull), 2 * kQBytes);
-          const int y = sg.i * p.R + sg.mt * kMTile + c.cta * kRowsCta;
-          tma_load_3d_pair(c.base + kOffQ, &p.tm_q, c.lead_bar(kBarQFull), 0, y, 0);
-        }
-      }
-      if (good) MLA_TRACE(0, gi);
+      MLA_TRACE(0, gi);
       for (int pn = 0; pn < 9 && good; ++pn, ++ks) {
         const uint32_t slot = ks % kKRing;
         if (ks >= kKRing) good = wait_bar(c, c.bar(kBarKEmpty + slot), ((ks / kKRing) - 1) & 1);
@@ -301,10 +315,9 @@ __device__ void producer_k(const DecodeParams& p, const Ctx& c, int s_begin, int
         }
       }
     }
-    if (gr.first) ++seg_it;
     ++gi;
     return __shfl_sync(0xffffffffu, good, 0) != 0;
-  });
+  }, load_q);
 }
 
 // Warp 2: this CTA's value tile of every page (all 64 tokens, its 256 value
