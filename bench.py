@@ -9,9 +9,11 @@ batch 16, s_q 1, h_q 128, lengths uniform in [1024, 4096] (64-token pages,
 1.25x shuffled pool, bf16 N(0, 1)).  Calls rotate over several independent
 pools whose total size is at least 3x the L2 cache, so each step reads its
 cache from HBM.  The timed region replays CUDA graphs of those steps (exactly
-K steps), bracketed by a barrier and a device synchronisation, timed with CUDA
-events on the launching stream; the split-KV kernel is also timed on its own
-through events recorded around it inside the graphs.
+K steps, no event nodes between the kernels so that programmatic dependent
+launch applies), bracketed by a barrier and a device synchronisation, timed
+with CUDA events on the launching stream; the split-KV kernel is also timed on
+its own, by graphs of the same steps with events recorded around it, replayed
+right after the timed region.
 
 With --gpus N > 1 (launched by torchrun, one process per GPU, NCCL), every
 rank runs its own batch (batch rows are independent: weak scaling, no
