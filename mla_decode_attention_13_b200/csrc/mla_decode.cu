@@ -31,9 +31,10 @@
 //     columns [256h + 128c, 256h + 128c + 128) (h = 0, 1): a 32 KB tile per
 //     page, read from L2 (the pair has just brought the page in), in a ring
 //     of two.
-//   * Softmax: thread r (= TMEM lane r) handles row r mod 64, 128 scores (32
-//     tokens of each page); the two threads of a row trade their maxima
-//     through shared memory.  Online softmax in the log2 domain with a lazy
+//   * Softmax: eight warps; warps 4-7 take pages 0-1 of each group, warps
+//     8-11 pages 2-3.  A thread (TMEM lane r) handles row r mod 64, 64 scores
+//     (32 tokens of each of its two pages); the four threads of a row trade
+//     their maxima (and, at the end, their sums) through shared memory.  Online softmax in the log2 domain with a lazy
 //     rescale (the running max only moves when a block's max exceeds it by
 //     more than kTau; O and the running sums are rescaled together, so the
 //     result is exact).  The bf16-rounded weights P of each page go to a ring
@@ -47,9 +48,9 @@
 //   producer warps read page ids 32 at a time.
 // A row the plan splits writes fp32 (O / l, lse) partials to the workspace
 // for the combine kernel; an unsplit row writes bf16 out and lse.
-// Warp roles per CTA (256 threads): warp 0 = key/Q producer, warp 1 = TMEM
+// Warp roles per CTA (384 threads): warp 0 = key/Q producer, warp 1 = TMEM
 // owner and (leader only) QK issuer, warp 2 = value producer, warp 3 =
-// (leader only) PV issuer, warps 4-7 = softmax and epilogue.  (A bulk L2 prefetch of the pages ahead of the key
+// (leader only) PV issuer, warps 4-11 = softmax and epilogue.  (A bulk L2 prefetch of the pages ahead of the key
 // loads was measured on B200 and made the kernel slower; there is none.)
 //
 // Cross-CTA signals are relaxed arrivals after a CTA-scope fence (see
@@ -85,7 +86,7 @@ namespace {
 
 using namespace ptx;
 
-constexpr int kThreads = 256;
+constexpr int kThreads = 384;
 constexpr int kGroup = 4;             // pages per QK group
 constexpr int kKRing = 4;             // key panel slots
 constexpr int kVRing = 2;             // value tiles (and P tiles)
@@ -107,8 +108,8 @@ constexpr uint32_t kOffQ = 0;
 constexpr uint32_t kOffK = kOffQ + kQBytes;
 constexpr uint32_t kOffV = kOffK + kKRing * kKSlot;
 constexpr uint32_t kOffP = kOffV + kVRing * kVTile;
-constexpr uint32_t kOffX = kOffP + kVRing * kPTile;     // float [2][128] row exchange
-constexpr uint32_t kOffBar = kOffX + 2 * 128 * 4;
+constexpr uint32_t kOffX = kOffP + kVRing * kPTile;     // float [2][256] row exchange
+constexpr uint32_t kOffBar = kOffX + 2 * 256 * 4;
 
 enum Bar : uint32_t {
   kBarKFull = 0,                       // [kKRing] (leader) both CTAs' key panel landed
@@ -122,8 +123,8 @@ enum Bar : uint32_t {
   kBarQEmpty = kBarQFull + 1,          // (both) last QK of the segment done
   kBarOEmpty = kBarQEmpty + 1,         // (leader) both CTAs' softmax warps read O out
   kBarFinal = kBarOEmpty + 1,          // (leader) MMA drain at teardown: both issuer threads
-  kBarXch = kBarFinal + 1,             // [2] (both) warps 4+6 / 5+7 published row values
-  kBarStageFree = kBarXch + 2,         // (both, local) the epilogue's stores have read their staging
+  kBarXch = kBarFinal + 1,             // (both) the 8 softmax warps published row values
+  kBarStageFree = kBarXch + 1,         // (both, local) the epilogue's stores have read their staging
   kNumBars = kBarStageFree + 1,
 };
 constexpr uint32_t kOffTmemSlot = kOffBar + 8 * kNumBars;  // u32
@@ -480,33 +481,36 @@ __device__ __forceinline__ float exp_pack(const float (&sv)[32], int nvalid, flo
 }
 
 __device__ void softmax_epilogue(const DecodeParams& p, const Ctx& c, uint32_t tmem, int s_begin, int s_end) {
-  const int r = threadIdx.x - 128;  // TMEM lane
+  const int r = threadIdx.x - 128;  // 0-255: softmax thread
+  const int sp = r >> 7;            // page pair: pages 2 sp, 2 sp + 1 of each group (S columns 64 sp ..)
+  const int rr = r & 127;           // TMEM lane
   const int lane = threadIdx.x & 31;
-  const int hr = r & (kRowsCta - 1);  // query row within this CTA
-  const int half = r >> 6;            // 0: tokens 0-31 of each page / first column half; 1: the rest
-  const uint32_t lane_off = static_cast<uint32_t>(r & ~31) << 16;
-  const uint32_t t_s = tmem + lane_off + kColS;
-  const uint32_t t_o = tmem + lane_off + kColO;
-  const uint32_t xbar = c.bar(kBarXch + ((r >> 5) & 1));  // warps 4+6 and 5+7 hold the two halves of rows
+  const int hr = rr & (kRowsCta - 1);  // query row within this CTA
+  const int half = rr >> 6;            // 0: tokens 0-31 of each page / first column half; 1: the rest
+  const uint32_t lane_off = static_cast<uint32_t>(rr & ~31) << 16;
+  const uint32_t t_s = tmem + lane_off + kColS + 64 * sp;
+  const uint32_t t_o = tmem + lane_off + kColO + 128 * sp;  // this thread's 128 O columns
   float* xbuf = reinterpret_cast<float*>(c.gbase + kOffX);
   // This thread's 32 weights of a page: 64 bytes of P row hr, 16-byte chunks
   // 4 half .. 4 half + 3, swizzled by the row.
   const uint32_t prow_off = (hr >> 3) * 1024 + (hr & 7) * 128;
   const float sl2 = p.scale_log2;
-  // gi: groups, ps: pages consumed so far (select buffers and phases);
-  // x_cnt: row exchanges with the partner thread.
+  // gi: groups, ps: pages before the current group (select buffers and
+  // phases); x_cnt: row exchanges among the row's four threads.
   uint32_t gi = 0, ps = 0, x_cnt = 0;
   auto pv_done = [&](uint32_t k) -> bool { return wait_bar(c, c.bar(kBarPvDone + k % kVRing), (k / kVRing) & 1); };
-  // Publish v for the partner thread (same row, other half) and return its
-  // value; the two warps meet on an mbarrier (bounded wait).
-  auto trade = [&](float v, float* out) -> bool {
-    float* buf = xbuf + (x_cnt & 1) * 128;
+  // Publish v for the other three threads of this row (the other half of its
+  // tokens, the other page pair) and return the max or the sum of the four;
+  // the eight softmax warps meet on an mbarrier (bounded wait).
+  auto trade = [&](float v, bool sum, float* out) -> bool {
+    float* buf = xbuf + (x_cnt & 1) * 256;
     buf[r] = v;
     __syncwarp();
-    if (lane == 0) mbar_arrive(xbar);
-    const bool ok = wait_bar(c, xbar, x_cnt & 1);
+    if (lane == 0) mbar_arrive(c.bar(kBarXch));
+    const bool ok = wait_bar(c, c.bar(kBarXch), x_cnt & 1);
     ++x_cnt;
-    *out = buf[r ^ 64];
+    const float a = buf[r ^ 64], b = buf[r ^ 128], d = buf[r ^ 192];
+    *out = sum ? (v + a) + (b + d) : fmaxf(fmaxf(v, a), fmaxf(b, d));
     return ok;
   };
 
@@ -529,7 +533,7 @@ __device__ void softmax_epilogue(const DecodeParams& p, const Ctx& c, uint32_t t
     }
     const int last_page = ceil_div(sg.L, kPage) - 1;
 
-    float m = -INFINITY, l = 0.0f;  // l: this thread's half of the row sum
+    float m = -INFINITY, l = 0.0f;  // l: this thread's share of the row sum
     for (int j = 0; j < n; j += kGroup, ++gi) {
       const int blk = sg.b0 + j;
       const int np = min(kGroup, n - j);
@@ -537,39 +541,39 @@ __device__ void softmax_epilogue(const DecodeParams& p, const Ctx& c, uint32_t t
       if (!wait_bar(c, c.bar(kBarSFull + sb), (gi >> 1) & 1)) return;
       if (r == 0) MLA_TRACE(4, gi);
       tc_fence_after();
-      float sv[kGroup][32];
-#pragma unroll
-      for (int q = 0; q < kGroup; ++q) tmem_ld32(t_s + 128 * sb + 32 * q, sv[q]);
+      float sv[2][32];
+      tmem_ld32(t_s + 128 * sb, sv[0]);
+      tmem_ld32(t_s + 128 * sb + 32, sv[1]);
       tmem_wait_ld();
       tc_fence_before();
       __syncwarp();
       if (lane == 0) arrive_leader(c, kBarSEmpty + sb);  // S buffer read
 
       // ---- mask; max over the group's pages and both halves of the row ----
-      int nv[kGroup];
+      int nv[2];
       float mx = -INFINITY;
 #pragma unroll
-      for (int q = 0; q < kGroup; ++q) {
-        int v = limit - (blk + q) * kPage - kHalfPage * half;
-        nv[q] = (q >= np || v < 0) ? 0 : (v > 32 ? 32 : v);
-        mx = fmaxf(mx, masked_max(sv[q], nv[q]));
+      for (int e = 0; e < 2; ++e) {
+        const int q = 2 * sp + e;
+        const int v = limit - (blk + q) * kPage - kHalfPage * half;
+        nv[e] = (q >= np || v < 0) ? 0 : (v > 32 ? 32 : v);
+        mx = fmaxf(mx, masked_max(sv[e], nv[e]));
       }
       mx = (nv[0] > 0) ? mx * sl2 : -INFINITY;  // tokens are valid from the left; softmax_scale >= 0
-      float mx_peer;
-      if (!trade(mx, &mx_peer)) return;
+      if (!trade(mx, false, &mx)) return;
       if (r == 0) MLA_TRACE(5, gi);
-      mx = fmaxf(mx, mx_peer);
       float m_new = m;
       if (mx > m + kTau) m_new = mx;  // also true for the first finite block
       const float alpha = (m_new == m) ? 1.0f : ex2(m - m_new);  // 0 when m was -inf
       const float neg_m = (m_new == -INFINITY) ? 0.0f : -m_new;
 
-      // ---- rescale O (rare): after PV of every earlier page of the segment ----
+      // ---- rescale this thread's O columns (rare): after PV of every earlier
+      //      page of the segment ----
       if (j > 0 && __any_sync(0xffffffffu, alpha < 1.0f)) {
         if (!pv_done(ps - 1)) return;
         tc_fence_after();
 #pragma unroll 1
-        for (int cc = 0; cc < 256; cc += 32) {
+        for (int cc = 0; cc < 128; cc += 32) {
           float o[32];
           tmem_ld32(t_o + cc, o);
           tmem_wait_ld();
@@ -582,14 +586,16 @@ __device__ void softmax_epilogue(const DecodeParams& p, const Ctx& c, uint32_t t
 
       float lsum = 0.0f;
 #pragma unroll
-      for (int q = 0; q < kGroup; ++q) {
+      for (int e = 0; e < 2; ++e) {
+        const int q = 2 * sp + e;
         if (q >= np) break;
+        const uint32_t pg = ps + q;  // global page index
         uint32_t packed[16];
-        lsum += exp_pack(sv[q], nv[q], sl2, neg_m, packed);
-        const uint32_t slot = ps % kVRing;
+        lsum += exp_pack(sv[e], nv[e], sl2, neg_m, packed);
+        const uint32_t slot = pg % kVRing;
         // ---- P tile free (PV two pages back) ----
-        if (ps >= kVRing && !pv_done(ps - kVRing)) return;
-        if (r == 0) MLA_TRACE(6, ps);
+        if (pg >= kVRing && !pv_done(pg - kVRing)) return;
+        if (r == 0 || r == 128) MLA_TRACE(6, pg);
         {
           uint8_t* prow = c.gbase + kOffP + slot * kPTile + prow_off;
 #pragma unroll
@@ -600,13 +606,13 @@ __device__ void softmax_epilogue(const DecodeParams& p, const Ctx& c, uint32_t t
         // ---- this CTA's value tile has landed; the last page of a row may
         //      hold garbage (even NaN) past L: zero the value rows there, so
         //      that 0 * garbage cannot reach O ----
-        if (!wait_bar(c, c.bar(kBarVFull + slot), (ps / kVRing) & 1)) return;
-        if (r == 0) MLA_TRACE(7, ps);
+        if (!wait_bar(c, c.bar(kBarVFull + slot), (pg / kVRing) & 1)) return;
+        if (r == 0 || r == 128) MLA_TRACE(7, pg);
         if (blk + q == last_page && (sg.L & (kPage - 1))) {
           const int first_bad = sg.L - last_page * kPage;
           const int chunks = (kPage - first_bad) * 4 * 8;  // tokens x panels x 16-byte chunks
           uint8_t* vt = c.gbase + kOffV + slot * kVTile;
-          for (int e2 = r; e2 < chunks; e2 += 128) {
+          for (int e2 = rr; e2 < chunks; e2 += 128) {
             const int tok = first_bad + (e2 >> 5);
             *reinterpret_cast<uint4*>(vt + ((e2 >> 3) & 3) * kVPanel + tok * 128 + (e2 & 7) * 16) =
                 make_uint4(0, 0, 0, 0);
@@ -616,74 +622,65 @@ __device__ void softmax_epilogue(const DecodeParams& p, const Ctx& c, uint32_t t
         tc_fence_before();
         __syncwarp();
         if (lane == 0) arrive_leader(c, kBarPFull + slot);
-        if (r == 0) MLA_TRACE(8, ps);
-        ++ps;
+        if (r == 0 || r == 128) MLA_TRACE(8, pg);
       }
       l = l * alpha + lsum;
       m = m_new;
+      ps += np;
     }
 
     // ---- epilogue ----
     if (!pv_done(ps - 1)) return;
     if (r == 0) MLA_TRACE(12, s - s_begin);
     tc_fence_after();
-    float l_peer;
-    if (!trade(l, &l_peer)) return;
-    const float lt = l + l_peer;
+    float lt;
+    if (!trade(l, true, &lt)) return;
     const float inv_l = lt > 0.0f ? 1.0f / lt : 0.0f;
     const float lse_v = lt > 0.0f ? (m + __log2f(lt)) * 0.69314718055994530942f : -INFINITY;
     // Output through TMA stores: each warp stages its 32 rows x 128 bytes of
     // columns in shared memory (128B-swizzled, two buffers per warp in the
     // value ring, idle now) and stores the box; rows past R (or tile_rows)
     // lie outside the store tensor and are dropped by the copy engine.  This
-    // thread's O columns: for each half h of the 512, columns
-    // [256h + 128*half, 256h + 128*half + 128).
-    const int wq = r >> 5;  // softmax warp 0-3: rows 32 (wq & 1) .., column half wq >> 1
-    const uint32_t stage0 = c.base + kOffV + wq * 8192;
-    uint8_t* stage0_g = c.gbase + kOffV + wq * 8192;
-    const int row0 = c.cta * kRowsCta + 32 * (wq & 1);  // first row of this warp's box in the tile
+    // thread's O columns: [256 sp + 128 half, +128).
+    const int ws = (threadIdx.x >> 5) - 4;  // softmax warp 0-7
+    const uint32_t stage0 = c.base + kOffV + ws * 8192;
+    uint8_t* stage0_g = c.gbase + kOffV + ws * 8192;
+    const int row0 = c.cta * kRowsCta + 32 * ((rr >> 5) & 1);  // first row of this warp's box in the tile
     const uint32_t swz = lane & 7;
+    const int col0 = 256 * sp + 128 * half;
     if (sg.slot < 0) {
       const int y = sg.mt * kMTile + row0;
       const bool any = y < p.R;
 #pragma unroll 1
-      for (int k = 0; k < 4; ++k) {  // 64 columns (128 bytes of bf16) per box
+      for (int k = 0; k < 2; ++k) {  // 64 columns (128 bytes of bf16) per box
         float o[64];
         tmem_ld32(t_o + 64 * k, *reinterpret_cast<float(*)[32]>(o));
         tmem_ld32(t_o + 64 * k + 32, *reinterpret_cast<float(*)[32]>(o + 32));
         tmem_wait_ld();
-        const uint32_t buf = k & 1;
-        if (k >= 2) {
-          if (lane == 0) bulk_wait_group_read<1>();
-          __syncwarp();
-        }
-        uint8_t* srow = stage0_g + buf * 4096 + lane * 128;
+        uint8_t* srow = stage0_g + k * 4096 + lane * 128;
 #pragma unroll
-        for (int j = 0; j < 8; ++j) {
-          __nv_bfloat162 h0 = __floats2bfloat162_rn(o[8 * j + 0] * inv_l, o[8 * j + 1] * inv_l);
-          __nv_bfloat162 h1 = __floats2bfloat162_rn(o[8 * j + 2] * inv_l, o[8 * j + 3] * inv_l);
-          __nv_bfloat162 h2 = __floats2bfloat162_rn(o[8 * j + 4] * inv_l, o[8 * j + 5] * inv_l);
-          __nv_bfloat162 h3 = __floats2bfloat162_rn(o[8 * j + 6] * inv_l, o[8 * j + 7] * inv_l);
+        for (int jj = 0; jj < 8; ++jj) {
+          __nv_bfloat162 h0 = __floats2bfloat162_rn(o[8 * jj + 0] * inv_l, o[8 * jj + 1] * inv_l);
+          __nv_bfloat162 h1 = __floats2bfloat162_rn(o[8 * jj + 2] * inv_l, o[8 * jj + 3] * inv_l);
+          __nv_bfloat162 h2 = __floats2bfloat162_rn(o[8 * jj + 4] * inv_l, o[8 * jj + 5] * inv_l);
+          __nv_bfloat162 h3 = __floats2bfloat162_rn(o[8 * jj + 6] * inv_l, o[8 * jj + 7] * inv_l);
           uint4 v;
           v.x = *reinterpret_cast<uint32_t*>(&h0);
           v.y = *reinterpret_cast<uint32_t*>(&h1);
           v.z = *reinterpret_cast<uint32_t*>(&h2);
           v.w = *reinterpret_cast<uint32_t*>(&h3);
-          *reinterpret_cast<uint4*>(srow + ((j ^ swz) << 4)) = v;
+          *reinterpret_cast<uint4*>(srow + ((jj ^ swz) << 4)) = v;
         }
         fence_proxy_async_smem();
         __syncwarp();
-        if (lane == 0 && any) {
-          const int col = (k >> 1) * 256 + 128 * half + (k & 1) * 64;
-          tma_store_3d(&p.tm_out, stage0 + buf * 4096, col, y, sg.i);
-        }
+        if (lane == 0 && any) tma_store_3d(&p.tm_out, stage0 + k * 4096, col0 + 64 * k, y, sg.i);
         if (lane == 0) bulk_commit_group();
       }
-      if (row_valid && half == 0) p.lse[(static_cast<long long>(sg.i) * p.h_q + hh) * p.s_q + t] = lse_v;
+      if (row_valid && half == 0 && sp == 0) p.lse[(static_cast<long long>(sg.i) * p.h_q + hh) * p.s_q + t] = lse_v;
     } else {
       const bool any = row0 < p.tile_rows;
 #pragma unroll 1
-      for (int k = 0; k < 8; ++k) {  // 32 columns (128 bytes of fp32) per box
+      for (int k = 0; k < 4; ++k) {  // 32 columns (128 bytes of fp32) per box
         float o[32];
         tmem_ld32(t_o + 32 * k, o);
         tmem_wait_ld();
@@ -694,18 +691,16 @@ __device__ void softmax_epilogue(const DecodeParams& p, const Ctx& c, uint32_t t
         }
         uint8_t* srow = stage0_g + buf * 4096 + lane * 128;
 #pragma unroll
-        for (int j = 0; j < 8; ++j)
-          *reinterpret_cast<float4*>(srow + ((j ^ swz) << 4)) =
-              make_float4(o[4 * j] * inv_l, o[4 * j + 1] * inv_l, o[4 * j + 2] * inv_l, o[4 * j + 3] * inv_l);
+        for (int jj = 0; jj < 8; ++jj)
+          *reinterpret_cast<float4*>(srow + ((jj ^ swz) << 4)) =
+              make_float4(o[4 * jj] * inv_l, o[4 * jj + 1] * inv_l, o[4 * jj + 2] * inv_l, o[4 * jj + 3] * inv_l);
         fence_proxy_async_smem();
         __syncwarp();
-        if (lane == 0 && any) {
-          const int col = (k >> 2) * 256 + 128 * half + (k & 3) * 32;
-          tma_store_3d(&p.tm_opart, stage0 + buf * 4096, col, row0, sg.slot);
-        }
+        if (lane == 0 && any) tma_store_3d(&p.tm_opart, stage0 + buf * 4096, col0 + 32 * k, row0, sg.slot);
         if (lane == 0) bulk_commit_group();
       }
-      if (row_valid && half == 0) p.lse_part[static_cast<long long>(sg.slot) * p.tile_rows + q_row] = lse_v;
+      if (row_valid && half == 0 && sp == 0)
+        p.lse_part[static_cast<long long>(sg.slot) * p.tile_rows + q_row] = lse_v;
     }
     tc_fence_before();
     __syncwarp();
@@ -749,14 +744,14 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     }
     for (int k = 0; k < 2; ++k) {
       mbar_init(c.bar(kBarSFull + k), 1);
-      mbar_init(c.bar(kBarSEmpty + k), 8);
-      mbar_init(c.bar(kBarXch + k), 2);
+      mbar_init(c.bar(kBarSEmpty + k), 16);
     }
     mbar_init(c.bar(kBarQFull), 1);
     mbar_init(c.bar(kBarQEmpty), 1);
-    mbar_init(c.bar(kBarOEmpty), 8);
+    mbar_init(c.bar(kBarOEmpty), 16);
+    mbar_init(c.bar(kBarXch), 8);
     mbar_init(c.bar(kBarFinal), 2);
-    mbar_init(c.bar(kBarStageFree), 4);
+    mbar_init(c.bar(kBarStageFree), 8);
     *c.abort_flag = 0u;
     fence_mbar_init_cluster();
   }
