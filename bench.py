@@ -350,6 +350,9 @@ def ours(args, world, rank, local):
         err = binding.mla_check_device_error(m, stream=stream)
         if err:
             raise RuntimeError(f"device error word {err:#x} during warm-up")
+    err = binding.mla_take_device_errors(stream=stream)  # every plan rewrites its metadata word: check the sticky bits
+    if err:
+        raise RuntimeError(f"device error bits {err:#x} during warm-up")
 
     # CUDA graphs: one cycle over all pools (with events around each split-KV
     # kernel) and one single-step graph per pool, so that exactly K steps run.
@@ -421,10 +424,11 @@ def ours(args, world, rank, local):
         stream.synchronize()
         k2_ms = [a.elapsed_time(b) for a, b in ev_pairs]
     k2_avg_ms = sum(k2_ms) / len(k2_ms)
-    for m in metas:
-        err = binding.mla_check_device_error(m, stream=stream)
-        if err:
-            raise RuntimeError(f"device error word {err:#x} in the timed region")
+    # The sticky bits cover every step since warm-up (each plan rewrites the
+    # word in its own metadata, so those only show the last cycle).
+    err = binding.mla_take_device_errors(stream=stream)
+    if err:
+        raise RuntimeError(f"device error bits {err:#x} in the timed region or the kernel timing replays")
 
     # end to end through the API: pinned host inputs in, result out, every step
     e2e_steps = min(K, 500)
@@ -454,6 +458,9 @@ def ours(args, world, rank, local):
             h_lse.copy_(lse, non_blocking=True)
         e1.record(stream)
     stream.synchronize()
+    err = binding.mla_take_device_errors(stream=stream)
+    if err:
+        raise RuntimeError(f"device error bits {err:#x} in the end-to-end steps")
     e2e_ms = max_over_ranks(e0.elapsed_time(e1) / e2e_steps, world, dev)
     h2d = h_q_host.numel() * 2 + h_table.numel() * 4 + h_lens.numel() * 4
     d2h = h_out.numel() * 2 + h_lse.numel() * 4

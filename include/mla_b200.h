@@ -201,6 +201,19 @@ int mla_decode_noalloc(const void* q, const void* kv_cache, int64_t num_pages, c
  */
 int mla_check_device_error(const void* metadata, void* stream, uint32_t* error_word);
 
+/*
+ * The error bits any call raised on the current device since the last
+ * mla_take_device_errors, whatever metadata buffer it used: unlike the word in
+ * `metadata`, which the next mla_get_metadata on that buffer rewrites, these
+ * bits stay set until taken.  For callers that replay many steps (a captured
+ * graph, a benchmark loop) and check once at the end.  Enqueues an atomic
+ * read-and-clear on `stream` (one tiny kernel), synchronises the stream and
+ * writes the bits to *error_word (if not NULL).  Returns MLA_OK when they are
+ * zero, MLA_ERR_DEVICE when not, MLA_ERR_CUDA if the launch, copy or sync
+ * failed.
+ */
+int mla_take_device_errors(void* stream, uint32_t* error_word);
+
 /* Static text for a status code. */
 const char* mla_error_string(int status);
 

@@ -38,6 +38,7 @@ EXPORTED = (
     "mla_decode_timed",
     "mla_decode_noalloc",
     "mla_check_device_error",
+    "mla_take_device_errors",
     "mla_error_string",
 )
 
@@ -77,6 +78,8 @@ def lib() -> ctypes.CDLL:
         L.mla_decode_noalloc.argtypes = dec[:14] + [_vp]
         L.mla_check_device_error.restype = ctypes.c_int
         L.mla_check_device_error.argtypes = [_vp, _vp, ctypes.POINTER(ctypes.c_uint32)]
+        L.mla_take_device_errors.restype = ctypes.c_int
+        L.mla_take_device_errors.argtypes = [_vp, ctypes.POINTER(ctypes.c_uint32)]
         L.mla_error_string.restype = ctypes.c_char_p
         L.mla_error_string.argtypes = [ctypes.c_int]
         _lib = L
@@ -193,6 +196,16 @@ def mla_decode_noalloc(q: torch.Tensor, kv_cache: torch.Tensor, block_table: tor
                                     int(block_table.shape[1]), _ptr(seqlens), batch, s_q, h_q, float(softmax_scale),
                                     int(bool(causal)), _ptr(out), _ptr(lse), _ptr(metadata), _stream_ptr(stream)))
     return out, lse
+
+
+def mla_take_device_errors(stream=None) -> int:
+    """Read and clear the device's sticky error bits (raised by any call
+    since the last take); synchronises the stream."""
+    word = ctypes.c_uint32(0)
+    status = lib().mla_take_device_errors(_stream_ptr(stream), ctypes.byref(word))
+    if status not in (MLA_OK, MLA_ERR_DEVICE):
+        raise MLAError("mla_take_device_errors", status)
+    return int(word.value)
 
 
 def mla_check_device_error(metadata: torch.Tensor, stream=None) -> int:

@@ -110,6 +110,21 @@ int noalloc_scratch(void** out) {
   return MLA_OK;
 }
 
+// The cache as (64 cols, rows, 4 panels, 2 halves of 256 columns) with strides
+// (1152 B, 128 B, 512 B): box (64, 64, 2, 2) at (0, y, 2c, 0) lands as the
+// value tile of CTA c (columns [256h + 128c, +128) of 64 tokens, panels in
+// [h][e] order, 128B-swizzled).
+int encode_value_tiles(PFN_cuTensorMapEncodeTiled_v12000 enc, CUtensorMap* map, const void* base, uint64_t rows) {
+  const cuuint64_t dims[4] = {64, static_cast<cuuint64_t>(rows), 4, 2};
+  const cuuint64_t strides[3] = {static_cast<cuuint64_t>(kDqk) * 2, 128, 512};
+  const cuuint32_t box[4] = {64, static_cast<cuuint32_t>(kPage), 2, 2};
+  const cuuint32_t elem[4] = {1, 1, 1, 1};
+  const CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void*>(base), dims, strides, box, elem,
+                         CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                         CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS ? MLA_OK : MLA_ERR_CUDA;
+}
+
 // A row-major [outer][rows][512] tensor of 2- or 4-byte elements as (512
 // cols, rows, outer), box (128 bytes of columns, 32 rows, 1), 128B swizzle:
 // the TMA-store view of the output and of the split partials.
@@ -160,8 +175,8 @@ int decode_impl(const void* q, const void* kv_cache, int64_t num_pages, const in
   DecodeParams p;
   const uint64_t kv_rows = static_cast<uint64_t>(num_pages) * kPage;
   const uint64_t q_rows = static_cast<uint64_t>(batch) * R;
-  if ((st = encode_panels576(enc, &p.tm_k, kv_cache, kv_rows, kPage / 2, 1)) != MLA_OK ||
-      (st = encode_panels576(enc, &p.tm_v, kv_cache, kv_rows, kPage, 2)) != MLA_OK ||
+  if ((st = encode_panels576(enc, &p.tm_k, kv_cache, kv_rows, kPage, 1)) != MLA_OK ||
+      (st = encode_value_tiles(enc, &p.tm_v, kv_cache, kv_rows)) != MLA_OK ||
       (st = encode_panels576(enc, &p.tm_q, q, q_rows, kMTile / 2, kDqk / 64)) != MLA_OK ||
       (st = encode_store_map(enc, &p.tm_out, out, static_cast<uint64_t>(R), static_cast<uint64_t>(batch), false)) !=
           MLA_OK)
@@ -301,6 +316,16 @@ MLA_API int mla_check_device_error(const void* metadata, void* stream, uint32_t*
   if (cudaMemcpyAsync(&word, static_cast<const int32_t*>(metadata) + kHError, sizeof(word), cudaMemcpyDeviceToHost,
                       s) != cudaSuccess ||
       cudaStreamSynchronize(s) != cudaSuccess) {
+    cudaGetLastError();
+    return MLA_ERR_CUDA;
+  }
+  if (error_word) *error_word = word;
+  return word == 0 ? MLA_OK : MLA_ERR_DEVICE;
+}
+
+MLA_API int mla_take_device_errors(void* stream, uint32_t* error_word) {
+  uint32_t word = 0;
+  if (take_sticky_error(static_cast<cudaStream_t>(stream), &word) != cudaSuccess) {
     cudaGetLastError();
     return MLA_ERR_CUDA;
   }

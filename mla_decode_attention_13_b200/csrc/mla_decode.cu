@@ -19,21 +19,23 @@
 // A tcgen05.mma costs at least ~64 cycles whatever its size, and a pair MMA
 // only reaches the tensor peak at N = 256, so QK^T runs over four pages at a
 // time (a group, 256 tokens); PV runs page by page at N = 256.
-//   * Keys: CTA c supplies tokens [32c, 32c + 32) of each page of the group,
-//     all 576 columns, so a page leaves HBM once for the pair.  They stream
-//     through a ring of panels (64 columns x 128 token rows, 16 KB); a panel
-//     is free again as soon as its four K = 16 MMAs are done.
+//   * Keys: CTA c supplies pages 2c and 2c + 1 of the group, all 64 tokens
+//     and 576 columns, so a page leaves HBM once for the pair.  They stream
+//     through a ring of panels (64 columns x 128 token rows, 16 KB, one TMA
+//     box per page); a panel is free again as soon as its four K = 16 MMAs
+//     are done.
 //   * QK^T: A = Q (64 rows x 576, shared memory, loaded once per segment),
 //     B = the group's panels, N = 256.  S (64 rows x 256 tokens per CTA)
-//     lands in 128 TMEM columns: lane r < 64 holds tokens 0-31 of the four
-//     pages for row r, lane r + 64 tokens 32-63.
+//     lands in 128 TMEM columns: lane r < 64 holds pages 0 and 1 of the group
+//     for row r, lane r + 64 pages 2 and 3.
 //   * Values: for PV, CTA c needs all 64 tokens of a page in its value
 //     columns [256h + 128c, 256h + 128c + 128) (h = 0, 1): a 32 KB tile per
-//     page, read from L2 (the pair has just brought the page in), in a ring
-//     of two.
-//   * Softmax: eight warps; warps 4-7 take pages 0-1 of each group, warps
-//     8-11 pages 2-3.  A thread (TMEM lane r) handles row r mod 64, 64 scores
-//     (32 tokens of each of its two pages); the four threads of a row trade
+//     page (one 4-D TMA box), read from L2 (the pair has just brought the
+//     page in), in a ring of two.
+//   * Softmax: eight warps; warps 4-7 read S columns 0-63, warps 8-11 columns
+//     64-127.  A thread (TMEM lane r) handles row r mod 64 and one page of
+//     the group (all 64 of its tokens), so each row of a P tile comes from a
+//     single thread; the four threads of a row trade
 //     their maxima (and, at the end, their sums) through shared memory.  Online softmax in the log2 domain with a lazy
 //     rescale (the running max only moves when a block's max exceeds it by
 //     more than kTau; O and the running sums are rescaled together, so the
@@ -70,6 +72,16 @@ namespace mla {
 #ifdef MLA_DECODE_TRACE
 __device__ unsigned long long g_mla_trace[4][16][512];  // [traced CTA][event][index]
 __device__ unsigned long long g_mla_span[160][4];  // [pair][start, end, segments, pages] (globaltimer)
+// First wait that ran out of time: [taken, barrier index, parity, thread, block, clock].
+__device__ unsigned long long g_mla_abort[6];
+// Per block and warp: the wait it left on abort (1 << 32 | barrier << 8 | parity)
+// and the role's last loop position.
+__device__ unsigned long long g_mla_stuck[160 * 2][12];
+__device__ unsigned long long g_mla_step[160 * 2][12];
+#define MLA_STEP(v) \
+  do {              \
+    g_mla_step[blockIdx.x][threadIdx.x >> 5] = static_cast<unsigned long long>(v); \
+  } while (0)
 #define MLA_TRACE(ev, k)                                                                         \
   do {                                                                                           \
     const int tr_pair_ = static_cast<int>(blockIdx.x >> 1);                                      \
@@ -80,27 +92,46 @@ __device__ unsigned long long g_mla_span[160][4];  // [pair][start, end, segment
 #define MLA_TRACE(ev, k) \
   do {                   \
   } while (0)
+#define MLA_STEP(v) \
+  do {              \
+  } while (0)
 #endif
+
+// Error bits raised on this device since the host last took them (see
+// mla_take_device_errors): the metadata's error word is rewritten by every
+// plan, this one is only cleared by the host.
+__device__ unsigned int g_mla_sticky_error;
 
 namespace {
 
 using namespace ptx;
 
+__device__ __forceinline__ void set_error(int32_t* meta, uint32_t bits) {
+  atomicOr(reinterpret_cast<unsigned int*>(meta + kHError), bits);
+  atomicOr(&g_mla_sticky_error, bits);
+}
+
 constexpr int kThreads = 384;
 constexpr int kGroup = 4;             // pages per QK group
 constexpr int kKRing = 4;             // key panel slots
 constexpr int kVRing = 2;             // value tiles (and P tiles)
+// PV completion barriers, one per page mod kPvBars.  A parity wait on page k's
+// barrier is only right while the PV of page k - kPvBars is known to be done
+// and that of page k + kPvBars is not; with four, every wait below has that
+// window by construction (a page's writers learn of PV up to three pages
+// before their group from the previous group's writers, through the row
+// exchange).
+constexpr int kPvBars = 4;
 constexpr float kTau = 8.0f;          // lazy-rescale threshold, log2 units
 constexpr uint64_t kTimeoutNs = 500ull * 1000ull * 1000ull;
 constexpr int kRowsCta = kMTile / 2;  // 64 query rows per CTA
-constexpr int kHalfPage = kPage / 2;  // 32 tokens of a page per CTA
 
 // Shared-memory layout (offsets from a 1024-byte aligned base).  All operand
 // tiles are 128-byte swizzled panels of 64 bf16 columns.
 constexpr uint32_t kQPanel = kRowsCta * 128;            // 64 rows x 64 cols
 constexpr uint32_t kQBytes = 9 * kQPanel;               // 64 query rows x 576 cols
-constexpr uint32_t kHalfPageBytes = kHalfPage * 128;    // 32 token rows x 64 cols
-constexpr uint32_t kKSlot = kGroup * kHalfPageBytes;    // one panel of a group: 128 token rows
+constexpr uint32_t kPagePanel = kPage * 128;            // 64 token rows x 64 cols
+constexpr uint32_t kKSlot = 2 * kPagePanel;             // one panel of a CTA's two pages: 128 token rows
 constexpr uint32_t kVPanel = kPage * 128;               // 64 tokens x 64 cols
 constexpr uint32_t kVTile = 4 * kVPanel;                // 64 tokens x this CTA's 256 value cols
 constexpr uint32_t kPTile = kRowsCta * 128;             // 64 rows x 64 tokens bf16
@@ -112,12 +143,12 @@ constexpr uint32_t kOffX = kOffP + kVRing * kPTile;     // float [2][256] row ex
 constexpr uint32_t kOffBar = kOffX + 2 * 256 * 4;
 
 enum Bar : uint32_t {
-  kBarKFull = 0,                       // [kKRing] (leader) both CTAs' key panel landed
+  kBarKFull = 0,                       // [kKRing] (leader) both CTAs' key panel landed (2 arrivals + bytes)
   kBarKEmpty = kBarKFull + kKRing,     // [kKRing] (both) the panel's QK MMAs are done
   kBarVFull = kBarKEmpty + kKRing,     // [kVRing] (both, local) this CTA's value tile landed
-  kBarPFull = kBarVFull + kVRing,      // [kVRing] (leader) P written by both CTAs' 4 softmax warps
-  kBarPvDone = kBarPFull + kVRing,     // [kVRing] (both) PV of that page done: P and value tiles free
-  kBarSFull = kBarPvDone + kVRing,     // [2] (both) S buffer written
+  kBarPFull = kBarVFull + kVRing,      // [kVRing] (leader) P written by both CTAs' 2 softmax warps of the page
+  kBarPvDone = kBarPFull + kVRing,     // [kPvBars] (both) PV of page k (mod kPvBars) done: its P and value tiles free
+  kBarSFull = kBarPvDone + kPvBars,    // [2] (both) S buffer written
   kBarSEmpty = kBarSFull + 2,          // [2] (leader) both CTAs' softmax warps read the S buffer
   kBarQFull = kBarSEmpty + 2,          // (leader) both CTAs' Q rows landed
   kBarQEmpty = kBarQFull + 1,          // (both) last QK of the segment done
@@ -125,7 +156,8 @@ enum Bar : uint32_t {
   kBarFinal = kBarOEmpty + 1,          // (leader) MMA drain at teardown: both issuer threads
   kBarXch = kBarFinal + 1,             // (both) the 8 softmax warps published row values
   kBarStageFree = kBarXch + 1,         // (both, local) the epilogue's stores have read their staging
-  kNumBars = kBarStageFree + 1,
+  kBarResc = kBarStageFree + 1,        // [2] (both, local) the 4 warps of rows 32k..32k+31 rescaled O
+  kNumBars = kBarResc + 2,
 };
 constexpr uint32_t kOffTmemSlot = kOffBar + 8 * kNumBars;  // u32
 constexpr uint32_t kOffAbort = kOffTmemSlot + 4;           // u32
@@ -158,7 +190,7 @@ struct Ctx {
 };
 
 __device__ void raise_abort(const Ctx& c, uint32_t err_bits) {
-  if (err_bits) atomicOr(reinterpret_cast<unsigned int*>(c.meta + kHError), err_bits);
+  if (err_bits) set_error(c.meta, err_bits);
   *c.abort_flag = 1u;
   st_cluster_u32(c.peer_abort, 1u);
 }
@@ -171,11 +203,26 @@ __device__ bool wait_bar(const Ctx& c, uint32_t bar, uint32_t parity) {
   while (true) {
     if (mbar_try_wait(bar, parity)) return true;
     if ((++spins & 63u) == 0) {
-      if (*c.abort_flag) return false;
+      if (*c.abort_flag) {
+#ifdef MLA_DECODE_TRACE
+        g_mla_stuck[blockIdx.x][threadIdx.x >> 5] =
+            (1ull << 32) | (static_cast<unsigned long long>((bar - c.base - kOffBar) / 8) << 8) | parity;
+#endif
+        return false;
+      }
       const uint64_t now = globaltimer();
       if (t0 == 0) {
         t0 = now;
       } else if (now - t0 > kTimeoutNs) {
+#ifdef MLA_DECODE_TRACE
+        if (atomicCAS(&g_mla_abort[0], 0ull, 1ull) == 0ull) {
+          g_mla_abort[1] = (bar - c.base - kOffBar) / 8;
+          g_mla_abort[2] = parity;
+          g_mla_abort[3] = threadIdx.x;
+          g_mla_abort[4] = blockIdx.x;
+          g_mla_abort[5] = clock64();
+        }
+#endif
         raise_abort(c, MLA_DEVERR_TIMEOUT);
         return false;
       }
@@ -227,7 +274,7 @@ __device__ __forceinline__ int load_page(const DecodeParams& p, const Ctx& c, co
   if (blk >= end) return 0;
   int page = table[blk];
   if (page < 0 || page >= p.num_pages) {
-    atomicOr(reinterpret_cast<unsigned int*>(c.meta + kHError), MLA_DEVERR_PAGE);
+    set_error(c.meta, MLA_DEVERR_PAGE);
     page = 0;  // keep the copy inside the pool; the result is flagged
   }
   return page;
@@ -279,9 +326,9 @@ __device__ __forceinline__ void walk_groups(const DecodeParams& p, const Ctx& c,
 }
 
 // ------------------------------------------------------------- producers --
-// Warp 0: each segment's Q rows of this CTA, then this CTA's key half of the
-// group's pages, panel by panel, into the key ring (bytes complete on the
-// leader's barriers).
+// Warp 0: each segment's Q rows of this CTA, then this CTA's two pages of
+// the group (pages 2c and 2c + 1, those that exist), panel by panel, into the
+// key ring (bytes complete on the leader's barriers).
 __device__ void producer_k(const DecodeParams& p, const Ctx& c, int s_begin, int s_end) {
   const int lane = threadIdx.x & 31;
   uint32_t gi = 0, seg_it = 0, ks = 0;  // groups, segments started, key panels loaded
@@ -309,10 +356,20 @@ __device__ void producer_k(const DecodeParams& p, const Ctx& c, int s_begin, int
         if (ks >= kKRing) good = wait_bar(c, c.bar(kBarKEmpty + slot), ((ks / kKRing) - 1) & 1);
         if (good) {
           MLA_TRACE(10, ks);
-          if (c.cta == 0) mbar_arrive_expect_tx(c.bar(kBarKFull + slot), 2 * gr.np * kHalfPageBytes);
-          for (int q = 0; q < gr.np; ++q)
-            tma_load_3d_pair(c.kslot(slot) + q * kHalfPageBytes, &p.tm_k, c.lead_bar(kBarKFull + slot), 0,
-                             gr.page[q] * kPage + static_cast<int>(c.cta) * kHalfPage, pn);
+          MLA_STEP(ks);
+          if (c.cta == 0) mbar_arrive_expect_tx(c.bar(kBarKFull + slot), gr.np * kPagePanel);
+#pragma unroll
+          for (int q = 0; q < 2; ++q) {
+            const int gq = 2 * static_cast<int>(c.cta) + q;
+            if (gq < gr.np)
+              tma_load_3d_pair(c.kslot(slot) + q * kPagePanel, &p.tm_k, c.lead_bar(kBarKFull + slot), 0,
+                               gr.page[gq] * kPage, pn);
+          }
+          // The other CTA also arrives, even when it has no page in the group:
+          // otherwise the slot could fill and drain without it, and its
+          // parity wait on the slot's empty barrier would fall two phases
+          // behind.
+          if (c.cta != 0) mbar_arrive_remote(c.lead_bar(kBarKFull + slot));
         }
       }
     }
@@ -336,15 +393,16 @@ __device__ void producer_v(const DecodeParams& p, const Ctx& c, int s_begin, int
       if (gr.first && seg_it > 0) good = wait_bar(c, c.bar(kBarStageFree), (seg_it - 1) & 1);
       for (int q = 0; q < gr.np && good; ++q, ++ps) {
         const uint32_t slot = ps % kVRing;
-        if (ps >= kVRing) good = wait_bar(c, c.bar(kBarPvDone + slot), ((ps - kVRing) / kVRing) & 1);
+        if (ps >= kVRing) {
+          const uint32_t k = ps - kVRing;  // the tile's previous page: its PV must be done
+          good = wait_bar(c, c.bar(kBarPvDone + k % kPvBars), (k / kPvBars) & 1);
+        }
         if (good) {
           MLA_TRACE(3, ps);
+          MLA_STEP(ps);
           const uint32_t bar = c.bar(kBarVFull + slot);
           mbar_arrive_expect_tx(bar, kVTile);
-#pragma unroll
-          for (int h = 0; h < 2; ++h)
-            tma_load_3d(c.vtile(slot) + h * 2 * kVPanel, &p.tm_v, bar, 0, gr.page[q] * kPage,
-                        4 * h + 2 * static_cast<int>(c.cta));
+          tma_load_4d(c.vtile(slot), &p.tm_v, bar, 0, gr.page[q] * kPage, 2 * static_cast<int>(c.cta), 0);
         }
       }
     }
@@ -408,6 +466,7 @@ __device__ void qk_issuer(const DecodeParams& p, const Ctx& c, uint32_t tmem, in
         const uint32_t slot = ks % kKRing;
         if (!wait_bar(c, c.bar(kBarKFull + slot), (ks / kKRing) & 1)) return;
         MLA_TRACE(9, ks);
+        MLA_STEP(ks);
         tc_fence_after();
         issue_qk_panel(c, tmem, slot, pn, sb);
         umma_commit_pair(c.bar(kBarKEmpty + slot), both);
@@ -431,9 +490,10 @@ __device__ void pv_issuer(const DecodeParams& p, const Ctx& c, uint32_t tmem, in
       if (!wait_bar(c, c.bar(kBarPFull + slot), (pg / kVRing) & 1)) return;
       if (jp == 0 && seg_it > 0 && !wait_bar(c, c.bar(kBarOEmpty), (seg_it - 1) & 1)) return;
       MLA_TRACE(2, pg);
+      MLA_STEP(pg);
       tc_fence_after();
       issue_pv_page(c, tmem, slot, jp == 0);
-      umma_commit_pair(c.bar(kBarPvDone + slot), both);
+      umma_commit_pair(c.bar(kBarPvDone + pg % kPvBars), both);
     }
     ++seg_it;
   }
@@ -482,23 +542,27 @@ __device__ __forceinline__ float exp_pack(const float (&sv)[32], int nvalid, flo
 
 __device__ void softmax_epilogue(const DecodeParams& p, const Ctx& c, uint32_t tmem, int s_begin, int s_end) {
   const int r = threadIdx.x - 128;  // 0-255: softmax thread
-  const int sp = r >> 7;            // page pair: pages 2 sp, 2 sp + 1 of each group (S columns 64 sp ..)
+  const int sp = r >> 7;            // S columns 64 sp .. 64 sp + 63 of each lane
   const int rr = r & 127;           // TMEM lane
   const int lane = threadIdx.x & 31;
   const int hr = rr & (kRowsCta - 1);  // query row within this CTA
-  const int half = rr >> 6;            // 0: tokens 0-31 of each page / first column half; 1: the rest
+  const int half = rr >> 6;            // 0: pages 0-1 of each group / first O column half; 1: the rest
+  const int q = 2 * half + sp;         // this thread's page of each group
   const uint32_t lane_off = static_cast<uint32_t>(rr & ~31) << 16;
   const uint32_t t_s = tmem + lane_off + kColS + 64 * sp;
   const uint32_t t_o = tmem + lane_off + kColO + 128 * sp;  // this thread's 128 O columns
   float* xbuf = reinterpret_cast<float*>(c.gbase + kOffX);
-  // This thread's 32 weights of a page: 64 bytes of P row hr, 16-byte chunks
-  // 4 half .. 4 half + 3, swizzled by the row.
+  // This thread's 64 weights of a page: row hr of the P tile (128 bytes,
+  // 16-byte chunks swizzled by the row).
   const uint32_t prow_off = (hr >> 3) * 1024 + (hr & 7) * 128;
   const float sl2 = p.scale_log2;
   // gi: groups, ps: pages before the current group (select buffers and
-  // phases); x_cnt: row exchanges among the row's four threads.
-  uint32_t gi = 0, ps = 0, x_cnt = 0;
-  auto pv_done = [&](uint32_t k) -> bool { return wait_bar(c, c.bar(kBarPvDone + k % kVRing), (k / kVRing) & 1); };
+  // phases); x_cnt: row exchanges among the row's four threads; n_resc: O
+  // rescales of this warp's rows (the four warps holding rows 32 kr ..
+  // 32 kr + 31 take the same decisions, so they count alike).
+  uint32_t gi = 0, ps = 0, x_cnt = 0, n_resc = 0;
+  const int kr = (rr >> 5) & 1;
+  auto pv_done = [&](uint32_t k) -> bool { return wait_bar(c, c.bar(kBarPvDone + k % kPvBars), (k / kPvBars) & 1); };
   // Publish v for the other three threads of this row (the other half of its
   // tokens, the other page pair) and return the max or the sum of the four;
   // the eight softmax warps meet on an mbarrier (bounded wait).
@@ -517,7 +581,7 @@ __device__ void softmax_epilogue(const DecodeParams& p, const Ctx& c, uint32_t t
   for (int s = s_begin; s < s_end; ++s) {
     const Segment sg = load_segment(p, s);
     if (sg.bad) {
-      if (r == 0 && c.cta == 0) atomicOr(reinterpret_cast<unsigned int*>(c.meta + kHError), MLA_DEVERR_SEQLEN);
+      if (r == 0 && c.cta == 0) set_error(c.meta, MLA_DEVERR_SEQLEN);
       continue;
     }
     const int n = sg.b1 - sg.b0;
@@ -534,12 +598,15 @@ __device__ void softmax_epilogue(const DecodeParams& p, const Ctx& c, uint32_t t
     const int last_page = ceil_div(sg.L, kPage) - 1;
 
     float m = -INFINITY, l = 0.0f;  // l: this thread's share of the row sum
+    int np_last = 0;                // pages in the segment's last group
     for (int j = 0; j < n; j += kGroup, ++gi) {
       const int blk = sg.b0 + j;
       const int np = min(kGroup, n - j);
+      np_last = np;
       const uint32_t sb = gi & 1;
       if (!wait_bar(c, c.bar(kBarSFull + sb), (gi >> 1) & 1)) return;
       if (r == 0) MLA_TRACE(4, gi);
+      MLA_STEP((1ull << 40) | (static_cast<unsigned long long>(gi) << 20) | ps);
       tc_fence_after();
       float sv[2][32];
       tmem_ld32(t_s + 128 * sb, sv[0]);
@@ -549,13 +616,12 @@ __device__ void softmax_epilogue(const DecodeParams& p, const Ctx& c, uint32_t t
       __syncwarp();
       if (lane == 0) arrive_leader(c, kBarSEmpty + sb);  // S buffer read
 
-      // ---- mask; max over the group's pages and both halves of the row ----
+      // ---- mask; max over the group's four pages ----
       int nv[2];
       float mx = -INFINITY;
 #pragma unroll
       for (int e = 0; e < 2; ++e) {
-        const int q = 2 * sp + e;
-        const int v = limit - (blk + q) * kPage - kHalfPage * half;
+        const int v = limit - (blk + q) * kPage - 32 * e;
         nv[e] = (q >= np || v < 0) ? 0 : (v > 32 ? 32 : v);
         mx = fmaxf(mx, masked_max(sv[e], nv[e]));
       }
@@ -568,8 +634,11 @@ __device__ void softmax_epilogue(const DecodeParams& p, const Ctx& c, uint32_t t
       const float neg_m = (m_new == -INFINITY) ? 0.0f : -m_new;
 
       // ---- rescale this thread's O columns (rare): after PV of every earlier
-      //      page of the segment ----
-      if (j > 0 && __any_sync(0xffffffffu, alpha < 1.0f)) {
+      //      page of the segment, and before PV of this group's first page,
+      //      whose P writers wait on the row half's rescale barrier ----
+      const bool resc = j > 0 && __any_sync(0xffffffffu, alpha < 1.0f);
+      if (resc) {
+        MLA_STEP((5ull << 40) | ps);
         if (!pv_done(ps - 1)) return;
         tc_fence_after();
 #pragma unroll 1
@@ -582,59 +651,71 @@ __device__ void softmax_epilogue(const DecodeParams& p, const Ctx& c, uint32_t t
           tmem_st32(t_o + cc, o);
         }
         tmem_wait_st();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(c.bar(kBarResc + kr));
+        ++n_resc;
+        MLA_STEP((6ull << 40) | n_resc);
       }
 
       float lsum = 0.0f;
-#pragma unroll
-      for (int e = 0; e < 2; ++e) {
-        const int q = 2 * sp + e;
-        if (q >= np) break;
+      if (q < np) {
         const uint32_t pg = ps + q;  // global page index
-        uint32_t packed[16];
-        lsum += exp_pack(sv[e], nv[e], sl2, neg_m, packed);
+        uint32_t packed[2][16];
+        lsum = exp_pack(sv[0], nv[0], sl2, neg_m, packed[0]) + exp_pack(sv[1], nv[1], sl2, neg_m, packed[1]);
         const uint32_t slot = pg % kVRing;
         // ---- P tile free (PV two pages back) ----
         if (pg >= kVRing && !pv_done(pg - kVRing)) return;
-        if (r == 0 || r == 128) MLA_TRACE(6, pg);
+        MLA_STEP((2ull << 40) | pg);
+        if (rr == 0) MLA_TRACE(6, pg);
         {
           uint8_t* prow = c.gbase + kOffP + slot * kPTile + prow_off;
 #pragma unroll
-          for (int ci = 0; ci < 4; ++ci)
-            *reinterpret_cast<uint4*>(prow + (((4 * half + ci) ^ (hr & 7)) << 4)) =
-                make_uint4(packed[4 * ci], packed[4 * ci + 1], packed[4 * ci + 2], packed[4 * ci + 3]);
+          for (int ci = 0; ci < 8; ++ci)
+            *reinterpret_cast<uint4*>(prow + ((ci ^ (hr & 7)) << 4)) =
+                make_uint4(packed[ci >> 2][4 * (ci & 3)], packed[ci >> 2][4 * (ci & 3) + 1],
+                           packed[ci >> 2][4 * (ci & 3) + 2], packed[ci >> 2][4 * (ci & 3) + 3]);
         }
         // ---- this CTA's value tile has landed; the last page of a row may
         //      hold garbage (even NaN) past L: zero the value rows there, so
         //      that 0 * garbage cannot reach O ----
         if (!wait_bar(c, c.bar(kBarVFull + slot), (pg / kVRing) & 1)) return;
-        if (r == 0 || r == 128) MLA_TRACE(7, pg);
+        MLA_STEP((3ull << 40) | pg);
+        if (rr == 0) MLA_TRACE(7, pg);
         if (blk + q == last_page && (sg.L & (kPage - 1))) {
           const int first_bad = sg.L - last_page * kPage;
           const int chunks = (kPage - first_bad) * 4 * 8;  // tokens x panels x 16-byte chunks
           uint8_t* vt = c.gbase + kOffV + slot * kVTile;
-          for (int e2 = rr; e2 < chunks; e2 += 128) {
+          for (int e2 = hr; e2 < chunks; e2 += kRowsCta) {
             const int tok = first_bad + (e2 >> 5);
             *reinterpret_cast<uint4*>(vt + ((e2 >> 3) & 3) * kVPanel + tok * 128 + (e2 & 7) * 16) =
                 make_uint4(0, 0, 0, 0);
           }
         }
+        // The group's first PV adds to O: every warp of these rows must have
+        // rescaled its O columns first.
+        if (resc && q == 0 && !wait_bar(c, c.bar(kBarResc + kr), (n_resc - 1) & 1)) return;
         fence_proxy_async_smem();
         tc_fence_before();
         __syncwarp();
         if (lane == 0) arrive_leader(c, kBarPFull + slot);
-        if (r == 0 || r == 128) MLA_TRACE(8, pg);
+        MLA_STEP((4ull << 40) | pg);
+        if (rr == 0) MLA_TRACE(8, pg);
       }
       l = l * alpha + lsum;
       m = m_new;
       ps += np;
     }
 
-    // ---- epilogue ----
-    if (!pv_done(ps - 1)) return;
+    // ---- epilogue: the writers of the last page (whose own P-slot wait
+    //      makes this parity wait exact) wait for its PV; the row exchange
+    //      then orders everyone's O reads after it ----
+    MLA_STEP((7ull << 40) | ps);
+    if (q == np_last - 1 && !pv_done(ps - 1)) return;
     if (r == 0) MLA_TRACE(12, s - s_begin);
-    tc_fence_after();
     float lt;
     if (!trade(l, true, &lt)) return;
+    tc_fence_after();
     const float inv_l = lt > 0.0f ? 1.0f / lt : 0.0f;
     const float lse_v = lt > 0.0f ? (m + __log2f(lt)) * 0.69314718055994530942f : -INFINITY;
     // Output through TMA stores: each warp stages its 32 rows x 128 bytes of
@@ -734,14 +815,14 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     // Barriers of the leader's pipeline are only used in the leader, the
     // rest in both CTAs; initialise all of them everywhere.
     for (int k = 0; k < kKRing; ++k) {
-      mbar_init(c.bar(kBarKFull + k), 1);
+      mbar_init(c.bar(kBarKFull + k), 2);
       mbar_init(c.bar(kBarKEmpty + k), 1);
     }
     for (int k = 0; k < kVRing; ++k) {
       mbar_init(c.bar(kBarVFull + k), 1);
-      mbar_init(c.bar(kBarPFull + k), 8);
-      mbar_init(c.bar(kBarPvDone + k), 1);
+      mbar_init(c.bar(kBarPFull + k), 4);
     }
+    for (int k = 0; k < kPvBars; ++k) mbar_init(c.bar(kBarPvDone + k), 1);
     for (int k = 0; k < 2; ++k) {
       mbar_init(c.bar(kBarSFull + k), 1);
       mbar_init(c.bar(kBarSEmpty + k), 16);
@@ -752,6 +833,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     mbar_init(c.bar(kBarXch), 8);
     mbar_init(c.bar(kBarFinal), 2);
     mbar_init(c.bar(kBarStageFree), 8);
+    mbar_init(c.bar(kBarResc), 4);
+    mbar_init(c.bar(kBarResc + 1), 4);
     *c.abort_flag = 0u;
     fence_mbar_init_cluster();
   }
@@ -788,8 +871,12 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     const MetaLayout lo = meta_layout(p.batch, p.h_q, p.s_q);
     s_begin = p.meta[lo.pair_off + pair];
     s_end = p.meta[lo.pair_off + pair + 1];
+    // Bits the plan raised (lengths past the table, slot overflow) go to the
+    // sticky word too.
+    if (threadIdx.x == 0 && c.cta == 0 && pair == 0 && p.meta[kHError] != 0)
+      atomicOr(&g_mla_sticky_error, static_cast<unsigned int>(p.meta[kHError]));
   } else if (threadIdx.x == 0 && c.cta == 0 && pair == 0) {
-    atomicOr(reinterpret_cast<unsigned int*>(c.meta + kHError), MLA_DEVERR_PLAN);
+    set_error(c.meta, MLA_DEVERR_PLAN);
   }
 
   if (threadIdx.x == 128) MLA_TRACE(11, 0);
@@ -847,6 +934,14 @@ extern "C" __attribute__((visibility("default"))) int mla_trace_read(void* host)
 extern "C" __attribute__((visibility("default"))) int mla_trace_span(void* host) {
   return static_cast<int>(cudaMemcpyFromSymbol(host, g_mla_span, sizeof(g_mla_span)));
 }
+extern "C" __attribute__((visibility("default"))) int mla_trace_abort(void* host) {
+  return static_cast<int>(cudaMemcpyFromSymbol(host, g_mla_abort, sizeof(g_mla_abort)));
+}
+extern "C" __attribute__((visibility("default"))) int mla_trace_stuck(void* stuck, void* step) {
+  cudaError_t e = cudaMemcpyFromSymbol(stuck, g_mla_stuck, sizeof(g_mla_stuck));
+  if (e == cudaSuccess) e = cudaMemcpyFromSymbol(step, g_mla_step, sizeof(g_mla_step));
+  return static_cast<int>(e);
+}
 extern "C" __attribute__((visibility("default"))) int mla_trace_clear() {
   static unsigned long long zero[4][16][512];
   return static_cast<int>(cudaMemcpyToSymbol(g_mla_trace, zero, sizeof(zero)));
@@ -854,6 +949,19 @@ extern "C" __attribute__((visibility("default"))) int mla_trace_clear() {
 #endif
 
 size_t decode_kernel_smem_bytes() { return kSmemBytes; }
+
+__device__ unsigned int g_mla_sticky_taken;
+
+__global__ void take_sticky_kernel() { g_mla_sticky_taken = atomicExch(&g_mla_sticky_error, 0u); }
+
+cudaError_t take_sticky_error(cudaStream_t stream, uint32_t* word) {
+  take_sticky_kernel<<<1, 1, 0, stream>>>();
+  cudaError_t e = cudaGetLastError();
+  if (e == cudaSuccess)
+    e = cudaMemcpyFromSymbolAsync(word, g_mla_sticky_taken, sizeof(unsigned int), 0, cudaMemcpyDeviceToHost, stream);
+  if (e == cudaSuccess) e = cudaStreamSynchronize(stream);
+  return e;
+}
 
 cudaError_t decode_kernel_prepare() {
   return cudaFuncSetAttribute(mla_decode_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,

@@ -96,8 +96,11 @@ struct DecodeParams {
   // All three view a [rows][576] bf16 tensor as (64 cols, rows, 9 panels),
   // strides (1152 B, 128 B), so that a 3-D box lands as panels of 64
   // columns x box rows, 128B-swizzled.
-  CUtensorMap tm_k;  // cache: box (64, 32, 1), one panel of a page's 32 key tokens
-  CUtensorMap tm_v;  // cache: box (64, 64, 2), two value panels of a page's 64 tokens
+  CUtensorMap tm_k;  // cache: box (64, 64, 1), one panel of a page's 64 tokens
+  // cache as (64 cols, rows, 4 panels of a 256-column half, 2 halves), strides
+  // (1152 B, 128 B, 512 B): box (64, 64, 2, 2) is one CTA's value tile of a
+  // page (its 128 columns of each half), panels in [half][panel] order.
+  CUtensorMap tm_v;
   CUtensorMap tm_q;  // q: box (64, 64, 9), 64 query rows
   // Stores, with 128B swizzle: out as (512 cols, R rows, batch), box (64,
   // 32, 1) bf16; o_part as (512 cols, tile_rows, max_slots), box (32, 32, 1)
@@ -134,6 +137,8 @@ cudaError_t launch_sched(const int32_t* seqlens, int batch, int h_q, int s_q, in
 cudaError_t decode_kernel_prepare();
 cudaError_t decode_kernel_pairs(int* pairs);
 size_t decode_kernel_smem_bytes();
+// Reads and clears (atomically, on `stream`) the device's sticky error bits.
+cudaError_t take_sticky_error(cudaStream_t stream, uint32_t* word);
 cudaError_t launch_decode(const DecodeParams& p, int pairs, cudaStream_t stream);
 cudaError_t launch_combine(const CombineParams& p, int grid, cudaStream_t stream);
 

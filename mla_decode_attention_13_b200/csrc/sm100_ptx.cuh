@@ -128,6 +128,17 @@ __device__ __forceinline__ void tma_load_3d(uint32_t dst, const CUtensorMap* m, 
       : "memory");
 }
 
+// 4-D tiled bulk copy global -> this CTA's shared memory, completing its
+// bytes on `bar` (a barrier of this CTA).  x is 0 for every caller.
+__device__ __forceinline__ void tma_load_4d(uint32_t dst, const CUtensorMap* m, uint32_t bar, int32_t x, int32_t y,
+                                            int32_t z, int32_t w) {
+  asm volatile(
+      "cp.async.bulk.tensor.4d.shared::cluster.global.tile.mbarrier::complete_tx::bytes [%0], [%1, {%3, %4, %5, "
+      "%6}], [%2];" ::"r"(dst),
+      "l"(reinterpret_cast<uint64_t>(m)), "r"(bar), "r"(x), "r"(y), "r"(z), "r"(w)
+      : "memory");
+}
+
 // 3-D tiled load into this CTA's shared memory whose byte count completes on
 // `bar_cluster`, a barrier that may sit in either CTA of the 2-CTA pair
 // (shared::cluster address): both CTAs' halves of an MMA operand signal the

@@ -203,6 +203,22 @@ def test_increasing_scores_exercise_rescale():
     assert_parity(x, out, lse)
 
 
+@pytest.mark.parametrize("slope,h_q,s_q,causal", [(0.2, 128, 2, True), (0.05, 128, 1, False), (0.2, 64, 1, False)])
+def test_steep_score_ramp_rescales_every_group(slope, h_q, s_q, causal):
+    # With a per-token score increase of slope * 4 * softmax_scale, the running
+    # max of a 256-token group rises by 5-21 log2 units, so the lazy rescale
+    # (threshold 8) fires at almost every group; long rows are also split
+    # across SM pairs, and the row lengths leave ragged last groups.
+    lens = [9000, 2500, 700, 130]
+    x = inputs.make_inputs(lens, h_q, s_q, seed=710, causal=causal)
+    x.q[..., 512] = 4.0
+    for i, n in enumerate(lens):
+        for j in range(0, n):
+            x.kv_cache[int(x.block_table[i, j // 64]), j % 64, 0, 512] = slope * j
+    out, lse, _ = run(x)
+    assert_parity(x, out, lse)
+
+
 def test_peaked_softmax():
     x = inputs.make_inputs([500, 64], 32, seed=800, softmax_scale=1.0)
     out, lse, _ = run(x)
