@@ -30,8 +30,6 @@ constexpr uint32_t kMagic = 0x314C4D42u;  // "BML1"
 //   row_info  [W][2]                    (first slot or -1, pieces)
 //   split_rows [W]                      work rows cut into >1 pieces
 //   empty_rows [W]                      work rows with no pages
-//   scratch   [W][4]                    plan construction: end cost (int64),
-//                                       first segment, first pair
 // A work row is (batch row i, m-tile mt) with index w = mt * batch + i.
 // ---------------------------------------------------------------------------
 enum HeaderWord : int {
@@ -55,7 +53,7 @@ enum HeaderWord : int {
 
 struct MetaLayout {
   int W;
-  size_t pair_off, segs, row_info, split_rows, empty_rows, scratch, words;
+  size_t pair_off, segs, row_info, split_rows, empty_rows, words;
 };
 
 __host__ __device__ inline int ceil_div(int a, int b) { return (a + b - 1) / b; }
@@ -68,8 +66,7 @@ __host__ __device__ inline MetaLayout meta_layout(int batch, int h_q, int s_q) {
   L.row_info = L.segs + size_t(4) * (L.W + kMaxPairs);
   L.split_rows = L.row_info + size_t(2) * L.W;
   L.empty_rows = L.split_rows + L.W;
-  L.scratch = (L.empty_rows + L.W + 1) & ~size_t(1);  // 8-byte aligned
-  L.words = L.scratch + size_t(4) * L.W;
+  L.words = L.empty_rows + L.W;
   return L;
 }
 

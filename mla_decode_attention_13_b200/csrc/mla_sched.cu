@@ -20,7 +20,8 @@
 //   * a row whose pages land on k > 1 pairs is cut into k pieces with k
 //     consecutive partial slots (row order); its output comes from the combine.
 // Everything follows from prefix sums, so one CTA computes it with block-wide
-// scans over chunks of 1024 rows and one binary search per pair.
+// scans over chunks of 1024 rows (one pass when the rows fit one chunk); each
+// row also writes the start offset of every pair whose range begins inside it.
 #include "mla_internal.h"
 #include "sm100_ptx.cuh"
 
@@ -85,54 +86,73 @@ __global__ void __launch_bounds__(kSchedThreads) mla_sched_kernel(const int32_t*
   int32_t* row_info = meta + lo.row_info;
   int32_t* split_rows = meta + lo.split_rows;
   int32_t* empty_rows = meta + lo.empty_rows;
-  long long* end_cost = reinterpret_cast<long long*>(meta + lo.scratch);  // [W]
-  int32_t* first_seg = meta + lo.scratch + 2 * W;                         // [W]
-  int32_t* first_pair = meta + lo.scratch + 3 * W;                        // [W]
 
   __shared__ long long s_wl[kWarps];
-  __shared__ int s_wi[kWarps];
+  __shared__ unsigned long long s_wp[kWarps];
   __shared__ long long s_tot_l;
-  __shared__ int s_tot_i;
+  __shared__ unsigned long long s_tot_p;
   __shared__ int s_err;
   if (threadIdx.x == 0) s_err = 0;
-  __syncthreads();
   int err = 0;
+  const bool one_chunk = W <= kSchedThreads;
 
-  // Pass 1: total cost T.
-  long long local = 0;
-  for (int w = threadIdx.x; w < W; w += kSchedThreads) {
-    const int n = row_pages(seqlens, batch, w, &err);
-    if (n > 0) local += n + kKappa;
+  // Pass 1: total cost T.  With at most one row per thread, the row's pages
+  // and cost prefix are kept for pass 2 instead of being read and scanned
+  // again.
+  int n_own = 0;
+  long long C_own = 0, T = 0;
+  if (one_chunk) {
+    n_own = threadIdx.x < W ? row_pages(seqlens, batch, threadIdx.x, &err) : 0;
+    C_own = block_exclusive_scan<long long>(n_own > 0 ? n_own + kKappa : 0, s_wl, &s_tot_l);
+    T = s_tot_l;
+  } else {
+    long long local = 0;
+    for (int w = threadIdx.x; w < W; w += kSchedThreads) {
+      const int n = row_pages(seqlens, batch, w, &err);
+      if (n > 0) local += n + kKappa;
+    }
+    block_exclusive_scan<long long>(local, s_wl, &s_tot_l);
+    T = s_tot_l;
   }
-  block_exclusive_scan<long long>(local, s_wl, &s_tot_l);
-  const long long T = s_tot_l;
   const long long cap = T > 0 ? (T + pairs - 1) / pairs : 1;
 
-  // Pass 2: per-row prefix sums (cost, segments, slots, split and empty
-  // lists), chunk by chunk with carries.
+  // Pass 2: per-row prefix sums, chunk by chunk with carries.  The four
+  // counts (segments, partial slots, split rows, empty rows) are scanned
+  // together as 16-bit fields of one 64-bit word: within a chunk of 1024 rows
+  // each stays below 1024 + pairs.
   long long carry_cost = 0;
   int carry_seg = 0, carry_slot = 0, carry_split = 0, carry_empty = 0;
   for (int base = 0; base < W; base += kSchedThreads) {
     const int w = base + threadIdx.x;
     const bool in = w < W;
-    const int n = in ? row_pages(seqlens, batch, w, &err) : 0;
+    int n;
+    long long C, chunk_cost;
+    if (one_chunk) {
+      n = n_own;
+      C = C_own;
+      chunk_cost = T;
+    } else {
+      n = in ? row_pages(seqlens, batch, w, &err) : 0;
+      C = carry_cost + block_exclusive_scan<long long>(n > 0 ? n + kKappa : 0, s_wl, &s_tot_l);
+      chunk_cost = s_tot_l;
+    }
     const long long c = n > 0 ? n + kKappa : 0;
-    const long long C = carry_cost + block_exclusive_scan<long long>(c, s_wl, &s_tot_l);
-    const long long chunk_cost = s_tot_l;
     int f = 0, pieces = 0;
     if (n > 0) {
       f = static_cast<int>((C + kKappa) / cap);
       const int l = static_cast<int>((C + kKappa + n - 1) / cap);
       pieces = l - f + 1;
     }
-    const int seg0 = carry_seg + block_exclusive_scan<int>(pieces, s_wi, &s_tot_i);
-    const int chunk_seg = s_tot_i;
-    const int slot0 = carry_slot + block_exclusive_scan<int>(pieces > 1 ? pieces : 0, s_wi, &s_tot_i);
-    const int chunk_slot = s_tot_i;
-    const int split_i = carry_split + block_exclusive_scan<int>(pieces > 1 ? 1 : 0, s_wi, &s_tot_i);
-    const int chunk_split = s_tot_i;
-    const int empty_i = carry_empty + block_exclusive_scan<int>(in && n == 0 ? 1 : 0, s_wi, &s_tot_i);
-    const int chunk_empty = s_tot_i;
+    const unsigned long long v = static_cast<unsigned long long>(pieces) |
+                                 (static_cast<unsigned long long>(pieces > 1 ? pieces : 0) << 16) |
+                                 (static_cast<unsigned long long>(pieces > 1 ? 1 : 0) << 32) |
+                                 (static_cast<unsigned long long>(in && n == 0 ? 1 : 0) << 48);
+    const unsigned long long pre = block_exclusive_scan<unsigned long long>(v, s_wp, &s_tot_p);
+    const unsigned long long tot = s_tot_p;
+    const int seg0 = carry_seg + static_cast<int>(pre & 0xffffu);
+    const int slot0 = carry_slot + static_cast<int>((pre >> 16) & 0xffffu);
+    const int split_i = carry_split + static_cast<int>((pre >> 32) & 0xffffu);
+    const int empty_i = carry_empty + static_cast<int>((pre >> 48) & 0xffffu);
     if (in) {
       row_info[2 * w + 0] = pieces > 1 ? slot0 : -1;
       row_info[2 * w + 1] = pieces;
@@ -149,37 +169,27 @@ __global__ void __launch_bounds__(kSchedThreads) mla_sched_kernel(const int32_t*
       }
       if (pieces > 1) split_rows[split_i] = w;
       if (n == 0) empty_rows[empty_i] = w;
-      end_cost[w] = C + c;
-      first_seg[w] = seg0;
-      first_pair[w] = f;
+      // Pair p's segments start with the first one on a pair >= p.  When
+      // p * cap falls in this row's cost range [C, C + c), every segment of
+      // the rows before sits on a pair < p, and of this row's pieces (pairs
+      // f, f + 1, ...) those before pair p; later rows start at or past p.
+      if (c > 0) {
+        const long long p_end = (C + c + cap - 1) / cap;
+        for (long long p = (C + cap - 1) / cap; p < p_end && p < pairs; ++p)
+          pair_off[p] = seg0 + (p > f ? static_cast<int>(p - f) : 0);
+      }
     }
     carry_cost += chunk_cost;
-    carry_seg += chunk_seg;
-    carry_slot += chunk_slot;
-    carry_split += chunk_split;
-    carry_empty += chunk_empty;
+    carry_seg += static_cast<int>(tot & 0xffffu);
+    carry_slot += static_cast<int>((tot >> 16) & 0xffffu);
+    carry_split += static_cast<int>((tot >> 32) & 0xffffu);
+    carry_empty += static_cast<int>((tot >> 48) & 0xffffu);
   }
   if (err) s_err = 1;
-  __syncthreads();  // scratch written and visible to the whole CTA
-
-  // Pass 3: pair p starts at the first row whose pages reach cost position
-  // p * cap (end cost > p * cap); its first segment there is p - first pair.
-  for (int p = threadIdx.x; p <= pairs; p += kSchedThreads) {
-    int off = carry_seg;
-    if (p < pairs) {
-      const long long x = static_cast<long long>(p) * cap;
-      int lo_w = 0, hi_w = W;  // first w with end_cost[w] > x
-      while (lo_w < hi_w) {
-        const int mid = (lo_w + hi_w) >> 1;
-        if (end_cost[mid] > x) hi_w = mid; else lo_w = mid + 1;
-      }
-      if (lo_w < W) {
-        const int d = p - first_pair[lo_w];
-        off = first_seg[lo_w] + (d > 0 ? d : 0);
-      }
-    }
-    pair_off[p] = off;
-  }
+  // Pairs past the total cost (and the end marker) take no segment.
+  for (int p = threadIdx.x; p <= pairs; p += kSchedThreads)
+    if (p == pairs || static_cast<long long>(p) * cap >= T) pair_off[p] = carry_seg;
+  __syncthreads();  // s_err
 
   if (threadIdx.x == 0) {
     uint32_t e = s_err ? MLA_DEVERR_SEQLEN : 0u;

@@ -118,6 +118,8 @@ def decode_plan(meta, batch, h_q, s_q):
 PLAN_CASES = [
     ([256], 16, 1), ([0], 16, 1), ([0, 5, 0, 7000], 128, 1), ([4096] * 8, 128, 2), ([131072, 1024, 32768, 8192], 16, 1),
     ([1] * 300, 64, 1), ([77, 64, 65, 129, 4000, 1, 0, 99999], 128, 3), (list(range(0, 4000, 37)), 32, 2),
+    # more than 1024 work rows: the plan kernel's chunked path
+    ([(37 * k) % 900 for k in range(1100)], 64, 1), ([0, 1, 64, 65, 4000] * 250, 128, 2),
 ]
 
 
