@@ -348,33 +348,35 @@ __device__ void producer_k(const DecodeParams& p, const Ctx& c, int s_begin, int
     return __shfl_sync(0xffffffffu, good, 0) != 0;
   };
   walk_groups(p, c, s_begin, s_end, [&](const Segment& sg, const Group& gr) -> bool {
+    if (lane == 0) MLA_TRACE(0, gi);
+    // This CTA's two pages of the group; lanes 0 and 1 issue their boxes in
+    // one instruction (a TMA issue holds its thread for ~300 cycles; two
+    // lanes of one instruction take ~420 together instead of ~660 in turn).
+    const int my_page = c.cta == 0 ? (lane == 0 ? gr.page[0] : gr.page[1]) : (lane == 0 ? gr.page[2] : gr.page[3]);
+    const bool my_load = lane < 2 && 2 * static_cast<int>(c.cta) + lane < gr.np;
     int good = 1;
-    if (lane == 0) {
-      MLA_TRACE(0, gi);
-      for (int pn = 0; pn < 9 && good; ++pn, ++ks) {
-        const uint32_t slot = ks % kKRing;
-        if (ks >= kKRing) good = wait_bar(c, c.bar(kBarKEmpty + slot), ((ks / kKRing) - 1) & 1);
-        if (good) {
-          MLA_TRACE(10, ks);
-          MLA_STEP(ks);
-          if (c.cta == 0) mbar_arrive_expect_tx(c.bar(kBarKFull + slot), gr.np * kPagePanel);
-#pragma unroll
-          for (int q = 0; q < 2; ++q) {
-            const int gq = 2 * static_cast<int>(c.cta) + q;
-            if (gq < gr.np)
-              tma_load_3d_pair(c.kslot(slot) + q * kPagePanel, &p.tm_k, c.lead_bar(kBarKFull + slot), 0,
-                               gr.page[gq] * kPage, pn);
-          }
-          // The other CTA also arrives, even when it has no page in the group:
-          // otherwise the slot could fill and drain without it, and its
-          // parity wait on the slot's empty barrier would fall two phases
-          // behind.
-          if (c.cta != 0) mbar_arrive_remote(c.lead_bar(kBarKFull + slot));
-        }
+    for (int pn = 0; pn < 9; ++pn, ++ks) {
+      const uint32_t slot = ks % kKRing;
+      if (lane == 0 && ks >= kKRing) good = wait_bar(c, c.bar(kBarKEmpty + slot), ((ks / kKRing) - 1) & 1);
+      good = __shfl_sync(0xffffffffu, good, 0);
+      if (!good) break;
+      if (lane == 0) {
+        MLA_TRACE(10, ks);
+        MLA_STEP(ks);
+        if (c.cta == 0) mbar_arrive_expect_tx(c.bar(kBarKFull + slot), gr.np * kPagePanel);
       }
+      __syncwarp();
+      if (my_load)
+        tma_load_3d_pair(c.kslot(slot) + lane * kPagePanel, &p.tm_k, c.lead_bar(kBarKFull + slot), 0,
+                         my_page * kPage, pn);
+      if (lane == 0) MLA_TRACE(15, ks);
+      // The other CTA also arrives, even when it has no page in the group:
+      // otherwise the slot could fill and drain without it, and its parity
+      // wait on the slot's empty barrier would fall two phases behind.
+      if (lane == 0 && c.cta != 0) mbar_arrive_remote(c.lead_bar(kBarKFull + slot));
     }
     ++gi;
-    return __shfl_sync(0xffffffffu, good, 0) != 0;
+    return good != 0;
   }, load_q);
 }
 
