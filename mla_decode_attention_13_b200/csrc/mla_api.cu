@@ -125,22 +125,6 @@ int encode_value_tiles(PFN_cuTensorMapEncodeTiled_v12000 enc, CUtensorMap* map, 
   return r == CUDA_SUCCESS ? MLA_OK : MLA_ERR_CUDA;
 }
 
-// A row-major [outer][rows][512] tensor of 2- or 4-byte elements as (512
-// cols, rows, outer), box (128 bytes of columns, 32 rows, 1), 128B swizzle:
-// the TMA-store view of the output and of the split partials.
-int encode_store_map(PFN_cuTensorMapEncodeTiled_v12000 enc, CUtensorMap* map, void* base, uint64_t rows,
-                     uint64_t outer, bool fp32) {
-  const cuuint64_t esz = fp32 ? 4 : 2;
-  const cuuint64_t dims[3] = {static_cast<cuuint64_t>(kDv), rows, outer};
-  const cuuint64_t strides[2] = {kDv * esz, rows * kDv * esz};
-  const cuuint32_t box[3] = {static_cast<cuuint32_t>(128 / esz), 32, 1};
-  const cuuint32_t elem[3] = {1, 1, 1};
-  const CUresult r = enc(map, fp32 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT32 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, base,
-                         dims, strides, box, elem, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
-                         CU_TENSOR_MAP_L2_PROMOTION_NONE, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
-  return r == CUDA_SUCCESS ? MLA_OK : MLA_ERR_CUDA;
-}
-
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
 bool shape_ok(int batch, int h_q, int s_q) {
@@ -177,18 +161,8 @@ int decode_impl(const void* q, const void* kv_cache, int64_t num_pages, const in
   const uint64_t q_rows = static_cast<uint64_t>(batch) * R;
   if ((st = encode_panels576(enc, &p.tm_k, kv_cache, kv_rows, kPage, 1)) != MLA_OK ||
       (st = encode_value_tiles(enc, &p.tm_v, kv_cache, kv_rows)) != MLA_OK ||
-      (st = encode_panels576(enc, &p.tm_q, q, q_rows, kMTile / 2, kDqk / 64)) != MLA_OK ||
-      (st = encode_store_map(enc, &p.tm_out, out, static_cast<uint64_t>(R), static_cast<uint64_t>(batch), false)) !=
-          MLA_OK)
+      (st = encode_panels576(enc, &p.tm_q, q, q_rows, kMTile / 2, kDqk / 64)) != MLA_OK)
     return st;
-  if (slots > 0 && workspace) {
-    if ((st = encode_store_map(enc, &p.tm_opart, workspace, static_cast<uint64_t>(tr), static_cast<uint64_t>(slots),
-                               true)) != MLA_OK)
-      return st;
-  } else {
-    p.tm_opart = p.tm_out;  // never used: the plan splits no row without slots
-  }
-  p.kv = kv_cache;
   p.block_table = block_table;
   p.seqlens = seqlens;
   p.out = out;

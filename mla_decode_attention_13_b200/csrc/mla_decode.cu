@@ -70,7 +70,7 @@ namespace mla {
 // Optional clock64 timeline of the pipeline roles, for profiling builds only
 // (compile with -DMLA_DECODE_TRACE; the default build records nothing).
 #ifdef MLA_DECODE_TRACE
-__device__ unsigned long long g_mla_trace[4][16][512];  // [traced CTA][event][index]
+__device__ unsigned long long g_mla_trace[4][20][512];  // [traced CTA][event][index]
 __device__ unsigned long long g_mla_span[160][4];  // [pair][start, end, segments, pages] (globaltimer)
 // First wait that ran out of time: [taken, barrier index, parity, thread, block, clock].
 __device__ unsigned long long g_mla_abort[6];
@@ -717,30 +717,36 @@ __device__ void softmax_epilogue(const DecodeParams& p, const Ctx& c, uint32_t t
     if (r == 0) MLA_TRACE(12, s - s_begin);
     float lt;
     if (!trade(l, true, &lt)) return;
+    if ((threadIdx.x & 31) == 0) MLA_TRACE(16, 8 * (s - s_begin) + ((threadIdx.x >> 5) - 4));
     tc_fence_after();
     const float inv_l = lt > 0.0f ? 1.0f / lt : 0.0f;
     const float lse_v = lt > 0.0f ? (m + __log2f(lt)) * 0.69314718055994530942f : -INFINITY;
-    // Output through TMA stores: each warp stages its 32 rows x 128 bytes of
-    // columns in shared memory (128B-swizzled, two buffers per warp in the
-    // value ring, idle now) and stores the box; rows past R (or tile_rows)
-    // lie outside the store tensor and are dropped by the copy engine.  This
-    // thread's O columns: [256 sp + 128 half, +128).
+    // Output: each warp owns 32 rows x 128 columns of this CTA's tile (its
+    // TMEM lanes, O columns [256 sp + 128 half, +128)).  In steps of 128
+    // bytes of columns it stages them in shared memory (a 4 KB buffer per
+    // warp in the value ring, idle now; 16-byte chunks swizzled by row), then
+    // reads them back four rows per instruction and writes whole 128-byte
+    // lines with coalesced 16-byte stores, skipping rows past R (or
+    // tile_rows).  (Measured: TMA stores of 4 KB boxes took ~4,500 cycles
+    // for a CTA's 128 KB of fp32 partials, ~140 cycles per box.)
     const int ws = (threadIdx.x >> 5) - 4;  // softmax warp 0-7
-    const uint32_t stage0 = c.base + kOffV + ws * 8192;
-    uint8_t* stage0_g = c.gbase + kOffV + ws * 8192;
-    const int row0 = c.cta * kRowsCta + 32 * ((rr >> 5) & 1);  // first row of this warp's box in the tile
+    uint8_t* stage = c.gbase + kOffV + ws * 4096;
+    const int row0 = c.cta * kRowsCta + 32 * ((rr >> 5) & 1);  // first row of this warp in the tile
     const uint32_t swz = lane & 7;
     const int col0 = 256 * sp + 128 * half;
+    const int rd_row = lane >> 3;   // read-back: rows rd_row + 4 i, chunk lane % 8
+    const int rd_chunk = lane & 7;
     if (sg.slot < 0) {
-      const int y = sg.mt * kMTile + row0;
-      const bool any = y < p.R;
+      __nv_bfloat16* obase = reinterpret_cast<__nv_bfloat16*>(p.out) +
+                             (static_cast<long long>(sg.i) * p.R + sg.mt * kMTile + row0) * kDv + col0;
+      const int rows_ok = p.R - (sg.mt * kMTile + row0);  // rows of this warp that exist
 #pragma unroll 1
-      for (int k = 0; k < 2; ++k) {  // 64 columns (128 bytes of bf16) per box
+      for (int k = 0; k < 2; ++k) {  // 64 columns (128 bytes of bf16) per step
         float o[64];
         tmem_ld32(t_o + 64 * k, *reinterpret_cast<float(*)[32]>(o));
         tmem_ld32(t_o + 64 * k + 32, *reinterpret_cast<float(*)[32]>(o + 32));
         tmem_wait_ld();
-        uint8_t* srow = stage0_g + k * 4096 + lane * 128;
+        uint8_t* srow = stage + lane * 128;
 #pragma unroll
         for (int jj = 0; jj < 8; ++jj) {
           __nv_bfloat162 h0 = __floats2bfloat162_rn(o[8 * jj + 0] * inv_l, o[8 * jj + 1] * inv_l);
@@ -754,48 +760,55 @@ __device__ void softmax_epilogue(const DecodeParams& p, const Ctx& c, uint32_t t
           v.w = *reinterpret_cast<uint32_t*>(&h3);
           *reinterpret_cast<uint4*>(srow + ((jj ^ swz) << 4)) = v;
         }
-        fence_proxy_async_smem();
         __syncwarp();
-        if (lane == 0 && any) tma_store_3d(&p.tm_out, stage0 + k * 4096, col0 + 64 * k, y, sg.i);
-        if (lane == 0) bulk_commit_group();
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+          const int r2 = rd_row + 4 * i;
+          const uint4 v = *reinterpret_cast<const uint4*>(stage + r2 * 128 + ((rd_chunk ^ (r2 & 7)) << 4));
+          if (r2 < rows_ok)
+            *reinterpret_cast<uint4*>(obase + static_cast<long long>(r2) * kDv + 64 * k + 8 * rd_chunk) = v;
+        }
+        __syncwarp();
       }
       if (row_valid && half == 0 && sp == 0) p.lse[(static_cast<long long>(sg.i) * p.h_q + hh) * p.s_q + t] = lse_v;
     } else {
-      const bool any = row0 < p.tile_rows;
+      float* obase = p.o_part + (static_cast<long long>(sg.slot) * p.tile_rows + row0) * kDv + col0;
+      const int rows_ok = p.tile_rows - row0;
 #pragma unroll 1
-      for (int k = 0; k < 4; ++k) {  // 32 columns (128 bytes of fp32) per box
+      for (int k = 0; k < 4; ++k) {  // 32 columns (128 bytes of fp32) per step
         float o[32];
         tmem_ld32(t_o + 32 * k, o);
         tmem_wait_ld();
-        const uint32_t buf = k & 1;
-        if (k >= 2) {
-          if (lane == 0) bulk_wait_group_read<1>();
-          __syncwarp();
-        }
-        uint8_t* srow = stage0_g + buf * 4096 + lane * 128;
+        uint8_t* srow = stage + lane * 128;
 #pragma unroll
         for (int jj = 0; jj < 8; ++jj)
           *reinterpret_cast<float4*>(srow + ((jj ^ swz) << 4)) =
               make_float4(o[4 * jj] * inv_l, o[4 * jj + 1] * inv_l, o[4 * jj + 2] * inv_l, o[4 * jj + 3] * inv_l);
-        fence_proxy_async_smem();
         __syncwarp();
-        if (lane == 0 && any) tma_store_3d(&p.tm_opart, stage0 + buf * 4096, col0 + 32 * k, row0, sg.slot);
-        if (lane == 0) bulk_commit_group();
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+          const int r2 = rd_row + 4 * i;
+          const float4 v = *reinterpret_cast<const float4*>(stage + r2 * 128 + ((rd_chunk ^ (r2 & 7)) << 4));
+          if (r2 < rows_ok)
+            *reinterpret_cast<float4*>(obase + static_cast<long long>(r2) * kDv + 32 * k + 4 * rd_chunk) = v;
+        }
+        __syncwarp();
       }
       if (row_valid && half == 0 && sp == 0)
         p.lse_part[static_cast<long long>(sg.slot) * p.tile_rows + q_row] = lse_v;
     }
     tc_fence_before();
     __syncwarp();
+    if (lane == 0) MLA_TRACE(17, 8 * (s - s_begin) + ((threadIdx.x >> 5) - 4));
     if (lane == 0) arrive_leader(c, kBarOEmpty);  // O is read out: the next segment's PV may overwrite it
     if (lane == 0) {
-      bulk_wait_group_read<0>();
+      MLA_TRACE(18, 8 * (s - s_begin) + ((threadIdx.x >> 5) - 4));
       mbar_arrive(c.bar(kBarStageFree));  // staging read: the value ring may be refilled
     }
     __syncwarp();
     if (r == 0) MLA_TRACE(13, s - s_begin);
   }
-  if (lane == 0) bulk_wait_group_all();  // this warp's output stores have landed
+  if (lane == 0) MLA_TRACE(19, (threadIdx.x >> 5) - 4);
   __syncwarp();
 }
 
@@ -945,7 +958,7 @@ extern "C" __attribute__((visibility("default"))) int mla_trace_stuck(void* stuc
   return static_cast<int>(e);
 }
 extern "C" __attribute__((visibility("default"))) int mla_trace_clear() {
-  static unsigned long long zero[4][16][512];
+  static unsigned long long zero[4][20][512];
   return static_cast<int>(cudaMemcpyToSymbol(g_mla_trace, zero, sizeof(zero)));
 }
 #endif

@@ -99,13 +99,6 @@ struct DecodeParams {
   // page (its 128 columns of each half), panels in [half][panel] order.
   CUtensorMap tm_v;
   CUtensorMap tm_q;  // q: box (64, 64, 9), 64 query rows
-  // Stores, with 128B swizzle: out as (512 cols, R rows, batch), box (64,
-  // 32, 1) bf16; o_part as (512 cols, tile_rows, max_slots), box (32, 32, 1)
-  // fp32.  Rows past R (or tile_rows) fall outside the tensor and are not
-  // written.
-  CUtensorMap tm_out;
-  CUtensorMap tm_opart;
-  const void* kv;          // cache base (bf16 [num_pages*64][576]), for L2 prefetch
   const int32_t* block_table;
   const int32_t* seqlens;
   void* out;               // bf16
