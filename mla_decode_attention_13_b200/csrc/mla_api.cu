@@ -195,6 +195,7 @@ int decode_impl(const void* q, const void* kv_cache, int64_t num_pages, const in
   cp.tile_rows = tr;
   cp.pairs = dev.pairs;
   cp.max_slots = slots;
+  cp.slices = combine_slices(batch * p.n_mt, tr, dev.sms);
 
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   // Inside a stream capture the events must become event-record nodes of the
@@ -210,7 +211,7 @@ int decode_impl(const void* q, const void* kv_cache, int64_t num_pages, const in
   if (launch_decode(p, dev.pairs, s) != cudaSuccess) return MLA_ERR_CUDA;
   if (ev_after && cudaEventRecordWithFlags(static_cast<cudaEvent_t>(ev_after), s, ev_flags) != cudaSuccess)
     return MLA_ERR_CUDA;
-  if (launch_combine(cp, 2 * dev.sms, s) != cudaSuccess) return MLA_ERR_CUDA;
+  if (launch_combine(cp, 4 * dev.sms, s) != cudaSuccess) return MLA_ERR_CUDA;
   return MLA_OK;
 }
 

@@ -72,6 +72,12 @@ namespace mla {
 #ifdef MLA_DECODE_TRACE
 __device__ unsigned long long g_mla_trace[4][20][512];  // [traced CTA][event][index]
 __device__ unsigned long long g_mla_span[160][4];  // [pair][start, end, segments, pages] (globaltimer)
+// Prologue of the leader CTA of each pair: [entry, after cluster sync, after the grid dependency, exit].
+__device__ unsigned long long g_mla_pro[160][4];
+#define MLA_PRO(k)                                                                    \
+  do {                                                                                \
+    if (threadIdx.x == 0 && cluster_ctarank() == 0) g_mla_pro[blockIdx.x >> 1][k] = globaltimer(); \
+  } while (0)
 // First wait that ran out of time: [taken, barrier index, parity, thread, block, clock].
 __device__ unsigned long long g_mla_abort[6];
 // Per block and warp: the wait it left on abort (1 << 32 | barrier << 8 | parity)
@@ -94,6 +100,9 @@ __device__ unsigned long long g_mla_step[160 * 2][12];
   } while (0)
 #define MLA_STEP(v) \
   do {              \
+  } while (0)
+#define MLA_PRO(k) \
+  do {             \
   } while (0)
 #endif
 
@@ -815,6 +824,7 @@ __device__ void softmax_epilogue(const DecodeParams& p, const Ctx& c, uint32_t t
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     mla_decode_kernel(const __grid_constant__ DecodeParams p) {
   extern __shared__ uint8_t smem_raw[];
+  MLA_PRO(0);
   const uint32_t raw = smem_u32(smem_raw);
   const uint32_t base = (raw + 1023u) & ~1023u;
   Ctx c;
@@ -866,6 +876,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
   __syncthreads();
   tc_fence_after();
   cluster_sync();  // both CTAs' barriers exist before any remote arrival
+  MLA_PRO(1);
   const uint32_t tmem = *reinterpret_cast<volatile uint32_t*>(c.gbase + kOffTmemSlot);
   c.peer_abort = map_to_rank(base + kOffAbort, c.cta ^ 1u);
   c.lead_bars = map_to_rank(base + kOffBar, 0);
@@ -875,6 +886,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
   // may start launching now (it waits for this kernel in turn).
   griddep_launch_dependents();
   griddep_wait();
+  MLA_PRO(2);
 
   // The plan must be the one built for this call's shape on this many pairs.
   const int pair = static_cast<int>(blockIdx.x >> 1);
@@ -938,6 +950,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     tc_fence_after();
     tmem_dealloc_pair(tmem, kTmemCols);
   }
+  MLA_PRO(3);
 }
 
 }  // namespace
@@ -948,6 +961,9 @@ extern "C" __attribute__((visibility("default"))) int mla_trace_read(void* host)
 }
 extern "C" __attribute__((visibility("default"))) int mla_trace_span(void* host) {
   return static_cast<int>(cudaMemcpyFromSymbol(host, g_mla_span, sizeof(g_mla_span)));
+}
+extern "C" __attribute__((visibility("default"))) int mla_trace_pro(void* host) {
+  return static_cast<int>(cudaMemcpyFromSymbol(host, g_mla_pro, sizeof(g_mla_pro)));
 }
 extern "C" __attribute__((visibility("default"))) int mla_trace_abort(void* host) {
   return static_cast<int>(cudaMemcpyFromSymbol(host, g_mla_abort, sizeof(g_mla_abort)));

@@ -19,7 +19,7 @@ constexpr int kMTile = 128;       // query rows per work row (UMMA M)
 constexpr int kMaxPairs = 160;    // upper bound on SM pairs of any sm_100 part
 constexpr int kMaxHq = 128;
 constexpr int kMaxSq = 16;
-constexpr int kKappa = 2;         // fixed per-piece cost of the plan, in pages
+constexpr int kKappa = 4;         // fixed per-piece cost of the plan, in pages
 constexpr uint32_t kMagic = 0x314C4D42u;  // "BML1"
 
 // ---------------------------------------------------------------------------
@@ -30,6 +30,8 @@ constexpr uint32_t kMagic = 0x314C4D42u;  // "BML1"
 //   row_info  [W][2]                    (first slot or -1, pieces)
 //   split_rows [W]                      work rows cut into >1 pieces
 //   empty_rows [W]                      work rows with no pages
+//   tasks     [W][4]                    per split row: (work row, first slot, pieces, 0),
+//                                       so the combine finds a row's pieces in one load
 // A work row is (batch row i, m-tile mt) with index w = mt * batch + i.
 // ---------------------------------------------------------------------------
 enum HeaderWord : int {
@@ -53,7 +55,7 @@ enum HeaderWord : int {
 
 struct MetaLayout {
   int W;
-  size_t pair_off, segs, row_info, split_rows, empty_rows, words;
+  size_t pair_off, segs, row_info, split_rows, empty_rows, tasks, words;
 };
 
 __host__ __device__ inline int ceil_div(int a, int b) { return (a + b - 1) / b; }
@@ -66,7 +68,8 @@ __host__ __device__ inline MetaLayout meta_layout(int batch, int h_q, int s_q) {
   L.row_info = L.segs + size_t(4) * (L.W + kMaxPairs);
   L.split_rows = L.row_info + size_t(2) * L.W;
   L.empty_rows = L.split_rows + L.W;
-  L.words = L.empty_rows + L.W;
+  L.tasks = (L.empty_rows + L.W + 3) & ~size_t(3);
+  L.words = L.tasks + size_t(4) * L.W;
   return L;
 }
 
@@ -119,6 +122,7 @@ struct CombineParams {
   void* out;
   float* lse;
   int batch, s_q, h_q, R, tile_rows, pairs, max_slots;
+  int slices;  // warps per query row (1, 2, 4 or 8), each merging 512 / slices columns
 };
 
 // Launch wrappers (each returns a cudaError_t).
@@ -131,5 +135,8 @@ size_t decode_kernel_smem_bytes();
 cudaError_t take_sticky_error(cudaStream_t stream, uint32_t* word);
 cudaError_t launch_decode(const DecodeParams& p, int pairs, cudaStream_t stream);
 cudaError_t launch_combine(const CombineParams& p, int grid, cudaStream_t stream);
+// Warps per query row of the combine (CombineParams::slices) for this many
+// work rows of tile_rows query rows on a device with `sms` SMs.
+int combine_slices(int work_rows, int tile_rows, int sms);
 
 }  // namespace mla

@@ -14,9 +14,11 @@
 //     read the same pages, land on pairs far apart and run at the same time;
 //   * a row with n > 0 pages costs n + kappa (kappa: fixed cost of starting a
 //     row: Q load, pipeline fill, epilogue); C_w is the cost of the rows before
-//     w and T the total; cap = max(1, ceil(T / P));
-//   * page b of row w sits at cost position C_w + kappa + b and belongs to pair
-//     floor(position / cap), so every pair takes one contiguous page range;
+//     w and T the total;
+//   * page b of row w sits at cost position C_w + kappa + b; pair p owns the
+//     positions [B(p), B(p + 1)) with B(p) = floor(p T / P) when T >= P (each
+//     pair gets floor(T / P) or ceil(T / P) positions, so none is idle) and
+//     B(p) = min(p, T) otherwise, so every pair takes one contiguous range;
 //   * a row whose pages land on k > 1 pairs is cut into k pieces with k
 //     consecutive partial slots (row order); its output comes from the combine.
 // Everything follows from prefix sums, so one CTA computes it with block-wide
@@ -26,6 +28,12 @@
 #include "sm100_ptx.cuh"
 
 namespace mla {
+
+#ifdef MLA_DECODE_TRACE
+// Profiling builds only: [entry, after the grid dependency, exit] of the last launch (globaltimer).
+__device__ unsigned long long g_mla_sched_times[3];
+#endif
+
 namespace {
 
 constexpr int kSchedThreads = 1024;
@@ -61,6 +69,40 @@ __device__ T block_exclusive_scan(T v, T* warp_tot, T* total) {
   return res;
 }
 
+// The pairs' cost boundaries B(p) (see the header), the pair owning cost
+// position x (B(p) <= x < B(p + 1)), and the first pair p with B(p) >= x.
+// next() steps (B(p), its remainder) to B(p + 1) without a division.
+struct Bounds {
+  long long T;
+  int P;
+  long long tq, tr;  // T / P and T % P
+  __device__ Bounds(long long T_, int P_) : T(T_), P(P_), tq(T_ / P_), tr(T_ % P_) {}
+  __device__ long long owner(long long x) const { return T >= P ? ((x + 1) * P - 1) / T : x; }
+  __device__ long long first_at_or_past(long long x) const { return T >= P ? (x * P + T - 1) / T : x; }
+  // B(p) as a quotient and remainder of p * T / P.
+  __device__ void at(long long p, long long* q, long long* r) const {
+    if (T >= P) {
+      *q = (p * T) / P;
+      *r = p * T - *q * P;
+    } else {
+      *q = p < T ? p : T;
+      *r = 0;
+    }
+  }
+  __device__ void next(long long p, long long* q, long long* r) const {  // from B(p) to B(p + 1)
+    if (T >= P) {
+      *q += tq;
+      *r += tr;
+      if (*r >= P) {
+        *r -= P;
+        ++*q;
+      }
+    } else {
+      *q = p + 1 < T ? p + 1 : T;
+    }
+  }
+};
+
 __device__ __forceinline__ int row_pages(const int32_t* seqlens, int batch, int w, int* err) {
   int L = seqlens[w % batch];
   if (L < 0) {
@@ -75,8 +117,14 @@ __global__ void __launch_bounds__(kSchedThreads) mla_sched_kernel(const int32_t*
   // Programmatic dependent launch: the decode kernel may start its set-up now;
   // this kernel itself waits until the previous kernel in the stream (which
   // may still read the metadata, or have written the lengths) has completed.
+#ifdef MLA_DECODE_TRACE
+  if (threadIdx.x == 0) g_mla_sched_times[0] = ptx::globaltimer();
+#endif
   ptx::griddep_launch_dependents();
   ptx::griddep_wait();
+#ifdef MLA_DECODE_TRACE
+  if (threadIdx.x == 0) g_mla_sched_times[1] = ptx::globaltimer();
+#endif
   const MetaLayout lo = meta_layout(batch, h_q, s_q);
   const int W = lo.W;
   const int R = s_q * h_q;
@@ -86,6 +134,7 @@ __global__ void __launch_bounds__(kSchedThreads) mla_sched_kernel(const int32_t*
   int32_t* row_info = meta + lo.row_info;
   int32_t* split_rows = meta + lo.split_rows;
   int32_t* empty_rows = meta + lo.empty_rows;
+  int32_t* tasks = meta + lo.tasks;
 
   __shared__ long long s_wl[kWarps];
   __shared__ unsigned long long s_wp[kWarps];
@@ -114,7 +163,8 @@ __global__ void __launch_bounds__(kSchedThreads) mla_sched_kernel(const int32_t*
     block_exclusive_scan<long long>(local, s_wl, &s_tot_l);
     T = s_tot_l;
   }
-  const long long cap = T > 0 ? (T + pairs - 1) / pairs : 1;
+  const long long cap = T > 0 ? (T + pairs - 1) / pairs : 1;  // the longest range (reported only)
+  const Bounds bd(T, pairs);
 
   // Pass 2: per-row prefix sums, chunk by chunk with carries.  The four
   // counts (segments, partial slots, split rows, empty rows) are scanned
@@ -139,8 +189,8 @@ __global__ void __launch_bounds__(kSchedThreads) mla_sched_kernel(const int32_t*
     const long long c = n > 0 ? n + kKappa : 0;
     int f = 0, pieces = 0;
     if (n > 0) {
-      f = static_cast<int>((C + kKappa) / cap);
-      const int l = static_cast<int>((C + kKappa + n - 1) / cap);
+      f = static_cast<int>(bd.owner(C + kKappa));
+      const int l = static_cast<int>(bd.owner(C + kKappa + n - 1));
       pieces = l - f + 1;
     }
     const unsigned long long v = static_cast<unsigned long long>(pieces) |
@@ -156,10 +206,13 @@ __global__ void __launch_bounds__(kSchedThreads) mla_sched_kernel(const int32_t*
     if (in) {
       row_info[2 * w + 0] = pieces > 1 ? slot0 : -1;
       row_info[2 * w + 1] = pieces;
+      long long bq, br;  // B(p) of the piece's pair p, stepped along
+      bd.at(f, &bq, &br);
       for (int k = 0; k < pieces; ++k) {
         const long long p = f + k;
-        const long long b0 = p * cap - C - kKappa;
-        const long long b1 = (p + 1) * cap - C - kKappa;
+        const long long b0 = bq - C - kKappa;
+        bd.next(p, &bq, &br);
+        const long long b1 = bq - C - kKappa;
         int4 sg;
         sg.x = w;
         sg.y = b0 > 0 ? static_cast<int>(b0) : 0;
@@ -167,15 +220,18 @@ __global__ void __launch_bounds__(kSchedThreads) mla_sched_kernel(const int32_t*
         sg.w = pieces > 1 ? slot0 + k : -1;
         *reinterpret_cast<int4*>(segs + 4 * (seg0 + k)) = sg;
       }
-      if (pieces > 1) split_rows[split_i] = w;
+      if (pieces > 1) {
+        split_rows[split_i] = w;
+        *reinterpret_cast<int4*>(tasks + 4 * split_i) = make_int4(w, slot0, pieces, 0);
+      }
       if (n == 0) empty_rows[empty_i] = w;
       // Pair p's segments start with the first one on a pair >= p.  When
-      // p * cap falls in this row's cost range [C, C + c), every segment of
-      // the rows before sits on a pair < p, and of this row's pieces (pairs
-      // f, f + 1, ...) those before pair p; later rows start at or past p.
+      // B(p) falls in this row's cost range [C, C + c), every segment of the
+      // rows before sits on a pair < p, and of this row's pieces (pairs f,
+      // f + 1, ...) those before pair p; later rows start at or past p.
       if (c > 0) {
-        const long long p_end = (C + c + cap - 1) / cap;
-        for (long long p = (C + cap - 1) / cap; p < p_end && p < pairs; ++p)
+        const long long p_end = bd.first_at_or_past(C + c);
+        for (long long p = bd.first_at_or_past(C); p < p_end && p < pairs; ++p)
           pair_off[p] = seg0 + (p > f ? static_cast<int>(p - f) : 0);
       }
     }
@@ -186,9 +242,11 @@ __global__ void __launch_bounds__(kSchedThreads) mla_sched_kernel(const int32_t*
     carry_empty += static_cast<int>((tot >> 48) & 0xffffu);
   }
   if (err) s_err = 1;
-  // Pairs past the total cost (and the end marker) take no segment.
+  // Pairs whose range starts at the total cost (the end marker, and when
+  // T < P the pairs past T) take no segment.
+  const long long p_tail = bd.first_at_or_past(T);
   for (int p = threadIdx.x; p <= pairs; p += kSchedThreads)
-    if (p == pairs || static_cast<long long>(p) * cap >= T) pair_off[p] = carry_seg;
+    if (p >= p_tail) pair_off[p] = carry_seg;
   __syncthreads();  // s_err
 
   if (threadIdx.x == 0) {
@@ -210,9 +268,19 @@ __global__ void __launch_bounds__(kSchedThreads) mla_sched_kernel(const int32_t*
     meta[kHSq] = s_q;
     meta[kHCap] = static_cast<int32_t>(cap < 0x7fffffffLL ? cap : 0x7fffffffLL);
   }
+#ifdef MLA_DECODE_TRACE
+  __syncthreads();
+  if (threadIdx.x == 0) g_mla_sched_times[2] = ptx::globaltimer();
+#endif
 }
 
 }  // namespace
+
+#ifdef MLA_DECODE_TRACE
+extern "C" __attribute__((visibility("default"))) int mla_trace_sched_times(void* host) {
+  return static_cast<int>(cudaMemcpyFromSymbol(host, g_mla_sched_times, sizeof(g_mla_sched_times)));
+}
+#endif
 
 cudaError_t launch_sched(const int32_t* seqlens, int batch, int h_q, int s_q, int pairs, int32_t* meta,
                          cudaStream_t stream) {

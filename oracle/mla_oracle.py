@@ -281,10 +281,13 @@ def split_plan(seqlens, h_q, s_q, num_pairs: int, kappa: int) -> dict:
     ordered m-tile major (w = mt * batch + i).  A work row with n > 0 pages
     costs c = n + kappa (kappa: the fixed cost of starting a row, in page
     units), else 0.  With C_w the cost of the rows before w and T the total,
-    page b of row w sits at cost position C_w + kappa + b and belongs to pair
-    floor(position / cap), cap = max(1, ceil(T / P)).  Each pair thus takes one
-    contiguous range of pages; a row whose pages land on k > 1 pairs is cut
-    into k pieces and gets k consecutive partial slots, numbered in row order.
+    page b of row w sits at cost position C_w + kappa + b.  Pair p owns the
+    positions [B(p), B(p + 1)), with B(p) = floor(p * T / P) when T >= P (every
+    pair gets floor(T / P) or ceil(T / P) positions) and B(p) = min(p, T)
+    otherwise (one position each; the pairs past T get none).  Each pair thus
+    takes one contiguous range of pages; a row whose pages land on k > 1 pairs
+    is cut into k pieces and gets k consecutive partial slots, numbered in row
+    order.  ``cap`` reports the longest range, max(1, ceil(T / P)).
     """
     lens = [int(x) for x in as_int(seqlens)]
     batch = len(lens)
@@ -297,18 +300,20 @@ def split_plan(seqlens, h_q, s_q, num_pairs: int, kappa: int) -> dict:
             n_blk[mt * batch + i] = (max(lens[i], 0) + PAGE - 1) // PAGE
     cost = [(n + kappa) if n > 0 else 0 for n in n_blk]
     T = sum(cost)
-    cap = max(1, (T + num_pairs - 1) // num_pairs)
+    P = num_pairs
+    cap = max(1, (T + P - 1) // P)
+    bound = [(p * T) // P if T >= P else min(p, T) for p in range(P + 1)]
     segs = []  # (pair, w, b0, b1)
     C = 0
     for w in range(W):
         n = n_blk[w]
         if n > 0:
-            first = (C + kappa) // cap
-            last = (C + kappa + n - 1) // cap
-            for p in range(first, last + 1):
-                b0 = max(0, p * cap - C - kappa)
-                b1 = min(n, (p + 1) * cap - C - kappa)
-                segs.append([p, w, b0, b1])
+            lo, hi = C + kappa, C + kappa + n  # this row's page positions
+            for p in range(P):
+                b0 = max(lo, bound[p]) - lo
+                b1 = min(hi, bound[p + 1]) - lo
+                if b0 < b1:
+                    segs.append([p, w, b0, b1])
         C += cost[w]
     pieces = [0] * W
     for sg in segs:

@@ -99,6 +99,7 @@ def decode_plan(meta, batch, h_q, s_q):
     row0 = seg0 + 4 * (W + maxp)
     split0 = row0 + 2 * W
     empty0 = split0 + W
+    tasks0 = (empty0 + W + 3) & ~3
     segs = m[seg0:seg0 + 4 * nseg].reshape(nseg, 4)
     pair_off = m[hdr:hdr + P + 1].tolist()
     seg_pair = []
@@ -112,6 +113,7 @@ def decode_plan(meta, batch, h_q, s_q):
         "num_slots": int(m[5]), "kappa": int(m[9]),
         "split_rows": [int(v) for v in m[split0:split0 + int(m[10])]],
         "empty_rows": [int(v) for v in m[empty0:empty0 + int(m[11])]],
+        "tasks": [tuple(int(v) for v in t) for t in m[tasks0:tasks0 + 4 * int(m[10])].reshape(-1, 4)],
     }
 
 
@@ -137,6 +139,8 @@ def test_plan_matches_oracle_bit_for_bit(lens, h_q, s_q):
         if key == "segments":
             want_v = [tuple(s) for s in want_v]
         assert got[key] == want_v, key
+    # one combine task per split row: (work row, first slot, pieces, 0)
+    assert got["tasks"] == [(w, want["slot_base"][w], want["pieces"][w], 0) for w in want["split_rows"]]
 
 
 def test_num_sm_pairs_is_half_the_sms():

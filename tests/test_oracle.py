@@ -340,9 +340,17 @@ def test_plan_covers_every_page_once_and_balances(case, kappa):
     assert owners == sorted(owners)
     # per-pair load stays within cap
     load = [0] * P
+    pages = [0] * P
     for (w, b0, b1, _), p in zip(plan["segments"], plan["segment_pair"]):
         load[p] += b1 - b0 + kappa
+        pages[p] += b1 - b0
     assert max(load, default=0) <= plan["cap"] + 2 * kappa
+    assert max(pages, default=0) <= plan["cap"]
+    # proportional ranges: when every range is longer than kappa, no pair is idle
+    T = sum(-(-max(L, 0) // 64) + kappa for L in lens if L > 0) * n_mt
+    assert plan["cap"] == max(1, -(-T // P))
+    if T >= (kappa + 1) * P:
+        assert min(pages) >= 1
     # pair offsets index the segment list
     offs = plan["pair_offsets"]
     assert offs[0] == 0 and offs[-1] == len(plan["segments"])
