@@ -71,7 +71,9 @@ extern "C" {
 #define MLA_DEVERR_SEQLEN 0x1u   /* L_i < 0 or L_i > 64 * max_pages_per_seq */
 #define MLA_DEVERR_PAGE 0x2u     /* block-table entry outside [0, num_pages) */
 #define MLA_DEVERR_TIMEOUT 0x4u  /* a bounded wait inside a kernel gave up   */
-#define MLA_DEVERR_PLAN 0x8u     /* metadata does not match this call        */
+#define MLA_DEVERR_PLAN 0x8u     /* metadata does not match this call (its
+                                    shape, or lengths that changed since it
+                                    was built)                               */
 
 /* Fixed dimensions of the absorbed cache row and of a page. */
 #define MLA_D_QK 576
@@ -123,7 +125,9 @@ int mla_get_metadata(const int32_t* seqlens, int batch, int h_q, int s_q, void* 
  *   block_table  [device] int32 [batch][max_pages_per_seq]; entries past a
  *                row's ceil(L_i / 64) pages are never read.
  *   seqlens      [device] int32 [batch], 0 <= L_i <= 64 * max_pages_per_seq;
- *                must hold the values the metadata was built from.
+ *                must hold the values the metadata was built from: the
+ *                kernels work from the lengths the plan read, and a length
+ *                that differs from them sets MLA_DEVERR_PLAN.
  *   softmax_scale  multiplies <q, k>; finite and >= 0.
  *   causal       0 or 1 (see the header comment).
  *   out          [device] bf16 [batch][s_q][h_q][512], 16-byte aligned.

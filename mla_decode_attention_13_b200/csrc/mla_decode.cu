@@ -183,6 +183,12 @@ constexpr uint32_t kColS = 256;  // 2 x 128
 constexpr uint32_t kIdescQK = idesc_bf16_f32(kMTile, kGroup * kPage, false);
 constexpr uint32_t kIdescPV = idesc_bf16_f32(kMTile, 256, true);
 
+struct Segment {
+  int w, b0, b1, slot;
+  int i, mt, L;
+  bool bad;
+};
+
 struct Ctx {
   uint32_t base;     // shared::cta address of the aligned base
   uint8_t* gbase;    // generic pointer to the same place
@@ -191,6 +197,8 @@ struct Ctx {
   uint32_t lead_bars;  // shared::cluster address of the leader's barrier block
   volatile uint32_t* abort_flag;
   int32_t* meta;
+  int s_begin;       // this pair's first segment, read with the pair's record
+  Segment first;
   __device__ uint32_t bar(uint32_t k) const { return base + kOffBar + 8 * k; }
   __device__ uint32_t lead_bar(uint32_t k) const { return lead_bars + 8 * k; }
   __device__ uint32_t kslot(uint32_t k) const { return base + kOffK + k * kKSlot; }
@@ -251,20 +259,16 @@ __device__ __forceinline__ void arrive_leader(const Ctx& c, uint32_t k) {
   }
 }
 
-struct Segment {
-  int w, b0, b1, slot;
-  int i, mt, L;
-  bool bad;
-};
-
-__device__ __forceinline__ Segment load_segment(const DecodeParams& p, int s) {
-  const MetaLayout lo = meta_layout(p.batch, p.h_q, p.s_q);
-  const int4 v = *reinterpret_cast<const int4*>(p.meta + lo.segs + 4 * s);
+// A segment from its record (work row, first page, end page, slot; length).
+// The length is the one the plan read, so every role takes the same decision
+// on a bad segment whatever the lengths hold now (the softmax warps check
+// them against it).
+__device__ __forceinline__ Segment make_segment(const DecodeParams& p, int4 a, int L) {
   Segment g;
-  g.w = v.x;
-  g.b0 = v.y;
-  g.b1 = v.z;
-  g.slot = v.w;
+  g.w = a.x;
+  g.b0 = a.y;
+  g.b1 = a.z;
+  g.slot = a.w;
   if (g.w < 0 || g.w >= p.batch * p.n_mt) {
     g.i = g.mt = g.L = 0;
     g.bad = true;
@@ -272,10 +276,20 @@ __device__ __forceinline__ Segment load_segment(const DecodeParams& p, int s) {
   }
   g.i = g.w % p.batch;
   g.mt = g.w / p.batch;
-  g.L = p.seqlens[g.i];
+  g.L = L;
   g.bad = g.L < 0 || g.L > kPage * p.max_pages || g.b1 > ceil_div(g.L, kPage) || g.b0 < 0 || g.b0 >= g.b1 ||
           g.slot >= p.max_slots;
   return g;
+}
+
+// Segment s of this pair: the first one came with the pair's record.
+__device__ __forceinline__ Segment load_segment(const DecodeParams& p, const Ctx& c, int s) {
+  if (s == c.s_begin) return c.first;
+  const MetaLayout lo = meta_layout(p.batch, p.h_q, p.s_q);
+  const int32_t* rec = p.meta + lo.segs + kSegWords * s;
+  const int4 a = *reinterpret_cast<const int4*>(rec);
+  const int L = rec[4];
+  return make_segment(p, a, L);
 }
 
 __device__ __forceinline__ int load_page(const DecodeParams& p, const Ctx& c, const int32_t* table, int blk,
@@ -312,7 +326,7 @@ __device__ __forceinline__ void walk_groups(const DecodeParams& p, const Ctx& c,
   static_assert(32 % kGroup == 0, "groups never straddle a chunk of page ids");
   const int lane = threadIdx.x & 31;
   for (int s = s_begin; s < s_end; ++s) {
-    const Segment sg = load_segment(p, s);
+    const Segment sg = load_segment(p, c, s);
     if (sg.bad) continue;
     if (!on_segment(sg)) return;
     const int32_t* table = p.block_table + static_cast<long long>(sg.i) * p.max_pages;
@@ -465,7 +479,7 @@ __device__ void qk_issuer(const DecodeParams& p, const Ctx& c, uint32_t tmem, in
   uint32_t gi = 0, ks = 0, seg_it = 0;  // groups, key panels consumed, segments
   const uint16_t both = 0x3;
   for (int s = s_begin; s < s_end; ++s) {
-    const Segment sg = load_segment(p, s);
+    const Segment sg = load_segment(p, c, s);
     if (sg.bad) continue;
     const int ng = ceil_div(sg.b1 - sg.b0, kGroup);
     if (!wait_bar(c, c.bar(kBarQFull), seg_it & 1)) return;
@@ -493,7 +507,7 @@ __device__ void pv_issuer(const DecodeParams& p, const Ctx& c, uint32_t tmem, in
   uint32_t pg = 0, seg_it = 0;  // pages, segments
   const uint16_t both = 0x3;
   for (int s = s_begin; s < s_end; ++s) {
-    const Segment sg = load_segment(p, s);
+    const Segment sg = load_segment(p, c, s);
     if (sg.bad) continue;
     const int n = sg.b1 - sg.b0;
     for (int jp = 0; jp < n; ++jp, ++pg) {
@@ -590,11 +604,14 @@ __device__ void softmax_epilogue(const DecodeParams& p, const Ctx& c, uint32_t t
   };
 
   for (int s = s_begin; s < s_end; ++s) {
-    const Segment sg = load_segment(p, s);
+    const Segment sg = load_segment(p, c, s);
     if (sg.bad) {
       if (r == 0 && c.cta == 0) set_error(c.meta, MLA_DEVERR_SEQLEN);
       continue;
     }
+    // The plan was made for these lengths (off the critical path: these warps
+    // wait for the segment's first scores anyway).
+    if (r == 0 && c.cta == 0 && p.seqlens[sg.i] != sg.L) set_error(c.meta, MLA_DEVERR_PLAN);
     const int n = sg.b1 - sg.b0;
     const int q_row = c.cta * kRowsCta + hr;  // row within the 128-row tile
     const int row_g = sg.mt * kMTile + q_row;
@@ -889,22 +906,35 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
   MLA_PRO(2);
 
   // The plan must be the one built for this call's shape on this many pairs.
+  // The header, this pair's record (its first segment and where its segments
+  // start) and where they end are independent loads: one round trip.
   const int pair = static_cast<int>(blockIdx.x >> 1);
   const int pairs = static_cast<int>(gridDim.x >> 1);
-  const bool plan_ok = p.meta[kHMagic] == static_cast<int32_t>(kMagic) && p.meta[kHPairs] == pairs &&
-                       p.meta[kHBatch] == p.batch && p.meta[kHHq] == p.h_q && p.meta[kHSq] == p.s_q;
+  const MetaLayout lo = meta_layout(p.batch, p.h_q, p.s_q);
+  const int4 hdr0 = *reinterpret_cast<const int4*>(p.meta);               // magic, error, pairs, work rows
+  const int4 hdr2 = *reinterpret_cast<const int4*>(p.meta + 8);           // batch, kappa, splits, empties
+  const int4 hdr3 = *reinterpret_cast<const int4*>(p.meta + 12);          // h_q, s_q, cap, -
+  const int32_t* prec = p.meta + lo.pair_rec + kSegWords * pair;
+  const int4 rec0 = *reinterpret_cast<const int4*>(prec);
+  const int4 rec1 = *reinterpret_cast<const int4*>(prec + 4);
+  const int s_end_raw = p.meta[lo.pair_off + pair + 1];
+  static_assert(kHMagic == 0 && kHError == 1 && kHPairs == 2 && kHBatch == 8 && kHHq == 12 && kHSq == 13,
+                "header words read as int4s");
+  const bool plan_ok = hdr0.x == static_cast<int32_t>(kMagic) && hdr0.z == pairs && hdr2.x == p.batch &&
+                       hdr3.x == p.h_q && hdr3.y == p.s_q;
   int s_begin = 0, s_end = 0;
   if (plan_ok) {
-    const MetaLayout lo = meta_layout(p.batch, p.h_q, p.s_q);
-    s_begin = p.meta[lo.pair_off + pair];
-    s_end = p.meta[lo.pair_off + pair + 1];
+    s_begin = rec1.y;
+    s_end = s_end_raw;
     // Bits the plan raised (lengths past the table, slot overflow) go to the
     // sticky word too.
-    if (threadIdx.x == 0 && c.cta == 0 && pair == 0 && p.meta[kHError] != 0)
-      atomicOr(&g_mla_sticky_error, static_cast<unsigned int>(p.meta[kHError]));
+    if (threadIdx.x == 0 && c.cta == 0 && pair == 0 && hdr0.y != 0)
+      atomicOr(&g_mla_sticky_error, static_cast<unsigned int>(hdr0.y));
   } else if (threadIdx.x == 0 && c.cta == 0 && pair == 0) {
     set_error(c.meta, MLA_DEVERR_PLAN);
   }
+  c.s_begin = s_begin;
+  c.first = make_segment(p, rec0, rec1.x);
 
   if (threadIdx.x == 128) MLA_TRACE(11, 0);
 #ifdef MLA_DECODE_TRACE

@@ -26,7 +26,13 @@ constexpr uint32_t kMagic = 0x314C4D42u;  // "BML1"
 // Metadata: int32 words.
 //   header [kHdrWords]
 //   pair_off  [kMaxPairs + 1]           segment range of each pair
-//   segs      [W + kMaxPairs][4]        (work row, first page, end page, slot)
+//   pair_rec  [kMaxPairs][8]            per pair: its first segment's record
+//                                       (words 0-4, as in segs; work row -1 if
+//                                       it has none) and its first segment
+//                                       index (word 5), so a pair starts from
+//                                       one load
+//   segs      [W + kMaxPairs][8]        (work row, first page, end page, slot,
+//                                       length, 0, 0, 0)
 //   row_info  [W][2]                    (first slot or -1, pieces)
 //   split_rows [W]                      work rows cut into >1 pieces
 //   empty_rows [W]                      work rows with no pages
@@ -53,9 +59,11 @@ enum HeaderWord : int {
   kHdrWords = 32,
 };
 
+constexpr int kSegWords = 8;  // words of a segment record (pair_rec and segs)
+
 struct MetaLayout {
   int W;
-  size_t pair_off, segs, row_info, split_rows, empty_rows, tasks, words;
+  size_t pair_off, pair_rec, segs, row_info, split_rows, empty_rows, tasks, words;
 };
 
 __host__ __device__ inline int ceil_div(int a, int b) { return (a + b - 1) / b; }
@@ -64,8 +72,9 @@ __host__ __device__ inline MetaLayout meta_layout(int batch, int h_q, int s_q) {
   MetaLayout L;
   L.W = batch * ceil_div(s_q * h_q, kMTile);
   L.pair_off = kHdrWords;
-  L.segs = (L.pair_off + kMaxPairs + 1 + 3) & ~size_t(3);
-  L.row_info = L.segs + size_t(4) * (L.W + kMaxPairs);
+  L.pair_rec = (L.pair_off + kMaxPairs + 1 + 7) & ~size_t(7);
+  L.segs = L.pair_rec + size_t(kSegWords) * kMaxPairs;
+  L.row_info = L.segs + size_t(kSegWords) * (L.W + kMaxPairs);
   L.split_rows = L.row_info + size_t(2) * L.W;
   L.empty_rows = L.split_rows + L.W;
   L.tasks = (L.empty_rows + L.W + 3) & ~size_t(3);

@@ -103,13 +103,14 @@ struct Bounds {
   }
 };
 
-__device__ __forceinline__ int row_pages(const int32_t* seqlens, int batch, int w, int* err) {
+// Length of work row w's batch row (a negative length is flagged and read as 0).
+__device__ __forceinline__ int row_length(const int32_t* seqlens, int batch, int w, int* err) {
   int L = seqlens[w % batch];
   if (L < 0) {
     *err = 1;
     L = 0;
   }
-  return ceil_div(L, kPage);
+  return L;
 }
 
 __global__ void __launch_bounds__(kSchedThreads) mla_sched_kernel(const int32_t* __restrict__ seqlens, int batch,
@@ -130,6 +131,7 @@ __global__ void __launch_bounds__(kSchedThreads) mla_sched_kernel(const int32_t*
   const int R = s_q * h_q;
   const int n_mt = ceil_div(R, kMTile);
   int32_t* pair_off = meta + lo.pair_off;
+  int32_t* pair_rec = meta + lo.pair_rec;
   int32_t* segs = meta + lo.segs;
   int32_t* row_info = meta + lo.row_info;
   int32_t* split_rows = meta + lo.split_rows;
@@ -148,16 +150,17 @@ __global__ void __launch_bounds__(kSchedThreads) mla_sched_kernel(const int32_t*
   // Pass 1: total cost T.  With at most one row per thread, the row's pages
   // and cost prefix are kept for pass 2 instead of being read and scanned
   // again.
-  int n_own = 0;
+  int L_own = 0, n_own = 0;
   long long C_own = 0, T = 0;
   if (one_chunk) {
-    n_own = threadIdx.x < W ? row_pages(seqlens, batch, threadIdx.x, &err) : 0;
+    L_own = threadIdx.x < W ? row_length(seqlens, batch, threadIdx.x, &err) : 0;
+    n_own = ceil_div(L_own, kPage);
     C_own = block_exclusive_scan<long long>(n_own > 0 ? n_own + kKappa : 0, s_wl, &s_tot_l);
     T = s_tot_l;
   } else {
     long long local = 0;
     for (int w = threadIdx.x; w < W; w += kSchedThreads) {
-      const int n = row_pages(seqlens, batch, w, &err);
+      const int n = ceil_div(row_length(seqlens, batch, w, &err), kPage);
       if (n > 0) local += n + kKappa;
     }
     block_exclusive_scan<long long>(local, s_wl, &s_tot_l);
@@ -175,14 +178,16 @@ __global__ void __launch_bounds__(kSchedThreads) mla_sched_kernel(const int32_t*
   for (int base = 0; base < W; base += kSchedThreads) {
     const int w = base + threadIdx.x;
     const bool in = w < W;
-    int n;
+    int L, n;
     long long C, chunk_cost;
     if (one_chunk) {
+      L = L_own;
       n = n_own;
       C = C_own;
       chunk_cost = T;
     } else {
-      n = in ? row_pages(seqlens, batch, w, &err) : 0;
+      L = in ? row_length(seqlens, batch, w, &err) : 0;
+      n = ceil_div(L, kPage);
       C = carry_cost + block_exclusive_scan<long long>(n > 0 ? n + kKappa : 0, s_wl, &s_tot_l);
       chunk_cost = s_tot_l;
     }
@@ -218,7 +223,9 @@ __global__ void __launch_bounds__(kSchedThreads) mla_sched_kernel(const int32_t*
         sg.y = b0 > 0 ? static_cast<int>(b0) : 0;
         sg.z = b1 < n ? static_cast<int>(b1) : n;
         sg.w = pieces > 1 ? slot0 + k : -1;
-        *reinterpret_cast<int4*>(segs + 4 * (seg0 + k)) = sg;
+        int32_t* rec = segs + kSegWords * (seg0 + k);
+        *reinterpret_cast<int4*>(rec) = sg;
+        *reinterpret_cast<int4*>(rec + 4) = make_int4(L, 0, 0, 0);
       }
       if (pieces > 1) {
         split_rows[split_i] = w;
@@ -228,11 +235,31 @@ __global__ void __launch_bounds__(kSchedThreads) mla_sched_kernel(const int32_t*
       // Pair p's segments start with the first one on a pair >= p.  When
       // B(p) falls in this row's cost range [C, C + c), every segment of the
       // rows before sits on a pair < p, and of this row's pieces (pairs f,
-      // f + 1, ...) those before pair p; later rows start at or past p.
+      // f + 1, ...) those before pair p; later rows start at or past p.  Its
+      // first segment is then this row's piece p - f (a pair p < f ends
+      // inside the row's fixed-cost positions and has no segment at all).
       if (c > 0) {
+        const long long p_begin = bd.first_at_or_past(C);
         const long long p_end = bd.first_at_or_past(C + c);
-        for (long long p = bd.first_at_or_past(C); p < p_end && p < pairs; ++p)
-          pair_off[p] = seg0 + (p > f ? static_cast<int>(p - f) : 0);
+        long long bq, br;
+        bd.at(p_begin, &bq, &br);
+        for (long long p = p_begin; p < p_end && p < pairs; ++p) {
+          const long long b0 = bq - C - kKappa;
+          bd.next(p, &bq, &br);
+          const long long b1 = bq - C - kKappa;
+          const int s0 = seg0 + (p > f ? static_cast<int>(p - f) : 0);
+          pair_off[p] = s0;
+          int32_t* rec = pair_rec + kSegWords * p;
+          if (p >= f) {
+            *reinterpret_cast<int4*>(rec) =
+                make_int4(w, b0 > 0 ? static_cast<int>(b0) : 0, b1 < n ? static_cast<int>(b1) : n,
+                          pieces > 1 ? slot0 + static_cast<int>(p - f) : -1);
+            *reinterpret_cast<int4*>(rec + 4) = make_int4(L, s0, 0, 0);
+          } else {
+            *reinterpret_cast<int4*>(rec) = make_int4(-1, 0, 0, -1);
+            *reinterpret_cast<int4*>(rec + 4) = make_int4(0, s0, 0, 0);
+          }
+        }
       }
     }
     carry_cost += chunk_cost;
@@ -245,8 +272,15 @@ __global__ void __launch_bounds__(kSchedThreads) mla_sched_kernel(const int32_t*
   // Pairs whose range starts at the total cost (the end marker, and when
   // T < P the pairs past T) take no segment.
   const long long p_tail = bd.first_at_or_past(T);
-  for (int p = threadIdx.x; p <= pairs; p += kSchedThreads)
-    if (p >= p_tail) pair_off[p] = carry_seg;
+  for (int p = threadIdx.x; p <= pairs; p += kSchedThreads) {
+    if (p >= p_tail) {
+      pair_off[p] = carry_seg;
+      if (p < pairs) {
+        *reinterpret_cast<int4*>(pair_rec + kSegWords * p) = make_int4(-1, 0, 0, -1);
+        *reinterpret_cast<int4*>(pair_rec + kSegWords * p + 4) = make_int4(0, carry_seg, 0, 0);
+      }
+    }
+  }
   __syncthreads();  // s_err
 
   if (threadIdx.x == 0) {

@@ -95,12 +95,14 @@ def decode_plan(meta, batch, h_q, s_q):
     W = int(m[3])
     nseg = int(m[4])
     hdr, maxp = 32, 160
-    seg0 = (hdr + maxp + 1 + 3) & ~3
-    row0 = seg0 + 4 * (W + maxp)
+    rec0 = (hdr + maxp + 1 + 7) & ~7
+    seg0 = rec0 + 8 * maxp
+    row0 = seg0 + 8 * (W + maxp)
     split0 = row0 + 2 * W
     empty0 = split0 + W
     tasks0 = (empty0 + W + 3) & ~3
-    segs = m[seg0:seg0 + 4 * nseg].reshape(nseg, 4)
+    recs = m[seg0:seg0 + 8 * nseg].reshape(nseg, 8)
+    segs = recs[:, :4]
     pair_off = m[hdr:hdr + P + 1].tolist()
     seg_pair = []
     for p in range(P):
@@ -114,6 +116,8 @@ def decode_plan(meta, batch, h_q, s_q):
         "split_rows": [int(v) for v in m[split0:split0 + int(m[10])]],
         "empty_rows": [int(v) for v in m[empty0:empty0 + int(m[11])]],
         "tasks": [tuple(int(v) for v in t) for t in m[tasks0:tasks0 + 4 * int(m[10])].reshape(-1, 4)],
+        "seg_lengths": [int(v) for v in recs[:, 4]],
+        "pair_records": m[rec0:rec0 + 8 * P].reshape(P, 8),
     }
 
 
@@ -141,6 +145,18 @@ def test_plan_matches_oracle_bit_for_bit(lens, h_q, s_q):
         assert got[key] == want_v, key
     # one combine task per split row: (work row, first slot, pieces, 0)
     assert got["tasks"] == [(w, want["slot_base"][w], want["pieces"][w], 0) for w in want["split_rows"]]
+    # every segment carries its row's length; every pair's record holds its first segment
+    b = len(lens)
+    assert got["seg_lengths"] == [max(lens[w % b], 0) for (w, *_rest) in want["segments"]]
+    for p in range(got["num_pairs"]):
+        rec = [int(v) for v in got["pair_records"][p]]
+        s0, s1 = want["pair_offsets"][p], want["pair_offsets"][p + 1]
+        assert rec[5] == s0
+        if s0 < s1:
+            w, b0, b1, slot = want["segments"][s0]
+            assert rec[:5] == [w, b0, b1, slot, max(lens[w % b], 0)]
+        else:
+            assert rec[0] == -1
 
 
 def test_num_sm_pairs_is_half_the_sms():

@@ -96,3 +96,16 @@ def test_clean_calls_leave_the_sticky_word_clear():
     for _ in range(3):
         _decode(x)
     assert binding.mla_take_device_errors() == 0
+
+
+def test_lengths_changed_since_the_plan_are_flagged():
+    binding.mla_take_device_errors()
+    x = inputs.make_inputs([900, 300, 1200], 64, seed=1600)
+    g = x.to("cuda")
+    meta = binding.mla_get_metadata(g.seqlens, g.h_q, g.s_q)
+    changed = g.seqlens.clone()
+    changed[2] -= 100  # same pages table, shorter row: the plan no longer matches
+    binding.mla_decode(g.q, g.kv_cache, g.block_table, changed, g.softmax_scale, g.causal, meta)
+    torch.cuda.synchronize()
+    assert binding.mla_check_device_error(meta) & binding.MLA_DEVERR_PLAN
+    assert binding.mla_take_device_errors() & binding.MLA_DEVERR_PLAN
