@@ -36,7 +36,7 @@ __device__ unsigned long long g_mla_sched_times[3];
 
 namespace {
 
-constexpr int kSchedThreads = 1024;
+constexpr int kSchedThreads = 1024;  // the most threads a launch uses (and rows per chunk)
 constexpr int kWarps = kSchedThreads / 32;
 
 // Block-wide exclusive scan of one value per thread; returns the exclusive
@@ -53,15 +53,16 @@ __device__ T block_exclusive_scan(T v, T* warp_tot, T* total) {
   if (lane == 31) warp_tot[warp] = incl;
   __syncthreads();
   if (warp == 0) {
-    T t = lane < kWarps ? warp_tot[lane] : T(0);
+    const int nwarps = static_cast<int>(blockDim.x >> 5);
+    T t = lane < nwarps ? warp_tot[lane] : T(0);
     T ti = t;
 #pragma unroll
     for (int off = 1; off < 32; off <<= 1) {
       const T o = __shfl_up_sync(0xffffffffu, ti, off);
       if (lane >= off) ti += o;
     }
-    if (lane < kWarps) warp_tot[lane] = ti - t;  // exclusive warp offsets
-    if (lane == kWarps - 1) *total = ti;
+    if (lane < nwarps) warp_tot[lane] = ti - t;  // exclusive warp offsets
+    if (lane == nwarps - 1) *total = ti;
   }
   __syncthreads();
   const T res = warp_tot[warp] + incl - v;
@@ -71,39 +72,27 @@ __device__ T block_exclusive_scan(T v, T* warp_tot, T* total) {
 
 // The pairs' cost boundaries B(p) (see the header), the pair owning cost
 // position x (B(p) <= x < B(p + 1)), and the first pair p with B(p) >= x.
-// next() steps (B(p), its remainder) to B(p + 1) without a division.
 struct Bounds {
   long long T;
   int P;
-  long long tq, tr;  // T / P and T % P
-  __device__ Bounds(long long T_, int P_) : T(T_), P(P_), tq(T_ / P_), tr(T_ % P_) {}
+  __device__ Bounds(long long T_, int P_) : T(T_), P(P_) {}
+  __device__ long long b(long long p) const { return T >= P ? (p * T) / P : (p < T ? p : T); }
   __device__ long long owner(long long x) const { return T >= P ? ((x + 1) * P - 1) / T : x; }
   __device__ long long first_at_or_past(long long x) const { return T >= P ? (x * P + T - 1) / T : x; }
-  // B(p) as a quotient and remainder of p * T / P.
-  __device__ void at(long long p, long long* q, long long* r) const {
-    if (T >= P) {
-      *q = (p * T) / P;
-      *r = p * T - *q * P;
-    } else {
-      *q = p < T ? p : T;
-      *r = 0;
-    }
-  }
-  __device__ void next(long long p, long long* q, long long* r) const {  // from B(p) to B(p + 1)
-    if (T >= P) {
-      *q += tq;
-      *r += tr;
-      if (*r >= P) {
-        *r -= P;
-        ++*q;
-      }
-    } else {
-      *q = p + 1 < T ? p + 1 : T;
-    }
-  }
 };
 
 // Length of work row w's batch row (a negative length is flagged and read as 0).
+// One work row of a chunk, as the segment and pair writers need it.
+struct RowPlan {
+  long long C;  // cost before the row
+  long long c;  // its cost (0 for an empty row)
+  int L, n;     // length and pages
+  int f;        // pair of its first page
+  int pieces;
+  int seg0;     // its first segment, counted from the chunk's first
+  int slot0;    // its first partial slot (split rows)
+};
+
 __device__ __forceinline__ int row_length(const int32_t* seqlens, int batch, int w, int* err) {
   int L = seqlens[w % batch];
   if (L < 0) {
@@ -143,9 +132,11 @@ __global__ void __launch_bounds__(kSchedThreads) mla_sched_kernel(const int32_t*
   __shared__ long long s_tot_l;
   __shared__ unsigned long long s_tot_p;
   __shared__ int s_err;
+  __shared__ RowPlan s_row[kSchedThreads];
   if (threadIdx.x == 0) s_err = 0;
   int err = 0;
-  const bool one_chunk = W <= kSchedThreads;
+  const int nthr = static_cast<int>(blockDim.x);  // a multiple of 32, at most kSchedThreads
+  const bool one_chunk = W <= nthr;
 
   // Pass 1: total cost T.  With at most one row per thread, the row's pages
   // and cost prefix are kept for pass 2 instead of being read and scanned
@@ -159,7 +150,7 @@ __global__ void __launch_bounds__(kSchedThreads) mla_sched_kernel(const int32_t*
     T = s_tot_l;
   } else {
     long long local = 0;
-    for (int w = threadIdx.x; w < W; w += kSchedThreads) {
+    for (int w = threadIdx.x; w < W; w += nthr) {
       const int n = ceil_div(row_length(seqlens, batch, w, &err), kPage);
       if (n > 0) local += n + kKappa;
     }
@@ -175,7 +166,7 @@ __global__ void __launch_bounds__(kSchedThreads) mla_sched_kernel(const int32_t*
   // each stays below 1024 + pairs.
   long long carry_cost = 0;
   int carry_seg = 0, carry_slot = 0, carry_split = 0, carry_empty = 0;
-  for (int base = 0; base < W; base += kSchedThreads) {
+  for (int base = 0; base < W; base += nthr) {
     const int w = base + threadIdx.x;
     const bool in = w < W;
     int L, n;
@@ -211,57 +202,69 @@ __global__ void __launch_bounds__(kSchedThreads) mla_sched_kernel(const int32_t*
     if (in) {
       row_info[2 * w + 0] = pieces > 1 ? slot0 : -1;
       row_info[2 * w + 1] = pieces;
-      long long bq, br;  // B(p) of the piece's pair p, stepped along
-      bd.at(f, &bq, &br);
-      for (int k = 0; k < pieces; ++k) {
-        const long long p = f + k;
-        const long long b0 = bq - C - kKappa;
-        bd.next(p, &bq, &br);
-        const long long b1 = bq - C - kKappa;
-        int4 sg;
-        sg.x = w;
-        sg.y = b0 > 0 ? static_cast<int>(b0) : 0;
-        sg.z = b1 < n ? static_cast<int>(b1) : n;
-        sg.w = pieces > 1 ? slot0 + k : -1;
-        int32_t* rec = segs + kSegWords * (seg0 + k);
-        *reinterpret_cast<int4*>(rec) = sg;
-        *reinterpret_cast<int4*>(rec + 4) = make_int4(L, 0, 0, 0);
-      }
       if (pieces > 1) {
         split_rows[split_i] = w;
         *reinterpret_cast<int4*>(tasks + 4 * split_i) = make_int4(w, slot0, pieces, 0);
       }
       if (n == 0) empty_rows[empty_i] = w;
-      // Pair p's segments start with the first one on a pair >= p.  When
-      // B(p) falls in this row's cost range [C, C + c), every segment of the
-      // rows before sits on a pair < p, and of this row's pieces (pairs f,
-      // f + 1, ...) those before pair p; later rows start at or past p.  Its
-      // first segment is then this row's piece p - f (a pair p < f ends
-      // inside the row's fixed-cost positions and has no segment at all).
-      if (c > 0) {
-        const long long p_begin = bd.first_at_or_past(C);
-        const long long p_end = bd.first_at_or_past(C + c);
-        long long bq, br;
-        bd.at(p_begin, &bq, &br);
-        for (long long p = p_begin; p < p_end && p < pairs; ++p) {
-          const long long b0 = bq - C - kKappa;
-          bd.next(p, &bq, &br);
-          const long long b1 = bq - C - kKappa;
-          const int s0 = seg0 + (p > f ? static_cast<int>(p - f) : 0);
-          pair_off[p] = s0;
-          int32_t* rec = pair_rec + kSegWords * p;
-          if (p >= f) {
-            *reinterpret_cast<int4*>(rec) =
-                make_int4(w, b0 > 0 ? static_cast<int>(b0) : 0, b1 < n ? static_cast<int>(b1) : n,
-                          pieces > 1 ? slot0 + static_cast<int>(p - f) : -1);
-            *reinterpret_cast<int4*>(rec + 4) = make_int4(L, s0, 0, 0);
-          } else {
-            *reinterpret_cast<int4*>(rec) = make_int4(-1, 0, 0, -1);
-            *reinterpret_cast<int4*>(rec + 4) = make_int4(0, s0, 0, 0);
-          }
-        }
+    }
+    // The chunk's rows to shared memory; then every segment and every pair
+    // whose range starts in the chunk is written by a thread of its own (a
+    // long row's pieces and pairs would otherwise be one thread's serial
+    // work), which finds its row by binary search.
+    s_row[threadIdx.x] = RowPlan{C, c, L, n, f, pieces, seg0 - carry_seg, slot0};
+    __syncthreads();
+    const int rows_here = min(nthr, W - base);
+    const int segs_here = static_cast<int>(tot & 0xffffu);
+    for (int j = threadIdx.x; j < segs_here; j += nthr) {
+      // the last row whose first segment is at or before j (it has pieces)
+      int lo_r = 0, hi_r = rows_here - 1;
+      while (lo_r < hi_r) {
+        const int mid = (lo_r + hi_r + 1) >> 1;
+        if (s_row[mid].seg0 <= j) lo_r = mid; else hi_r = mid - 1;
+      }
+      const RowPlan& rp = s_row[lo_r];
+      const int k = j - rp.seg0;
+      const long long p = rp.f + k;
+      const long long b0 = bd.b(p) - rp.C - kKappa;
+      const long long b1 = bd.b(p + 1) - rp.C - kKappa;
+      int32_t* rec = segs + kSegWords * (carry_seg + j);
+      *reinterpret_cast<int4*>(rec) =
+          make_int4(base + lo_r, b0 > 0 ? static_cast<int>(b0) : 0, b1 < rp.n ? static_cast<int>(b1) : rp.n,
+                    rp.pieces > 1 ? rp.slot0 + k : -1);
+      *reinterpret_cast<int4*>(rec + 4) = make_int4(rp.L, 0, 0, 0);
+    }
+    // Pair p's segments start with the first one on a pair >= p.  When B(p)
+    // falls in a row's cost range [C, C + c), every segment of the rows
+    // before sits on a pair < p, and of this row's pieces (pairs f, f + 1,
+    // ...) those before pair p; later rows start at or past p.  Its first
+    // segment is then this row's piece p - f (a pair p < f ends inside the
+    // row's fixed-cost positions and has no segment at all).
+    for (int p = threadIdx.x; p < pairs; p += nthr) {
+      const long long x = bd.b(p);
+      if (x < carry_cost || x >= carry_cost + chunk_cost) continue;
+      int lo_r = 0, hi_r = rows_here - 1;  // the last row whose cost range starts at or before x
+      while (lo_r < hi_r) {
+        const int mid = (lo_r + hi_r + 1) >> 1;
+        if (s_row[mid].C <= x) lo_r = mid; else hi_r = mid - 1;
+      }
+      const RowPlan& rp = s_row[lo_r];
+      const int s0 = carry_seg + rp.seg0 + (p > rp.f ? p - rp.f : 0);
+      pair_off[p] = s0;
+      int32_t* rec = pair_rec + kSegWords * p;
+      if (p >= rp.f) {
+        const long long b0 = x - rp.C - kKappa;
+        const long long b1 = bd.b(p + 1) - rp.C - kKappa;
+        *reinterpret_cast<int4*>(rec) =
+            make_int4(base + lo_r, b0 > 0 ? static_cast<int>(b0) : 0, b1 < rp.n ? static_cast<int>(b1) : rp.n,
+                      rp.pieces > 1 ? rp.slot0 + (p - rp.f) : -1);
+        *reinterpret_cast<int4*>(rec + 4) = make_int4(rp.L, s0, 0, 0);
+      } else {
+        *reinterpret_cast<int4*>(rec) = make_int4(-1, 0, 0, -1);
+        *reinterpret_cast<int4*>(rec + 4) = make_int4(0, s0, 0, 0);
       }
     }
+    __syncthreads();  // s_row is rewritten by the next chunk
     carry_cost += chunk_cost;
     carry_seg += static_cast<int>(tot & 0xffffu);
     carry_slot += static_cast<int>((tot >> 16) & 0xffffu);
@@ -272,7 +275,7 @@ __global__ void __launch_bounds__(kSchedThreads) mla_sched_kernel(const int32_t*
   // Pairs whose range starts at the total cost (the end marker, and when
   // T < P the pairs past T) take no segment.
   const long long p_tail = bd.first_at_or_past(T);
-  for (int p = threadIdx.x; p <= pairs; p += kSchedThreads) {
+  for (int p = threadIdx.x; p <= pairs; p += nthr) {
     if (p >= p_tail) {
       pair_off[p] = carry_seg;
       if (p < pairs) {
@@ -320,7 +323,13 @@ cudaError_t launch_sched(const int32_t* seqlens, int batch, int h_q, int s_q, in
                          cudaStream_t stream) {
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(1, 1, 1);
-  cfg.blockDim = dim3(kSchedThreads, 1, 1);
+  // One thread per work row (and at least one per pair), up to kSchedThreads:
+  // small plans then pay for few warps at every block-wide scan.
+  const int W = batch * ceil_div(s_q * h_q, kMTile);
+  int threads = (W > pairs + 1 ? W : pairs + 1) + 31;
+  threads = threads & ~31;
+  if (threads > kSchedThreads) threads = kSchedThreads;
+  cfg.blockDim = dim3(static_cast<unsigned>(threads), 1, 1);
   cfg.stream = stream;
   cudaLaunchAttribute attr[1];
   attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
