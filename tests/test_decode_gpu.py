@@ -284,3 +284,51 @@ def test_workload_full_size_sampled_rows(index):
     rows = list(range(x.batch)) if x.batch <= 4 else _sample_rows(x, seed=index)
     assert_parity(x, out, lse, rows=rows, strict=True)
     assert torch.isfinite(out.float()).all()
+
+
+def test_one_plan_serves_many_calls():
+    """The plan is made once per decode step and reused by every layer: calls
+    on one metadata buffer with different queries and caches (same lengths)
+    each match the oracle, the split rows' merge included."""
+    lens = [3000, 70, 1500, 4100, 900]
+    xs = [inputs.make_inputs(lens, 128, seed=1700 + k) for k in range(3)]
+    g0 = xs[0].to("cuda")
+    meta = binding.mla_get_metadata(g0.seqlens, g0.h_q, g0.s_q)
+    for x in xs * 2:
+        g = x.to("cuda")
+        out, lse = binding.mla_decode(g.q, g.kv_cache, g.block_table, g.seqlens, g.softmax_scale, g.causal, meta)
+        torch.cuda.synchronize()
+        assert binding.mla_check_device_error(meta) == 0
+        assert_parity(x, out.cpu(), lse.cpu())
+
+
+def test_graph_replays_on_one_plan():
+    """A CUDA graph of the decode call, replayed on one plan: the merge's
+    per-call bookkeeping lives on the device, so every replay is right."""
+    x = inputs.make_inputs([2000, 333, 5000], 64, seed=1800)
+    g = x.to("cuda")
+    meta = binding.mla_get_metadata(g.seqlens, g.h_q, g.s_q)
+    ws = torch.empty(binding.mla_workspace_bytes(3, 64, 1), dtype=torch.uint8, device="cuda")
+    out = torch.empty(3, 1, 64, 512, dtype=torch.bfloat16, device="cuda")
+    lse = torch.empty(3, 64, 1, dtype=torch.float32, device="cuda")
+    q_alt = inputs.make_inputs([2000, 333, 5000], 64, seed=1801).q.to("cuda")
+    q_buf = g.q.clone()
+    st = torch.cuda.Stream()
+    with torch.cuda.stream(st):
+        binding.mla_decode(q_buf, g.kv_cache, g.block_table, g.seqlens, g.softmax_scale, g.causal, meta,
+                           workspace=ws, out=out, lse=lse, stream=st)
+    st.synchronize()
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph, stream=st):
+        binding.mla_decode(q_buf, g.kv_cache, g.block_table, g.seqlens, g.softmax_scale, g.causal, meta,
+                           workspace=ws, out=out, lse=lse, stream=st)
+    x_alt = inputs.DecodeInputs(**{**x.__dict__, "q": q_alt.cpu()})
+    for k in range(4):
+        src = x_alt if k % 2 else x
+        with torch.cuda.stream(st):
+            q_buf.copy_(src.q.to("cuda"))
+            graph.replay()
+        st.synchronize()
+        assert binding.mla_check_device_error(meta) == 0
+        assert_parity(src, out.cpu(), lse.cpu())
+    del graph
