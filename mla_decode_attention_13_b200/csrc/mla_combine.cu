@@ -94,41 +94,45 @@ __global__ void __launch_bounds__(kCombineThreads, 4) mla_combine_kernel(const C
   if (threadIdx.x == 0) atomicMin(&g_mla_comb_times[0], ptx::globaltimer());
 #endif
   ptx::griddep_launch_dependents();
-  ptx::griddep_wait();  // the decode kernel's partials and the plan are complete
-#ifdef MLA_DECODE_TRACE
-  if (threadIdx.x == 0) atomicMin(&g_mla_comb_times[1], ptx::globaltimer());
-#endif
+  // The plan is complete before this grid launches (the decode kernel lets it
+  // launch only after its own wait for the plan), so the plan's words and this
+  // warp's first task are read now; only the partials wait for the decode
+  // kernel's completion.
   const int32_t* meta = p.meta;
   const MetaLayout lo = meta_layout(p.batch, p.h_q, p.s_q);
   // Only a plan built for this call's shape on this many pairs is used.
-  if (meta[kHMagic] != static_cast<int32_t>(kMagic) || meta[kHBatch] != p.batch || meta[kHHq] != p.h_q ||
-      meta[kHSq] != p.s_q || meta[kHPairs] != p.pairs)
-    return;
+  const bool plan_ok = meta[kHMagic] == static_cast<int32_t>(kMagic) && meta[kHBatch] == p.batch &&
+                       meta[kHHq] == p.h_q && meta[kHSq] == p.s_q && meta[kHPairs] == p.pairs;
   const int n_split = meta[kHSplitRows];
   const int n_empty = meta[kHEmptyRows];
   const int W = lo.W;
-  if (n_split < 0 || n_split > W || n_empty < 0 || n_empty > W) return;
   const int per_row = p.tile_rows * S;
-  const int n_items = (n_split + n_empty) * per_row;
   const int lane = threadIdx.x & 31;
   const int warp_g = blockIdx.x * kWarpsPerCta + (threadIdx.x >> 5);
   const int stride = gridDim.x * kWarpsPerCta;
+  const bool counts_ok = plan_ok && n_split >= 0 && n_split <= W && n_empty >= 0 && n_empty <= W;
+  const int n_items = counts_ok ? (n_split + n_empty) * per_row : 0;
+  // A work row's task: (work row, first slot, pieces) for a split row, or the
+  // work row alone for an empty one.
+  auto task_of = [&](int k) -> int4 {
+    if (k < n_split) return *reinterpret_cast<const int4*>(meta + lo.tasks + 4 * k);
+    return make_int4(meta[lo.empty_rows + (k - n_split)], 0, 0, 0);
+  };
+  int4 first_task = make_int4(-1, 0, 0, 0);
+  if (warp_g < n_items) first_task = task_of(warp_g / per_row);
+  ptx::griddep_wait();  // the decode kernel's partials are complete
+#ifdef MLA_DECODE_TRACE
+  if (threadIdx.x == 0) atomicMin(&g_mla_comb_times[1], ptx::globaltimer());
+#endif
 
   for (int item = warp_g; item < n_items; item += stride) {
     const int k = item / per_row;
     const int rem = item - k * per_row;
     const int r = rem / S;
     const int slice = rem - r * S;
-    int w, base = 0, pieces = 0;
-    if (k < n_split) {
-      const int4 task = *reinterpret_cast<const int4*>(meta + lo.tasks + 4 * k);
-      w = task.x;
-      base = task.y;
-      pieces = task.z;
-      if (base < 0 || pieces < 2 || base + pieces > p.max_slots) continue;
-    } else {
-      w = meta[lo.empty_rows + (k - n_split)];
-    }
+    const int4 task = item == warp_g ? first_task : task_of(k);
+    const int w = task.x, base = task.y, pieces = task.z;
+    if (k < n_split && (base < 0 || pieces < 2 || base + pieces > p.max_slots)) continue;
     if (w < 0 || w >= W) continue;
     const int i = w % p.batch;
     const int mt = w / p.batch;

@@ -900,9 +900,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
   // Programmatic dependent launch: the set-up above overlapped the previous
   // kernel (the plan, or the previous call's combine); wait for its
   // completion before reading the plan or writing any output.  The combine
-  // may start launching now (it waits for this kernel in turn).
-  griddep_launch_dependents();
+  // may launch from then on: it reads the plan at once and waits for this
+  // kernel only before it reads the partials.
   griddep_wait();
+  griddep_launch_dependents();
   MLA_PRO(2);
 
   // The plan must be the one built for this call's shape on this many pairs.
