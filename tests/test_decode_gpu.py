@@ -126,6 +126,8 @@ PLAN_CASES = [
     ([1] * 300, 64, 1), ([77, 64, 65, 129, 4000, 1, 0, 99999], 128, 3), (list(range(0, 4000, 37)), 32, 2),
     # more than 1024 work rows: the plan kernel's chunked path
     ([(37 * k) % 900 for k in range(1100)], 64, 1), ([0, 1, 64, 65, 4000] * 250, 128, 2),
+    # a total cost past 2^32 / (pairs + 1): the plan's 64-bit quotients (a plan reads only the lengths)
+    ([3_600_000] * 1100, 128, 1),
 ]
 
 
