@@ -199,6 +199,50 @@ int mla_decode_noalloc(const void* q, const void* kv_cache, int64_t num_pages, c
                        float softmax_scale, int causal, void* out, float* lse, void* metadata, void* stream);
 
 /*
+ * The projections either side of the absorbed decode.  "MLA 和 MHA 的 Kernel
+ * 区别", section "内存布局和 KV Cache 大小 / MLA": a head's keys and values are
+ * up-projections of the cached latent, K^h = c W_UK^h and V^h = c W_UV^h.
+ * Since <q_nope^h, c W_UK^h> = <W_UK^h q_nope^h, c> (W_UK^h taken as [512][128]
+ * with the latent index first) and sum_j p_j c_j W_UV^h = (sum_j p_j c_j)
+ * W_UV^h, both matrices move off the cache: onto the query before the decode
+ * (mla_absorb_q) and onto the latent output after it (mla_up_project), which
+ * leaves the decode above reading each cached row once.  Both are batched
+ * GEMMs over the heads on the tensor cores (fp32 accumulation, bf16 results).
+ *
+ * mla_absorb_q: for every token t and head h
+ *     q_out[t][h][0:512]   = W_UK^h q_nope[t][h]      (sum over 128 columns)
+ *     q_out[t][h][512:576] = q_rope[t][h]             (copied)
+ * so that q_out is mla_decode's q (t = i * s_q + token).
+ *   q_nope  [device] bf16 [tokens][h_q][128].
+ *   q_rope  [device] bf16 [tokens][h_q][64].
+ *   w_uk    [device] bf16 [h_q][512][128]: w_uk[h][c][n] is W_UK^h's entry for
+ *           latent dim c and no-position dim n.
+ *   tokens  >= 1 rows of every tensor; at most 65535 * 128.
+ *   h_q     1..128.
+ *   q_out   [device] bf16 [tokens][h_q][576].
+ * Every pointer 16-byte aligned.  Returns MLA_ERR_ARG for a NULL or misaligned
+ * pointer or a count below 1, MLA_ERR_UNSUPPORTED for h_q or tokens past the
+ * limits, MLA_ERR_UNSUPPORTED / MLA_ERR_CUDA if the device is not sm_100 or a
+ * launch failed.  A kernel wait that ran past its time limit leaves q_out
+ * unwritten for that head and token tile and sets MLA_DEVERR_TIMEOUT in the
+ * bits mla_take_device_errors reports.
+ */
+int mla_absorb_q(const void* q_nope, const void* q_rope, const void* w_uk, int tokens, int h_q, void* q_out,
+                 void* stream);
+
+/*
+ * mla_up_project: for every token t and head h
+ *     o_out[t][h][v] = sum_c o_latent[t][h][c] * W_UV^h[c][v]
+ * where o_latent is mla_decode's out (t = i * s_q + token).
+ *   o_latent [device] bf16 [tokens][h_q][512].
+ *   w_uv     [device] bf16 [h_q][512][128]: w_uv[h][c][v] is W_UV^h's entry
+ *            for latent dim c and value dim v.
+ *   tokens, h_q, errors: as mla_absorb_q.
+ *   o_out    [device] bf16 [tokens][h_q][128].
+ */
+int mla_up_project(const void* o_latent, const void* w_uv, int tokens, int h_q, void* o_out, void* stream);
+
+/*
  * Synchronise `stream` and read the device error word from `metadata`.
  * Writes the word to *error_word (if not NULL).  Returns MLA_OK when it is
  * zero, MLA_ERR_DEVICE when not, MLA_ERR_CUDA if the copy or sync failed.
@@ -207,7 +251,8 @@ int mla_check_device_error(const void* metadata, void* stream, uint32_t* error_w
 
 /*
  * The error bits any call raised on the current device since the last
- * mla_take_device_errors, whatever metadata buffer it used: unlike the word in
+ * mla_take_device_errors, whatever metadata buffer it used (and those of
+ * mla_absorb_q and mla_up_project, which have none): unlike the word in
  * `metadata`, which the next mla_get_metadata on that buffer rewrites, these
  * bits stay set until taken.  For callers that replay many steps (a captured
  * graph, a benchmark loop) and check once at the end.  Enqueues an atomic

@@ -37,6 +37,8 @@ EXPORTED = (
     "mla_decode",
     "mla_decode_timed",
     "mla_decode_noalloc",
+    "mla_absorb_q",
+    "mla_up_project",
     "mla_check_device_error",
     "mla_take_device_errors",
     "mla_error_string",
@@ -76,6 +78,10 @@ def lib() -> ctypes.CDLL:
         L.mla_decode_timed.argtypes = dec + [_vp, _vp]
         L.mla_decode_noalloc.restype = ctypes.c_int
         L.mla_decode_noalloc.argtypes = dec[:14] + [_vp]
+        L.mla_absorb_q.restype = ctypes.c_int
+        L.mla_absorb_q.argtypes = [_vp, _vp, _vp, ctypes.c_int, ctypes.c_int, _vp, _vp]
+        L.mla_up_project.restype = ctypes.c_int
+        L.mla_up_project.argtypes = [_vp, _vp, ctypes.c_int, ctypes.c_int, _vp, _vp]
         L.mla_check_device_error.restype = ctypes.c_int
         L.mla_check_device_error.argtypes = [_vp, _vp, ctypes.POINTER(ctypes.c_uint32)]
         L.mla_take_device_errors.restype = ctypes.c_int
@@ -196,6 +202,60 @@ def mla_decode_noalloc(q: torch.Tensor, kv_cache: torch.Tensor, block_table: tor
                                     int(block_table.shape[1]), _ptr(seqlens), batch, s_q, h_q, float(softmax_scale),
                                     int(bool(causal)), _ptr(out), _ptr(lse), _ptr(metadata), _stream_ptr(stream)))
     return out, lse
+
+
+def _projection_shapes(func: str, x: torch.Tensor, cols: int, w: torch.Tensor) -> Tuple[int, int]:
+    """(tokens, h_q) of x [..., h_q, cols] against weights [h_q, 512, 128]."""
+    if x.dim() < 2 or x.shape[-1] != cols or x.dtype != torch.bfloat16 or not x.is_contiguous():
+        raise MLAError(func, MLA_ERR_ARG)
+    h_q = int(x.shape[-2])
+    if tuple(w.shape) != (h_q, 512, 128) or w.dtype != torch.bfloat16 or not w.is_contiguous():
+        raise MLAError(func, MLA_ERR_ARG)
+    tokens = x.numel() // (h_q * cols)
+    return tokens, h_q
+
+
+def mla_absorb_q(q_nope: torch.Tensor, q_rope: torch.Tensor, w_uk: torch.Tensor, out: Optional[torch.Tensor] = None,
+                 stream=None) -> torch.Tensor:
+    """Absorbed query [..., h_q, 576] = [W_UK^h q_nope, q_rope] per token and head.
+
+    q_nope [..., h_q, 128], q_rope [..., h_q, 64], w_uk [h_q, 512, 128] (latent
+    index first), all bf16 on the device.
+    """
+    tokens, h_q = _projection_shapes("mla_absorb_q", q_nope, 128, w_uk)
+    if tuple(q_rope.shape) != tuple(q_nope.shape[:-1]) + (64,) or q_rope.dtype != torch.bfloat16 \
+            or not q_rope.is_contiguous():
+        raise MLAError("mla_absorb_q", MLA_ERR_ARG)
+    if out is None:
+        out = torch.empty(*q_nope.shape[:-1], 576, dtype=torch.bfloat16, device=q_nope.device)
+    elif tuple(out.shape) != tuple(q_nope.shape[:-1]) + (576,) or out.dtype != torch.bfloat16 \
+            or not out.is_contiguous():
+        raise MLAError("mla_absorb_q", MLA_ERR_ARG)
+    if tokens == 0:
+        return out
+    _check("mla_absorb_q", lib().mla_absorb_q(_ptr(q_nope), _ptr(q_rope), _ptr(w_uk), tokens, h_q, _ptr(out),
+                                              _stream_ptr(stream)))
+    return out
+
+
+def mla_up_project(o_latent: torch.Tensor, w_uv: torch.Tensor, out: Optional[torch.Tensor] = None,
+                   stream=None) -> torch.Tensor:
+    """Per-head output [..., h_q, 128] = o_latent W_UV^h.
+
+    o_latent [..., h_q, 512] (mla_decode's out), w_uv [h_q, 512, 128] (latent
+    index first), bf16 on the device.
+    """
+    tokens, h_q = _projection_shapes("mla_up_project", o_latent, 512, w_uv)
+    if out is None:
+        out = torch.empty(*o_latent.shape[:-1], 128, dtype=torch.bfloat16, device=o_latent.device)
+    elif tuple(out.shape) != tuple(o_latent.shape[:-1]) + (128,) or out.dtype != torch.bfloat16 \
+            or not out.is_contiguous():
+        raise MLAError("mla_up_project", MLA_ERR_ARG)
+    if tokens == 0:
+        return out
+    _check("mla_up_project", lib().mla_up_project(_ptr(o_latent), _ptr(w_uv), tokens, h_q, _ptr(out),
+                                                  _stream_ptr(stream)))
+    return out
 
 
 def mla_take_device_errors(stream=None) -> int:

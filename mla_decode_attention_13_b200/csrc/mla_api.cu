@@ -127,6 +127,66 @@ int encode_value_tiles(PFN_cuTensorMapEncodeTiled_v12000 enc, CUtensorMap* map, 
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
+// A [tokens][h_q][cols] bf16 tensor as (64 cols, tokens, cols / 64 panels,
+// h_q) with strides (h_q * cols * 2 B, 128 B, cols * 2 B): box (64, 128, 2, 1)
+// at (0, t0, z, h) lands as 2 panels of 128 tokens x 128 bytes of head h,
+// 128B-swizzled; tokens past the end read as zeros.
+int encode_token_rows(PFN_cuTensorMapEncodeTiled_v12000 enc, CUtensorMap* map, const void* base, uint64_t tokens,
+                      int h_q, int cols) {
+  const cuuint64_t dims[4] = {64, static_cast<cuuint64_t>(tokens), static_cast<cuuint64_t>(cols / 64),
+                              static_cast<cuuint64_t>(h_q)};
+  const cuuint64_t strides[3] = {static_cast<cuuint64_t>(h_q) * cols * 2, 128, static_cast<cuuint64_t>(cols) * 2};
+  const cuuint32_t box[4] = {64, 128, 2, 1};
+  const cuuint32_t elem[4] = {1, 1, 1, 1};
+  const CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void*>(base), dims, strides, box, elem,
+                         CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                         CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS ? MLA_OK : MLA_ERR_CUDA;
+}
+
+// Per-head weights [h_q][512][128] bf16 as (64 cols, h_q * 512 rows, 2 panels)
+// with strides (256 B, 128 B): box (64, box_rows, 2) lands as 2 panels of
+// box_rows x 128 bytes, 128B-swizzled.
+int encode_head_weights(PFN_cuTensorMapEncodeTiled_v12000 enc, CUtensorMap* map, const void* base, int h_q,
+                        uint32_t box_rows) {
+  const cuuint64_t dims[3] = {64, static_cast<cuuint64_t>(h_q) * kDv, 2};
+  const cuuint64_t strides[2] = {256, 128};
+  const cuuint32_t box[3] = {64, box_rows, 2};
+  const cuuint32_t elem[3] = {1, 1, 1};
+  const CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box, elem,
+                         CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                         CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS ? MLA_OK : MLA_ERR_CUDA;
+}
+
+// Shared argument checks and launch of mla_absorb_q / mla_up_project.
+int projection_impl(const void* a, const void* extra, const void* w, int tokens, int h_q, void* out, bool absorb,
+                    void* stream) {
+  if (!a || !w || !out || (absorb && !extra)) return MLA_ERR_ARG;
+  if (tokens < 1 || h_q < 1) return MLA_ERR_ARG;
+  if (!aligned16(a) || !aligned16(w) || !aligned16(out) || (absorb && !aligned16(extra))) return MLA_ERR_ARG;
+  // grid (h_q, tokens / 128) and 32-bit row offsets
+  if (h_q > kMaxHq || tokens > 65535 * 128) return MLA_ERR_UNSUPPORTED;
+  DeviceInfo dev;
+  int st = current_device_info(&dev);
+  if (st != MLA_OK) return st;
+  PFN_cuTensorMapEncodeTiled_v12000 enc = nullptr;
+  if ((st = tensor_map_encoder(&enc)) != MLA_OK) return st;
+  ProjParams p;
+  if ((st = encode_token_rows(enc, &p.tm_a, a, static_cast<uint64_t>(tokens), h_q, absorb ? 128 : kDv)) != MLA_OK ||
+      (st = encode_head_weights(enc, &p.tm_b, w, h_q, absorb ? 256 : 128)) != MLA_OK)
+    return st;
+  p.extra = extra;
+  p.out = out;
+  p.tokens = tokens;
+  p.h_q = h_q;
+  if (launch_projection(p, absorb, static_cast<cudaStream_t>(stream)) != cudaSuccess) {
+    cudaGetLastError();
+    return MLA_ERR_CUDA;
+  }
+  return MLA_OK;
+}
+
 bool shape_ok(int batch, int h_q, int s_q) {
   return batch >= 1 && h_q >= 1 && h_q <= kMaxHq && s_q >= 1 && s_q <= kMaxSq &&
          static_cast<long long>(batch) * s_q * h_q <= (1LL << 30);
@@ -284,6 +344,15 @@ MLA_API int mla_decode_noalloc(const void* q, const void* kv_cache, int64_t num_
                      causal, out, lse, metadata, scratch, MLA_NOALLOC_SCRATCH_BYTES, stream, nullptr, nullptr);
 }
 
+MLA_API int mla_absorb_q(const void* q_nope, const void* q_rope, const void* w_uk, int tokens, int h_q, void* q_out,
+                         void* stream) {
+  return projection_impl(q_nope, q_rope, w_uk, tokens, h_q, q_out, true, stream);
+}
+
+MLA_API int mla_up_project(const void* o_latent, const void* w_uv, int tokens, int h_q, void* o_out, void* stream) {
+  return projection_impl(o_latent, nullptr, w_uv, tokens, h_q, o_out, false, stream);
+}
+
 MLA_API int mla_check_device_error(const void* metadata, void* stream, uint32_t* error_word) {
   if (!metadata) return MLA_ERR_ARG;
   uint32_t word = 0;
@@ -300,10 +369,13 @@ MLA_API int mla_check_device_error(const void* metadata, void* stream, uint32_t*
 
 MLA_API int mla_take_device_errors(void* stream, uint32_t* error_word) {
   uint32_t word = 0;
-  if (take_sticky_error(static_cast<cudaStream_t>(stream), &word) != cudaSuccess) {
+  uint32_t proj = 0;
+  if (take_sticky_error(static_cast<cudaStream_t>(stream), &word) != cudaSuccess ||
+      take_project_sticky_error(static_cast<cudaStream_t>(stream), &proj) != cudaSuccess) {
     cudaGetLastError();
     return MLA_ERR_CUDA;
   }
+  word |= proj;
   if (error_word) *error_word = word;
   return word == 0 ? MLA_OK : MLA_ERR_DEVICE;
 }

@@ -134,6 +134,19 @@ struct CombineParams {
   int slices;  // warps per query row (1, 2, 4 or 8), each merging 512 / slices columns
 };
 
+// The projections either side of the decode (mla_absorb_q, mla_up_project).
+struct ProjParams {
+  // absorb:     q_nope as (64 cols, tokens, 2 panels, h_q), box (64, 128, 2, 1);
+  // up-project: latent output as (64 cols, tokens, 8 panels, h_q), same box.
+  CUtensorMap tm_a;
+  // The per-head weights [h_q][512][128] as (64 cols, h_q * 512 rows, 2
+  // panels): box (64, 256, 2) for absorb, (64, 128, 2) for the up-projection.
+  CUtensorMap tm_b;
+  const void* extra;  // absorb: q_rope [tokens][h_q][64] bf16 (copied through)
+  void* out;          // absorb: [tokens][h_q][576]; up-project: [tokens][h_q][128]
+  int tokens, h_q;
+};
+
 // Launch wrappers (each returns a cudaError_t).
 cudaError_t launch_sched(const int32_t* seqlens, int batch, int h_q, int s_q, int pairs, int32_t* meta,
                          cudaStream_t stream);
@@ -144,6 +157,9 @@ size_t decode_kernel_smem_bytes();
 cudaError_t take_sticky_error(cudaStream_t stream, uint32_t* word);
 cudaError_t launch_decode(const DecodeParams& p, int pairs, cudaStream_t stream);
 cudaError_t launch_combine(const CombineParams& p, int grid, cudaStream_t stream);
+cudaError_t launch_projection(const ProjParams& p, bool absorb, cudaStream_t stream);
+// Reads and clears the projection kernels' sticky error bits.
+cudaError_t take_project_sticky_error(cudaStream_t stream, uint32_t* word);
 // Warps per query row of the combine (CombineParams::slices) for this many
 // work rows of tile_rows query rows on a device with `sms` SMs.
 int combine_slices(int work_rows, int tile_rows, int sms);

@@ -202,3 +202,43 @@ def workload_inputs(index_or_name, *, device: str = "cpu", seed_offset: int = 0,
     kwargs.update(overrides)
     return make_inputs(lens, wl.h_q, wl.s_q, **kwargs)
 
+
+
+D_NOPE = 128  # per-head query dims without position (W_UK^h: [512][128])
+D_VH = 128    # per-head value dims (W_UV^h: [512][128])
+
+
+@dataclasses.dataclass
+class ProjectionInputs:
+    """Tensors of the projections either side of the absorbed decode."""
+
+    q_nope: torch.Tensor    # [tokens, h_q, 128] bf16
+    q_rope: torch.Tensor    # [tokens, h_q, 64] bf16
+    w_uk: torch.Tensor      # [h_q, 512, 128] bf16, latent index first
+    w_uv: torch.Tensor      # [h_q, 512, 128] bf16, latent index first
+    o_latent: torch.Tensor  # [tokens, h_q, 512] bf16
+
+    def to(self, device) -> "ProjectionInputs":
+        return ProjectionInputs(*(t.to(device) for t in dataclasses.astuple(self)))
+
+
+def make_projection_inputs(tokens: int, h_q: int, *, seed: int = 0) -> ProjectionInputs:
+    """Seeded N(0, 1) activations and N(0, 1 / fan-in) weights, rounded to bf16.
+
+    The weights are scaled by the inverse square root of the summed dimension
+    (128 for W_UK, 512 for W_UV) so that both products come out O(1), as a
+    trained layer's would.  Drawn on the CPU generator.
+    """
+    gen = torch.Generator()
+    gen.manual_seed(seed)
+
+    def draw(*shape, scale=1.0):
+        return (torch.randn(*shape, generator=gen) * scale).to(torch.bfloat16)
+
+    return ProjectionInputs(
+        q_nope=draw(tokens, h_q, D_NOPE),
+        q_rope=draw(tokens, h_q, D_ROPE),
+        w_uk=draw(h_q, D_LATENT, D_NOPE, scale=D_NOPE ** -0.5),
+        w_uv=draw(h_q, D_LATENT, D_VH, scale=D_LATENT ** -0.5),
+        o_latent=draw(tokens, h_q, D_LATENT),
+    )

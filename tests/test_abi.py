@@ -119,3 +119,33 @@ def test_get_metadata_rejects_bad_arguments_on_host(lib):
 def test_check_device_error_rejects_null(lib):
     w = ctypes.c_uint32(0)
     assert lib.mla_check_device_error(None, None, ctypes.byref(w)) == binding.MLA_ERR_ARG
+
+
+@pytest.mark.parametrize("args,status", [
+    ((None, 16, 16, 4, 16, 16), binding.MLA_ERR_ARG),   # q_nope
+    ((16, None, 16, 4, 16, 16), binding.MLA_ERR_ARG),   # q_rope
+    ((16, 16, None, 4, 16, 16), binding.MLA_ERR_ARG),   # w_uk
+    ((16, 16, 16, 4, 16, None), binding.MLA_ERR_ARG),   # q_out
+    ((24, 16, 16, 4, 16, 16), binding.MLA_ERR_ARG),     # misaligned for TMA
+    ((16, 8, 16, 4, 16, 16), binding.MLA_ERR_ARG),
+    ((16, 16, 16, 4, 16, 40), binding.MLA_ERR_ARG),
+    ((16, 16, 16, 0, 16, 16), binding.MLA_ERR_ARG),     # tokens
+    ((16, 16, 16, 4, 0, 16), binding.MLA_ERR_ARG),      # h_q
+    ((16, 16, 16, 4, 129, 16), binding.MLA_ERR_UNSUPPORTED),
+    ((16, 16, 16, 65535 * 128 + 1, 16, 16), binding.MLA_ERR_UNSUPPORTED),
+])
+def test_absorb_q_rejects_bad_arguments_on_host(lib, args, status):
+    assert lib.mla_absorb_q(*args, None) == status
+
+
+@pytest.mark.parametrize("args,status", [
+    ((None, 16, 4, 16, 16), binding.MLA_ERR_ARG),
+    ((16, None, 4, 16, 16), binding.MLA_ERR_ARG),
+    ((16, 16, 4, 16, None), binding.MLA_ERR_ARG),
+    ((16, 32 + 8, 4, 16, 16), binding.MLA_ERR_ARG),
+    ((16, 16, -1, 16, 16), binding.MLA_ERR_ARG),
+    ((16, 16, 4, 0, 16), binding.MLA_ERR_ARG),
+    ((16, 16, 4, 200, 16), binding.MLA_ERR_UNSUPPORTED),
+])
+def test_up_project_rejects_bad_arguments_on_host(lib, args, status):
+    assert lib.mla_up_project(*args, None) == status
