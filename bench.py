@@ -494,6 +494,7 @@ def ours(args, world, rank, local):
     stream.synchronize()
     layer_us = max_over_ranks(l0.elapsed_time(l1) * 1e3 / (n_rep * n_layers), world, dev)
     del layer_graph
+    proj = projection_timing(wl, pools, metas[0], ws, out, lse, stream, dev, l2, world, local, n_layers)
     # The sticky bits cover every step since warm-up (each plan rewrites the
     # word in its own metadata, so those only show the last cycle).
     err = binding.mla_take_device_errors(stream=stream)
@@ -594,6 +595,7 @@ def ours(args, world, rank, local):
         "per_layer": {"value": round(layer_us, 3), "unit": "us/call",
                       "note": (f"one plan, then {n_layers} decode calls (split-KV + combine) on it over the rotating "
                                f"pools, graph-replayed {n_rep} times; the plan's cost spread over the calls")},
+        "projections": proj,
         "gpu_launches": 3 * K,
         "clocks": clocks.summary(),
     }
@@ -602,6 +604,96 @@ def ours(args, world, rank, local):
     del cycle, singles
     if rank == 0:
         print(json.dumps(line), flush=True)
+
+
+def projection_work(tokens, h_q):
+    """Algorithmic bytes of one absorb and one up-projection launch: the head
+    weights once, the tokens' inputs once, the outputs once (bf16)."""
+    w = h_q * 512 * 128 * 2
+    absorb = w + tokens * h_q * (128 + 64) * 2 + tokens * h_q * 576 * 2
+    up = w + tokens * h_q * 512 * 2 + tokens * h_q * 128 * 2
+    return absorb, up
+
+
+def projection_timing(wl, pools, meta, ws, out, lse, stream, dev, l2, world, local, n_layers):
+    """The projections either side of the decode, on the workload's tokens.
+
+    Each kernel is timed as the mean launch of a graph that runs it over
+    rotating weight sets (more than 3x L2 in all, so the weights come from
+    HBM), back to back; then one layer call (absorb -> decode -> up-project)
+    is timed the same way, with the plan made once per graph."""
+    tokens = wl.batch * wl.s_q
+    sets, total = [], 0
+    while len(sets) < 2 or total < 3 * l2:
+        x = inputs.make_projection_inputs(tokens, wl.h_q, seed=5000 + len(sets)).to(dev)
+        sets.append(x)
+        total += sum(t.numel() * 2 for t in (x.w_uk, x.w_uv, x.q_nope, x.q_rope, x.o_latent))
+        if len(sets) >= 128:
+            break
+    n = len(sets)
+    with torch.cuda.stream(stream):
+        q_abs = torch.empty(tokens, wl.h_q, 576, dtype=torch.bfloat16, device=dev)
+        o_up = torch.empty(tokens, wl.h_q, 128, dtype=torch.bfloat16, device=dev)
+    graphs = {}
+    for name in ("absorb", "up_project"):
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g, stream=stream):
+            for x in sets:
+                if name == "absorb":
+                    binding.mla_absorb_q(x.q_nope, x.q_rope, x.w_uk, out=q_abs, stream=stream)
+                else:
+                    binding.mla_up_project(x.o_latent, x.w_uv, out=o_up, stream=stream)
+        graphs[name] = g
+    layer = torch.cuda.CUDAGraph()
+    q_layer = [torch.empty_like(p.q) for p in pools[:2]]
+    with torch.cuda.graph(layer, stream=stream):
+        x0 = pools[0]
+        binding.mla_get_metadata(x0.seqlens, x0.h_q, x0.s_q, metadata=meta, stream=stream)
+        for k in range(n_layers):
+            x, w = pools[k % len(pools)], sets[k % n]
+            qb = q_layer[k & 1]
+            binding.mla_absorb_q(w.q_nope, w.q_rope, w.w_uk, out=qb.view(tokens, wl.h_q, 576), stream=stream)
+            binding.mla_decode(qb, x.kv_cache, x.block_table, x.seqlens, x.softmax_scale, x.causal, meta,
+                               workspace=ws, out=out, lse=lse, stream=stream)
+            binding.mla_up_project(out.view(tokens, wl.h_q, 512), w.w_uv, out=o_up, stream=stream)
+    graphs["layer"] = layer
+    with torch.cuda.stream(stream):
+        for g in graphs.values():
+            g.replay()
+    stream.synchronize()
+    res = {}
+    for name, g in graphs.items():
+        e0 = torch.cuda.Event(enable_timing=True)
+        e1 = torch.cuda.Event(enable_timing=True)
+        reps = 10
+        time.sleep(0.3)  # from an idle GPU, as the other timed phases
+        with ClockSampler(local) as clk:
+            with torch.cuda.stream(stream):
+                e0.record(stream)
+                for _ in range(reps):
+                    g.replay()
+                e1.record(stream)
+            stream.synchronize()
+        per = n_layers if name == "layer" else n
+        res[name] = (max_over_ranks(e0.elapsed_time(e1) * 1e3 / (reps * per), world, dev), clk.summary())
+    del graphs, layer
+    hbm_peak = measured_peaks()[0]
+    b_abs, b_up = projection_work(tokens, wl.h_q)
+    entry = {}
+    for name, nbytes in (("absorb", b_abs), ("up_project", b_up)):
+        us = res[name][0]
+        gbs = nbytes / (us * 1e-6) / 1e9
+        entry[name] = {"us": round(us, 3), "bytes": nbytes,
+                       "roofline": {"bound": "hbm", "achieved": round(gbs, 1), "peak": hbm_peak, "unit": "GB/s",
+                                    "frac": round(gbs / hbm_peak, 3)},
+                       "clocks": res[name][1]}
+    entry["layer_with_projections"] = {
+        "value": round(res["layer"][0], 3), "unit": "us/call", "clocks": res["layer"][1],
+        "note": (f"one plan, then {n_layers} calls of absorb -> decode (split-KV + combine) -> up-project, "
+                 f"graph-replayed; weights rotate over {n} sets")}
+    entry["note"] = (f"{tokens} tokens x {wl.h_q} heads; each kernel is the mean launch of a graph over {n} weight "
+                     f"sets ({total / 2**20:.0f} MiB > 3x L2), launched back to back")
+    return entry
 
 
 def main():

@@ -128,15 +128,15 @@ int encode_value_tiles(PFN_cuTensorMapEncodeTiled_v12000 enc, CUtensorMap* map, 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
 // A [tokens][h_q][cols] bf16 tensor as (64 cols, tokens, cols / 64 panels,
-// h_q) with strides (h_q * cols * 2 B, 128 B, cols * 2 B): box (64, 128, 2, 1)
-// at (0, t0, z, h) lands as 2 panels of 128 tokens x 128 bytes of head h,
-// 128B-swizzled; tokens past the end read as zeros.
+// h_q) with strides (h_q * cols * 2 B, 128 B, cols * 2 B): box (64, box_rows,
+// 2, 1) at (0, t0, z, h) lands as 2 panels of box_rows tokens x 128 bytes of
+// head h, 128B-swizzled; tokens past the end read as zeros.
 int encode_token_rows(PFN_cuTensorMapEncodeTiled_v12000 enc, CUtensorMap* map, const void* base, uint64_t tokens,
-                      int h_q, int cols) {
+                      int h_q, int cols, uint32_t box_rows) {
   const cuuint64_t dims[4] = {64, static_cast<cuuint64_t>(tokens), static_cast<cuuint64_t>(cols / 64),
                               static_cast<cuuint64_t>(h_q)};
   const cuuint64_t strides[3] = {static_cast<cuuint64_t>(h_q) * cols * 2, 128, static_cast<cuuint64_t>(cols) * 2};
-  const cuuint32_t box[4] = {64, 128, 2, 1};
+  const cuuint32_t box[4] = {64, box_rows, 2, 1};
   const cuuint32_t elem[4] = {1, 1, 1, 1};
   const CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void*>(base), dims, strides, box, elem,
                          CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
@@ -173,9 +173,12 @@ int projection_impl(const void* a, const void* extra, const void* w, int tokens,
   PFN_cuTensorMapEncodeTiled_v12000 enc = nullptr;
   if ((st = tensor_map_encoder(&enc)) != MLA_OK) return st;
   ProjParams p;
-  if ((st = encode_token_rows(enc, &p.tm_a, a, static_cast<uint64_t>(tokens), h_q, absorb ? 128 : kDv)) != MLA_OK ||
-      (st = encode_head_weights(enc, &p.tm_b, w, h_q, absorb ? 256 : 128)) != MLA_OK)
+  p.nb = proj_box_rows(tokens, absorb ? kProjAbsorbTile : kProjUpTile);
+  if ((st = encode_token_rows(enc, &p.tm_a, a, static_cast<uint64_t>(tokens), h_q, absorb ? 128 : kDv,
+                              static_cast<uint32_t>(p.nb))) != MLA_OK ||
+      (st = encode_head_weights(enc, &p.tm_b, w, h_q, 128)) != MLA_OK)
     return st;
+  p.w = w;
   p.extra = extra;
   p.out = out;
   p.tokens = tokens;

@@ -135,16 +135,31 @@ struct CombineParams {
 };
 
 // The projections either side of the decode (mla_absorb_q, mla_up_project).
+// A CTA takes one head and a tile of tokens (up to kProjAbsorbTile for the
+// absorb, kProjUpTile for the up-projection).
+constexpr int kProjAbsorbTile = 128;
+constexpr int kProjUpTile = 64;
+
+// Token rows of a tile's box (the MMA's N): the token count rounded up to 16,
+// capped at the tile.
+__host__ __device__ inline int proj_box_rows(int tokens, int tile) {
+  const int r = (tokens + 15) & ~15;
+  return r < tile ? r : tile;
+}
+
 struct ProjParams {
-  // absorb:     q_nope as (64 cols, tokens, 2 panels, h_q), box (64, 128, 2, 1);
-  // up-project: latent output as (64 cols, tokens, 8 panels, h_q), same box.
+  // absorb:     q_nope as (64 cols, tokens, 2 panels, h_q);
+  // up-project: latent output as (64 cols, tokens, 8 panels, h_q);
+  // box (64, nb, 2, 1): 2 panels of nb tokens of one head.
   CUtensorMap tm_a;
   // The per-head weights [h_q][512][128] as (64 cols, h_q * 512 rows, 2
-  // panels): box (64, 256, 2) for absorb, (64, 128, 2) for the up-projection.
+  // panels): box (64, 128, 2), one 128-row chunk.
   CUtensorMap tm_b;
+  const void* w;      // the weights' base address (for the L2 prefetch)
   const void* extra;  // absorb: q_rope [tokens][h_q][64] bf16 (copied through)
   void* out;          // absorb: [tokens][h_q][576]; up-project: [tokens][h_q][128]
   int tokens, h_q;
+  int nb;             // proj_box_rows(tokens, tile)
 };
 
 // Launch wrappers (each returns a cudaError_t).

@@ -10,21 +10,29 @@
 // with W_UK^h and W_UV^h stored [512 latent rows][128 columns] per head.
 //
 // Both are batched GEMMs over the heads whose bytes are the weights (128 KB
-// per head and product) and the tokens' rows; with decode's few tokens per
-// head they are bound by memory.  One CTA takes one head and a tile of up to
-// 128 tokens: the tokens are the MMA's M (so each TMEM lane holds one token's
-// output row, stored whole with 16-byte stores), the head's weight rows its N.
-//   * absorb: A = the tokens' q_nope (128 x 128, K-major), B = W_UK^h (512 x
-//     128, K-major), D = 128 tokens x 512 fp32 in all 512 TMEM columns, as two
-//     N = 256 products over 8 K steps.
-//   * up-project: A = the tokens' latent output (128 x 512, K-major), B =
-//     W_UV^h (K = 512 rows, N = 128 columns, MN-major), D = 128 x 128 fp32, over
-//     32 K steps streamed through two 64 KB stages.
-// One thread issues the TMA loads and the MMAs; four warps read TMEM out.  Every
+// per head and product); a decode step has few tokens (16 to a few hundred),
+// so they are bound by memory.  The weight rows are the MMA's M and the tokens
+// its N (N = the token box, a multiple of 16), so a short token list costs no
+// padded MMA rows, each TMEM lane holds one output dimension, and a warp
+// stores 32 consecutive dimensions of a token (64 bytes) per instruction.
+//   * absorb: one CTA per (head, 128-row chunk of W_UK^h, tile of up to 128
+//     tokens): one M = 128 product of the chunk (K-major, 32 KB) with the
+//     tokens' q_nope (K-major), 8 K steps.  Small CTAs (32 KB + the token box)
+//     let several share an SM, the next launch's included.
+//   * up-project: one CTA per (head, tile of up to 64 tokens): one M = 128
+//     product over K = 512: A = W_UV^h seen as 128 value dims x 512 latent
+//     dims (MN-major: the value dim is contiguous in memory), B = the tokens'
+//     latent output (K-major), in four 128-deep K chunks, each with a barrier
+//     of its own, all in flight at once, each chunk's MMAs issued as it lands.
+// Shared memory is sized by the token box.  Before waiting for the previous
+// kernel on the stream (programmatic dependent launch) each CTA asks L2 to
+// fetch its weights, which no kernel of the decode writes; a prefetch is only
+// a hint and L2 is the point of coherence, so it cannot return stale data.  One
+// thread issues the TMA loads and the MMAs; four warps read TMEM out.  Every
 // wait is bounded by %globaltimer; on expiry the kernel raises
 // MLA_DEVERR_TIMEOUT in this file's sticky error word (taken with the decode
-// kernel's by mla_take_device_errors), waits for its copies, frees TMEM and
-// returns without writing.
+// kernel's by mla_take_device_errors), skips the affected stores, waits for
+// its copies and MMAs, frees TMEM and returns.
 #include <cuda_bf16.h>
 
 #include "mla_internal.h"
@@ -39,27 +47,33 @@ namespace {
 using namespace ptx;
 
 constexpr int kProjThreads = 128;
-constexpr int kTokTile = 128;
 constexpr uint64_t kProjTimeoutNs = 1000ull * 1000ull * 1000ull;
+constexpr int kChunks = 4;                      // 128-row weight chunks per head
+constexpr uint32_t kWChunk = 128 * 256;         // 128 rows x 128 bf16 columns: 32 KB
+constexpr uint32_t kAMajorMN = 1u << 15;        // instruction descriptor: A is MN-major
 
-// K-major 128B-swizzled panel of 64 bf16 columns: rows x 128 bytes.
-constexpr uint32_t kPanelTok = kTokTile * 128;  // 128 token rows: 16 KB
+// Shared memory (sized by the token box nb at launch), then barriers:
+//   absorb:     one 32 KB chunk of W_UK^h, then q_nope (2 panels x nb rows x 128 B)
+//   up-project: 4 x 32 KB of W_UV^h, then 4 chunks of the latent output
+//               (2 panels x nb rows x 128 B each)
+constexpr uint32_t kAbsTokens = kProjAbsorbTile;
+constexpr uint32_t kUpTokens = kProjUpTile;
+constexpr uint32_t kBarBytes = 128;
+__host__ __device__ constexpr uint32_t absorb_bar_offset(int nb) { return kWChunk + 2u * nb * 128u; }
+__host__ __device__ constexpr uint32_t up_bar_offset(int nb) { return kChunks * kWChunk + kChunks * 2u * nb * 128u; }
+__host__ __device__ constexpr uint32_t absorb_smem(int nb) { return absorb_bar_offset(nb) + kBarBytes + 1024; }
+__host__ __device__ constexpr uint32_t up_smem(int nb) { return up_bar_offset(nb) + kBarBytes + 1024; }
+static_assert(absorb_smem(kProjAbsorbTile) <= 227 * 1024 && up_smem(kProjUpTile) <= 227 * 1024, "shared memory");
 
-// absorb: A = 2 panels (K = 128), B = 2 N-halves x 2 panels of 256 rows.
-constexpr uint32_t kAbsA = 2 * kPanelTok;          // 32 KB
-constexpr uint32_t kAbsBPanel = 256 * 128;         // 32 KB
-constexpr uint32_t kAbsB = 4 * kAbsBPanel;         // 128 KB
-constexpr uint32_t kAbsBar = kAbsA + kAbsB;
-constexpr uint32_t kAbsSmem = kAbsBar + 64 + 1024;
+// Barrier words (byte offsets from the barrier area): w[c] at 8c (data of
+// chunk c; absorb uses w[0]), accumulator ready at 40, final drain at 72;
+// TMEM address at 80; ok flag at 84.
+constexpr uint32_t kBW = 0, kBD = 40, kBFin = 72, kTmemSlot = 80, kOkFlag = 84;
 
-// up-project: 2 stages of (A: 2 panels of 128 tokens, B: 2 column panels of
-// 128 latent rows), one stage per 128 latent columns.
-constexpr uint32_t kUpStage = 2 * kPanelTok + 2 * (128 * 128);  // 64 KB
-constexpr uint32_t kUpBar = 2 * kUpStage;
-constexpr uint32_t kUpSmem = kUpBar + 64 + 1024;
-
-constexpr uint32_t kIdescAbs = idesc_bf16_f32(128, 256, false);
-constexpr uint32_t kIdescUp = idesc_bf16_f32(128, 128, true);
+// Ask L2 to fetch [ptr, ptr + bytes) from memory (no shared-memory write).
+__device__ __forceinline__ void prefetch_l2(const void* ptr, uint32_t bytes) {
+  asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(ptr), "r"(bytes) : "memory");
+}
 
 __device__ __forceinline__ void tma_load_3d(uint32_t dst, const CUtensorMap* m, uint32_t bar, int32_t x, int32_t y,
                                             int32_t z) {
@@ -90,48 +104,70 @@ __device__ bool wait_proj(uint32_t bar, uint32_t parity, bool raise = true) {
   }
 }
 
-// Four warps, one token per thread: row t of D (its TMEM lane), columns
-// [c0, c0 + 32), as bf16 to dst (32 contiguous elements, 16-byte stores).
-__device__ __forceinline__ void store_row32(uint32_t taddr, __nv_bfloat16* dst, bool ok) {
+// Width of one accumulator of nb token columns: nb rounded up to 32, so that
+// the read-out's 32-column loads stay inside it.
+__device__ __forceinline__ uint32_t slot_width(int nb) { return (static_cast<uint32_t>(nb) + 31u) & ~31u; }
+
+// TMEM columns to allocate for `slots` accumulators: a power of two from 32 to
+// 512 (4 x 128 at most).
+__device__ __forceinline__ uint32_t tmem_cols(int slots, int nb) {
+  const uint32_t need = static_cast<uint32_t>(slots) * slot_width(nb);
+  uint32_t c = 32;
+  while (c < need) c <<= 1;
+  return c;
+}
+
+// Four warps, one output dimension per thread (its TMEM lane): columns
+// [j0, j0 + 32) of the accumulator at `taddr` are the tile's tokens j0 + j;
+// token j is stored as bf16 at dst + j * row_stride, for j below `count`.
+__device__ __forceinline__ void store_tokens32(uint32_t taddr, __nv_bfloat16* dst, long long row_stride, int j0,
+                                               int count) {
   float v[32];
   tmem_ld32(taddr, v);
   tmem_wait_ld();
-  if (!ok) return;
-  uint4* d4 = reinterpret_cast<uint4*>(dst);
 #pragma unroll
-  for (int j = 0; j < 4; ++j) {
-    __nv_bfloat162 a = __floats2bfloat162_rn(v[8 * j + 0], v[8 * j + 1]);
-    __nv_bfloat162 b = __floats2bfloat162_rn(v[8 * j + 2], v[8 * j + 3]);
-    __nv_bfloat162 c = __floats2bfloat162_rn(v[8 * j + 4], v[8 * j + 5]);
-    __nv_bfloat162 e = __floats2bfloat162_rn(v[8 * j + 6], v[8 * j + 7]);
-    uint4 u;
-    u.x = *reinterpret_cast<uint32_t*>(&a);
-    u.y = *reinterpret_cast<uint32_t*>(&b);
-    u.z = *reinterpret_cast<uint32_t*>(&c);
-    u.w = *reinterpret_cast<uint32_t*>(&e);
-    d4[j] = u;
-  }
+  for (int j = 0; j < 32; ++j)
+    if (j0 + j < count) dst[static_cast<long long>(j0 + j) * row_stride] = __float2bfloat16_rn(v[j]);
+}
+
+struct ProjSmem {
+  uint32_t base;   // 1024-aligned shared address
+  uint8_t* gbase;  // the same, generic
+};
+
+__device__ __forceinline__ ProjSmem proj_smem() {
+  extern __shared__ uint8_t smem_raw[];
+  const uint32_t raw = smem_u32(smem_raw);
+  ProjSmem s;
+  s.base = (raw + 1023u) & ~1023u;
+  s.gbase = smem_raw + (s.base - raw);
+  return s;
 }
 
 __global__ void __launch_bounds__(kProjThreads, 1) mla_absorb_kernel(const __grid_constant__ ProjParams p) {
-  extern __shared__ uint8_t smem_raw[];
-  const uint32_t raw = smem_u32(smem_raw);
-  const uint32_t base = (raw + 1023u) & ~1023u;
-  uint8_t* gbase = smem_raw + (base - raw);
-  const int h = blockIdx.x;
-  const int t0 = blockIdx.y * kTokTile;
+  const ProjSmem sm = proj_smem();
+  const uint32_t base = sm.base;
+  const int h = blockIdx.x >> 2, c = blockIdx.x & 3;  // head, 128-row chunk of W_UK^h
+  const int t0 = blockIdx.y * kAbsTokens;
+  const int nb = p.nb;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const uint32_t bar_full = base + kAbsBar, bar_done = base + kAbsBar + 8;
-  volatile uint32_t* tmem_slot = reinterpret_cast<volatile uint32_t*>(gbase + kAbsBar + 16);
-  volatile uint32_t* ok_flag = reinterpret_cast<volatile uint32_t*>(gbase + kAbsBar + 20);
+  const uint32_t q_smem = base + kWChunk;
+  const uint32_t bar_area = absorb_bar_offset(nb);
+  const uint32_t bars = base + bar_area;
+  volatile uint32_t* tmem_slot = reinterpret_cast<volatile uint32_t*>(sm.gbase + bar_area + kTmemSlot);
+  volatile uint32_t* ok_flag = reinterpret_cast<volatile uint32_t*>(sm.gbase + bar_area + kOkFlag);
+  const uint32_t ncols = tmem_cols(1, nb);
+  const char* w_chunk = static_cast<const char*>(p.w) + (static_cast<size_t>(h) * kDv + c * 128) * 256;
   if (threadIdx.x == 0) {
-    mbar_init(bar_full, 1);
-    mbar_init(bar_done, 1);
+    mbar_init(bars + kBW, 1);
+    mbar_init(bars + kBD, 1);
+    mbar_init(bars + kBFin, 1);
     *ok_flag = 1u;
     fence_mbar_init_cluster();
+    prefetch_l2(w_chunk, kWChunk);  // the weights are not written by the kernels this one waits for
   }
   if (warp == 0) {
-    tmem_alloc(base + kAbsBar + 16, 512);
+    tmem_alloc(bars + kTmemSlot, ncols);
     tmem_relinquish();
   }
   tc_fence_before();
@@ -139,85 +175,90 @@ __global__ void __launch_bounds__(kProjThreads, 1) mla_absorb_kernel(const __gri
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
   griddep_launch_dependents();
-  griddep_wait();  // the tokens' q_nope may come from the previous kernel
+  griddep_wait();  // q_nope may come from the previous kernel on the stream
 
   if (threadIdx.x == 0) {
-    mbar_arrive_expect_tx(bar_full, kAbsA + kAbsB);
-    tma_load_4d(base, &p.tm_a, bar_full, 0, t0, 0, h);  // q_nope: 2 panels x 128 tokens
-#pragma unroll
-    for (int nh = 0; nh < 2; ++nh)  // W_UK^h rows [256 nh, +256): 2 panels
-      tma_load_3d(base + kAbsA + nh * 2 * kAbsBPanel, &p.tm_b, bar_full, 0, h * 512 + nh * 256, 0);
-    bool good = wait_proj(bar_full, 0);
-    if (good) {
+    mbar_arrive_expect_tx(bars + kBW, kWChunk + 2u * nb * 128u);
+    tma_load_3d(base, &p.tm_b, bars + kBW, 0, h * kDv + c * 128, 0);  // W_UK^h rows [128 c, +128): 2 panels
+    tma_load_4d(q_smem, &p.tm_a, bars + kBW, 0, t0, 0, h);            // q_nope: 2 panels x nb tokens
+    const uint32_t idesc = idesc_bf16_f32(128, static_cast<uint32_t>(nb), false);
+    if (wait_proj(bars + kBW, 0)) {
       tc_fence_after();
 #pragma unroll
-      for (int nh = 0; nh < 2; ++nh) {
-#pragma unroll
-        for (int ks = 0; ks < 8; ++ks) {
-          const uint64_t a = smem_desc(base + (ks >> 2) * kPanelTok + (ks & 3) * 32, 16, 1024, kSwizzle128B);
-          const uint64_t b = smem_desc(base + kAbsA + (2 * nh + (ks >> 2)) * kAbsBPanel + (ks & 3) * 32, 16, 1024,
-                                       kSwizzle128B);
-          umma_ss(tmem + 256 * nh, a, b, kIdescAbs, ks > 0 ? 1u : 0u);
-        }
-      }
-      umma_commit(bar_done);
-      if (!wait_proj(bar_done, 0)) {
-        good = false;
-        wait_proj(bar_done, 0, false);  // drain the MMAs before TMEM is freed
+      for (int ks = 0; ks < 8; ++ks) {
+        const uint64_t a = smem_desc(base + (ks >> 2) * (128 * 128) + (ks & 3) * 32, 16, 1024, kSwizzle128B);
+        const uint64_t b = smem_desc(q_smem + (ks >> 2) * (nb * 128) + (ks & 3) * 32, 16, 1024, kSwizzle128B);
+        umma_ss(tmem, a, b, idesc, ks > 0 ? 1u : 0u);
       }
     } else {
-      wait_proj(bar_full, 0, false);  // drain the copies before the CTA exits
+      *ok_flag = 0u;
+      wait_proj(bars + kBW, 0, false);  // drain the copies
     }
-    if (!good) *ok_flag = 0u;
+    umma_commit(bars + kBD);  // after the MMAs (or at once, with none issued)
   }
-  __syncthreads();
+  __syncwarp();
+
+  // Read-out: the accumulator holds latent dims [128 c, +128) of the tile's
+  // tokens; thread (warp, lane) owns dim 128 c + 32 warp + lane.
+  __nv_bfloat16* out = reinterpret_cast<__nv_bfloat16*>(p.out);
+  const long long row_stride = static_cast<long long>(p.h_q) * kDqk;
+  const int count = min(static_cast<int>(kAbsTokens), p.tokens - t0);
+  __nv_bfloat16* tile_out = out + static_cast<long long>(t0) * row_stride + static_cast<long long>(h) * kDqk;
+  const bool ready = __all_sync(0xffffffffu, wait_proj(bars + kBD, 0));  // warp-uniform, as the TMEM loads are
   tc_fence_after();
-  const bool ok = *ok_flag != 0u;
-  const int t = t0 + 32 * warp + lane;
-  const bool row_ok = ok && t < p.tokens;
-  __nv_bfloat16* orow = reinterpret_cast<__nv_bfloat16*>(p.out) + (static_cast<long long>(t) * p.h_q + h) * kDqk;
-  const uint32_t lane_addr = tmem + (static_cast<uint32_t>(32 * warp) << 16);
-  if (ok) {
-#pragma unroll 1
-    for (int c0 = 0; c0 < 512; c0 += 32) store_row32(lane_addr + c0, orow + c0, row_ok);
-    if (row_ok) {  // the rope part passes through
-      const uint4* src = reinterpret_cast<const uint4*>(reinterpret_cast<const __nv_bfloat16*>(p.extra) +
-                                                        (static_cast<long long>(t) * p.h_q + h) * 64);
-      uint4* dst = reinterpret_cast<uint4*>(orow + 512);
-#pragma unroll
-      for (int j = 0; j < 8; ++j) dst[j] = src[j];
+  if (ready && *ok_flag != 0u) {
+    const uint32_t lane_base = tmem + (static_cast<uint32_t>(32 * warp) << 16);
+    for (int j0 = 0; j0 < nb; j0 += 32)
+      store_tokens32(lane_base + j0, tile_out + c * 128 + 32 * warp + lane, row_stride, j0, count);
+    // The rope columns pass through (chunk 0's CTA): 16-byte pieces.
+    if (c == 0) {
+      const __nv_bfloat16* rope = reinterpret_cast<const __nv_bfloat16*>(p.extra);
+      for (int k = threadIdx.x; k < count * 8; k += kProjThreads) {
+        const long long t = t0 + (k >> 3);
+        const uint4 v = reinterpret_cast<const uint4*>(rope + (t * p.h_q + h) * 64)[k & 7];
+        reinterpret_cast<uint4*>(out + t * row_stride + static_cast<long long>(h) * kDqk + kDv)[k & 7] = v;
+      }
     }
+  }
+
+  // Teardown: every MMA done before TMEM is freed.
+  if (threadIdx.x == 0) {
+    umma_commit(bars + kBFin);
+    wait_proj(bars + kBFin, 0, false);
   }
   tc_fence_before();
   __syncthreads();
   if (warp == 0) {
     tc_fence_after();
-    tmem_dealloc(tmem, 512);
+    tmem_dealloc(tmem, ncols);
   }
 }
 
 __global__ void __launch_bounds__(kProjThreads, 1) mla_up_project_kernel(const __grid_constant__ ProjParams p) {
-  extern __shared__ uint8_t smem_raw[];
-  const uint32_t raw = smem_u32(smem_raw);
-  const uint32_t base = (raw + 1023u) & ~1023u;
-  uint8_t* gbase = smem_raw + (base - raw);
+  const ProjSmem sm = proj_smem();
+  const uint32_t bar_area = up_bar_offset(p.nb);
+  const uint32_t base = sm.base, bars = sm.base + bar_area;
   const int h = blockIdx.x;
-  const int t0 = blockIdx.y * kTokTile;
+  const int t0 = blockIdx.y * kUpTokens;
+  const int nb = p.nb;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const uint32_t bar_full = base + kUpBar, bar_empty = base + kUpBar + 16, bar_done = base + kUpBar + 32;
-  volatile uint32_t* tmem_slot = reinterpret_cast<volatile uint32_t*>(gbase + kUpBar + 40);
-  volatile uint32_t* ok_flag = reinterpret_cast<volatile uint32_t*>(gbase + kUpBar + 44);
+  const uint32_t o_smem = base + kChunks * kWChunk;  // chunk c at o_smem + c * o_chunk
+  const uint32_t o_chunk = 2u * nb * 128u;
+  volatile uint32_t* tmem_slot = reinterpret_cast<volatile uint32_t*>(sm.gbase + bar_area + kTmemSlot);
+  volatile uint32_t* ok_flag = reinterpret_cast<volatile uint32_t*>(sm.gbase + bar_area + kOkFlag);
+  const uint32_t ncols = tmem_cols(1, nb);
   if (threadIdx.x == 0) {
-    for (int s = 0; s < 2; ++s) {
-      mbar_init(bar_full + 8 * s, 1);
-      mbar_init(bar_empty + 8 * s, 1);
-    }
-    mbar_init(bar_done, 1);
+    for (int c = 0; c < kChunks; ++c) mbar_init(bars + kBW + 8 * c, 1);
+    mbar_init(bars + kBD, 1);
+    mbar_init(bars + kBFin, 1);
     *ok_flag = 1u;
     fence_mbar_init_cluster();
+    // W_UV^h is not written by the kernels this one waits for
+    const char* w_head = static_cast<const char*>(p.w) + static_cast<size_t>(h) * kDv * 256;
+    for (int c = 0; c < kChunks; ++c) prefetch_l2(w_head + c * kWChunk, kWChunk);
   }
   if (warp == 0) {
-    tmem_alloc(base + kUpBar + 40, 128);
+    tmem_alloc(bars + kTmemSlot, ncols);
     tmem_relinquish();
   }
   tc_fence_before();
@@ -225,72 +266,62 @@ __global__ void __launch_bounds__(kProjThreads, 1) mla_up_project_kernel(const _
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
   griddep_launch_dependents();
-  griddep_wait();  // the latent output comes from the decode (combine) kernel
+  griddep_wait();  // the latent output comes from the decode's combine kernel
 
   if (threadIdx.x == 0) {
-    // Stage s holds latent columns [128 c, +128) of chunk c: the tokens' rows
-    // (2 panels) and W_UV^h's rows (2 panels of 64 output columns).
-    auto load = [&](int c) {
-      const int s = c & 1;
-      const uint32_t st = base + s * kUpStage;
-      mbar_arrive_expect_tx(bar_full + 8 * s, kUpStage);
-      tma_load_4d(st, &p.tm_a, bar_full + 8 * s, 0, t0, 2 * c, h);
-      tma_load_3d(st + 2 * kPanelTok, &p.tm_b, bar_full + 8 * s, 0, h * 512 + c * 128, 0);
-    };
-    int issued = 0, landed = 0;  // chunks loaded, chunks whose load was waited for
-    load(0);
-    load(1);
-    issued = 2;
+    // Chunk c: latent dims [128 c, +128) of W_UV^h (2 panels of 64 value
+    // dims x 128 rows) and of the tokens' output (2 panels x nb rows).
+    for (int c = 0; c < kChunks; ++c) {
+      mbar_arrive_expect_tx(bars + kBW + 8 * c, kWChunk + o_chunk);
+      tma_load_3d(base + c * kWChunk, &p.tm_b, bars + kBW + 8 * c, 0, h * kDv + c * 128, 0);
+      tma_load_4d(o_smem + c * o_chunk, &p.tm_a, bars + kBW + 8 * c, 0, t0, 2 * c, h);
+    }
+    const uint32_t idesc = idesc_bf16_f32(128, static_cast<uint32_t>(nb), false) | kAMajorMN;
     bool good = true;
-    for (int c = 0; c < 4 && good; ++c) {
-      const int s = c & 1;
-      const uint32_t st = base + s * kUpStage;
-      good = wait_proj(bar_full + 8 * s, (c >> 1) & 1);
+    int landed = 0;
+    for (int c = 0; c < kChunks && good; ++c) {
+      good = wait_proj(bars + kBW + 8 * c, 0);
       if (!good) break;
       landed = c + 1;
       tc_fence_after();
 #pragma unroll
       for (int ks = 0; ks < 8; ++ks) {
-        const uint64_t a = smem_desc(st + (ks >> 2) * kPanelTok + (ks & 3) * 32, 16, 1024, kSwizzle128B);
-        // MN-major: 16 latent rows of both 64-column panels (leading byte
-        // offset = one panel of 128 rows)
-        const uint64_t b = smem_desc(st + 2 * kPanelTok + ks * 16 * 128, 128 * 128, 1024, kSwizzle128B);
-        umma_ss(tmem, a, b, kIdescUp, (c > 0 || ks > 0) ? 1u : 0u);
-      }
-      if (c + 2 < 4) {  // refill the stage once this chunk's MMAs are done with it
-        umma_commit(bar_empty + 8 * s);
-        good = wait_proj(bar_empty + 8 * s, (c >> 1) & 1);
-        if (good) {
-          load(c + 2);
-          issued = c + 3;
-        }
+        // MN-major A: 16 latent rows of both 64-value-dim panels (leading
+        // byte offset = one panel of 128 rows)
+        const uint64_t a = smem_desc(base + c * kWChunk + ks * 16 * 128, 128 * 128, 1024, kSwizzle128B);
+        const uint64_t b = smem_desc(o_smem + c * o_chunk + (ks >> 2) * (nb * 128) + (ks & 3) * 32, 16, 1024,
+                                     kSwizzle128B);
+        umma_ss(tmem, a, b, idesc, (c > 0 || ks > 0) ? 1u : 0u);
       }
     }
-    umma_commit(bar_done);  // every MMA issued so far
-    if (!wait_proj(bar_done, 0, good)) {
-      good = false;
-      wait_proj(bar_done, 0, false);
+    umma_commit(bars + kBD);  // after the last MMA issued (or none)
+    if (!good) {
+      *ok_flag = 0u;
+      for (int c = landed; c < kChunks; ++c) wait_proj(bars + kBW + 8 * c, 0, false);
     }
-    if (!good)  // drain copies still in flight before the CTA exits
-      for (int c = landed; c < issued; ++c) wait_proj(bar_full + 8 * (c & 1), (c >> 1) & 1, false);
-    if (!good) *ok_flag = 0u;
   }
-  __syncthreads();
+  __syncwarp();
+
+  __nv_bfloat16* out = reinterpret_cast<__nv_bfloat16*>(p.out);
+  const long long row_stride = static_cast<long long>(p.h_q) * 128;
+  const int count = min(static_cast<int>(kUpTokens), p.tokens - t0);
+  const bool ready = __all_sync(0xffffffffu, wait_proj(bars + kBD, 0));  // warp-uniform, as the TMEM loads are
   tc_fence_after();
-  const bool ok = *ok_flag != 0u;
-  const int t = t0 + 32 * warp + lane;
-  const bool row_ok = ok && t < p.tokens;
-  __nv_bfloat16* orow = reinterpret_cast<__nv_bfloat16*>(p.out) + (static_cast<long long>(t) * p.h_q + h) * 128;
-  const uint32_t lane_addr = tmem + (static_cast<uint32_t>(32 * warp) << 16);
-  if (ok) {
-#pragma unroll 1
-    for (int c0 = 0; c0 < 128; c0 += 32) store_row32(lane_addr + c0, orow + c0, row_ok);
+  if (ready && *ok_flag != 0u) {
+    __nv_bfloat16* dst = out + static_cast<long long>(t0) * row_stride + h * 128 + 32 * warp + lane;
+    const uint32_t lane_base = tmem + (static_cast<uint32_t>(32 * warp) << 16);
+    for (int j0 = 0; j0 < nb; j0 += 32) store_tokens32(lane_base + j0, dst, row_stride, j0, count);
+  }
+
+  if (threadIdx.x == 0) {
+    umma_commit(bars + kBFin);
+    wait_proj(bars + kBFin, 0, false);
   }
   tc_fence_before();
   __syncthreads();
   if (warp == 0) {
     tc_fence_after();
-    tmem_dealloc(tmem, 128);
+    tmem_dealloc(tmem, ncols);
   }
 }
 
@@ -299,11 +330,14 @@ __global__ void __launch_bounds__(kProjThreads, 1) mla_up_project_kernel(const _
 cudaError_t launch_projection(const ProjParams& p, bool absorb, cudaStream_t stream) {
   const void* fn = absorb ? reinterpret_cast<const void*>(mla_absorb_kernel)
                           : reinterpret_cast<const void*>(mla_up_project_kernel);
-  const int smem = static_cast<int>(absorb ? kAbsSmem : kUpSmem);
-  cudaError_t e = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+  const int smem = static_cast<int>(absorb ? absorb_smem(p.nb) : up_smem(p.nb));
+  const int max_smem = static_cast<int>(absorb ? absorb_smem(kProjAbsorbTile) : up_smem(kProjUpTile));
+  const int tile = absorb ? kProjAbsorbTile : kProjUpTile;
+  cudaError_t e = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, max_smem);
   if (e != cudaSuccess) return e;
   cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3(static_cast<unsigned>(p.h_q), static_cast<unsigned>((p.tokens + kTokTile - 1) / kTokTile), 1);
+  cfg.gridDim = dim3(static_cast<unsigned>(absorb ? kChunks * p.h_q : p.h_q),
+                     static_cast<unsigned>((p.tokens + tile - 1) / tile), 1);
   cfg.blockDim = dim3(kProjThreads, 1, 1);
   cfg.dynamicSmemBytes = static_cast<size_t>(smem);
   cfg.stream = stream;

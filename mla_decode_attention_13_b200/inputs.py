@@ -219,7 +219,7 @@ class ProjectionInputs:
     o_latent: torch.Tensor  # [tokens, h_q, 512] bf16
 
     def to(self, device) -> "ProjectionInputs":
-        return ProjectionInputs(*(t.to(device) for t in dataclasses.astuple(self)))
+        return ProjectionInputs(*(getattr(self, f.name).to(device) for f in dataclasses.fields(self)))
 
 
 def make_projection_inputs(tokens: int, h_q: int, *, seed: int = 0) -> ProjectionInputs:
