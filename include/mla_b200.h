@@ -243,6 +243,33 @@ int mla_absorb_q(const void* q_nope, const void* q_rope, const void* w_uk, int t
 int mla_up_project(const void* o_latent, const void* w_uv, int tokens, int h_q, void* o_out, void* stream);
 
 /*
+ * Merge decode results computed over disjoint token ranges of the same rows:
+ * one long row split across GPUs, each decoding (mla_get_metadata and
+ * mla_decode on its own cache, block table and lengths) the pages it holds,
+ * then exchanging (out, lse).  "Unlocking GPU Potential: The Impact of
+ * FlashAttention and KV Cache Optimization in Long-Text Inference": attend to
+ * each chunk of the keys separately, then rescale the partial results by
+ * their log-sum-exp.  For each query row, over splits k:
+ *     lse = ln sum_k exp(lse_k),   out = sum_k exp(lse_k - lse) * out_k
+ * in fp32; a split with lse_k = -inf adds nothing, and a row with no visible
+ * token in any split gets out = 0, lse = -inf.  The result equals one
+ * mla_decode over the union of the ranges when every split saw the query rows'
+ * visible tokens of its range (for a causal step: all splits but the one
+ * holding the row's last tokens run with causal = 0).
+ *   outs   [device] bf16 [splits][batch][s_q][h_q][512]: the splits' `out`,
+ *          stacked; 16-byte aligned.
+ *   lses   [device] fp32 [splits][batch][h_q][s_q]: the splits' `lse`.
+ *   splits >= 1; batch, s_q, h_q as for mla_decode.
+ *   out    [device] bf16 [batch][s_q][h_q][512], 16-byte aligned; lse [device]
+ *          fp32 [batch][h_q][s_q].  Neither may overlap the inputs.
+ * Returns MLA_ERR_ARG for a NULL or misaligned pointer or a count below 1,
+ * MLA_ERR_UNSUPPORTED for shapes mla_decode refuses, MLA_ERR_CUDA if the
+ * launch failed.  One small kernel; no device error bits.
+ */
+int mla_merge_splits(const void* outs, const float* lses, int splits, int batch, int s_q, int h_q, void* out,
+                     float* lse, void* stream);
+
+/*
  * Synchronise `stream` and read the device error word from `metadata`.
  * Writes the word to *error_word (if not NULL).  Returns MLA_OK when it is
  * zero, MLA_ERR_DEVICE when not, MLA_ERR_CUDA if the copy or sync failed.

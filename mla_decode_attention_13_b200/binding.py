@@ -39,6 +39,7 @@ EXPORTED = (
     "mla_decode_noalloc",
     "mla_absorb_q",
     "mla_up_project",
+    "mla_merge_splits",
     "mla_check_device_error",
     "mla_take_device_errors",
     "mla_error_string",
@@ -82,6 +83,8 @@ def lib() -> ctypes.CDLL:
         L.mla_absorb_q.argtypes = [_vp, _vp, _vp, ctypes.c_int, ctypes.c_int, _vp, _vp]
         L.mla_up_project.restype = ctypes.c_int
         L.mla_up_project.argtypes = [_vp, _vp, ctypes.c_int, ctypes.c_int, _vp, _vp]
+        L.mla_merge_splits.restype = ctypes.c_int
+        L.mla_merge_splits.argtypes = [_vp, _vp] + [ctypes.c_int] * 4 + [_vp, _vp, _vp]
         L.mla_check_device_error.restype = ctypes.c_int
         L.mla_check_device_error.argtypes = [_vp, _vp, ctypes.POINTER(ctypes.c_uint32)]
         L.mla_take_device_errors.restype = ctypes.c_int
@@ -256,6 +259,28 @@ def mla_up_project(o_latent: torch.Tensor, w_uv: torch.Tensor, out: Optional[tor
     _check("mla_up_project", lib().mla_up_project(_ptr(o_latent), _ptr(w_uv), tokens, h_q, _ptr(out),
                                                   _stream_ptr(stream)))
     return out
+
+
+def mla_merge_splits(outs: torch.Tensor, lses: torch.Tensor, out: Optional[torch.Tensor] = None,
+                     lse: Optional[torch.Tensor] = None, stream=None) -> Tuple[torch.Tensor, torch.Tensor]:
+    """Merge decode results over disjoint token ranges of the same rows.
+
+    outs [splits, batch, s_q, h_q, 512] bf16 and lses [splits, batch, h_q, s_q]
+    fp32 (the splits' mla_decode results, stacked); returns (out, lse) as
+    mla_decode would over the union of the ranges.
+    """
+    if outs.dim() != 5 or outs.shape[-1] != 512 or outs.dtype != torch.bfloat16 or not outs.is_contiguous():
+        raise MLAError("mla_merge_splits", MLA_ERR_ARG)
+    splits, batch, s_q, h_q, _ = outs.shape
+    if tuple(lses.shape) != (splits, batch, h_q, s_q) or lses.dtype != torch.float32 or not lses.is_contiguous():
+        raise MLAError("mla_merge_splits", MLA_ERR_ARG)
+    if out is None:
+        out = torch.empty(batch, s_q, h_q, 512, dtype=torch.bfloat16, device=outs.device)
+    if lse is None:
+        lse = torch.empty(batch, h_q, s_q, dtype=torch.float32, device=outs.device)
+    _check("mla_merge_splits", lib().mla_merge_splits(_ptr(outs), _ptr(lses), splits, batch, s_q, h_q, _ptr(out),
+                                                      _ptr(lse), _stream_ptr(stream)))
+    return out, lse
 
 
 def mla_take_device_errors(stream=None) -> int:

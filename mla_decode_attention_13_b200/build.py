@@ -23,7 +23,7 @@ INCLUDE = os.path.join(ROOT, "include")
 BUILD = os.path.join(ROOT, "_build")
 LIB = os.path.join(PKG, "libmla_b200.so")
 
-SOURCES = ["mla_api.cu", "mla_sched.cu", "mla_decode.cu", "mla_combine.cu", "mla_project.cu"]
+SOURCES = ["mla_api.cu", "mla_sched.cu", "mla_decode.cu", "mla_combine.cu", "mla_project.cu", "mla_merge.cu"]
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 FLAGS = ["-O3", "-lineinfo", "-std=c++17", "-Xcompiler", "-fPIC,-fvisibility=hidden", "-I", INCLUDE, "-I", CSRC]
 

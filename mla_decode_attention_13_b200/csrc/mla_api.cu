@@ -356,6 +356,32 @@ MLA_API int mla_up_project(const void* o_latent, const void* w_uv, int tokens, i
   return projection_impl(o_latent, nullptr, w_uv, tokens, h_q, o_out, false, stream);
 }
 
+MLA_API int mla_merge_splits(const void* outs, const float* lses, int splits, int batch, int s_q, int h_q, void* out,
+                             float* lse, void* stream) {
+  if (!outs || !lses || !out || !lse) return MLA_ERR_ARG;
+  if (splits < 1 || batch < 1 || s_q < 1 || h_q < 1) return MLA_ERR_ARG;
+  if (!aligned16(outs) || !aligned16(out)) return MLA_ERR_ARG;
+  if (!shape_ok(batch, h_q, s_q)) return MLA_ERR_UNSUPPORTED;
+  if (static_cast<long long>(splits) * batch * s_q * h_q > (1LL << 31)) return MLA_ERR_UNSUPPORTED;
+  DeviceInfo dev;
+  const int st = current_device_info(&dev);
+  if (st != MLA_OK) return st;
+  MergeParams p;
+  p.outs = outs;
+  p.lses = lses;
+  p.out = out;
+  p.lse = lse;
+  p.splits = splits;
+  p.batch = batch;
+  p.s_q = s_q;
+  p.h_q = h_q;
+  if (launch_merge(p, dev.sms, static_cast<cudaStream_t>(stream)) != cudaSuccess) {
+    cudaGetLastError();
+    return MLA_ERR_CUDA;
+  }
+  return MLA_OK;
+}
+
 MLA_API int mla_check_device_error(const void* metadata, void* stream, uint32_t* error_word) {
   if (!metadata) return MLA_ERR_ARG;
   uint32_t word = 0;

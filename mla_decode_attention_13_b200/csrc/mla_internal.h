@@ -162,6 +162,15 @@ struct ProjParams {
   int nb;             // proj_box_rows(tokens, tile)
 };
 
+// Merge of per-split decode results (mla_merge_splits).
+struct MergeParams {
+  const void* outs;   // bf16 [splits][batch][s_q][h_q][512]
+  const float* lses;  // [splits][batch][h_q][s_q]
+  void* out;          // bf16 [batch][s_q][h_q][512]
+  float* lse;         // [batch][h_q][s_q]
+  int splits, batch, s_q, h_q;
+};
+
 // Launch wrappers (each returns a cudaError_t).
 cudaError_t launch_sched(const int32_t* seqlens, int batch, int h_q, int s_q, int pairs, int32_t* meta,
                          cudaStream_t stream);
@@ -173,6 +182,7 @@ cudaError_t take_sticky_error(cudaStream_t stream, uint32_t* word);
 cudaError_t launch_decode(const DecodeParams& p, int pairs, cudaStream_t stream);
 cudaError_t launch_combine(const CombineParams& p, int grid, cudaStream_t stream);
 cudaError_t launch_projection(const ProjParams& p, bool absorb, cudaStream_t stream);
+cudaError_t launch_merge(const MergeParams& p, int sms, cudaStream_t stream);
 // Reads and clears the projection kernels' sticky error bits.
 cudaError_t take_project_sticky_error(cudaStream_t stream, uint32_t* word);
 // Warps per query row of the combine (CombineParams::slices) for this many

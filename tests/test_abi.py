@@ -149,3 +149,21 @@ def test_absorb_q_rejects_bad_arguments_on_host(lib, args, status):
 ])
 def test_up_project_rejects_bad_arguments_on_host(lib, args, status):
     assert lib.mla_up_project(*args, None) == status
+
+
+@pytest.mark.parametrize("args,status", [
+    ((None, 16, 2, 1, 1, 16, 16, 16), binding.MLA_ERR_ARG),
+    ((16, None, 2, 1, 1, 16, 16, 16), binding.MLA_ERR_ARG),
+    ((16, 16, 2, 1, 1, 16, None, 16), binding.MLA_ERR_ARG),
+    ((16, 16, 2, 1, 1, 16, 16, None), binding.MLA_ERR_ARG),
+    ((8, 16, 2, 1, 1, 16, 16, 16), binding.MLA_ERR_ARG),   # misaligned
+    ((16, 16, 2, 1, 1, 16, 24, 16), binding.MLA_ERR_ARG),
+    ((16, 16, 0, 1, 1, 16, 16, 16), binding.MLA_ERR_ARG),  # splits
+    ((16, 16, 2, 0, 1, 16, 16, 16), binding.MLA_ERR_ARG),
+    ((16, 16, 2, 1, 0, 16, 16, 16), binding.MLA_ERR_ARG),
+    ((16, 16, 2, 1, 1, 0, 16, 16), binding.MLA_ERR_ARG),
+    ((16, 16, 2, 1, 1, 129, 16, 16), binding.MLA_ERR_UNSUPPORTED),
+    ((16, 16, 2, 1, 17, 16, 16, 16), binding.MLA_ERR_UNSUPPORTED),
+])
+def test_merge_splits_rejects_bad_arguments_on_host(lib, args, status):
+    assert lib.mla_merge_splits(*args, None) == status

@@ -34,9 +34,10 @@ ATOL = 5e-4
 RTOL = 2.0 ** -8
 MIN_EXACT = 0.98
 
-# (tokens, h_q): one token; the decode workloads' 16 and 256 tokens of 128
-# heads; a ragged second tile (200 = 128 + 72); an odd head count; one head.
-CASES = [(1, 128), (16, 128), (256, 128), (200, 16), (300, 3), (129, 1)]
+# (tokens, h_q): one token; every decode workload's tokens (batch * s_q) and
+# heads (1 x 16, 16 x 128, 64 x 128, 256 x 128, 4 x 16); a ragged second tile
+# (200 = 128 + 72); an odd head count; one head.
+CASES = [(1, 128), (1, 16), (16, 128), (64, 128), (256, 128), (4, 16), (200, 16), (300, 3), (129, 1)]
 
 
 def bf16_round(x: np.ndarray) -> np.ndarray:
