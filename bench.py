@@ -495,6 +495,7 @@ def ours(args, world, rank, local):
     layer_us = max_over_ranks(l0.elapsed_time(l1) * 1e3 / (n_rep * n_layers), world, dev)
     del layer_graph
     proj = projection_timing(wl, pools, metas[0], ws, out, lse, stream, dev, l2, world, local, n_layers)
+    split = long_row_timing(wl, pools, stream, dev, world, local)
     # The sticky bits cover every step since warm-up (each plan rewrites the
     # word in its own metadata, so those only show the last cycle).
     err = binding.mla_take_device_errors(stream=stream)
@@ -596,6 +597,7 @@ def ours(args, world, rank, local):
                       "note": (f"one plan, then {n_layers} decode calls (split-KV + combine) on it over the rotating "
                                f"pools, graph-replayed {n_rep} times; the plan's cost spread over the calls")},
         "projections": proj,
+        "long_row_split": split,
         "gpu_launches": 3 * K,
         "clocks": clocks.summary(),
     }
@@ -694,6 +696,99 @@ def projection_timing(wl, pools, meta, ws, out, lse, stream, dev, l2, world, loc
     entry["note"] = (f"{tokens} tokens x {wl.h_q} heads; each kernel is the mean launch of a graph over {n} weight "
                      f"sets ({total / 2**20:.0f} MiB > 3x L2), launched back to back")
     return entry
+
+
+def long_row_timing(wl, pools, stream, dev, world, local):
+    """The split of each row across W ranks (longrow), with the ranks emulated
+    one after another on this GPU: each rank's plan + decode call on its share
+    of the pages (graph over the rotating pools, mean per call), and the merge
+    of the W partial results.  The exchange between GPUs is not timed here
+    (one GPU); its bytes per rank are reported."""
+    from mla_decode_attention_13_b200 import longrow
+
+    lens = [int(v) for v in pools[0].seqlens.cpu()]
+    rows = wl.batch * wl.s_q * wl.h_q
+    res = {}
+    for W in (2, 4):
+        rank_us, outs, lses = [], [], []
+        for r in range(W):
+            shards = [longrow.shard_block_table(x.block_table, lens, W, r, wl.s_q) for x in pools]
+            with torch.cuda.stream(stream):
+                meta = torch.empty(binding.mla_metadata_bytes(wl.batch, wl.h_q, wl.s_q) // 4, dtype=torch.int32,
+                                   device=dev)
+                ws = torch.empty(max(binding.mla_workspace_bytes(wl.batch, wl.h_q, wl.s_q), 16), dtype=torch.uint8,
+                                 device=dev)
+                o = torch.empty(wl.batch, wl.s_q, wl.h_q, 512, dtype=torch.bfloat16, device=dev)
+                l = torch.empty(wl.batch, wl.h_q, wl.s_q, dtype=torch.float32, device=dev)
+            causal_r = bool(wl.causal) and r == W - 1
+
+            def call(k):
+                x, (tab, ln) = pools[k], shards[k]
+                binding.mla_get_metadata(ln, x.h_q, x.s_q, metadata=meta, stream=stream)
+                binding.mla_decode(x.q, x.kv_cache, tab, ln, x.softmax_scale, causal_r, meta, workspace=ws, out=o,
+                                   lse=l, stream=stream)
+
+            for k in range(len(pools)):
+                call(k)
+            g = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(g, stream=stream):
+                for k in range(len(pools)):
+                    call(k)
+            with torch.cuda.stream(stream):
+                g.replay()
+            stream.synchronize()
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            reps = 10
+            time.sleep(0.3)
+            with torch.cuda.stream(stream):
+                e0.record(stream)
+                for _ in range(reps):
+                    g.replay()
+                e1.record(stream)
+            stream.synchronize()
+            rank_us.append(max_over_ranks(e0.elapsed_time(e1) * 1e3 / (reps * len(pools)), world, dev))
+            del g
+            # the last pool's partial result, for the merge
+            outs.append(o.clone())
+            lses.append(l.clone())
+        outs_t, lses_t = torch.stack(outs), torch.stack(lses)
+        with torch.cuda.stream(stream):
+            m_out = torch.empty_like(outs[0])
+            m_lse = torch.empty_like(lses[0])
+            binding.mla_merge_splits(outs_t, lses_t, out=m_out, lse=m_lse, stream=stream)
+        stream.synchronize()
+        g = torch.cuda.CUDAGraph()
+        n_merge = 20
+        with torch.cuda.graph(g, stream=stream):
+            for _ in range(n_merge):
+                binding.mla_merge_splits(outs_t, lses_t, out=m_out, lse=m_lse, stream=stream)
+        with torch.cuda.stream(stream):
+            g.replay()
+        stream.synchronize()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        time.sleep(0.3)
+        with torch.cuda.stream(stream):
+            e0.record(stream)
+            for _ in range(5):
+                g.replay()
+            e1.record(stream)
+        stream.synchronize()
+        merge_us = max_over_ranks(e0.elapsed_time(e1) * 1e3 / (5 * n_merge), world, dev)
+        del g
+        merge_bytes = (W + 1) * rows * (512 * 2 + 4)
+        res[f"ranks_{W}"] = {
+            "rank_call_us": [round(u, 3) for u in rank_us],
+            "max_rank_call_us": round(max(rank_us), 3),
+            "merge_us": round(merge_us, 3),
+            "merge_bytes": merge_bytes,
+            "merge_achieved_gbs": round(merge_bytes / (merge_us * 1e-6) / 1e9, 1),
+            "exchange_bytes_per_rank": (W - 1) * rows * (512 * 2 + 4),
+        }
+    res["note"] = ("each row's pages cut over W ranks (page-aligned, the last rank masks); ranks emulated one after "
+                   "another on this GPU, each a plan + decode call on its share (graph over the rotating pools, mean "
+                   "per call); merge = mla_merge_splits of the W partials (graph, mean per launch, L2-resident "
+                   "inputs as after an exchange); the all-gather between GPUs is not run on one GPU")
+    return res
 
 
 def main():
