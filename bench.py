@@ -603,6 +603,7 @@ def ours(args, world, rank, local):
     }
     if world == 1 and rank == 0 and not args.no_cpu_baseline:
         line["cpu_baseline"] = cpu_baseline(idx, budget_s=10.0)
+        line["projections"]["cpu_baseline"] = oracle_projection_and_merge(wl)
     del cycle, singles
     if rank == 0:
         print(json.dumps(line), flush=True)
@@ -696,6 +697,39 @@ def projection_timing(wl, pools, meta, ws, out, lse, stream, dev, l2, world, loc
     entry["note"] = (f"{tokens} tokens x {wl.h_q} heads; each kernel is the mean launch of a graph over {n} weight "
                      f"sets ({total / 2**20:.0f} MiB > 3x L2), launched back to back")
     return entry
+
+
+def oracle_projection_and_merge(wl, budget_s=4.0):
+    """The oracle, as it stands, on bounded samples of the same shapes: the two
+    projections on one token of every head (scaled to the step's tokens), and
+    the merge of 4 splits over a sample of query rows (scaled to all rows)."""
+    from oracle import mla_oracle
+
+    tokens = wl.batch * wl.s_q
+    x = inputs.make_projection_inputs(1, wl.h_q, seed=99)
+    res = {}
+    for name, fn in (("absorb", lambda: mla_oracle.absorb_query(x.q_nope[0], x.q_rope[0], x.w_uk)),
+                     ("up_project", lambda: mla_oracle.expand_output(x.o_latent[0], x.w_uv))):
+        times = []
+        t_start = time.perf_counter()
+        while not times or (time.perf_counter() - t_start < budget_s / 3 and len(times) < 20):
+            t0 = time.perf_counter()
+            fn()
+            times.append(time.perf_counter() - t0)
+        res[name + "_us"] = round(sum(times) / len(times) * tokens * 1e6, 1)
+    rows = wl.batch * wl.s_q * wl.h_q
+    sample = min(rows, 256)
+    gen = torch.Generator()
+    gen.manual_seed(98)
+    parts = [((torch.randn(sample, 512, generator=gen) * 0.25).double().numpy(),
+              torch.randn(sample, generator=gen).double().numpy()) for _ in range(4)]
+    t0 = time.perf_counter()
+    mla_oracle.combine_partials(parts)
+    res["merge_4_splits_us"] = round((time.perf_counter() - t0) * rows / sample * 1e6, 1)
+    res.update(unit="us/call", cores=cpu_threads(), kind="oracle",
+               sample=(f"projections: one token of all {wl.h_q} heads, x {tokens} tokens; merge: {sample} of "
+                       f"{rows} query rows, x {rows / sample:g}"))
+    return res
 
 
 def long_row_timing(wl, pools, stream, dev, world, local):

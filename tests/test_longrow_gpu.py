@@ -84,3 +84,28 @@ def test_split_decode_emulated_on_one_gpu_matches_unsplit_oracle(world, case):
     assert np.array_equal(np.isneginf(got_lse), np.isneginf(want_lse))
     fin = np.isfinite(want_lse)
     assert np.max(np.abs(got_lse[fin] - want_lse[fin])) <= 1e-3
+
+
+def test_split_of_the_long_context_workload_at_full_size():
+    # b4_h16_L128k-1k (rows of 131072, 1024, 32768 and 8192 tokens, 16 heads)
+    # over 4 emulated ranks, every output against the oracle's unsplit decode.
+    x = inputs.workload_inputs("b4_h16_L128k-1k")
+    lens = [int(v) for v in x.seqlens]
+    g = x.to("cuda")
+    world = 4
+    outs, lses = [], []
+    for rank in range(world):
+        table, local = longrow.shard_block_table(g.block_table, lens, world, rank, x.s_q)
+        meta = binding.mla_get_metadata(local, x.h_q, x.s_q)
+        o, l = binding.mla_decode(g.q, g.kv_cache, table, local, x.softmax_scale, x.causal and rank == world - 1, meta)
+        assert binding.mla_check_device_error(meta) == 0
+        outs.append(o)
+        lses.append(l)
+    out, lse = binding.mla_merge_splits(torch.stack(outs), torch.stack(lses))
+    torch.cuda.synchronize()
+    want_out, want_lse = mla_oracle.decode(x.q, x.kv_cache, x.block_table, x.seqlens, x.softmax_scale, x.causal)
+    err = np.abs(mla_oracle.as_f64(out.cpu()) - want_out)
+    parts_max = max(float(o.abs().max()) for o in outs)
+    bar = 8e-3 + 2.0 ** -9 * (parts_max + float(np.abs(want_out).max()))
+    assert err.max() <= bar and err.mean() <= 1e-3, (err.max(), bar, err.mean())
+    assert np.max(np.abs(mla_oracle.as_f64(lse.cpu()) - want_lse)) <= 1e-3
