@@ -440,8 +440,30 @@ def _mut_combine_mean(mp):
     mp.setattr(O, "combine_partials", comb)
 
 
+def _mut_absorb_one_head(mp):
+    # every head absorbed with head 0's W_UK
+    orig = O.absorb_query
+    mp.setattr(O, "absorb_query", lambda qn, qr, w: orig(qn, qr, np.broadcast_to(O.as_f64(w)[:1], np.shape(w))))
+
+
+def _mut_absorb_drops_rope(mp):
+    orig = O.absorb_query
+
+    def absorb(qn, qr, w):
+        q = orig(qn, qr, w)
+        q[:, 512:] = 0.0
+        return q
+    mp.setattr(O, "absorb_query", absorb)
+
+
+def _mut_expand_heads_reversed(mp):
+    orig = O.expand_output
+    mp.setattr(O, "expand_output", lambda o, w: orig(o, O.as_f64(w)[::-1]))
+
+
 MUTATIONS = [_mut_drop_rope, _mut_rope_sign, _mut_value_window, _mut_no_scale, _mut_causal_off_by_one,
-             _mut_ignore_table, _mut_slot_major, _mut_log2_lse, _mut_unnormalised, _mut_combine_mean]
+             _mut_ignore_table, _mut_slot_major, _mut_log2_lse, _mut_unnormalised, _mut_combine_mean,
+             _mut_absorb_one_head, _mut_absorb_drops_rope, _mut_expand_heads_reversed]
 
 
 @pytest.mark.parametrize("mutation", MUTATIONS, ids=lambda f: f.__name__)
