@@ -5,7 +5,7 @@
 #include <cmath>
 #include <mutex>
 
-#include "mla_internal.h"
+#include "mla_layer.h"
 
 #define MLA_API extern "C" __attribute__((visibility("default")))
 

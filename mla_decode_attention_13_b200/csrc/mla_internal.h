@@ -134,43 +134,6 @@ struct CombineParams {
   int slices;  // warps per query row (1, 2, 4 or 8), each merging 512 / slices columns
 };
 
-// The projections either side of the decode (mla_absorb_q, mla_up_project).
-// A CTA takes one head and a tile of tokens (up to kProjAbsorbTile for the
-// absorb, kProjUpTile for the up-projection).
-constexpr int kProjAbsorbTile = 128;
-constexpr int kProjUpTile = 64;
-
-// Token rows of a tile's box (the MMA's N): the token count rounded up to 16,
-// capped at the tile.
-__host__ __device__ inline int proj_box_rows(int tokens, int tile) {
-  const int r = (tokens + 15) & ~15;
-  return r < tile ? r : tile;
-}
-
-struct ProjParams {
-  // absorb:     q_nope as (64 cols, tokens, 2 panels, h_q);
-  // up-project: latent output as (64 cols, tokens, 8 panels, h_q);
-  // box (64, nb, 2, 1): 2 panels of nb tokens of one head.
-  CUtensorMap tm_a;
-  // The per-head weights [h_q][512][128] as (64 cols, h_q * 512 rows, 2
-  // panels): box (64, 128, 2), one 128-row chunk.
-  CUtensorMap tm_b;
-  const void* w;      // the weights' base address (for the L2 prefetch)
-  const void* extra;  // absorb: q_rope [tokens][h_q][64] bf16 (copied through)
-  void* out;          // absorb: [tokens][h_q][576]; up-project: [tokens][h_q][128]
-  int tokens, h_q;
-  int nb;             // proj_box_rows(tokens, tile)
-};
-
-// Merge of per-split decode results (mla_merge_splits).
-struct MergeParams {
-  const void* outs;   // bf16 [splits][batch][s_q][h_q][512]
-  const float* lses;  // [splits][batch][h_q][s_q]
-  void* out;          // bf16 [batch][s_q][h_q][512]
-  float* lse;         // [batch][h_q][s_q]
-  int splits, batch, s_q, h_q;
-};
-
 // Launch wrappers (each returns a cudaError_t).
 cudaError_t launch_sched(const int32_t* seqlens, int batch, int h_q, int s_q, int pairs, int32_t* meta,
                          cudaStream_t stream);
@@ -181,10 +144,6 @@ size_t decode_kernel_smem_bytes();
 cudaError_t take_sticky_error(cudaStream_t stream, uint32_t* word);
 cudaError_t launch_decode(const DecodeParams& p, int pairs, cudaStream_t stream);
 cudaError_t launch_combine(const CombineParams& p, int grid, cudaStream_t stream);
-cudaError_t launch_projection(const ProjParams& p, bool absorb, cudaStream_t stream);
-cudaError_t launch_merge(const MergeParams& p, int sms, cudaStream_t stream);
-// Reads and clears the projection kernels' sticky error bits.
-cudaError_t take_project_sticky_error(cudaStream_t stream, uint32_t* word);
 // Warps per query row of the combine (CombineParams::slices) for this many
 // work rows of tile_rows query rows on a device with `sms` SMs.
 int combine_slices(int work_rows, int tile_rows, int sms);

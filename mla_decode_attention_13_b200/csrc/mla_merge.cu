@@ -21,7 +21,7 @@
 
 #include <cmath>
 
-#include "mla_internal.h"
+#include "mla_layer.h"
 #include "sm100_ptx.cuh"
 
 namespace mla {

@@ -35,7 +35,7 @@
 // its copies and MMAs, frees TMEM and returns.
 #include <cuda_bf16.h>
 
-#include "mla_internal.h"
+#include "mla_layer.h"
 #include "sm100_ptx.cuh"
 
 namespace mla {
