@@ -24,7 +24,10 @@
 //     dims (MN-major: the value dim is contiguous in memory), B = the tokens'
 //     latent output (K-major), in four 128-deep K chunks, each with a barrier
 //     of its own, all in flight at once, each chunk's MMAs issued as it lands.
-// Shared memory is sized by the token box.  Before waiting for the previous
+// Shared memory is sized by the token box, and TMEM is read out 16 columns at
+// a time so that both kernels fit in 64 registers a thread: up to five absorb
+// CTAs (at 16 tokens) share an SM, which leaves room for the next launch's
+// CTAs to start early.  Before waiting for the previous
 // kernel on the stream (programmatic dependent launch) each CTA asks L2 to
 // fetch its weights, which no kernel of the decode writes; a prefetch is only
 // a hint and L2 is the point of coherence, so it cannot return stale data.  One
@@ -117,17 +120,32 @@ __device__ __forceinline__ uint32_t tmem_cols(int slots, int nb) {
   return c;
 }
 
+// Each thread of the warp reads its own lane, 16 consecutive fp32 columns.
+__device__ __forceinline__ void tmem_ld16(uint32_t taddr, float (&v)[16]) {
+  uint32_t* r = reinterpret_cast<uint32_t*>(v);
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x16.b32 "
+      "{%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15}, [%16];"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
+        "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15])
+      : "r"(taddr)
+      : "memory");
+}
+
 // Four warps, one output dimension per thread (its TMEM lane): columns
-// [j0, j0 + 32) of the accumulator at `taddr` are the tile's tokens j0 + j;
+// [j0, j0 + 16) of the accumulator at `taddr` are the tile's tokens j0 + j;
 // token j is stored as bf16 at dst + j * row_stride, for j below `count`.
-__device__ __forceinline__ void store_tokens32(uint32_t taddr, __nv_bfloat16* dst, long long row_stride, int j0,
+__device__ __forceinline__ void store_tokens16(uint32_t taddr, __nv_bfloat16* dst, long long row_stride, int j0,
                                                int count) {
-  float v[32];
-  tmem_ld32(taddr, v);
+  float v[16];
+  tmem_ld16(taddr, v);
   tmem_wait_ld();
+  __nv_bfloat16* d = dst + static_cast<long long>(j0) * row_stride;
 #pragma unroll
-  for (int j = 0; j < 32; ++j)
-    if (j0 + j < count) dst[static_cast<long long>(j0 + j) * row_stride] = __float2bfloat16_rn(v[j]);
+  for (int j = 0; j < 16; ++j) {
+    if (j0 + j < count) *d = __float2bfloat16_rn(v[j]);
+    d += row_stride;
+  }
 }
 
 struct ProjSmem {
@@ -144,7 +162,7 @@ __device__ __forceinline__ ProjSmem proj_smem() {
   return s;
 }
 
-__global__ void __launch_bounds__(kProjThreads, 1) mla_absorb_kernel(const __grid_constant__ ProjParams p) {
+__global__ void __launch_bounds__(kProjThreads, 8) mla_absorb_kernel(const __grid_constant__ ProjParams p) {
   const ProjSmem sm = proj_smem();
   const uint32_t base = sm.base;
   const int h = blockIdx.x >> 2, c = blockIdx.x & 3;  // head, 128-row chunk of W_UK^h
@@ -208,8 +226,8 @@ __global__ void __launch_bounds__(kProjThreads, 1) mla_absorb_kernel(const __gri
   tc_fence_after();
   if (ready && *ok_flag != 0u) {
     const uint32_t lane_base = tmem + (static_cast<uint32_t>(32 * warp) << 16);
-    for (int j0 = 0; j0 < nb; j0 += 32)
-      store_tokens32(lane_base + j0, tile_out + c * 128 + 32 * warp + lane, row_stride, j0, count);
+    for (int j0 = 0; j0 < nb; j0 += 16)
+      store_tokens16(lane_base + j0, tile_out + c * 128 + 32 * warp + lane, row_stride, j0, count);
     // The rope columns pass through (chunk 0's CTA): 16-byte pieces.
     if (c == 0) {
       const __nv_bfloat16* rope = reinterpret_cast<const __nv_bfloat16*>(p.extra);
@@ -234,7 +252,7 @@ __global__ void __launch_bounds__(kProjThreads, 1) mla_absorb_kernel(const __gri
   }
 }
 
-__global__ void __launch_bounds__(kProjThreads, 1) mla_up_project_kernel(const __grid_constant__ ProjParams p) {
+__global__ void __launch_bounds__(kProjThreads, 4) mla_up_project_kernel(const __grid_constant__ ProjParams p) {
   const ProjSmem sm = proj_smem();
   const uint32_t bar_area = up_bar_offset(p.nb);
   const uint32_t base = sm.base, bars = sm.base + bar_area;
@@ -310,7 +328,7 @@ __global__ void __launch_bounds__(kProjThreads, 1) mla_up_project_kernel(const _
   if (ready && *ok_flag != 0u) {
     __nv_bfloat16* dst = out + static_cast<long long>(t0) * row_stride + h * 128 + 32 * warp + lane;
     const uint32_t lane_base = tmem + (static_cast<uint32_t>(32 * warp) << 16);
-    for (int j0 = 0; j0 < nb; j0 += 32) store_tokens32(lane_base + j0, dst, row_stride, j0, count);
+    for (int j0 = 0; j0 < nb; j0 += 16) store_tokens16(lane_base + j0, dst, row_stride, j0, count);
   }
 
   if (threadIdx.x == 0) {
