@@ -290,6 +290,17 @@ int mla_check_device_error(const void* metadata, void* stream, uint32_t* error_w
  */
 int mla_take_device_errors(void* stream, uint32_t* error_word);
 
+/*
+ * Self-test of the kernels' bounded waits, for failure-detection tests: one
+ * tiny kernel waits on a barrier that nothing arrives at, with the limit the
+ * projection kernels use (1 s of %globaltimer).  The wait gives up, sets
+ * MLA_DEVERR_TIMEOUT in the bits mla_take_device_errors reports, and the
+ * kernel returns: no fault, and the context stays usable.  Enqueued on
+ * `stream`; returns MLA_OK, or MLA_ERR_UNSUPPORTED / MLA_ERR_CUDA if the
+ * device is not sm_100 or the launch failed.
+ */
+int mla_selftest_bounded_wait(void* stream);
+
 /* Static text for a status code. */
 const char* mla_error_string(int status);
 

@@ -40,6 +40,7 @@ EXPORTED = (
     "mla_absorb_q",
     "mla_up_project",
     "mla_merge_splits",
+    "mla_selftest_bounded_wait",
     "mla_check_device_error",
     "mla_take_device_errors",
     "mla_error_string",
@@ -85,6 +86,8 @@ def lib() -> ctypes.CDLL:
         L.mla_up_project.argtypes = [_vp, _vp, ctypes.c_int, ctypes.c_int, _vp, _vp]
         L.mla_merge_splits.restype = ctypes.c_int
         L.mla_merge_splits.argtypes = [_vp, _vp] + [ctypes.c_int] * 4 + [_vp, _vp, _vp]
+        L.mla_selftest_bounded_wait.restype = ctypes.c_int
+        L.mla_selftest_bounded_wait.argtypes = [_vp]
         L.mla_check_device_error.restype = ctypes.c_int
         L.mla_check_device_error.argtypes = [_vp, _vp, ctypes.POINTER(ctypes.c_uint32)]
         L.mla_take_device_errors.restype = ctypes.c_int
@@ -281,6 +284,11 @@ def mla_merge_splits(outs: torch.Tensor, lses: torch.Tensor, out: Optional[torch
     _check("mla_merge_splits", lib().mla_merge_splits(_ptr(outs), _ptr(lses), splits, batch, s_q, h_q, _ptr(out),
                                                       _ptr(lse), _stream_ptr(stream)))
     return out, lse
+
+
+def mla_selftest_bounded_wait(stream=None) -> None:
+    """Enqueue one bounded wait that runs out (raises MLA_DEVERR_TIMEOUT after ~1 s)."""
+    _check("mla_selftest_bounded_wait", lib().mla_selftest_bounded_wait(_stream_ptr(stream)))
 
 
 def mla_take_device_errors(stream=None) -> int:

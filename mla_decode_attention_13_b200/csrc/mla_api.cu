@@ -382,6 +382,17 @@ MLA_API int mla_merge_splits(const void* outs, const float* lses, int splits, in
   return MLA_OK;
 }
 
+MLA_API int mla_selftest_bounded_wait(void* stream) {
+  DeviceInfo dev;
+  const int st = current_device_info(&dev);
+  if (st != MLA_OK) return st;
+  if (launch_wait_selftest(static_cast<cudaStream_t>(stream)) != cudaSuccess) {
+    cudaGetLastError();
+    return MLA_ERR_CUDA;
+  }
+  return MLA_OK;
+}
+
 MLA_API int mla_check_device_error(const void* metadata, void* stream, uint32_t* error_word) {
   if (!metadata) return MLA_ERR_ARG;
   uint32_t word = 0;

@@ -46,6 +46,8 @@ struct MergeParams {
 
 cudaError_t launch_projection(const ProjParams& p, bool absorb, cudaStream_t stream);
 cudaError_t launch_merge(const MergeParams& p, int sms, cudaStream_t stream);
+// One bounded wait that runs out (see mla_selftest_bounded_wait).
+cudaError_t launch_wait_selftest(cudaStream_t stream);
 // Reads and clears the projection kernels' sticky error bits.
 cudaError_t take_project_sticky_error(cudaStream_t stream, uint32_t* word);
 

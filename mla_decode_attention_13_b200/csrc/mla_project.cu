@@ -367,6 +367,24 @@ cudaError_t launch_projection(const ProjParams& p, bool absorb, cudaStream_t str
   return absorb ? cudaLaunchKernelEx(&cfg, mla_absorb_kernel, p) : cudaLaunchKernelEx(&cfg, mla_up_project_kernel, p);
 }
 
+// Self-test of the bounded wait: one thread waits on a barrier that nothing
+// arrives at; the wait gives up after its limit, raises MLA_DEVERR_TIMEOUT in
+// the sticky word and the kernel returns.
+__global__ void mla_wait_selftest_kernel() {
+  __shared__ __align__(8) uint64_t bar;
+  if (threadIdx.x == 0) {
+    const uint32_t b = smem_u32(&bar);
+    mbar_init(b, 1);
+    fence_mbar_init_cluster();
+    wait_proj(b, 0);
+  }
+}
+
+cudaError_t launch_wait_selftest(cudaStream_t stream) {
+  mla_wait_selftest_kernel<<<1, 32, 0, stream>>>();
+  return cudaGetLastError();
+}
+
 __device__ unsigned int g_mla_project_taken;
 
 __global__ void take_project_sticky_kernel() {

@@ -109,3 +109,23 @@ def test_lengths_changed_since_the_plan_are_flagged():
     torch.cuda.synchronize()
     assert binding.mla_check_device_error(meta) & binding.MLA_DEVERR_PLAN
     assert binding.mla_take_device_errors() & binding.MLA_DEVERR_PLAN
+
+
+def test_a_bounded_wait_that_runs_out_reports_a_timeout_and_the_context_stays_usable():
+    # A barrier nothing arrives at: the wait gives up after its limit (1 s),
+    # raises the timeout bit and the kernel returns; later calls still work.
+    import time
+
+    binding.mla_take_device_errors()
+    t0 = time.perf_counter()
+    binding.mla_selftest_bounded_wait()
+    assert binding.mla_take_device_errors() == binding.MLA_DEVERR_TIMEOUT
+    assert 0.9 < time.perf_counter() - t0 < 30
+    x = inputs.workload_inputs(0)
+    g = x.to("cuda")
+    meta = binding.mla_get_metadata(g.seqlens, g.h_q, g.s_q)
+    out, lse = binding.mla_decode(g.q, g.kv_cache, g.block_table, g.seqlens, g.softmax_scale, g.causal, meta)
+    assert binding.mla_check_device_error(meta) == 0
+    assert binding.mla_take_device_errors() == 0
+    want_out, _ = mla_oracle.decode(x.q, x.kv_cache, x.block_table, x.seqlens, x.softmax_scale, x.causal)
+    assert np.abs(out.cpu().double().numpy() - want_out).max() <= 8e-3
