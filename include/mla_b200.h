@@ -237,8 +237,10 @@ int mla_absorb_q(const void* q_nope, const void* q_rope, const void* w_uk, int t
  *   o_latent [device] bf16 [tokens][h_q][512].
  *   w_uv     [device] bf16 [h_q][512][128]: w_uv[h][c][v] is W_UV^h's entry
  *            for latent dim c and value dim v.
- *   tokens, h_q, errors: as mla_absorb_q.
+ *   h_q      1..128.
  *   o_out    [device] bf16 [tokens][h_q][128].
+ * tokens may be at most 65535 * 64 (the kernel's token tiles are 64 wide);
+ * the other limits and errors are those of mla_absorb_q.
  */
 int mla_up_project(const void* o_latent, const void* w_uv, int tokens, int h_q, void* o_out, void* stream);
 

@@ -165,8 +165,8 @@ int projection_impl(const void* a, const void* extra, const void* w, int tokens,
   if (!a || !w || !out || (absorb && !extra)) return MLA_ERR_ARG;
   if (tokens < 1 || h_q < 1) return MLA_ERR_ARG;
   if (!aligned16(a) || !aligned16(w) || !aligned16(out) || (absorb && !aligned16(extra))) return MLA_ERR_ARG;
-  // grid (h_q, tokens / 128) and 32-bit row offsets
-  if (h_q > kMaxHq || tokens > 65535 * 128) return MLA_ERR_UNSUPPORTED;
+  // the grid's y dimension counts token tiles: at most 65535 of them
+  if (h_q > kMaxHq || tokens > 65535 * (absorb ? kProjAbsorbTile : kProjUpTile)) return MLA_ERR_UNSUPPORTED;
   DeviceInfo dev;
   int st = current_device_info(&dev);
   if (st != MLA_OK) return st;

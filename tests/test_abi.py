@@ -146,6 +146,7 @@ def test_absorb_q_rejects_bad_arguments_on_host(lib, args, status):
     ((16, 16, -1, 16, 16), binding.MLA_ERR_ARG),
     ((16, 16, 4, 0, 16), binding.MLA_ERR_ARG),
     ((16, 16, 4, 200, 16), binding.MLA_ERR_UNSUPPORTED),
+    ((16, 16, 65535 * 64 + 1, 16, 16), binding.MLA_ERR_UNSUPPORTED),  # token tiles past the grid's limit
 ])
 def test_up_project_rejects_bad_arguments_on_host(lib, args, status):
     assert lib.mla_up_project(*args, None) == status
