@@ -189,6 +189,16 @@ def test_causal_multi_token(s_q, h_q):
     assert_parity(x, out, lse)
 
 
+@pytest.mark.parametrize("s_q,h_q,causal", [(16, 128, True), (16, 128, False), (8, 16, True), (16, 1, True),
+                                            (5, 100, True)])
+def test_many_query_tokens_up_to_the_limits(s_q, h_q, causal):
+    # Speculative / multi-token steps up to s_q = 16 and s_q * h_q = 2048 query
+    # rows per batch row (16 work rows of 128), with rows shorter than s_q.
+    x = inputs.make_inputs([7, 16, 17, 300, 1500], h_q, s_q, seed=900 + s_q + h_q, causal=causal)
+    out, lse, _ = run(x)
+    assert_parity(x, out, lse)
+
+
 def test_noncausal_multi_token():
     x = inputs.make_inputs([50, 300], 64, 2, seed=301, causal=False)
     out, lse, _ = run(x)
