@@ -109,3 +109,19 @@ def test_split_of_the_long_context_workload_at_full_size():
     bar = 8e-3 + 2.0 ** -9 * (parts_max + float(np.abs(want_out).max()))
     assert err.max() <= bar and err.mean() <= 1e-3, (err.max(), bar, err.mean())
     assert np.max(np.abs(mla_oracle.as_f64(lse.cpu()) - want_lse)) <= 1e-3
+
+
+def test_decode_sharded_on_one_rank_equals_the_unsplit_call():
+    # Without a process group (one rank) the exchange is the identity and the
+    # merge of a single split must reproduce mla_decode's result exactly
+    # (lse) and to the bf16 rounding of a value that is already bf16 (out).
+    lens = [900, 64, 1]
+    x = inputs.make_inputs(lens, 32, 2, seed=77, causal=True)
+    g = x.to("cuda")
+    table, local = longrow.shard_block_table(g.block_table, lens, 1, 0, x.s_q)
+    out, lse = longrow.decode_sharded(g.q, g.kv_cache, table, local, x.softmax_scale, True)
+    meta = binding.mla_get_metadata(g.seqlens, x.h_q, x.s_q)
+    ref_out, ref_lse = binding.mla_decode(g.q, g.kv_cache, g.block_table, g.seqlens, x.softmax_scale, True, meta)
+    torch.cuda.synchronize()
+    assert torch.equal(out, ref_out)
+    assert torch.allclose(lse, ref_lse, rtol=0, atol=1e-6) or torch.equal(lse, ref_lse)
