@@ -242,3 +242,80 @@ def make_projection_inputs(tokens: int, h_q: int, *, seed: int = 0) -> Projectio
         w_uv=draw(h_q, D_LATENT, D_VH, scale=D_LATENT ** -0.5),
         o_latent=draw(tokens, h_q, D_LATENT),
     )
+
+
+@dataclasses.dataclass
+class Fp8DecodeInputs:
+    """One decode step over an FP8 latent cache: E4M3 codes for the 512 latent
+    dims with one power-of-two scale 2^exp per cached token, bf16 rope."""
+
+    q: torch.Tensor             # [batch, s_q, h_q, 576] bf16
+    latent_codes: torch.Tensor  # [num_pages, 64, 512] uint8 (E4M3 bit patterns)
+    rope: torch.Tensor          # [num_pages, 64, 64] bf16
+    exps: torch.Tensor          # [num_pages, 64] int8 (token scale 2^exp)
+    block_table: torch.Tensor   # [batch, max_pages_per_row] int32
+    seqlens: torch.Tensor       # [batch] int32
+    s_q: int
+    h_q: int
+    causal: bool
+    softmax_scale: float
+
+    @property
+    def batch(self) -> int:
+        return int(self.seqlens.shape[0])
+
+    def to(self, device) -> "Fp8DecodeInputs":
+        return dataclasses.replace(self, q=self.q.to(device), latent_codes=self.latent_codes.to(device),
+                                   rope=self.rope.to(device), exps=self.exps.to(device),
+                                   block_table=self.block_table.to(device), seqlens=self.seqlens.to(device))
+
+
+E4M3_NAN = 0x7F   # S.1111.111
+E4M3_MAX = 0x7E   # 448
+
+
+def make_fp8_inputs(seqlens: Sequence[int], h_q: int, s_q: int = 1, *, seed: int = 0, causal: bool = False,
+                    softmax_scale: float = DEFAULT_SCALE, pool_factor: Optional[float] = 1.25,
+                    exp_range: tuple = (-8, -5)) -> Fp8DecodeInputs:
+    """Paged FP8 decode step drawn on the CPU generator.
+
+    The latent codes are N(0, 64^2) values rounded to E4M3 (so that the
+    codes span the format's range, |v| < 448), each token's exponent is
+    uniform in ``exp_range`` (dequantised values ~ N(0, 1/16 .. 1)), rope and
+    Q are N(0, 1) rounded to bf16.  Pages as in ``make_inputs``: a shuffled
+    pool, table entries past a row's pages on a spare page whose codes are
+    NaN, and slots past L in a row's last page holding the largest code with
+    exponent 5 (14336: finite, large enough to be noticed if read).
+    """
+    gen = torch.Generator()
+    gen.manual_seed(seed)
+    batch = len(seqlens)
+    pages_per_row = [(int(L) + PAGE - 1) // PAGE for L in seqlens]
+    needed = sum(pages_per_row)
+    pool = max(needed, 1) if pool_factor is None else max(int(math.ceil(pool_factor * needed)), needed + 1)
+    perm = torch.randperm(pool, generator=gen)
+    spare = int(perm[needed]) if pool > needed else 0
+    width = max(max(pages_per_row, default=0), 1)
+    table = torch.full((batch, width), spare, dtype=torch.int32)
+    cursor = 0
+    for i, n in enumerate(pages_per_row):
+        table[i, :n] = perm[cursor:cursor + n].to(torch.int32)
+        cursor += n
+    q = torch.randn(batch, s_q, h_q, D_QK, generator=gen).to(torch.bfloat16)
+    codes = (torch.randn(pool, PAGE, D_LATENT, generator=gen) * 64.0).to(torch.float8_e4m3fn).view(torch.uint8)
+    rope = torch.randn(pool, PAGE, D_ROPE, generator=gen).to(torch.bfloat16)
+    exps = torch.randint(exp_range[0], exp_range[1] + 1, (pool, PAGE), generator=gen, dtype=torch.int64).to(torch.int8)
+    used = torch.zeros(pool, dtype=torch.bool)
+    used[perm[:needed]] = True
+    unused = (~used).nonzero().flatten()
+    if unused.numel():
+        codes[unused] = E4M3_NAN
+        rope[unused] = float("nan")
+    for i, (L, n) in enumerate(zip(seqlens, pages_per_row)):
+        if n and int(L) % PAGE:
+            last = int(table[i, n - 1])
+            codes[last, int(L) % PAGE:] = E4M3_MAX
+            exps[last, int(L) % PAGE:] = 5
+    return Fp8DecodeInputs(q=q, latent_codes=codes.contiguous(), rope=rope, exps=exps, block_table=table,
+                           seqlens=torch.tensor([int(L) for L in seqlens], dtype=torch.int32), s_q=s_q, h_q=h_q,
+                           causal=causal, softmax_scale=softmax_scale)

@@ -31,6 +31,15 @@ are split across processors and merged.  ``partial_attention`` and
 the integer tile-scheduler plan of the CUDA path's metadata kernel, restated
 here from its definition so that the plan can be compared bit for bit.
 
+"MLA 和 MHA 的 Kernel 区别", section "量化友好性": the latent ``c_KV`` may be
+cached quantised (FP8 or INT8), the dequantisation fused with the load.  The
+pages fix no format; ``e4m3_value``, ``dequantize_latent`` and ``decode_fp8``
+take the plainest reading: the 512 latent dims of a cached token are OCP FP8
+E4M3 codes with one power-of-two scale 2^e per token, and the 64 rope dims
+(not part of ``c_KV``) stay bf16.  Every E4M3 value times a power of two is
+exact in bf16, so the attention over the dequantised cache is again the
+definition above.
+
 Readings where the pages are silent (parity unpinned by the pages themselves;
 the tests pin them only to these stated conventions):
   * causal decode with ``s_q > 1``: the ``s_q`` new tokens are the last
@@ -219,6 +228,45 @@ def decode_unabsorbed(c_kv, k_rope, q_nope, q_rope, w_uk, w_uv, scale: float,
         o, l = attend(q_h, k_h, v_h, scale, [L])
         out[h], lse[h] = o[0], l[0]
     return out, lse
+
+
+# --------------------------------------------------------------------------
+# FP8 (E4M3) latent cache
+# --------------------------------------------------------------------------
+
+def e4m3_value(codes) -> np.ndarray:
+    """float64 value of OCP FP8 E4M3 codes (uint8): 1 sign bit, 4 exponent
+    bits with bias 7, 3 mantissa bits; exponent field 0 is subnormal
+    (m / 8 * 2^-6); no infinities; S.1111.111 is NaN; the largest finite
+    value is 448."""
+    c = np.asarray(codes, dtype=np.int64)
+    sign = np.where(c & 0x80, -1.0, 1.0)
+    e = (c >> 3) & 0xF
+    m = c & 0x7
+    normal = (1.0 + m / 8.0) * np.power(2.0, e - 7)
+    subnormal = (m / 8.0) * 2.0 ** -6
+    v = sign * np.where(e == 0, subnormal, normal)
+    return np.where((c & 0x7F) == 0x7F, np.nan, v)
+
+
+def dequantize_latent(codes, exps) -> np.ndarray:
+    """Latent rows from FP8 codes [..., 512] and per-token exponents [...]:
+    e4m3_value(code) * 2^exp, in float64."""
+    e = np.asarray(as_int(exps), dtype=np.float64)
+    return e4m3_value(as_int(codes)) * np.power(2.0, e)[..., None]
+
+
+def decode_fp8(q, latent_codes, rope, exps, block_table, seqlens, softmax_scale: float, causal: bool,
+               rows: Sequence[int] = None) -> Tuple[np.ndarray, np.ndarray]:
+    """``decode`` over an FP8 latent cache.
+
+    latent_codes [num_pages, 64, 512] uint8 (E4M3), rope [num_pages, 64, 64]
+    (bf16 or float), exps [num_pages, 64] integer (token scale 2^exp).  Each
+    cached row is [dequantised latent, rope]; the rest is ``decode``.
+    """
+    lat = dequantize_latent(latent_codes, exps)
+    pool = np.concatenate([lat, as_f64(rope)], axis=-1)[:, :, None, :]  # [pages, 64, 1, 576]
+    return decode(q, pool, block_table, seqlens, softmax_scale, causal, rows=rows)
 
 
 def absorb_query(q_nope, q_rope, w_uk) -> np.ndarray:

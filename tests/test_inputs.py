@@ -47,3 +47,26 @@ def test_length_recipes():
     assert min(u) >= 1024 and max(u) <= 4096
     n = I.draw_lengths(("normal", 8192.0, 2048.0, 256, 16384), 500, g)
     assert min(n) >= 256 and max(n) <= 16384 and 7500 < sum(n) / len(n) < 8900
+
+
+def test_fp8_inputs_layout():
+    x = I.make_fp8_inputs([300, 64, 1, 0, 130], 8, 2, seed=5)
+    pool = x.latent_codes.shape[0]
+    assert x.latent_codes.dtype == torch.uint8 and x.latent_codes.shape[1:] == (64, 512)
+    assert x.rope.shape == (pool, 64, 64) and x.exps.shape == (pool, 64)
+    lens = [int(v) for v in x.seqlens]
+    used = set()
+    for i, L in enumerate(lens):
+        n = (L + 63) // 64
+        pages = [int(p) for p in x.block_table[i, :n]]
+        used |= set(pages)
+        for j in range(L):  # every visible token: finite codes, exponent in range
+            p, sl = pages[j // 64], j % 64
+            assert not bool(((x.latent_codes[p, sl] & 0x7F) == 0x7F).any())
+            assert -8 <= int(x.exps[p, sl]) <= -5
+        if n and L % 64:  # slots past L in the last page: largest code, exponent 5
+            assert bool((x.latent_codes[pages[-1], L % 64:] == 0x7E).all())
+            assert bool((x.exps[pages[-1], L % 64:] == 5).all())
+    assert len(used) == sum((L + 63) // 64 for L in lens)
+    for p in set(range(pool)) - used:  # pages no row holds: NaN codes
+        assert bool((x.latent_codes[p] == 0x7F).all())

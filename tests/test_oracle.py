@@ -286,12 +286,62 @@ def pin_monotone_scores(O):
         assert abs(lse[0, k, 0] - (m + math.log(s))) < 1e-12
 
 
+def pin_e4m3_codes(O):
+    # Every E4M3 bit pattern against torch's float8_e4m3fn conversion (a
+    # library routine), and closed forms of the format: 0x7E = 448 (largest),
+    # 0x01 = 2^-9 (smallest subnormal), 0x08 = 2^-6 (smallest normal),
+    # 0x38 = 1, 0xB8 = -1, 0x00 = 0, S.1111.111 = NaN.
+    import torch
+
+    codes = np.arange(256, dtype=np.uint8)
+    mine = O.e4m3_value(codes)
+    lib = torch.from_numpy(codes).view(torch.float8_e4m3fn).to(torch.float64).numpy()
+    assert np.array_equal(np.isnan(mine), np.isnan(lib))
+    assert np.array_equal(mine[~np.isnan(mine)], lib[~np.isnan(lib)])
+    want = {0x7E: 448.0, 0x01: 2.0 ** -9, 0x08: 2.0 ** -6, 0x38: 1.0, 0xB8: -1.0, 0x00: 0.0}
+    for c, v in want.items():
+        assert O.e4m3_value([c])[0] == v, hex(c)
+    assert np.isnan(O.e4m3_value([0x7F, 0xFF])).all()
+
+
+def pin_fp8_dequantized_values_are_bf16_exact(O):
+    import torch
+
+    rng = np.random.default_rng(31)
+    codes = rng.integers(0, 256, size=(64, 512)).astype(np.uint8)
+    codes[(codes & 0x7F) == 0x7F] = 0x7E
+    exps = rng.integers(-20, 21, size=64)
+    lat = O.dequantize_latent(codes, exps)
+    back = torch.from_numpy(lat).to(torch.bfloat16).double().numpy()
+    assert np.array_equal(back, lat)
+
+
+def pin_fp8_decode_equals_bf16_decode(O):
+    # The FP8 path against the pinned bf16 decode over a cache assembled
+    # independently: torch's float8 conversion times 2^exp, rope appended.
+    import torch
+
+    from mla_decode_attention_13_b200 import inputs as I
+
+    x = I.make_fp8_inputs([300, 64, 1, 0, 130], 8, 2, seed=21, causal=True)
+    lat = x.latent_codes.view(torch.float8_e4m3fn).to(torch.float64) * torch.pow(2.0, x.exps.to(torch.float64))[..., None]
+    pool = torch.cat([lat, x.rope.to(torch.float64)], dim=-1)[:, :, None, :].numpy()
+    want_o, want_l = O.decode(x.q, pool, x.block_table, x.seqlens, x.softmax_scale, True)
+    got_o, got_l = O.decode_fp8(x.q, x.latent_codes, x.rope, x.exps, x.block_table, x.seqlens, x.softmax_scale,
+                                True)
+    np.testing.assert_allclose(got_o, want_o, rtol=0, atol=1e-12)
+    np.testing.assert_array_equal(np.isneginf(got_l), np.isneginf(want_l))
+    fin = np.isfinite(want_l)
+    np.testing.assert_allclose(got_l[fin], want_l[fin], rtol=0, atol=1e-12)
+
+
 NUMERIC_PINS = [
     pin_golden_three_tokens, pin_single_token, pin_two_tokens, pin_brute_force_small,
     pin_constant_cache, pin_weights_sum_to_one, pin_absorbed_equals_unabsorbed,
     pin_paged_equals_contiguous, pin_split_combine_equals_single, pin_head_permutation,
     pin_constant_shift, pin_causal_single_token_is_noncausal, pin_causal_two_tokens,
     pin_library_sdpa, pin_empty_rows, pin_monotone_scores,
+    pin_e4m3_codes, pin_fp8_dequantized_values_are_bf16_exact, pin_fp8_decode_equals_bf16_decode,
 ]
 
 
@@ -461,9 +511,41 @@ def _mut_expand_heads_reversed(mp):
     mp.setattr(O, "expand_output", lambda o, w: orig(o, O.as_f64(w)[::-1]))
 
 
+def _mut_e4m3_bias_8(mp):
+    orig = O.e4m3_value
+    mp.setattr(O, "e4m3_value", lambda c: orig(c) / 2.0)
+
+
+def _mut_e4m3_subnormal_scale(mp):
+    orig = O.e4m3_value
+
+    def v(c):
+        out = orig(c)
+        sub = ((np.asarray(c, dtype=np.int64) >> 3) & 0xF) == 0
+        return np.where(sub, out / 2.0, out)
+    mp.setattr(O, "e4m3_value", v)
+
+
+def _mut_fp8_scale_inverted(mp):
+    mp.setattr(O, "dequantize_latent",
+               lambda codes, exps: O.e4m3_value(O.as_int(codes)) * np.power(2.0, -O.as_int(exps).astype(float))[..., None])
+
+
+def _mut_fp8_rope_scaled(mp):
+    orig = O.decode
+
+    def decode_fp8(q, codes, rope, exps, table, lens, scale, causal, rows=None):
+        lat = O.dequantize_latent(codes, exps)
+        r = O.as_f64(rope) * np.power(2.0, O.as_int(exps).astype(float))[..., None]
+        pool = np.concatenate([lat, r], axis=-1)[:, :, None, :]
+        return orig(q, pool, table, lens, scale, causal, rows=rows)
+    mp.setattr(O, "decode_fp8", decode_fp8)
+
+
 MUTATIONS = [_mut_drop_rope, _mut_rope_sign, _mut_value_window, _mut_no_scale, _mut_causal_off_by_one,
              _mut_ignore_table, _mut_slot_major, _mut_log2_lse, _mut_unnormalised, _mut_combine_mean,
-             _mut_absorb_one_head, _mut_absorb_drops_rope, _mut_expand_heads_reversed]
+             _mut_absorb_one_head, _mut_absorb_drops_rope, _mut_expand_heads_reversed,
+             _mut_e4m3_bias_8, _mut_e4m3_subnormal_scale, _mut_fp8_scale_inverted, _mut_fp8_rope_scaled]
 
 
 @pytest.mark.parametrize("mutation", MUTATIONS, ids=lambda f: f.__name__)
