@@ -214,7 +214,9 @@ __global__ void __launch_bounds__(kProjThreads, 8) mla_absorb_kernel(const __gri
     }
     umma_commit(bars + kBD);  // after the MMAs (or at once, with none issued)
   }
-  __syncwarp();
+  // Every thread sees the issuer's ok flag past here (the accumulator
+  // barrier's arrive comes from the tensor core and orders only its results).
+  __syncthreads();
 
   // Read-out: the accumulator holds latent dims [128 c, +128) of the tile's
   // tokens; thread (warp, lane) owns dim 128 c + 32 warp + lane.
@@ -318,7 +320,7 @@ __global__ void __launch_bounds__(kProjThreads, 4) mla_up_project_kernel(const _
       for (int c = landed; c < kChunks; ++c) wait_proj(bars + kBW + 8 * c, 0, false);
     }
   }
-  __syncwarp();
+  __syncthreads();  // the issuer's ok flag, as in the absorb kernel
 
   __nv_bfloat16* out = reinterpret_cast<__nv_bfloat16*>(p.out);
   const long long row_stride = static_cast<long long>(p.h_q) * 128;
