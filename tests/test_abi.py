@@ -168,3 +168,28 @@ def test_up_project_rejects_bad_arguments_on_host(lib, args, status):
 ])
 def test_merge_splits_rejects_bad_arguments_on_host(lib, args, status):
     assert lib.mla_merge_splits(*args, None) == status
+
+
+def test_binding_checks_projection_and_merge_shapes_before_the_library(lib):
+    # Shape and dtype errors are raised by the binding itself (MLA_ERR_ARG),
+    # before any pointer reaches the library; CPU tensors suffice.
+    import torch
+
+    bf = torch.bfloat16
+    w = torch.zeros(4, 512, 128, dtype=bf)
+    cases = [
+        lambda: binding.mla_absorb_q(torch.zeros(2, 4, 127, dtype=bf), torch.zeros(2, 4, 64, dtype=bf), w),
+        lambda: binding.mla_absorb_q(torch.zeros(2, 4, 128, dtype=bf), torch.zeros(2, 4, 32, dtype=bf), w),
+        lambda: binding.mla_absorb_q(torch.zeros(2, 4, 128), torch.zeros(2, 4, 64, dtype=bf), w),
+        lambda: binding.mla_absorb_q(torch.zeros(2, 3, 128, dtype=bf), torch.zeros(2, 3, 64, dtype=bf), w),
+        lambda: binding.mla_up_project(torch.zeros(2, 4, 511, dtype=bf), w),
+        lambda: binding.mla_up_project(torch.zeros(2, 4, 512, dtype=bf), w.transpose(1, 2)),
+        lambda: binding.mla_up_project(torch.zeros(2, 4, 512, dtype=bf), w, out=torch.zeros(2, 4, 64, dtype=bf)),
+        lambda: binding.mla_merge_splits(torch.zeros(2, 1, 1, 4, 512, dtype=bf), torch.zeros(2, 1, 1, 4)),
+        lambda: binding.mla_merge_splits(torch.zeros(2, 1, 1, 4, 512), torch.zeros(2, 1, 4, 1)),
+        lambda: binding.mla_merge_splits(torch.zeros(1, 4, 512, dtype=bf), torch.zeros(1, 4)),
+    ]
+    for k, call in enumerate(cases):
+        with pytest.raises(binding.MLAError) as e:
+            call()
+        assert e.value.status == binding.MLA_ERR_ARG, k
