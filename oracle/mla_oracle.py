@@ -256,6 +256,44 @@ def dequantize_latent(codes, exps) -> np.ndarray:
     return e4m3_value(as_int(codes)) * np.power(2.0, e)[..., None]
 
 
+def _e4m3_table() -> Tuple[np.ndarray, np.ndarray]:
+    """The finite E4M3 values in increasing order, with their codes."""
+    codes = np.array([c for c in range(256) if (c & 0x7F) != 0x7F], dtype=np.int64)
+    vals = e4m3_value(codes)
+    order = np.lexsort((codes, vals))
+    return vals[order], codes[order]
+
+
+def quantize_latent(rows) -> Tuple[np.ndarray, np.ndarray]:
+    """The cache writer's side of the FP8 format: per token (last axis = 512
+    latent dims) the exponent e is the smallest integer with
+    max|x| / 2^e <= 448 (e = 0 for an all-zero row), and each code is x / 2^e
+    rounded to the nearest E4M3 value, ties to the even mantissa.  Returns
+    (codes uint8 [..., 512], exps int64 [...])."""
+    x = as_f64(rows)
+    amax = np.max(np.abs(x), axis=-1)
+    e = np.zeros(amax.shape, dtype=np.int64)
+    nz = amax > 0
+    e[nz] = np.ceil(np.log2(amax[nz] / 448.0)).astype(np.int64)
+    # log2 rounding can leave e one too small or too large: settle it exactly
+    e[nz] += (amax[nz] / np.power(2.0, e[nz]) > 448.0)
+    e[nz] -= (amax[nz] / np.power(2.0, e[nz] - 1) <= 448.0)
+    y = x / np.power(2.0, e.astype(np.float64))[..., None]
+    vals, codes = _e4m3_table()
+    # the codes with the sign bit clear (+0 .. 448), for rounding |y|
+    pos = (codes & 0x80) == 0
+    pv, pc = vals[pos], codes[pos]
+    a = np.abs(y)
+    hi = np.clip(np.searchsorted(pv, a, side="left"), 1, len(pv) - 1)
+    lo = hi - 1
+    d_lo, d_hi = a - pv[lo], pv[hi] - a
+    take_hi = (d_hi < d_lo) | ((d_hi == d_lo) & ((pc[hi] & 1) == 0))
+    mag = np.where(take_hi, pc[hi], pc[lo])
+    mag = np.where(a >= pv[-1], pc[-1], mag)
+    code = np.where(np.signbit(y), mag | 0x80, mag)  # the sign is kept, on zero too
+    return code.astype(np.uint8), e
+
+
 def decode_fp8(q, latent_codes, rope, exps, block_table, seqlens, softmax_scale: float, causal: bool,
                rows: Sequence[int] = None) -> Tuple[np.ndarray, np.ndarray]:
     """``decode`` over an FP8 latent cache.

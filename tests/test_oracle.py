@@ -335,6 +335,32 @@ def pin_fp8_decode_equals_bf16_decode(O):
     np.testing.assert_allclose(got_l[fin], want_l[fin], rtol=0, atol=1e-12)
 
 
+def pin_fp8_quantizer(O):
+    # The writer's exponent puts each row's largest magnitude in (224, 448];
+    # codes equal torch's float8_e4m3fn rounding (nearest, ties to even) of
+    # x / 2^e; the round trip errs by at most half an E4M3 step, 2^-4 |x| in
+    # the normal range and 2^-10 2^e below it; dequantised rows quantise back
+    # to the same values; an all-zero row gets e = 0 and zero codes.
+    import torch
+
+    rng = np.random.default_rng(41)
+    x = rng.standard_normal((300, 512)) * rng.uniform(1e-3, 1e3, size=(300, 1))
+    x[7] = 0.0
+    codes, e = O.quantize_latent(x)
+    amax = np.abs(x).max(axis=1)
+    r = amax[amax > 0] / np.power(2.0, e[amax > 0])
+    assert np.all((r > 224.0) & (r <= 448.0))
+    assert e[7] == 0 and not codes[7].any()
+    y = x / np.power(2.0, e)[:, None]
+    lib = torch.from_numpy(y).to(torch.float8_e4m3fn).view(torch.uint8).numpy()
+    assert np.array_equal(lib, codes)
+    deq = O.dequantize_latent(codes, e)
+    step = np.maximum(2.0 ** -4 * np.abs(x), 2.0 ** -10 * np.power(2.0, e)[:, None])
+    assert np.all(np.abs(deq - x) <= step)
+    codes2, e2 = O.quantize_latent(deq)
+    assert np.array_equal(O.dequantize_latent(codes2, e2), deq)
+
+
 NUMERIC_PINS = [
     pin_golden_three_tokens, pin_single_token, pin_two_tokens, pin_brute_force_small,
     pin_constant_cache, pin_weights_sum_to_one, pin_absorbed_equals_unabsorbed,
@@ -342,6 +368,7 @@ NUMERIC_PINS = [
     pin_constant_shift, pin_causal_single_token_is_noncausal, pin_causal_two_tokens,
     pin_library_sdpa, pin_empty_rows, pin_monotone_scores,
     pin_e4m3_codes, pin_fp8_dequantized_values_are_bf16_exact, pin_fp8_decode_equals_bf16_decode,
+    pin_fp8_quantizer,
 ]
 
 
@@ -542,10 +569,20 @@ def _mut_fp8_rope_scaled(mp):
     mp.setattr(O, "decode_fp8", decode_fp8)
 
 
+def _mut_quantize_exponent_high(mp):
+    orig = O.quantize_latent
+
+    def q(rows):
+        codes, e = orig(rows)
+        return orig(O.as_f64(rows) / 2.0)[0], e + 1
+    mp.setattr(O, "quantize_latent", q)
+
+
 MUTATIONS = [_mut_drop_rope, _mut_rope_sign, _mut_value_window, _mut_no_scale, _mut_causal_off_by_one,
              _mut_ignore_table, _mut_slot_major, _mut_log2_lse, _mut_unnormalised, _mut_combine_mean,
              _mut_absorb_one_head, _mut_absorb_drops_rope, _mut_expand_heads_reversed,
-             _mut_e4m3_bias_8, _mut_e4m3_subnormal_scale, _mut_fp8_scale_inverted, _mut_fp8_rope_scaled]
+             _mut_e4m3_bias_8, _mut_e4m3_subnormal_scale, _mut_fp8_scale_inverted, _mut_fp8_rope_scaled,
+             _mut_quantize_exponent_high]
 
 
 @pytest.mark.parametrize("mutation", MUTATIONS, ids=lambda f: f.__name__)
