@@ -107,8 +107,8 @@ __device__ bool wait_proj(uint32_t bar, uint32_t parity, bool raise = true) {
   }
 }
 
-// Width of one accumulator of nb token columns: nb rounded up to 32, so that
-// the read-out's 32-column loads stay inside it.
+// Width of one accumulator of nb token columns: nb rounded up to 32 (the
+// smallest TMEM allocation); the read-out's 16-column loads stay inside it.
 __device__ __forceinline__ uint32_t slot_width(int nb) { return (static_cast<uint32_t>(nb) + 31u) & ~31u; }
 
 // TMEM columns to allocate for `slots` accumulators: a power of two from 32 to
@@ -182,7 +182,9 @@ __global__ void __launch_bounds__(kProjThreads, 8) mla_absorb_kernel(const __gri
     mbar_init(bars + kBFin, 1);
     *ok_flag = 1u;
     fence_mbar_init_cluster();
-    prefetch_l2(w_chunk, kWChunk);  // the weights are not written by the kernels this one waits for
+    // Before the dependency wait: a prefetch only warms L2, the point of
+    // coherence, so it cannot return stale data whatever runs before.
+    prefetch_l2(w_chunk, kWChunk);
   }
   if (warp == 0) {
     tmem_alloc(bars + kTmemSlot, ncols);
@@ -273,7 +275,7 @@ __global__ void __launch_bounds__(kProjThreads, 4) mla_up_project_kernel(const _
     mbar_init(bars + kBFin, 1);
     *ok_flag = 1u;
     fence_mbar_init_cluster();
-    // W_UV^h is not written by the kernels this one waits for
+    // W_UV^h into L2 before the dependency wait (a hint, as in the absorb)
     const char* w_head = static_cast<const char*>(p.w) + static_cast<size_t>(h) * kDv * 256;
     for (int c = 0; c < kChunks; ++c) prefetch_l2(w_head + c * kWChunk, kWChunk);
   }
