@@ -124,3 +124,75 @@ def test_gloo_ranks_exchange_partials_that_merge_to_the_unsplit_decode(world, ca
     res = sorted(q.get(timeout=5) for _ in range(world))
     for rank, err, lerr, same_inf in res:
         assert err < 1e-12 and lerr < 1e-12 and same_inf, (rank, err, lerr, same_inf)
+
+
+def _sharded_worker(rank, world, port, case, q):
+    # longrow.decode_sharded itself across gloo ranks, with the library calls
+    # replaced by oracle-backed stand-ins: this checks the orchestration (which
+    # rank masks, the gather order, what reaches the merge).
+    sys.path.insert(0, ROOT)
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port), RANK=str(rank), WORLD_SIZE=str(world))
+    import datetime
+    import types
+
+    import torch.distributed as dist
+
+    from mla_decode_attention_13_b200 import inputs, longrow
+    from oracle import mla_oracle
+
+    calls = []
+
+    def get_metadata(seqlens, h_q, s_q, metadata=None, stream=None):
+        return ("plan", tuple(int(v) for v in seqlens))
+
+    def decode(q, kv, table, seqlens, scale, causal, meta, **kw):
+        assert meta == ("plan", tuple(int(v) for v in seqlens))
+        calls.append(bool(causal))
+        o, l = mla_oracle.decode(q, kv, table, seqlens, scale, causal)
+        return torch.from_numpy(o), torch.from_numpy(l)
+
+    def merge(outs, lses, **kw):
+        w, b, s, h, _ = outs.shape
+        parts = [(outs[k].numpy().reshape(b * s * h, 512), lses[k].numpy().transpose(0, 2, 1).reshape(-1))
+                 for k in range(w)]
+        o, l = mla_oracle.combine_partials(parts)
+        return torch.from_numpy(o.reshape(b, s, h, 512)), torch.from_numpy(l.reshape(b, s, h).transpose(0, 2, 1))
+
+    longrow.binding = types.SimpleNamespace(mla_get_metadata=get_metadata, mla_decode=decode,
+                                            mla_merge_splits=merge)
+    dist.init_process_group("gloo", rank=rank, world_size=world, timeout=datetime.timedelta(seconds=60))
+    try:
+        lens, h_q, s_q, causal = case
+        x = inputs.make_inputs(lens, h_q, s_q, seed=23, causal=causal)
+        table, local = longrow.shard_block_table(x.block_table, lens, world, rank, s_q)
+        out, lse = longrow.decode_sharded(x.q, x.kv_cache, table, local, x.softmax_scale, causal)
+        want_out, want_lse = mla_oracle.decode(x.q, x.kv_cache, x.block_table, x.seqlens, x.softmax_scale, causal)
+        err = float(np.max(np.abs(out.numpy() - want_out)))
+        fin = np.isfinite(want_lse)
+        lerr = float(np.max(np.abs(lse.numpy()[fin] - want_lse[fin]))) if fin.any() else 0.0
+        same_inf = bool(np.array_equal(np.isneginf(lse.numpy()), np.isneginf(want_lse)))
+        q.put((rank, err, lerr, same_inf, calls))
+    finally:
+        dist.destroy_process_group()
+
+
+@pytest.mark.timeout(180)
+@pytest.mark.parametrize("world,case", [
+    (2, ([300, 65, 3, 130, 700], 4, 3, True)),
+    (3, ([1000, 129, 64, 2, 0], 2, 1, False)),
+])
+def test_decode_sharded_over_gloo_ranks_equals_the_unsplit_decode(world, case):
+    port = _free_port()
+    ctx = mp.get_context("spawn")
+    q = ctx.Queue()
+    procs = [ctx.Process(target=_sharded_worker, args=(r, world, port, case, q)) for r in range(world)]
+    for p in procs:
+        p.start()
+    for p in procs:
+        p.join(170)
+    assert all(p.exitcode == 0 for p in procs)
+    res = sorted(q.get(timeout=5) for _ in range(world))
+    causal = case[3]
+    for rank, err, lerr, same_inf, calls in res:
+        assert err < 1e-12 and lerr < 1e-12 and same_inf, (rank, err, lerr)
+        assert calls == [causal and rank == world - 1]  # one decode per rank; only the last one masks
