@@ -1,19 +1,35 @@
 """Benchmark of the MLA decode hot path on B200 (one JSON line on rank 0).
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference] [--workload I]
+                    [--no-cpu-baseline] [--headline-only]
 
 A step is one pass of the whole path over one batch: the split-KV plan
 (mla_get_metadata), the split-KV decode kernel and the log-sum-exp combine
-(mla_decode), on inputs already resident in HBM.  The workload defaults to
-batch 16, s_q 1, h_q 128, lengths uniform in [1024, 4096] (64-token pages,
-1.25x shuffled pool, bf16 N(0, 1)).  Calls rotate over several independent
-pools whose total size is at least 3x the L2 cache, so each step reads its
-cache from HBM.  The timed region replays CUDA graphs of those steps (exactly
-K steps, no event nodes between the kernels so that programmatic dependent
-launch applies), bracketed by a barrier and a device synchronisation, timed
-with CUDA events on the launching stream; the split-KV kernel is also timed on
-its own, by graphs of the same steps with events recorded around it, replayed
-right after the timed region.
+(mla_decode), on inputs already resident in HBM.  The workload defaults to the
+largest one-GPU configuration: the compute-bound speculative decode, batch
+128, s_q 2 (causal within the two new tokens), h_q 128, 4096 cached tokens
+per row (64-token pages, 1.25x shuffled pool, bf16 N(0, 1)).  Calls rotate
+over several independent pools whose total size is at least 3x the L2 cache,
+so each step reads its cache from HBM.  The timed region replays CUDA graphs
+of those steps (exactly K steps, no event nodes between the kernels so that
+programmatic dependent launch applies), bracketed by a barrier and a device
+synchronisation, timed with CUDA events on the launching stream; the split-KV
+kernel is also timed on its own, by graphs of the same steps with events
+recorded around it, replayed right after the timed region.
+
+The line also carries, for the headline workload:
+  * `parity`: the GPU result on the workload's seeded inputs against the fp64
+    oracle, element by element (every row when the oracle finishes them in
+    about 25 s, else a seeded sample of at least 8 rows with the shortest and
+    longest), with the benchmark spec's bars;
+  * `cpu_baseline`: that same oracle run, timed and scaled to a full call;
+  * `e2e`: the public API with pinned host buffers, inputs in and results out
+    every step (at least 200 steps, rotating over the pools);
+  * the projections either side of the decode and the split of one row over
+    emulated ranks;
+and, unless --headline-only, the same decode-kernel roofline, step time and
+parity sample for the other four workloads (`memory_bound` is the
+memory-bound sweep, `other_workloads` the rest).
 
 With --gpus N > 1 (launched by torchrun, one process per GPU, NCCL), every
 rank runs its own batch (batch rows are independent: weak scaling, no
@@ -32,11 +48,11 @@ import hashlib
 import json
 import math
 import os
-import re
 import sys
 import threading
 import time
 
+import numpy as np
 import torch
 
 ROOT = os.path.dirname(os.path.abspath(__file__))
@@ -45,9 +61,15 @@ sys.path.insert(0, ROOT)
 from mla_decode_attention_13_b200 import binding, inputs  # noqa: E402
 
 METRIC = "MLA decode µs/call, achieved HBM GB/s and TFLOPS vs B200 roofline (1 GPU)"
+DEFAULT_WORKLOAD = 3  # b128_s2_h128_L4k_causal: the largest configuration by bytes and FLOPs
 FALLBACK_HBM_GBS = 6650.0
 FALLBACK_BF16_TFLOPS = 1590.0
 KERNEL_SOURCES = ("mla_decode.cu", "sm100_ptx.cuh", "mla_internal.h")
+TRAFFIC_FILE = os.path.join(ROOT, "profiles", "mla_decode_kernel_traffic.json")
+TOL_MAX, TOL_MEAN, TOL_LSE = 8e-3, 1e-3, 1e-3
+# How every workload keeps its reads out of L2 between timed steps (the same
+# words in both arms' config).
+L2_NOTE = "inputs larger than L2: calls rotate over cache pools totalling at least 3x the L2 size"
 
 
 # ----------------------------------------------------------------------------
@@ -128,18 +150,18 @@ def kernel_source_sha():
 
 
 def committed_traffic(workload_name):
-    """DRAM bytes per decode-kernel launch from the committed ncu summary, if
-    it was taken on the current kernel source (else None)."""
-    path = os.path.join(ROOT, "profiles", "mla_decode_kernel_traffic.md")
-    if not os.path.exists(path):
+    """DRAM bytes (read + write) per decode-kernel launch from the ncu capture
+    recorded in profiles/mla_decode_kernel_traffic.json, if that capture was
+    taken on the current kernel source (else None)."""
+    try:
+        with open(TRAFFIC_FILE) as f:
+            d = json.load(f)
+    except (OSError, ValueError):
         return None
-    sha = kernel_source_sha()
-    pat = re.compile(r"traffic_bytes_per_launch:\s*(\d+)\s+workload:\s*(\S+)\s+source_sha:\s*([0-9a-f]+)")
-    for line in open(path):
-        m = pat.search(line)
-        if m and m.group(2) == workload_name and m.group(3) == sha:
-            return int(m.group(1))
-    return None
+    if d.get("source_sha") != kernel_source_sha():
+        return None
+    v = d.get("workloads", {}).get(workload_name)
+    return int(v) if v is not None else None
 
 
 # ----------------------------------------------------------------------------
@@ -249,7 +271,7 @@ def dist_teardown(world: int):
 
 
 # ----------------------------------------------------------------------------
-# the reference arm: the fp64 CPU oracle
+# the oracle: the reference arm, the CPU baseline and the parity check
 # ----------------------------------------------------------------------------
 
 def cpu_threads():
@@ -277,20 +299,19 @@ def time_oracle_rows(x, rows_per_step, steps, warmup):
     return times
 
 
-def cpu_baseline(idx, budget_s):
-    """The oracle, as it stands, on whole calls of the workload for about budget_s."""
-    from oracle import mla_oracle
+def workload_config(wl, idx, lens):
+    """The workload's description, the same in both arms."""
+    rec = wl.lengths
+    return {"workload": wl.name, "batch": wl.batch, "s_q": wl.s_q, "h_q": wl.h_q, "h_kv": 1, "d_qk": 576,
+            "d_v": 512, "page": 64, "causal": wl.causal, "lengths": str(rec[0]) + str(list(rec[1:]))[:60],
+            "tokens": int(sum(lens)), "seed": 1000 + idx, "l2": L2_NOTE}
 
-    x = inputs.workload_inputs(idx)
-    times = []
-    t_start = time.perf_counter()
-    while not times or (time.perf_counter() - t_start < budget_s and len(times) < 50):
-        t0 = time.perf_counter()
-        mla_oracle.decode(x.q, x.kv_cache, x.block_table, x.seqlens, x.softmax_scale, x.causal)
-        times.append(time.perf_counter() - t0)
-    per_call = sum(times) / len(times)
-    return {"value": round(per_call * 1e6, 1), "unit": "us/call", "cores": cpu_threads(), "kind": "oracle",
-            "sample": f"{len(times)} whole oracle calls (fp64 NumPy, all {x.batch} rows) of the same workload"}
+
+def workload_lengths(idx):
+    wl = inputs.WORKLOADS[idx]
+    gen = torch.Generator()
+    gen.manual_seed(1000 + idx)
+    return inputs.draw_lengths(wl.lengths, wl.batch, gen)
 
 
 def reference_arm(args, world, rank):
@@ -313,7 +334,7 @@ def reference_arm(args, world, rank):
         "impl": "reference", "metric": METRIC, "value": round(us_per_call, 3), "unit": "us/call", "n_gpus": world,
         "steps": steps, "warmup": warmup, "ms_per_step": round(per_row * 1e3, 4), "higher_is_better": False,
         "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-        "config": workload_config(wl, idx, lens, None),
+        "config": workload_config(wl, idx, lens),
         "achieved_gbs": round(nbytes / (us_per_call * 1e-6) / 1e9, 3),
         "achieved_tflops": round(flops / (us_per_call * 1e-6) / 1e12, 6),
         "cpu_baseline": {"value": round(us_per_call, 3), "unit": "us/call", "cores": cpu_threads(), "kind": "oracle",
@@ -324,193 +345,248 @@ def reference_arm(args, world, rank):
     print(json.dumps(line), flush=True)
 
 
-def workload_config(wl, idx, lens, l2_note):
-    rec = wl.lengths
-    c = {"workload": wl.name, "batch": wl.batch, "s_q": wl.s_q, "h_q": wl.h_q, "h_kv": 1, "d_qk": 576, "d_v": 512,
-         "page": 64, "causal": wl.causal, "lengths": str(rec[0]) + str(list(rec[1:]))[:60],
-         "tokens": int(sum(lens)), "seed": 1000 + idx}
-    if l2_note:
-        c["l2"] = l2_note
-    return c
+def sample_rows(lens, k, seed):
+    """A seeded sample of k batch rows that includes the shortest and the longest."""
+    order = sorted(range(len(lens)), key=lambda i: (lens[i], i))
+    rows = {order[0], order[-1]}
+    rng = np.random.default_rng(seed)
+    for i in rng.permutation(len(lens)):
+        if len(rows) >= k:
+            break
+        rows.add(int(i))
+    return sorted(rows)
+
+
+def parity_check(idx, dev, budget_s, min_rows=8, all_rows_ok=True):
+    """The GPU result on the workload's seeded inputs (drawn on the CPU, as the
+    tests draw them) against the fp64 oracle on the same inputs.
+
+    Rows: all of them if the oracle's estimated time fits budget_s (and
+    all_rows_ok), else a seeded sample of at least min_rows with the shortest
+    and longest.  Returns (parity entry, oracle seconds per batch row, rows)."""
+    from oracle import mla_oracle
+
+    x = inputs.workload_inputs(idx)
+    lens = [int(v) for v in x.seqlens]
+    g = x.to(dev)
+    meta = binding.mla_get_metadata(g.seqlens, g.h_q, g.s_q)
+    out, lse = binding.mla_decode(g.q, g.kv_cache, g.block_table, g.seqlens, g.softmax_scale, g.causal, meta)
+    torch.cuda.synchronize(dev)
+    err = binding.mla_check_device_error(meta)
+    got_o = out.cpu().double().numpy()
+    got_l = lse.cpu().double().numpy()
+    del g, meta, out, lse
+    # the longest row first: it calibrates the oracle's cost per row
+    longest = max(range(len(lens)), key=lambda i: (lens[i], i))
+    t0 = time.perf_counter()
+    mla_oracle.decode(x.q, x.kv_cache, x.block_table, x.seqlens, x.softmax_scale, x.causal, rows=[longest])
+    t_longest = time.perf_counter() - t0
+    if all_rows_ok and t_longest * x.batch <= budget_s:
+        rows = list(range(x.batch))
+    else:
+        k = max(min_rows, min(x.batch, int(budget_s / max(t_longest, 1e-6))))
+        rows = sample_rows(lens, min(k, x.batch), seed=idx)
+    t0 = time.perf_counter()
+    want_o, want_l = mla_oracle.decode(x.q, x.kv_cache, x.block_table, x.seqlens, x.softmax_scale, x.causal,
+                                       rows=rows)
+    t_oracle = time.perf_counter() - t0
+    go, gl, wo, wl_ = got_o[rows], got_l[rows], want_o[rows], want_l[rows]
+    d = np.abs(go - wo)
+    inf = np.isneginf(wl_)
+    neg_inf_match = bool(np.array_equal(np.isneginf(gl), inf))
+    lse_max = float(np.abs(gl[~inf] - wl_[~inf]).max()) if (~inf).any() else 0.0
+    finite = bool(np.isfinite(go).all())
+    entry = {
+        "max_abs": float(d.max()), "mean_abs": float(d.mean()), "lse_max_abs": lse_max,
+        "neg_inf_match": neg_inf_match, "finite": finite, "device_error_word": int(err),
+        "rows": len(rows) if len(rows) == x.batch else rows, "of_rows": x.batch,
+        "elements": int(d.size),
+        "tolerance": {"max_abs": TOL_MAX, "mean_abs": TOL_MEAN, "lse_max_abs": TOL_LSE},
+        "pass": bool(d.max() <= TOL_MAX and d.mean() <= TOL_MEAN and lse_max <= TOL_LSE and neg_inf_match
+                     and finite and err == 0),
+        "inputs": "the workload's seeded inputs (seed 1000 + index, drawn on the CPU), one mla_decode call",
+    }
+    return entry, t_oracle / len(rows), rows
 
 
 # ----------------------------------------------------------------------------
 # our arm
 # ----------------------------------------------------------------------------
 
-def ours(args, world, rank, local):
-    dev = torch.device("cuda", local)
-    torch.cuda.set_device(dev)
-    idx = args.workload
-    wl = inputs.WORKLOADS[idx]
-    gen = torch.Generator()
-    gen.manual_seed(1000 + idx)
-    lens = inputs.draw_lengths(wl.lengths, wl.batch, gen)
-    l2 = torch.cuda.get_device_properties(dev).L2_cache_size
-    one = None
-    pools = []
-    total = 0
-    while len(pools) < 2 or total < 3 * l2:
-        seed = 1000 + idx + 7919 * (len(pools) + 1) + 104729 * rank
-        one = inputs.make_inputs(lens, wl.h_q, wl.s_q, seed=seed, causal=wl.causal, softmax_scale=wl.softmax_scale,
-                                 pool_factor=wl.pool_factor, device=str(dev), name=wl.name)
-        pools.append(one)
-        total += one.kv_cache.numel() * 2 + one.q.numel() * 2
-        if len(pools) >= 64:
-            break
-    npool = len(pools)
-    stream = torch.cuda.Stream(dev)
-    ws_bytes = max(binding.mla_workspace_bytes(wl.batch, wl.h_q, wl.s_q), 16)
-    with torch.cuda.stream(stream):
-        metas = [torch.empty(binding.mla_metadata_bytes(wl.batch, wl.h_q, wl.s_q) // 4, dtype=torch.int32, device=dev)
-                 for _ in range(npool)]
-        ws = torch.empty(ws_bytes, dtype=torch.uint8, device=dev)
-        out = torch.empty(wl.batch, wl.s_q, wl.h_q, 512, dtype=torch.bfloat16, device=dev)
-        lse = torch.empty(wl.batch, wl.h_q, wl.s_q, dtype=torch.float32, device=dev)
-    torch.cuda.synchronize(dev)
+class Bench:
+    """One workload's rotating pools, buffers and step graphs on this GPU."""
 
-    def step(r, events=None):
-        x = pools[r]
-        binding.mla_get_metadata(x.seqlens, x.h_q, x.s_q, metadata=metas[r], stream=stream)
-        binding.mla_decode(x.q, x.kv_cache, x.block_table, x.seqlens, x.softmax_scale, x.causal, metas[r],
-                           workspace=ws, out=out, lse=lse, stream=stream, events=events)
-
-    # warm-up (eager), and a check that no device error was raised
-    for k in range(max(args.warmup, 1)):
-        step(k % npool)
-    stream.synchronize()
-    for m in metas:
-        err = binding.mla_check_device_error(m, stream=stream)
-        if err:
-            raise RuntimeError(f"device error word {err:#x} during warm-up")
-    err = binding.mla_take_device_errors(stream=stream)  # every plan rewrites its metadata word: check the sticky bits
-    if err:
-        raise RuntimeError(f"device error bits {err:#x} during warm-up")
-
-    # CUDA graphs: one cycle over all pools (with events around each split-KV
-    # kernel) and one single-step graph per pool, so that exactly K steps run.
-    ev_pairs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(npool)]
-    for a, b in ev_pairs:
-        a.record(stream)
-        b.record(stream)
-    stream.synchronize()
-    # The timed graphs hold no event nodes between the kernels, so that each
-    # kernel can launch while its predecessor finishes (programmatic dependent
-    # launch); a separate graph with events around each split-KV kernel times
-    # that kernel alone, replayed right after the timed region.
-    cycle = torch.cuda.CUDAGraph()
-    with torch.cuda.graph(cycle, stream=stream):
-        for r in range(npool):
-            step(r)
-    cycle_k2 = torch.cuda.CUDAGraph()
-    with torch.cuda.graph(cycle_k2, stream=stream):
-        for r in range(npool):
-            step(r, events=ev_pairs[r])
-    singles = []
-    for r in range(npool):
-        g = torch.cuda.CUDAGraph()
-        with torch.cuda.graph(g, stream=stream):
-            step(r)
-        singles.append(g)
-    with torch.cuda.stream(stream):
-        for _ in range(2):
-            cycle.replay()
-            cycle_k2.replay()
-    stream.synchronize()
-
-    K = args.steps
-    reps, rem = divmod(K, npool)
-    start = torch.cuda.Event(enable_timing=True)
-    end = torch.cuda.Event(enable_timing=True)
-    barrier(world)
-    torch.cuda.synchronize(dev)
-    with ClockSampler(local) as clocks:
+    def __init__(self, idx, dev, rank, stream):
+        self.idx = idx
+        self.wl = wl = inputs.WORKLOADS[idx]
+        self.dev = dev
+        self.stream = stream
+        self.lens = workload_lengths(idx)
+        self.l2 = torch.cuda.get_device_properties(dev).L2_cache_size
+        pools, total = [], 0
+        while len(pools) < 2 or total < 3 * self.l2:
+            seed = 1000 + idx + 7919 * (len(pools) + 1) + 104729 * rank
+            one = inputs.make_inputs(self.lens, wl.h_q, wl.s_q, seed=seed, causal=wl.causal,
+                                     softmax_scale=wl.softmax_scale, pool_factor=wl.pool_factor, device=str(dev),
+                                     name=wl.name)
+            pools.append(one)
+            total += one.kv_cache.numel() * 2 + one.q.numel() * 2
+            if len(pools) >= 64:
+                break
+        self.pools, self.total = pools, total
+        self.npool = len(pools)
+        ws_bytes = max(binding.mla_workspace_bytes(wl.batch, wl.h_q, wl.s_q), 16)
         with torch.cuda.stream(stream):
-            start.record(stream)
-            for _ in range(reps):
-                cycle.replay()
-            for r in range(rem):
-                singles[r].replay()
-            end.record(stream)
-        stream.synchronize()
-    torch.cuda.synchronize(dev)
-    barrier(world)
-    ms_total = start.elapsed_time(end)
-    ms_total = max_over_ranks(ms_total, world, dev)
-    ms_step = ms_total / K
-    n_cycles = max(1, min(reps, 20))
-    k2_source = ("events around the split-KV kernel, graph replays of the same steps right after the timed "
-                 "region and a 0.3 s idle pause (median of %d launches: %d cycles over the pools)"
-                 % (n_cycles * npool, n_cycles))
-    k2_ms = []
-    # Under sustained load the GPU's power cap lowers the SM clock within a
-    # tenth of a second; each timed phase therefore starts from an idle GPU,
-    # as the timed region did, and its clocks are sampled too.
-    time.sleep(0.3)
-    with ClockSampler(local) as k2_clocks:
-        try:
-            for _ in range(n_cycles):
-                with torch.cuda.stream(stream):
-                    cycle_k2.replay()
-                stream.synchronize()
-                k2_ms += [a.elapsed_time(b) for a, b in ev_pairs]
-        except Exception:
-            k2_ms = []
-        if not k2_ms:
-            # Eager launches with the same events, right after the timed region.
-            k2_source = "events around the split-KV kernel, eager launches after the timed region (median)"
-            for _ in range(n_cycles):
-                for r in range(npool):
-                    step(r, events=ev_pairs[r])
-                stream.synchronize()
-                k2_ms += [a.elapsed_time(b) for a, b in ev_pairs]
-    k2_med_ms = sorted(k2_ms)[len(k2_ms) // 2]
+            self.metas = [torch.empty(binding.mla_metadata_bytes(wl.batch, wl.h_q, wl.s_q) // 4, dtype=torch.int32,
+                                      device=dev) for _ in range(self.npool)]
+            self.ws = torch.empty(ws_bytes, dtype=torch.uint8, device=dev)
+            self.out = torch.empty(wl.batch, wl.s_q, wl.h_q, 512, dtype=torch.bfloat16, device=dev)
+            self.lse = torch.empty(wl.batch, wl.h_q, wl.s_q, dtype=torch.float32, device=dev)
+        torch.cuda.synchronize(dev)
 
-    # Per layer: the plan is made once per decode step and reused by every
-    # layer, so a step of a model is one plan and then one decode call (split
-    # KV + combine) per layer.  One graph: a plan on the shared lengths, then
-    # a decode call over each pool in turn (a pool stands for a layer's
-    # cache; all pools share the lengths), timed whole and divided by the
-    # calls.
-    n_layers = max(8, npool)
-    layer_graph = torch.cuda.CUDAGraph()
-    with torch.cuda.graph(layer_graph, stream=stream):
-        x0p = pools[0]
-        binding.mla_get_metadata(x0p.seqlens, x0p.h_q, x0p.s_q, metadata=metas[0], stream=stream)
+    def step(self, r, events=None):
+        x = self.pools[r]
+        binding.mla_get_metadata(x.seqlens, x.h_q, x.s_q, metadata=self.metas[r], stream=self.stream)
+        binding.mla_decode(x.q, x.kv_cache, x.block_table, x.seqlens, x.softmax_scale, x.causal, self.metas[r],
+                           workspace=self.ws, out=self.out, lse=self.lse, stream=self.stream, events=events)
+
+    def warm_up(self, n):
+        for k in range(max(n, 1)):
+            self.step(k % self.npool)
+        self.stream.synchronize()
+        for m in self.metas:
+            err = binding.mla_check_device_error(m, stream=self.stream)
+            if err:
+                raise RuntimeError(f"device error word {err:#x} during warm-up ({self.wl.name})")
+        err = binding.mla_take_device_errors(stream=self.stream)  # each plan rewrites its own word: the sticky bits
+        if err:
+            raise RuntimeError(f"device error bits {err:#x} during warm-up ({self.wl.name})")
+
+    def capture(self):
+        """One graph cycling over the pools, the same with events around each
+        split-KV kernel, and one single-step graph per pool (so that exactly K
+        steps can run)."""
+        s = self.stream
+        self.ev_pairs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+                         for _ in range(self.npool)]
+        for a, b in self.ev_pairs:
+            a.record(s)
+            b.record(s)
+        s.synchronize()
+        # The timed graphs hold no event nodes between the kernels, so that each
+        # kernel can launch while its predecessor finishes (programmatic
+        # dependent launch); the graph with events times the split-KV kernel.
+        self.cycle = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(self.cycle, stream=s):
+            for r in range(self.npool):
+                self.step(r)
+        self.cycle_k2 = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(self.cycle_k2, stream=s):
+            for r in range(self.npool):
+                self.step(r, events=self.ev_pairs[r])
+        self.singles = []
+        for r in range(self.npool):
+            g = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(g, stream=s):
+                self.step(r)
+            self.singles.append(g)
+        with torch.cuda.stream(s):
+            for _ in range(2):
+                self.cycle.replay()
+                self.cycle_k2.replay()
+        s.synchronize()
+
+    def timed_steps(self, K, world, local):
+        """Exactly K steps, bracketed by a barrier and a device sync; max over ranks."""
+        reps, rem = divmod(K, self.npool)
+        start = torch.cuda.Event(enable_timing=True)
+        end = torch.cuda.Event(enable_timing=True)
+        s = self.stream
+        barrier(world)
+        torch.cuda.synchronize(self.dev)
+        with ClockSampler(local) as clocks:
+            with torch.cuda.stream(s):
+                start.record(s)
+                for _ in range(reps):
+                    self.cycle.replay()
+                for r in range(rem):
+                    self.singles[r].replay()
+                end.record(s)
+            s.synchronize()
+        torch.cuda.synchronize(self.dev)
+        barrier(world)
+        ms_total = max_over_ranks(start.elapsed_time(end), world, self.dev)
+        return ms_total / K, clocks.summary()
+
+    def decode_kernel_timing(self, K, local):
+        """The split-KV kernel alone: events around it in graph replays of the
+        same steps, started from an idle GPU (the power cap lowers the SM clock
+        within a tenth of a second of sustained load), median of the launches."""
+        n_cycles = max(1, min(max(K // self.npool, 1), 20))
+        source = ("events around the split-KV kernel, graph replays of the same steps after a 0.3 s idle pause "
+                  "(median of %d launches: %d cycles over the pools)" % (n_cycles * self.npool, n_cycles))
+        k2_ms = []
+        time.sleep(0.3)
+        with ClockSampler(local) as clk:
+            for _ in range(n_cycles):
+                with torch.cuda.stream(self.stream):
+                    self.cycle_k2.replay()
+                self.stream.synchronize()
+                k2_ms += [a.elapsed_time(b) for a, b in self.ev_pairs]
+        return sorted(k2_ms)[len(k2_ms) // 2], source, clk.summary()
+
+    def release(self):
+        for name in ("cycle", "cycle_k2", "singles", "pools", "metas", "ws", "out", "lse"):
+            if hasattr(self, name):
+                delattr(self, name)
+        torch.cuda.synchronize(self.dev)
+        torch.cuda.empty_cache()
+
+
+def per_layer_timing(B, K, world):
+    """The plan is made once per decode step and reused by every layer: one
+    graph of a plan on the shared lengths, then a decode call over each pool in
+    turn (a pool stands for a layer's cache; all pools share the lengths),
+    timed whole and divided by the calls."""
+    n_layers = max(8, B.npool)
+    s = B.stream
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g, stream=s):
+        x0 = B.pools[0]
+        binding.mla_get_metadata(x0.seqlens, x0.h_q, x0.s_q, metadata=B.metas[0], stream=s)
         for layer in range(n_layers):
-            x = pools[layer % npool]
-            binding.mla_decode(x.q, x.kv_cache, x.block_table, x.seqlens, x.softmax_scale, x.causal, metas[0],
-                               workspace=ws, out=out, lse=lse, stream=stream)
+            x = B.pools[layer % B.npool]
+            binding.mla_decode(x.q, x.kv_cache, x.block_table, x.seqlens, x.softmax_scale, x.causal, B.metas[0],
+                               workspace=B.ws, out=B.out, lse=B.lse, stream=s)
     l0 = torch.cuda.Event(enable_timing=True)
     l1 = torch.cuda.Event(enable_timing=True)
     time.sleep(0.3)
-    with torch.cuda.stream(stream):
-        layer_graph.replay()
-        l0.record(stream)
+    with torch.cuda.stream(s):
+        g.replay()
+        l0.record(s)
         n_rep = max(1, min(20, K // n_layers))
         for _ in range(n_rep):
-            layer_graph.replay()
-        l1.record(stream)
-    stream.synchronize()
-    layer_us = max_over_ranks(l0.elapsed_time(l1) * 1e3 / (n_rep * n_layers), world, dev)
-    del layer_graph
-    proj = projection_timing(wl, pools, metas[0], ws, out, lse, stream, dev, l2, world, local, n_layers)
-    split = long_row_timing(wl, pools, stream, dev, world, local)
-    # The sticky bits cover every step since warm-up (each plan rewrites the
-    # word in its own metadata, so those only show the last cycle).
-    err = binding.mla_take_device_errors(stream=stream)
-    if err:
-        raise RuntimeError(f"device error bits {err:#x} in the timed region or the kernel timing replays")
+            g.replay()
+        l1.record(s)
+    s.synchronize()
+    us = max_over_ranks(l0.elapsed_time(l1) * 1e3 / (n_rep * n_layers), world, B.dev)
+    del g
+    return {"value": round(us, 3), "unit": "us/call",
+            "note": (f"one plan, then {n_layers} decode calls (split-KV + combine) on it over the rotating pools, "
+                     f"graph-replayed {n_rep} times; the plan's cost spread over the calls")}
 
-    # End to end through the API: every step copies its inputs in from pinned
-    # host memory and its result (out, lse) back, as a serving loop would:
-    # copies run on their own streams, double-buffered, so that step n + 1's
-    # inputs go in and step n - 1's result comes out while step n computes.
-    e2e_steps = min(K, 500)
-    x0 = pools[0]
+
+def e2e_timing(B, K, world):
+    """End to end through the public API: every step copies its inputs (q,
+    block table, lengths) in from pinned host memory and its result (out, lse)
+    back, as a serving loop would, rotating over the pools (each pool's inputs
+    have a pinned host copy of their own).  Copies run on two copy streams,
+    double-buffered, so that step n + 1's inputs go in and step n - 1's result
+    comes out while step n computes."""
+    dev, stream = B.dev, B.stream
+    steps = max(200, min(K, 2000))
 
     def layout(tensors):
-        """Byte offsets of the tensors packed back to back, each 16-byte aligned."""
         offs, n = [], 0
         for t in tensors:
             offs.append(n)
@@ -520,70 +596,138 @@ def ours(args, world, rank, local):
     def views(buf, offs, like):
         return [buf[o:o + t.numel() * t.element_size()].view(t.dtype).view(t.shape) for o, t in zip(offs, like)]
 
-    # One pinned buffer per direction: q, block table and lengths go in with
-    # one copy, out and lse come back with one copy (the device tensors the
-    # API calls take are views into the matching device buffers).
-    ins = [x0.q, x0.block_table, x0.seqlens]
-    in_offs, in_bytes = layout(ins)
-    h_in = torch.empty(in_bytes, dtype=torch.uint8).pin_memory()
-    for v, t in zip(views(h_in, in_offs, ins), ins):
-        v.copy_(t.cpu())
-    res_like = [out, lse]
+    like_in = [B.pools[0].q, B.pools[0].block_table, B.pools[0].seqlens]
+    in_offs, in_bytes = layout(like_in)
+    h_in = []
+    for x in B.pools:
+        h = torch.empty(in_bytes, dtype=torch.uint8).pin_memory()
+        for v, t in zip(views(h, in_offs, like_in), (x.q, x.block_table, x.seqlens)):
+            v.copy_(t.cpu())
+        h_in.append(h)
+    res_like = [B.out, B.lse]
     res_offs, res_bytes = layout(res_like)
     h_res = [torch.empty(res_bytes, dtype=torch.uint8).pin_memory() for _ in range(2)]
     d_in = [torch.empty(in_bytes, dtype=torch.uint8, device=dev) for _ in range(2)]
     d_res = [torch.empty(res_bytes, dtype=torch.uint8, device=dev) for _ in range(2)]
-    d_q, d_table, d_lens = zip(*[views(d, in_offs, ins) for d in d_in])
+    d_q, d_table, d_lens = zip(*[views(d, in_offs, like_in) for d in d_in])
     d_out, d_lse = zip(*[views(d, res_offs, res_like) for d in d_res])
     s_in = torch.cuda.Stream(device=dev)
     s_out = torch.cuda.Stream(device=dev)
-    ev = lambda: torch.cuda.Event()
-    in_done = [ev(), ev()]
-    comp_done = [ev(), ev()]
-    out_done = [ev(), ev()]
+    in_done = [torch.cuda.Event(), torch.cuda.Event()]
+    comp_done = [torch.cuda.Event(), torch.cuda.Event()]
+    out_done = [torch.cuda.Event(), torch.cuda.Event()]
     e0 = torch.cuda.Event(enable_timing=True)
     e1 = torch.cuda.Event(enable_timing=True)
-    barrier(world)
-    torch.cuda.synchronize(dev)
-    time.sleep(0.3)  # start from an idle GPU, as the other timed phases do
-    e0.record(s_in)
-    for n in range(e2e_steps):
-        b = n & 1
+    wl = B.wl
+
+    def run(n):
+        b, r = n & 1, n % B.npool
         with torch.cuda.stream(s_in):
             if n >= 2:
                 s_in.wait_event(comp_done[b])  # step n - 2 no longer reads these inputs
-            d_in[b].copy_(h_in, non_blocking=True)
+            d_in[b].copy_(h_in[r], non_blocking=True)
             in_done[b].record(s_in)
         stream.wait_event(in_done[b])
         if n >= 2:
             stream.wait_event(out_done[b])  # step n - 2's result has left this buffer
-        binding.mla_get_metadata(d_lens[b], x0.h_q, x0.s_q, metadata=metas[b], stream=stream)
-        binding.mla_decode(d_q[b], x0.kv_cache, d_table[b], d_lens[b], x0.softmax_scale, x0.causal, metas[b],
-                           workspace=ws, out=d_out[b], lse=d_lse[b], stream=stream)
+        binding.mla_get_metadata(d_lens[b], wl.h_q, wl.s_q, metadata=B.metas[b % B.npool], stream=stream)
+        binding.mla_decode(d_q[b], B.pools[r].kv_cache, d_table[b], d_lens[b], wl.softmax_scale, wl.causal,
+                           B.metas[b % B.npool], workspace=B.ws, out=d_out[b], lse=d_lse[b], stream=stream)
         comp_done[b].record(stream)
         with torch.cuda.stream(s_out):
             s_out.wait_event(comp_done[b])
             h_res[b].copy_(d_res[b], non_blocking=True)
             out_done[b].record(s_out)
-    s_out.wait_event(comp_done[(e2e_steps - 1) & 1])
+
+    for n in range(4):  # untimed: first calls of the copy streams and of the API on these buffers
+        run(n)
+    torch.cuda.synchronize(dev)
+    barrier(world)
+    time.sleep(0.3)  # start from an idle GPU, as the other timed phases do
+    e0.record(s_in)
+    for n in range(steps):
+        run(n)
+    s_out.wait_event(comp_done[(steps - 1) & 1])
     e1.record(s_out)
     torch.cuda.synchronize(dev)
     err = binding.mla_take_device_errors(stream=stream)
     if err:
         raise RuntimeError(f"device error bits {err:#x} in the end-to-end steps")
-    # the last step's result, as it came back, against a call on the device-resident inputs
-    binding.mla_decode(x0.q, x0.kv_cache, x0.block_table, x0.seqlens, x0.softmax_scale, x0.causal, metas[0],
-                       workspace=ws, out=out, lse=lse, stream=stream)
+    # the last step's result, as it came back, against a call on that pool's device-resident inputs
+    last = steps - 1
+    x = B.pools[last % B.npool]
+    binding.mla_get_metadata(x.seqlens, x.h_q, x.s_q, metadata=B.metas[0], stream=stream)
+    binding.mla_decode(x.q, x.kv_cache, x.block_table, x.seqlens, x.softmax_scale, x.causal, B.metas[0],
+                       workspace=B.ws, out=B.out, lse=B.lse, stream=stream)
     stream.synchronize()
-    last = views(h_res[(e2e_steps - 1) & 1], res_offs, res_like)
-    e2e_same = bool(torch.equal(last[0], out.cpu()) and torch.equal(last[1], lse.cpu()))
-    e2e_ms = max_over_ranks(e0.elapsed_time(e1) / e2e_steps, world, dev)
-    h2d = in_bytes
-    d2h = res_bytes
+    got = views(h_res[last & 1], res_offs, res_like)
+    same = bool(torch.equal(got[0], B.out.cpu()) and torch.equal(got[1], B.lse.cpu()))
+    ms = max_over_ranks(e0.elapsed_time(e1) / steps, world, dev)
+    return {"value": round(ms * 1e3 / world, 3), "unit": "us/call", "h2d_bytes_per_step": in_bytes,
+            "d2h_bytes_per_step": res_bytes, "steps": steps,
+            "pcie_gbs_each_way": round(max(in_bytes, res_bytes) / (ms * 1e-3) / 1e9, 1),
+            "last_result_equals_device_call": same,
+            "note": ("pinned q/block_table/seqlens in (one packed copy per step, from the step's pool), out/lse "
+                     "back (one packed copy), every step, on copy streams of their own, double-buffered so that "
+                     "copies overlap the neighbouring steps' compute; calls rotate over the cache pools, which stay "
+                     "resident in HBM (the model state a decode step appends to)")}
 
-    nbytes, flops = algorithmic_work(lens, wl.h_q, wl.s_q, wl.causal)
-    hbm_peak, tf_peak, tf_sustained, peak_kind = measured_peaks()
-    k2_s = k2_med_ms * 1e-3
+
+def roofline_for(B, k2_ms, k2_source, peaks):
+    hbm_peak, tf_peak, _, peak_kind = peaks
+    nbytes, flops = algorithmic_work(B.lens, B.wl.h_q, B.wl.s_q, B.wl.causal)
+    return roofline_entry(nbytes, flops, k2_ms * 1e-3, hbm_peak, tf_peak, peak_kind, committed_traffic(B.wl.name),
+                          k2_source), nbytes, flops
+
+
+def other_workload(idx, args, world, rank, local, dev, stream, peaks):
+    """Another workload's step time, decode-kernel roofline and parity sample."""
+    B = Bench(idx, dev, rank, stream)
+    B.warm_up(args.warmup)
+    B.capture()
+    K = max(B.npool, min(args.steps, 200))
+    ms_step, clocks = B.timed_steps(K, world, local)
+    k2_ms, k2_source, k2_clocks = B.decode_kernel_timing(K, local)
+    roof, _, _ = roofline_for(B, k2_ms, k2_source, peaks)
+    entry = {"config": workload_config(B.wl, idx, B.lens), "step_us": round(ms_step * 1e3 / world, 3),
+             "steps": K, "decode_kernel_us": round(k2_ms * 1e3, 3), "roofline": roof,
+             "decode_kernel_clocks": k2_clocks, "clocks": clocks}
+    B.release()
+    if world == 1 and not args.no_cpu_baseline:
+        entry["parity"], _, _ = parity_check(idx, dev, budget_s=3.0, min_rows=8, all_rows_ok=False)
+    return entry
+
+
+def ours(args, world, rank, local):
+    dev = torch.device("cuda", local)
+    torch.cuda.set_device(dev)
+    idx = args.workload
+    stream = torch.cuda.Stream(dev)
+    peaks = measured_peaks()
+    K = args.steps
+
+    B = Bench(idx, dev, rank, stream)
+    wl = B.wl
+    B.warm_up(args.warmup)
+    B.capture()
+    ms_step, clocks = B.timed_steps(K, world, local)
+    k2_ms, k2_source, k2_clocks = B.decode_kernel_timing(K, local)
+    layer = per_layer_timing(B, K, world)
+    proj = split = None
+    if not args.headline_only:
+        proj = projection_timing(wl, B.pools, B.metas[0], B.ws, B.out, B.lse, stream, dev, B.l2, world, local,
+                                 max(8, B.npool))
+        split = long_row_timing(wl, B.pools, stream, dev, world, local)
+    # The sticky bits cover every call since warm-up (each plan rewrites the
+    # word in its own metadata, so those only show the last cycle).
+    err = binding.mla_take_device_errors(stream=stream)
+    if err:
+        raise RuntimeError(f"device error bits {err:#x} in the timed region or the kernel timing replays")
+    e2e = e2e_timing(B, K, world)
+    roof, nbytes, flops = roofline_for(B, k2_ms, k2_source, peaks)
+    npool, total, l2 = B.npool, B.total, B.l2
+    B.release()
+
     line = {
         "metric": METRIC,
         # Whole job: the calls all ranks made over the time they took (each
@@ -599,33 +743,41 @@ def ours(args, world, rank, local):
         "vs_baseline": None,
         "dtype": "bf16",
         "data": "synthetic",
-        "config": workload_config(wl, idx, lens, f"{npool} rotating pools, {total / 2**20:.0f} MiB > 3x "
-                                                 f"{l2 / 2**20:.0f} MiB L2; timed via CUDA graph replay"),
+        "config": workload_config(wl, idx, B.lens),
+        "pools": f"{npool} rotating pools, {total / 2**20:.0f} MiB > 3x {l2 / 2**20:.0f} MiB L2; timed via CUDA "
+                 f"graph replay",
         "achieved_gbs": round(world * nbytes / (ms_step * 1e-3) / 1e9, 1),
         "achieved_tflops": round(world * flops / (ms_step * 1e-3) / 1e12, 2),
         "calls_per_s_all_ranks": round(world / (ms_step * 1e-3), 1),
-        "decode_kernel_us": round(k2_med_ms * 1e3, 3),
-        "roofline": roofline_entry(nbytes, flops, k2_s, hbm_peak, tf_peak, peak_kind, committed_traffic(wl.name),
-                                   k2_source),
-        "decode_kernel_clocks": k2_clocks.summary(),
-        "e2e": {"value": round(e2e_ms * 1e3 / world, 3), "unit": "us/call", "h2d_bytes_per_step": h2d,
-                "d2h_bytes_per_step": d2h, "steps": e2e_steps,
-                "last_result_equals_device_call": e2e_same,
-                "note": ("pinned q/block_table/seqlens in (one packed copy), out/lse back (one packed copy), "
-                         "every step, on copy streams of their own, double-buffered so that copies overlap the "
-                         "neighbouring steps' compute; cache resident in HBM")},
-        "per_layer": {"value": round(layer_us, 3), "unit": "us/call",
-                      "note": (f"one plan, then {n_layers} decode calls (split-KV + combine) on it over the rotating "
-                               f"pools, graph-replayed {n_rep} times; the plan's cost spread over the calls")},
-        "projections": proj,
-        "long_row_split": split,
+        "decode_kernel_us": round(k2_ms * 1e3, 3),
+        "roofline": roof,
+        "decode_kernel_clocks": k2_clocks,
+        "e2e": e2e,
+        "per_layer": layer,
         "gpu_launches": 3 * K,
-        "clocks": clocks.summary(),
+        "clocks": clocks,
     }
+    if proj is not None:
+        line["projections"] = proj
+        line["long_row_split"] = split
     if world == 1 and rank == 0 and not args.no_cpu_baseline:
-        line["cpu_baseline"] = cpu_baseline(idx, budget_s=10.0)
-        line["projections"]["cpu_baseline"] = oracle_projection_and_merge(wl)
-    del cycle, singles
+        par, t_row, rows = parity_check(idx, dev, budget_s=25.0)
+        line["parity"] = par
+        line["cpu_baseline"] = {
+            "value": round(t_row * wl.batch * 1e6, 1), "unit": "us/call", "cores": cpu_threads(), "kind": "oracle",
+            "sample": (f"the parity check's oracle run (fp64 NumPy) over {len(rows)} of {wl.batch} batch rows of the "
+                       f"same workload, scaled to all {wl.batch} rows")}
+        if proj is not None:
+            line["projections"]["cpu_baseline"] = oracle_projection_and_merge(wl)
+    if not args.headline_only:
+        others = {}
+        for j in range(len(inputs.WORKLOADS)):
+            if j != idx:
+                others[inputs.WORKLOADS[j].name] = other_workload(j, args, world, rank, local, dev, stream, peaks)
+        mb = inputs.WORKLOADS[2].name
+        if mb in others:
+            line["memory_bound"] = others.pop(mb)
+        line["other_workloads"] = others
     if rank == 0:
         print(json.dumps(line), flush=True)
 
@@ -852,8 +1004,11 @@ def main():
     ap.add_argument("--steps", type=int, default=3000)
     ap.add_argument("--warmup", type=int, default=10)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
-    ap.add_argument("--workload", type=int, default=1, help="index into inputs.WORKLOADS (1 = headline)")
-    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--workload", type=int, default=DEFAULT_WORKLOAD,
+                    help=f"index into inputs.WORKLOADS ({DEFAULT_WORKLOAD} = headline)")
+    ap.add_argument("--no-cpu-baseline", action="store_true", help="run no oracle (no parity, no CPU baseline)")
+    ap.add_argument("--headline-only", action="store_true",
+                    help="time only the headline workload's step (no projections, split or other workloads)")
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3

@@ -47,6 +47,12 @@
  *   - No exception or C++ type crosses the ABI.  The functions are
  *     thread-compatible: concurrent calls must use distinct metadata and
  *     workspace buffers.
+ *   - Per device, the library caches the kernels' launch geometry (looked up
+ *     on the first call there) and the device address of its fixed scratch
+ *     array (mla_decode_noalloc); per host thread, the TMA descriptors of
+ *     recently used (pointer, size) pairs.  None of these survive a device
+ *     reset (cudaDeviceReset) or the destruction of the device's primary
+ *     context: the library must not be used on a device after either.
  */
 #ifndef MLA_B200_H
 #define MLA_B200_H
@@ -145,6 +151,22 @@ int mla_decode(const void* q, const void* kv_cache, int64_t num_pages, const int
                int max_pages_per_seq, const int32_t* seqlens, int batch, int s_q, int h_q, float softmax_scale,
                int causal, void* out, float* lse, void* metadata, void* workspace, size_t workspace_bytes,
                void* stream);
+
+/*
+ * mla_decode with an fp32 output: the same attention, with out written as
+ * fp32 [batch][s_q][h_q][512] (16-byte aligned) instead of bf16, unrounded.
+ * For results that are merged again before they are rounded: the split of
+ * one long row across GPUs ("Unlocking GPU Potential: The Impact of
+ * FlashAttention and KV Cache Optimization in Long-Text Inference": each
+ * chunk of the keys is attended to separately, and the partial results are
+ * rescaled by their log-sum-exp), whose per-GPU results go to
+ * mla_merge_splits_f32.  Every other argument, the limits and the errors are
+ * those of mla_decode.
+ */
+int mla_decode_f32(const void* q, const void* kv_cache, int64_t num_pages, const int32_t* block_table,
+                   int max_pages_per_seq, const int32_t* seqlens, int batch, int s_q, int h_q, float softmax_scale,
+                   int causal, float* out, float* lse, void* metadata, void* workspace, size_t workspace_bytes,
+                   void* stream);
 
 /*
  * mla_decode, plus CUDA events recorded on `stream` immediately before and
@@ -270,6 +292,15 @@ int mla_up_project(const void* o_latent, const void* w_uv, int tokens, int h_q, 
  */
 int mla_merge_splits(const void* outs, const float* lses, int splits, int batch, int s_q, int h_q, void* out,
                      float* lse, void* stream);
+
+/*
+ * mla_merge_splits over fp32 partial outputs (mla_decode_f32's `out`): outs
+ * is fp32 [splits][batch][s_q][h_q][512], 16-byte aligned; the result `out` is
+ * bf16 as for mla_merge_splits, rounded once after the merge.  Arguments,
+ * limits and errors as for mla_merge_splits.
+ */
+int mla_merge_splits_f32(const float* outs, const float* lses, int splits, int batch, int s_q, int h_q, void* out,
+                         float* lse, void* stream);
 
 /*
  * Synchronise `stream` and read the device error word from `metadata`.

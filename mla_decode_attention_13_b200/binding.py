@@ -35,11 +35,13 @@ EXPORTED = (
     "mla_num_sm_pairs",
     "mla_get_metadata",
     "mla_decode",
+    "mla_decode_f32",
     "mla_decode_timed",
     "mla_decode_noalloc",
     "mla_absorb_q",
     "mla_up_project",
     "mla_merge_splits",
+    "mla_merge_splits_f32",
     "mla_selftest_bounded_wait",
     "mla_check_device_error",
     "mla_take_device_errors",
@@ -76,6 +78,8 @@ def lib() -> ctypes.CDLL:
                ctypes.c_float, ctypes.c_int, _vp, _vp, _vp, _vp, ctypes.c_size_t, _vp]
         L.mla_decode.restype = ctypes.c_int
         L.mla_decode.argtypes = dec
+        L.mla_decode_f32.restype = ctypes.c_int
+        L.mla_decode_f32.argtypes = dec
         L.mla_decode_timed.restype = ctypes.c_int
         L.mla_decode_timed.argtypes = dec + [_vp, _vp]
         L.mla_decode_noalloc.restype = ctypes.c_int
@@ -86,6 +90,8 @@ def lib() -> ctypes.CDLL:
         L.mla_up_project.argtypes = [_vp, _vp, ctypes.c_int, ctypes.c_int, _vp, _vp]
         L.mla_merge_splits.restype = ctypes.c_int
         L.mla_merge_splits.argtypes = [_vp, _vp] + [ctypes.c_int] * 4 + [_vp, _vp, _vp]
+        L.mla_merge_splits_f32.restype = ctypes.c_int
+        L.mla_merge_splits_f32.argtypes = [_vp, _vp] + [ctypes.c_int] * 4 + [_vp, _vp, _vp]
         L.mla_selftest_bounded_wait.restype = ctypes.c_int
         L.mla_selftest_bounded_wait.argtypes = [_vp]
         L.mla_check_device_error.restype = ctypes.c_int
@@ -180,6 +186,35 @@ def mla_decode(q: torch.Tensor, kv_cache: torch.Tensor, block_table: torch.Tenso
             ev.append(None if e is None else int(e.cuda_event))
         status = lib().mla_decode_timed(*args, *ev)
     _check("mla_decode", status)
+    return out, lse
+
+
+def mla_decode_f32(q: torch.Tensor, kv_cache: torch.Tensor, block_table: torch.Tensor, seqlens: torch.Tensor,
+                   softmax_scale: float, causal: bool, metadata: torch.Tensor, workspace: Optional[torch.Tensor] = None,
+                   out: Optional[torch.Tensor] = None, lse: Optional[torch.Tensor] = None,
+                   stream=None) -> Tuple[torch.Tensor, torch.Tensor]:
+    """mla_decode with an fp32 output: returns (out [b, s_q, h_q, 512] fp32,
+    lse [b, h_q, s_q] fp32), for results that are merged again before they are
+    rounded (mla_merge_splits_f32)."""
+    batch, s_q, h_q, d = q.shape
+    if d != 576 or kv_cache.shape[-1] != 576 or q.dtype != torch.bfloat16 or kv_cache.dtype != torch.bfloat16:
+        raise MLAError("mla_decode_f32", MLA_ERR_ARG)
+    for t in (q, kv_cache, block_table, seqlens):
+        if not t.is_contiguous():
+            raise MLAError("mla_decode_f32", MLA_ERR_ARG)
+    if out is None:
+        out = torch.empty(batch, s_q, h_q, 512, dtype=torch.float32, device=q.device)
+    elif tuple(out.shape) != (batch, s_q, h_q, 512) or out.dtype != torch.float32 or not out.is_contiguous():
+        raise MLAError("mla_decode_f32", MLA_ERR_ARG)
+    if lse is None:
+        lse = torch.empty(batch, h_q, s_q, dtype=torch.float32, device=q.device)
+    if workspace is None:
+        workspace = torch.empty(max(mla_workspace_bytes(batch, h_q, s_q), 16), dtype=torch.uint8, device=q.device)
+    _check("mla_decode_f32",
+           lib().mla_decode_f32(_ptr(q), _ptr(kv_cache), int(kv_cache.shape[0]), _ptr(block_table),
+                                int(block_table.shape[1]), _ptr(seqlens), batch, s_q, h_q, float(softmax_scale),
+                                int(bool(causal)), _ptr(out), _ptr(lse), _ptr(metadata), _ptr(workspace),
+                                int(workspace.numel() * workspace.element_size()), _stream_ptr(stream)))
     return out, lse
 
 
@@ -283,6 +318,24 @@ def mla_merge_splits(outs: torch.Tensor, lses: torch.Tensor, out: Optional[torch
         lse = torch.empty(batch, h_q, s_q, dtype=torch.float32, device=outs.device)
     _check("mla_merge_splits", lib().mla_merge_splits(_ptr(outs), _ptr(lses), splits, batch, s_q, h_q, _ptr(out),
                                                       _ptr(lse), _stream_ptr(stream)))
+    return out, lse
+
+
+def mla_merge_splits_f32(outs: torch.Tensor, lses: torch.Tensor, out: Optional[torch.Tensor] = None,
+                         lse: Optional[torch.Tensor] = None, stream=None) -> Tuple[torch.Tensor, torch.Tensor]:
+    """mla_merge_splits over fp32 partial outputs (mla_decode_f32's out):
+    outs [splits, batch, s_q, h_q, 512] fp32; returns (out bf16, lse fp32)."""
+    if outs.dim() != 5 or outs.shape[-1] != 512 or outs.dtype != torch.float32 or not outs.is_contiguous():
+        raise MLAError("mla_merge_splits_f32", MLA_ERR_ARG)
+    splits, batch, s_q, h_q, _ = outs.shape
+    if tuple(lses.shape) != (splits, batch, h_q, s_q) or lses.dtype != torch.float32 or not lses.is_contiguous():
+        raise MLAError("mla_merge_splits_f32", MLA_ERR_ARG)
+    if out is None:
+        out = torch.empty(batch, s_q, h_q, 512, dtype=torch.bfloat16, device=outs.device)
+    if lse is None:
+        lse = torch.empty(batch, h_q, s_q, dtype=torch.float32, device=outs.device)
+    _check("mla_merge_splits_f32", lib().mla_merge_splits_f32(_ptr(outs), _ptr(lses), splits, batch, s_q, h_q,
+                                                              _ptr(out), _ptr(lse), _stream_ptr(stream)))
     return out, lse
 
 

@@ -2,6 +2,7 @@
 // TMA tensor-map encoding, per-device launch geometry, and the launches.
 #include <cudaTypedefs.h>
 
+#include <atomic>
 #include <cmath>
 #include <mutex>
 
@@ -17,12 +18,16 @@ constexpr int kMaxDevices = 64;
 struct DeviceInfo {
   int pairs = 0;  // co-resident 2-CTA clusters of the decode kernel
   int sms = 0;
-  bool ready = false;
 };
 
+// Per-device launch geometry, looked up on the first call on a device (under
+// g_mu) and read without the lock afterwards: g_dev_ready is published with
+// release order after the fields are written.  The library assumes the
+// device keeps its context for as long as the library is loaded.
 std::mutex g_mu;
 DeviceInfo g_dev[kMaxDevices];
-PFN_cuTensorMapEncodeTiled_v12000 g_encode = nullptr;
+std::atomic<bool> g_dev_ready[kMaxDevices];
+std::atomic<PFN_cuTensorMapEncodeTiled_v12000> g_encode{nullptr};
 
 int current_device_info(DeviceInfo* out) {
   int dev = 0;
@@ -31,9 +36,13 @@ int current_device_info(DeviceInfo* out) {
     return MLA_ERR_CUDA;
   }
   if (dev < 0 || dev >= kMaxDevices) return MLA_ERR_UNSUPPORTED;
+  if (g_dev_ready[dev].load(std::memory_order_acquire)) {
+    *out = g_dev[dev];
+    return MLA_OK;
+  }
   std::lock_guard<std::mutex> lock(g_mu);
   DeviceInfo& d = g_dev[dev];
-  if (!d.ready) {
+  if (!g_dev_ready[dev].load(std::memory_order_relaxed)) {
     int major = 0;
     if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess) return MLA_ERR_CUDA;
     if (major != 10) return MLA_ERR_UNSUPPORTED;  // built for sm_100a only
@@ -43,25 +52,70 @@ int current_device_info(DeviceInfo* out) {
       return MLA_ERR_CUDA;
     }
     if (d.pairs < 1) return MLA_ERR_UNSUPPORTED;
-    d.ready = true;
+    g_dev_ready[dev].store(true, std::memory_order_release);
   }
   *out = d;
   return MLA_OK;
 }
 
 int tensor_map_encoder(PFN_cuTensorMapEncodeTiled_v12000* fn) {
-  std::lock_guard<std::mutex> lock(g_mu);
-  if (!g_encode) {
-    void* ptr = nullptr;
-    cudaDriverEntryPointQueryResult q = cudaDriverEntryPointSymbolNotFound;
-    const cudaError_t e = cudaGetDriverEntryPointByVersion("cuTensorMapEncodeTiled", &ptr, 12000, cudaEnableDefault, &q);
-    if (e != cudaSuccess || q != cudaDriverEntryPointSuccess || ptr == nullptr) {
-      cudaGetLastError();
-      return MLA_ERR_CUDA;
+  PFN_cuTensorMapEncodeTiled_v12000 f = g_encode.load(std::memory_order_acquire);
+  if (!f) {
+    std::lock_guard<std::mutex> lock(g_mu);
+    f = g_encode.load(std::memory_order_relaxed);
+    if (!f) {
+      void* ptr = nullptr;
+      cudaDriverEntryPointQueryResult q = cudaDriverEntryPointSymbolNotFound;
+      const cudaError_t e =
+          cudaGetDriverEntryPointByVersion("cuTensorMapEncodeTiled", &ptr, 12000, cudaEnableDefault, &q);
+      if (e != cudaSuccess || q != cudaDriverEntryPointSuccess || ptr == nullptr) {
+        cudaGetLastError();
+        return MLA_ERR_CUDA;
+      }
+      f = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(ptr);
+      g_encode.store(f, std::memory_order_release);
     }
-    g_encode = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(ptr);
   }
-  *fn = g_encode;
+  *fn = f;
+  return MLA_OK;
+}
+
+// Recently encoded tensor maps of this host thread, keyed by what they encode
+// (which map, base address, rows).  A serving loop calls the decode with the
+// same cache and a few rotating query buffers, so their maps are encoded once
+// instead of on every call.  A map holds only the address and the layout, so
+// it stays right for any later buffer at the same address and size.
+enum MapKind : int { kMapK = 0, kMapV = 1, kMapQ = 2, kMapKinds = 3 };
+
+struct MapCache {
+  static constexpr int kWays = 8;
+  struct Entry {
+    const void* base = nullptr;
+    uint64_t rows = 0;
+    CUtensorMap map;
+  };
+  Entry e[kMapKinds][kWays];
+  int next[kMapKinds] = {};
+};
+
+thread_local MapCache t_maps;
+
+template <typename EncodeFn>
+int cached_map(int kind, const void* base, uint64_t rows, CUtensorMap* out, EncodeFn&& encode) {
+  MapCache::Entry* ways = t_maps.e[kind];
+  for (int k = 0; k < MapCache::kWays; ++k) {
+    if (ways[k].base == base && ways[k].rows == rows) {
+      *out = ways[k].map;
+      return MLA_OK;
+    }
+  }
+  const int st = encode(out);
+  if (st != MLA_OK) return st;
+  MapCache::Entry& slot = ways[t_maps.next[kind]];
+  t_maps.next[kind] = (t_maps.next[kind] + 1) % MapCache::kWays;
+  slot.base = base;
+  slot.rows = rows;
+  slot.map = *out;
   return MLA_OK;
 }
 
@@ -198,7 +252,7 @@ bool shape_ok(int batch, int h_q, int s_q) {
 int decode_impl(const void* q, const void* kv_cache, int64_t num_pages, const int32_t* block_table,
                 int max_pages_per_seq, const int32_t* seqlens, int batch, int s_q, int h_q, float softmax_scale,
                 int causal, void* out, float* lse, void* metadata, void* workspace, size_t workspace_bytes,
-                void* stream, void* ev_before, void* ev_after) {
+                void* stream, void* ev_before, void* ev_after, int out_f32) {
   if (!q || !kv_cache || !block_table || !seqlens || !out || !lse || !metadata) return MLA_ERR_ARG;
   if (batch < 1 || h_q < 1 || s_q < 1 || max_pages_per_seq < 1 || num_pages < 1) return MLA_ERR_ARG;
   if (causal != 0 && causal != 1) return MLA_ERR_ARG;
@@ -222,9 +276,14 @@ int decode_impl(const void* q, const void* kv_cache, int64_t num_pages, const in
   DecodeParams p;
   const uint64_t kv_rows = static_cast<uint64_t>(num_pages) * kPage;
   const uint64_t q_rows = static_cast<uint64_t>(batch) * R;
-  if ((st = encode_panels576(enc, &p.tm_k, kv_cache, kv_rows, kPage, 1)) != MLA_OK ||
-      (st = encode_value_tiles(enc, &p.tm_v, kv_cache, kv_rows)) != MLA_OK ||
-      (st = encode_panels576(enc, &p.tm_q, q, q_rows, kMTile / 2, kDqk / 64)) != MLA_OK)
+  if ((st = cached_map(kMapK, kv_cache, kv_rows, &p.tm_k,
+                       [&](CUtensorMap* m) { return encode_panels576(enc, m, kv_cache, kv_rows, kPage, 1); })) !=
+          MLA_OK ||
+      (st = cached_map(kMapV, kv_cache, kv_rows, &p.tm_v,
+                       [&](CUtensorMap* m) { return encode_value_tiles(enc, m, kv_cache, kv_rows); })) != MLA_OK ||
+      (st = cached_map(kMapQ, q, q_rows, &p.tm_q,
+                       [&](CUtensorMap* m) { return encode_panels576(enc, m, q, q_rows, kMTile / 2, kDqk / 64); })) !=
+          MLA_OK)
     return st;
   p.block_table = block_table;
   p.seqlens = seqlens;
@@ -243,6 +302,7 @@ int decode_impl(const void* q, const void* kv_cache, int64_t num_pages, const in
   p.causal = causal;
   p.tile_rows = tr;
   p.max_slots = slots;
+  p.out_f32 = out_f32;
   p.scale_log2 = softmax_scale * 1.4426950408889634f;
 
   CombineParams cp;
@@ -259,6 +319,7 @@ int decode_impl(const void* q, const void* kv_cache, int64_t num_pages, const in
   cp.pairs = dev.pairs;
   cp.max_slots = slots;
   cp.slices = combine_slices(batch * p.n_mt, tr, dev.sms);
+  cp.out_f32 = out_f32;
 
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   // Inside a stream capture the events must become event-record nodes of the
@@ -320,7 +381,15 @@ MLA_API int mla_decode(const void* q, const void* kv_cache, int64_t num_pages, c
                        int causal, void* out, float* lse, void* metadata, void* workspace, size_t workspace_bytes,
                        void* stream) {
   return decode_impl(q, kv_cache, num_pages, block_table, max_pages_per_seq, seqlens, batch, s_q, h_q, softmax_scale,
-                     causal, out, lse, metadata, workspace, workspace_bytes, stream, nullptr, nullptr);
+                     causal, out, lse, metadata, workspace, workspace_bytes, stream, nullptr, nullptr, 0);
+}
+
+MLA_API int mla_decode_f32(const void* q, const void* kv_cache, int64_t num_pages, const int32_t* block_table,
+                           int max_pages_per_seq, const int32_t* seqlens, int batch, int s_q, int h_q,
+                           float softmax_scale, int causal, float* out, float* lse, void* metadata, void* workspace,
+                           size_t workspace_bytes, void* stream) {
+  return decode_impl(q, kv_cache, num_pages, block_table, max_pages_per_seq, seqlens, batch, s_q, h_q, softmax_scale,
+                     causal, out, lse, metadata, workspace, workspace_bytes, stream, nullptr, nullptr, 1);
 }
 
 MLA_API int mla_decode_timed(const void* q, const void* kv_cache, int64_t num_pages, const int32_t* block_table,
@@ -330,7 +399,7 @@ MLA_API int mla_decode_timed(const void* q, const void* kv_cache, int64_t num_pa
                              void* event_after_decode) {
   return decode_impl(q, kv_cache, num_pages, block_table, max_pages_per_seq, seqlens, batch, s_q, h_q, softmax_scale,
                      causal, out, lse, metadata, workspace, workspace_bytes, stream, event_before_decode,
-                     event_after_decode);
+                     event_after_decode, 0);
 }
 
 MLA_API int mla_decode_noalloc(const void* q, const void* kv_cache, int64_t num_pages, const int32_t* block_table,
@@ -344,7 +413,7 @@ MLA_API int mla_decode_noalloc(const void* q, const void* kv_cache, int64_t num_
   void* scratch = nullptr;
   if ((st = noalloc_scratch(&scratch)) != MLA_OK) return st;
   return decode_impl(q, kv_cache, num_pages, block_table, max_pages_per_seq, seqlens, batch, s_q, h_q, softmax_scale,
-                     causal, out, lse, metadata, scratch, MLA_NOALLOC_SCRATCH_BYTES, stream, nullptr, nullptr);
+                     causal, out, lse, metadata, scratch, MLA_NOALLOC_SCRATCH_BYTES, stream, nullptr, nullptr, 0);
 }
 
 MLA_API int mla_absorb_q(const void* q_nope, const void* q_rope, const void* w_uk, int tokens, int h_q, void* q_out,
@@ -356,8 +425,11 @@ MLA_API int mla_up_project(const void* o_latent, const void* w_uv, int tokens, i
   return projection_impl(o_latent, nullptr, w_uv, tokens, h_q, o_out, false, stream);
 }
 
-MLA_API int mla_merge_splits(const void* outs, const float* lses, int splits, int batch, int s_q, int h_q, void* out,
-                             float* lse, void* stream) {
+namespace mla {
+namespace {
+
+int merge_impl(const void* outs, const float* lses, int splits, int batch, int s_q, int h_q, void* out, float* lse,
+               void* stream, int in_f32) {
   if (!outs || !lses || !out || !lse) return MLA_ERR_ARG;
   if (splits < 1 || batch < 1 || s_q < 1 || h_q < 1) return MLA_ERR_ARG;
   if (!aligned16(outs) || !aligned16(out)) return MLA_ERR_ARG;
@@ -375,11 +447,25 @@ MLA_API int mla_merge_splits(const void* outs, const float* lses, int splits, in
   p.batch = batch;
   p.s_q = s_q;
   p.h_q = h_q;
+  p.in_f32 = in_f32;
   if (launch_merge(p, dev.sms, static_cast<cudaStream_t>(stream)) != cudaSuccess) {
     cudaGetLastError();
     return MLA_ERR_CUDA;
   }
   return MLA_OK;
+}
+
+}  // namespace
+}  // namespace mla
+
+MLA_API int mla_merge_splits(const void* outs, const float* lses, int splits, int batch, int s_q, int h_q, void* out,
+                             float* lse, void* stream) {
+  return merge_impl(outs, lses, splits, batch, s_q, h_q, out, lse, stream, 0);
+}
+
+MLA_API int mla_merge_splits_f32(const float* outs, const float* lses, int splits, int batch, int s_q, int h_q,
+                                 void* out, float* lse, void* stream) {
+  return merge_impl(outs, lses, splits, batch, s_q, h_q, out, lse, stream, 1);
 }
 
 MLA_API int mla_selftest_bounded_wait(void* stream) {

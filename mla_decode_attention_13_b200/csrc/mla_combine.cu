@@ -6,7 +6,8 @@
 // normalised output o_k and lse_k = ln sum_{j in piece} exp(z_j); the merge is
 //     lse = ln sum_k exp(lse_k),    out = sum_k exp(lse_k - lse) * o_k,
 // computed with the maximum lse_k subtracted first.  Work rows the plan gave
-// no pages (L = 0) produce out = 0 and lse = -inf here.
+// no pages (L = 0) produce out = 0 and lse = -inf here.  out is bf16, or fp32
+// for mla_decode_f32.
 //
 // Grid-stride over items (work row, query row, slice of the 512 output
 // columns); one warp per item.  The host picks the slices per query row (1,
@@ -83,6 +84,17 @@ struct Slice {
       }
     }
   }
+  __device__ static void store(float* orow, int slice, int lane, const float (&a)[kFloats], float scale) {
+#pragma unroll
+    for (int j = 0; j < kNVec; ++j) {
+      if constexpr (kVec == 4) {
+        *reinterpret_cast<float4*>(orow + col(slice, lane, j)) =
+            make_float4(a[4 * j] * scale, a[4 * j + 1] * scale, a[4 * j + 2] * scale, a[4 * j + 3] * scale);
+      } else {
+        *reinterpret_cast<float2*>(orow + col(slice, lane, j)) = make_float2(a[2 * j] * scale, a[2 * j + 1] * scale);
+      }
+    }
+  }
 };
 
 template <int S>
@@ -140,7 +152,7 @@ __global__ void __launch_bounds__(kCombineThreads, 4) mla_combine_kernel(const C
     if (row_g >= p.R) continue;
     const int t = row_g / p.h_q;
     const int hh = row_g - t * p.h_q;
-    __nv_bfloat16* orow = reinterpret_cast<__nv_bfloat16*>(p.out) + (static_cast<long long>(i) * p.R + row_g) * kDv;
+    const long long orow_off = (static_cast<long long>(i) * p.R + row_g) * kDv;
 
     // Online merge: m = running max of lse_k, s = sum exp(lse_k - m),
     // acc = sum exp(lse_k - m) o_k.
@@ -180,7 +192,10 @@ __global__ void __launch_bounds__(kCombineThreads, 4) mla_combine_kernel(const C
       m = m_new;
     }
     const bool any = s > 0.0f;
-    Sl::store(orow, slice, lane, acc, any ? 1.0f / s : 0.0f);
+    if (p.out_f32)
+      Sl::store(static_cast<float*>(p.out) + orow_off, slice, lane, acc, any ? 1.0f / s : 0.0f);
+    else
+      Sl::store(static_cast<__nv_bfloat16*>(p.out) + orow_off, slice, lane, acc, any ? 1.0f / s : 0.0f);
     if (slice == 0 && lane == 0)
       p.lse[(static_cast<long long>(i) * p.h_q + hh) * p.s_q + t] = any ? m + __logf(s) : -INFINITY;
   }

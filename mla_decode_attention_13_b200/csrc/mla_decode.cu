@@ -49,7 +49,8 @@
 //   block table ("FlashMLA overview": paged kvcache, block size 64); the
 //   producer warps read page ids 32 at a time.
 // A row the plan splits writes fp32 (O / l, lse) partials to the workspace
-// for the combine kernel; an unsplit row writes bf16 out and lse.
+// for the combine kernel; an unsplit row writes out (bf16, or fp32 for
+// mla_decode_f32) and lse.
 // Warp roles per CTA (384 threads): warp 0 = key/Q producer, warp 1 = TMEM
 // owner and (leader only) QK issuer, warp 2 = value producer, warp 3 =
 // (leader only) PV issuer, warps 4-11 = softmax and epilogue.  (A bulk L2 prefetch of the pages ahead of the key
@@ -133,6 +134,7 @@ constexpr int kVRing = 2;             // value tiles (and P tiles)
 constexpr int kPvBars = 4;
 constexpr float kTau = 8.0f;          // lazy-rescale threshold, log2 units
 constexpr uint64_t kTimeoutNs = 500ull * 1000ull * 1000ull;
+constexpr uint64_t kDrainNs = 2ull * 1000ull * 1000ull;  // teardown wait for in-flight copies after an abort
 constexpr int kRowsCta = kMTile / 2;  // 64 query rows per CTA
 
 // Shared-memory layout (offsets from a 1024-byte aligned base).  All operand
@@ -170,7 +172,13 @@ enum Bar : uint32_t {
 };
 constexpr uint32_t kOffTmemSlot = kOffBar + 8 * kNumBars;  // u32
 constexpr uint32_t kOffAbort = kOffTmemSlot + 4;           // u32
-constexpr uint32_t kSmemUsed = kOffAbort + 4;
+// u32 fill counts of the barriers that TMA copies complete on: [kKRing] key
+// slots and [1] Q (leader: the expect_tx it posted), [kVRing] value slots
+// (each CTA); read at teardown to wait for copies still in flight on abort.
+constexpr uint32_t kOffFill = kOffAbort + 4;
+constexpr uint32_t kFillQ = kKRing;
+constexpr uint32_t kFillV = kKRing + 1;
+constexpr uint32_t kSmemUsed = kOffFill + 4 * (kKRing + 1 + kVRing);
 constexpr uint32_t kSmemBytes = kSmemUsed + 1024;  // slack for aligning the base
 static_assert(kSmemBytes <= 232448, "shared memory budget");
 static_assert(kOffK % 1024 == 0 && kOffV % 1024 == 0 && kOffP % 1024 == 0, "1024-byte aligned tiles");
@@ -204,6 +212,7 @@ struct Ctx {
   __device__ uint32_t kslot(uint32_t k) const { return base + kOffK + k * kKSlot; }
   __device__ uint32_t vtile(uint32_t k) const { return base + kOffV + k * kVTile; }
   __device__ uint32_t ptile(uint32_t k) const { return base + kOffP + k * kPTile; }
+  __device__ volatile uint32_t* fill() const { return reinterpret_cast<volatile uint32_t*>(gbase + kOffFill); }
 };
 
 __device__ void raise_abort(const Ctx& c, uint32_t err_bits) {
@@ -362,7 +371,10 @@ __device__ void producer_k(const DecodeParams& p, const Ctx& c, int s_begin, int
       good = seg_it == 0 || wait_bar(c, c.bar(kBarQEmpty), (seg_it - 1) & 1);
       if (good) {
         MLA_TRACE(14, seg_it);
-        if (c.cta == 0) mbar_arrive_expect_tx(c.bar(kBarQFull), 2 * kQBytes);
+        if (c.cta == 0) {
+          mbar_arrive_expect_tx(c.bar(kBarQFull), 2 * kQBytes);
+          c.fill()[kFillQ] += 1;
+        }
         const int y = sg.i * p.R + sg.mt * kMTile + c.cta * kRowsCta;
         tma_load_3d_pair(c.base + kOffQ, &p.tm_q, c.lead_bar(kBarQFull), 0, y, 0);
       }
@@ -386,7 +398,10 @@ __device__ void producer_k(const DecodeParams& p, const Ctx& c, int s_begin, int
       if (lane == 0) {
         MLA_TRACE(10, ks);
         MLA_STEP(ks);
-        if (c.cta == 0) mbar_arrive_expect_tx(c.bar(kBarKFull + slot), gr.np * kPagePanel);
+        if (c.cta == 0) {
+          mbar_arrive_expect_tx(c.bar(kBarKFull + slot), gr.np * kPagePanel);
+          c.fill()[slot] += 1;
+        }
       }
       __syncwarp();
       if (my_load)
@@ -427,6 +442,7 @@ __device__ void producer_v(const DecodeParams& p, const Ctx& c, int s_begin, int
           MLA_STEP(ps);
           const uint32_t bar = c.bar(kBarVFull + slot);
           mbar_arrive_expect_tx(bar, kVTile);
+          c.fill()[kFillV + slot] += 1;
           tma_load_4d(c.vtile(slot), &p.tm_v, bar, 0, gr.page[q] * kPage, 2 * static_cast<int>(c.cta), 0);
         }
       }
@@ -762,7 +778,7 @@ __device__ void softmax_epilogue(const DecodeParams& p, const Ctx& c, uint32_t t
     const int col0 = 256 * sp + 128 * half;
     const int rd_row = lane >> 3;   // read-back: rows rd_row + 4 i, chunk lane % 8
     const int rd_chunk = lane & 7;
-    if (sg.slot < 0) {
+    if (sg.slot < 0 && !p.out_f32) {
       __nv_bfloat16* obase = reinterpret_cast<__nv_bfloat16*>(p.out) +
                              (static_cast<long long>(sg.i) * p.R + sg.mt * kMTile + row0) * kDv + col0;
       const int rows_ok = p.R - (sg.mt * kMTile + row0);  // rows of this warp that exist
@@ -798,8 +814,17 @@ __device__ void softmax_epilogue(const DecodeParams& p, const Ctx& c, uint32_t t
       }
       if (row_valid && half == 0 && sp == 0) p.lse[(static_cast<long long>(sg.i) * p.h_q + hh) * p.s_q + t] = lse_v;
     } else {
-      float* obase = p.o_part + (static_cast<long long>(sg.slot) * p.tile_rows + row0) * kDv + col0;
-      const int rows_ok = p.tile_rows - row0;
+      // fp32: a piece of a split row (its partial, in the workspace), or a
+      // whole row of an fp32 output.
+      float* obase;
+      int rows_ok;
+      if (sg.slot < 0) {
+        obase = static_cast<float*>(p.out) + (static_cast<long long>(sg.i) * p.R + sg.mt * kMTile + row0) * kDv + col0;
+        rows_ok = p.R - (sg.mt * kMTile + row0);
+      } else {
+        obase = p.o_part + (static_cast<long long>(sg.slot) * p.tile_rows + row0) * kDv + col0;
+        rows_ok = p.tile_rows - row0;
+      }
 #pragma unroll 1
       for (int k = 0; k < 4; ++k) {  // 32 columns (128 bytes of fp32) per step
         float o[32];
@@ -820,8 +845,12 @@ __device__ void softmax_epilogue(const DecodeParams& p, const Ctx& c, uint32_t t
         }
         __syncwarp();
       }
-      if (row_valid && half == 0 && sp == 0)
-        p.lse_part[static_cast<long long>(sg.slot) * p.tile_rows + q_row] = lse_v;
+      if (row_valid && half == 0 && sp == 0) {
+        if (sg.slot < 0)
+          p.lse[(static_cast<long long>(sg.i) * p.h_q + hh) * p.s_q + t] = lse_v;
+        else
+          p.lse_part[static_cast<long long>(sg.slot) * p.tile_rows + q_row] = lse_v;
+      }
     }
     tc_fence_before();
     __syncwarp();
@@ -836,6 +865,35 @@ __device__ void softmax_epilogue(const DecodeParams& p, const Ctx& c, uint32_t t
   }
   if (lane == 0) MLA_TRACE(19, (threadIdx.x >> 5) - 4);
   __syncwarp();
+}
+
+// After an abort: wait, bounded, for the last phase of every barrier that a
+// TMA copy of this CTA completes on, so that no copy is still writing this
+// CTA's shared memory when it exits.  A barrier filled n times has at most its
+// phase n - 1 outstanding (a slot is refilled only after its previous phase
+// completed).  The leader waits for the key and Q barriers, which count the
+// other CTA's bytes too; the other CTA then leaves only after the cluster
+// barrier that follows.  Returns false if a wait ran out (a copy that was
+// never issued by the other CTA, whose abort came first).
+__device__ __noinline__ bool drain_copies(const Ctx& c) {
+  volatile uint32_t* fill = c.fill();
+  bool ok = true;
+  auto wait_last = [&](uint32_t bar, uint32_t n) {
+    if (n == 0 || !ok) return;
+    const uint64_t t0 = globaltimer();
+    while (!mbar_try_wait(bar, (n - 1) & 1u)) {
+      if (globaltimer() - t0 > kDrainNs) {
+        ok = false;
+        return;
+      }
+    }
+  };
+  if (c.cta == 0) {
+    for (int k = 0; k < kKRing; ++k) wait_last(c.bar(kBarKFull + k), fill[k]);
+    wait_last(c.bar(kBarQFull), fill[kFillQ]);
+  }
+  for (int k = 0; k < kVRing; ++k) wait_last(c.bar(kBarVFull + k), fill[kFillV + k]);
+  return ok;
 }
 
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
@@ -878,6 +936,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     mbar_init(c.bar(kBarResc), 4);
     mbar_init(c.bar(kBarResc + 1), 4);
     *c.abort_flag = 0u;
+    for (uint32_t k = 0; k < kKRing + 1 + kVRing; ++k) c.fill()[k] = 0u;
     fence_mbar_init_cluster();
   }
   if (warp == 1) {
@@ -962,8 +1021,13 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     if (lane == 0) {
       umma_commit_pair(c.bar(kBarFinal), 0x1);  // QK issuer's MMAs
       const uint64_t t0 = globaltimer();
-      while (!mbar_try_wait(c.bar(kBarFinal), 0) && globaltimer() - t0 < kTimeoutNs) {
+      bool done = false;
+      while (!(done = mbar_try_wait(c.bar(kBarFinal), 0)) && globaltimer() - t0 < kTimeoutNs) {
       }
+      // MMAs that never completed are recorded; TMEM is still freed below:
+      // a CTA that exits holding TMEM would leave the next kernel's
+      // allocation on this SM pair waiting for good.
+      if (!done) set_error(c.meta, MLA_DEVERR_TIMEOUT);
     }
     __syncwarp();
   }
@@ -973,7 +1037,13 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     g_mla_span[blockIdx.x >> 1][2] = s_end - s_begin;
   }
 #endif
-  if (*c.abort_flag) __nanosleep(20000);  // let in-flight copies and arrivals land
+  // On abort: wait for this CTA's copies still in flight; the fixed pause is
+  // only a backstop for copies no barrier here can see (the other CTA's key
+  // or Q boxes for a phase this CTA never posted).
+  if (*c.abort_flag && threadIdx.x == 0) {
+    drain_copies(c);
+    __nanosleep(20000);
+  }
   tc_fence_before();
   __syncthreads();
   cluster_sync();

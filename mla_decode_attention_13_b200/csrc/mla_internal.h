@@ -121,6 +121,7 @@ struct DecodeParams {
   long long num_pages;
   int max_pages;
   int batch, s_q, h_q, R, n_mt, causal, tile_rows, max_slots;
+  int out_f32;             // 1: out is fp32 [batch][s_q][h_q][512] (mla_decode_f32), 0: bf16
   float scale_log2;        // softmax_scale * log2(e)
 };
 
@@ -132,6 +133,7 @@ struct CombineParams {
   float* lse;
   int batch, s_q, h_q, R, tile_rows, pairs, max_slots;
   int slices;  // warps per query row (1, 2, 4 or 8), each merging 512 / slices columns
+  int out_f32;  // as DecodeParams::out_f32
 };
 
 // Launch wrappers (each returns a cudaError_t).

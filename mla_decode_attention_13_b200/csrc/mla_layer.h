@@ -37,11 +37,12 @@ struct ProjParams {
 
 // Merge of per-split decode results (mla_merge_splits).
 struct MergeParams {
-  const void* outs;   // bf16 [splits][batch][s_q][h_q][512]
+  const void* outs;   // [splits][batch][s_q][h_q][512], bf16 or (in_f32) fp32
   const float* lses;  // [splits][batch][h_q][s_q]
   void* out;          // bf16 [batch][s_q][h_q][512]
   float* lse;         // [batch][h_q][s_q]
   int splits, batch, s_q, h_q;
+  int in_f32;
 };
 
 cudaError_t launch_projection(const ProjParams& p, bool absorb, cudaStream_t stream);

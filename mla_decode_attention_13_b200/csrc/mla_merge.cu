@@ -15,8 +15,9 @@
 // no visible token in any split gets out = 0 and lse = -inf.
 //
 // One warp per query row; each lane holds 16 of the 512 columns (two 16-byte
-// loads of bf16 per split).  The loads of the next split are issued before the
-// current one is folded in.
+// loads per split of bf16 partial outputs, four of fp32 ones from
+// mla_decode_f32).  The loads of the next split are issued before the current
+// one is folded in.
 #include <cuda_bf16.h>
 
 #include <cmath>
@@ -50,14 +51,49 @@ __device__ __forceinline__ uint4 pack8(const float* f) {
   return u;
 }
 
+// A lane's 16 columns of one split's row: [8 lane, +8) and [256 + 8 lane, +8),
+// from bf16 (two 16-byte loads) or fp32 (four) partial outputs.
+template <bool kF32>
+struct Part {
+  uint4 u[kF32 ? 4 : 2];
+  __device__ void load(const void* outs, long long row_elem, int lane) {
+    if constexpr (kF32) {
+      const uint4* b = static_cast<const uint4*>(outs);
+      const long long c0 = (row_elem + 8 * lane) / 4, c1 = (row_elem + 256 + 8 * lane) / 4;
+      u[0] = b[c0];
+      u[1] = b[c0 + 1];
+      u[2] = b[c1];
+      u[3] = b[c1 + 1];
+    } else {
+      const uint4* b = static_cast<const uint4*>(outs);
+      u[0] = b[(row_elem + 8 * lane) / 8];
+      u[1] = b[(row_elem + 256 + 8 * lane) / 8];
+    }
+  }
+  __device__ void unpack(float* f) const {
+    if constexpr (kF32) {
+#pragma unroll
+      for (int k = 0; k < 4; ++k) {
+        f[4 * k] = __uint_as_float(u[k].x);
+        f[4 * k + 1] = __uint_as_float(u[k].y);
+        f[4 * k + 2] = __uint_as_float(u[k].z);
+        f[4 * k + 3] = __uint_as_float(u[k].w);
+      }
+    } else {
+      unpack8(u[0], f);
+      unpack8(u[1], f + 8);
+    }
+  }
+};
+
+template <bool kF32>
 __global__ void __launch_bounds__(32 * kMergeWarps) mla_merge_kernel(const MergeParams p) {
   ptx::griddep_launch_dependents();
   ptx::griddep_wait();  // the partial results may come from the previous kernels
   const int lane = threadIdx.x & 31;
   const long long rows = static_cast<long long>(p.batch) * p.s_q * p.h_q;
-  const long long split_stride = rows * kDv;  // bf16 elements per split
+  const long long split_stride = rows * kDv;  // elements per split
   const long long lse_split_stride = rows;
-  const uint4* outs = static_cast<const uint4*>(p.outs);
   for (long long r = static_cast<long long>(blockIdx.x) * kMergeWarps + (threadIdx.x >> 5); r < rows;
        r += static_cast<long long>(gridDim.x) * kMergeWarps) {
     // out rows are [batch][s_q][h_q]; lse is [batch][h_q][s_q]
@@ -70,17 +106,14 @@ __global__ void __launch_bounds__(32 * kMergeWarps) mla_merge_kernel(const Merge
 #pragma unroll
     for (int k = 0; k < 16; ++k) acc[k] = 0.0f;
     float m = -INFINITY, s = 0.0f;
-    // lane's columns: [8 lane, +8) and [256 + 8 lane, +8)
-    const long long col0 = (r * kDv + 8 * lane) / 8, col1 = (r * kDv + 256 + 8 * lane) / 8;
-    uint4 u0 = outs[col0], u1 = outs[col1];
+    Part<kF32> cur;
+    cur.load(p.outs, r * kDv, lane);
     float l = p.lses[lse_idx];
     for (int k = 0; k < p.splits; ++k) {
-      uint4 n0 = u0, n1 = u1;
+      Part<kF32> nxt = cur;
       float nl = l;
       if (k + 1 < p.splits) {  // next split's loads before this one is folded in
-        const long long off = (k + 1) * split_stride / 8;
-        n0 = outs[col0 + off];
-        n1 = outs[col1 + off];
+        nxt.load(p.outs, (k + 1) * split_stride + r * kDv, lane);
         nl = p.lses[(k + 1) * lse_split_stride + lse_idx];
       }
       if (l != -INFINITY) {
@@ -88,15 +121,13 @@ __global__ void __launch_bounds__(32 * kMergeWarps) mla_merge_kernel(const Merge
         const float a = __expf(m - m2);  // 0 when m is -inf
         const float b = __expf(l - m2);
         float f[16];
-        unpack8(u0, f);
-        unpack8(u1, f + 8);
+        cur.unpack(f);
         s = s * a + b;
 #pragma unroll
         for (int c = 0; c < 16; ++c) acc[c] = acc[c] * a + b * f[c];
         m = m2;
       }
-      u0 = n0;
-      u1 = n1;
+      cur = nxt;
       l = nl;
     }
     uint4* out = static_cast<uint4*>(p.out);
@@ -133,7 +164,8 @@ cudaError_t launch_merge(const MergeParams& p, int sms, cudaStream_t stream) {
   attr[0].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  return cudaLaunchKernelEx(&cfg, mla_merge_kernel, p);
+  return p.in_f32 ? cudaLaunchKernelEx(&cfg, mla_merge_kernel<true>, p)
+                  : cudaLaunchKernelEx(&cfg, mla_merge_kernel<false>, p);
 }
 
 }  // namespace mla

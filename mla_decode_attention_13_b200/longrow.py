@@ -19,8 +19,13 @@ The shard rule (page-aligned, contiguous):
     shifted by 64 b_{W-1} positions.
 Ranks with no pages of a row get lse = -inf for it, which the merge ignores.
 
+The partial results cross between ranks unrounded: each rank decodes with
+mla_decode_f32 (fp32 out, 2052 bytes per query row with its lse) and
+mla_merge_splits_f32 merges them in fp32 and rounds once to bf16, so the split
+result keeps the error bars of an unsplit decode.
+
 Only host logic lives here: the compute is the library's kernels
-(mla_get_metadata, mla_decode, mla_merge_splits) and the exchange is
+(mla_get_metadata, mla_decode_f32, mla_merge_splits_f32) and the exchange is
 torch.distributed (NCCL between GPUs).
 """
 
@@ -115,7 +120,7 @@ def decode_sharded(q: torch.Tensor, kv_cache: torch.Tensor, local_table: torch.T
     rank = dist.get_rank(group) if dist.is_initialized() else 0
     _, s_q, h_q, _ = q.shape
     meta = binding.mla_get_metadata(local_seqlens, h_q, s_q, metadata=metadata)
-    out_r, lse_r = binding.mla_decode(q, kv_cache, local_table, local_seqlens, softmax_scale,
-                                      bool(causal) and rank == world - 1, meta)
+    out_r, lse_r = binding.mla_decode_f32(q, kv_cache, local_table, local_seqlens, softmax_scale,
+                                          bool(causal) and rank == world - 1, meta)
     outs, lses = gather_partials(out_r, lse_r, group)
-    return binding.mla_merge_splits(outs, lses)
+    return binding.mla_merge_splits_f32(outs, lses)

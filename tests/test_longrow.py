@@ -145,21 +145,23 @@ def _sharded_worker(rank, world, port, case, q):
     def get_metadata(seqlens, h_q, s_q, metadata=None, stream=None):
         return ("plan", tuple(int(v) for v in seqlens))
 
-    def decode(q, kv, table, seqlens, scale, causal, meta, **kw):
+    def decode_f32(q, kv, table, seqlens, scale, causal, meta, **kw):
+        # the split exchanges unrounded partials: fp32 out, as mla_decode_f32 writes
         assert meta == ("plan", tuple(int(v) for v in seqlens))
         calls.append(bool(causal))
         o, l = mla_oracle.decode(q, kv, table, seqlens, scale, causal)
-        return torch.from_numpy(o), torch.from_numpy(l)
+        return torch.from_numpy(o).float(), torch.from_numpy(l).float()
 
-    def merge(outs, lses, **kw):
+    def merge_f32(outs, lses, **kw):
+        assert outs.dtype == torch.float32 and lses.dtype == torch.float32
         w, b, s, h, _ = outs.shape
         parts = [(outs[k].numpy().reshape(b * s * h, 512), lses[k].numpy().transpose(0, 2, 1).reshape(-1))
                  for k in range(w)]
         o, l = mla_oracle.combine_partials(parts)
         return torch.from_numpy(o.reshape(b, s, h, 512)), torch.from_numpy(l.reshape(b, s, h).transpose(0, 2, 1))
 
-    longrow.binding = types.SimpleNamespace(mla_get_metadata=get_metadata, mla_decode=decode,
-                                            mla_merge_splits=merge)
+    longrow.binding = types.SimpleNamespace(mla_get_metadata=get_metadata, mla_decode_f32=decode_f32,
+                                            mla_merge_splits_f32=merge_f32)
     dist.init_process_group("gloo", rank=rank, world_size=world, timeout=datetime.timedelta(seconds=60))
     try:
         lens, h_q, s_q, causal = case
@@ -194,5 +196,6 @@ def test_decode_sharded_over_gloo_ranks_equals_the_unsplit_decode(world, case):
     res = sorted(q.get(timeout=5) for _ in range(world))
     causal = case[3]
     for rank, err, lerr, same_inf, calls in res:
-        assert err < 1e-12 and lerr < 1e-12 and same_inf, (rank, err, lerr)
+        # the stand-ins pass fp32 partials, as the library's do: fp32 rounding only
+        assert err < 1e-5 and lerr < 1e-5 and same_inf, (rank, err, lerr)
         assert calls == [causal and rank == world - 1]  # one decode per rank; only the last one masks

@@ -8,14 +8,20 @@ buffer already; what they cannot provide is the scratch workspace that
 mla_decode takes for the partial results of rows split across SM pairs.
 mla_decode_noalloc keeps that scratch in a fixed array inside the library.
 
-These tests call it through the C ABI and check its results against those of
-mla_decode with a caller-allocated workspace, on two calls in a row (the
-second with different inputs, so that scratch left over from the first call
-must not matter), on a shape whose plan does split rows.  The bar is the one
-the other GPU tests use (max-abs 8e-3, mean-abs 1e-3 on the bf16 output,
-|lse difference| <= 1e-3, -inf in the same places).
+These tests call it through the C ABI on two calls in a row (the second with
+different inputs, so that scratch left over from the first call must not
+matter), on shapes whose plans do split rows, and check its results two ways:
 
-The file is named so that pytest collects it last.
+  * against the fp64 oracle, with the bar the other GPU tests use (max-abs
+    8e-3, mean-abs 1e-3 on the bf16 output, |lse difference| <= 1e-3, -inf in
+    the same places);
+  * against mla_decode with a caller-allocated workspace, bit for bit: both
+    run the same plan through the same deterministic kernels and differ only
+    in where the partials live, so any difference at all (stale or partly
+    overwritten scratch) is a fault.
+
+One call runs on a non-default stream and is synchronised through that stream
+alone.  The file is named so that pytest collects it last.
 """
 
 import numpy as np
@@ -23,6 +29,7 @@ import pytest
 import torch
 
 from mla_decode_attention_13_b200 import binding, inputs
+from oracle import mla_oracle
 
 pytestmark = pytest.mark.gpu
 
@@ -35,33 +42,47 @@ CASES = [
 ]
 
 
-def _compare(ref, got):
-    (ro, rl), (go, gl) = ref, got
-    d = (ro.float() - go.float()).abs()
-    assert torch.isfinite(go.float()).all(), "non-finite output"
-    assert d.max().item() <= TOL_MAX, f"max-abs {d.max().item():.3e}"
-    assert d.mean().item() <= TOL_MEAN, f"mean-abs {d.mean().item():.3e}"
-    rl, gl = rl.cpu().numpy(), gl.cpu().numpy()
-    inf = np.isneginf(rl)
-    assert np.array_equal(inf, np.isneginf(gl)), "lse -inf pattern differs"
+def _against_oracle(x, out, lse):
+    want_o, want_l = mla_oracle.decode(x.q, x.kv_cache, x.block_table, x.seqlens, x.softmax_scale, x.causal)
+    got_o = out.cpu().double().numpy()
+    got_l = lse.cpu().double().numpy()
+    assert np.isfinite(got_o).all(), "non-finite output"
+    d = np.abs(got_o - want_o)
+    assert d.max() <= TOL_MAX, f"max-abs {d.max():.3e}"
+    assert d.mean() <= TOL_MEAN, f"mean-abs {d.mean():.3e}"
+    inf = np.isneginf(want_l)
+    assert np.array_equal(inf, np.isneginf(got_l)), "lse -inf pattern differs"
     if (~inf).any():
-        assert np.abs(rl[~inf] - gl[~inf]).max() <= TOL_LSE
+        assert np.abs(got_l[~inf] - want_l[~inf]).max() <= TOL_LSE
+
+
+def _bitwise_equal(ref, got):
+    (ro, rl), (go, gl) = ref, got
+    assert torch.equal(ro.view(torch.int16), go.view(torch.int16)), "out differs from mla_decode"
+    assert torch.equal(rl.view(torch.int32), gl.view(torch.int32)), "lse differs from mla_decode"
 
 
 @pytest.mark.parametrize("lens,h_q,s_q,causal", CASES)
-def test_noalloc_matches_decode_on_two_calls(lens, h_q, s_q, causal):
+def test_noalloc_matches_oracle_and_decode_on_two_calls(lens, h_q, s_q, causal):
+    side = torch.cuda.Stream()
     for call in range(2):
-        x = inputs.make_inputs(lens, h_q, s_q, seed=70 + call, causal=causal).to("cuda")
+        xc = inputs.make_inputs(lens, h_q, s_q, seed=70 + call, causal=causal)
+        x = xc.to("cuda")
         meta = binding.mla_get_metadata(x.seqlens, x.h_q, x.s_q)
         torch.cuda.synchronize()
         assert int(meta[5].item()) > 0, "the plan should split at least one row"
         ref = binding.mla_decode(x.q, x.kv_cache, x.block_table, x.seqlens, x.softmax_scale, x.causal, meta)
+        torch.cuda.synchronize()
         out = torch.full((x.batch, x.s_q, x.h_q, 512), float("nan"), dtype=torch.bfloat16, device="cuda")
         lse = torch.full((x.batch, x.h_q, x.s_q), float("nan"), dtype=torch.float32, device="cuda")
+        torch.cuda.synchronize()
+        # the second call goes through an explicit non-default stream, synchronised on that stream only
+        stream = side if call == 1 else None
         got = binding.mla_decode_noalloc(x.q, x.kv_cache, x.block_table, x.seqlens, x.softmax_scale, x.causal, meta,
-                                         out, lse)
-        assert binding.mla_check_device_error(meta) == 0
-        _compare(ref, got)
+                                         out, lse, stream=stream)
+        assert binding.mla_check_device_error(meta, stream=stream) == 0
+        _against_oracle(xc, got[0], got[1])
+        _bitwise_equal(ref, got)
 
 
 def test_noalloc_rejects_bad_arguments_before_launch():
