@@ -85,6 +85,19 @@ def visible_pairs(lens, h_q, s_q, causal):
     return n
 
 
+def algorithmic_work_fp8(lens, h_q, s_q, causal):
+    """As algorithmic_work for an FP8 latent cache: every cached token once as
+    512 E4M3 codes, 64 bf16 rope values and one exponent byte (641 B instead
+    of 1152 B); the rest (Q, output, lse, table, lengths) and the FLOPs are
+    unchanged."""
+    rows = s_q * h_q
+    tokens = sum(lens)
+    pages = sum((L + 63) // 64 for L in lens)
+    nbytes = tokens * (512 + 64 * 2 + 1) + len(lens) * rows * (576 * 2 + 512 * 2 + 4) + pages * 4 + len(lens) * 4
+    flops = 2 * (576 + 512) * visible_pairs(lens, h_q, s_q, causal)
+    return nbytes, flops
+
+
 def algorithmic_work(lens, h_q, s_q, causal):
     """Bytes the decode kernel must move and FLOPs it must do.
 
@@ -414,10 +427,12 @@ def parity_check(idx, dev, budget_s, min_rows=8, all_rows_ok=True):
 # ----------------------------------------------------------------------------
 
 class Bench:
-    """One workload's rotating pools, buffers and step graphs on this GPU."""
+    """One workload's rotating pools, buffers and step graphs on this GPU
+    (bf16 cache, or with fp8 the FP8 latent cache of mla_decode_fp8)."""
 
-    def __init__(self, idx, dev, rank, stream):
+    def __init__(self, idx, dev, rank, stream, fp8=False):
         self.idx = idx
+        self.fp8 = fp8
         self.wl = wl = inputs.WORKLOADS[idx]
         self.dev = dev
         self.stream = stream
@@ -426,11 +441,17 @@ class Bench:
         pools, total = [], 0
         while len(pools) < 2 or total < 3 * self.l2:
             seed = 1000 + idx + 7919 * (len(pools) + 1) + 104729 * rank
-            one = inputs.make_inputs(self.lens, wl.h_q, wl.s_q, seed=seed, causal=wl.causal,
-                                     softmax_scale=wl.softmax_scale, pool_factor=wl.pool_factor, device=str(dev),
-                                     name=wl.name)
+            if fp8:
+                one = inputs.make_fp8_inputs(self.lens, wl.h_q, wl.s_q, seed=seed, causal=wl.causal,
+                                             softmax_scale=wl.softmax_scale, pool_factor=wl.pool_factor,
+                                             device=str(dev))
+                total += sum(t.numel() * t.element_size() for t in (one.latent_codes, one.rope, one.exps, one.q))
+            else:
+                one = inputs.make_inputs(self.lens, wl.h_q, wl.s_q, seed=seed, causal=wl.causal,
+                                         softmax_scale=wl.softmax_scale, pool_factor=wl.pool_factor, device=str(dev),
+                                         name=wl.name)
+                total += one.kv_cache.numel() * 2 + one.q.numel() * 2
             pools.append(one)
-            total += one.kv_cache.numel() * 2 + one.q.numel() * 2
             if len(pools) >= 64:
                 break
         self.pools, self.total = pools, total
@@ -447,8 +468,13 @@ class Bench:
     def step(self, r, events=None):
         x = self.pools[r]
         binding.mla_get_metadata(x.seqlens, x.h_q, x.s_q, metadata=self.metas[r], stream=self.stream)
-        binding.mla_decode(x.q, x.kv_cache, x.block_table, x.seqlens, x.softmax_scale, x.causal, self.metas[r],
-                           workspace=self.ws, out=self.out, lse=self.lse, stream=self.stream, events=events)
+        if self.fp8:
+            binding.mla_decode_fp8(x.q, x.latent_codes, x.rope, x.exps, x.block_table, x.seqlens, x.softmax_scale,
+                                   x.causal, self.metas[r], workspace=self.ws, out=self.out, lse=self.lse,
+                                   stream=self.stream, events=events)
+        else:
+            binding.mla_decode(x.q, x.kv_cache, x.block_table, x.seqlens, x.softmax_scale, x.causal, self.metas[r],
+                               workspace=self.ws, out=self.out, lse=self.lse, stream=self.stream, events=events)
 
     def warm_up(self, n):
         for k in range(max(n, 1)):
@@ -675,9 +701,72 @@ def e2e_timing(B, K, world):
 
 def roofline_for(B, k2_ms, k2_source, peaks):
     hbm_peak, tf_peak, _, peak_kind = peaks
-    nbytes, flops = algorithmic_work(B.lens, B.wl.h_q, B.wl.s_q, B.wl.causal)
-    return roofline_entry(nbytes, flops, k2_ms * 1e-3, hbm_peak, tf_peak, peak_kind, committed_traffic(B.wl.name),
-                          k2_source), nbytes, flops
+    work = algorithmic_work_fp8 if B.fp8 else algorithmic_work
+    nbytes, flops = work(B.lens, B.wl.h_q, B.wl.s_q, B.wl.causal)
+    traffic = committed_traffic(("fp8:" if B.fp8 else "") + B.wl.name)
+    entry = roofline_entry(nbytes, flops, k2_ms * 1e-3, hbm_peak, tf_peak, peak_kind, traffic, k2_source)
+    if B.fp8:
+        entry["kernel"] = "mla_decode_kernel (FP8 latent cache)"
+    return entry, nbytes, flops
+
+
+def parity_check_fp8(idx, dev, min_rows=8):
+    """The FP8-cache decode on seeded inputs of the workload's shape (drawn on
+    the CPU) against the oracle's decode_fp8, on a seeded sample of at least
+    min_rows rows with the shortest and longest (every row when there are
+    no more)."""
+    from oracle import mla_oracle
+
+    wl = inputs.WORKLOADS[idx]
+    lens = workload_lengths(idx)
+    x = inputs.make_fp8_inputs(lens, wl.h_q, wl.s_q, seed=3000 + idx, causal=wl.causal,
+                               softmax_scale=wl.softmax_scale, pool_factor=wl.pool_factor)
+    g = x.to(dev)
+    meta = binding.mla_get_metadata(g.seqlens, g.h_q, g.s_q)
+    out, lse = binding.mla_decode_fp8(g.q, g.latent_codes, g.rope, g.exps, g.block_table, g.seqlens,
+                                      g.softmax_scale, g.causal, meta)
+    torch.cuda.synchronize(dev)
+    err = binding.mla_check_device_error(meta)
+    got_o = out.cpu().double().numpy()
+    got_l = lse.cpu().double().numpy()
+    del g, meta, out, lse
+    rows = sample_rows(lens, min(min_rows, wl.batch), seed=idx)
+    want_o, want_l = mla_oracle.decode_fp8(x.q, x.latent_codes, x.rope, x.exps, x.block_table, x.seqlens,
+                                           x.softmax_scale, x.causal, rows=rows)
+    go, gl, wo, wl_ = got_o[rows], got_l[rows], want_o[rows], want_l[rows]
+    d = np.abs(go - wo)
+    inf = np.isneginf(wl_)
+    neg_inf_match = bool(np.array_equal(np.isneginf(gl), inf))
+    lse_max = float(np.abs(gl[~inf] - wl_[~inf]).max()) if (~inf).any() else 0.0
+    finite = bool(np.isfinite(go).all())
+    return {"max_abs": float(d.max()), "mean_abs": float(d.mean()), "lse_max_abs": lse_max,
+            "neg_inf_match": neg_inf_match, "finite": finite, "device_error_word": int(err),
+            "rows": rows, "of_rows": wl.batch, "elements": int(d.size),
+            "tolerance": {"max_abs": TOL_MAX, "mean_abs": TOL_MEAN, "lse_max_abs": TOL_LSE},
+            "pass": bool(d.max() <= TOL_MAX and d.mean() <= TOL_MEAN and lse_max <= TOL_LSE and neg_inf_match
+                         and finite and err == 0),
+            "inputs": "seeded FP8 inputs of the workload's shape (seed 3000 + index, drawn on the CPU): E4M3 codes "
+                      "of N(0, 64^2) values, token exponents uniform in [-8, -5], bf16 rope and q ~ N(0, 1)"}
+
+
+def fp8_workload(idx, args, world, rank, local, dev, stream, peaks):
+    """The FP8 latent cache (mla_decode_fp8) on a workload's shape: step
+    time, decode-kernel roofline on the FP8 bytes, and a parity sample."""
+    B = Bench(idx, dev, rank, stream, fp8=True)
+    B.warm_up(args.warmup)
+    B.capture()
+    K = max(B.npool, min(args.steps, 200))
+    ms_step, clocks = B.timed_steps(K, world, local)
+    k2_ms, k2_source, k2_clocks = B.decode_kernel_timing(K, local)
+    roof, nbytes, _ = roofline_for(B, k2_ms, k2_source, peaks)
+    entry = {"config": {**workload_config(B.wl, idx, B.lens), "cache": "fp8 e4m3 latent + per-token 2^e + bf16 rope"},
+             "step_us": round(ms_step * 1e3 / world, 3), "steps": K, "decode_kernel_us": round(k2_ms * 1e3, 3),
+             "roofline": roof, "decode_kernel_clocks": k2_clocks, "clocks": clocks,
+             "pools": f"{B.npool} rotating pools, {B.total / 2**20:.0f} MiB"}
+    B.release()
+    if world == 1 and not args.no_cpu_baseline:
+        entry["parity"] = parity_check_fp8(idx, dev)
+    return entry
 
 
 def other_workload(idx, args, world, rank, local, dev, stream, peaks):
@@ -778,6 +867,10 @@ def ours(args, world, rank, local):
         if mb in others:
             line["memory_bound"] = others.pop(mb)
         line["other_workloads"] = others
+        # The FP8 latent cache on the memory-bound sweep's shape and the
+        # headline's.
+        line["fp8_cache"] = {inputs.WORKLOADS[j].name: fp8_workload(j, args, world, rank, local, dev, stream, peaks)
+                             for j in (2, idx) if j < len(inputs.WORKLOADS)}
     if rank == 0:
         print(json.dumps(line), flush=True)
 

@@ -80,6 +80,9 @@ extern "C" {
 #define MLA_DEVERR_PLAN 0x8u     /* metadata does not match this call (its
                                     shape, or lengths that changed since it
                                     was built)                               */
+#define MLA_DEVERR_FP8_RANGE 0x10u /* mla_decode_fp8: a visible token's scale
+                                      exponent outside [-15, 7], or a query
+                                      value past the f16 range              */
 
 /* Fixed dimensions of the absorbed cache row and of a page. */
 #define MLA_D_QK 576
@@ -167,6 +170,46 @@ int mla_decode_f32(const void* q, const void* kv_cache, int64_t num_pages, const
                    int max_pages_per_seq, const int32_t* seqlens, int batch, int s_q, int h_q, float softmax_scale,
                    int causal, float* out, float* lse, void* metadata, void* workspace, size_t workspace_bytes,
                    void* stream);
+
+/*
+ * MLA decode over an FP8 latent cache.  "MLA 和 MHA 的 Kernel 区别", section
+ * "量化友好性": the compressed latent c_KV tolerates FP8 (or INT8) storage,
+ * with the dequantisation fused into the load, which halves the bytes a
+ * memory-bound decode reads.  The pages fix no format; this call takes:
+ *
+ *   latent_codes [device] uint8 [num_pages][64][512]: OCP FP8 E4M3 codes of
+ *                the 512 latent dims of each cached token (1 sign, 4
+ *                exponent bits with bias 7, 3 mantissa bits; largest finite
+ *                value 448), 16-byte aligned;
+ *   rope         [device] bf16 [num_pages][64][64]: the 64 rope dims, which
+ *                are not part of c_KV and stay bf16, 16-byte aligned;
+ *   exps         [device] int8 [num_pages][64]: each token's scale exponent
+ *                e, 16-byte aligned.
+ *
+ * Cached token j of a page is the 576-wide row [code_value(latent_codes[j])
+ * * 2^exps[j], rope[j]], and the result is mla_decode's over those rows:
+ * every other argument, the plan (one mla_get_metadata serves both calls),
+ * the outputs and the errors are those of mla_decode.  Every E4M3 value
+ * times 2^e with -15 <= e <= 7 is exact in f16; the kernel computes the
+ * latent products in f16 (the latent part of q converted to f16, the rope
+ * part in bf16) and accumulates in fp32.  A visible token whose exponent is
+ * outside [-15, 7], or a query value past the f16 range (|q| >= 65520), sets
+ * MLA_DEVERR_FP8_RANGE in the device error word (its results are then not
+ * those of the definition); query values below 2^-14 in magnitude keep an
+ * absolute precision of 2^-25.
+ */
+int mla_decode_fp8(const void* q, const void* latent_codes, const void* rope, const int8_t* exps, int64_t num_pages,
+                   const int32_t* block_table, int max_pages_per_seq, const int32_t* seqlens, int batch, int s_q,
+                   int h_q, float softmax_scale, int causal, void* out, float* lse, void* metadata, void* workspace,
+                   size_t workspace_bytes, void* stream);
+
+/* mla_decode_fp8 with events around its split-KV decode kernel, as
+   mla_decode_timed. */
+int mla_decode_fp8_timed(const void* q, const void* latent_codes, const void* rope, const int8_t* exps,
+                         int64_t num_pages, const int32_t* block_table, int max_pages_per_seq, const int32_t* seqlens,
+                         int batch, int s_q, int h_q, float softmax_scale, int causal, void* out, float* lse,
+                         void* metadata, void* workspace, size_t workspace_bytes, void* stream,
+                         void* event_before_decode, void* event_after_decode);
 
 /*
  * mla_decode, plus CUDA events recorded on `stream` immediately before and

@@ -28,6 +28,7 @@ MLA_DEVERR_SEQLEN = 0x1
 MLA_DEVERR_PAGE = 0x2
 MLA_DEVERR_TIMEOUT = 0x4
 MLA_DEVERR_PLAN = 0x8
+MLA_DEVERR_FP8_RANGE = 0x10
 
 EXPORTED = (
     "mla_metadata_bytes",
@@ -36,6 +37,8 @@ EXPORTED = (
     "mla_get_metadata",
     "mla_decode",
     "mla_decode_f32",
+    "mla_decode_fp8",
+    "mla_decode_fp8_timed",
     "mla_decode_timed",
     "mla_decode_noalloc",
     "mla_absorb_q",
@@ -80,6 +83,10 @@ def lib() -> ctypes.CDLL:
         L.mla_decode.argtypes = dec
         L.mla_decode_f32.restype = ctypes.c_int
         L.mla_decode_f32.argtypes = dec
+        L.mla_decode_fp8.restype = ctypes.c_int
+        L.mla_decode_fp8.argtypes = [_vp, _vp, _vp, _vp] + dec[2:]
+        L.mla_decode_fp8_timed.restype = ctypes.c_int
+        L.mla_decode_fp8_timed.argtypes = [_vp, _vp, _vp, _vp] + dec[2:] + [_vp, _vp]
         L.mla_decode_timed.restype = ctypes.c_int
         L.mla_decode_timed.argtypes = dec + [_vp, _vp]
         L.mla_decode_noalloc.restype = ctypes.c_int
@@ -215,6 +222,53 @@ def mla_decode_f32(q: torch.Tensor, kv_cache: torch.Tensor, block_table: torch.T
                                 int(block_table.shape[1]), _ptr(seqlens), batch, s_q, h_q, float(softmax_scale),
                                 int(bool(causal)), _ptr(out), _ptr(lse), _ptr(metadata), _ptr(workspace),
                                 int(workspace.numel() * workspace.element_size()), _stream_ptr(stream)))
+    return out, lse
+
+
+def mla_decode_fp8(q: torch.Tensor, latent_codes: torch.Tensor, rope: torch.Tensor, exps: torch.Tensor,
+                   block_table: torch.Tensor, seqlens: torch.Tensor, softmax_scale: float, causal: bool,
+                   metadata: torch.Tensor, workspace: Optional[torch.Tensor] = None,
+                   out: Optional[torch.Tensor] = None, lse: Optional[torch.Tensor] = None, stream=None,
+                   events: Optional[Tuple] = None) -> Tuple[torch.Tensor, torch.Tensor]:
+    """MLA decode over an FP8 latent cache: latent_codes [pages, 64, 512]
+    uint8 (E4M3), rope [pages, 64, 64] bf16, exps [pages, 64] int8 (token
+    scale 2^exp).  Returns (out [b, s_q, h_q, 512] bf16, lse [b, h_q, s_q]).
+
+    ``events`` = (before, after) torch.cuda.Event recorded around the split-KV
+    kernel (timing only: mla_decode_fp8_timed)."""
+    batch, s_q, h_q, d = q.shape
+    pages = int(latent_codes.shape[0])
+    if d != 576 or q.dtype != torch.bfloat16:
+        raise MLAError("mla_decode_fp8", MLA_ERR_ARG)
+    if tuple(latent_codes.shape) != (pages, 64, 512) or latent_codes.dtype != torch.uint8:
+        raise MLAError("mla_decode_fp8", MLA_ERR_ARG)
+    if tuple(rope.shape) != (pages, 64, 64) or rope.dtype != torch.bfloat16:
+        raise MLAError("mla_decode_fp8", MLA_ERR_ARG)
+    if tuple(exps.shape) != (pages, 64) or exps.dtype != torch.int8:
+        raise MLAError("mla_decode_fp8", MLA_ERR_ARG)
+    for t in (q, latent_codes, rope, exps, block_table, seqlens):
+        if not t.is_contiguous():
+            raise MLAError("mla_decode_fp8", MLA_ERR_ARG)
+    if out is None:
+        out = torch.empty(batch, s_q, h_q, 512, dtype=torch.bfloat16, device=q.device)
+    if lse is None:
+        lse = torch.empty(batch, h_q, s_q, dtype=torch.float32, device=q.device)
+    if workspace is None:
+        workspace = torch.empty(max(mla_workspace_bytes(batch, h_q, s_q), 16), dtype=torch.uint8, device=q.device)
+    args = [_ptr(q), _ptr(latent_codes), _ptr(rope), _ptr(exps), pages, _ptr(block_table),
+            int(block_table.shape[1]), _ptr(seqlens), batch, s_q, h_q, float(softmax_scale), int(bool(causal)),
+            _ptr(out), _ptr(lse), _ptr(metadata), _ptr(workspace), int(workspace.numel() * workspace.element_size()),
+            _stream_ptr(stream)]
+    if events is None:
+        status = lib().mla_decode_fp8(*args)
+    else:
+        ev = []
+        for e in events:
+            if e is not None and int(e.cuda_event) == 0:
+                e.record()  # torch creates the CUDA event lazily, on first record
+            ev.append(None if e is None else int(e.cuda_event))
+        status = lib().mla_decode_fp8_timed(*args, *ev)
+    _check("mla_decode_fp8", status)
     return out, lse
 
 

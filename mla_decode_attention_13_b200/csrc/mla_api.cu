@@ -85,7 +85,7 @@ int tensor_map_encoder(PFN_cuTensorMapEncodeTiled_v12000* fn) {
 // same cache and a few rotating query buffers, so their maps are encoded once
 // instead of on every call.  A map holds only the address and the layout, so
 // it stays right for any later buffer at the same address and size.
-enum MapKind : int { kMapK = 0, kMapV = 1, kMapQ = 2, kMapKinds = 3 };
+enum MapKind : int { kMapK = 0, kMapV = 1, kMapQ = 2, kMapCodes = 3, kMapRope = 4, kMapKinds = 5 };
 
 struct MapCache {
   static constexpr int kWays = 8;
@@ -179,6 +179,32 @@ int encode_value_tiles(PFN_cuTensorMapEncodeTiled_v12000 enc, CUtensorMap* map, 
   return r == CUDA_SUCCESS ? MLA_OK : MLA_ERR_CUDA;
 }
 
+// FP8 cache: the latent codes [rows][512] u8 as (512 cols, rows), box (64
+// codes, 64 tokens), unswizzled (64-byte rows in shared memory).
+int encode_codes(PFN_cuTensorMapEncodeTiled_v12000 enc, CUtensorMap* map, const void* base, uint64_t rows) {
+  const cuuint64_t dims[2] = {static_cast<cuuint64_t>(kDv), static_cast<cuuint64_t>(rows)};
+  const cuuint64_t strides[1] = {static_cast<cuuint64_t>(kDv)};
+  const cuuint32_t box[2] = {64, static_cast<cuuint32_t>(kPage)};
+  const cuuint32_t elem[2] = {1, 1};
+  const CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void*>(base), dims, strides, box, elem,
+                         CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                         CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS ? MLA_OK : MLA_ERR_CUDA;
+}
+
+// FP8 cache: the bf16 rope [rows][64] as (64 cols, rows), box (64, 64 tokens),
+// 128B-swizzled: one page lands as a key panel's 64 rows.
+int encode_rope(PFN_cuTensorMapEncodeTiled_v12000 enc, CUtensorMap* map, const void* base, uint64_t rows) {
+  const cuuint64_t dims[2] = {64, static_cast<cuuint64_t>(rows)};
+  const cuuint64_t strides[1] = {128};
+  const cuuint32_t box[2] = {64, static_cast<cuuint32_t>(kPage)};
+  const cuuint32_t elem[2] = {1, 1};
+  const CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box, elem,
+                         CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                         CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS ? MLA_OK : MLA_ERR_CUDA;
+}
+
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
 // A [tokens][h_q][cols] bf16 tensor as (64 cols, tokens, cols / 64 panels,
@@ -249,15 +275,27 @@ bool shape_ok(int batch, int h_q, int s_q) {
          static_cast<long long>(batch) * s_q * h_q <= (1LL << 30);
 }
 
-int decode_impl(const void* q, const void* kv_cache, int64_t num_pages, const int32_t* block_table,
+// The cache of one call: a bf16 cache (kv), or an FP8 one (codes, rope, exps).
+struct CacheRef {
+  const void* kv = nullptr;
+  const void* codes = nullptr;
+  const void* rope = nullptr;
+  const void* exps = nullptr;
+  bool fp8() const { return kv == nullptr; }
+  bool ok() const { return fp8() ? (codes && rope && exps && aligned16(codes) && aligned16(rope) && aligned16(exps))
+                                 : aligned16(kv); }
+};
+
+int decode_impl(const void* q, const CacheRef& cache, int64_t num_pages, const int32_t* block_table,
                 int max_pages_per_seq, const int32_t* seqlens, int batch, int s_q, int h_q, float softmax_scale,
                 int causal, void* out, float* lse, void* metadata, void* workspace, size_t workspace_bytes,
                 void* stream, void* ev_before, void* ev_after, int out_f32) {
-  if (!q || !kv_cache || !block_table || !seqlens || !out || !lse || !metadata) return MLA_ERR_ARG;
+  if (!q || !block_table || !seqlens || !out || !lse || !metadata) return MLA_ERR_ARG;
+  if (!cache.ok()) return MLA_ERR_ARG;
   if (batch < 1 || h_q < 1 || s_q < 1 || max_pages_per_seq < 1 || num_pages < 1) return MLA_ERR_ARG;
   if (causal != 0 && causal != 1) return MLA_ERR_ARG;
   if (!std::isfinite(softmax_scale) || softmax_scale < 0.0f) return MLA_ERR_ARG;
-  if (!aligned16(q) || !aligned16(kv_cache) || !aligned16(out) || !aligned16(metadata)) return MLA_ERR_ARG;
+  if (!aligned16(q) || !aligned16(out) || !aligned16(metadata)) return MLA_ERR_ARG;
   if (workspace && !aligned16(workspace)) return MLA_ERR_ARG;
   if (!shape_ok(batch, h_q, s_q)) return MLA_ERR_UNSUPPORTED;
   if (num_pages > (1LL << 25)) return MLA_ERR_UNSUPPORTED;  // row coordinates stay below 2^31
@@ -273,18 +311,31 @@ int decode_impl(const void* q, const void* kv_cache, int64_t num_pages, const in
   const int R = s_q * h_q;
   const int tr = tile_rows(h_q, s_q);
   const int slots = max_slots(dev.pairs);
-  DecodeParams p;
+  DecodeParams p = {};
   const uint64_t kv_rows = static_cast<uint64_t>(num_pages) * kPage;
   const uint64_t q_rows = static_cast<uint64_t>(batch) * R;
-  if ((st = cached_map(kMapK, kv_cache, kv_rows, &p.tm_k,
-                       [&](CUtensorMap* m) { return encode_panels576(enc, m, kv_cache, kv_rows, kPage, 1); })) !=
-          MLA_OK ||
-      (st = cached_map(kMapV, kv_cache, kv_rows, &p.tm_v,
-                       [&](CUtensorMap* m) { return encode_value_tiles(enc, m, kv_cache, kv_rows); })) != MLA_OK ||
-      (st = cached_map(kMapQ, q, q_rows, &p.tm_q,
+  if ((st = cached_map(kMapQ, q, q_rows, &p.tm_q,
                        [&](CUtensorMap* m) { return encode_panels576(enc, m, q, q_rows, kMTile / 2, kDqk / 64); })) !=
-          MLA_OK)
+      MLA_OK)
     return st;
+  p.fp8 = cache.fp8() ? 1 : 0;
+  p.codes = static_cast<const uint8_t*>(cache.codes);
+  p.exps = static_cast<const int8_t*>(cache.exps);
+  if (cache.fp8()) {
+    if ((st = cached_map(kMapCodes, cache.codes, kv_rows, &p.tm_codes,
+                         [&](CUtensorMap* m) { return encode_codes(enc, m, cache.codes, kv_rows); })) != MLA_OK ||
+        (st = cached_map(kMapRope, cache.rope, kv_rows, &p.tm_rope,
+                         [&](CUtensorMap* m) { return encode_rope(enc, m, cache.rope, kv_rows); })) != MLA_OK)
+      return st;
+  } else {
+    const void* kv_cache = cache.kv;
+    if ((st = cached_map(kMapK, kv_cache, kv_rows, &p.tm_k,
+                         [&](CUtensorMap* m) { return encode_panels576(enc, m, kv_cache, kv_rows, kPage, 1); })) !=
+            MLA_OK ||
+        (st = cached_map(kMapV, kv_cache, kv_rows, &p.tm_v,
+                         [&](CUtensorMap* m) { return encode_value_tiles(enc, m, kv_cache, kv_rows); })) != MLA_OK)
+      return st;
+  }
   p.block_table = block_table;
   p.seqlens = seqlens;
   p.out = out;
@@ -380,7 +431,9 @@ MLA_API int mla_decode(const void* q, const void* kv_cache, int64_t num_pages, c
                        int max_pages_per_seq, const int32_t* seqlens, int batch, int s_q, int h_q, float softmax_scale,
                        int causal, void* out, float* lse, void* metadata, void* workspace, size_t workspace_bytes,
                        void* stream) {
-  return decode_impl(q, kv_cache, num_pages, block_table, max_pages_per_seq, seqlens, batch, s_q, h_q, softmax_scale,
+  CacheRef cache;
+  cache.kv = kv_cache;
+  return decode_impl(q, cache, num_pages, block_table, max_pages_per_seq, seqlens, batch, s_q, h_q, softmax_scale,
                      causal, out, lse, metadata, workspace, workspace_bytes, stream, nullptr, nullptr, 0);
 }
 
@@ -388,8 +441,38 @@ MLA_API int mla_decode_f32(const void* q, const void* kv_cache, int64_t num_page
                            int max_pages_per_seq, const int32_t* seqlens, int batch, int s_q, int h_q,
                            float softmax_scale, int causal, float* out, float* lse, void* metadata, void* workspace,
                            size_t workspace_bytes, void* stream) {
-  return decode_impl(q, kv_cache, num_pages, block_table, max_pages_per_seq, seqlens, batch, s_q, h_q, softmax_scale,
+  CacheRef cache;
+  cache.kv = kv_cache;
+  return decode_impl(q, cache, num_pages, block_table, max_pages_per_seq, seqlens, batch, s_q, h_q, softmax_scale,
                      causal, out, lse, metadata, workspace, workspace_bytes, stream, nullptr, nullptr, 1);
+}
+
+MLA_API int mla_decode_fp8(const void* q, const void* latent_codes, const void* rope, const int8_t* exps,
+                           int64_t num_pages, const int32_t* block_table, int max_pages_per_seq, const int32_t* seqlens,
+                           int batch, int s_q, int h_q, float softmax_scale, int causal, void* out, float* lse,
+                           void* metadata, void* workspace, size_t workspace_bytes, void* stream) {
+  if (!latent_codes || !rope || !exps) return MLA_ERR_ARG;
+  CacheRef cache;
+  cache.codes = latent_codes;
+  cache.rope = rope;
+  cache.exps = exps;
+  return decode_impl(q, cache, num_pages, block_table, max_pages_per_seq, seqlens, batch, s_q, h_q, softmax_scale,
+                     causal, out, lse, metadata, workspace, workspace_bytes, stream, nullptr, nullptr, 0);
+}
+
+MLA_API int mla_decode_fp8_timed(const void* q, const void* latent_codes, const void* rope, const int8_t* exps,
+                                 int64_t num_pages, const int32_t* block_table, int max_pages_per_seq,
+                                 const int32_t* seqlens, int batch, int s_q, int h_q, float softmax_scale, int causal,
+                                 void* out, float* lse, void* metadata, void* workspace, size_t workspace_bytes,
+                                 void* stream, void* event_before_decode, void* event_after_decode) {
+  if (!latent_codes || !rope || !exps) return MLA_ERR_ARG;
+  CacheRef cache;
+  cache.codes = latent_codes;
+  cache.rope = rope;
+  cache.exps = exps;
+  return decode_impl(q, cache, num_pages, block_table, max_pages_per_seq, seqlens, batch, s_q, h_q, softmax_scale,
+                     causal, out, lse, metadata, workspace, workspace_bytes, stream, event_before_decode,
+                     event_after_decode, 0);
 }
 
 MLA_API int mla_decode_timed(const void* q, const void* kv_cache, int64_t num_pages, const int32_t* block_table,
@@ -397,7 +480,9 @@ MLA_API int mla_decode_timed(const void* q, const void* kv_cache, int64_t num_pa
                              float softmax_scale, int causal, void* out, float* lse, void* metadata, void* workspace,
                              size_t workspace_bytes, void* stream, void* event_before_decode,
                              void* event_after_decode) {
-  return decode_impl(q, kv_cache, num_pages, block_table, max_pages_per_seq, seqlens, batch, s_q, h_q, softmax_scale,
+  CacheRef cache;
+  cache.kv = kv_cache;
+  return decode_impl(q, cache, num_pages, block_table, max_pages_per_seq, seqlens, batch, s_q, h_q, softmax_scale,
                      causal, out, lse, metadata, workspace, workspace_bytes, stream, event_before_decode,
                      event_after_decode, 0);
 }
@@ -412,7 +497,9 @@ MLA_API int mla_decode_noalloc(const void* q, const void* kv_cache, int64_t num_
   if (workspace_bytes_for(dev.pairs, h_q, s_q) > MLA_NOALLOC_SCRATCH_BYTES) return MLA_ERR_SCRATCH;
   void* scratch = nullptr;
   if ((st = noalloc_scratch(&scratch)) != MLA_OK) return st;
-  return decode_impl(q, kv_cache, num_pages, block_table, max_pages_per_seq, seqlens, batch, s_q, h_q, softmax_scale,
+  CacheRef cache;
+  cache.kv = kv_cache;
+  return decode_impl(q, cache, num_pages, block_table, max_pages_per_seq, seqlens, batch, s_q, h_q, softmax_scale,
                      causal, out, lse, metadata, scratch, MLA_NOALLOC_SCRATCH_BYTES, stream, nullptr, nullptr, 0);
 }
 

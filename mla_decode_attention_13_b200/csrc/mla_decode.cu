@@ -121,9 +121,7 @@ __device__ __forceinline__ void set_error(int32_t* meta, uint32_t bits) {
   atomicOr(&g_mla_sticky_error, bits);
 }
 
-constexpr int kThreads = 384;
 constexpr int kGroup = 4;             // pages per QK group
-constexpr int kKRing = 4;             // key panel slots
 constexpr int kVRing = 2;             // value tiles (and P tiles)
 // PV completion barriers, one per page mod kPvBars.  A parity wait on page k's
 // barrier is only right while the PV of page k - kPvBars is known to be done
@@ -137,51 +135,94 @@ constexpr uint64_t kTimeoutNs = 500ull * 1000ull * 1000ull;
 constexpr uint64_t kDrainNs = 2ull * 1000ull * 1000ull;  // teardown wait for in-flight copies after an abort
 constexpr int kRowsCta = kMTile / 2;  // 64 query rows per CTA
 
+// The two cache formats the kernel is built for.
+//   * bf16: the cache row is 576 bf16 values; key panels and value tiles come
+//     straight from TMA.  12 warps.
+//   * fp8: the 512 latent values of a row are E4M3 codes with one power-of-two
+//     scale 2^e per token, the 64 rope values bf16 ("MLA 和 MHA 的 Kernel 区别",
+//     section "量化友好性": the latent cache tolerates FP8 or INT8, dequantised
+//     as it is loaded).  The codes land by TMA in a staging ring; converter
+//     warps dequantise them into the key panels and build the value tiles
+//     from L2.  The latent products run as f16 MMAs: every E4M3 value times
+//     2^e with e in [-15, 7] is exact in f16, and the latent part of Q is
+//     converted to f16 once per segment; the rope panel stays bf16 in both Q
+//     and the keys.  16 warps (four converter warps).
+struct CfgBf16 {
+  static constexpr bool kFp8 = false;
+  static constexpr int kThreads = 384;
+  static constexpr int kKRing = 4;  // key panel slots
+  static constexpr int kSRing = 0;  // staging slots
+};
+struct CfgFp8 {
+  static constexpr bool kFp8 = true;
+  static constexpr int kThreads = 512;
+  static constexpr int kKRing = 2;
+  static constexpr int kSRing = 4;
+};
+// FP8 kernel registers per thread: 128 at launch (65,536 / 512); the eight
+// softmax warps run with 168, the other eight with 88 (256 x 168 + 256 x 88 =
+// 65,536).
+constexpr uint32_t kRegsLaunch = 128;
+constexpr uint32_t kRegsSoftmax = 168;
+constexpr uint32_t kRegsSide = 88;
+static_assert(256 * kRegsSoftmax + 256 * kRegsSide <= 65536, "register split");
+
 // Shared-memory layout (offsets from a 1024-byte aligned base).  All operand
-// tiles are 128-byte swizzled panels of 64 bf16 columns.
+// tiles are 128-byte swizzled panels of 64 16-bit columns.
 constexpr uint32_t kQPanel = kRowsCta * 128;            // 64 rows x 64 cols
 constexpr uint32_t kQBytes = 9 * kQPanel;               // 64 query rows x 576 cols
 constexpr uint32_t kPagePanel = kPage * 128;            // 64 token rows x 64 cols
 constexpr uint32_t kKSlot = 2 * kPagePanel;             // one panel of a CTA's two pages: 128 token rows
 constexpr uint32_t kVPanel = kPage * 128;               // 64 tokens x 64 cols
 constexpr uint32_t kVTile = 4 * kVPanel;                // 64 tokens x this CTA's 256 value cols
-constexpr uint32_t kPTile = kRowsCta * 128;             // 64 rows x 64 tokens bf16
-constexpr uint32_t kOffQ = 0;
-constexpr uint32_t kOffK = kOffQ + kQBytes;
-constexpr uint32_t kOffV = kOffK + kKRing * kKSlot;
-constexpr uint32_t kOffP = kOffV + kVRing * kVTile;
-constexpr uint32_t kOffX = kOffP + kVRing * kPTile;     // float [2][256] row exchange
-constexpr uint32_t kOffBar = kOffX + 2 * 256 * 4;
+constexpr uint32_t kPTile = kRowsCta * 128;             // 64 rows x 64 tokens, 16-bit
+constexpr uint32_t kSSlot = 8192;                       // fp8 staging: 128 token rows x 64 codes, or 64 x 64 bf16
 
-enum Bar : uint32_t {
-  kBarKFull = 0,                       // [kKRing] (leader) both CTAs' key panel landed (2 arrivals + bytes)
-  kBarKEmpty = kBarKFull + kKRing,     // [kKRing] (both) the panel's QK MMAs are done
-  kBarVFull = kBarKEmpty + kKRing,     // [kVRing] (both, local) this CTA's value tile landed
-  kBarPFull = kBarVFull + kVRing,      // [kVRing] (leader) P written by both CTAs' 2 softmax warps of the page
-  kBarPvDone = kBarPFull + kVRing,     // [kPvBars] (both) PV of page k (mod kPvBars) done: its P and value tiles free
-  kBarSFull = kBarPvDone + kPvBars,    // [2] (both) S buffer written
-  kBarSEmpty = kBarSFull + 2,          // [2] (leader) both CTAs' softmax warps read the S buffer
-  kBarQFull = kBarSEmpty + 2,          // (leader) both CTAs' Q rows landed
-  kBarQEmpty = kBarQFull + 1,          // (both) last QK of the segment done
-  kBarOEmpty = kBarQEmpty + 1,         // (leader) both CTAs' softmax warps read O out
-  kBarFinal = kBarOEmpty + 1,          // (leader) MMA drain at teardown: both issuer threads
-  kBarXch = kBarFinal + 1,             // (both) the 8 softmax warps published row values
-  kBarStageFree = kBarXch + 1,         // (both, local) the epilogue's stores have read their staging
-  kBarResc = kBarStageFree + 1,        // [2] (both, local) the 4 warps of rows 32k..32k+31 rescaled O
-  kNumBars = kBarResc + 2,
+template <class C>
+struct Lay {
+  static constexpr uint32_t kOffQ = 0;
+  static constexpr uint32_t kOffK = kOffQ + kQBytes;
+  static constexpr uint32_t kOffS = kOffK + C::kKRing * kKSlot;
+  static constexpr uint32_t kOffV = kOffS + C::kSRing * kSSlot;
+  static constexpr uint32_t kOffP = kOffV + kVRing * kVTile;
+  static constexpr uint32_t kOffX = kOffP + kVRing * kPTile;  // float [2][256] row exchange
+  static constexpr uint32_t kOffBar = kOffX + 2 * 256 * 4;
+  // Barriers.
+  static constexpr uint32_t kBarKFull = 0;                          // [kKRing] (leader) both CTAs' key panel ready
+  static constexpr uint32_t kBarKEmpty = kBarKFull + C::kKRing;     // [kKRing] (both) the panel's QK MMAs are done
+  static constexpr uint32_t kBarVFull = kBarKEmpty + C::kKRing;     // [kVRing] (both, local) this CTA's value tile ready
+  static constexpr uint32_t kBarPFull = kBarVFull + kVRing;         // [kVRing] (leader) P written by both CTAs
+  static constexpr uint32_t kBarPvDone = kBarPFull + kVRing;        // [kPvBars] (both) PV of page k (mod kPvBars) done
+  static constexpr uint32_t kBarSFull = kBarPvDone + kPvBars;       // [2] (both) S buffer written
+  static constexpr uint32_t kBarSEmpty = kBarSFull + 2;             // [2] (leader) both CTAs' softmax warps read S
+  static constexpr uint32_t kBarQFull = kBarSEmpty + 2;             // bf16: (leader) both CTAs' Q landed; fp8: (local)
+  static constexpr uint32_t kBarQEmpty = kBarQFull + 1;             // (both) last QK of the segment done
+  static constexpr uint32_t kBarOEmpty = kBarQEmpty + 1;            // (leader) both CTAs' softmax warps read O out
+  static constexpr uint32_t kBarFinal = kBarOEmpty + 1;             // (leader) MMA drain at teardown
+  static constexpr uint32_t kBarXch = kBarFinal + 1;                // (both) the 8 softmax warps published row values
+  static constexpr uint32_t kBarStageFree = kBarXch + 1;            // (both, local) the epilogue read its staging
+  static constexpr uint32_t kBarResc = kBarStageFree + 1;           // [2] (both, local) rows 32k.. rescaled O
+  static constexpr uint32_t kBarQReady = kBarResc + 2;              // fp8: (leader) both CTAs' Q converted
+  static constexpr uint32_t kBarStFull = kBarQReady + 1;            // fp8: [kSRing] (local) staging slot landed
+  static constexpr uint32_t kBarStEmpty = kBarStFull + C::kSRing;   // fp8: [kSRing] (local) staging slot converted
+  static constexpr uint32_t kNumBars = kBarStEmpty + C::kSRing;
+  static constexpr uint32_t kOffTmemSlot = kOffBar + 8 * kNumBars;  // u32
+  static constexpr uint32_t kOffAbort = kOffTmemSlot + 4;           // u32
+  // u32 fill counts of the barriers that TMA copies complete on: [kKRing] key
+  // slots (bf16) and [1] Q (the expect_tx posted: bf16 leader, fp8 each CTA),
+  // [kVRing] value slots (bf16), [kSRing] staging slots (fp8); read at
+  // teardown to wait for copies still in flight on abort.
+  static constexpr uint32_t kOffFill = kOffAbort + 4;
+  static constexpr uint32_t kFillQ = C::kKRing;
+  static constexpr uint32_t kFillV = kFillQ + 1;
+  static constexpr uint32_t kFillS = kFillV + kVRing;
+  static constexpr uint32_t kNumFill = kFillS + C::kSRing;
+  static constexpr uint32_t kSmemUsed = kOffFill + 4 * kNumFill;
+  static constexpr uint32_t kSmemBytes = kSmemUsed + 1024;  // slack for aligning the base
+  static_assert(kSmemBytes <= 232448, "shared memory budget");
+  static_assert(kOffK % 1024 == 0 && kOffS % 1024 == 0 && kOffV % 1024 == 0 && kOffP % 1024 == 0,
+                "1024-byte aligned tiles");
 };
-constexpr uint32_t kOffTmemSlot = kOffBar + 8 * kNumBars;  // u32
-constexpr uint32_t kOffAbort = kOffTmemSlot + 4;           // u32
-// u32 fill counts of the barriers that TMA copies complete on: [kKRing] key
-// slots and [1] Q (leader: the expect_tx it posted), [kVRing] value slots
-// (each CTA); read at teardown to wait for copies still in flight on abort.
-constexpr uint32_t kOffFill = kOffAbort + 4;
-constexpr uint32_t kFillQ = kKRing;
-constexpr uint32_t kFillV = kKRing + 1;
-constexpr uint32_t kSmemUsed = kOffFill + 4 * (kKRing + 1 + kVRing);
-constexpr uint32_t kSmemBytes = kSmemUsed + 1024;  // slack for aligning the base
-static_assert(kSmemBytes <= 232448, "shared memory budget");
-static_assert(kOffK % 1024 == 0 && kOffV % 1024 == 0 && kOffP % 1024 == 0, "1024-byte aligned tiles");
 
 // Tensor-memory columns (per CTA; the pair allocation mirrors them).
 constexpr uint32_t kTmemCols = 512;
@@ -190,6 +231,8 @@ constexpr uint32_t kColS = 256;  // 2 x 128
 
 constexpr uint32_t kIdescQK = idesc_bf16_f32(kMTile, kGroup * kPage, false);
 constexpr uint32_t kIdescPV = idesc_bf16_f32(kMTile, 256, true);
+constexpr uint32_t kIdescQK16 = idesc_f16_f32(kMTile, kGroup * kPage, false);
+constexpr uint32_t kIdescPV16 = idesc_f16_f32(kMTile, 256, true);
 
 struct Segment {
   int w, b0, b1, slot;
@@ -197,7 +240,9 @@ struct Segment {
   bool bad;
 };
 
+template <class C>
 struct Ctx {
+  using L = Lay<C>;
   uint32_t base;     // shared::cta address of the aligned base
   uint8_t* gbase;    // generic pointer to the same place
   uint32_t cta;      // rank in the pair; 0 is the leader
@@ -207,15 +252,18 @@ struct Ctx {
   int32_t* meta;
   int s_begin;       // this pair's first segment, read with the pair's record
   Segment first;
-  __device__ uint32_t bar(uint32_t k) const { return base + kOffBar + 8 * k; }
+  __device__ uint32_t bar(uint32_t k) const { return base + L::kOffBar + 8 * k; }
   __device__ uint32_t lead_bar(uint32_t k) const { return lead_bars + 8 * k; }
-  __device__ uint32_t kslot(uint32_t k) const { return base + kOffK + k * kKSlot; }
-  __device__ uint32_t vtile(uint32_t k) const { return base + kOffV + k * kVTile; }
-  __device__ uint32_t ptile(uint32_t k) const { return base + kOffP + k * kPTile; }
-  __device__ volatile uint32_t* fill() const { return reinterpret_cast<volatile uint32_t*>(gbase + kOffFill); }
+  __device__ uint32_t kslot(uint32_t k) const { return base + L::kOffK + k * kKSlot; }
+  __device__ uint32_t stage(uint32_t k) const { return base + L::kOffS + k * kSSlot; }
+  __device__ uint32_t vtile(uint32_t k) const { return base + L::kOffV + k * kVTile; }
+  __device__ uint32_t ptile(uint32_t k) const { return base + L::kOffP + k * kPTile; }
+  __device__ volatile uint32_t* fill() const { return reinterpret_cast<volatile uint32_t*>(gbase + L::kOffFill); }
 };
 
-__device__ void raise_abort(const Ctx& c, uint32_t err_bits) {
+template <class C>
+__device__ void raise_abort(const Ctx<C>& c, uint32_t err_bits) {
+  using L = Lay<C>;
   if (err_bits) set_error(c.meta, err_bits);
   *c.abort_flag = 1u;
   st_cluster_u32(c.peer_abort, 1u);
@@ -223,7 +271,9 @@ __device__ void raise_abort(const Ctx& c, uint32_t err_bits) {
 
 // Bounded wait on an mbarrier phase.  Returns false when the kernel is
 // aborting (this wait timed out, or another role or the peer CTA gave up).
-__device__ bool wait_bar(const Ctx& c, uint32_t bar, uint32_t parity) {
+template <class C>
+__device__ bool wait_bar(const Ctx<C>& c, uint32_t bar, uint32_t parity) {
+  using L = Lay<C>;
   uint32_t spins = 0;
   uint64_t t0 = 0;
   while (true) {
@@ -232,7 +282,7 @@ __device__ bool wait_bar(const Ctx& c, uint32_t bar, uint32_t parity) {
       if (*c.abort_flag) {
 #ifdef MLA_DECODE_TRACE
         g_mla_stuck[blockIdx.x][threadIdx.x >> 5] =
-            (1ull << 32) | (static_cast<unsigned long long>((bar - c.base - kOffBar) / 8) << 8) | parity;
+            (1ull << 32) | (static_cast<unsigned long long>((bar - c.base - L::kOffBar) / 8) << 8) | parity;
 #endif
         return false;
       }
@@ -242,7 +292,7 @@ __device__ bool wait_bar(const Ctx& c, uint32_t bar, uint32_t parity) {
       } else if (now - t0 > kTimeoutNs) {
 #ifdef MLA_DECODE_TRACE
         if (atomicCAS(&g_mla_abort[0], 0ull, 1ull) == 0ull) {
-          g_mla_abort[1] = (bar - c.base - kOffBar) / 8;
+          g_mla_abort[1] = (bar - c.base - L::kOffBar) / 8;
           g_mla_abort[2] = parity;
           g_mla_abort[3] = threadIdx.x;
           g_mla_abort[4] = blockIdx.x;
@@ -259,7 +309,9 @@ __device__ bool wait_bar(const Ctx& c, uint32_t bar, uint32_t parity) {
 // Arrive on one of the leader's barriers (locally in the leader, remotely from
 // the other CTA).  The caller's warp has written what the arrival publishes
 // (shared memory of its own CTA, or TMEM reads that completed) and synced.
-__device__ __forceinline__ void arrive_leader(const Ctx& c, uint32_t k) {
+template <class C>
+__device__ __forceinline__ void arrive_leader(const Ctx<C>& c, uint32_t k) {
+  using L = Lay<C>;
   if (c.cta == 0) {
     mbar_arrive(c.bar(k));
   } else {
@@ -292,7 +344,8 @@ __device__ __forceinline__ Segment make_segment(const DecodeParams& p, int4 a, i
 }
 
 // Segment s of this pair: the first one came with the pair's record.
-__device__ __forceinline__ Segment load_segment(const DecodeParams& p, const Ctx& c, int s) {
+template <class C>
+__device__ __forceinline__ Segment load_segment(const DecodeParams& p, const Ctx<C>& c, int s) {
   if (s == c.s_begin) return c.first;
   const MetaLayout lo = meta_layout(p.batch, p.h_q, p.s_q);
   const int32_t* rec = p.meta + lo.segs + kSegWords * s;
@@ -301,8 +354,10 @@ __device__ __forceinline__ Segment load_segment(const DecodeParams& p, const Ctx
   return make_segment(p, a, L);
 }
 
-__device__ __forceinline__ int load_page(const DecodeParams& p, const Ctx& c, const int32_t* table, int blk,
+template <class C>
+__device__ __forceinline__ int load_page(const DecodeParams& p, const Ctx<C>& c, const int32_t* table, int blk,
                                          int end) {
+  using L = Lay<C>;
   if (blk >= end) return 0;
   int page = table[blk];
   if (page < 0 || page >= p.num_pages) {
@@ -329,9 +384,10 @@ struct NoSegmentHook {
   __device__ bool operator()(const Segment&) const { return true; }
 };
 
-template <typename Fn, typename SegFn = NoSegmentHook>
-__device__ __forceinline__ void walk_groups(const DecodeParams& p, const Ctx& c, int s_begin, int s_end, Fn&& fn,
+template <class C, typename Fn, typename SegFn = NoSegmentHook>
+__device__ __forceinline__ void walk_groups(const DecodeParams& p, const Ctx<C>& c, int s_begin, int s_end, Fn&& fn,
                                             SegFn&& on_segment = SegFn()) {
+  using L = Lay<C>;
   static_assert(32 % kGroup == 0, "groups never straddle a chunk of page ids");
   const int lane = threadIdx.x & 31;
   for (int s = s_begin; s < s_end; ++s) {
@@ -361,27 +417,72 @@ __device__ __forceinline__ void walk_groups(const DecodeParams& p, const Ctx& c,
 // Warp 0: each segment's Q rows of this CTA, then this CTA's two pages of
 // the group (pages 2c and 2c + 1, those that exist), panel by panel, into the
 // key ring (bytes complete on the leader's barriers).
-__device__ void producer_k(const DecodeParams& p, const Ctx& c, int s_begin, int s_end) {
+template <class C>
+__device__ void producer_k(const DecodeParams& p, const Ctx<C>& c, int s_begin, int s_end) {
+  using L = Lay<C>;
   const int lane = threadIdx.x & 31;
   uint32_t gi = 0, seg_it = 0, ks = 0;  // groups, segments started, key panels loaded
   // The segment's Q rows first, before its page ids are even read.
   auto load_q = [&](const Segment& sg) -> bool {
     int good = 1;
     if (lane == 0) {
-      good = seg_it == 0 || wait_bar(c, c.bar(kBarQEmpty), (seg_it - 1) & 1);
+      good = seg_it == 0 || wait_bar(c, c.bar(L::kBarQEmpty), (seg_it - 1) & 1);
       if (good) {
         MLA_TRACE(14, seg_it);
-        if (c.cta == 0) {
-          mbar_arrive_expect_tx(c.bar(kBarQFull), 2 * kQBytes);
-          c.fill()[kFillQ] += 1;
-        }
         const int y = sg.i * p.R + sg.mt * kMTile + c.cta * kRowsCta;
-        tma_load_3d_pair(c.base + kOffQ, &p.tm_q, c.lead_bar(kBarQFull), 0, y, 0);
+        if constexpr (C::kFp8) {
+          // Each CTA converts its own rows: a local copy on its own barrier.
+          mbar_arrive_expect_tx(c.bar(L::kBarQFull), kQBytes);
+          c.fill()[L::kFillQ] += 1;
+          tma_load_3d(c.base + L::kOffQ, &p.tm_q, c.bar(L::kBarQFull), 0, y, 0);
+        } else {
+          if (c.cta == 0) {
+            mbar_arrive_expect_tx(c.bar(L::kBarQFull), 2 * kQBytes);
+            c.fill()[L::kFillQ] += 1;
+          }
+          tma_load_3d_pair(c.base + L::kOffQ, &p.tm_q, c.lead_bar(L::kBarQFull), 0, y, 0);
+        }
       }
     }
     ++seg_it;
     return __shfl_sync(0xffffffffu, good, 0) != 0;
   };
+  if constexpr (C::kFp8) {
+    // FP8 cache: this CTA's two pages of the group (2c and 2c + 1, those that
+    // exist) go to the staging ring, ten 8 KB fills per group: the latent
+    // codes of 64 columns of both pages (fills 0-7, one box per page, lanes 0
+    // and 1 together), then the bf16 rope of each page (fills 8 and 9).  A
+    // fill of a missing page posts no bytes but still completes, so that the
+    // converters see every fill of every group.
+    uint32_t sf = 0;
+    walk_groups(p, c, s_begin, s_end, [&](const Segment&, const Group& gr) -> bool {
+      const int my_np = min(max(gr.np - 2 * static_cast<int>(c.cta), 0), 2);
+      const int page_a = gr.page[2 * c.cta], page_b = gr.page[2 * c.cta + 1];
+      int good = 1;
+      for (int f = 0; f < 10; ++f, ++sf) {
+        const uint32_t slot = sf % C::kSRing;
+        if (lane == 0 && sf >= C::kSRing)
+          good = wait_bar(c, c.bar(L::kBarStEmpty + slot), ((sf / C::kSRing) - 1) & 1);
+        good = __shfl_sync(0xffffffffu, good, 0);
+        if (!good) break;
+        const uint32_t bytes = f < 8 ? my_np * (kSSlot / 2) : (f - 8 < my_np ? kSSlot : 0u);
+        if (lane == 0) {
+          mbar_arrive_expect_tx(c.bar(L::kBarStFull + slot), bytes);
+          c.fill()[L::kFillS + slot] += 1;
+        }
+        __syncwarp();
+        if (f < 8) {
+          if (lane < my_np)
+            tma_load_2d(c.stage(slot) + lane * (kSSlot / 2), &p.tm_codes, c.bar(L::kBarStFull + slot), 64 * f,
+                        (lane == 0 ? page_a : page_b) * kPage);
+        } else if (lane == 0 && f - 8 < my_np) {
+          tma_load_2d(c.stage(slot), &p.tm_rope, c.bar(L::kBarStFull + slot), 0, (f == 8 ? page_a : page_b) * kPage);
+        }
+      }
+      return good != 0;
+    }, load_q);
+    return;
+  }
   walk_groups(p, c, s_begin, s_end, [&](const Segment& sg, const Group& gr) -> bool {
     if (lane == 0) MLA_TRACE(0, gi);
     // This CTA's two pages of the group; lanes 0 and 1 issue their boxes in
@@ -391,27 +492,27 @@ __device__ void producer_k(const DecodeParams& p, const Ctx& c, int s_begin, int
     const bool my_load = lane < 2 && 2 * static_cast<int>(c.cta) + lane < gr.np;
     int good = 1;
     for (int pn = 0; pn < 9; ++pn, ++ks) {
-      const uint32_t slot = ks % kKRing;
-      if (lane == 0 && ks >= kKRing) good = wait_bar(c, c.bar(kBarKEmpty + slot), ((ks / kKRing) - 1) & 1);
+      const uint32_t slot = ks % C::kKRing;
+      if (lane == 0 && ks >= C::kKRing) good = wait_bar(c, c.bar(L::kBarKEmpty + slot), ((ks / C::kKRing) - 1) & 1);
       good = __shfl_sync(0xffffffffu, good, 0);
       if (!good) break;
       if (lane == 0) {
         MLA_TRACE(10, ks);
         MLA_STEP(ks);
         if (c.cta == 0) {
-          mbar_arrive_expect_tx(c.bar(kBarKFull + slot), gr.np * kPagePanel);
+          mbar_arrive_expect_tx(c.bar(L::kBarKFull + slot), gr.np * kPagePanel);
           c.fill()[slot] += 1;
         }
       }
       __syncwarp();
       if (my_load)
-        tma_load_3d_pair(c.kslot(slot) + lane * kPagePanel, &p.tm_k, c.lead_bar(kBarKFull + slot), 0,
+        tma_load_3d_pair(c.kslot(slot) + lane * kPagePanel, &p.tm_k, c.lead_bar(L::kBarKFull + slot), 0,
                          my_page * kPage, pn);
       if (lane == 0) MLA_TRACE(15, ks);
       // The other CTA also arrives, even when it has no page in the group:
       // otherwise the slot could fill and drain without it, and its parity
       // wait on the slot's empty barrier would fall two phases behind.
-      if (lane == 0 && c.cta != 0) mbar_arrive_remote(c.lead_bar(kBarKFull + slot));
+      if (lane == 0 && c.cta != 0) mbar_arrive_remote(c.lead_bar(L::kBarKFull + slot));
     }
     ++gi;
     return good != 0;
@@ -422,7 +523,9 @@ __device__ void producer_k(const DecodeParams& p, const Ctx& c, int s_begin, int
 // columns) into the value ring once PV two pages back has released the slot;
 // bytes complete on this CTA's own barrier (the softmax warps wait for it
 // before releasing P, so PV never runs ahead of it).
-__device__ void producer_v(const DecodeParams& p, const Ctx& c, int s_begin, int s_end) {
+template <class C>
+__device__ void producer_v(const DecodeParams& p, const Ctx<C>& c, int s_begin, int s_end) {
+  using L = Lay<C>;
   const int lane = threadIdx.x & 31;
   uint32_t ps = 0, seg_it = 0;  // pages, segments
   walk_groups(p, c, s_begin, s_end, [&](const Segment&, const Group& gr) -> bool {
@@ -430,19 +533,19 @@ __device__ void producer_v(const DecodeParams& p, const Ctx& c, int s_begin, int
     if (lane == 0) {
       // The epilogue of the previous segment stages its output in the value
       // ring: a new segment's first tile waits until those stores have read it.
-      if (gr.first && seg_it > 0) good = wait_bar(c, c.bar(kBarStageFree), (seg_it - 1) & 1);
+      if (gr.first && seg_it > 0) good = wait_bar(c, c.bar(L::kBarStageFree), (seg_it - 1) & 1);
       for (int q = 0; q < gr.np && good; ++q, ++ps) {
         const uint32_t slot = ps % kVRing;
         if (ps >= kVRing) {
           const uint32_t k = ps - kVRing;  // the tile's previous page: its PV must be done
-          good = wait_bar(c, c.bar(kBarPvDone + k % kPvBars), (k / kPvBars) & 1);
+          good = wait_bar(c, c.bar(L::kBarPvDone + k % kPvBars), (k / kPvBars) & 1);
         }
         if (good) {
           MLA_TRACE(3, ps);
           MLA_STEP(ps);
-          const uint32_t bar = c.bar(kBarVFull + slot);
+          const uint32_t bar = c.bar(L::kBarVFull + slot);
           mbar_arrive_expect_tx(bar, kVTile);
-          c.fill()[kFillV + slot] += 1;
+          c.fill()[L::kFillV + slot] += 1;
           tma_load_4d(c.vtile(slot), &p.tm_v, bar, 0, gr.page[q] * kPage, 2 * static_cast<int>(c.cta), 0);
         }
       }
@@ -452,23 +555,234 @@ __device__ void producer_v(const DecodeParams& p, const Ctx& c, int s_begin, int
   });
 }
 
+// ------------------------------------------------ converters (FP8 cache) --
+// f16 bits of 2^e, exact for e in [-24, 15] (subnormal below -14); e is
+// clamped to that range (exponents outside [-15, 7] are flagged by the key
+// converter, as E4M3 values times 2^e are exact in f16 only there).
+__device__ __forceinline__ uint32_t f16_pow2(int e) {
+  e = max(-24, min(15, e));
+  return e >= -14 ? static_cast<uint32_t>(e + 15) << 10 : 1u << (e + 24);
+}
+
+// 16 E4M3 codes (a 16-byte chunk, first code in the lowest byte) times the
+// f16x2 scale, as 16 f16 values in memory order (two 16-byte chunks).
+__device__ __forceinline__ void dequant16(const uint4& v, uint32_t scale2, uint4& lo, uint4& hi) {
+  const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+  uint32_t r[8];
+#pragma unroll
+  for (int k = 0; k < 4; ++k) {
+    r[2 * k] = mul_f16x2(e4m3x2_to_f16x2(static_cast<uint16_t>(w[k] & 0xFFFFu)), scale2);
+    r[2 * k + 1] = mul_f16x2(e4m3x2_to_f16x2(static_cast<uint16_t>(w[k] >> 16)), scale2);
+  }
+  lo = make_uint4(r[0], r[1], r[2], r[3]);
+  hi = make_uint4(r[4], r[5], r[6], r[7]);
+}
+
+// Two bf16 values (low half first) to f16, rounded to nearest.
+__device__ __forceinline__ uint32_t bf16x2_to_f16x2(uint32_t w) {
+  return f32x2_to_f16x2(__uint_as_float(w & 0xFFFF0000u), __uint_as_float(w << 16));
+}
+
+// Warps 12-13 (64 threads), FP8 cache only.
+//   * At each segment start: this CTA's Q rows to f16 in place (the latent
+//     panels 0-7; the rope panel stays bf16), then one arrival per warp on the
+//     leader's Q barrier.  A query value past the f16 range is flagged.
+//   * Per group, the nine key panels in order: a latent panel's staging slot
+//     (64 codes of 128 token rows: this CTA's two pages) is dequantised with
+//     each token's 2^e into a key slot (f16, 128B-swizzled, the layout of the
+//     bf16 cache's key panels); the rope panel is two staging slots (one page
+//     each, already bf16 and swizzled) copied into one key slot.  Each key
+//     slot then gets one arrival per warp on the leader's full barrier.
+template <class C>
+__device__ void key_converter(const DecodeParams& p, const Ctx<C>& c, int s_begin, int s_end) {
+  using L = Lay<C>;
+  const int kt = static_cast<int>(threadIdx.x) - 12 * 32;  // 0-63
+  const int lane = threadIdx.x & 31;
+  uint32_t seg_it = 0, sf = 0, kf = 0;  // segments, staging fills, key panels
+  bool out_of_range = false;
+  auto conv_q = [&](const Segment&) -> bool {
+    if (!wait_bar(c, c.bar(L::kBarQFull), seg_it & 1)) return false;
+    ++seg_it;
+    uint4* q = reinterpret_cast<uint4*>(c.gbase + L::kOffQ);
+    uint32_t inf_seen = 0;  // bit 15 of a half: an f16 result with the all-ones exponent
+    for (int k = kt; k < static_cast<int>(8 * kQPanel / 16); k += 64) {
+      uint4 v = q[k];
+      v.x = bf16x2_to_f16x2(v.x);
+      v.y = bf16x2_to_f16x2(v.y);
+      v.z = bf16x2_to_f16x2(v.z);
+      v.w = bf16x2_to_f16x2(v.w);
+      inf_seen |= ((v.x & 0x7C007C00u) + 0x04000400u) | ((v.y & 0x7C007C00u) + 0x04000400u) |
+                  ((v.z & 0x7C007C00u) + 0x04000400u) | ((v.w & 0x7C007C00u) + 0x04000400u);
+      q[k] = v;
+    }
+    if (inf_seen & 0x80008000u) out_of_range = true;
+    fence_proxy_async_smem();
+    __syncwarp();
+    if (lane == 0) arrive_leader(c, L::kBarQReady);
+    return true;
+  };
+  walk_groups(p, c, s_begin, s_end, [&](const Segment& sg, const Group& gr) -> bool {
+    const int my_np = min(max(gr.np - 2 * static_cast<int>(c.cta), 0), 2);
+    // Exponents of this CTA's two pages: lane l holds those of rows 4l to
+    // 4l + 3 (rows 0-63: page 2c, rows 64-127: page 2c + 1).
+    const int half = lane >> 4;
+    uint32_t ew = 0;
+    if (half < my_np) {
+      const int page = gr.page[2 * c.cta + half];
+      ew = *reinterpret_cast<const uint32_t*>(p.exps + static_cast<long long>(page) * kPage + 4 * (lane & 15));
+      const int tok0 = (gr.blk + 2 * static_cast<int>(c.cta) + half) * kPage + 4 * (lane & 15);
+#pragma unroll
+      for (int b = 0; b < 4; ++b) {
+        const int e = static_cast<int8_t>((ew >> (8 * b)) & 0xFFu);
+        if (tok0 + b < sg.L && (e < -15 || e > 7)) out_of_range = true;
+      }
+    }
+    for (int pn = 0; pn < 9; ++pn, ++kf) {
+      const uint32_t ks = kf % C::kKRing;
+      if (kf >= C::kKRing && !wait_bar(c, c.bar(L::kBarKEmpty + ks), ((kf / C::kKRing) - 1) & 1)) return false;
+      uint8_t* dst = c.gbase + L::kOffK + ks * kKSlot;
+      if (pn < 8) {
+        const uint32_t st = sf % C::kSRing;
+        if (!wait_bar(c, c.bar(L::kBarStFull + st), (sf / C::kSRing) & 1)) return false;
+        ++sf;
+        // 16-byte chunk kt + 64 j of the slot: row kt / 4 + 16 j (64 bytes of
+        // codes per row), codes 16 (kt % 4) to +15 -> f16 chunks 2 (kt % 4)
+        // and + 1 of the row, swizzled by row % 8 = (kt / 4) % 8.
+        const int row0 = kt >> 2, c4 = kt & 3;
+        const uint8_t* src = c.gbase + L::kOffS + st * kSSlot + 16 * kt;
+        uint8_t* drow = dst + row0 * 128;
+        const uint32_t off_lo = ((2 * c4) ^ (row0 & 7)) << 4, off_hi = ((2 * c4 + 1) ^ (row0 & 7)) << 4;
+#pragma unroll 4
+        for (int j = 0; j < 8; ++j) {
+          const uint4 v = *reinterpret_cast<const uint4*>(src + 1024 * j);
+          const int row = row0 + 16 * j;
+          const int e = static_cast<int8_t>((__shfl_sync(0xffffffffu, ew, row >> 2) >> (8 * (row & 3))) & 0xFFu);
+          const uint32_t sc = f16_pow2(e);
+          uint4 lo, hi;
+          dequant16(v, sc | (sc << 16), lo, hi);
+          *reinterpret_cast<uint4*>(drow + 2048 * j + off_lo) = lo;
+          *reinterpret_cast<uint4*>(drow + 2048 * j + off_hi) = hi;
+        }
+        __syncwarp();
+        if (lane == 0) mbar_arrive(c.bar(L::kBarStEmpty + st));
+      } else {
+        for (int h = 0; h < 2; ++h, ++sf) {
+          const uint32_t st = sf % C::kSRing;
+          if (!wait_bar(c, c.bar(L::kBarStFull + st), (sf / C::kSRing) & 1)) return false;
+          const uint4* src = reinterpret_cast<const uint4*>(c.gbase + L::kOffS + st * kSSlot);
+          uint4* d = reinterpret_cast<uint4*>(dst + h * kSSlot);
+#pragma unroll
+          for (int k = kt; k < static_cast<int>(kSSlot / 16); k += 64) d[k] = src[k];
+          __syncwarp();
+          if (lane == 0) mbar_arrive(c.bar(L::kBarStEmpty + st));
+        }
+      }
+      fence_proxy_async_smem();
+      __syncwarp();
+      if (lane == 0) arrive_leader(c, L::kBarKFull + ks);
+    }
+    return true;
+  }, conv_q);
+  if (out_of_range) set_error(c.meta, MLA_DEVERR_FP8_RANGE);
+}
+
+// Warps 14-15 (64 threads), FP8 cache only: this CTA's value tile of every
+// page (its 256 value columns [256h + 128c, +128), h = 0, 1, of all 64
+// tokens, f16, the layout of the bf16 cache's value tiles), built from the
+// page's codes in L2 (the pair has just staged the page) and each token's
+// 2^e, once PV two pages back has released the slot.  The loads are issued
+// before that wait.
+template <class C>
+__device__ void value_converter(const DecodeParams& p, const Ctx<C>& c, int s_begin, int s_end) {
+  using L = Lay<C>;
+  const int vt = static_cast<int>(threadIdx.x) - 14 * 32;  // 0-63
+  const int lane = threadIdx.x & 31;
+  uint32_t ps = 0, seg_it = 0;  // pages, segments
+  walk_groups(p, c, s_begin, s_end, [&](const Segment&, const Group& gr) -> bool {
+    for (int q = 0; q < gr.np; ++q, ++ps) {
+      const uint32_t slot = ps % kVRing;
+      const long long row0 = static_cast<long long>(gr.page[q]) * kPage;
+      // 16-byte chunk vt + 64 j (j = 0-15) of the tile: token tok0 + 4 j
+      // (tok0 = vt / 16), half h = (vt / 8) % 2, codes 16 i8 to +15 (i8 =
+      // vt % 8) of the half's 128 columns; only the token moves with j.
+      const int tok0 = vt >> 4, h = (vt >> 3) & 1, i8 = vt & 7;
+      const uint8_t* src = p.codes + (row0 + tok0) * kDv + 256 * h + 128 * static_cast<int>(c.cta) + 16 * i8;
+      // The first half of the tile's codes is loaded before the wait, the
+      // second while the first is converted.
+      uint4 v[8];
+#pragma unroll
+      for (int j = 0; j < 8; ++j) v[j] = ld_nc_v4(src + 4 * kDv * j);
+      const uint32_t ew = *reinterpret_cast<const uint16_t*>(p.exps + row0 + 2 * lane);  // tokens 2 lane, + 1
+      int good = 1;
+      if (lane == 0) {
+        // The previous segment's epilogue stages its output in the value ring.
+        if (gr.first && q == 0 && seg_it > 0) good = wait_bar(c, c.bar(L::kBarStageFree), (seg_it - 1) & 1);
+        if (good && ps >= kVRing) {
+          const uint32_t k = ps - kVRing;  // the tile's previous page: its PV must be done
+          good = wait_bar(c, c.bar(L::kBarPvDone + k % kPvBars), (k / kPvBars) & 1);
+        }
+      }
+      if (!__shfl_sync(0xffffffffu, good, 0)) return false;
+      // panel [h][i8 / 4]; f16 chunks 2 (i8 % 4) and + 1 of the token's
+      // 128-byte row, swizzled by tok % 8 = (tok0 % 8) ^ (4 (j % 2)).
+      uint8_t* drow = c.gbase + L::kOffV + slot * kVTile + (2 * h + (i8 >> 2)) * kVPanel + tok0 * 128;
+      const uint32_t ch = 2 * (i8 & 3);
+#pragma unroll
+      for (int half = 0; half < 2; ++half) {
+        uint4 w[8];
+        if (half == 0) {
+#pragma unroll
+          for (int j = 0; j < 8; ++j) w[j] = ld_nc_v4(src + 4 * kDv * (8 + j));
+        }
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {
+          const int jj = 8 * half + j;
+          const int tok = tok0 + 4 * jj;
+          const int e = static_cast<int8_t>((__shfl_sync(0xffffffffu, ew, tok >> 1) >> (8 * (tok & 1))) & 0xFFu);
+          const uint32_t sc = f16_pow2(e);
+          uint4 lo, hi;
+          dequant16(v[j], sc | (sc << 16), lo, hi);
+          const uint32_t sw = (tok0 & 7) ^ (4 * (j & 1));
+          *reinterpret_cast<uint4*>(drow + 512 * jj + ((ch ^ sw) << 4)) = lo;
+          *reinterpret_cast<uint4*>(drow + 512 * jj + (((ch + 1) ^ sw) << 4)) = hi;
+        }
+        if (half == 0) {
+#pragma unroll
+          for (int j = 0; j < 8; ++j) v[j] = w[j];
+        }
+      }
+      fence_proxy_async_smem();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(c.bar(L::kBarVFull + slot));
+    }
+    if (gr.first) ++seg_it;
+    return true;
+  });
+}
+
 // ------------------------------------------------------ MMA (leader only) --
 // One key panel of QK^T: four K = 16 steps over its 64 columns.
-__device__ __forceinline__ void issue_qk_panel(const Ctx& c, uint32_t tmem, uint32_t slot, int pn, uint32_t sb) {
-  const uint32_t q = c.base + kOffQ + pn * kQPanel;
+template <class C>
+__device__ __forceinline__ void issue_qk_panel(const Ctx<C>& c, uint32_t tmem, uint32_t slot, int pn, uint32_t sb) {
+  using L = Lay<C>;
+  const uint32_t q = c.base + L::kOffQ + pn * kQPanel;
   const uint32_t k = c.kslot(slot);
+  // FP8 cache: the latent panels (0-7) are f16 on both sides, the rope panel bf16.
+  const uint32_t idesc = (C::kFp8 && pn < 8) ? kIdescQK16 : kIdescQK;
 #pragma unroll
   for (int s = 0; s < 4; ++s) {
     const uint64_t a = smem_desc(q + s * 32, 16, 1024, kSwizzle128B);
     const uint64_t b = smem_desc(k + s * 32, 16, 1024, kSwizzle128B);
-    umma_ss_pair(tmem + kColS + 128 * sb, a, b, kIdescQK, (pn > 0 || s > 0) ? 1u : 0u);
+    umma_ss_pair(tmem + kColS + 128 * sb, a, b, idesc, (pn > 0 || s > 0) ? 1u : 0u);
   }
 }
 
 // O (+)= P V for one page.  For the N = 256 half h, each CTA's 128 value
 // columns are two adjacent panels (leading byte offset = one panel); K step k
 // takes tokens [16k, 16k + 16).
-__device__ __forceinline__ void issue_pv_page(const Ctx& c, uint32_t tmem, uint32_t slot, bool first) {
+template <class C>
+__device__ __forceinline__ void issue_pv_page(const Ctx<C>& c, uint32_t tmem, uint32_t slot, bool first) {
+  using L = Lay<C>;
   const uint32_t pt = c.ptile(slot);
   const uint32_t vt = c.vtile(slot);
 #pragma unroll
@@ -477,7 +791,7 @@ __device__ __forceinline__ void issue_pv_page(const Ctx& c, uint32_t tmem, uint3
     for (int k = 0; k < 4; ++k) {
       const uint64_t a = smem_desc(pt + k * 32, 16, 1024, kSwizzle128B);
       const uint64_t b = smem_desc(vt + h * 2 * kVPanel + k * 16 * 128, kVPanel, 1024, kSwizzle128B);
-      umma_ss_pair(tmem + kColO + 128 * h, a, b, kIdescPV, (!first || k > 0) ? 1u : 0u);
+      umma_ss_pair(tmem + kColO + 128 * h, a, b, C::kFp8 ? kIdescPV16 : kIdescPV, (!first || k > 0) ? 1u : 0u);
     }
   }
 }
@@ -491,35 +805,40 @@ __device__ __forceinline__ void issue_pv_page(const Ctx& c, uint32_t tmem, uint3
 //   * PV (warp 3): per page, in order, once both CTAs have written its P
 //     (which they do after reading S, so QK of its group is complete); the
 //     first page of a segment also waits until O has been read out.
-__device__ void qk_issuer(const DecodeParams& p, const Ctx& c, uint32_t tmem, int s_begin, int s_end) {
+template <class C>
+__device__ void qk_issuer(const DecodeParams& p, const Ctx<C>& c, uint32_t tmem, int s_begin, int s_end) {
+  using L = Lay<C>;
   uint32_t gi = 0, ks = 0, seg_it = 0;  // groups, key panels consumed, segments
   const uint16_t both = 0x3;
   for (int s = s_begin; s < s_end; ++s) {
     const Segment sg = load_segment(p, c, s);
     if (sg.bad) continue;
     const int ng = ceil_div(sg.b1 - sg.b0, kGroup);
-    if (!wait_bar(c, c.bar(kBarQFull), seg_it & 1)) return;
+    // FP8 cache: both CTAs' Q rows converted; bf16: both CTAs' Q rows landed.
+    if (!wait_bar(c, c.bar(C::kFp8 ? L::kBarQReady : L::kBarQFull), seg_it & 1)) return;
     for (int gq = 0; gq < ng; ++gq, ++gi) {
       const uint32_t sb = gi & 1;
-      if (gi >= 2 && !wait_bar(c, c.bar(kBarSEmpty + sb), ((gi - 2) >> 1) & 1)) return;
+      if (gi >= 2 && !wait_bar(c, c.bar(L::kBarSEmpty + sb), ((gi - 2) >> 1) & 1)) return;
       MLA_TRACE(1, gi);
       for (int pn = 0; pn < 9; ++pn, ++ks) {
-        const uint32_t slot = ks % kKRing;
-        if (!wait_bar(c, c.bar(kBarKFull + slot), (ks / kKRing) & 1)) return;
+        const uint32_t slot = ks % C::kKRing;
+        if (!wait_bar(c, c.bar(L::kBarKFull + slot), (ks / C::kKRing) & 1)) return;
         MLA_TRACE(9, ks);
         MLA_STEP(ks);
         tc_fence_after();
         issue_qk_panel(c, tmem, slot, pn, sb);
-        umma_commit_pair(c.bar(kBarKEmpty + slot), both);
+        umma_commit_pair(c.bar(L::kBarKEmpty + slot), both);
       }
-      umma_commit_pair(c.bar(kBarSFull + sb), both);
+      umma_commit_pair(c.bar(L::kBarSFull + sb), both);
     }
-    umma_commit_pair(c.bar(kBarQEmpty), both);  // Q free once the segment's last QK is done
+    umma_commit_pair(c.bar(L::kBarQEmpty), both);  // Q free once the segment's last QK is done
     ++seg_it;
   }
 }
 
-__device__ void pv_issuer(const DecodeParams& p, const Ctx& c, uint32_t tmem, int s_begin, int s_end) {
+template <class C>
+__device__ void pv_issuer(const DecodeParams& p, const Ctx<C>& c, uint32_t tmem, int s_begin, int s_end) {
+  using L = Lay<C>;
   uint32_t pg = 0, seg_it = 0;  // pages, segments
   const uint16_t both = 0x3;
   for (int s = s_begin; s < s_end; ++s) {
@@ -528,13 +847,13 @@ __device__ void pv_issuer(const DecodeParams& p, const Ctx& c, uint32_t tmem, in
     const int n = sg.b1 - sg.b0;
     for (int jp = 0; jp < n; ++jp, ++pg) {
       const uint32_t slot = pg % kVRing;
-      if (!wait_bar(c, c.bar(kBarPFull + slot), (pg / kVRing) & 1)) return;
-      if (jp == 0 && seg_it > 0 && !wait_bar(c, c.bar(kBarOEmpty), (seg_it - 1) & 1)) return;
+      if (!wait_bar(c, c.bar(L::kBarPFull + slot), (pg / kVRing) & 1)) return;
+      if (jp == 0 && seg_it > 0 && !wait_bar(c, c.bar(L::kBarOEmpty), (seg_it - 1) & 1)) return;
       MLA_TRACE(2, pg);
       MLA_STEP(pg);
       tc_fence_after();
       issue_pv_page(c, tmem, slot, jp == 0);
-      umma_commit_pair(c.bar(kBarPvDone + pg % kPvBars), both);
+      umma_commit_pair(c.bar(L::kBarPvDone + pg % kPvBars), both);
     }
     ++seg_it;
   }
@@ -558,7 +877,9 @@ __device__ __forceinline__ float masked_max(float (&sv)[32], int nvalid) {
 }
 
 // p = 2^(s * sl2 - m) for the first nvalid scores, 0 past them; packs the
-// bf16-rounded weights in pairs and returns their unrounded fp32 sum.
+// weights in pairs, rounded to bf16 (or to f16 for the FP8 cache, whose PV
+// product is f16), and returns their unrounded fp32 sum.
+template <bool kF16>
 __device__ __forceinline__ float exp_pack(const float (&sv)[32], int nvalid, float sl2, float neg_m,
                                           uint32_t (&packed)[16]) {
   float e[16];
@@ -571,8 +892,12 @@ __device__ __forceinline__ float exp_pack(const float (&sv)[32], int nvalid, flo
       b = (2 * k + 1 < nvalid) ? b : 0.0f;
     }
     e[k] = a + b;
-    const __nv_bfloat162 pr = __floats2bfloat162_rn(a, b);
-    packed[k] = *reinterpret_cast<const uint32_t*>(&pr);
+    if constexpr (kF16) {
+      packed[k] = f32x2_to_f16x2(b, a);
+    } else {
+      const __nv_bfloat162 pr = __floats2bfloat162_rn(a, b);
+      packed[k] = *reinterpret_cast<const uint32_t*>(&pr);
+    }
   }
 #pragma unroll
   for (int k = 0; k < 8; ++k) e[k] += e[k + 8];
@@ -581,7 +906,9 @@ __device__ __forceinline__ float exp_pack(const float (&sv)[32], int nvalid, flo
   return (e[0] + e[2]) + (e[1] + e[3]);
 }
 
-__device__ void softmax_epilogue(const DecodeParams& p, const Ctx& c, uint32_t tmem, int s_begin, int s_end) {
+template <class C>
+__device__ void softmax_epilogue(const DecodeParams& p, const Ctx<C>& c, uint32_t tmem, int s_begin, int s_end) {
+  using L = Lay<C>;
   const int r = threadIdx.x - 128;  // 0-255: softmax thread
   const int sp = r >> 7;            // S columns 64 sp .. 64 sp + 63 of each lane
   const int rr = r & 127;           // TMEM lane
@@ -592,7 +919,7 @@ __device__ void softmax_epilogue(const DecodeParams& p, const Ctx& c, uint32_t t
   const uint32_t lane_off = static_cast<uint32_t>(rr & ~31) << 16;
   const uint32_t t_s = tmem + lane_off + kColS + 64 * sp;
   const uint32_t t_o = tmem + lane_off + kColO + 128 * sp;  // this thread's 128 O columns
-  float* xbuf = reinterpret_cast<float*>(c.gbase + kOffX);
+  float* xbuf = reinterpret_cast<float*>(c.gbase + L::kOffX);
   // This thread's 64 weights of a page: row hr of the P tile (128 bytes,
   // 16-byte chunks swizzled by the row).
   const uint32_t prow_off = (hr >> 3) * 1024 + (hr & 7) * 128;
@@ -603,7 +930,7 @@ __device__ void softmax_epilogue(const DecodeParams& p, const Ctx& c, uint32_t t
   // 32 kr + 31 take the same decisions, so they count alike).
   uint32_t gi = 0, ps = 0, x_cnt = 0, n_resc = 0;
   const int kr = (rr >> 5) & 1;
-  auto pv_done = [&](uint32_t k) -> bool { return wait_bar(c, c.bar(kBarPvDone + k % kPvBars), (k / kPvBars) & 1); };
+  auto pv_done = [&](uint32_t k) -> bool { return wait_bar(c, c.bar(L::kBarPvDone + k % kPvBars), (k / kPvBars) & 1); };
   // Publish v for the other three threads of this row (the other half of its
   // tokens, the other page pair) and return the max or the sum of the four;
   // the eight softmax warps meet on an mbarrier (bounded wait).
@@ -611,8 +938,8 @@ __device__ void softmax_epilogue(const DecodeParams& p, const Ctx& c, uint32_t t
     float* buf = xbuf + (x_cnt & 1) * 256;
     buf[r] = v;
     __syncwarp();
-    if (lane == 0) mbar_arrive(c.bar(kBarXch));
-    const bool ok = wait_bar(c, c.bar(kBarXch), x_cnt & 1);
+    if (lane == 0) mbar_arrive(c.bar(L::kBarXch));
+    const bool ok = wait_bar(c, c.bar(L::kBarXch), x_cnt & 1);
     ++x_cnt;
     const float a = buf[r ^ 64], b = buf[r ^ 128], d = buf[r ^ 192];
     *out = sum ? (v + a) + (b + d) : fmaxf(fmaxf(v, a), fmaxf(b, d));
@@ -648,7 +975,7 @@ __device__ void softmax_epilogue(const DecodeParams& p, const Ctx& c, uint32_t t
       const int np = min(kGroup, n - j);
       np_last = np;
       const uint32_t sb = gi & 1;
-      if (!wait_bar(c, c.bar(kBarSFull + sb), (gi >> 1) & 1)) return;
+      if (!wait_bar(c, c.bar(L::kBarSFull + sb), (gi >> 1) & 1)) return;
       if (r == 0) MLA_TRACE(4, gi);
       MLA_STEP((1ull << 40) | (static_cast<unsigned long long>(gi) << 20) | ps);
       tc_fence_after();
@@ -658,7 +985,7 @@ __device__ void softmax_epilogue(const DecodeParams& p, const Ctx& c, uint32_t t
       tmem_wait_ld();
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) arrive_leader(c, kBarSEmpty + sb);  // S buffer read
+      if (lane == 0) arrive_leader(c, L::kBarSEmpty + sb);  // S buffer read
 
       // ---- mask; max over the group's four pages ----
       int nv[2];
@@ -697,7 +1024,7 @@ __device__ void softmax_epilogue(const DecodeParams& p, const Ctx& c, uint32_t t
         tmem_wait_st();
         tc_fence_before();
         __syncwarp();
-        if (lane == 0) mbar_arrive(c.bar(kBarResc + kr));
+        if (lane == 0) mbar_arrive(c.bar(L::kBarResc + kr));
         ++n_resc;
         MLA_STEP((6ull << 40) | n_resc);
       }
@@ -706,14 +1033,15 @@ __device__ void softmax_epilogue(const DecodeParams& p, const Ctx& c, uint32_t t
       if (q < np) {
         const uint32_t pg = ps + q;  // global page index
         uint32_t packed[2][16];
-        lsum = exp_pack(sv[0], nv[0], sl2, neg_m, packed[0]) + exp_pack(sv[1], nv[1], sl2, neg_m, packed[1]);
+        lsum = exp_pack<C::kFp8>(sv[0], nv[0], sl2, neg_m, packed[0]) +
+               exp_pack<C::kFp8>(sv[1], nv[1], sl2, neg_m, packed[1]);
         const uint32_t slot = pg % kVRing;
         // ---- P tile free (PV two pages back) ----
         if (pg >= kVRing && !pv_done(pg - kVRing)) return;
         MLA_STEP((2ull << 40) | pg);
         if (rr == 0) MLA_TRACE(6, pg);
         {
-          uint8_t* prow = c.gbase + kOffP + slot * kPTile + prow_off;
+          uint8_t* prow = c.gbase + L::kOffP + slot * kPTile + prow_off;
 #pragma unroll
           for (int ci = 0; ci < 8; ++ci)
             *reinterpret_cast<uint4*>(prow + ((ci ^ (hr & 7)) << 4)) =
@@ -723,13 +1051,13 @@ __device__ void softmax_epilogue(const DecodeParams& p, const Ctx& c, uint32_t t
         // ---- this CTA's value tile has landed; the last page of a row may
         //      hold garbage (even NaN) past L: zero the value rows there, so
         //      that 0 * garbage cannot reach O ----
-        if (!wait_bar(c, c.bar(kBarVFull + slot), (pg / kVRing) & 1)) return;
+        if (!wait_bar(c, c.bar(L::kBarVFull + slot), (pg / kVRing) & 1)) return;
         MLA_STEP((3ull << 40) | pg);
         if (rr == 0) MLA_TRACE(7, pg);
         if (blk + q == last_page && (sg.L & (kPage - 1))) {
           const int first_bad = sg.L - last_page * kPage;
           const int chunks = (kPage - first_bad) * 4 * 8;  // tokens x panels x 16-byte chunks
-          uint8_t* vt = c.gbase + kOffV + slot * kVTile;
+          uint8_t* vt = c.gbase + L::kOffV + slot * kVTile;
           for (int e2 = hr; e2 < chunks; e2 += kRowsCta) {
             const int tok = first_bad + (e2 >> 5);
             *reinterpret_cast<uint4*>(vt + ((e2 >> 3) & 3) * kVPanel + tok * 128 + (e2 & 7) * 16) =
@@ -738,11 +1066,11 @@ __device__ void softmax_epilogue(const DecodeParams& p, const Ctx& c, uint32_t t
         }
         // The group's first PV adds to O: every warp of these rows must have
         // rescaled its O columns first.
-        if (resc && q == 0 && !wait_bar(c, c.bar(kBarResc + kr), (n_resc - 1) & 1)) return;
+        if (resc && q == 0 && !wait_bar(c, c.bar(L::kBarResc + kr), (n_resc - 1) & 1)) return;
         fence_proxy_async_smem();
         tc_fence_before();
         __syncwarp();
-        if (lane == 0) arrive_leader(c, kBarPFull + slot);
+        if (lane == 0) arrive_leader(c, L::kBarPFull + slot);
         MLA_STEP((4ull << 40) | pg);
         if (rr == 0) MLA_TRACE(8, pg);
       }
@@ -772,7 +1100,7 @@ __device__ void softmax_epilogue(const DecodeParams& p, const Ctx& c, uint32_t t
     // tile_rows).  (Measured: TMA stores of 4 KB boxes took ~4,500 cycles
     // for a CTA's 128 KB of fp32 partials, ~140 cycles per box.)
     const int ws = (threadIdx.x >> 5) - 4;  // softmax warp 0-7
-    uint8_t* stage = c.gbase + kOffV + ws * 4096;
+    uint8_t* stage = c.gbase + L::kOffV + ws * 4096;
     const int row0 = c.cta * kRowsCta + 32 * ((rr >> 5) & 1);  // first row of this warp in the tile
     const uint32_t swz = lane & 7;
     const int col0 = 256 * sp + 128 * half;
@@ -855,10 +1183,10 @@ __device__ void softmax_epilogue(const DecodeParams& p, const Ctx& c, uint32_t t
     tc_fence_before();
     __syncwarp();
     if (lane == 0) MLA_TRACE(17, 8 * (s - s_begin) + ((threadIdx.x >> 5) - 4));
-    if (lane == 0) arrive_leader(c, kBarOEmpty);  // O is read out: the next segment's PV may overwrite it
+    if (lane == 0) arrive_leader(c, L::kBarOEmpty);  // O is read out: the next segment's PV may overwrite it
     if (lane == 0) {
       MLA_TRACE(18, 8 * (s - s_begin) + ((threadIdx.x >> 5) - 4));
-      mbar_arrive(c.bar(kBarStageFree));  // staging read: the value ring may be refilled
+      mbar_arrive(c.bar(L::kBarStageFree));  // staging read: the value ring may be refilled
     }
     __syncwarp();
     if (r == 0) MLA_TRACE(13, s - s_begin);
@@ -875,7 +1203,9 @@ __device__ void softmax_epilogue(const DecodeParams& p, const Ctx& c, uint32_t t
 // other CTA's bytes too; the other CTA then leaves only after the cluster
 // barrier that follows.  Returns false if a wait ran out (a copy that was
 // never issued by the other CTA, whose abort came first).
-__device__ __noinline__ bool drain_copies(const Ctx& c) {
+template <class C>
+__device__ __noinline__ bool drain_copies(const Ctx<C>& c) {
+  using L = Lay<C>;
   volatile uint32_t* fill = c.fill();
   bool ok = true;
   auto wait_last = [&](uint32_t bar, uint32_t n) {
@@ -888,64 +1218,85 @@ __device__ __noinline__ bool drain_copies(const Ctx& c) {
       }
     }
   };
-  if (c.cta == 0) {
-    for (int k = 0; k < kKRing; ++k) wait_last(c.bar(kBarKFull + k), fill[k]);
-    wait_last(c.bar(kBarQFull), fill[kFillQ]);
+  if constexpr (C::kFp8) {
+    // every copy lands on this CTA's own barriers: Q and the staging slots
+    wait_last(c.bar(L::kBarQFull), fill[L::kFillQ]);
+    for (int k = 0; k < C::kSRing; ++k) wait_last(c.bar(L::kBarStFull + k), fill[L::kFillS + k]);
+  } else {
+    if (c.cta == 0) {
+      for (int k = 0; k < C::kKRing; ++k) wait_last(c.bar(L::kBarKFull + k), fill[k]);
+      wait_last(c.bar(L::kBarQFull), fill[L::kFillQ]);
+    }
+    for (int k = 0; k < kVRing; ++k) wait_last(c.bar(L::kBarVFull + k), fill[L::kFillV + k]);
   }
-  for (int k = 0; k < kVRing; ++k) wait_last(c.bar(kBarVFull + k), fill[kFillV + k]);
   return ok;
 }
 
-__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
+template <class C>
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(C::kThreads, 1)
     mla_decode_kernel(const __grid_constant__ DecodeParams p) {
+  using L = Lay<C>;
   extern __shared__ uint8_t smem_raw[];
   MLA_PRO(0);
   const uint32_t raw = smem_u32(smem_raw);
   const uint32_t base = (raw + 1023u) & ~1023u;
-  Ctx c;
+  Ctx<C> c;
   c.base = base;
   c.gbase = smem_raw + (base - raw);
   c.cta = cluster_ctarank();
   c.meta = p.meta;
-  c.abort_flag = reinterpret_cast<volatile uint32_t*>(c.gbase + kOffAbort);
+  c.abort_flag = reinterpret_cast<volatile uint32_t*>(c.gbase + L::kOffAbort);
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
 
   if (threadIdx.x == 0) {
     // Barriers of the leader's pipeline are only used in the leader, the
     // rest in both CTAs; initialise all of them everywhere.
-    for (int k = 0; k < kKRing; ++k) {
-      mbar_init(c.bar(kBarKFull + k), 2);
-      mbar_init(c.bar(kBarKEmpty + k), 1);
+    // Key panels: bf16, the leader's expect_tx arrival plus one from the other
+    // CTA; fp8, one arrival per key-converter warp of both CTAs.  Value tiles:
+    // bf16, the copy's expect_tx arrival; fp8, one per value-converter warp.
+    for (int k = 0; k < C::kKRing; ++k) {
+      mbar_init(c.bar(L::kBarKFull + k), C::kFp8 ? 4 : 2);
+      mbar_init(c.bar(L::kBarKEmpty + k), 1);
     }
     for (int k = 0; k < kVRing; ++k) {
-      mbar_init(c.bar(kBarVFull + k), 1);
-      mbar_init(c.bar(kBarPFull + k), 4);
+      mbar_init(c.bar(L::kBarVFull + k), C::kFp8 ? 2 : 1);
+      mbar_init(c.bar(L::kBarPFull + k), 4);
     }
-    for (int k = 0; k < kPvBars; ++k) mbar_init(c.bar(kBarPvDone + k), 1);
+    mbar_init(c.bar(L::kBarQReady), 4);
+    for (int k = 0; k < C::kSRing; ++k) {
+      mbar_init(c.bar(L::kBarStFull + k), 1);
+      mbar_init(c.bar(L::kBarStEmpty + k), 2);
+    }
+    for (int k = 0; k < kPvBars; ++k) mbar_init(c.bar(L::kBarPvDone + k), 1);
     for (int k = 0; k < 2; ++k) {
-      mbar_init(c.bar(kBarSFull + k), 1);
-      mbar_init(c.bar(kBarSEmpty + k), 16);
+      mbar_init(c.bar(L::kBarSFull + k), 1);
+      mbar_init(c.bar(L::kBarSEmpty + k), 16);
     }
-    mbar_init(c.bar(kBarQFull), 1);
-    mbar_init(c.bar(kBarQEmpty), 1);
-    mbar_init(c.bar(kBarOEmpty), 16);
-    mbar_init(c.bar(kBarXch), 8);
-    mbar_init(c.bar(kBarFinal), 2);
-    mbar_init(c.bar(kBarStageFree), 8);
-    mbar_init(c.bar(kBarResc), 4);
-    mbar_init(c.bar(kBarResc + 1), 4);
+    mbar_init(c.bar(L::kBarQFull), 1);
+    mbar_init(c.bar(L::kBarQEmpty), 1);
+    mbar_init(c.bar(L::kBarOEmpty), 16);
+    mbar_init(c.bar(L::kBarXch), 8);
+    mbar_init(c.bar(L::kBarFinal), 2);
+    mbar_init(c.bar(L::kBarStageFree), 8);
+    mbar_init(c.bar(L::kBarResc), 4);
+    mbar_init(c.bar(L::kBarResc + 1), 4);
     *c.abort_flag = 0u;
-    for (uint32_t k = 0; k < kKRing + 1 + kVRing; ++k) c.fill()[k] = 0u;
+    for (uint32_t k = 0; k < L::kNumFill; ++k) c.fill()[k] = 0u;
     fence_mbar_init_cluster();
   }
   if (warp == 1) {
-    tmem_alloc_pair(base + kOffTmemSlot, kTmemCols);
+    tmem_alloc_pair(base + L::kOffTmemSlot, kTmemCols);
     tmem_relinquish_pair();
   }
   if (warp == 0 && lane == 0) {
-    tma_prefetch_desc(&p.tm_k);
-    tma_prefetch_desc(&p.tm_v);
+    if constexpr (C::kFp8) {
+      tma_prefetch_desc(&p.tm_codes);
+      tma_prefetch_desc(&p.tm_rope);
+    } else {
+      tma_prefetch_desc(&p.tm_k);
+      tma_prefetch_desc(&p.tm_v);
+    }
     tma_prefetch_desc(&p.tm_q);
   }
   tc_fence_before();
@@ -953,9 +1304,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
   tc_fence_after();
   cluster_sync();  // both CTAs' barriers exist before any remote arrival
   MLA_PRO(1);
-  const uint32_t tmem = *reinterpret_cast<volatile uint32_t*>(c.gbase + kOffTmemSlot);
-  c.peer_abort = map_to_rank(base + kOffAbort, c.cta ^ 1u);
-  c.lead_bars = map_to_rank(base + kOffBar, 0);
+  const uint32_t tmem = *reinterpret_cast<volatile uint32_t*>(c.gbase + L::kOffTmemSlot);
+  c.peer_abort = map_to_rank(base + L::kOffAbort, c.cta ^ 1u);
+  c.lead_bars = map_to_rank(base + L::kOffBar, 0);
   // Programmatic dependent launch: the set-up above overlapped the previous
   // kernel (the plan, or the previous call's combine); wait for its
   // completion before reading the plan or writing any output.  The combine
@@ -1000,29 +1351,51 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
 #ifdef MLA_DECODE_TRACE
   if (threadIdx.x == 0 && c.cta == 0) g_mla_span[blockIdx.x >> 1][0] = globaltimer();
 #endif
+  // FP8 cache: 512 threads launched with 128 registers each; the two softmax
+  // warpgroups take what the producer/issuer warpgroup and the converter
+  // warpgroup give up, and everyone returns to 128 before the teardown.
+  if constexpr (C::kFp8) {
+    if (warp >= 4 && warp < 12)
+      regs_inc<kRegsSoftmax>();
+    else
+      regs_dec<kRegsSide>();
+  }
   if (warp == 0) {
     producer_k(p, c, s_begin, s_end);
   } else if (warp == 1) {
     if (lane == 0 && c.cta == 0) qk_issuer(p, c, tmem, s_begin, s_end);
     __syncwarp();
   } else if (warp == 2) {
-    producer_v(p, c, s_begin, s_end);
+    if constexpr (!C::kFp8) producer_v(p, c, s_begin, s_end);
   } else if (warp == 3) {
     if (lane == 0 && c.cta == 0) pv_issuer(p, c, tmem, s_begin, s_end);
     __syncwarp();
-  } else {
+  } else if (warp < 12) {
     softmax_epilogue(p, c, tmem, s_begin, s_end);
+  } else {
+    if constexpr (C::kFp8) {
+      if (warp < 14)
+        key_converter(p, c, s_begin, s_end);
+      else
+        value_converter(p, c, s_begin, s_end);
+    }
+  }
+  if constexpr (C::kFp8) {
+    if (warp >= 4 && warp < 12)
+      regs_dec<kRegsLaunch>();
+    else
+      regs_inc<kRegsLaunch>();
   }
 
   // ---- teardown: drain the pair MMAs, wait for the peer, free TMEM ----
   __syncthreads();
-  if (warp == 3 && c.cta == 0 && lane == 0) umma_commit_pair(c.bar(kBarFinal), 0x1);  // PV issuer's MMAs
+  if (warp == 3 && c.cta == 0 && lane == 0) umma_commit_pair(c.bar(L::kBarFinal), 0x1);  // PV issuer's MMAs
   if (warp == 1 && c.cta == 0) {
     if (lane == 0) {
-      umma_commit_pair(c.bar(kBarFinal), 0x1);  // QK issuer's MMAs
+      umma_commit_pair(c.bar(L::kBarFinal), 0x1);  // QK issuer's MMAs
       const uint64_t t0 = globaltimer();
       bool done = false;
-      while (!(done = mbar_try_wait(c.bar(kBarFinal), 0)) && globaltimer() - t0 < kTimeoutNs) {
+      while (!(done = mbar_try_wait(c.bar(L::kBarFinal), 0)) && globaltimer() - t0 < kTimeoutNs) {
       }
       // MMAs that never completed are recorded; TMEM is still freed below:
       // a CTA that exits holding TMEM would leave the next kernel's
@@ -1080,7 +1453,7 @@ extern "C" __attribute__((visibility("default"))) int mla_trace_clear() {
 }
 #endif
 
-size_t decode_kernel_smem_bytes() { return kSmemBytes; }
+size_t decode_kernel_smem_bytes(bool fp8) { return fp8 ? Lay<CfgFp8>::kSmemBytes : Lay<CfgBf16>::kSmemBytes; }
 
 __device__ unsigned int g_mla_sticky_taken;
 
@@ -1095,21 +1468,21 @@ cudaError_t take_sticky_error(cudaStream_t stream, uint32_t* word) {
   return e;
 }
 
-cudaError_t decode_kernel_prepare() {
-  return cudaFuncSetAttribute(mla_decode_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                              static_cast<int>(kSmemBytes));
+namespace {
+
+template <class C>
+cudaError_t prepare_one() {
+  return cudaFuncSetAttribute(mla_decode_kernel<C>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                              static_cast<int>(Lay<C>::kSmemBytes));
 }
 
-cudaError_t decode_kernel_pairs(int* pairs) {
-  cudaError_t e = decode_kernel_prepare();
-  if (e != cudaSuccess) return e;
-  int dev = 0, sms = 0;
-  if ((e = cudaGetDevice(&dev)) != cudaSuccess) return e;
-  if ((e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev)) != cudaSuccess) return e;
+// Co-resident 2-CTA clusters of one build of the kernel.
+template <class C>
+cudaError_t pairs_one(int sms, int* clusters) {
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(static_cast<unsigned>(sms & ~1), 1, 1);
-  cfg.blockDim = dim3(kThreads, 1, 1);
-  cfg.dynamicSmemBytes = kSmemBytes;
+  cfg.blockDim = dim3(C::kThreads, 1, 1);
+  cfg.dynamicSmemBytes = Lay<C>::kSmemBytes;
   cudaLaunchAttribute attr[1];
   attr[0].id = cudaLaunchAttributeClusterDimension;
   attr[0].val.clusterDim.x = 2;
@@ -1117,25 +1490,50 @@ cudaError_t decode_kernel_pairs(int* pairs) {
   attr[0].val.clusterDim.z = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  int clusters = 0;
-  e = cudaOccupancyMaxActiveClusters(&clusters, mla_decode_kernel, &cfg);
-  if (e != cudaSuccess) return e;
-  *pairs = clusters < kMaxPairs ? clusters : kMaxPairs;
-  return cudaSuccess;
+  return cudaOccupancyMaxActiveClusters(clusters, mla_decode_kernel<C>, &cfg);
 }
 
-cudaError_t launch_decode(const DecodeParams& p, int pairs, cudaStream_t stream) {
+template <class C>
+cudaError_t launch_one(const DecodeParams& p, int pairs, cudaStream_t stream) {
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(static_cast<unsigned>(2 * pairs), 1, 1);
-  cfg.blockDim = dim3(kThreads, 1, 1);
-  cfg.dynamicSmemBytes = kSmemBytes;
+  cfg.blockDim = dim3(C::kThreads, 1, 1);
+  cfg.dynamicSmemBytes = Lay<C>::kSmemBytes;
   cfg.stream = stream;
   cudaLaunchAttribute attr[1];
   attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
   attr[0].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  return cudaLaunchKernelEx(&cfg, mla_decode_kernel, p);
+  return cudaLaunchKernelEx(&cfg, mla_decode_kernel<C>, p);
+}
+
+}  // namespace
+
+cudaError_t decode_kernel_prepare() {
+  cudaError_t e = prepare_one<CfgBf16>();
+  if (e == cudaSuccess) e = prepare_one<CfgFp8>();
+  return e;
+}
+
+// Both builds (bf16 and FP8 cache) run on the same pairs, as one plan serves
+// both: the smaller of their co-resident cluster counts.
+cudaError_t decode_kernel_pairs(int* pairs) {
+  cudaError_t e = decode_kernel_prepare();
+  if (e != cudaSuccess) return e;
+  int dev = 0, sms = 0;
+  if ((e = cudaGetDevice(&dev)) != cudaSuccess) return e;
+  if ((e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev)) != cudaSuccess) return e;
+  int c_bf16 = 0, c_fp8 = 0;
+  if ((e = pairs_one<CfgBf16>(sms, &c_bf16)) != cudaSuccess) return e;
+  if ((e = pairs_one<CfgFp8>(sms, &c_fp8)) != cudaSuccess) return e;
+  int clusters = c_bf16 < c_fp8 ? c_bf16 : c_fp8;
+  *pairs = clusters < kMaxPairs ? clusters : kMaxPairs;
+  return cudaSuccess;
+}
+
+cudaError_t launch_decode(const DecodeParams& p, int pairs, cudaStream_t stream) {
+  return p.fp8 ? launch_one<CfgFp8>(p, pairs, stream) : launch_one<CfgBf16>(p, pairs, stream);
 }
 
 }  // namespace mla

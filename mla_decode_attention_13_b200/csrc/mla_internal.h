@@ -111,6 +111,15 @@ struct DecodeParams {
   // page (its 128 columns of each half), panels in [half][panel] order.
   CUtensorMap tm_v;
   CUtensorMap tm_q;  // q: box (64, 64, 9), 64 query rows
+  // FP8 cache only (fp8 = 1; tm_k and tm_v unused then):
+  //   latent codes [rows][512] u8 as (512 cols, rows), box (64, 64), no
+  //   swizzle: 64 codes of a page's 64 tokens;
+  //   rope [rows][64] bf16 as (64 cols, rows), box (64, 64), 128B-swizzled.
+  CUtensorMap tm_codes;
+  CUtensorMap tm_rope;
+  const uint8_t* codes;    // [rows][512] E4M3 (value tiles are built from it)
+  const int8_t* exps;      // [rows]: token scale 2^exp
+  int fp8;
   const int32_t* block_table;
   const int32_t* seqlens;
   void* out;               // bf16
@@ -141,7 +150,7 @@ cudaError_t launch_sched(const int32_t* seqlens, int batch, int h_q, int s_q, in
                          cudaStream_t stream);
 cudaError_t decode_kernel_prepare();
 cudaError_t decode_kernel_pairs(int* pairs);
-size_t decode_kernel_smem_bytes();
+size_t decode_kernel_smem_bytes(bool fp8);
 // Reads and clears (atomically, on `stream`) the device's sticky error bits.
 cudaError_t take_sticky_error(cudaStream_t stream, uint32_t* word);
 cudaError_t launch_decode(const DecodeParams& p, int pairs, cudaStream_t stream);

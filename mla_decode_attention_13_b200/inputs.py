@@ -276,7 +276,7 @@ E4M3_MAX = 0x7E   # 448
 
 def make_fp8_inputs(seqlens: Sequence[int], h_q: int, s_q: int = 1, *, seed: int = 0, causal: bool = False,
                     softmax_scale: float = DEFAULT_SCALE, pool_factor: Optional[float] = 1.25,
-                    exp_range: tuple = (-8, -5)) -> Fp8DecodeInputs:
+                    exp_range: tuple = (-8, -5), device: str = "cpu") -> Fp8DecodeInputs:
     """Paged FP8 decode step drawn on the CPU generator.
 
     The latent codes are N(0, 64^2) values rounded to E4M3 (so that the
@@ -286,14 +286,16 @@ def make_fp8_inputs(seqlens: Sequence[int], h_q: int, s_q: int = 1, *, seed: int
     pool, table entries past a row's pages on a spare page whose codes are
     NaN, and slots past L in a row's last page holding the largest code with
     exponent 5 (14336: finite, large enough to be noticed if read).
+    ``device`` only chooses where the random numbers are drawn (as in
+    ``make_inputs``: parity tests draw on the CPU).
     """
-    gen = torch.Generator()
+    gen = torch.Generator(device=device)
     gen.manual_seed(seed)
     batch = len(seqlens)
     pages_per_row = [(int(L) + PAGE - 1) // PAGE for L in seqlens]
     needed = sum(pages_per_row)
     pool = max(needed, 1) if pool_factor is None else max(int(math.ceil(pool_factor * needed)), needed + 1)
-    perm = torch.randperm(pool, generator=gen)
+    perm = torch.randperm(pool, generator=gen, device=device).to("cpu")
     spare = int(perm[needed]) if pool > needed else 0
     width = max(max(pages_per_row, default=0), 1)
     table = torch.full((batch, width), spare, dtype=torch.int32)
@@ -301,13 +303,19 @@ def make_fp8_inputs(seqlens: Sequence[int], h_q: int, s_q: int = 1, *, seed: int
     for i, n in enumerate(pages_per_row):
         table[i, :n] = perm[cursor:cursor + n].to(torch.int32)
         cursor += n
-    q = torch.randn(batch, s_q, h_q, D_QK, generator=gen).to(torch.bfloat16)
-    codes = (torch.randn(pool, PAGE, D_LATENT, generator=gen) * 64.0).to(torch.float8_e4m3fn).view(torch.uint8)
-    rope = torch.randn(pool, PAGE, D_ROPE, generator=gen).to(torch.bfloat16)
-    exps = torch.randint(exp_range[0], exp_range[1] + 1, (pool, PAGE), generator=gen, dtype=torch.int64).to(torch.int8)
+    q = torch.randn(batch, s_q, h_q, D_QK, generator=gen, device=device).to(torch.bfloat16)
+    codes = torch.empty(pool, PAGE, D_LATENT, dtype=torch.uint8, device=device)
+    chunk = 4096
+    for p0 in range(0, pool, chunk):
+        p1 = min(pool, p0 + chunk)
+        codes[p0:p1] = (torch.randn(p1 - p0, PAGE, D_LATENT, generator=gen, device=device) * 64.0).to(
+            torch.float8_e4m3fn).view(torch.uint8)
+    rope = torch.randn(pool, PAGE, D_ROPE, generator=gen, device=device).to(torch.bfloat16)
+    exps = torch.randint(exp_range[0], exp_range[1] + 1, (pool, PAGE), generator=gen, dtype=torch.int64,
+                         device=device).to(torch.int8)
     used = torch.zeros(pool, dtype=torch.bool)
     used[perm[:needed]] = True
-    unused = (~used).nonzero().flatten()
+    unused = (~used).nonzero().flatten().to(device)
     if unused.numel():
         codes[unused] = E4M3_NAN
         rope[unused] = float("nan")
@@ -316,6 +324,6 @@ def make_fp8_inputs(seqlens: Sequence[int], h_q: int, s_q: int = 1, *, seed: int
             last = int(table[i, n - 1])
             codes[last, int(L) % PAGE:] = E4M3_MAX
             exps[last, int(L) % PAGE:] = 5
-    return Fp8DecodeInputs(q=q, latent_codes=codes.contiguous(), rope=rope, exps=exps, block_table=table,
-                           seqlens=torch.tensor([int(L) for L in seqlens], dtype=torch.int32), s_q=s_q, h_q=h_q,
-                           causal=causal, softmax_scale=softmax_scale)
+    return Fp8DecodeInputs(q=q, latent_codes=codes.contiguous(), rope=rope, exps=exps, block_table=table.to(device),
+                           seqlens=torch.tensor([int(L) for L in seqlens], dtype=torch.int32, device=device),
+                           s_q=s_q, h_q=h_q, causal=causal, softmax_scale=softmax_scale)

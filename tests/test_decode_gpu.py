@@ -26,6 +26,7 @@ import torch
 
 from mla_decode_attention_13_b200 import binding, inputs
 from oracle import mla_oracle
+from parity_bounds import bf16_weight_bound
 
 pytestmark = pytest.mark.gpu
 
@@ -40,28 +41,6 @@ def run(x, check_error=True):
     if check_error:
         assert err == 0, f"device error word {err:#x}"
     return out.cpu(), lse.cpu(), meta
-
-
-def bf16_weight_bound(x, want_o, rows):
-    """Per-element bound 1.01 * 2^-8 (|out| + sum_j w_j |v_j|) + 1e-4 (module docstring)."""
-    B = np.zeros_like(want_o)
-    for n, i in enumerate(rows):
-        L = int(x.seqlens[i])
-        pages = (L + 63) // 64
-        kv = x.kv_cache[x.block_table[i, :pages].long()].reshape(pages * 64, 576)[:L].double().numpy()
-        for t in range(x.s_q):
-            lim = min(max((L - x.s_q + t + 1) if x.causal else L, 0), L)
-            q = x.q[i, t].double().numpy()
-            for h in range(x.h_q):
-                o = want_o[n, t, h]
-                if lim == 0:
-                    continue
-                z = x.softmax_scale * (kv[:lim] @ q[h])
-                w = np.exp(z - z.max())
-                w /= w.sum()
-                mag = w @ np.abs(kv[:lim, :512])
-                B[n, t, h] = 1.01 * 2.0 ** -8 * (np.abs(o) + mag) + 1e-4
-    return B
 
 
 def assert_parity(x, out, lse, rows=None, strict=False):

@@ -9,9 +9,12 @@ Tolerances.  The merge reads bf16 (mla_merge_splits) or fp32
 rounds once to bf16: |out - oracle| <= 2^-8 |oracle| + 1e-5 and
 |lse - oracle| <= 1e-5 (1 + |lse|).  The emulated split runs each rank's
 decode with fp32 output (mla_decode_f32) and merges the fp32 partials, so
-nothing is rounded before the merge: the merge weights sum to one, the merged
-error stays within each rank's decode error, and the result is held to the
-plain decode bars (max-abs 8e-3, mean-abs 1e-3, lse 1e-3).
+nothing is rounded before the merge: the merge weights sum to one and the
+merged error stays within an unsplit decode's.  The result is held to the
+unsplit decode's bars: mean-abs 1e-3 and lse 1e-3, and per element the larger
+of 8e-3 and the bf16-weight bound of parity_bounds, which exceeds 8e-3 only on
+rows where a few tokens carry the weight (the cases below include rows of 1
+to 3 tokens, causal); the long-context workload's split is held to 8e-3.
 """
 
 import numpy as np
@@ -20,6 +23,7 @@ import torch
 
 from mla_decode_attention_13_b200 import binding, inputs, longrow
 from oracle import mla_oracle
+from parity_bounds import bf16_weight_bound
 
 pytestmark = pytest.mark.gpu
 
@@ -83,7 +87,8 @@ def test_split_decode_emulated_on_one_gpu_matches_unsplit_oracle(world, case):
     want_out, want_lse = mla_oracle.decode(x.q, x.kv_cache, x.block_table, x.seqlens, x.softmax_scale, causal)
     got = mla_oracle.as_f64(out.cpu())
     err = np.abs(got - want_out)
-    assert err.max() <= 8e-3 and err.mean() <= 1e-3, (err.max(), err.mean())
+    tol = np.maximum(8e-3, bf16_weight_bound(x, want_out, list(range(x.batch))))
+    assert (err <= tol).all() and err.mean() <= 1e-3, (err.max(), err.mean())
     got_lse = mla_oracle.as_f64(lse.cpu())
     assert np.array_equal(np.isneginf(got_lse), np.isneginf(want_lse))
     fin = np.isfinite(want_lse)
