@@ -83,8 +83,8 @@ __device__ unsigned long long g_mla_pro[160][4];
 __device__ unsigned long long g_mla_abort[6];
 // Per block and warp: the wait it left on abort (1 << 32 | barrier << 8 | parity)
 // and the role's last loop position.
-__device__ unsigned long long g_mla_stuck[160 * 2][12];
-__device__ unsigned long long g_mla_step[160 * 2][12];
+__device__ unsigned long long g_mla_stuck[160 * 2][16];
+__device__ unsigned long long g_mla_step[160 * 2][16];
 #define MLA_STEP(v) \
   do {              \
     g_mla_step[blockIdx.x][threadIdx.x >> 5] = static_cast<unsigned long long>(v); \
@@ -159,13 +159,8 @@ struct CfgFp8 {
   static constexpr int kKRing = 2;
   static constexpr int kSRing = 4;
 };
-// FP8 kernel registers per thread: 128 at launch (65,536 / 512); the eight
-// softmax warps run with 168, the other eight with 88 (256 x 168 + 256 x 88 =
-// 65,536).
-constexpr uint32_t kRegsLaunch = 128;
-constexpr uint32_t kRegsSoftmax = 168;
-constexpr uint32_t kRegsSide = 88;
-static_assert(256 * kRegsSoftmax + 256 * kRegsSide <= 65536, "register split");
+// The FP8 build's 512 threads run with 128 registers each (65,536 / 512), the
+// softmax warps included; no warp changes its register count at run time.
 
 // Shared-memory layout (offsets from a 1024-byte aligned base).  All operand
 // tiles are 128-byte swizzled panels of 64 16-bit columns.
@@ -601,6 +596,7 @@ __device__ void key_converter(const DecodeParams& p, const Ctx<C>& c, int s_begi
   uint32_t seg_it = 0, sf = 0, kf = 0;  // segments, staging fills, key panels
   bool out_of_range = false;
   auto conv_q = [&](const Segment&) -> bool {
+    MLA_STEP((10ull << 40) | seg_it);
     if (!wait_bar(c, c.bar(L::kBarQFull), seg_it & 1)) return false;
     ++seg_it;
     uint4* q = reinterpret_cast<uint4*>(c.gbase + L::kOffQ);
@@ -639,6 +635,7 @@ __device__ void key_converter(const DecodeParams& p, const Ctx<C>& c, int s_begi
     }
     for (int pn = 0; pn < 9; ++pn, ++kf) {
       const uint32_t ks = kf % C::kKRing;
+      MLA_STEP((8ull << 40) | (static_cast<unsigned long long>(sf) << 20) | kf);
       if (kf >= C::kKRing && !wait_bar(c, c.bar(L::kBarKEmpty + ks), ((kf / C::kKRing) - 1) & 1)) return false;
       uint8_t* dst = c.gbase + L::kOffK + ks * kKSlot;
       if (pn < 8) {
@@ -714,6 +711,7 @@ __device__ void value_converter(const DecodeParams& p, const Ctx<C>& c, int s_be
       for (int j = 0; j < 8; ++j) v[j] = ld_nc_v4(src + 4 * kDv * j);
       const uint32_t ew = *reinterpret_cast<const uint16_t*>(p.exps + row0 + 2 * lane);  // tokens 2 lane, + 1
       int good = 1;
+      MLA_STEP((9ull << 40) | ps);
       if (lane == 0) {
         // The previous segment's epilogue stages its output in the value ring.
         if (gr.first && q == 0 && seg_it > 0) good = wait_bar(c, c.bar(L::kBarStageFree), (seg_it - 1) & 1);
@@ -1351,15 +1349,6 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(C::kThreads, 1)
 #ifdef MLA_DECODE_TRACE
   if (threadIdx.x == 0 && c.cta == 0) g_mla_span[blockIdx.x >> 1][0] = globaltimer();
 #endif
-  // FP8 cache: 512 threads launched with 128 registers each; the two softmax
-  // warpgroups take what the producer/issuer warpgroup and the converter
-  // warpgroup give up, and everyone returns to 128 before the teardown.
-  if constexpr (C::kFp8) {
-    if (warp >= 4 && warp < 12)
-      regs_inc<kRegsSoftmax>();
-    else
-      regs_dec<kRegsSide>();
-  }
   if (warp == 0) {
     producer_k(p, c, s_begin, s_end);
   } else if (warp == 1) {
@@ -1379,12 +1368,6 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(C::kThreads, 1)
       else
         value_converter(p, c, s_begin, s_end);
     }
-  }
-  if constexpr (C::kFp8) {
-    if (warp >= 4 && warp < 12)
-      regs_dec<kRegsLaunch>();
-    else
-      regs_inc<kRegsLaunch>();
   }
 
   // ---- teardown: drain the pair MMAs, wait for the peer, free TMEM ----

@@ -301,17 +301,6 @@ __host__ __device__ constexpr uint32_t idesc_bf16_f32(uint32_t m, uint32_t n, bo
   return (1u << 4) | (1u << 7) | (1u << 10) | ((b_mn_major ? 1u : 0u) << 16) | ((n >> 3) << 17) | ((m >> 4) << 24);
 }
 
-// Warp-group register re-allocation (all four warps of the warpgroup execute
-// it): give up registers down to N, or wait for registers up to N, per thread.
-template <uint32_t N>
-__device__ __forceinline__ void regs_dec() {
-  asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(N));
-}
-template <uint32_t N>
-__device__ __forceinline__ void regs_inc() {
-  asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(N));
-}
-
 // Two E4M3 codes (low byte first) to two f16 values, exactly (every E4M3
 // value is an f16 value).
 __device__ __forceinline__ uint32_t e4m3x2_to_f16x2(uint16_t codes) {

@@ -276,7 +276,7 @@ E4M3_MAX = 0x7E   # 448
 
 def make_fp8_inputs(seqlens: Sequence[int], h_q: int, s_q: int = 1, *, seed: int = 0, causal: bool = False,
                     softmax_scale: float = DEFAULT_SCALE, pool_factor: Optional[float] = 1.25,
-                    exp_range: tuple = (-8, -5), device: str = "cpu") -> Fp8DecodeInputs:
+                    exp_range: tuple = (-8, -6), device: str = "cpu") -> Fp8DecodeInputs:
     """Paged FP8 decode step drawn on the CPU generator.
 
     The latent codes are N(0, 64^2) values rounded to E4M3 (so that the

@@ -300,11 +300,28 @@ def decode_fp8(q, latent_codes, rope, exps, block_table, seqlens, softmax_scale:
 
     latent_codes [num_pages, 64, 512] uint8 (E4M3), rope [num_pages, 64, 64]
     (bf16 or float), exps [num_pages, 64] integer (token scale 2^exp).  Each
-    cached row is [dequantised latent, rope]; the rest is ``decode``.
+    cached row is [dequantised latent, rope]; the rest is ``decode``.  Only
+    the pages the computed rows read are dequantised (a pool of those pages,
+    with the block table renumbered into it), so that a large pool costs no
+    more than the rows asked for.
     """
-    lat = dequantize_latent(latent_codes, exps)
-    pool = np.concatenate([lat, as_f64(rope)], axis=-1)[:, :, None, :]  # [pages, 64, 1, 576]
-    return decode(q, pool, block_table, seqlens, softmax_scale, causal, rows=rows)
+    table = as_int(block_table)
+    lens = as_int(seqlens)
+    batch = table.shape[0]
+    sel = range(batch) if rows is None else rows
+    used = sorted({int(table[i, j]) for i in sel for j in range((max(int(lens[i]), 0) + PAGE - 1) // PAGE)})
+    index = {page: k for k, page in enumerate(used)}
+    local = np.zeros_like(table)
+    for i in sel:
+        for j in range((max(int(lens[i]), 0) + PAGE - 1) // PAGE):
+            local[i, j] = index[int(table[i, j])]
+    if not used:
+        pool = np.zeros((0, PAGE, D_QK))
+    else:
+        # index first (a plain list works for arrays and tensors), then convert
+        lat = dequantize_latent(as_int(latent_codes[used]), as_int(exps[used]))
+        pool = np.concatenate([lat, as_f64(rope[used])], axis=-1)
+    return decode(q, pool[:, :, None, :], local, seqlens, softmax_scale, causal, rows=rows)
 
 
 def absorb_query(q_nope, q_rope, w_uk) -> np.ndarray:

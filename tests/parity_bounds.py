@@ -35,3 +35,36 @@ def bf16_weight_bound(x, want_o, rows):
                 mag = w @ np.abs(kv[:lim, :512])
                 B[n, t, h] = 1.01 * 2.0 ** -8 * (np.abs(o) + mag) + 1e-4
     return B
+
+
+def fp8_weight_bound(x, want_o, rows):
+    """The same bound for the FP8-cache kernel (mla_decode_fp8), whose weights
+    go to the PV product as f16 (|e| <= 2^-11) and whose output is rounded to
+    bf16 once (bf16's unit roundoff: 2^-8 |out|):
+        |out_gpu - out| <= 1.01 * (2^-8 |out| + 2^-11 sum_j w_j |v_j|) + 1e-4.
+    x is an Fp8DecodeInputs; the values are the dequantised latent dims."""
+    from oracle import mla_oracle
+
+    B = np.zeros_like(want_o)
+    table = x.block_table.numpy()
+    for n, i in enumerate(rows):
+        L = int(x.seqlens[i])
+        if L <= 0:
+            continue
+        pages = (L + 63) // 64
+        ids = [int(v) for v in table[i, :pages]]
+        lat = mla_oracle.dequantize_latent(x.latent_codes[ids], x.exps[ids]).reshape(pages * 64, 512)[:L]
+        rope = x.rope[ids].double().numpy().reshape(pages * 64, 64)[:L]
+        keys = np.concatenate([lat, rope], axis=1)
+        for t in range(x.s_q):
+            lim = min(max((L - x.s_q + t + 1) if x.causal else L, 0), L)
+            if lim == 0:
+                continue
+            q = x.q[i, t].double().numpy()
+            for h in range(x.h_q):
+                z = x.softmax_scale * (keys[:lim] @ q[h])
+                w = np.exp(z - z.max())
+                w /= w.sum()
+                mag = w @ np.abs(lat[:lim])
+                B[n, t, h] = 1.01 * (2.0 ** -8 * np.abs(want_o[n, t, h]) + 2.0 ** -11 * mag) + 1e-4
+    return B

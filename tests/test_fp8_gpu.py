@@ -5,13 +5,18 @@ The cache format ("MLA 和 MHA 的 Kernel 区别", section "量化友好性"): E
 for the 512 latent dims of each token with one power-of-two scale 2^e per
 token, bf16 rope.  decode_fp8 dequantises exactly and runs the fp64 decode.
 
-Tolerances: the benchmark spec's bars on every case, max-abs 8e-3 and mean-abs 1e-3 on
-the bf16 output, |lse difference| <= 1e-3, -inf where the oracle has no
-visible token.  The kernel's arithmetic differs from the bf16 cache's only in
+Tolerances.  The kernel's arithmetic differs from the bf16 cache's only in
 formats that lose nothing or less: the dequantised values are exact in f16
 (e in [-15, 7]), q's latent part is exact in f16 for these N(0, 1) draws
 except below 2^-14 (absolute error <= 2^-25), and the softmax weights go to
-the PV product as f16 (relative error <= 2^-11 instead of bf16's 2^-8).
+the PV product as f16 (relative error <= 2^-11 instead of bf16's 2^-8).  The
+five workload shapes are held to the benchmark spec's bars: max-abs 8e-3 and
+mean-abs 1e-3 on the bf16 output, |lse difference| <= 1e-3, -inf where the
+oracle has no visible token.  The other cases keep the mean-abs and lse bars;
+per element they take the larger of 8e-3 and parity_bounds.fp8_weight_bound,
+1.01 (2^-8 |out| + 2^-11 sum_j w_j |v_j|) + 1e-4, which passes 8e-3 only on
+rows where a few tokens carry the weight and |out| reaches a few units (the
+bf16 rounding of the exact output alone can reach 2^-8 |out|).
 """
 
 import numpy as np
@@ -20,6 +25,7 @@ import torch
 
 from mla_decode_attention_13_b200 import binding, inputs
 from oracle import mla_oracle
+from parity_bounds import fp8_weight_bound
 
 pytestmark = pytest.mark.gpu
 
@@ -36,7 +42,7 @@ def run_fp8(x, meta=None):
     return out.cpu(), lse.cpu(), err
 
 
-def assert_parity(x, out, lse, rows=None):
+def assert_parity(x, out, lse, rows=None, strict=False):
     want_o, want_l = mla_oracle.decode_fp8(x.q, x.latent_codes, x.rope, x.exps, x.block_table, x.seqlens,
                                            x.softmax_scale, x.causal, rows=rows)
     sel = list(range(x.batch)) if rows is None else list(rows)
@@ -45,7 +51,12 @@ def assert_parity(x, out, lse, rows=None):
     want_o, want_l = want_o[sel], want_l[sel]
     assert np.isfinite(got_o).all(), "non-finite output"
     d = np.abs(got_o - want_o)
-    assert d.max() <= TOL_MAX, f"max-abs {d.max():.3e}"
+    if strict:
+        assert d.max() <= TOL_MAX, f"max-abs {d.max():.3e}"
+    else:
+        tol = np.maximum(TOL_MAX, fp8_weight_bound(x, want_o, sel))
+        worst = np.unravel_index(np.argmax(d - tol), d.shape)
+        assert (d <= tol).all(), f"max-abs {d.max():.3e}; worst excess at {worst}: {d[worst]:.3e} > {tol[worst]:.3e}"
     assert d.mean() <= TOL_MEAN, f"mean-abs {d.mean():.3e}"
     inf = np.isneginf(want_l)
     assert np.array_equal(np.isneginf(got_l), inf), "lse -inf pattern differs"
@@ -93,7 +104,7 @@ def test_exponents_at_the_ends_of_the_supported_range(exp_range, q_scale):
     # smallest subnormal) and the high end (up to 448 * 2^7) of [-15, 7].  The
     # latent part of q is scaled so that the scores stay O(1); the outputs
     # then scale with 2^e, so the bar is relative to their size: 2^-7 of the
-    # largest |out| (bf16 rounding of the output is 2^-9 of it).
+    # largest |out| (bf16 rounding of the output is at most 2^-8 of it).
     x = inputs.make_fp8_inputs([3000, 77, 640], 64, seed=40 + exp_range[0], exp_range=exp_range)
     x.q[..., :512] = (x.q[..., :512].float() * q_scale).to(torch.bfloat16)
     out, lse, err = run_fp8(x)
@@ -132,7 +143,7 @@ def test_workload_shapes_full_size(index):
     out, lse, err = run_fp8(x)
     assert err == 0
     rows = None if wl.batch <= 16 else _sample_rows(lens, 8, seed=index)
-    assert_parity(x, out, lse, rows=rows)
+    assert_parity(x, out, lse, rows=rows, strict=True)
 
 
 def test_one_plan_serves_fp8_and_bf16_calls():
@@ -179,6 +190,7 @@ def test_matches_the_bf16_kernel_on_the_dequantised_cache():
 
 
 def test_out_of_range_exponent_and_query_are_flagged():
+    binding.mla_take_device_errors()  # start from a clear sticky word
     lens = [300, 200]
     # a visible token with exponent 9 (E4M3 values times 2^9 overflow f16)
     x = inputs.make_fp8_inputs(lens, 16, seed=70)
@@ -207,3 +219,4 @@ def test_out_of_range_exponent_and_query_are_flagged():
     assert err == 0
     assert_parity(x, out, lse)
     assert binding.mla_take_device_errors() & binding.MLA_DEVERR_FP8_RANGE
+    assert binding.mla_take_device_errors() == 0

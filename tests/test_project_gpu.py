@@ -55,6 +55,7 @@ def check(gpu: np.ndarray, ref: np.ndarray):
 
 @pytest.mark.parametrize("tokens,h_q", CASES)
 def test_absorb_matches_oracle(tokens, h_q):
+    binding.mla_take_device_errors()  # start from a clear sticky word
     x = inputs.make_projection_inputs(tokens, h_q, seed=tokens * 131 + h_q)
     g = x.to("cuda")
     out = binding.mla_absorb_q(g.q_nope, g.q_rope, g.w_uk)
@@ -68,6 +69,7 @@ def test_absorb_matches_oracle(tokens, h_q):
 
 @pytest.mark.parametrize("tokens,h_q", CASES)
 def test_up_project_matches_oracle(tokens, h_q):
+    binding.mla_take_device_errors()
     x = inputs.make_projection_inputs(tokens, h_q, seed=7 + tokens * 131 + h_q)
     g = x.to("cuda")
     out = binding.mla_up_project(g.o_latent, g.w_uv)
@@ -99,6 +101,7 @@ def test_zero_tokens_is_a_no_op():
 
 
 def test_layer_absorb_decode_up_project_matches_unabsorbed_definition():
+    binding.mla_take_device_errors()
     lens = [300, 64, 1000, 129]
     h_q = 16
     d = inputs.make_inputs(lens, h_q, 1, seed=11, pool_factor=1.5)
