@@ -746,7 +746,7 @@ def parity_check_fp8(idx, dev, min_rows=8):
             "pass": bool(d.max() <= TOL_MAX and d.mean() <= TOL_MEAN and lse_max <= TOL_LSE and neg_inf_match
                          and finite and err == 0),
             "inputs": "seeded FP8 inputs of the workload's shape (seed 3000 + index, drawn on the CPU): E4M3 codes "
-                      "of N(0, 64^2) values, token exponents uniform in [-8, -5], bf16 rope and q ~ N(0, 1)"}
+                      "of N(0, 64^2) values, token exponents uniform in [-8, -6], bf16 rope and q ~ N(0, 1)"}
 
 
 def fp8_workload(idx, args, world, rank, local, dev, stream, peaks):

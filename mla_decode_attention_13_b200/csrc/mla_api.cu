@@ -85,7 +85,7 @@ int tensor_map_encoder(PFN_cuTensorMapEncodeTiled_v12000* fn) {
 // same cache and a few rotating query buffers, so their maps are encoded once
 // instead of on every call.  A map holds only the address and the layout, so
 // it stays right for any later buffer at the same address and size.
-enum MapKind : int { kMapK = 0, kMapV = 1, kMapQ = 2, kMapCodes = 3, kMapRope = 4, kMapKinds = 5 };
+enum MapKind : int { kMapK = 0, kMapV = 1, kMapQ = 2, kMapCodes = 3, kMapRope = 4, kMapVCodes = 5, kMapKinds = 6 };
 
 struct MapCache {
   static constexpr int kWays = 8;
@@ -187,6 +187,21 @@ int encode_codes(PFN_cuTensorMapEncodeTiled_v12000 enc, CUtensorMap* map, const 
   const cuuint32_t box[2] = {64, static_cast<cuuint32_t>(kPage)};
   const cuuint32_t elem[2] = {1, 1};
   const CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void*>(base), dims, strides, box, elem,
+                         CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                         CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS ? MLA_OK : MLA_ERR_CUDA;
+}
+
+// FP8 cache: the latent codes as (128 cols, rows, 2 column blocks c, 2
+// halves h) with strides (512 B, 128 B, 256 B): box (128, 64, 1, 2) at (0, y,
+// c, 0) is CTA c's value columns [256h + 128c, +128) of 64 tokens, landing as
+// [h][token][128 codes], unswizzled.
+int encode_vcodes(PFN_cuTensorMapEncodeTiled_v12000 enc, CUtensorMap* map, const void* base, uint64_t rows) {
+  const cuuint64_t dims[4] = {128, static_cast<cuuint64_t>(rows), 2, 2};
+  const cuuint64_t strides[3] = {static_cast<cuuint64_t>(kDv), 128, 256};
+  const cuuint32_t box[4] = {128, static_cast<cuuint32_t>(kPage), 1, 2};
+  const cuuint32_t elem[4] = {1, 1, 1, 1};
+  const CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 4, const_cast<void*>(base), dims, strides, box, elem,
                          CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                          CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   return r == CUDA_SUCCESS ? MLA_OK : MLA_ERR_CUDA;
@@ -325,7 +340,9 @@ int decode_impl(const void* q, const CacheRef& cache, int64_t num_pages, const i
     if ((st = cached_map(kMapCodes, cache.codes, kv_rows, &p.tm_codes,
                          [&](CUtensorMap* m) { return encode_codes(enc, m, cache.codes, kv_rows); })) != MLA_OK ||
         (st = cached_map(kMapRope, cache.rope, kv_rows, &p.tm_rope,
-                         [&](CUtensorMap* m) { return encode_rope(enc, m, cache.rope, kv_rows); })) != MLA_OK)
+                         [&](CUtensorMap* m) { return encode_rope(enc, m, cache.rope, kv_rows); })) != MLA_OK ||
+        (st = cached_map(kMapVCodes, cache.codes, kv_rows, &p.tm_vcodes,
+                         [&](CUtensorMap* m) { return encode_vcodes(enc, m, cache.codes, kv_rows); })) != MLA_OK)
       return st;
   } else {
     const void* kv_cache = cache.kv;

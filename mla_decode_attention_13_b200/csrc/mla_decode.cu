@@ -200,13 +200,15 @@ struct Lay {
   static constexpr uint32_t kBarQReady = kBarResc + 2;              // fp8: (leader) both CTAs' Q converted
   static constexpr uint32_t kBarStFull = kBarQReady + 1;            // fp8: [kSRing] (local) staging slot landed
   static constexpr uint32_t kBarStEmpty = kBarStFull + C::kSRing;   // fp8: [kSRing] (local) staging slot converted
-  static constexpr uint32_t kNumBars = kBarStEmpty + C::kSRing;
+  static constexpr uint32_t kBarVCodes = kBarStEmpty + C::kSRing;   // fp8: [kVRing] (local) a tile's value codes landed
+  static constexpr uint32_t kNumBars = kBarVCodes + (C::kFp8 ? kVRing : 0);
   static constexpr uint32_t kOffTmemSlot = kOffBar + 8 * kNumBars;  // u32
   static constexpr uint32_t kOffAbort = kOffTmemSlot + 4;           // u32
   // u32 fill counts of the barriers that TMA copies complete on: [kKRing] key
   // slots (bf16) and [1] Q (the expect_tx posted: bf16 leader, fp8 each CTA),
-  // [kVRing] value slots (bf16), [kSRing] staging slots (fp8); read at
-  // teardown to wait for copies still in flight on abort.
+  // [kVRing] value slots (bf16: the tiles; fp8: their codes), [kSRing]
+  // staging slots (fp8); read at teardown to wait for copies still in flight
+  // on abort.
   static constexpr uint32_t kOffFill = kOffAbort + 4;
   static constexpr uint32_t kFillQ = C::kKRing;
   static constexpr uint32_t kFillV = kFillQ + 1;
@@ -517,7 +519,8 @@ __device__ void producer_k(const DecodeParams& p, const Ctx<C>& c, int s_begin, 
 // Warp 2: this CTA's value tile of every page (all 64 tokens, its 256 value
 // columns) into the value ring once PV two pages back has released the slot;
 // bytes complete on this CTA's own barrier (the softmax warps wait for it
-// before releasing P, so PV never runs ahead of it).
+// before releasing P, so PV never runs ahead of it).  FP8 cache: the tile's
+// codes instead, into the slot's upper half, for the value converters.
 template <class C>
 __device__ void producer_v(const DecodeParams& p, const Ctx<C>& c, int s_begin, int s_end) {
   using L = Lay<C>;
@@ -538,10 +541,21 @@ __device__ void producer_v(const DecodeParams& p, const Ctx<C>& c, int s_begin, 
         if (good) {
           MLA_TRACE(3, ps);
           MLA_STEP(ps);
-          const uint32_t bar = c.bar(L::kBarVFull + slot);
-          mbar_arrive_expect_tx(bar, kVTile);
-          c.fill()[L::kFillV + slot] += 1;
-          tma_load_4d(c.vtile(slot), &p.tm_v, bar, 0, gr.page[q] * kPage, 2 * static_cast<int>(c.cta), 0);
+          if constexpr (C::kFp8) {
+            // The page's E4M3 codes of this CTA's value columns ([h][64
+            // tokens][128 codes], 16 KB) into the upper half of the tile's
+            // slot; the value converters dequantise them over the whole slot.
+            const uint32_t bar = c.bar(L::kBarVCodes + slot);
+            mbar_arrive_expect_tx(bar, kVTile / 2);
+            c.fill()[L::kFillV + slot] += 1;
+            tma_load_4d(c.vtile(slot) + kVTile / 2, &p.tm_vcodes, bar, 0, gr.page[q] * kPage,
+                        static_cast<int>(c.cta), 0);
+          } else {
+            const uint32_t bar = c.bar(L::kBarVFull + slot);
+            mbar_arrive_expect_tx(bar, kVTile);
+            c.fill()[L::kFillV + slot] += 1;
+            tma_load_4d(c.vtile(slot), &p.tm_v, bar, 0, gr.page[q] * kPage, 2 * static_cast<int>(c.cta), 0);
+          }
         }
       }
     }
@@ -685,75 +699,57 @@ __device__ void key_converter(const DecodeParams& p, const Ctx<C>& c, int s_begi
 
 // Warps 14-15 (64 threads), FP8 cache only: this CTA's value tile of every
 // page (its 256 value columns [256h + 128c, +128), h = 0, 1, of all 64
-// tokens, f16, the layout of the bf16 cache's value tiles), built from the
-// page's codes in L2 (the pair has just staged the page) and each token's
-// 2^e, once PV two pages back has released the slot.  The loads are issued
-// before that wait.
+// tokens, f16, the layout of the bf16 cache's value tiles).  Warp 2 has
+// copied the page's codes of those columns into the upper half of the tile's
+// slot (once PV two pages back released it); each warp reads its tokens'
+// codes into registers and writes their dequantised rows (each token's 2^e
+// applied) over the whole slot.  A token belongs to one warp, and its f16 rows
+// in the upper half lie exactly over its own codes ([h][token][128] there,
+// panels 2 and 3 row `token`), so no warp overwrites codes another still
+// reads.
 template <class C>
 __device__ void value_converter(const DecodeParams& p, const Ctx<C>& c, int s_begin, int s_end) {
   using L = Lay<C>;
   const int vt = static_cast<int>(threadIdx.x) - 14 * 32;  // 0-63
   const int lane = threadIdx.x & 31;
-  uint32_t ps = 0, seg_it = 0;  // pages, segments
+  uint32_t ps = 0;  // pages
+  // 16-byte chunk vt + 64 j (j = 0-15) of the tile: token tok0 + 4 j (tok0 =
+  // vt / 16), half h = (vt / 8) % 2, codes 16 i8 to +15 (i8 = vt % 8) of the
+  // half's 128 columns; only the token moves with j.
+  const int tok0 = vt >> 4, h = (vt >> 3) & 1, i8 = vt & 7;
+  const uint32_t ch = 2 * (i8 & 3);
   walk_groups(p, c, s_begin, s_end, [&](const Segment&, const Group& gr) -> bool {
     for (int q = 0; q < gr.np; ++q, ++ps) {
       const uint32_t slot = ps % kVRing;
-      const long long row0 = static_cast<long long>(gr.page[q]) * kPage;
-      // 16-byte chunk vt + 64 j (j = 0-15) of the tile: token tok0 + 4 j
-      // (tok0 = vt / 16), half h = (vt / 8) % 2, codes 16 i8 to +15 (i8 =
-      // vt % 8) of the half's 128 columns; only the token moves with j.
-      const int tok0 = vt >> 4, h = (vt >> 3) & 1, i8 = vt & 7;
-      const uint8_t* src = p.codes + (row0 + tok0) * kDv + 256 * h + 128 * static_cast<int>(c.cta) + 16 * i8;
-      // The first half of the tile's codes is loaded before the wait, the
-      // second while the first is converted.
-      uint4 v[8];
-#pragma unroll
-      for (int j = 0; j < 8; ++j) v[j] = ld_nc_v4(src + 4 * kDv * j);
-      const uint32_t ew = *reinterpret_cast<const uint16_t*>(p.exps + row0 + 2 * lane);  // tokens 2 lane, + 1
-      int good = 1;
       MLA_STEP((9ull << 40) | ps);
-      if (lane == 0) {
-        // The previous segment's epilogue stages its output in the value ring.
-        if (gr.first && q == 0 && seg_it > 0) good = wait_bar(c, c.bar(L::kBarStageFree), (seg_it - 1) & 1);
-        if (good && ps >= kVRing) {
-          const uint32_t k = ps - kVRing;  // the tile's previous page: its PV must be done
-          good = wait_bar(c, c.bar(L::kBarPvDone + k % kPvBars), (k / kPvBars) & 1);
-        }
-      }
-      if (!__shfl_sync(0xffffffffu, good, 0)) return false;
+      const long long row0 = static_cast<long long>(gr.page[q]) * kPage;
+      const uint32_t ew = *reinterpret_cast<const uint16_t*>(p.exps + row0 + 2 * lane);  // tokens 2 lane, + 1
+      if (!wait_bar(c, c.bar(L::kBarVCodes + slot), (ps / kVRing) & 1)) return false;
+      uint8_t* tile = c.gbase + L::kOffV + slot * kVTile;
+      // codes: [h][token][128] in the slot's upper half
+      const uint8_t* src = tile + kVTile / 2 + (h * kPage + tok0) * 128 + 16 * i8;
+      uint4 v[16];
+#pragma unroll
+      for (int j = 0; j < 16; ++j) v[j] = *reinterpret_cast<const uint4*>(src + 512 * j);
+      __syncwarp();  // the warp's codes are in registers before its rows overwrite them
       // panel [h][i8 / 4]; f16 chunks 2 (i8 % 4) and + 1 of the token's
       // 128-byte row, swizzled by tok % 8 = (tok0 % 8) ^ (4 (j % 2)).
-      uint8_t* drow = c.gbase + L::kOffV + slot * kVTile + (2 * h + (i8 >> 2)) * kVPanel + tok0 * 128;
-      const uint32_t ch = 2 * (i8 & 3);
+      uint8_t* drow = tile + (2 * h + (i8 >> 2)) * kVPanel + tok0 * 128;
 #pragma unroll
-      for (int half = 0; half < 2; ++half) {
-        uint4 w[8];
-        if (half == 0) {
-#pragma unroll
-          for (int j = 0; j < 8; ++j) w[j] = ld_nc_v4(src + 4 * kDv * (8 + j));
-        }
-#pragma unroll
-        for (int j = 0; j < 8; ++j) {
-          const int jj = 8 * half + j;
-          const int tok = tok0 + 4 * jj;
-          const int e = static_cast<int8_t>((__shfl_sync(0xffffffffu, ew, tok >> 1) >> (8 * (tok & 1))) & 0xFFu);
-          const uint32_t sc = f16_pow2(e);
-          uint4 lo, hi;
-          dequant16(v[j], sc | (sc << 16), lo, hi);
-          const uint32_t sw = (tok0 & 7) ^ (4 * (j & 1));
-          *reinterpret_cast<uint4*>(drow + 512 * jj + ((ch ^ sw) << 4)) = lo;
-          *reinterpret_cast<uint4*>(drow + 512 * jj + (((ch + 1) ^ sw) << 4)) = hi;
-        }
-        if (half == 0) {
-#pragma unroll
-          for (int j = 0; j < 8; ++j) v[j] = w[j];
-        }
+      for (int j = 0; j < 16; ++j) {
+        const int tok = tok0 + 4 * j;
+        const int e = static_cast<int8_t>((__shfl_sync(0xffffffffu, ew, tok >> 1) >> (8 * (tok & 1))) & 0xFFu);
+        const uint32_t sc = f16_pow2(e);
+        uint4 lo, hi;
+        dequant16(v[j], sc | (sc << 16), lo, hi);
+        const uint32_t sw = (tok0 & 7) ^ (4 * (j & 1));
+        *reinterpret_cast<uint4*>(drow + 512 * j + ((ch ^ sw) << 4)) = lo;
+        *reinterpret_cast<uint4*>(drow + 512 * j + (((ch + 1) ^ sw) << 4)) = hi;
       }
       fence_proxy_async_smem();
       __syncwarp();
       if (lane == 0) mbar_arrive(c.bar(L::kBarVFull + slot));
     }
-    if (gr.first) ++seg_it;
     return true;
   });
 }
@@ -1220,6 +1216,7 @@ __device__ __noinline__ bool drain_copies(const Ctx<C>& c) {
     // every copy lands on this CTA's own barriers: Q and the staging slots
     wait_last(c.bar(L::kBarQFull), fill[L::kFillQ]);
     for (int k = 0; k < C::kSRing; ++k) wait_last(c.bar(L::kBarStFull + k), fill[L::kFillS + k]);
+    for (int k = 0; k < kVRing; ++k) wait_last(c.bar(L::kBarVCodes + k), fill[L::kFillV + k]);
   } else {
     if (c.cta == 0) {
       for (int k = 0; k < C::kKRing; ++k) wait_last(c.bar(L::kBarKFull + k), fill[k]);
@@ -1266,6 +1263,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(C::kThreads, 1)
       mbar_init(c.bar(L::kBarStFull + k), 1);
       mbar_init(c.bar(L::kBarStEmpty + k), 2);
     }
+    if constexpr (C::kFp8)
+      for (int k = 0; k < kVRing; ++k) mbar_init(c.bar(L::kBarVCodes + k), 1);
     for (int k = 0; k < kPvBars; ++k) mbar_init(c.bar(L::kBarPvDone + k), 1);
     for (int k = 0; k < 2; ++k) {
       mbar_init(c.bar(L::kBarSFull + k), 1);
@@ -1291,6 +1290,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(C::kThreads, 1)
     if constexpr (C::kFp8) {
       tma_prefetch_desc(&p.tm_codes);
       tma_prefetch_desc(&p.tm_rope);
+      tma_prefetch_desc(&p.tm_vcodes);
     } else {
       tma_prefetch_desc(&p.tm_k);
       tma_prefetch_desc(&p.tm_v);
@@ -1355,7 +1355,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(C::kThreads, 1)
     if (lane == 0 && c.cta == 0) qk_issuer(p, c, tmem, s_begin, s_end);
     __syncwarp();
   } else if (warp == 2) {
-    if constexpr (!C::kFp8) producer_v(p, c, s_begin, s_end);
+    producer_v(p, c, s_begin, s_end);
   } else if (warp == 3) {
     if (lane == 0 && c.cta == 0) pv_issuer(p, c, tmem, s_begin, s_end);
     __syncwarp();

@@ -117,6 +117,10 @@ struct DecodeParams {
   //   rope [rows][64] bf16 as (64 cols, rows), box (64, 64), 128B-swizzled.
   CUtensorMap tm_codes;
   CUtensorMap tm_rope;
+  //   the same codes as (128 cols, rows, 2 blocks c, 2 halves h), strides
+  //   (512 B, 128 B, 256 B): box (128, 64, 1, 2) at (0, y, c, 0) is CTA c's
+  //   value columns [256h + 128c, +128) of 64 tokens, [h][token][128].
+  CUtensorMap tm_vcodes;
   const uint8_t* codes;    // [rows][512] E4M3 (value tiles are built from it)
   const int8_t* exps;      // [rows]: token scale 2^exp
   int fp8;
