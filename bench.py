@@ -875,6 +875,21 @@ def ours(args, world, rank, local):
         print(json.dumps(line), flush=True)
 
 
+def ours_fp8(args, world, rank, local):
+    """--fp8: the workload's step on the FP8 latent cache, one JSON line (for
+    profiling runs of that kernel; the default line carries the same entry
+    under fp8_cache)."""
+    dev = torch.device("cuda", local)
+    torch.cuda.set_device(dev)
+    stream = torch.cuda.Stream(dev)
+    e = fp8_workload(args.workload, args, world, rank, local, dev, stream, measured_peaks())
+    if rank == 0:
+        print(json.dumps({"metric": METRIC, "value": e["step_us"], "unit": "us/call", "n_gpus": world,
+                          "steps": e["steps"], "warmup": args.warmup, "higher_is_better": False, "scaling": "weak",
+                          "vs_baseline": None, "dtype": "fp8 cache, f16/bf16 MMAs", "data": "synthetic", **e}),
+              flush=True)
+
+
 def projection_work(tokens, h_q):
     """Algorithmic bytes of one absorb and one up-projection launch: the head
     weights once, the tokens' inputs once, the outputs once (bf16)."""
@@ -1102,6 +1117,8 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true", help="run no oracle (no parity, no CPU baseline)")
     ap.add_argument("--headline-only", action="store_true",
                     help="time only the headline workload's step (no projections, split or other workloads)")
+    ap.add_argument("--fp8", action="store_true",
+                    help="time the workload's step on the FP8 latent cache (mla_decode_fp8) only")
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3
@@ -1109,6 +1126,8 @@ def main():
     try:
         if args.impl == "reference":
             reference_arm(args, world, rank)
+        elif args.fp8:
+            ours_fp8(args, world, rank, local)
         else:
             ours(args, world, rank, local)
     finally:

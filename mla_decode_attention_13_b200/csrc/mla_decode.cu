@@ -71,7 +71,7 @@ namespace mla {
 // Optional clock64 timeline of the pipeline roles, for profiling builds only
 // (compile with -DMLA_DECODE_TRACE; the default build records nothing).
 #ifdef MLA_DECODE_TRACE
-__device__ unsigned long long g_mla_trace[4][20][512];  // [traced CTA][event][index]
+__device__ unsigned long long g_mla_trace[4][24][512];  // [traced CTA][event][index]
 __device__ unsigned long long g_mla_span[160][4];  // [pair][start, end, segments, pages] (globaltimer)
 // Prologue of the leader CTA of each pair: [entry, after cluster sync, after the grid dependency, exit].
 __device__ unsigned long long g_mla_pro[160][4];
@@ -464,6 +464,7 @@ __device__ void producer_k(const DecodeParams& p, const Ctx<C>& c, int s_begin, 
         if (!good) break;
         const uint32_t bytes = f < 8 ? my_np * (kSSlot / 2) : (f - 8 < my_np ? kSSlot : 0u);
         if (lane == 0) {
+          MLA_TRACE(10, sf);
           mbar_arrive_expect_tx(c.bar(L::kBarStFull + slot), bytes);
           c.fill()[L::kFillS + slot] += 1;
         }
@@ -655,6 +656,7 @@ __device__ void key_converter(const DecodeParams& p, const Ctx<C>& c, int s_begi
       if (pn < 8) {
         const uint32_t st = sf % C::kSRing;
         if (!wait_bar(c, c.bar(L::kBarStFull + st), (sf / C::kSRing) & 1)) return false;
+        if (kt == 0) MLA_TRACE(20, kf);
         ++sf;
         // 16-byte chunk kt + 64 j of the slot: row kt / 4 + 16 j (64 bytes of
         // codes per row), codes 16 (kt % 4) to +15 -> f16 chunks 2 (kt % 4)
@@ -690,6 +692,7 @@ __device__ void key_converter(const DecodeParams& p, const Ctx<C>& c, int s_begi
       }
       fence_proxy_async_smem();
       __syncwarp();
+      if (kt == 0) MLA_TRACE(21, kf);
       if (lane == 0) arrive_leader(c, L::kBarKFull + ks);
     }
     return true;
@@ -725,6 +728,7 @@ __device__ void value_converter(const DecodeParams& p, const Ctx<C>& c, int s_be
       const long long row0 = static_cast<long long>(gr.page[q]) * kPage;
       const uint32_t ew = *reinterpret_cast<const uint16_t*>(p.exps + row0 + 2 * lane);  // tokens 2 lane, + 1
       if (!wait_bar(c, c.bar(L::kBarVCodes + slot), (ps / kVRing) & 1)) return false;
+      if (vt == 0) MLA_TRACE(22, ps);
       uint8_t* tile = c.gbase + L::kOffV + slot * kVTile;
       // codes: [h][token][128] in the slot's upper half
       const uint8_t* src = tile + kVTile / 2 + (h * kPage + tok0) * 128 + 16 * i8;
@@ -748,6 +752,7 @@ __device__ void value_converter(const DecodeParams& p, const Ctx<C>& c, int s_be
       }
       fence_proxy_async_smem();
       __syncwarp();
+      if (vt == 0) MLA_TRACE(23, ps);
       if (lane == 0) mbar_arrive(c.bar(L::kBarVFull + slot));
     }
     return true;
@@ -1431,7 +1436,7 @@ extern "C" __attribute__((visibility("default"))) int mla_trace_stuck(void* stuc
   return static_cast<int>(e);
 }
 extern "C" __attribute__((visibility("default"))) int mla_trace_clear() {
-  static unsigned long long zero[4][20][512];
+  static unsigned long long zero[4][24][512];
   return static_cast<int>(cudaMemcpyToSymbol(g_mla_trace, zero, sizeof(zero)));
 }
 #endif
