@@ -593,7 +593,7 @@ __device__ __forceinline__ uint32_t bf16x2_to_f16x2(uint32_t w) {
   return f32x2_to_f16x2(__uint_as_float(w & 0xFFFF0000u), __uint_as_float(w << 16));
 }
 
-// Warps 12-13 (64 threads), FP8 cache only.
+// Warps 12-15 (128 threads), FP8 cache only.
 //   * At each segment start: this CTA's Q rows to f16 in place (the latent
 //     panels 0-7; the rope panel stays bf16), then one arrival per warp on the
 //     leader's Q barrier.  A query value past the f16 range is flagged.
@@ -606,7 +606,7 @@ __device__ __forceinline__ uint32_t bf16x2_to_f16x2(uint32_t w) {
 template <class C>
 __device__ void key_converter(const DecodeParams& p, const Ctx<C>& c, int s_begin, int s_end) {
   using L = Lay<C>;
-  const int kt = static_cast<int>(threadIdx.x) - 12 * 32;  // 0-63
+  const int kt = static_cast<int>(threadIdx.x) - 12 * 32;  // 0-127
   const int lane = threadIdx.x & 31;
   uint32_t seg_it = 0, sf = 0, kf = 0;  // segments, staging fills, key panels
   bool out_of_range = false;
@@ -616,7 +616,7 @@ __device__ void key_converter(const DecodeParams& p, const Ctx<C>& c, int s_begi
     ++seg_it;
     uint4* q = reinterpret_cast<uint4*>(c.gbase + L::kOffQ);
     uint32_t inf_seen = 0;  // bit 15 of a half: an f16 result with the all-ones exponent
-    for (int k = kt; k < static_cast<int>(8 * kQPanel / 16); k += 64) {
+    for (int k = kt; k < static_cast<int>(8 * kQPanel / 16); k += 128) {
       uint4 v = q[k];
       v.x = bf16x2_to_f16x2(v.x);
       v.y = bf16x2_to_f16x2(v.y);
@@ -658,23 +658,26 @@ __device__ void key_converter(const DecodeParams& p, const Ctx<C>& c, int s_begi
         if (!wait_bar(c, c.bar(L::kBarStFull + st), (sf / C::kSRing) & 1)) return false;
         if (kt == 0) MLA_TRACE(20, kf);
         ++sf;
-        // 16-byte chunk kt + 64 j of the slot: row kt / 4 + 16 j (64 bytes of
-        // codes per row), codes 16 (kt % 4) to +15 -> f16 chunks 2 (kt % 4)
+        // 16-byte chunk kt + 128 j of the slot: row kt / 4 + 32 j (64 bytes
+        // of codes per row), codes 16 (kt % 4) to +15 -> f16 chunks 2 (kt % 4)
         // and + 1 of the row, swizzled by row % 8 = (kt / 4) % 8.
         const int row0 = kt >> 2, c4 = kt & 3;
         const uint8_t* src = c.gbase + L::kOffS + st * kSSlot + 16 * kt;
         uint8_t* drow = dst + row0 * 128;
         const uint32_t off_lo = ((2 * c4) ^ (row0 & 7)) << 4, off_hi = ((2 * c4 + 1) ^ (row0 & 7)) << 4;
-#pragma unroll 4
-        for (int j = 0; j < 8; ++j) {
-          const uint4 v = *reinterpret_cast<const uint4*>(src + 1024 * j);
-          const int row = row0 + 16 * j;
+        uint4 v4[4];
+#pragma unroll
+        for (int j = 0; j < 4; ++j) v4[j] = *reinterpret_cast<const uint4*>(src + 2048 * j);
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+          const uint4 v = v4[j];
+          const int row = row0 + 32 * j;
           const int e = static_cast<int8_t>((__shfl_sync(0xffffffffu, ew, row >> 2) >> (8 * (row & 3))) & 0xFFu);
           const uint32_t sc = f16_pow2(e);
           uint4 lo, hi;
           dequant16(v, sc | (sc << 16), lo, hi);
-          *reinterpret_cast<uint4*>(drow + 2048 * j + off_lo) = lo;
-          *reinterpret_cast<uint4*>(drow + 2048 * j + off_hi) = hi;
+          *reinterpret_cast<uint4*>(drow + 4096 * j + off_lo) = lo;
+          *reinterpret_cast<uint4*>(drow + 4096 * j + off_hi) = hi;
         }
         __syncwarp();
         if (lane == 0) mbar_arrive(c.bar(L::kBarStEmpty + st));
@@ -685,7 +688,7 @@ __device__ void key_converter(const DecodeParams& p, const Ctx<C>& c, int s_begi
           const uint4* src = reinterpret_cast<const uint4*>(c.gbase + L::kOffS + st * kSSlot);
           uint4* d = reinterpret_cast<uint4*>(dst + h * kSSlot);
 #pragma unroll
-          for (int k = kt; k < static_cast<int>(kSSlot / 16); k += 64) d[k] = src[k];
+          for (int k = kt; k < static_cast<int>(kSSlot / 16); k += 128) d[k] = src[k];
           __syncwarp();
           if (lane == 0) mbar_arrive(c.bar(L::kBarStEmpty + st));
         }
@@ -700,63 +703,51 @@ __device__ void key_converter(const DecodeParams& p, const Ctx<C>& c, int s_begi
   if (out_of_range) set_error(c.meta, MLA_DEVERR_FP8_RANGE);
 }
 
-// Warps 14-15 (64 threads), FP8 cache only: this CTA's value tile of every
-// page (its 256 value columns [256h + 128c, +128), h = 0, 1, of all 64
-// tokens, f16, the layout of the bf16 cache's value tiles).  Warp 2 has
-// copied the page's codes of those columns into the upper half of the tile's
-// slot (once PV two pages back released it); each warp reads its tokens'
-// codes into registers and writes their dequantised rows (each token's 2^e
-// applied) over the whole slot.  A token belongs to one warp, and its f16 rows
-// in the upper half lie exactly over its own codes ([h][token][128] there,
-// panels 2 and 3 row `token`), so no warp overwrites codes another still
-// reads.
+// FP8 cache: this CTA's value tile of one page (its 256 value columns [256h +
+// 128c, +128), h = 0, 1, of all 64 tokens, f16, the layout of the bf16 cache's
+// value tiles), dequantised in place by the 64 softmax threads that write the
+// page's P (vt = 0-63, two warps), once warp 2 has copied the page's codes of
+// those columns into the upper half of the tile's slot.  Each thread reads
+// its tokens' codes and writes their dequantised rows (each token's 2^e
+// applied; zeros for tokens at or past `valid`, whose codes may hold
+// anything) over the whole slot.  A token belongs to one warp (tokens 0 and 1
+// mod 4 to the first, 2 and 3 to the second), and its f16 rows in the upper
+// half lie exactly over its own codes ([h][token][128] there, panels 2 and 3
+// row `token`), so a warp sync between a pass's reads and its writes is the
+// only ordering needed.  ew: the page's exponent bytes of tokens 2 lane and
+// 2 lane + 1.
 template <class C>
-__device__ void value_converter(const DecodeParams& p, const Ctx<C>& c, int s_begin, int s_end) {
+__device__ __forceinline__ void convert_value_tile(const Ctx<C>& c, uint32_t slot, int vt, int valid, uint32_t ew) {
   using L = Lay<C>;
-  const int vt = static_cast<int>(threadIdx.x) - 14 * 32;  // 0-63
-  const int lane = threadIdx.x & 31;
-  uint32_t ps = 0;  // pages
   // 16-byte chunk vt + 64 j (j = 0-15) of the tile: token tok0 + 4 j (tok0 =
   // vt / 16), half h = (vt / 8) % 2, codes 16 i8 to +15 (i8 = vt % 8) of the
   // half's 128 columns; only the token moves with j.
   const int tok0 = vt >> 4, h = (vt >> 3) & 1, i8 = vt & 7;
   const uint32_t ch = 2 * (i8 & 3);
-  walk_groups(p, c, s_begin, s_end, [&](const Segment&, const Group& gr) -> bool {
-    for (int q = 0; q < gr.np; ++q, ++ps) {
-      const uint32_t slot = ps % kVRing;
-      MLA_STEP((9ull << 40) | ps);
-      const long long row0 = static_cast<long long>(gr.page[q]) * kPage;
-      const uint32_t ew = *reinterpret_cast<const uint16_t*>(p.exps + row0 + 2 * lane);  // tokens 2 lane, + 1
-      if (!wait_bar(c, c.bar(L::kBarVCodes + slot), (ps / kVRing) & 1)) return false;
-      if (vt == 0) MLA_TRACE(22, ps);
-      uint8_t* tile = c.gbase + L::kOffV + slot * kVTile;
-      // codes: [h][token][128] in the slot's upper half
-      const uint8_t* src = tile + kVTile / 2 + (h * kPage + tok0) * 128 + 16 * i8;
-      uint4 v[16];
+  uint8_t* tile = c.gbase + L::kOffV + slot * kVTile;
+  const uint8_t* src = tile + kVTile / 2 + (h * kPage + tok0) * 128 + 16 * i8;  // codes: [h][token][128]
+  // panel [h][i8 / 4]; f16 chunks 2 (i8 % 4) and + 1 of the token's 128-byte
+  // row, swizzled by tok % 8 = (tok0 % 8) ^ (4 (j % 2)).
+  uint8_t* drow = tile + (2 * h + (i8 >> 2)) * kVPanel + tok0 * 128;
 #pragma unroll
-      for (int j = 0; j < 16; ++j) v[j] = *reinterpret_cast<const uint4*>(src + 512 * j);
-      __syncwarp();  // the warp's codes are in registers before its rows overwrite them
-      // panel [h][i8 / 4]; f16 chunks 2 (i8 % 4) and + 1 of the token's
-      // 128-byte row, swizzled by tok % 8 = (tok0 % 8) ^ (4 (j % 2)).
-      uint8_t* drow = tile + (2 * h + (i8 >> 2)) * kVPanel + tok0 * 128;
+  for (int jb = 0; jb < 16; jb += 4) {  // four passes of four tokens
+    uint4 v[4];
 #pragma unroll
-      for (int j = 0; j < 16; ++j) {
-        const int tok = tok0 + 4 * j;
-        const int e = static_cast<int8_t>((__shfl_sync(0xffffffffu, ew, tok >> 1) >> (8 * (tok & 1))) & 0xFFu);
-        const uint32_t sc = f16_pow2(e);
-        uint4 lo, hi;
-        dequant16(v[j], sc | (sc << 16), lo, hi);
-        const uint32_t sw = (tok0 & 7) ^ (4 * (j & 1));
-        *reinterpret_cast<uint4*>(drow + 512 * j + ((ch ^ sw) << 4)) = lo;
-        *reinterpret_cast<uint4*>(drow + 512 * j + (((ch + 1) ^ sw) << 4)) = hi;
-      }
-      fence_proxy_async_smem();
-      __syncwarp();
-      if (vt == 0) MLA_TRACE(23, ps);
-      if (lane == 0) mbar_arrive(c.bar(L::kBarVFull + slot));
+    for (int u = 0; u < 4; ++u) v[u] = *reinterpret_cast<const uint4*>(src + 512 * (jb + u));
+    __syncwarp();  // the pass's codes are in registers before its rows overwrite them
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      const int j = jb + u;
+      const int tok = tok0 + 4 * j;
+      const int e = static_cast<int8_t>((__shfl_sync(0xffffffffu, ew, tok >> 1) >> (8 * (tok & 1))) & 0xFFu);
+      const uint32_t sc = f16_pow2(e);
+      uint4 lo = make_uint4(0, 0, 0, 0), hi = make_uint4(0, 0, 0, 0);
+      if (tok < valid) dequant16(v[u], sc | (sc << 16), lo, hi);
+      const uint32_t sw = (tok0 & 7) ^ (4 * (j & 1));
+      *reinterpret_cast<uint4*>(drow + 512 * j + ((ch ^ sw) << 4)) = lo;
+      *reinterpret_cast<uint4*>(drow + 512 * j + (((ch + 1) ^ sw) << 4)) = hi;
     }
-    return true;
-  });
+  }
 }
 
 // ------------------------------------------------------ MMA (leader only) --
@@ -974,6 +965,18 @@ __device__ void softmax_epilogue(const DecodeParams& p, const Ctx<C>& c, uint32_
       const int np = min(kGroup, n - j);
       np_last = np;
       const uint32_t sb = gi & 1;
+      // FP8 cache: this thread's page's exponent bytes (tokens 2 lane, + 1),
+      // for the value tile it dequantises; loaded before the scores are waited
+      // for.  (A page id outside the pool reads page 0, as the producers do;
+      // they flag it.)
+      uint32_t v_ew = 0;
+      if constexpr (C::kFp8) {
+        if (q < np) {
+          int page = p.block_table[static_cast<long long>(sg.i) * p.max_pages + blk + q];
+          page = (page < 0 || page >= p.num_pages) ? 0 : page;
+          v_ew = *reinterpret_cast<const uint16_t*>(p.exps + static_cast<long long>(page) * kPage + 2 * lane);
+        }
+      }
       if (!wait_bar(c, c.bar(L::kBarSFull + sb), (gi >> 1) & 1)) return;
       if (r == 0) MLA_TRACE(4, gi);
       MLA_STEP((1ull << 40) | (static_cast<unsigned long long>(gi) << 20) | ps);
@@ -1029,49 +1032,75 @@ __device__ void softmax_epilogue(const DecodeParams& p, const Ctx<C>& c, uint32_
       }
 
       float lsum = 0.0f;
-      if (q < np) {
-        const uint32_t pg = ps + q;  // global page index
-        uint32_t packed[2][16];
+      uint32_t packed[2][16];
+      if (q < np)
         lsum = exp_pack<C::kFp8>(sv[0], nv[0], sl2, neg_m, packed[0]) +
                exp_pack<C::kFp8>(sv[1], nv[1], sl2, neg_m, packed[1]);
+      // ---- P tile free (PV two pages back); write this thread's row of P ----
+      auto write_p = [&]() -> bool {
+        const uint32_t pg = ps + q;  // global page index
         const uint32_t slot = pg % kVRing;
-        // ---- P tile free (PV two pages back) ----
-        if (pg >= kVRing && !pv_done(pg - kVRing)) return;
+        if (pg >= kVRing && !pv_done(pg - kVRing)) return false;
         MLA_STEP((2ull << 40) | pg);
         if (rr == 0) MLA_TRACE(6, pg);
-        {
-          uint8_t* prow = c.gbase + L::kOffP + slot * kPTile + prow_off;
+        uint8_t* prow = c.gbase + L::kOffP + slot * kPTile + prow_off;
 #pragma unroll
-          for (int ci = 0; ci < 8; ++ci)
-            *reinterpret_cast<uint4*>(prow + ((ci ^ (hr & 7)) << 4)) =
-                make_uint4(packed[ci >> 2][4 * (ci & 3)], packed[ci >> 2][4 * (ci & 3) + 1],
-                           packed[ci >> 2][4 * (ci & 3) + 2], packed[ci >> 2][4 * (ci & 3) + 3]);
-        }
-        // ---- this CTA's value tile has landed; the last page of a row may
-        //      hold garbage (even NaN) past L: zero the value rows there, so
-        //      that 0 * garbage cannot reach O ----
-        if (!wait_bar(c, c.bar(L::kBarVFull + slot), (pg / kVRing) & 1)) return;
-        MLA_STEP((3ull << 40) | pg);
-        if (rr == 0) MLA_TRACE(7, pg);
-        if (blk + q == last_page && (sg.L & (kPage - 1))) {
-          const int first_bad = sg.L - last_page * kPage;
-          const int chunks = (kPage - first_bad) * 4 * 8;  // tokens x panels x 16-byte chunks
-          uint8_t* vt = c.gbase + L::kOffV + slot * kVTile;
-          for (int e2 = hr; e2 < chunks; e2 += kRowsCta) {
-            const int tok = first_bad + (e2 >> 5);
-            *reinterpret_cast<uint4*>(vt + ((e2 >> 3) & 3) * kVPanel + tok * 128 + (e2 & 7) * 16) =
-                make_uint4(0, 0, 0, 0);
-          }
-        }
-        // The group's first PV adds to O: every warp of these rows must have
-        // rescaled its O columns first.
-        if (resc && q == 0 && !wait_bar(c, c.bar(L::kBarResc + kr), (n_resc - 1) & 1)) return;
+        for (int ci = 0; ci < 8; ++ci)
+          *reinterpret_cast<uint4*>(prow + ((ci ^ (hr & 7)) << 4)) =
+              make_uint4(packed[ci >> 2][4 * (ci & 3)], packed[ci >> 2][4 * (ci & 3) + 1],
+                         packed[ci >> 2][4 * (ci & 3) + 2], packed[ci >> 2][4 * (ci & 3) + 3]);
+        return true;
+      };
+      // ---- page k's P and value tile are ready in this warp's share: the
+      //      group's first PV adds to O, so its P writers first wait until
+      //      every warp of these rows has rescaled its O columns ----
+      auto release = [&](int k) -> bool {
+        if (resc && k == 0 && q == 0 && !wait_bar(c, c.bar(L::kBarResc + kr), (n_resc - 1) & 1)) return false;
         fence_proxy_async_smem();
         tc_fence_before();
         __syncwarp();
-        if (lane == 0) arrive_leader(c, L::kBarPFull + slot);
-        MLA_STEP((4ull << 40) | pg);
-        if (rr == 0) MLA_TRACE(8, pg);
+        if (lane == 0) arrive_leader(c, L::kBarPFull + (ps + k) % kVRing);
+        MLA_STEP((4ull << 40) | (ps + k));
+        if (rr == 0) MLA_TRACE(8, ps + k);
+        return true;
+      };
+      if constexpr (!C::kFp8) {
+        if (q < np) {
+          if (!write_p()) return;
+          // ---- this CTA's value tile has landed; the last page of a row may
+          //      hold garbage (even NaN) past L: zero the value rows there, so
+          //      that 0 * garbage cannot reach O ----
+          const uint32_t pg = ps + q;
+          const uint32_t slot = pg % kVRing;
+          if (!wait_bar(c, c.bar(L::kBarVFull + slot), (pg / kVRing) & 1)) return;
+          MLA_STEP((3ull << 40) | pg);
+          if (rr == 0) MLA_TRACE(7, pg);
+          if (blk + q == last_page && (sg.L & (kPage - 1))) {
+            const int first_bad = sg.L - last_page * kPage;
+            const int chunks = (kPage - first_bad) * 4 * 8;  // tokens x panels x 16-byte chunks
+            uint8_t* vt = c.gbase + L::kOffV + slot * kVTile;
+            for (int e2 = hr; e2 < chunks; e2 += kRowsCta) {
+              const int tok = first_bad + (e2 >> 5);
+              *reinterpret_cast<uint4*>(vt + ((e2 >> 3) & 3) * kVPanel + tok * 128 + (e2 & 7) * 16) =
+                  make_uint4(0, 0, 0, 0);
+            }
+          }
+          if (!release(q)) return;
+        }
+      } else {
+        // ---- FP8 cache: the page's codes have landed; its P writers
+        //      dequantise its value tile (zeros past L) ----
+        if (q < np) {
+          if (!write_p()) return;
+          const uint32_t pg = ps + q;
+          const uint32_t slot = pg % kVRing;
+          if (!wait_bar(c, c.bar(L::kBarVCodes + slot), (pg / kVRing) & 1)) return;
+          if (rr == 0) MLA_TRACE(22, pg);
+          const int valid = blk + q == last_page ? sg.L - last_page * kPage : kPage;
+          convert_value_tile(c, slot, hr, valid, v_ew);
+          if (rr == 0) MLA_TRACE(23, pg);
+          if (!release(q)) return;
+        }
       }
       l = l * alpha + lsum;
       m = m_new;
@@ -1254,19 +1283,21 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(C::kThreads, 1)
     // rest in both CTAs; initialise all of them everywhere.
     // Key panels: bf16, the leader's expect_tx arrival plus one from the other
     // CTA; fp8, one arrival per key-converter warp of both CTAs.  Value tiles:
-    // bf16, the copy's expect_tx arrival; fp8, one per value-converter warp.
+    // bf16, the copy's expect_tx arrival (fp8: the codes' copy completes
+    // VCodes, and the page's P writers dequantise the tile before releasing
+    // P).  P tiles: the page's two P-writer warps in both CTAs.
     for (int k = 0; k < C::kKRing; ++k) {
-      mbar_init(c.bar(L::kBarKFull + k), C::kFp8 ? 4 : 2);
+      mbar_init(c.bar(L::kBarKFull + k), C::kFp8 ? 8 : 2);
       mbar_init(c.bar(L::kBarKEmpty + k), 1);
     }
     for (int k = 0; k < kVRing; ++k) {
-      mbar_init(c.bar(L::kBarVFull + k), C::kFp8 ? 2 : 1);
+      mbar_init(c.bar(L::kBarVFull + k), 1);
       mbar_init(c.bar(L::kBarPFull + k), 4);
     }
-    mbar_init(c.bar(L::kBarQReady), 4);
+    mbar_init(c.bar(L::kBarQReady), 8);
     for (int k = 0; k < C::kSRing; ++k) {
       mbar_init(c.bar(L::kBarStFull + k), 1);
-      mbar_init(c.bar(L::kBarStEmpty + k), 2);
+      mbar_init(c.bar(L::kBarStEmpty + k), 4);
     }
     if constexpr (C::kFp8)
       for (int k = 0; k < kVRing; ++k) mbar_init(c.bar(L::kBarVCodes + k), 1);
@@ -1367,12 +1398,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(C::kThreads, 1)
   } else if (warp < 12) {
     softmax_epilogue(p, c, tmem, s_begin, s_end);
   } else {
-    if constexpr (C::kFp8) {
-      if (warp < 14)
-        key_converter(p, c, s_begin, s_end);
-      else
-        value_converter(p, c, s_begin, s_end);
-    }
+    if constexpr (C::kFp8) key_converter(p, c, s_begin, s_end);
   }
 
   // ---- teardown: drain the pair MMAs, wait for the peer, free TMEM ----
