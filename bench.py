@@ -154,11 +154,38 @@ def roofline_entry(nbytes, flops, k2_s, hbm_peak, tf_peak, peak_kind, traffic, t
                                   "timing")}
 
 
+def strip_comments(src):
+    """C/C++/CUDA source without its comments and blank lines, trailing
+    spaces dropped (string and character literals are kept as they are)."""
+    out, i, n = [], 0, len(src)
+    while i < n:
+        ch = src[i]
+        if src.startswith("//", i):
+            j = src.find("\n", i)
+            i = n if j < 0 else j
+        elif src.startswith("/*", i):
+            j = src.find("*/", i + 2)
+            i = n if j < 0 else j + 2
+        elif ch in "\"'":
+            j = i + 1
+            while j < n and src[j] != ch:
+                j += 2 if src[j] == "\\" else 1
+            out.append(src[i:j + 1])
+            i = j + 1
+        else:
+            out.append(ch)
+            i += 1
+    lines = (line.rstrip() for line in "".join(out).split("\n"))
+    return "\n".join(line for line in lines if line)
+
+
 def kernel_source_sha():
+    """Hash of the decode kernel's code (its comments and blank lines
+    removed): the ncu figures in TRAFFIC_FILE hold while it is unchanged."""
     h = hashlib.sha256()
     for name in KERNEL_SOURCES:
-        with open(os.path.join(ROOT, "mla_decode_attention_13_b200", "csrc", name), "rb") as f:
-            h.update(f.read())
+        with open(os.path.join(ROOT, "mla_decode_attention_13_b200", "csrc", name), encoding="utf-8") as f:
+            h.update(strip_comments(f.read()).encode("utf-8"))
     return h.hexdigest()[:16]
 
 

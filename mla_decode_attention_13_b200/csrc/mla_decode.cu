@@ -141,12 +141,13 @@ constexpr int kRowsCta = kMTile / 2;  // 64 query rows per CTA
 //   * fp8: the 512 latent values of a row are E4M3 codes with one power-of-two
 //     scale 2^e per token, the 64 rope values bf16 ("MLA 和 MHA 的 Kernel 区别",
 //     section "量化友好性": the latent cache tolerates FP8 or INT8, dequantised
-//     as it is loaded).  The codes land by TMA in a staging ring; converter
-//     warps dequantise them into the key panels and build the value tiles
-//     from L2.  The latent products run as f16 MMAs: every E4M3 value times
-//     2^e with e in [-15, 7] is exact in f16, and the latent part of Q is
-//     converted to f16 once per segment; the rope panel stays bf16 in both Q
-//     and the keys.  16 warps (four converter warps).
+//     as it is loaded).  The key codes land by TMA in a staging ring and
+//     four converter warps dequantise them into the key panels; each page's
+//     value codes land in its value tile's slot and the two softmax warps
+//     that write the page's P dequantise them in place.  The latent products
+//     run as f16 MMAs: every E4M3 value times 2^e with e in [-15, 7] is exact
+//     in f16, and the latent part of Q is converted to f16 once per segment;
+//     the rope panel stays bf16 in both Q and the keys.  16 warps.
 struct CfgBf16 {
   static constexpr bool kFp8 = false;
   static constexpr int kThreads = 384;
@@ -521,7 +522,8 @@ __device__ void producer_k(const DecodeParams& p, const Ctx<C>& c, int s_begin, 
 // columns) into the value ring once PV two pages back has released the slot;
 // bytes complete on this CTA's own barrier (the softmax warps wait for it
 // before releasing P, so PV never runs ahead of it).  FP8 cache: the tile's
-// codes instead, into the slot's upper half, for the value converters.
+// codes instead, into the slot's upper half, for the page's P writers to
+// dequantise.
 template <class C>
 __device__ void producer_v(const DecodeParams& p, const Ctx<C>& c, int s_begin, int s_end) {
   using L = Lay<C>;
@@ -545,7 +547,7 @@ __device__ void producer_v(const DecodeParams& p, const Ctx<C>& c, int s_begin, 
           if constexpr (C::kFp8) {
             // The page's E4M3 codes of this CTA's value columns ([h][64
             // tokens][128 codes], 16 KB) into the upper half of the tile's
-            // slot; the value converters dequantise them over the whole slot.
+            // slot; the page's P writers dequantise them over the whole slot.
             const uint32_t bar = c.bar(L::kBarVCodes + slot);
             mbar_arrive_expect_tx(bar, kVTile / 2);
             c.fill()[L::kFillV + slot] += 1;
