@@ -21,7 +21,7 @@ The line also carries, for the headline workload:
   * `parity`: the GPU result on the workload's seeded inputs against the fp64
     oracle, element by element (every row when the oracle finishes them in
     about 25 s, else a seeded sample of at least 8 rows with the shortest and
-    longest), with north_star's bars;
+    longest), with the parity bars (max-abs 8e-3, mean-abs 1e-3, lse 1e-3);
   * `cpu_baseline`: that same oracle run, timed and scaled to a full call;
   * `e2e`: the public API with pinned host buffers, inputs in and results out
     every step (at least 200 steps, rotating over the pools);

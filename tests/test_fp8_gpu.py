@@ -10,7 +10,7 @@ formats that lose nothing or less: the dequantised values are exact in f16
 (e in [-15, 7]), q's latent part is exact in f16 for these N(0, 1) draws
 except below 2^-14 (absolute error <= 2^-25), and the softmax weights go to
 the PV product as f16 (relative error <= 2^-11 instead of bf16's 2^-8).  The
-five workload shapes are held to the benchmark spec's bars: max-abs 8e-3 and
+five workload shapes are held to the parity bars: max-abs 8e-3 and
 mean-abs 1e-3 on the bf16 output, |lse difference| <= 1e-3, -inf where the
 oracle has no visible token.  The other cases keep the mean-abs and lse bars;
 per element they take the larger of 8e-3 and parity_bounds.fp8_weight_bound,
