@@ -220,3 +220,51 @@ def test_out_of_range_exponent_and_query_are_flagged():
     assert_parity(x, out, lse)
     assert binding.mla_take_device_errors() & binding.MLA_DEVERR_FP8_RANGE
     assert binding.mla_take_device_errors() == 0
+
+
+def test_graph_replays_on_one_plan():
+    # A CUDA graph of the FP8 call, replayed with a new query each time on
+    # one plan, gives what the oracle gives for that query.
+    lens = [2000, 333, 5000]
+    x = inputs.make_fp8_inputs(lens, 64, seed=80)
+    x_alt = inputs.make_fp8_inputs(lens, 64, seed=80)
+    x_alt.q = inputs.make_fp8_inputs(lens, 64, seed=81).q
+    g = x.to("cuda")
+    meta = binding.mla_get_metadata(g.seqlens, 64, 1)
+    ws = torch.empty(binding.mla_workspace_bytes(3, 64, 1), dtype=torch.uint8, device="cuda")
+    out = torch.empty(3, 1, 64, 512, dtype=torch.bfloat16, device="cuda")
+    lse = torch.empty(3, 64, 1, dtype=torch.float32, device="cuda")
+    q_buf = g.q.clone()
+    st = torch.cuda.Stream()
+
+    def call():
+        binding.mla_decode_fp8(q_buf, g.latent_codes, g.rope, g.exps, g.block_table, g.seqlens, g.softmax_scale,
+                               False, meta, workspace=ws, out=out, lse=lse, stream=st)
+
+    with torch.cuda.stream(st):
+        call()
+    st.synchronize()
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph, stream=st):
+        call()
+    for k in range(4):
+        src = x_alt if k % 2 else x
+        with torch.cuda.stream(st):
+            q_buf.copy_(src.q.to("cuda"))
+            graph.replay()
+        st.synchronize()
+        assert binding.mla_check_device_error(meta) == 0
+        assert_parity(src, out.cpu(), lse.cpu())
+    del graph
+
+
+def test_page_outside_pool_is_flagged_and_other_rows_hold():
+    binding.mla_take_device_errors()  # start from a clear sticky word
+    x = inputs.make_fp8_inputs([700, 1500, 300], 64, seed=82)
+    x.block_table[1, 3] = x.latent_codes.shape[0] + 7  # outside [0, num_pages)
+    out, lse, err = run_fp8(x)
+    assert err & binding.MLA_DEVERR_PAGE
+    assert torch.isfinite(out.float()).all()
+    x_ok = inputs.make_fp8_inputs([700, 1500, 300], 64, seed=82)
+    assert_parity(x_ok, out, lse, rows=[0, 2])
+    assert binding.mla_take_device_errors() & binding.MLA_DEVERR_PAGE
