@@ -85,7 +85,16 @@ int tensor_map_encoder(PFN_cuTensorMapEncodeTiled_v12000* fn) {
 // same cache and a few rotating query buffers, so their maps are encoded once
 // instead of on every call.  A map holds only the address and the layout, so
 // it stays right for any later buffer at the same address and size.
-enum MapKind : int { kMapK = 0, kMapV = 1, kMapQ = 2, kMapCodes = 3, kMapRope = 4, kMapVCodes = 5, kMapKinds = 6 };
+enum MapKind : int {
+  kMapK = 0,
+  kMapV = 1,
+  kMapQ = 2,
+  kMapCodes = 3,
+  kMapRope = 4,
+  kMapVCodes = 5,
+  kMapOut = 6,
+  kMapKinds = 7
+};
 
 struct MapCache {
   static constexpr int kWays = 8;
@@ -130,6 +139,22 @@ int encode_panels576(PFN_cuTensorMapEncodeTiled_v12000 enc, CUtensorMap* map, co
   const cuuint32_t elem[3] = {1, 1, 1};
   const CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box, elem,
                          CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                         CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS ? MLA_OK : MLA_ERR_CUDA;
+}
+
+// bf16 out [batch][R][512] as (512 cols, R rows, batch) with strides
+// (1024 B, R * 1024 B): box (64, 32, 1) is 32 rows x 64 columns of one batch
+// row's output, 128B-swizzled in shared memory (the decode kernel's bulk
+// stores of its output tiles; rows past R fall outside the map).
+int encode_out_rows(PFN_cuTensorMapEncodeTiled_v12000 enc, CUtensorMap* map, void* base, int R, int batch) {
+  const cuuint64_t dims[3] = {static_cast<cuuint64_t>(kDv), static_cast<cuuint64_t>(R),
+                              static_cast<cuuint64_t>(batch)};
+  const cuuint64_t strides[2] = {static_cast<cuuint64_t>(kDv) * 2, static_cast<cuuint64_t>(R) * kDv * 2};
+  const cuuint32_t box[3] = {64, 32, 1};
+  const cuuint32_t elem[3] = {1, 1, 1};
+  const CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, base, dims, strides, box, elem,
+                         CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_NONE,
                          CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   return r == CUDA_SUCCESS ? MLA_OK : MLA_ERR_CUDA;
 }
@@ -351,6 +376,13 @@ int decode_impl(const void* q, const CacheRef& cache, int64_t num_pages, const i
             MLA_OK ||
         (st = cached_map(kMapV, kv_cache, kv_rows, &p.tm_v,
                          [&](CUtensorMap* m) { return encode_value_tiles(enc, m, kv_cache, kv_rows); })) != MLA_OK)
+      return st;
+  }
+  if (!out_f32) {
+    // keyed by (batch, R): the same buffer viewed with another row count is another map
+    const uint64_t key = (static_cast<uint64_t>(batch) << 32) | static_cast<uint32_t>(R);
+    if ((st = cached_map(kMapOut, out, key, &p.tm_out,
+                         [&](CUtensorMap* m) { return encode_out_rows(enc, m, out, R, batch); })) != MLA_OK)
       return st;
   }
   p.block_table = block_table;

@@ -1137,16 +1137,19 @@ __device__ void softmax_epilogue(const DecodeParams& p, const Ctx<C>& c, uint32_
     const int rd_row = lane >> 3;   // read-back: rows rd_row + 4 i, chunk lane % 8
     const int rd_chunk = lane & 7;
     if (sg.slot < 0 && !p.out_f32) {
-      __nv_bfloat16* obase = reinterpret_cast<__nv_bfloat16*>(p.out) +
-                             (static_cast<long long>(sg.i) * p.R + sg.mt * kMTile + row0) * kDv + col0;
-      const int rows_ok = p.R - (sg.mt * kMTile + row0);  // rows of this warp that exist
+      // bf16 output of a whole row: the warp's 32 rows x 128 columns are
+      // staged as two 4 KB boxes (8 KB of the value ring per warp; the 128B
+      // swizzle above is the one the output tensor map expects) and written
+      // by two bulk tensor stores, which drain while the warp goes on; the
+      // value ring is released once they have read their staging.
+      uint8_t* stage8 = c.gbase + L::kOffV + ws * 8192;
 #pragma unroll 1
-      for (int k = 0; k < 2; ++k) {  // 64 columns (128 bytes of bf16) per step
+      for (int k = 0; k < 2; ++k) {  // 64 columns (128 bytes of bf16) per box
         float o[64];
         tmem_ld32(t_o + 64 * k, *reinterpret_cast<float(*)[32]>(o));
         tmem_ld32(t_o + 64 * k + 32, *reinterpret_cast<float(*)[32]>(o + 32));
         tmem_wait_ld();
-        uint8_t* srow = stage + lane * 128;
+        uint8_t* srow = stage8 + 4096 * k + lane * 128;
 #pragma unroll
         for (int jj = 0; jj < 8; ++jj) {
           __nv_bfloat162 h0 = __floats2bfloat162_rn(o[8 * jj + 0] * inv_l, o[8 * jj + 1] * inv_l);
@@ -1160,15 +1163,14 @@ __device__ void softmax_epilogue(const DecodeParams& p, const Ctx<C>& c, uint32_
           v.w = *reinterpret_cast<uint32_t*>(&h3);
           *reinterpret_cast<uint4*>(srow + ((jj ^ swz) << 4)) = v;
         }
-        __syncwarp();
-#pragma unroll
-        for (int i = 0; i < 8; ++i) {
-          const int r2 = rd_row + 4 * i;
-          const uint4 v = *reinterpret_cast<const uint4*>(stage + r2 * 128 + ((rd_chunk ^ (r2 & 7)) << 4));
-          if (r2 < rows_ok)
-            *reinterpret_cast<uint4*>(obase + static_cast<long long>(r2) * kDv + 64 * k + 8 * rd_chunk) = v;
-        }
-        __syncwarp();
+      }
+      fence_proxy_async_smem();
+      __syncwarp();
+      if (lane == 0) {
+        const uint32_t src = c.base + L::kOffV + ws * 8192;
+        tma_store_3d(&p.tm_out, src, col0, sg.mt * kMTile + row0, sg.i);
+        tma_store_3d(&p.tm_out, src + 4096, col0 + 64, sg.mt * kMTile + row0, sg.i);
+        bulk_commit_group();
       }
       if (row_valid && half == 0 && sp == 0) p.lse[(static_cast<long long>(sg.i) * p.h_q + hh) * p.s_q + t] = lse_v;
     } else {
@@ -1216,12 +1218,23 @@ __device__ void softmax_epilogue(const DecodeParams& p, const Ctx<C>& c, uint32_
     if (lane == 0) arrive_leader(c, L::kBarOEmpty);  // O is read out: the next segment's PV may overwrite it
     if (lane == 0) {
       MLA_TRACE(18, 8 * (s - s_begin) + ((threadIdx.x >> 5) - 4));
+      bulk_wait_read_all();                   // this warp's bulk stores (if any) have read their staging
       mbar_arrive(c.bar(L::kBarStageFree));  // staging read: the value ring may be refilled
     }
     __syncwarp();
     if (r == 0) MLA_TRACE(13, s - s_begin);
   }
   if (lane == 0) MLA_TRACE(19, (threadIdx.x >> 5) - 4);
+  __syncwarp();
+}
+
+// Softmax warps on their way out (normal or abort): this warp's bulk stores
+// of outputs are complete before the CTA's shared memory goes away.
+template <class C>
+__device__ void softmax_epilogue_then_drain(const DecodeParams& p, const Ctx<C>& c, uint32_t tmem, int s_begin,
+                                            int s_end) {
+  softmax_epilogue(p, c, tmem, s_begin, s_end);
+  if ((threadIdx.x & 31) == 0) bulk_wait_all();
   __syncwarp();
 }
 
@@ -1334,6 +1347,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(C::kThreads, 1)
       tma_prefetch_desc(&p.tm_v);
     }
     tma_prefetch_desc(&p.tm_q);
+    if (!p.out_f32) tma_prefetch_desc(&p.tm_out);
   }
   tc_fence_before();
   __syncthreads();
@@ -1398,7 +1412,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(C::kThreads, 1)
     if (lane == 0 && c.cta == 0) pv_issuer(p, c, tmem, s_begin, s_end);
     __syncwarp();
   } else if (warp < 12) {
-    softmax_epilogue(p, c, tmem, s_begin, s_end);
+    softmax_epilogue_then_drain(p, c, tmem, s_begin, s_end);
   } else {
     if constexpr (C::kFp8) key_converter(p, c, s_begin, s_end);
   }

@@ -111,6 +111,10 @@ struct DecodeParams {
   // page (its 128 columns of each half), panels in [half][panel] order.
   CUtensorMap tm_v;
   CUtensorMap tm_q;  // q: box (64, 64, 9), 64 query rows
+  // bf16 out [batch][R][512] as (512 cols, R rows, batch), strides (1024 B,
+  // R * 1024 B), 128B-swizzled: box (64, 32, 1) is 32 rows x 64 columns of a
+  // work row's output (rows past R are not written).  Unused for fp32 out.
+  CUtensorMap tm_out;
   // FP8 cache only (fp8 = 1; tm_k and tm_v unused then):
   //   latent codes [rows][512] u8 as (512 cols, rows), box (64, 64), no
   //   swizzle: 64 codes of a page's 64 tokens;
