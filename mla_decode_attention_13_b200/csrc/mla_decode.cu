@@ -1122,13 +1122,15 @@ __device__ void softmax_epilogue(const DecodeParams& p, const Ctx<C>& c, uint32_
     const float inv_l = lt > 0.0f ? 1.0f / lt : 0.0f;
     const float lse_v = lt > 0.0f ? (m + __log2f(lt)) * 0.69314718055994530942f : -INFINITY;
     // Output: each warp owns 32 rows x 128 columns of this CTA's tile (its
-    // TMEM lanes, O columns [256 sp + 128 half, +128)).  In steps of 128
-    // bytes of columns it stages them in shared memory (a 4 KB buffer per
-    // warp in the value ring, idle now; 16-byte chunks swizzled by row), then
-    // reads them back four rows per instruction and writes whole 128-byte
-    // lines with coalesced 16-byte stores, skipping rows past R (or
-    // tile_rows).  (Measured: TMA stores of 4 KB boxes took ~4,500 cycles
-    // for a CTA's 128 KB of fp32 partials, ~140 cycles per box.)
+    // TMEM lanes, O columns [256 sp + 128 half, +128)).  It stages them in
+    // shared memory, in the value ring (idle between segments), as 128-byte
+    // rows with 16-byte chunks swizzled by row (the 128B swizzle of a TMA
+    // box).  A whole row's bf16 output leaves by bulk tensor stores; fp32
+    // partials and fp32 outputs are read back four rows per instruction and
+    // written as whole 128-byte lines with coalesced 16-byte stores, skipping
+    // rows past R (or tile_rows).  (Measured: synchronous TMA stores of 4 KB
+    // boxes took ~4,500 cycles for a CTA's 128 KB of fp32 partials, ~140
+    // cycles per box, about what the coalesced stores take.)
     const int ws = (threadIdx.x >> 5) - 4;  // softmax warp 0-7
     uint8_t* stage = c.gbase + L::kOffV + ws * 4096;
     const int row0 = c.cta * kRowsCta + 32 * ((rr >> 5) & 1);  // first row of this warp in the tile
