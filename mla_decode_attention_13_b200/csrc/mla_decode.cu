@@ -1053,9 +1053,10 @@ __device__ void softmax_epilogue(const DecodeParams& p, const Ctx<C>& c, uint32_
                          packed[ci >> 2][4 * (ci & 3) + 2], packed[ci >> 2][4 * (ci & 3) + 3]);
         return true;
       };
-      // ---- page k's P and value tile are ready in this warp's share: the
-      //      group's first PV adds to O, so its P writers first wait until
-      //      every warp of these rows has rescaled its O columns ----
+      // ---- this warp's rows of page k's P (k = q, the thread's page) and its
+      //      share of the value tile are ready: release them to the PV
+      //      issuer.  The group's first PV adds to O, so its P writers first
+      //      wait until every warp of these rows has rescaled its O columns ----
       auto release = [&](int k) -> bool {
         if (resc && k == 0 && q == 0 && !wait_bar(c, c.bar(L::kBarResc + kr), (n_resc - 1) & 1)) return false;
         fence_proxy_async_smem();
