@@ -19,7 +19,7 @@ constexpr int kMTile = 128;       // query rows per work row (UMMA M)
 constexpr int kMaxPairs = 160;    // upper bound on SM pairs of any sm_100 part
 constexpr int kMaxHq = 128;
 constexpr int kMaxSq = 16;
-constexpr int kKappa = 4;         // fixed per-piece cost of the plan, in pages
+constexpr int kKappa = 5;         // fixed per-piece cost of the plan, in pages
 constexpr uint32_t kMagic = 0x314C4D42u;  // "BML1"
 
 // ---------------------------------------------------------------------------
